@@ -1,0 +1,219 @@
+"""CPU oracle for SAW-INT4 paged INT4 KV-cache compression.
+
+TEST INFRASTRUCTURE ONLY.  Only the tests, ``__graft_entry__.smoke()`` and the CPU-baseline
+leg of ``bench.py`` may import this package.  The product path (the CUDA library and its
+Python binding) never imports, links or executes anything here, and this package never
+imports the product package: the two share no code.
+
+The arithmetic lives in ``saw_oracle.c`` (plain C, ``-O2 -ffp-contract=off``, no fast-math);
+this module compiles it on first use with gcc and exposes numpy-level wrappers.  The method
+it restates is token-wise INT4 quantization with a block-diagonal Hadamard rotation, fused
+into a paged KV cache, and decode attention over that cache ("SAW-INT4: System-Aware 4-Bit
+KV-Cache Quantization for Real-World LLM Serving", Research Findings; restated on the idea
+page "Memory compression method reducing KV-cache size...", Core Innovation).
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+import threading
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "saw_oracle.c")
+_BUILD_DIR = os.path.join(_HERE, "_build")
+_LIB_PATH = os.path.join(_BUILD_DIR, "liboracle.so")
+_lock = threading.Lock()
+_lib = None
+
+GCC_FLAGS = ["-O2", "-ffp-contract=off", "-fno-fast-math", "-fPIC", "-shared", "-fopenmp",
+             "-std=gnu11"]
+
+
+def build(force: bool = False) -> str:
+    """Compile saw_oracle.c into _build/liboracle.so (a no-op when it is up to date)."""
+    os.makedirs(_BUILD_DIR, exist_ok=True)
+    if (not force and os.path.exists(_LIB_PATH)
+            and os.path.getmtime(_LIB_PATH) >= os.path.getmtime(_SRC)):
+        return _LIB_PATH
+    tmp = _LIB_PATH + f".tmp{os.getpid()}"
+    cmd = ["gcc", *GCC_FLAGS, "-o", tmp, _SRC, "-lm"]
+    subprocess.run(cmd, check=True)
+    os.replace(tmp, _LIB_PATH)
+    return _LIB_PATH
+
+
+def _load():
+    global _lib
+    with _lock:
+        if _lib is not None:
+            return _lib
+        lib = ctypes.CDLL(build())
+        P = ctypes.c_void_p
+        i32, i64, dbl = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        lib.oracle_bf16_to_f32.argtypes = [ctypes.c_uint16]
+        lib.oracle_bf16_to_f32.restype = ctypes.c_float
+        lib.oracle_f32_to_f16_bits.argtypes = [ctypes.c_float]
+        lib.oracle_f32_to_f16_bits.restype = ctypes.c_uint16
+        lib.oracle_f16_bits_to_f64.argtypes = [ctypes.c_uint16]
+        lib.oracle_f16_bits_to_f64.restype = dbl
+        lib.oracle_fwht_f32.argtypes = [P, i32]
+        lib.oracle_fwht_f32.restype = None
+        lib.oracle_rotate_f32.argtypes = [P, i32]
+        lib.oracle_rotate_f32.restype = None
+        lib.oracle_fwht_f64.argtypes = [P, i32]
+        lib.oracle_fwht_f64.restype = None
+        lib.oracle_rotate_f64.argtypes = [P, i32]
+        lib.oracle_rotate_f64.restype = None
+        lib.oracle_quantize_vec.argtypes = [P, i32, P, P, P, P, P]
+        lib.oracle_quantize_vec.restype = None
+        lib.oracle_rotate_quantize_paged.argtypes = [P, P, P, i64, i32, i32, i32, i64, P, P,
+                                                     i32, i32]
+        lib.oracle_rotate_quantize_paged.restype = i64
+        lib.oracle_dequant_row_f64.argtypes = [P, P, i32, i32, i32, i64, i32, i32, i32, P]
+        lib.oracle_dequant_row_f64.restype = None
+        lib.oracle_decode_fp64.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
+                                           i32, P, i32]
+        lib.oracle_decode_fp64.restype = None
+        _lib = lib
+        return lib
+
+
+def _ptr(a: np.ndarray) -> ctypes.c_void_p:
+    assert a.flags["C_CONTIGUOUS"], "oracle inputs must be C-contiguous"
+    return ctypes.c_void_p(a.ctypes.data)
+
+
+def _as(a, dtype) -> np.ndarray:
+    a = np.ascontiguousarray(a)
+    if a.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {a.dtype}")
+    return a
+
+
+# ---- scalar helpers ------------------------------------------------------------------
+
+def bf16_to_f32(bits: int) -> float:
+    return float(_load().oracle_bf16_to_f32(int(bits)))
+
+
+def f32_to_f16_bits(x: float) -> int:
+    return int(_load().oracle_f32_to_f16_bits(float(np.float32(x))))
+
+
+def f16_bits_to_f64(bits: int) -> float:
+    return float(_load().oracle_f16_bits_to_f64(int(bits)))
+
+
+# ---- rotation --------------------------------------------------------------------------
+
+def fwht_f32(x: np.ndarray) -> np.ndarray:
+    """Normalised Sylvester Hadamard transform of each length-n row (fp32 butterfly)."""
+    y = np.array(x, dtype=np.float32, copy=True, order="C")
+    n = y.shape[-1]
+    flat = y.reshape(-1, n)
+    lib = _load()
+    for r in range(flat.shape[0]):
+        row = flat[r]
+        lib.oracle_fwht_f32(ctypes.c_void_p(row.ctypes.data), n)
+    return y
+
+
+def rotate_f32(x: np.ndarray) -> np.ndarray:
+    """Block-diagonal (128-wide blocks) normalised Hadamard rotation of each row, fp32."""
+    y = np.array(x, dtype=np.float32, copy=True, order="C")
+    D = y.shape[-1]
+    flat = y.reshape(-1, D)
+    lib = _load()
+    for r in range(flat.shape[0]):
+        lib.oracle_rotate_f32(ctypes.c_void_p(flat[r].ctypes.data), D)
+    return y
+
+
+def rotate_f64(x: np.ndarray) -> np.ndarray:
+    y = np.array(x, dtype=np.float64, copy=True, order="C")
+    D = y.shape[-1]
+    flat = y.reshape(-1, D)
+    lib = _load()
+    for r in range(flat.shape[0]):
+        lib.oracle_rotate_f64(ctypes.c_void_p(flat[r].ctypes.data), D)
+    return y
+
+
+# ---- quantizer ---------------------------------------------------------------------------
+
+def quantize_vec(y: np.ndarray):
+    """Quantize one fp32 vector.  Returns (packed uint8[n/2], scale_f16_bits, zero_f16_bits,
+    scale_f32, min_f32)."""
+    y = _as(np.asarray(y, dtype=np.float32), np.float32)
+    n = y.shape[0]
+    assert y.ndim == 1 and n % 2 == 0
+    packed = np.zeros(n // 2, dtype=np.uint8)
+    sh = np.zeros(1, dtype=np.uint16)
+    zh = np.zeros(1, dtype=np.uint16)
+    sf = np.zeros(1, dtype=np.float32)
+    mf = np.zeros(1, dtype=np.float32)
+    _load().oracle_quantize_vec(_ptr(y), n, _ptr(packed), _ptr(sh), _ptr(zh), _ptr(sf), _ptr(mf))
+    return packed, int(sh[0]), int(zh[0]), float(sf[0]), float(mf[0])
+
+
+def rotate_quantize_paged(k_bits, v_bits, slot_mapping, kv_pages, scales, *, page_size=16,
+                          rotate=True, nthreads=1) -> int:
+    """Rotate, quantize and scatter tokens into the paged cache (in place).
+
+    k_bits, v_bits: uint16 bf16 bits [T][Hkv][D].  slot_mapping: int64 [T].
+    kv_pages: uint8 [num_pages][Hkv][2][page_size][D/2] (updated in place).
+    scales: uint16 fp16 bits [num_pages][Hkv][2][page_size][2] (updated in place).
+    Returns the number of out-of-range slots (skipped)."""
+    k_bits = _as(k_bits, np.uint16)
+    v_bits = _as(v_bits, np.uint16)
+    slot_mapping = _as(slot_mapping, np.int64)
+    assert kv_pages.dtype == np.uint8 and kv_pages.flags["C_CONTIGUOUS"]
+    assert scales.dtype == np.uint16 and scales.flags["C_CONTIGUOUS"]
+    T, Hkv, D = k_bits.shape
+    assert v_bits.shape == k_bits.shape and slot_mapping.shape == (T,)
+    num_pages = kv_pages.shape[0]
+    assert kv_pages.shape == (num_pages, Hkv, 2, page_size, D // 2)
+    assert scales.shape == (num_pages, Hkv, 2, page_size, 2)
+    return int(_load().oracle_rotate_quantize_paged(
+        _ptr(k_bits), _ptr(v_bits), _ptr(slot_mapping), T, Hkv, D, page_size, num_pages,
+        _ptr(kv_pages), _ptr(scales), 1 if rotate else 0, int(nthreads)))
+
+
+def dequant_row_f64(kv_pages, scales, page, h, sel, off) -> np.ndarray:
+    num_pages, Hkv, _, page_size, half = kv_pages.shape
+    D = 2 * half
+    y = np.zeros(D, dtype=np.float64)
+    _load().oracle_dequant_row_f64(_ptr(kv_pages), _ptr(scales), Hkv, D, page_size, int(page),
+                                   int(h), int(sel), int(off), _ptr(y))
+    return y
+
+
+def decode_fp64(q_bits, kv_pages, scales, block_table, seq_lens, *, sm_scale=None,
+                rotate=True, nthreads=1) -> np.ndarray:
+    """fp64 decode attention over the INT4 paged cache.
+
+    q_bits: uint16 bf16 bits [S][Hq][D]; block_table: int32 [S][max_blocks];
+    seq_lens: int32 [S].  Returns fp64 [S][Hq][D]."""
+    q_bits = _as(q_bits, np.uint16)
+    block_table = _as(block_table, np.int32)
+    seq_lens = _as(seq_lens, np.int32)
+    S, Hq, D = q_bits.shape
+    num_pages, Hkv, _, page_size, half = kv_pages.shape
+    assert half * 2 == D and Hq % Hkv == 0
+    assert block_table.ndim == 2 and block_table.shape[0] == S and seq_lens.shape == (S,)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    _load().oracle_decode_fp64(_ptr(q_bits), _ptr(kv_pages), _ptr(scales), _ptr(block_table),
+                               block_table.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, page_size,
+                               float(sm_scale), 1 if rotate else 0, _ptr(out), int(nthreads))
+    return out
+
+
+def empty_cache(num_pages: int, Hkv: int, D: int = 128, page_size: int = 16):
+    """Zero-filled cache arrays in the oracle's layout (pages, scales)."""
+    return (np.zeros((num_pages, Hkv, 2, page_size, D // 2), dtype=np.uint8),
+            np.zeros((num_pages, Hkv, 2, page_size, 2), dtype=np.uint16))

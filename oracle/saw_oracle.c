@@ -1,0 +1,300 @@
+/*
+ * saw_oracle.c -- plain, slow CPU oracle for SAW-INT4 paged INT4 KV-cache compression.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls this file:
+ * only the tests, the smoke check and the CPU-baseline leg of the benchmark do.  It shares
+ * no code, header, table or constant generator with the CUDA library.
+ *
+ * What it computes (source pages, all describing the same method):
+ *   - "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving"
+ *     (podcast-summary page, Research Findings): token-wise INT4 quantization combined with a
+ *     block-diagonal Hadamard rotation; a fused rotation-quantization kernel writes straight into
+ *     a paged KV-cache layout; the cache must stay compatible with paged memory, regular access
+ *     and fused attention.
+ *   - "Memory compression method reducing KV-cache size..." (idea page, Core Innovation and
+ *     Summary): the same method restated.
+ *   - "BitDecoding-FP4" (abstract): Hadamard rotation against key outliers under token-wise
+ *     scaling; stacked-query attention over paged caches.
+ * The pages give no formula.  The fixed build parameters used here are: Hadamard block B = 128,
+ * normalised by 1/sqrt(B), applied as an fp32 butterfly (natural Sylvester order, stages
+ * h = 1, 2, ..., 64, no FMA contraction: this file is compiled with -ffp-contract=off);
+ * asymmetric per-(token, kv-head) scale = (max - min) / 15 and zero = min computed in fp32 and
+ * stored as fp16; code = clamp(rint((y - min) / scale), 0, 15); two codes per byte, the even
+ * index in the low nibble; 16-token pages.
+ *
+ * Readings where the pages are silent:
+ *   - a vector whose fp32 scale is 0 (all elements equal) stores scale +0 and all codes 0;
+ *   - a zero minimum is stored as +0 (the stored zero point is min + 0.0f);
+ *   - page layout: codes   uint8 [num_pages][Hkv][2 (K,V)][page_size][D/2],
+ *                  scales  fp16  [num_pages][Hkv][2 (K,V)][page_size][2 (scale, zero)];
+ *   - decode: q is rotated by the same normalised Hadamard, scores use sm_scale, softmax over
+ *     the seq_len valid tokens, and the output is rotated back by the same (self-inverse)
+ *     normalised Hadamard; query head hq reads kv head hq / (Hq / Hkv).
+ * The decode reference runs entirely in fp64 on the dequantised cache.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <string.h>
+
+#define ORACLE_HADAMARD_BLOCK 128
+
+/* ---- scalar conversions -------------------------------------------------------------- */
+
+/* bf16 -> fp32 is exact: the bf16 bits are the high half of the fp32 bits. */
+float oracle_bf16_to_f32(uint16_t b)
+{
+    uint32_t u = (uint32_t)b << 16;
+    float f;
+    memcpy(&f, &u, sizeof f);
+    return f;
+}
+
+/* fp32 -> fp16 bits, IEEE round-to-nearest-even (overflow -> inf, subnormals kept). */
+uint16_t oracle_f32_to_f16_bits(float x)
+{
+    _Float16 h = (_Float16)x;
+    uint16_t b;
+    memcpy(&b, &h, sizeof b);
+    return b;
+}
+
+/* fp16 bits -> fp64, exact widening. */
+double oracle_f16_bits_to_f64(uint16_t b)
+{
+    _Float16 h;
+    memcpy(&h, &b, sizeof h);
+    return (double)h;
+}
+
+/* ---- rotation ----------------------------------------------------------------------- */
+
+/* Normalised Hadamard transform of one block of n = 2^m fp32 values, in place.
+ * Sylvester butterfly: for h = 1, 2, 4, ..., n/2 and every j with (j & h) == 0,
+ *     (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]),
+ * then every element is multiplied by the fp32 constant 1/sqrt(n).  Each step is one IEEE
+ * fp32 add, subtract or multiply, in exactly this order. */
+void oracle_fwht_f32(float *x, int n)
+{
+    for (int h = 1; h < n; h <<= 1) {
+        for (int j = 0; j < n; j++) {
+            if ((j & h) == 0) {
+                float a = x[j];
+                float b = x[j + h];
+                x[j] = a + b;
+                x[j + h] = a - b;
+            }
+        }
+    }
+    const float c = (float)(1.0 / sqrt((double)n));
+    for (int j = 0; j < n; j++)
+        x[j] = x[j] * c;
+}
+
+/* Block-diagonal rotation of a head vector of length D (a multiple of 128): each 128-wide
+ * block is rotated independently. */
+void oracle_rotate_f32(float *x, int D)
+{
+    for (int b = 0; b < D; b += ORACLE_HADAMARD_BLOCK)
+        oracle_fwht_f32(x + b, ORACLE_HADAMARD_BLOCK);
+}
+
+/* Same transform in fp64 (used on the decode side, where the reference is fp64). */
+void oracle_fwht_f64(double *x, int n)
+{
+    for (int h = 1; h < n; h <<= 1) {
+        for (int j = 0; j < n; j++) {
+            if ((j & h) == 0) {
+                double a = x[j];
+                double b = x[j + h];
+                x[j] = a + b;
+                x[j + h] = a - b;
+            }
+        }
+    }
+    const double c = 1.0 / sqrt((double)n);
+    for (int j = 0; j < n; j++)
+        x[j] = x[j] * c;
+}
+
+void oracle_rotate_f64(double *x, int D)
+{
+    for (int b = 0; b < D; b += ORACLE_HADAMARD_BLOCK)
+        oracle_fwht_f64(x + b, ORACLE_HADAMARD_BLOCK);
+}
+
+/* ---- token-wise asymmetric INT4 quantizer -------------------------------------------- */
+
+/* Quantize one vector y[0..n) (n even).  Writes n/2 packed bytes, and the fp16 bits of the
+ * scale and of the zero point.  Also returns the fp32 scale and min through out-pointers
+ * (may be NULL) so that tests can check the error bound against the unrounded values. */
+void oracle_quantize_vec(const float *y, int n, uint8_t *packed, uint16_t *scale_h,
+                         uint16_t *zero_h, float *scale_f32, float *min_f32)
+{
+    float mn = y[0];
+    float mx = y[0];
+    for (int i = 1; i < n; i++) {
+        if (y[i] < mn)
+            mn = y[i];
+        if (y[i] > mx)
+            mx = y[i];
+    }
+    float scale = (mx - mn) / 15.0f;
+    int degenerate = (scale == 0.0f);
+    if (degenerate)
+        scale = 0.0f; /* canonical +0 */
+
+    for (int j = 0; j < n / 2; j++) {
+        int code[2];
+        for (int e = 0; e < 2; e++) {
+            if (degenerate) {
+                code[e] = 0;
+            } else {
+                float q = (y[2 * j + e] - mn) / scale;
+                float r = rintf(q); /* default rounding mode: nearest, ties to even */
+                if (r < 0.0f)
+                    r = 0.0f;
+                if (r > 15.0f)
+                    r = 15.0f;
+                code[e] = (int)r;
+            }
+        }
+        packed[j] = (uint8_t)(code[0] | (code[1] << 4));
+    }
+    *scale_h = oracle_f32_to_f16_bits(scale);
+    *zero_h = oracle_f32_to_f16_bits(mn + 0.0f); /* a zero minimum is stored as +0 */
+    if (scale_f32)
+        *scale_f32 = scale;
+    if (min_f32)
+        *min_f32 = mn;
+}
+
+/* ---- fused rotate + quantize + scatter into the paged cache -------------------------- */
+
+/* k, v: bf16 bits [T][Hkv][D].  slot_mapping: int64 [T]; slot < 0 means "skip this token".
+ * kv_pages: uint8 [num_pages][Hkv][2][page_size][D/2].  scales: fp16 bits
+ * [num_pages][Hkv][2][page_size][2].  rotate = 0 gives the plain-INT4 variant (H = I).
+ * Returns the number of tokens whose slot was >= num_pages * page_size (those are skipped). */
+int64_t oracle_rotate_quantize_paged(const uint16_t *k, const uint16_t *v,
+                                     const int64_t *slot_mapping, int64_t T, int Hkv, int D,
+                                     int page_size, int64_t num_pages, uint8_t *kv_pages,
+                                     uint16_t *scales, int rotate, int nthreads)
+{
+    int64_t bad = 0;
+    const int64_t nslots = num_pages * (int64_t)page_size;
+#pragma omp parallel for schedule(static) num_threads(nthreads) reduction(+ : bad)
+    for (int64_t t = 0; t < T; t++) {
+        int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        if (slot >= nslots) {
+            bad += 1;
+            continue;
+        }
+        int64_t page = slot / page_size;
+        int64_t off = slot % page_size;
+        float y[1024];
+        for (int h = 0; h < Hkv; h++) {
+            for (int sel = 0; sel < 2; sel++) {
+                const uint16_t *src = (sel == 0 ? k : v) + ((size_t)t * Hkv + h) * D;
+                for (int d = 0; d < D; d++)
+                    y[d] = oracle_bf16_to_f32(src[d]);
+                if (rotate)
+                    oracle_rotate_f32(y, D);
+                size_t row = (((size_t)page * Hkv + h) * 2 + sel) * page_size + off;
+                oracle_quantize_vec(y, D, kv_pages + row * (D / 2), &scales[row * 2],
+                                    &scales[row * 2 + 1], NULL, NULL);
+            }
+        }
+    }
+    return bad;
+}
+
+/* ---- decode attention over the INT4 paged cache, fp64 -------------------------------- */
+
+/* Dequantise the head vector stored at (page, kv head h, sel, off) into y[0..D) in fp64:
+ * y[d] = zero + code[d] * scale, with the stored fp16 scale and zero widened exactly. */
+void oracle_dequant_row_f64(const uint8_t *kv_pages, const uint16_t *scales, int Hkv, int D,
+                            int page_size, int64_t page, int h, int sel, int off, double *y)
+{
+    size_t row = (((size_t)page * Hkv + h) * 2 + sel) * page_size + off;
+    const uint8_t *codes = kv_pages + row * (D / 2);
+    double scale = oracle_f16_bits_to_f64(scales[row * 2]);
+    double zero = oracle_f16_bits_to_f64(scales[row * 2 + 1]);
+    for (int j = 0; j < D / 2; j++) {
+        y[2 * j] = zero + (double)(codes[j] & 0xF) * scale;
+        y[2 * j + 1] = zero + (double)(codes[j] >> 4) * scale;
+    }
+}
+
+/* q: bf16 bits [S][Hq][D].  block_table: int32 [S][max_blocks].  seq_lens: int32 [S].
+ * out: fp64 [S][Hq][D].  For each (seq s, query head hq) with kv head h = hq / (Hq / Hkv):
+ *   q_r = H q (rotate != 0) or q,
+ *   s_t = sm_scale * <q_r, k_t>    for the seq_lens[s] tokens t (dequantised k_t),
+ *   p   = softmax(s),
+ *   o_r = sum_t p_t v_t,
+ *   out = H o_r (rotate != 0) or o_r.
+ * A sequence with seq_lens[s] <= 0 gets an all-zero output. */
+void oracle_decode_fp64(const uint16_t *q, const uint8_t *kv_pages, const uint16_t *scales,
+                        const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                        int S, int Hq, int Hkv, int D, int page_size, double sm_scale,
+                        int rotate, double *out, int nthreads)
+{
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic) num_threads(nthreads)
+    for (int s = 0; s < S; s++) {
+        for (int hq = 0; hq < Hq; hq++) {
+            const int h = hq / G;
+            const int L = seq_lens[s];
+            double qr[1024], kv[1024], o[1024];
+            double *dst = out + ((size_t)s * Hq + hq) * D;
+            if (L <= 0) {
+                for (int d = 0; d < D; d++)
+                    dst[d] = 0.0;
+                continue;
+            }
+            const uint16_t *qs = q + ((size_t)s * Hq + hq) * D;
+            for (int d = 0; d < D; d++)
+                qr[d] = (double)oracle_bf16_to_f32(qs[d]);
+            if (rotate)
+                oracle_rotate_f64(qr, D);
+
+            /* pass 1: scores and their maximum */
+            double m = -INFINITY;
+            for (int t = 0; t < L; t++) {
+                int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 0,
+                                       t % page_size, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qr[d] * kv[d];
+                double sc = sm_scale * acc;
+                if (sc > m)
+                    m = sc;
+            }
+            /* pass 2: softmax weights and the weighted sum of values */
+            double l = 0.0;
+            for (int d = 0; d < D; d++)
+                o[d] = 0.0;
+            for (int t = 0; t < L; t++) {
+                int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 0,
+                                       t % page_size, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qr[d] * kv[d];
+                double p = exp(sm_scale * acc - m);
+                l += p;
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 1,
+                                       t % page_size, kv);
+                for (int d = 0; d < D; d++)
+                    o[d] += p * kv[d];
+            }
+            for (int d = 0; d < D; d++)
+                o[d] /= l;
+            if (rotate)
+                oracle_rotate_f64(o, D);
+            for (int d = 0; d < D; d++)
+                dst[d] = o[d];
+        }
+    }
+}

@@ -1,0 +1,505 @@
+"""Pins for the CPU oracle: checks against things other than the oracle itself.
+
+Each test ties one oracle function to a closed form, an invariant, a library routine, a
+hand-derived worked case (tests/golden/quant_cases.json) or brute force, so that a dropped
+term, a wrong sign or index, a swapped nibble or a transposed operand fails somewhere.
+The method is SAW-INT4 ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
+LLM Serving", Research Findings): token-wise INT4 quantization with a block-diagonal Hadamard
+rotation, written into a paged KV cache that fused attention reads.
+"""
+import json
+import os
+from fractions import Fraction
+
+import numpy as np
+import pytest
+import torch
+from scipy.linalg import hadamard
+
+import oracle
+from bit_paged_kv_block_b200 import synth
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "quant_cases.json")
+C32 = np.float32(1.0 / np.sqrt(128.0))
+H128 = hadamard(128).astype(np.float64)          # library Sylvester matrix, entries +-1
+
+
+def popcount_sign(i, j):
+    return -1.0 if bin(i & j).count("1") % 2 else 1.0
+
+
+# ---------------------------------------------------------------------------------------
+# Hadamard rotation
+# ---------------------------------------------------------------------------------------
+
+def test_normalisation_constant_bits():
+    assert np.array(C32).view(np.uint32) == 0x3DB504F3
+
+
+def test_fwht_unit_vectors_are_signed_columns_exactly():
+    """e_j maps to column j of H, times c, bit-exactly: H[i][j] = (-1)^popcount(i & j)."""
+    cols = []
+    for j in range(128):
+        e = np.zeros(128, np.float32)
+        e[j] = 1.0
+        y = oracle.fwht_f32(e)
+        want = np.array([popcount_sign(i, j) for i in range(128)], np.float32) * C32
+        assert np.array_equal(y.view(np.uint32), want.view(np.uint32)), j
+        cols.append(np.sign(y))
+    S = np.stack(cols, axis=1).astype(np.int64)
+    assert np.array_equal(S, H128.astype(np.int64))                 # scipy's Sylvester order
+    assert np.array_equal(S @ S.T, 128 * np.eye(128, dtype=np.int64))  # H H^T = B I
+
+
+@pytest.mark.parametrize("scale", [1.0, 30.0, 1e-3])
+def test_fwht_matches_matrix_product(scale):
+    rng = np.random.default_rng(7)
+    H = H128 / np.sqrt(128.0)
+    for _ in range(200):
+        x = (rng.standard_normal(128) * scale).astype(np.float32)
+        x[rng.choice(128, 4, replace=False)] *= 20
+        y = oracle.fwht_f32(x)
+        exact = H @ x.astype(np.float64)
+        assert np.abs(y - exact).max() <= 2.5e-7 * np.linalg.norm(x.astype(np.float64))
+
+
+def test_fwht_constant_vector():
+    """a * 1 -> (fl(128 a * c), +0, ..., +0): every entry but the first is exactly +0."""
+    for a in [1.0, -3.5, 0.015625, 1000.0]:
+        y = oracle.fwht_f32(np.full(128, a, np.float32))
+        assert y[0] == np.float32(np.float32(128 * a) * C32)
+        assert np.all(y[1:].view(np.uint32) == 0)
+
+
+def test_fwht_round_trip_normwise():
+    """H_norm is symmetric and orthogonal, so it is its own inverse: within 1e-6 normwise."""
+    rng = np.random.default_rng(3)
+    for _ in range(200):
+        x = rng.standard_normal(128).astype(np.float32)
+        x[rng.choice(128, 4, replace=False)] *= 25
+        z = oracle.fwht_f32(oracle.fwht_f32(x))
+        assert np.abs(z - x).max() <= 1e-6 * np.abs(x).max()
+
+
+def test_fwht_f64_round_trip_absolute():
+    rng = np.random.default_rng(4)
+    x = rng.standard_normal((50, 128))
+    z = oracle.rotate_f64(oracle.rotate_f64(x))
+    assert np.abs(z - x).max() <= 1e-6
+    assert np.abs(oracle.rotate_f64(x) - x @ (H128 / np.sqrt(128.0)).T).max() <= 1e-12
+
+
+def test_rotation_is_block_diagonal():
+    """D = 256 rotates each 128 block on its own, which is not the 256-point transform."""
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((4, 256)).astype(np.float32)
+    y = oracle.rotate_f32(x)
+    assert np.array_equal(y[:, :128], oracle.fwht_f32(x[:, :128]))
+    assert np.array_equal(y[:, 128:], oracle.fwht_f32(x[:, 128:]))
+    full = x.astype(np.float64) @ (hadamard(256) / 16.0).T
+    assert np.abs(y - full).max() > 1e-2
+
+
+# ---------------------------------------------------------------------------------------
+# scalar conversions
+# ---------------------------------------------------------------------------------------
+
+def test_f32_to_f16_matches_numpy_rne():
+    rng = np.random.default_rng(11)
+    vals = np.concatenate([
+        rng.standard_normal(20000).astype(np.float32) * np.float32(10.0) ** rng.integers(
+            -9, 6, 20000).astype(np.float32),
+        np.array([0.0, -0.0, 65504.0, 65520.0, 65519.99, 1e9, -1e9, 6.1e-5, 5.96e-8,
+                  2.98e-8, 2.99e-8, 1.0 + 2.0 ** -11, 1.0 + 3 * 2.0 ** -11], np.float32),
+    ]).astype(np.float32)
+    # exact halfway points between adjacent fp16 values exercise ties-to-even
+    h = np.arange(0x0400, 0x7BFF, 37, dtype=np.uint16).view(np.float16).astype(np.float32)
+    h_next = (np.arange(0x0400, 0x7BFF, 37, dtype=np.uint16) + 1).view(np.float16).astype(
+        np.float32)
+    vals = np.concatenate([vals, (h + h_next) / 2]).astype(np.float32)
+    got = np.array([oracle.f32_to_f16_bits(v) for v in vals], np.uint16)
+    want = vals.astype(np.float16).view(np.uint16)
+    assert np.array_equal(got, want)
+
+
+def test_f16_to_f64_all_patterns():
+    bits = np.arange(0, 1 << 16, dtype=np.uint32).astype(np.uint16)
+    want = bits.view(np.float16).astype(np.float64)
+    sel = ~np.isnan(want)
+    got = np.array([oracle.f16_bits_to_f64(b) for b in bits[sel][::7]])
+    assert np.array_equal(got, want[sel][::7])
+
+
+def test_bf16_to_f32_matches_torch():
+    rng = np.random.default_rng(12)
+    bits = rng.integers(0, 1 << 16, 5000).astype(np.uint16)
+    want = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).float().numpy()
+    got = np.array([oracle.bf16_to_f32(b) for b in bits], np.float32)
+    fin = np.isfinite(want)
+    assert np.array_equal(got[fin].view(np.uint32), want[fin].view(np.uint32))
+
+
+# ---------------------------------------------------------------------------------------
+# quantizer
+# ---------------------------------------------------------------------------------------
+
+def _golden_input(spec):
+    x = np.zeros(128, np.float32)
+    if spec["kind"] == "sparse":
+        for k, v in spec["entries"].items():
+            x[int(k)] = v
+    elif spec["kind"] == "constant":
+        x[:] = spec["value"]
+    elif spec["kind"] == "list_then_fill":
+        x[:] = spec["fill"]
+        x[:len(spec["values"])] = spec["values"]
+    return x
+
+
+def _golden_cases():
+    with open(GOLDEN) as f:
+        return json.load(f)["cases"]
+
+
+@pytest.mark.parametrize("case", _golden_cases(), ids=lambda c: c["name"])
+def test_quantizer_golden(case):
+    x = _golden_input(case["input"])
+    y = oracle.fwht_f32(x) if case["rotate"] else x
+    packed, sh, zh, _, _ = oracle.quantize_vec(y)
+    if "packed_hex_all" in case:
+        want = bytes.fromhex(case["packed_hex_all"]) * 64
+    else:
+        pre = bytes.fromhex(case["packed_hex_prefix"])
+        want = pre + bytes.fromhex(case["packed_rest"]) * (64 - len(pre))
+    assert packed.tobytes() == want
+    assert sh == int(case["scale_f16"], 16)
+    assert zh == int(case["zero_f16"], 16)
+
+
+def _unpack(packed):
+    codes = np.empty(packed.size * 2, np.int64)
+    codes[0::2] = packed & 0xF
+    codes[1::2] = packed >> 4
+    return codes
+
+
+def _random_vectors(n, rng):
+    out = []
+    for i in range(n):
+        kind = i % 4
+        x = rng.standard_normal(128).astype(np.float32)
+        if kind == 1:
+            x[rng.choice(128, 4, replace=False)] *= np.float32(rng.uniform(10, 30))
+        if kind == 2:
+            x = (x * np.float32(10.0) ** rng.integers(-20, 20)).astype(np.float32)
+        if kind == 3:
+            x = np.round(x * 4) / 4            # many exact ties
+        out.append(oracle.fwht_f32(x) if i % 2 == 0 else x)
+    return out
+
+
+def test_quantizer_invariants_and_bound():
+    """min -> 0, max -> 15, monotone codes, |y - (min + code scale)| <= scale/2 (fp32 values),
+    and with the stored fp16 values the reading's widened bound holds."""
+    rng = np.random.default_rng(21)
+    for y in _random_vectors(400, rng):
+        packed, sh, zh, sf, mf = oracle.quantize_vec(y)
+        codes = _unpack(packed)
+        assert sf > 0
+        assert codes[np.argmin(y)] == 0 and codes[np.argmax(y)] == 15
+        order = np.argsort(y, kind="stable")
+        assert np.all(np.diff(codes[order]) >= 0)
+        yd = y.astype(np.float64)
+        err = np.abs(yd - (np.float64(mf) + codes * np.float64(sf)))
+        ulp = np.spacing(np.float32(np.abs(y).max())).astype(np.float64)
+        assert err.max() <= np.float64(sf) / 2 + 16 * ulp
+        s16, z16 = oracle.f16_bits_to_f64(sh), oracle.f16_bits_to_f64(zh)
+        if not (6.2e-5 < sf < 6e4 and abs(mf) < 6e4 and (mf == 0 or abs(mf) > 6.2e-5)):
+            continue                 # fp16 storage range: overflow/underflow is unsupported
+        err16 = np.abs(yd - (z16 + codes * s16))
+        bound16 = s16 / 2 + 15 * abs(sf - s16) + abs(mf - z16) + 16 * ulp + abs(sf - s16) / 2
+        assert err16.max() <= bound16
+
+
+def test_quantizer_brute_force_nearest_level():
+    """Each code is the level k in 0..15 nearest (exact rationals) to (y - min)/scale as the
+    fp32 values give it; within a hair of a half-integer either neighbour is allowed and an
+    exact half goes to the even level."""
+    rng = np.random.default_rng(22)
+    for y in _random_vectors(120, rng):
+        packed, _, _, sf, mf = oracle.quantize_vec(y)
+        codes = _unpack(packed)
+        S, M = Fraction(float(sf)), Fraction(float(mf))
+        for i in range(128):
+            d = Fraction(float(np.float32(y[i] - np.float32(mf))))   # the fp32 difference
+            q = d / S
+            lo = int(q)                                               # q >= 0
+            frac = q - lo
+            half = Fraction(1, 2)
+            if abs(frac - half) <= Fraction(1, 1 << 18):
+                assert codes[i] in (lo, min(lo + 1, 15))
+                if frac == half:
+                    assert codes[i] % 2 == 0 or codes[i] == 15
+            else:
+                want = lo + (1 if frac > half else 0)
+                assert codes[i] == min(max(want, 0), 15)
+        del M
+
+
+def test_quantizer_degenerate_and_signed_zero():
+    packed, sh, zh, sf, _ = oracle.quantize_vec(np.full(128, -2.5, np.float32))
+    assert sf == 0.0 and sh == 0 and zh == np.array(np.float16(-2.5)).view(np.uint16)
+    assert not packed.any()
+    y = np.zeros(128, np.float32)
+    y[5] = -0.0
+    y[9] = 1.0
+    packed, sh, zh, _, _ = oracle.quantize_vec(y)
+    assert zh == 0x0000                        # a zero minimum is stored as +0
+    assert _unpack(packed)[9] == 15 and _unpack(packed)[5] == 0
+
+
+def test_quantizer_subnormal_scale():
+    """Tiny vectors whose scale is subnormal still satisfy min -> 0 and max -> 15."""
+    y = np.zeros(128, np.float32)
+    y[3] = np.float32(1e-39)
+    y[7] = np.float32(-2e-39)
+    packed, _, _, sf, _ = oracle.quantize_vec(y)
+    codes = _unpack(packed)
+    assert 0 < sf < np.finfo(np.float32).tiny
+    assert codes[7] == 0 and codes[3] == 15
+
+
+# ---------------------------------------------------------------------------------------
+# scatter into the paged layout
+# ---------------------------------------------------------------------------------------
+
+def test_scatter_layout_and_skips():
+    rng = np.random.default_rng(31)
+    T, Hkv, D, P, num_pages = 40, 3, 128, 16, 6
+    k = synth.bf16_bits(torch.randn(T, Hkv, D).to(torch.bfloat16))
+    v = synth.bf16_bits(torch.randn(T, Hkv, D).to(torch.bfloat16))
+    slots = rng.permutation(num_pages * P)[:T].astype(np.int64)
+    slots[3] = -1
+    slots[11] = num_pages * P + 5          # out of range: skipped and counted
+    pages, scales = oracle.empty_cache(num_pages, Hkv, D, P)
+    pages[:] = 0xA5
+    scales[:] = 0x5A5A
+    bad = oracle.rotate_quantize_paged(k, v, slots, pages, scales, page_size=P)
+    assert bad == 1
+    touched = np.zeros((num_pages, P), bool)
+    for t in range(T):
+        s = slots[t]
+        if s < 0 or s >= num_pages * P:
+            continue
+        pg, off = divmod(int(s), P)
+        touched[pg, off] = True
+        for h in range(Hkv):
+            for sel, src in enumerate((k, v)):
+                x = src[t, h].view(np.int16).astype(np.int32) << 16
+                y = oracle.fwht_f32(x.astype(np.uint32).view(np.float32))
+                pk, sh, zh, _, _ = oracle.quantize_vec(y)
+                assert np.array_equal(pages[pg, h, sel, off], pk)
+                assert scales[pg, h, sel, off, 0] == sh and scales[pg, h, sel, off, 1] == zh
+    for pg in range(num_pages):
+        for off in range(P):
+            if not touched[pg, off]:
+                assert np.all(pages[pg, :, :, off] == 0xA5)
+                assert np.all(scales[pg, :, :, off] == 0x5A5A)
+
+
+def test_scatter_unrotated_variant():
+    T, Hkv, D = 4, 1, 128
+    k = synth.bf16_bits(torch.randn(T, Hkv, D).to(torch.bfloat16))
+    pages, scales = oracle.empty_cache(1, Hkv, D)
+    oracle.rotate_quantize_paged(k, k, np.arange(T, dtype=np.int64), pages, scales,
+                                 rotate=False)
+    x = (k[2, 0].view(np.int16).astype(np.int32) << 16).astype(np.uint32).view(np.float32)
+    pk, _, _, _, _ = oracle.quantize_vec(x)
+    assert np.array_equal(pages[0, 0, 0, 2], pk)
+
+
+def test_dequant_round_trip_bound():
+    """Dequantising the stored codes lands within the quantizer's error bound of y."""
+    rng = np.random.default_rng(41)
+    wl = synth.make_workload("tiny")
+    k = synth.bf16_bits(synth.kv_values(wl, "K"))
+    v = synth.bf16_bits(synth.kv_values(wl, "V"))
+    seq, pos = synth.token_index(wl)
+    slots = synth.slot_mapping(wl, seq, pos)
+    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
+    oracle.rotate_quantize_paged(k, v, slots, pages, scales)
+    for t in rng.choice(len(slots), 20, replace=False):
+        pg, off = divmod(int(slots[t]), 16)
+        for h in range(wl.num_kv_heads):
+            x = (k[t, h].view(np.int16).astype(np.int32) << 16).astype(np.uint32).view(
+                np.float32)
+            y = oracle.fwht_f32(x).astype(np.float64)
+            yhat = oracle.dequant_row_f64(pages, scales, pg, h, 0, off)
+            s16 = oracle.f16_bits_to_f64(scales[pg, h, 0, off, 0])
+            assert np.abs(yhat - y).max() <= 0.5 * s16 * 1.01 + 15 * s16 * 2 ** -11 + \
+                abs(y.min()) * 2 ** -11
+
+
+# ---------------------------------------------------------------------------------------
+# decode attention
+# ---------------------------------------------------------------------------------------
+
+def _cache_for(wl, rotate=True):
+    k = synth.bf16_bits(synth.kv_values(wl, "K"))
+    v = synth.bf16_bits(synth.kv_values(wl, "V"))
+    seq, pos = synth.token_index(wl)
+    slots = synth.slot_mapping(wl, seq, pos)
+    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads, wl.head_dim,
+                                       wl.page_size)
+    oracle.rotate_quantize_paged(k, v, slots, pages, scales, page_size=wl.page_size,
+                                 rotate=rotate)
+    return k, v, pages, scales
+
+
+def _dequant_seq(wl, pages, scales, s, h, sel):
+    L = int(wl.seq_lens[s])
+    rows = []
+    for t in range(L):
+        pg = wl.block_table[s, t // 16]
+        rows.append(oracle.dequant_row_f64(pages, scales, pg, h, sel, t % 16))
+    return np.stack(rows)
+
+
+def test_decode_single_token_is_rotated_value():
+    wl = synth.custom("one", [1], num_q_heads=4, num_kv_heads=2, seed=1)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens)
+    Hn = H128 / np.sqrt(128.0)
+    for hq in range(4):
+        vhat = _dequant_seq(wl, pages, scales, 0, hq // 2, 1)[0]
+        assert np.abs(out[0, hq] - Hn @ vhat).max() <= 1e-12
+
+
+def test_decode_matches_torch_sdpa_fp64():
+    """G = 1: the oracle equals torch's fp64 scaled-dot-product attention run on the rotated
+    query and the dequantised cache, rotated back."""
+    wl = synth.custom("sdpa", [37, 16, 17, 1, 64], num_q_heads=2, num_kv_heads=2, seed=2)
+    _, _, pages, scales = _cache_for(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(qb, pages, scales, wl.block_table, wl.seq_lens)
+    Hn = torch.tensor(H128 / np.sqrt(128.0))
+    qf = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).double()
+    for s in range(wl.num_seqs):
+        for h in range(2):
+            K = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 0))
+            V = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 1))
+            qr = Hn @ qf[s, h]
+            o = torch.nn.functional.scaled_dot_product_attention(
+                qr[None, None, None], K[None, None], V[None, None])[0, 0, 0]
+            assert torch.allclose(torch.from_numpy(out[s, h]), Hn @ o, atol=1e-12, rtol=0)
+
+
+def test_decode_identical_keys_and_zero_scale_give_mean():
+    """If every key is the same, or sm_scale is 0, the weights are uniform: the output is the
+    rotated mean of the dequantised values."""
+    wl = synth.custom("flat", [50], num_q_heads=2, num_kv_heads=1, seed=3)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    Hn = H128 / np.sqrt(128.0)
+    V = _dequant_seq(wl, pages, scales, 0, 0, 1)
+    out0 = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens, sm_scale=0.0)
+    assert np.abs(out0[0, 0] - Hn @ V.mean(0)).max() <= 1e-12
+    pages2, scales2 = pages.copy(), scales.copy()
+    first = wl.block_table[0, 0]
+    for t in range(50):
+        pg = wl.block_table[0, t // 16]
+        pages2[pg, 0, 0, t % 16] = pages[first, 0, 0, 0]
+        scales2[pg, 0, 0, t % 16] = scales[first, 0, 0, 0]
+    out = oracle.decode_fp64(q, pages2, scales2, wl.block_table, wl.seq_lens)
+    assert np.abs(out[0, 1] - Hn @ V.mean(0)).max() <= 1e-12
+
+
+def test_decode_dominant_key_selects_its_value():
+    wl = synth.custom("dom", [40], num_q_heads=1, num_kv_heads=1, seed=4)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    V = _dequant_seq(wl, pages, scales, 0, 0, 1)
+    K = _dequant_seq(wl, pages, scales, 0, 0, 0)
+    qf = (q[0, 0].view(np.int16).astype(np.int32) << 16).astype(np.uint32).view(np.float32)
+    qr = (H128 / np.sqrt(128.0)) @ qf.astype(np.float64)
+    t = int(np.argmax(K @ qr))
+    out = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens, sm_scale=1e4)
+    assert np.abs(out[0, 0] - (H128 / np.sqrt(128.0)) @ V[t]).max() <= 1e-9
+
+
+def test_decode_gqa_head_mapping():
+    """Query head hq reads kv head hq // G: the same as a G = 1 run on that head alone."""
+    wl = synth.custom("gqa", [33, 70], num_q_heads=8, num_kv_heads=2, seed=5)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens)
+    for hq in range(8):
+        h = hq // 4
+        p1 = np.ascontiguousarray(pages[:, h:h + 1])
+        s1 = np.ascontiguousarray(scales[:, h:h + 1])
+        o1 = oracle.decode_fp64(np.ascontiguousarray(q[:, hq:hq + 1]), p1, s1,
+                                wl.block_table, wl.seq_lens)
+        assert np.array_equal(o1[:, 0], out[:, hq])
+    assert np.abs(out[:, 0] - out[:, 4]).max() > 1e-3     # the two kv heads differ
+
+
+def test_decode_page_permutation_invariance():
+    wl = synth.custom("perm", [45, 16, 17], num_q_heads=4, num_kv_heads=1, seed=6)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens)
+    perm = np.random.default_rng(0).permutation(wl.num_pages)
+    inv = np.argsort(perm)
+    table2 = np.where(wl.block_table >= 0, inv[np.maximum(wl.block_table, 0)], -1).astype(
+        np.int32)
+    out2 = oracle.decode_fp64(q, np.ascontiguousarray(pages[perm]),
+                              np.ascontiguousarray(scales[perm]), table2, wl.seq_lens)
+    assert np.array_equal(out, out2)
+
+
+def test_decode_empty_sequence_is_zero():
+    wl = synth.custom("empty", [0, 5], num_q_heads=2, num_kv_heads=1, seed=7)
+    _, _, pages, scales = _cache_for(wl)
+    q = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(q, pages, scales, wl.block_table, wl.seq_lens)
+    assert not out[0].any() and np.abs(out[1]).max() > 0
+
+
+# ---------------------------------------------------------------------------------------
+# method-level check: rotation helps on outlier keys
+# ---------------------------------------------------------------------------------------
+
+def test_rotation_lowers_quantized_attention_error():
+    """On keys with outlier channels, rotating before the INT4 quantizer gives lower logit and
+    output error against unquantized fp64 attention than the plain INT4 quantizer does
+    ("SAW-INT4", Research Findings: naive INT4 degrades accuracy; the rotation recovers most
+    of it).  The size of the gain is not given on the pages (parity unpinned)."""
+    wl = synth.make_workload("tiny")
+    kb = synth.bf16_bits(synth.kv_values(wl, "K"))
+    vb = synth.bf16_bits(synth.kv_values(wl, "V"))
+    qb = synth.bf16_bits(synth.q_values(wl))
+    tof = lambda b: torch.from_numpy(b.view(np.int16)).view(torch.bfloat16).double()
+    K, V, Q = tof(kb), tof(vb), tof(qb)                 # [T][Hkv][D], [S][Hq][D]
+    G = wl.group
+    errs = {}
+    for rotate in (True, False):
+        seq, pos = synth.token_index(wl)
+        slots = synth.slot_mapping(wl, seq, pos)
+        pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
+        oracle.rotate_quantize_paged(kb, vb, slots, pages, scales, rotate=rotate)
+        out = oracle.decode_fp64(qb, pages, scales, wl.block_table, wl.seq_lens,
+                                 rotate=rotate)
+        o_err, l_err = [], []
+        for hq in range(wl.num_q_heads):
+            h = hq // G
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                Q[0, hq][None, None, None], K[:, h][None, None], V[:, h][None, None])[0, 0, 0]
+            o_err.append(np.abs(out[0, hq] - ref.numpy()).mean())
+            Kq = torch.from_numpy(_dequant_seq(wl, pages, scales, 0, h, 0))
+            Hn = torch.tensor(H128 / np.sqrt(128.0))
+            qr = Hn @ Q[0, hq] if rotate else Q[0, hq]
+            l_err.append((Kq @ qr - K[:, h] @ Q[0, hq]).abs().mean().item())
+        errs[rotate] = (np.mean(o_err), np.mean(l_err))
+    assert errs[True][0] < errs[False][0]
+    assert errs[True][1] < errs[False][1]
