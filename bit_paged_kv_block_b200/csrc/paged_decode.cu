@@ -1,0 +1,796 @@
+// paged_decode.cu -- decode attention over the INT4 paged KV cache (split-K, GQA-stacked).
+//
+// The read side of "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM
+// Serving" (Research Findings: the quantized cache must keep fused attention execution over
+// paged memory with regular access), with the query heads of one kv head stacked into one
+// tensor-core tile as in "BitDecoding-FP4" (abstract: stacked query MMA on paged KV caches).
+// Because H is orthogonal and symmetric, <q, k> = <Hq, Hk> and sum p_t v_t = H sum p_t (H v_t):
+// the kernel rotates q once, attends over the rotated codes and rotates the output back.
+//
+// Work split.  A (sequence s, kv head h) pair is a segment of ceil(len_s / 16) pages.  All
+// segments are laid end to end (seq-major, then kv head) and that flat page range P is cut into
+// C = min(gridDim.x, P / 4) equal slices, one per CTA; inside a CTA the 4 warps take every 4th
+// page.  Each
+// (segment, CTA) intersection is a piece: the warps' online-softmax states for a piece are
+// merged in shared memory; a segment that spans several CTAs has one partial per CTA in the
+// workspace (slot segment + CTA index, unique because both orders are monotone) and the CTA
+// that finishes it last (an atomic ticket, no waiting) merges them, rotates the result back
+// and writes it.
+//
+// Per page (16 tokens x one kv head, 2 KiB of codes + 128 B of scales), per warp:
+//   * one elected lane queues a 2-D tensor copy of the 32 code rows (64B swizzle, so both the
+//     K reads and the transposed V reads below are bank-conflict free) and a 1-D bulk copy of
+//     the scales into a 6-stage ring, completion on an mbarrier (bounded wait);
+//   * S^T[16 tok x 8 heads] = K_codes[16 x 128] . Q^T with mma.m16n8k16 (fp16 in, fp32 acc):
+//     the codes 0..15 are exact in fp16, and s = scale * acc + zero * sum(q) in fp32;
+//   * online softmax in the log2 domain (q carries sm_scale * log2 e);
+//   * O^T[128 d x 8 heads] += V_codes^T . P'^T with P' = p * scale_V in fp16 and the zero
+//     point added in fp32 through sum_t p_t zero_t.
+// The query dimension d of QK and the value dimension of PV are consumed in a permuted order
+// (both sides permuted alike), which lets every thread unpack whole 32-bit code words.
+#include <cfloat>
+#include <cudaTypedefs.h>
+
+#include "saw_device.cuh"
+#include "saw_internal.h"
+
+namespace saw {
+namespace {
+
+constexpr int kWarps = 4;
+constexpr int kThreads = 32 * kWarps;
+constexpr int kStages = 6;
+constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
+constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
+constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
+constexpr int kSlotFloats = 32 * 32 + 16;               // O (lane layout) + m[8] + l[8]
+constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a page wait after 1 s
+constexpr float kHadamardC = 0.0883883461356163f;
+
+// shared memory carve-up (bytes, from a 1024-aligned base)
+constexpr int kSmemCodes = 0;
+constexpr int kSmemScales = kSmemCodes + kWarps * kStages * kCodeBytes;
+constexpr int kSmemBars = kSmemScales + kWarps * kStages * kScaleBytes;
+constexpr int kSmemMergeO = kSmemBars + kWarps * kStages * 8;
+constexpr int kSmemMergeML = kSmemMergeO + (kWarps - 1) * 32 * 32 * 4;
+constexpr int kSmemFlags = kSmemMergeML + (kWarps - 1) * 16 * 4;
+constexpr int kSmemPrefix = kSmemFlags + 64;
+
+size_t decode_smem_bytes(int32_t num_seqs)
+{
+    return 1024 + kSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
+}
+
+struct DecodeParams {
+    const uint16_t *q;
+    const uint8_t *scales;       // bytes; 128 B per (page, kv head)
+    const int32_t *block_table;
+    const int32_t *seq_lens;
+    float *out;
+    uint32_t *tickets;
+    float *partials;
+    uint32_t *status;
+    int64_t num_pages;
+    int32_t max_blocks;
+    int32_t num_seqs;
+    int32_t hq;
+    int32_t hkv;
+    int32_t group;
+    float q_mult;                // fp32(1/sqrt(128)) * sm_scale * log2(e)
+};
+
+// ---- small helpers ----------------------------------------------------------------------
+
+// Largest s in [0, S) with hkv * pre[s] <= pos (pos < hkv * pre[S]).
+__device__ __forceinline__ int find_seq(const int32_t *pre, int S, int64_t pos, int64_t hkv)
+{
+    int lo = 0, hi = S;
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (hkv * pre[mid] <= pos)
+            lo = mid;
+        else
+            hi = mid;
+    }
+    return lo;
+}
+
+// Index of the CTA whose slice [c P / C, (c + 1) P / C) holds flat page pos.
+__device__ __forceinline__ int64_t cta_of(int64_t pos, int64_t P, int64_t C)
+{
+    return ((pos + 1) * C + P - 1) / P - 1;
+}
+
+// Unpack one 32-bit word of packed codes (bytes b0..b3, low nibble first) into four fp16x2
+// registers holding exact code values: (b0.lo, b2.lo), (b0.hi, b2.hi), (b1.lo, b3.lo),
+// (b1.hi, b3.hi).  OR-ing a nibble into the mantissa of 1024.0 gives 1024 + n (or 1024 + 16 n
+// for a high nibble), which one fp16 subtract / fma turns back into n exactly.
+__device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t y[4])
+{
+    const uint32_t magic = 0x64006400u;
+    const uint32_t w8 = w >> 8;
+    const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));   // 1024
+    const __half2 k1_16 = __half2half2(__ushort_as_half(0x2C00));   // 1/16
+    const __half2 km64 = __half2half2(__ushort_as_half(0xD400));    // -64
+    y[0] = half2_as_u32(__hsub2(u32_as_half2((w & 0x000F000Fu) | magic), k1024));
+    y[1] = half2_as_u32(__hfma2(u32_as_half2((w & 0x00F000F0u) | magic), k1_16, km64));
+    y[2] = half2_as_u32(__hsub2(u32_as_half2((w8 & 0x000F000Fu) | magic), k1024));
+    y[3] = half2_as_u32(__hfma2(u32_as_half2((w8 & 0x00F000F0u) | magic), k1_16, km64));
+}
+
+__device__ __forceinline__ float2 h2_to_f2(uint32_t u)
+{
+    return __half22float2(u32_as_half2(u));
+}
+
+// Per-warp running state of one piece, in mma accumulator layout: thread (g, t) holds heads
+// 2t and 2t + 1 and, for m-tile i = 2c + h2, the value rows d = 32c + 4g + 2h2 (+1).
+struct WarpState {
+    float o[8][4];
+    float m[2];
+    float l[2];
+    float z[2];
+};
+
+__device__ __forceinline__ void state_reset(WarpState &st)
+{
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+#pragma unroll
+        for (int k = 0; k < 4; k++)
+            st.o[i][k] = 0.0f;
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+        st.m[e] = -INFINITY;
+        st.l[e] = 0.0f;
+        st.z[e] = 0.0f;
+    }
+}
+
+// Rotated, scaled query of (seq s, kv head h) as fp16 mma B fragments.
+// Thread (g, t) owns query head g of the group and d in [32t, 32t + 32).
+__device__ __forceinline__ void load_query(const DecodeParams &p, int s, int h, int g, int t,
+                                           uint32_t bq[8][2], float sq_out[2])
+{
+    float x[32];
+    if (g < p.group) {
+        const uint16_t *src = p.q + ((static_cast<int64_t>(s) * p.hq + h * p.group + g) * kHeadDim + 32 * t);
+#pragma unroll
+        for (int c = 0; c < 4; c++) {
+            const uint4 u = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                x[8 * c + 2 * k] = __uint_as_float(w[k] << 16);
+                x[8 * c + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+            }
+        }
+    } else {
+#pragma unroll
+        for (int l = 0; l < 32; l++)
+            x[l] = 0.0f;
+    }
+    // Hadamard butterfly: d bits 0..4 in registers, bits 5, 6 across lanes t ^ 1, t ^ 2.
+#pragma unroll
+    for (int hb = 1; hb < 32; hb <<= 1)
+#pragma unroll
+        for (int l = 0; l < 32; l++)
+            if ((l & hb) == 0) {
+                const float a = x[l], b = x[l + hb];
+                x[l] = a + b;
+                x[l + hb] = a - b;
+            }
+#pragma unroll
+    for (int lb = 1; lb <= 2; lb <<= 1) {
+        const bool high = (t & lb) != 0;
+#pragma unroll
+        for (int l = 0; l < 32; l++) {
+            const float o = __shfl_xor_sync(0xFFFFFFFFu, x[l], lb);
+            x[l] = high ? o - x[l] : x[l] + o;
+        }
+    }
+    float sq = 0.0f;
+    __half hq[32];
+#pragma unroll
+    for (int l = 0; l < 32; l++) {
+        hq[l] = __float2half_rn(x[l] * p.q_mult);
+        sq += __half2float(hq[l]);
+    }
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
+    sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
+    // k-step (i, e): k slots (2t, 2t+1 | 2t+8, 2t+9) <-> d = 32t + 8i + 2e + (0, 4 | 1, 5)
+#pragma unroll
+    for (int i = 0; i < 4; i++)
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const int l0 = 8 * i + 2 * e;
+            bq[2 * i + e][0] = half2_as_u32(__halves2half2(hq[l0], hq[l0 + 4]));
+            bq[2 * i + e][1] = half2_as_u32(__halves2half2(hq[l0 + 1], hq[l0 + 5]));
+        }
+    // thread (g, t) needs sum(q) of heads 2t and 2t + 1 (held by lanes 4 (2t) and 4 (2t + 1))
+    sq_out[0] = __shfl_sync(0xFFFFFFFFu, sq, 8 * t);
+    sq_out[1] = __shfl_sync(0xFFFFFFFFu, sq, 8 * t + 4);
+}
+
+// One page of one warp: QK^T, online softmax, PV.
+__device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int valid,
+                                             const uint32_t bq[8][2], const float sq[2],
+                                             int lane, WarpState &st)
+{
+    const int g = lane >> 2, t = lane & 3;
+
+    // ---- S^T = K . Q^T over 16 tokens (rows g, g + 8) -----------------------------------
+    const uint4 k0 = lds128(cbase + g * 64 + ((t ^ ((g >> 1) & 3)) << 4));
+    const uint4 k1 = lds128(cbase + (g + 8) * 64 + ((t ^ (((g + 8) >> 1) & 3)) << 4));
+    const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
+    const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
+    float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+#pragma unroll
+    for (int i = 0; i < 4; i++) {
+        uint32_t ya[4], yb[4];
+        unpack_codes(kw0[i], ya);
+        unpack_codes(kw1[i], yb);
+        const uint32_t a0[4] = {ya[0], yb[0], ya[1], yb[1]};
+        const uint32_t a1[4] = {ya[2], yb[2], ya[3], yb[3]};
+        mma_16816(acc, a0, bq[2 * i][0], bq[2 * i][1]);
+        mma_16816(acc, a1, bq[2 * i + 1][0], bq[2 * i + 1][1]);
+    }
+
+    // ---- logits (log2 domain) ---------------------------------------------------------------
+    const bool v0 = g < valid, v1 = g + 8 < valid;
+    const float2 ksz0 = h2_to_f2(lds32(sbase + 4 * g));
+    const float2 ksz1 = h2_to_f2(lds32(sbase + 4 * (g + 8)));
+    float s[4];
+    s[0] = v0 ? fmaf(ksz0.x, acc[0], ksz0.y * sq[0]) : -INFINITY;
+    s[1] = v0 ? fmaf(ksz0.x, acc[1], ksz0.y * sq[1]) : -INFINITY;
+    s[2] = v1 ? fmaf(ksz1.x, acc[2], ksz1.y * sq[0]) : -INFINITY;
+    s[3] = v1 ? fmaf(ksz1.x, acc[3], ksz1.y * sq[1]) : -INFINITY;
+
+    float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 8));
+        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 16));
+    }
+    const bool grow = mx[0] > st.m[0] || mx[1] > st.m[1];
+    if (__any_sync(0xFFFFFFFFu, grow)) {
+        float alpha[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const float mn = fmaxf(st.m[e], mx[e]);
+            alpha[e] = ex2_approx(st.m[e] - mn);
+            st.m[e] = mn;
+            st.l[e] *= alpha[e];
+            st.z[e] *= alpha[e];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            st.o[i][0] *= alpha[0];
+            st.o[i][1] *= alpha[1];
+            st.o[i][2] *= alpha[0];
+            st.o[i][3] *= alpha[1];
+        }
+    }
+    float pr[4];
+    pr[0] = ex2_approx(s[0] - st.m[0]);
+    pr[1] = ex2_approx(s[1] - st.m[1]);
+    pr[2] = ex2_approx(s[2] - st.m[0]);
+    pr[3] = ex2_approx(s[3] - st.m[1]);
+
+    // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
+    float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));
+    float2 vsz1 = h2_to_f2(lds32(sbase + 64 + 4 * (g + 8)));
+    if (!v0)
+        vsz0 = make_float2(0.0f, 0.0f);
+    if (!v1)
+        vsz1 = make_float2(0.0f, 0.0f);
+    st.l[0] += pr[0] + pr[2];
+    st.l[1] += pr[1] + pr[3];
+    st.z[0] = fmaf(pr[0], vsz0.y, fmaf(pr[2], vsz1.y, st.z[0]));
+    st.z[1] = fmaf(pr[1], vsz0.y, fmaf(pr[3], vsz1.y, st.z[1]));
+    const uint32_t p01 = half2_as_u32(__floats2half2_rn(pr[0] * vsz0.x, pr[1] * vsz0.x));
+    const uint32_t p23 = half2_as_u32(__floats2half2_rn(pr[2] * vsz1.x, pr[3] * vsz1.x));
+    const uint32_t pb0 = movmatrix_trans(p01);   // B fragment: tokens 2t, 2t+1 of head g
+    const uint32_t pb1 = movmatrix_trans(p23);   // tokens 2t + 8, 2t + 9
+
+    // ---- O^T += V^T . P'^T -----------------------------------------------------------------
+    // ldmatrix.trans: lane L addresses row (L & 7) of matrix L >> 3; matrices are
+    // (tokens 0-7 | 8-15) x (16-byte chunk 2j | 2j + 1) of the V rows (rows 16..31).
+    const int vtok = ((lane >> 3) & 1) * 8 + (lane & 7);
+    const int vrow = 16 + vtok;
+    const uint32_t vrow_base = cbase + vrow * 64;
+    const int vsw = (vrow >> 1) & 3;
+#pragma unroll
+    for (int j = 0; j < 2; j++) {
+        const int chunk = 2 * j + (lane >> 4);
+        uint32_t r[4];
+        ldsm_x4_trans(vrow_base + ((chunk ^ vsw) << 4), r[0], r[1], r[2], r[3]);
+        // r[0]: tokens 0-7, chunk 2j; r[1]: tokens 8-15, chunk 2j; r[2], r[3]: chunk 2j + 1
+#pragma unroll
+        for (int cc = 0; cc < 2; cc++) {
+            uint32_t ylo[4], yhi[4];
+            unpack_codes(r[2 * cc], ylo);
+            unpack_codes(r[2 * cc + 1], yhi);
+            const int c = 2 * j + cc;
+#pragma unroll
+            for (int h2 = 0; h2 < 2; h2++) {
+                const uint32_t a[4] = {ylo[2 * h2], ylo[2 * h2 + 1], yhi[2 * h2], yhi[2 * h2 + 1]};
+                mma_16816(st.o[2 * c + h2], a, pb0, pb1);
+            }
+        }
+    }
+}
+
+// Fold (m, l, o) partial b (scaled by its own max) into the running partial a.
+__device__ __forceinline__ void merge_into(float am[2], float al[2], float ao[8][4],
+                                           const float bm[2], const float bl[2],
+                                           const float4 bo[8])
+{
+    float fa[2], fb[2];
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+        const float mn = fmaxf(am[e], bm[e]);
+        fa[e] = (mn == -INFINITY) ? 0.0f : ex2_approx(am[e] - mn);
+        fb[e] = (mn == -INFINITY) ? 0.0f : ex2_approx(bm[e] - mn);
+        am[e] = mn;
+        al[e] = al[e] * fa[e] + bl[e] * fb[e];
+    }
+#pragma unroll
+    for (int i = 0; i < 8; i++) {
+        ao[i][0] = ao[i][0] * fa[0] + bo[i].x * fb[0];
+        ao[i][1] = ao[i][1] * fa[1] + bo[i].y * fb[1];
+        ao[i][2] = ao[i][2] * fa[0] + bo[i].z * fb[0];
+        ao[i][3] = ao[i][3] * fa[1] + bo[i].w * fb[1];
+    }
+}
+
+// o_r = o / l, out = H o_r for the heads this thread holds; written to out[s][h G + 2t + e].
+__device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, int lane,
+                                         float o[8][4], const float l[2])
+{
+    const int g = lane >> 2, t = lane & 3;
+    const float inv[2] = {1.0f / l[0], 1.0f / l[1]};
+    // v[e][c][j]: head 2t + e, d = 32c + 4g + j
+    float v[2][4][4];
+#pragma unroll
+    for (int c = 0; c < 4; c++)
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            v[e][c][0] = o[2 * c][e] * inv[e];
+            v[e][c][1] = o[2 * c][2 + e] * inv[e];
+            v[e][c][2] = o[2 * c + 1][e] * inv[e];
+            v[e][c][3] = o[2 * c + 1][2 + e] * inv[e];
+        }
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+        // d bits 0, 1 (j) and 5, 6 (c) in registers
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+#pragma unroll
+            for (int jb = 1; jb <= 2; jb <<= 1)
+#pragma unroll
+                for (int j = 0; j < 4; j++)
+                    if ((j & jb) == 0) {
+                        const float a = v[e][c][j], b = v[e][c][j + jb];
+                        v[e][c][j] = a + b;
+                        v[e][c][j + jb] = a - b;
+                    }
+#pragma unroll
+        for (int cb = 1; cb <= 2; cb <<= 1)
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+                if ((c & cb) == 0)
+#pragma unroll
+                    for (int j = 0; j < 4; j++) {
+                        const float a = v[e][c][j], b = v[e][c + cb][j];
+                        v[e][c][j] = a + b;
+                        v[e][c + cb][j] = a - b;
+                    }
+        // d bits 2..4 (g) across lanes 4, 8, 16
+#pragma unroll
+        for (int gb = 1; gb <= 4; gb <<= 1) {
+            const bool high = (g & gb) != 0;
+#pragma unroll
+            for (int c = 0; c < 4; c++)
+#pragma unroll
+                for (int j = 0; j < 4; j++) {
+                    const float other = __shfl_xor_sync(0xFFFFFFFFu, v[e][c][j], 4 * gb);
+                    v[e][c][j] = high ? other - v[e][c][j] : v[e][c][j] + other;
+                }
+        }
+    }
+#pragma unroll
+    for (int e = 0; e < 2; e++) {
+        const int head = 2 * t + e;
+        if (head < p.group) {
+            float *dst = p.out + ((static_cast<int64_t>(s) * p.hq + h * p.group + head) * kHeadDim);
+#pragma unroll
+            for (int c = 0; c < 4; c++) {
+                const float4 val = make_float4(v[e][c][0] * kHadamardC, v[e][c][1] * kHadamardC,
+                                               v[e][c][2] * kHadamardC, v[e][c][3] * kHadamardC);
+                *reinterpret_cast<float4 *>(dst + 32 * c + 4 * g) = val;
+            }
+        }
+    }
+}
+
+__global__ void __launch_bounds__(kThreads, 3)
+    paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int g = lane >> 2, t = lane & 3;
+    const int S = p.num_seqs;
+    int32_t *pre = reinterpret_cast<int32_t *>(smem + kSmemPrefix);
+    volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + kSmemFlags);
+
+    // ---- 1. pages per sequence and their exclusive prefix ---------------------------------
+    {
+        const int per = (S + kThreads - 1) / kThreads;
+        const int s0 = tid * per, s1 = min(S, s0 + per);
+        int local = 0;
+        for (int s = s0; s < s1; s++) {
+            const int len = p.seq_lens[s];
+            const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
+            if (!ok && blockIdx.x == 0)
+                set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
+            local += ok ? (len + kPageSize - 1) / kPageSize : 0;
+        }
+        int incl = local;
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+            if (lane >= d)
+                incl += o;
+        }
+        if (lane == 31)
+            flags[warp] = incl;
+        __syncthreads();
+        int base = 0;
+        for (int w = 0; w < warp; w++)
+            base += flags[w];
+        int run = base + incl - local;
+        for (int s = s0; s < s1; s++) {
+            pre[s] = run;
+            const int len = p.seq_lens[s];
+            const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
+            run += ok ? (len + kPageSize - 1) / kPageSize : 0;
+        }
+        if (tid == kThreads - 1)
+            pre[S] = base + incl;
+        __syncthreads();
+    }
+    const int64_t hkv = p.hkv;
+    const int64_t P = hkv * pre[S];
+    const int64_t cta = blockIdx.x;
+
+    // ---- 2. sequences with no pages get a zero output ---------------------------------------
+    for (int s = blockIdx.x; s < S; s += gridDim.x) {
+        if (pre[s + 1] == pre[s]) {
+            float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<int64_t>(s) * p.hq * kHeadDim);
+            for (int i = tid; i < p.hq * kHeadDim / 4; i += kThreads)
+                dst[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        }
+    }
+    // Slice over C <= P / 4 CTAs so that every slice is non-empty (at least one page per
+    // warp); the remaining CTAs have no pages.  The merge counts rely on non-empty slices.
+    const int64_t C = max(int64_t(1), min(static_cast<int64_t>(gridDim.x), P / kWarps));
+    if (P == 0 || cta >= C)
+        return;
+    const int64_t Bc = (cta * P) / C, Bc1 = ((cta + 1) * P) / C;
+
+    // ---- 3. this warp's page stream: flat positions Bc + warp + 4 m ----------------------------
+    const uint32_t code0 = smem_u32(smem + kSmemCodes) + warp * kStages * kCodeBytes;
+    const uint32_t scale0 = smem_u32(smem + kSmemScales) + warp * kStages * kScaleBytes;
+    const uint32_t bar0 = smem_u32(smem + kSmemBars) + warp * kStages * 8;
+    if (lane == 0)
+        for (int i = 0; i < kStages; i++)
+            mbar_init(bar0 + 8 * i, 1);
+    mbar_init_fence();
+    __syncwarp();
+
+    const int64_t first = Bc + warp;
+    const int n_w = first < Bc1 ? static_cast<int>((Bc1 - first + kWarps - 1) / kWarps) : 0;
+
+    // tensor-map row (page * Hkv + h) * 32 of this warp's page m (-1 past the end)
+    auto lookup = [&](int m) -> int32_t {
+        if (m >= n_w)
+            return -1;
+        const int64_t pos = first + static_cast<int64_t>(kWarps) * m;
+        const int s = find_seq(pre, S, pos, hkv);
+        const int32_t n_s = pre[s + 1] - pre[s];
+        const int64_t u = pos - hkv * pre[s];
+        const int h = static_cast<int>(u / n_s);
+        const int i = static_cast<int>(u - static_cast<int64_t>(h) * n_s);
+        int32_t page = p.block_table[static_cast<int64_t>(s) * p.max_blocks + i];
+        if (page < 0 || page >= p.num_pages) {
+            set_status(p.status, SAW_DEV_BAD_PAGE);
+            page = 0;
+        }
+        return (page * p.hkv + h) * 32;
+    };
+
+    pdl_wait();   // the cache may be written by the kernel this one depends on
+
+    int32_t look_cur = lookup(lane), look_nxt = lookup(32 + lane);
+    int issued = 0;        // pages queued so far
+    bool aborted = false;
+    auto issue_next = [&]() {
+        if (issued >= n_w || aborted)
+            return;
+        const int m = issued;
+        if (m > 0 && (m & 31) == 0) {
+            look_cur = look_nxt;
+            look_nxt = lookup(m + 32 + lane);
+        }
+        const int32_t row = __shfl_sync(0xFFFFFFFFu, look_cur, m & 31);
+        if (lane == 0) {
+            const int stg = m % kStages;
+            const uint32_t bar = bar0 + 8 * stg;
+            mbar_arrive_expect_tx(bar, kTxBytes);
+            tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, row, bar);
+            bulk_g2s(scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(row) * 4,
+                     kScaleBytes, bar);
+        }
+        issued++;
+    };
+    for (int k = 0; k < kStages - 1; k++)
+        issue_next();
+
+    // ---- 4. pieces ----------------------------------------------------------------------------
+    int m = 0;
+    int64_t pos = Bc;
+    WarpState st;
+    while (pos < Bc1) {
+        const int s = find_seq(pre, S, pos, hkv);
+        const int32_t n_s = pre[s + 1] - pre[s];
+        const int64_t seq_start = hkv * pre[s];
+        const int h = static_cast<int>((pos - seq_start) / n_s);
+        const int64_t seg_start = seq_start + static_cast<int64_t>(h) * n_s;
+        const int64_t seg_end = seg_start + n_s;
+        const int64_t piece_end = seg_end < Bc1 ? seg_end : Bc1;
+        const int m_end = piece_end > first ? static_cast<int>((piece_end - first + kWarps - 1) / kWarps) : 0;
+        const int len = p.seq_lens[s];
+
+        state_reset(st);
+        if (m < m_end) {
+            uint32_t bq[8][2];
+            float sq[2];
+            load_query(p, s, h, g, t, bq, sq);
+            for (; m < m_end; m++) {
+                issue_next();
+                const int stg = m % kStages;
+                const bool ok = aborted ? false
+                                        : mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
+                if (!__all_sync(0xFFFFFFFFu, ok)) {
+                    if (!aborted && lane == 0)
+                        set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+                    aborted = true;
+                    continue;
+                }
+                const int i = static_cast<int>(first + static_cast<int64_t>(kWarps) * m - seg_start);
+                const int valid = len - kPageSize * i;
+                process_page(code0 + stg * kCodeBytes, scale0 + stg * kScaleBytes, valid, bq, sq,
+                             lane, st);
+                __syncwarp();
+            }
+            // reduce l and z over the 8 token rows (lanes differing in g)
+#pragma unroll
+            for (int e = 0; e < 2; e++) {
+#pragma unroll
+                for (int d = 4; d <= 16; d <<= 1) {
+                    st.l[e] += __shfl_xor_sync(0xFFFFFFFFu, st.l[e], d);
+                    st.z[e] += __shfl_xor_sync(0xFFFFFFFFu, st.z[e], d);
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 8; i++) {
+                st.o[i][0] += st.z[0];
+                st.o[i][1] += st.z[1];
+                st.o[i][2] += st.z[0];
+                st.o[i][3] += st.z[1];
+            }
+        }
+
+        // ---- merge the 4 warps' partials of this piece ----------------------------------------
+        __syncthreads();   // warp 0 has finished reading the previous piece's buffers
+        float *mO = reinterpret_cast<float *>(smem + kSmemMergeO);
+        float *mML = reinterpret_cast<float *>(smem + kSmemMergeML);
+        if (warp > 0) {
+            float4 *dst = reinterpret_cast<float4 *>(mO) + (warp - 1) * 8 * 32;
+#pragma unroll
+            for (int i = 0; i < 8; i++)
+                dst[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
+            if (g == 0) {
+                mML[(warp - 1) * 16 + 2 * t] = st.m[0];
+                mML[(warp - 1) * 16 + 2 * t + 1] = st.m[1];
+                mML[(warp - 1) * 16 + 8 + 2 * t] = st.l[0];
+                mML[(warp - 1) * 16 + 8 + 2 * t + 1] = st.l[1];
+            }
+        }
+        __syncthreads();
+        if (warp == 0) {
+            for (int w = 1; w < kWarps; w++) {
+                const float4 *src = reinterpret_cast<const float4 *>(mO) + (w - 1) * 8 * 32;
+                float4 bo[8];
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    bo[i] = src[i * 32 + lane];
+                const float bm[2] = {mML[(w - 1) * 16 + 2 * t], mML[(w - 1) * 16 + 2 * t + 1]};
+                const float bl[2] = {mML[(w - 1) * 16 + 8 + 2 * t], mML[(w - 1) * 16 + 8 + 2 * t + 1]};
+                merge_into(st.m, st.l, st.o, bm, bl, bo);
+            }
+            const int64_t seg = static_cast<int64_t>(s) * hkv + h;
+            const int64_t c_lo = cta_of(seg_start, P, C), c_hi = cta_of(seg_end - 1, P, C);
+            if (c_lo == c_hi) {
+                finalize(p, s, h, lane, st.o, st.l);
+            } else {
+                float *slot = p.partials + (seg + cta) * kSlotFloats;
+                float4 *so = reinterpret_cast<float4 *>(slot);
+#pragma unroll
+                for (int i = 0; i < 8; i++)
+                    so[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
+                if (g == 0) {
+                    slot[1024 + 2 * t] = st.m[0];
+                    slot[1024 + 2 * t + 1] = st.m[1];
+                    slot[1024 + 8 + 2 * t] = st.l[0];
+                    slot[1024 + 8 + 2 * t + 1] = st.l[1];
+                }
+                __threadfence();
+                __syncwarp();
+                uint32_t ticket = 0;
+                if (lane == 0)
+                    ticket = atomicAdd(p.tickets + seg, 1u);
+                ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
+                if (ticket == static_cast<uint32_t>(c_hi - c_lo)) {
+                    // last CTA of this segment: fold in every other CTA's partial
+                    __threadfence();
+                    for (int64_t c2 = c_lo; c2 <= c_hi; c2++) {
+                        if (c2 == cta)
+                            continue;
+                        const float *o2 = p.partials + (seg + c2) * kSlotFloats;
+                        const float4 *o24 = reinterpret_cast<const float4 *>(o2);
+                        float4 bo[8];
+#pragma unroll
+                        for (int i = 0; i < 8; i++)
+                            bo[i] = __ldcg(o24 + i * 32 + lane);
+                        const float bm[2] = {__ldcg(o2 + 1024 + 2 * t), __ldcg(o2 + 1024 + 2 * t + 1)};
+                        const float bl[2] = {__ldcg(o2 + 1032 + 2 * t), __ldcg(o2 + 1032 + 2 * t + 1)};
+                        merge_into(st.m, st.l, st.o, bm, bl, bo);
+                    }
+                    finalize(p, s, h, lane, st.o, st.l);
+                    if (lane == 0)
+                        p.tickets[seg] = 0u;   // ready for the next call
+                }
+            }
+        }
+        pos = piece_end;
+    }
+
+    // ---- 5. after an abort, let queued copies land before the CTA's shared memory is freed --
+    if (aborted) {
+        for (int k = m; k < issued; k++)
+            mbar_wait_bounded(bar0 + 8 * (k % kStages), (k / kStages) & 1, kWaitLimitNs / 10);
+    }
+}
+
+// Tensor map over kv_pages seen as [num_pages * Hkv * 32 rows][64 bytes], box 32 x 64
+// (one (page, kv head) block), 64-byte swizzle.
+PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+    if (fn == nullptr) {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }
+    return fn;
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs)
+{
+    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
+        return 0;
+    int dev = 0, sms = 0, occ = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+        return 0;
+    const size_t smem = decode_smem_bytes(num_seqs);
+    if (cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem)) != cudaSuccess ||
+        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, paged_decode_kernel, kThreads, smem) !=
+            cudaSuccess ||
+        occ <= 0)
+        return 0;
+    const size_t grid = static_cast<size_t>(sms) * occ;
+    const size_t segs = static_cast<size_t>(num_seqs) * num_kv_heads;
+    const size_t ticket_bytes = (segs * 4 + 255) & ~size_t(255);
+    return ticket_bytes + (grid + segs) * kSlotFloats * sizeof(float);
+}
+
+cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
+{
+    static thread_local struct {
+        const void *base = nullptr;
+        int64_t rows = 0;
+        CUtensorMap map;
+    } cache;
+    const int64_t rows = a.num_pages * a.num_kv_heads * 32;
+    if (cache.base != a.kv_pages || cache.rows != rows) {
+        auto encode = get_encode_fn();
+        if (encode == nullptr)
+            return cudaErrorNotSupported;
+        const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
+        const cuuint64_t strides[1] = {64};
+        const cuuint32_t box[2] = {64, 32};
+        const cuuint32_t estr[2] = {1, 1};
+        CUresult r = encode(&cache.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                            const_cast<uint8_t *>(a.kv_pages), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                            CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+        if (r != CUDA_SUCCESS) {
+            cache.base = nullptr;
+            return cudaErrorInvalidValue;
+        }
+        cache.base = a.kv_pages;
+        cache.rows = rows;
+    }
+
+    DecodeParams p;
+    p.q = static_cast<const uint16_t *>(a.q);
+    p.scales = static_cast<const uint8_t *>(a.scales);
+    p.block_table = a.block_table;
+    p.seq_lens = a.seq_lens;
+    p.out = a.out;
+    const size_t segs = static_cast<size_t>(a.num_seqs) * a.num_kv_heads;
+    const size_t ticket_bytes = (segs * 4 + 255) & ~size_t(255);
+    p.tickets = static_cast<uint32_t *>(a.workspace);
+    p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) + ticket_bytes);
+    p.status = a.status;
+    p.num_pages = a.num_pages;
+    p.max_blocks = a.max_blocks;
+    p.num_seqs = a.num_seqs;
+    p.hq = a.num_q_heads;
+    p.hkv = a.num_kv_heads;
+    p.group = a.num_q_heads / a.num_kv_heads;
+    p.q_mult = static_cast<float>(static_cast<double>(kHadamardC) * a.sm_scale * 1.4426950408889634);
+
+    int dev = 0, sms = 0, occ = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess)
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    const size_t smem = decode_smem_bytes(a.num_seqs);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, paged_decode_kernel, kThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (occ <= 0)
+        return cudaErrorInvalidConfiguration;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(sms * occ));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = programmatic ? 1 : 0;
+    e = cudaLaunchKernelEx(&cfg, paged_decode_kernel, cache.map, p);
+    if (e != cudaSuccess)
+        return e;
+    return cudaGetLastError();
+}
+
+}  // namespace saw

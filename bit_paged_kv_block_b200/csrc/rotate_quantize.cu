@@ -1,0 +1,327 @@
+// rotate_quantize.cu -- fused Hadamard rotation + token-wise INT4 quantization + paged scatter.
+//
+// Implements the fused rotation-quantization kernel of "SAW-INT4: System-Aware 4-Bit KV-Cache
+// Quantization for Real-World LLM Serving" (Research Findings): every new key and value head
+// vector is rotated by the normalised 128-point Hadamard transform, quantized token-wise to
+// asymmetric INT4 and written straight into its page of the paged KV cache.
+//
+// Results are bit-identical to the definition in saw.h:
+//   * the butterfly performs exactly the IEEE fp32 adds/subtracts of the natural-order
+//     Sylvester transform, stage h = 1, 2, ..., 64 in that order, then one multiply by
+//     fp32(1/sqrt(128)); two fp32 operations are issued per packed f32x2 instruction, each
+//     individually rounded, so the lane layout does not change any result;
+//   * scale = (max - min) / 15 uses the IEEE divide; the codes use a reciprocal, see
+//     quantize_fast() for why that gives the IEEE-divide code, and fall back to the IEEE
+//     divide where it might not.
+// This translation unit is compiled with -fmad=false as a second guard against contraction.
+//
+// Thread layout: two threads per head vector, 16 vectors (token, kv head) per warp.  Thread
+// half b of a vector holds the 64 elements j = 16a + 8b + r (a, r in 0..7): the 16-byte load a
+// covers elements 16a + 8b .. +7, so the two threads of a pair read one contiguous 32-byte
+// sector per load.  Stage h = 8 is the only one that crosses the pair (one shuffle); the
+// 64 elements are kept as 32 packed pairs X[8a + r] = (x[a][r], x[a + 4][r]) for a < 4.
+#include <cfloat>
+
+#include "saw_device.cuh"
+#include "saw_internal.h"
+
+namespace saw {
+namespace {
+
+constexpr int kRqThreads = 256;
+constexpr int kRqVecsPerWarp = 16;
+constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
+constexpr float kRoundMagic = 12582912.0f;           // 1.5 * 2^23
+// A code computed from the reciprocal is provably the IEEE-divide code unless the remainder
+// is within 2^-18 of one half (derivation at quantize_fast()).
+constexpr float kNearHalf = 0.5f - 1.0f / 262144.0f;
+
+__device__ __forceinline__ uint64_t shfl_xor_u64(uint32_t mask, uint64_t v, int delta)
+{
+    uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
+    lo = __shfl_xor_sync(mask, lo, delta);
+    hi = __shfl_xor_sync(mask, hi, delta);
+    return (static_cast<uint64_t>(hi) << 32) | lo;
+}
+
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+
+// Load this thread's 64 bf16 elements of one head vector (8 x 16 bytes).
+__device__ __forceinline__ void load_half_vec(const uint8_t *row, int b, uint4 raw[8])
+{
+#pragma unroll
+    for (int a = 0; a < 8; a++)
+        raw[a] = ldg_stream16(row + 32 * a + 16 * b);
+}
+
+__device__ __forceinline__ void to_pairs(const uint4 raw[8], uint64_t X[32])
+{
+#pragma unroll
+    for (int a = 0; a < 4; a++) {
+        const uint32_t lo[4] = {raw[a].x, raw[a].y, raw[a].z, raw[a].w};
+        const uint32_t hi[4] = {raw[a + 4].x, raw[a + 4].y, raw[a + 4].z, raw[a + 4].w};
+#pragma unroll
+        for (int q = 0; q < 4; q++) {
+            X[8 * a + 2 * q] = f2_pack(bf16_lo(lo[q]), bf16_lo(hi[q]));
+            X[8 * a + 2 * q + 1] = f2_pack(bf16_hi(lo[q]), bf16_hi(hi[q]));
+        }
+    }
+}
+
+// Normalised 128-point Hadamard transform of the vector held by a thread pair.
+// `mask` names the lanes executing this call (the full warp, or just this pair).
+__device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
+{
+    // h = 1, 2, 4: element bits r0..r2 = index bits 0..2 of X.
+#pragma unroll
+    for (int hb = 1; hb <= 4; hb <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            if ((i & hb) == 0) {
+                const uint64_t lo = X[i], hi = X[i + hb];
+                X[i] = f2_add(lo, hi);
+                X[i + hb] = f2_sub(lo, hi);
+            }
+        }
+    }
+    // h = 8: element bit 3 = the pair half b.  Low half: x + partner; high half:
+    // partner - x, computed as fma(x, -1, partner): the product is exact, so the single
+    // rounding gives exactly the IEEE difference.
+    {
+        const float sg = b ? -1.0f : 1.0f;
+        const uint64_t sgn = f2_pack(sg, sg);
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            const uint64_t other = shfl_xor_u64(mask, X[i], 1);
+            X[i] = f2_fma(X[i], sgn, other);
+        }
+    }
+    // h = 16, 32: element bits a0, a1 = index bits 3, 4 of X.
+#pragma unroll
+    for (int hb = 8; hb <= 16; hb <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            if ((i & hb) == 0) {
+                const uint64_t lo = X[i], hi = X[i + hb];
+                X[i] = f2_add(lo, hi);
+                X[i + hb] = f2_sub(lo, hi);
+            }
+        }
+    }
+    // h = 64: element bit a2 = the two halves of each packed pair.
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        X[i] = f2_pack(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+    }
+    const uint64_t cc = f2_pack(kHadamardC, kHadamardC);
+#pragma unroll
+    for (int i = 0; i < 32; i++)
+        X[i] = f2_mul(X[i], cc);
+}
+
+// Codes via the reciprocal.  With s = scale (a normal fp32 > 0), r = RN(1/s), d = RN(y - min)
+// and Q = d / s exactly (0 <= Q < 15 (1 + 2^-23)):
+//   t = RN(d r + M), M = 1.5 * 2^23: d r < 2^22, so t = M + k with k = rint(d r) (ties to even,
+//   since M is even) and k sits in the low mantissa bits of t;
+//   res = RN(d r - k) is the remainder to within 2^-26.
+// |d r - Q| <= Q 2^-24 < 2^-20 and |RN(Q) - Q| <= 2^-21, so if |res| < 0.5 - 2^-18 then
+// |RN(Q) - k| < 0.5 and rint(RN(d / s)) = k, which is the code the IEEE divide gives (no
+// clamp is needed: k <= 15).  Otherwise the caller recomputes with the IEEE divide.
+// On return X holds t (code = low 4 bits); the result is the largest |res| seen.
+__device__ __forceinline__ float quantize_fast(uint64_t X[32], float mn, float r)
+{
+    const uint64_t mn2 = f2_pack(mn, mn), r2 = f2_pack(r, r), m2 = f2_pack(kRoundMagic, kRoundMagic);
+    float worst = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        const uint64_t d = f2_sub(X[i], mn2);
+        const uint64_t t = f2_fma(d, r2, m2);
+        const uint64_t nk = f2_sub(m2, t);          // -k, exact
+        const uint64_t res = f2_fma(d, r2, nk);     // d r - k, one rounding
+        float a, c;
+        f2_unpack(res, a, c);
+        worst = fmax3(worst, fabsf(a), fabsf(c));
+        X[i] = t;
+    }
+    return worst;
+}
+
+// Codes through the IEEE divide, exactly as defined (used where quantize_fast cannot decide,
+// and when the scale is subnormal).
+__device__ __forceinline__ void quantize_exact(uint64_t X[32], float mn, float scale)
+{
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        float ql = rintf(__fdiv_rn(__fsub_rn(lo, mn), scale));
+        float qh = rintf(__fdiv_rn(__fsub_rn(hi, mn), scale));
+        ql = fminf(fmaxf(ql, 0.0f), 15.0f);
+        qh = fminf(fmaxf(qh, 0.0f), 15.0f);
+        X[i] = f2_pack(__fadd_rn(ql, kRoundMagic), __fadd_rn(qh, kRoundMagic));
+    }
+}
+
+// Gather the low nibbles of t_0..t_7 (codes of elements r = 0..7) into one word, element r at
+// bits 4r: bytes are [k0 | k1 << 4, k2 | k3 << 4, ...] (even index in the low nibble).
+__device__ __forceinline__ uint32_t pack8(const uint32_t tt[8])
+{
+    const uint32_t e01 = __byte_perm(tt[0], tt[2], 0x0040);
+    const uint32_t e23 = __byte_perm(tt[4], tt[6], 0x0040);
+    const uint32_t even = __byte_perm(e01, e23, 0x5410);   // [k0, k2, k4, k6]
+    const uint32_t o01 = __byte_perm(tt[1], tt[3], 0x0040);
+    const uint32_t o23 = __byte_perm(tt[5], tt[7], 0x0040);
+    const uint32_t odd = __byte_perm(o01, o23, 0x5410);    // [k1, k3, k5, k7]
+    return even | (odd << 4);
+}
+
+struct RqParams {
+    const uint8_t *k;
+    const uint8_t *v;
+    const int64_t *slot_mapping;
+    int64_t num_vecs;        // T * Hkv
+    int32_t hkv;
+    int64_t num_slots;       // num_pages * 16
+    uint8_t *kv_pages;
+    uint32_t *scales;        // fp16x2 (scale, zero) per row
+    uint32_t *status;
+};
+
+// Quantize the vector (held rotated in X) and store codes + scale for one of K (sel 0) / V (1).
+__device__ __forceinline__ void quantize_store(uint64_t X[32], const uint8_t *src_row, int b,
+                                               int lane, bool store, int64_t row,
+                                               const RqParams &p)
+{
+    // min / max over the pair's 128 elements
+    float mn = FLT_MAX, mx = -FLT_MAX;
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        mn = fmin3(mn, lo, hi);
+        mx = fmax3(mx, lo, hi);
+    }
+    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+
+    float scale = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
+    const bool degenerate = !(scale != 0.0f);
+    if (degenerate)
+        scale = 0.0f;                               // canonical +0
+    const float zero = __fadd_rn(mn, 0.0f);         // a zero minimum is stored as +0
+
+    bool exact = false;
+    if (degenerate) {
+        const uint64_t m2 = f2_pack(kRoundMagic, kRoundMagic);
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+            X[i] = m2;                              // every code 0
+    } else if (scale < FLT_MIN) {
+        exact = true;                               // subnormal scale: IEEE divide throughout
+    } else {
+        const float worst = quantize_fast(X, mn, __frcp_rn(scale));
+        exact = !(worst < kNearHalf);
+    }
+    // The two threads of a pair decide together (the recomputation shuffles within the pair).
+    const bool pair_exact = __shfl_xor_sync(0xFFFFFFFFu, exact ? 1 : 0, 1) != 0 || exact;
+    if (pair_exact) {
+        const uint32_t pair_mask = 3u << (lane & ~1);
+        uint4 raw[8];
+        load_half_vec(src_row, b, raw);
+        to_pairs(raw, X);
+        fwht128(X, b, pair_mask);
+        quantize_exact(X, mn, scale);
+    }
+
+    if (!store)
+        return;
+    uint8_t *dst = p.kv_pages + row * kRowBytes;
+#pragma unroll
+    for (int a = 0; a < 8; a++) {
+        uint32_t tt[8];
+#pragma unroll
+        for (int r = 0; r < 8; r++) {
+            float lo, hi;
+            f2_unpack(X[8 * (a & 3) + r], lo, hi);
+            tt[r] = __float_as_uint(a < 4 ? lo : hi);
+        }
+        *reinterpret_cast<uint32_t *>(dst + 8 * a + 4 * b) = pack8(tt);
+    }
+    if (b == 0) {
+        const __half2 sz = __halves2half2(__float2half_rn(scale), __float2half_rn(zero));
+        p.scales[row] = half2_as_u32(sz);
+    }
+}
+
+__global__ void __launch_bounds__(kRqThreads, 2) rotate_quantize_kernel(const RqParams p)
+{
+    pdl_launch_dependents();
+    const int lane = threadIdx.x & 31;
+    const int b = lane & 1;
+    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kRqThreads + threadIdx.x) >> 5;
+    const int64_t vec_raw = warp_global * kRqVecsPerWarp + (lane >> 1);
+    if (warp_global * kRqVecsPerWarp >= p.num_vecs)
+        return;                                      // whole warp past the end
+    const bool in_range = vec_raw < p.num_vecs;
+    const int64_t vec = in_range ? vec_raw : p.num_vecs - 1;   // tail lanes recompute the last
+    const int64_t tok = vec / p.hkv;
+    const int h = static_cast<int>(vec - tok * p.hkv);
+
+    const int64_t slot = p.slot_mapping[tok];
+    bool store = in_range && slot >= 0;
+    if (store && slot >= p.num_slots) {
+        if (b == 0)
+            set_status(p.status, SAW_DEV_BAD_SLOT);
+        store = false;
+    }
+    const int64_t page = store ? slot / kPageSize : 0;
+    const int64_t off = store ? slot - page * kPageSize : 0;
+    const int64_t row_k = ((page * p.hkv + h) * 2 + 0) * kPageSize + off;
+    const int64_t row_v = row_k + kPageSize;
+
+    const uint8_t *k_row = p.k + vec * (kHeadDim * 2);
+    const uint8_t *v_row = p.v + vec * (kHeadDim * 2);
+    uint4 raw_k[8], raw_v[8];
+    load_half_vec(k_row, b, raw_k);
+    load_half_vec(v_row, b, raw_v);
+
+    uint64_t X[32];
+    to_pairs(raw_k, X);
+    fwht128(X, b, 0xFFFFFFFFu);
+    quantize_store(X, k_row, b, lane, store, row_k, p);
+
+    to_pairs(raw_v, X);
+    fwht128(X, b, 0xFFFFFFFFu);
+    quantize_store(X, v_row, b, lane, store, row_v, p);
+}
+
+}  // namespace
+
+cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t stream,
+                                   bool trigger_dependents)
+{
+    (void)trigger_dependents;   // the kernel always releases dependents at its start
+    RqParams p;
+    p.k = static_cast<const uint8_t *>(a.k);
+    p.v = static_cast<const uint8_t *>(a.v);
+    p.slot_mapping = a.slot_mapping;
+    p.num_vecs = a.num_tokens * a.num_kv_heads;
+    p.hkv = a.num_kv_heads;
+    p.num_slots = a.num_pages * kPageSize;
+    p.kv_pages = a.kv_pages;
+    p.scales = static_cast<uint32_t *>(a.scales);
+    p.status = a.status;
+    if (p.num_vecs == 0)
+        return cudaSuccess;
+    const int64_t warps = (p.num_vecs + kRqVecsPerWarp - 1) / kRqVecsPerWarp;
+    const int64_t blocks = (warps * 32 + kRqThreads - 1) / kRqThreads;
+    if (blocks > 0x7FFFFFFF)
+        return cudaErrorInvalidValue;
+    rotate_quantize_kernel<<<static_cast<unsigned>(blocks), kRqThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
+
+}  // namespace saw

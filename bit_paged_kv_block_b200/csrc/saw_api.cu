@@ -1,0 +1,236 @@
+// saw_api.cu -- the extern "C" entry points declared in include/saw.h.
+//
+// Argument validation, workspace sizing and kernel launches.  Nothing here allocates device
+// memory; every launch is asynchronous on the caller's stream.
+#include <cmath>
+#include <cstdint>
+
+#include "saw.h"
+#include "saw_internal.h"
+
+namespace {
+
+bool aligned(const void *p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
+
+int check_cache(const saw_cache_desc *c)
+{
+    if (c == nullptr || c->num_kv_heads <= 0 || c->num_pages < 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (c->head_dim != 128 || c->page_size != 16)
+        return SAW_ERR_UNSUPPORTED;
+    // tensor-map rows (page * Hkv + h) * 32 must stay below 2^31
+    if (c->num_pages > (int64_t(1) << 31) / (int64_t(c->num_kv_heads) * 32))
+        return SAW_ERR_UNSUPPORTED;
+    return SAW_OK;
+}
+
+int check_append(const saw_cache_desc *cache, const void *k, const void *v,
+                 const int64_t *slot_mapping, int64_t num_tokens, const uint8_t *kv_pages,
+                 const void *scales)
+{
+    if (num_tokens < 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (num_tokens == 0)
+        return SAW_OK;
+    if (!k || !v || !slot_mapping || !kv_pages || !scales)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(kv_pages, 16) || !aligned(scales, 16) ||
+        !aligned(slot_mapping, 8))
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (num_tokens > INT64_MAX / (int64_t(cache->num_kv_heads) * 256))
+        return SAW_ERR_INVALID_ARGUMENT;
+    return SAW_OK;
+}
+
+int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                 const uint8_t *kv_pages, const void *scales, const int32_t *block_table,
+                 int32_t max_blocks, const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                 const float *out, const void *workspace, size_t workspace_bytes)
+{
+    if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (num_q_heads / cache->num_kv_heads > 8)
+        return SAW_ERR_UNSUPPORTED;
+    if (!std::isfinite(sm_scale))
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (num_seqs == 0)
+        return SAW_OK;
+    if (!q || !kv_pages || !scales || !block_table || !seq_lens || !out || max_blocks <= 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (!aligned(q, 16) || !aligned(kv_pages, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+        !aligned(block_table, 4) || !aligned(seq_lens, 4))
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (cache->num_pages == 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (int64_t(max_blocks) * 16 > INT32_MAX)
+        return SAW_ERR_INVALID_ARGUMENT;
+    const size_t need = saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+    if (need == 0)
+        return SAW_ERR_CUDA;
+    if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
+        return SAW_ERR_WORKSPACE;
+    return SAW_OK;
+}
+
+saw::DecodeArgs decode_args(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                            const uint8_t *kv_pages, const void *scales,
+                            const int32_t *block_table, int32_t max_blocks,
+                            const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                            float *out, void *workspace, size_t workspace_bytes,
+                            uint32_t *dev_status)
+{
+    saw::DecodeArgs a;
+    a.q = q;
+    a.kv_pages = kv_pages;
+    a.scales = scales;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks;
+    a.seq_lens = seq_lens;
+    a.num_seqs = num_seqs;
+    a.num_q_heads = num_q_heads;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.num_pages = cache->num_pages;
+    a.sm_scale = sm_scale;
+    a.out = out;
+    a.workspace = workspace;
+    a.workspace_bytes = workspace_bytes;
+    a.status = dev_status;
+    return a;
+}
+
+}  // namespace
+
+extern "C" {
+
+int saw_version(void) { return 100; }
+
+const char *saw_status_string(int status)
+{
+    switch (status) {
+    case SAW_OK:
+        return "ok";
+    case SAW_ERR_INVALID_ARGUMENT:
+        return "invalid argument (null pointer, bad size or alignment, Hq not a multiple of Hkv)";
+    case SAW_ERR_UNSUPPORTED:
+        return "unsupported shape (head_dim must be 128, page_size 16, Hq/Hkv at most 8)";
+    case SAW_ERR_CUDA:
+        return "CUDA runtime error";
+    case SAW_ERR_WORKSPACE:
+        return "workspace missing, misaligned or too small";
+    default:
+        return "unknown status";
+    }
+}
+
+int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const void *v,
+                              const int64_t *slot_mapping, int64_t num_tokens,
+                              uint8_t *kv_pages, void *scales, uint32_t *dev_status,
+                              void *stream)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k, v, slot_mapping, num_tokens, kv_pages, scales);
+    if (rc != SAW_OK || num_tokens == 0)
+        return rc;
+    saw::RotateQuantizeArgs a;
+    a.k = k;
+    a.v = v;
+    a.slot_mapping = slot_mapping;
+    a.num_tokens = num_tokens;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.num_pages = cache->num_pages;
+    a.kv_pages = kv_pages;
+    a.scales = scales;
+    a.status = dev_status;
+    return saw::launch_rotate_quantize(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? SAW_OK
+               : SAW_ERR_CUDA;
+}
+
+size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                        int32_t num_seqs)
+{
+    if (check_cache(cache) != SAW_OK || num_q_heads <= 0 ||
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 8)
+        return 0;
+    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+}
+
+int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
+{
+    if (workspace == nullptr && workspace_bytes != 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (workspace_bytes == 0)
+        return SAW_OK;
+    return cudaMemsetAsync(workspace, 0, workspace_bytes, static_cast<cudaStream_t>(stream)) ==
+                   cudaSuccess
+               ? SAW_OK
+               : SAW_ERR_CUDA;
+}
+
+int saw_paged_decode_attn(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                          const uint8_t *kv_pages, const void *scales,
+                          const int32_t *block_table, int32_t max_blocks_per_seq,
+                          const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                          float *out, void *workspace, size_t workspace_bytes,
+                          uint32_t *dev_status, void *stream)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    const saw::DecodeArgs a =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    return saw::launch_paged_decode(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? SAW_OK
+               : SAW_ERR_CUDA;
+}
+
+int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                    const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                    int64_t num_new_tokens, uint8_t *kv_pages, void *scales,
+                    const int32_t *block_table, int32_t max_blocks_per_seq,
+                    const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
+                    void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                    void *stream)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k_new, v_new, slot_mapping, num_new_tokens, kv_pages, scales);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
+    if (rc != SAW_OK)
+        return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool appended = num_new_tokens > 0;
+    if (appended) {
+        saw::RotateQuantizeArgs a;
+        a.k = k_new;
+        a.v = v_new;
+        a.slot_mapping = slot_mapping;
+        a.num_tokens = num_new_tokens;
+        a.num_kv_heads = cache->num_kv_heads;
+        a.num_pages = cache->num_pages;
+        a.kv_pages = kv_pages;
+        a.scales = scales;
+        a.status = dev_status;
+        if (saw::launch_rotate_quantize(a, s, true) != cudaSuccess)
+            return SAW_ERR_CUDA;
+    }
+    if (num_seqs == 0)
+        return SAW_OK;
+    const saw::DecodeArgs d =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    return saw::launch_paged_decode(d, s, appended) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+}
+
+}  // extern "C"

@@ -1,0 +1,52 @@
+// saw_internal.h -- launchers shared between the C-ABI layer and the kernel translation units.
+#pragma once
+
+#include <cstddef>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace saw {
+
+struct RotateQuantizeArgs {
+    const void *k;               // bf16 [T][Hkv][128]
+    const void *v;               // bf16 [T][Hkv][128]
+    const int64_t *slot_mapping; // [T]
+    int64_t num_tokens;
+    int32_t num_kv_heads;
+    int64_t num_pages;
+    uint8_t *kv_pages;           // [num_pages][Hkv][2][16][64]
+    void *scales;                // fp16 [num_pages][Hkv][2][16][2]
+    uint32_t *status;            // nullable
+};
+
+struct DecodeArgs {
+    const void *q;               // bf16 [S][Hq][128]
+    const uint8_t *kv_pages;
+    const void *scales;
+    const int32_t *block_table;  // [S][max_blocks]
+    int32_t max_blocks;
+    const int32_t *seq_lens;     // [S]
+    int32_t num_seqs;
+    int32_t num_q_heads;
+    int32_t num_kv_heads;
+    int64_t num_pages;
+    float sm_scale;
+    float *out;                  // fp32 [S][Hq][128]
+    void *workspace;
+    size_t workspace_bytes;
+    uint32_t *status;
+};
+
+// Queue the rotate+quantize+scatter kernel.  `trigger_dependents` makes the kernel release
+// a programmatic dependent launch early.  Returns a cudaError_t.
+cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t stream,
+                                   bool trigger_dependents);
+
+// Workspace bytes the decode kernel needs on the current device (0 if the shape is invalid).
+size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs);
+
+// Queue the decode kernel; `programmatic` launches it as a programmatic dependent of the
+// previous kernel on the stream.  Returns a cudaError_t.
+cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
+
+}  // namespace saw

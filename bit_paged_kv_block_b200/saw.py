@@ -1,0 +1,232 @@
+"""Python binding of libsaw (ctypes), with the C ABI's names.
+
+Argument marshalling only: each function checks tensor devices, dtypes, shapes and contiguity,
+then passes raw device pointers and the current CUDA stream to the C entry point.  Every step
+of the path runs in the library's CUDA kernels; there is no CPU path.  Importing this module
+loads libsaw.so from this package directory (building it with nvcc if it is missing) and raises
+if that fails.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+
+import torch
+
+from . import build as _build
+
+HEAD_DIM = 128
+PAGE_SIZE = 16
+
+SAW_OK = 0
+SAW_ERR_INVALID_ARGUMENT = 1
+SAW_ERR_UNSUPPORTED = 2
+SAW_ERR_CUDA = 3
+SAW_ERR_WORKSPACE = 4
+
+SAW_DEV_BAD_SLOT = 0x1
+SAW_DEV_BAD_PAGE = 0x2
+SAW_DEV_BAD_SEQ_LEN = 0x4
+SAW_DEV_WAIT_TIMEOUT = 0x8
+
+
+class SawError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: status {status}: {saw_status_string(status)}")
+
+
+class saw_cache_desc(ctypes.Structure):
+    _fields_ = [("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int64)]
+
+
+def _open_library() -> ctypes.CDLL:
+    path = _build.LIB
+    if not _build.up_to_date():
+        try:
+            _build.build()
+        except Exception as exc:  # the CUDA library is required: fail loudly
+            raise ImportError(f"libsaw.so is missing and could not be built: {exc}") from exc
+    lib = ctypes.CDLL(path)
+    P, i32, i64, f32, sz = (ctypes.c_void_p, ctypes.c_int32, ctypes.c_int64, ctypes.c_float,
+                            ctypes.c_size_t)
+    D = ctypes.POINTER(saw_cache_desc)
+    lib.saw_version.argtypes = []
+    lib.saw_version.restype = ctypes.c_int
+    lib.saw_status_string.argtypes = [ctypes.c_int]
+    lib.saw_status_string.restype = ctypes.c_char_p
+    lib.saw_rotate_quantize_paged.argtypes = [D, P, P, P, i64, P, P, P, P]
+    lib.saw_rotate_quantize_paged.restype = ctypes.c_int
+    lib.saw_paged_decode_workspace_bytes.argtypes = [D, i32, i32]
+    lib.saw_paged_decode_workspace_bytes.restype = sz
+    lib.saw_paged_decode_workspace_init.argtypes = [P, sz, P]
+    lib.saw_paged_decode_workspace_init.restype = ctypes.c_int
+    lib.saw_paged_decode_attn.argtypes = [D, i32, P, P, P, P, i32, P, i32, f32, P, P, sz, P, P]
+    lib.saw_paged_decode_attn.restype = ctypes.c_int
+    lib.saw_decode_step.argtypes = [D, i32, P, P, P, P, i64, P, P, P, i32, P, i32, f32, P, P,
+                                    sz, P, P]
+    lib.saw_decode_step.restype = ctypes.c_int
+    return lib
+
+
+lib = _open_library()
+
+
+def saw_version() -> int:
+    return int(lib.saw_version())
+
+
+def saw_status_string(status: int) -> str:
+    return lib.saw_status_string(int(status)).decode()
+
+
+def _check(rc: int, where: str) -> None:
+    if rc != SAW_OK:
+        raise SawError(rc, where)
+
+
+def _ptr(t) -> ctypes.c_void_p:
+    return ctypes.c_void_p(0 if t is None else t.data_ptr())
+
+
+def _stream(stream) -> ctypes.c_void_p:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream))
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim=None, cuda=True) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if cuda and t.device.type != "cuda":
+        raise ValueError(f"{name} must be on a CUDA device")
+    if ndim is not None and t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dimensions, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def cache_desc(kv_pages: torch.Tensor) -> saw_cache_desc:
+    """Descriptor of a cache tensor uint8 [num_pages][Hkv][2][16][64]."""
+    _need(kv_pages, "kv_pages", torch.uint8, 5, cuda=False)
+    num_pages, hkv, two, page, half = kv_pages.shape
+    if two != 2 or half * 2 != HEAD_DIM:
+        raise ValueError(f"kv_pages must be [num_pages][Hkv][2][16][64], got {tuple(kv_pages.shape)}")
+    return saw_cache_desc(int(hkv), HEAD_DIM, int(page), int(num_pages))
+
+
+def allocate_cache(num_pages: int, num_kv_heads: int, device="cuda"):
+    """Empty cache tensors: kv_pages uint8 [P][Hkv][2][16][64], scales fp16 [P][Hkv][2][16][2]."""
+    kv = torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, HEAD_DIM // 2), dtype=torch.uint8,
+                     device=device)
+    sc = torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, 2), dtype=torch.float16,
+                     device=device)
+    return kv, sc
+
+
+def saw_rotate_quantize_paged(k, v, slot_mapping, kv_pages, scales, dev_status=None,
+                              stream=None) -> None:
+    """Rotate, quantize and scatter new tokens k, v (bf16 [T][Hkv][128]) into the cache."""
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    desc = cache_desc(kv_pages)
+    T = k.shape[0]
+    if tuple(k.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
+        raise ValueError("k and v must be [T][Hkv][128] matching the cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have one entry per token")
+    if tuple(scales.shape) != (desc.num_pages, desc.num_kv_heads, 2, PAGE_SIZE, 2):
+        raise ValueError("scales must be [num_pages][Hkv][2][16][2]")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    rc = lib.saw_rotate_quantize_paged(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(slot_mapping),
+                                       T, _ptr(kv_pages), _ptr(scales), _ptr(dev_status),
+                                       _stream(stream))
+    _check(rc, "saw_rotate_quantize_paged")
+
+
+def saw_paged_decode_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,
+                                     num_pages: int = 1) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, int(num_pages))
+    return int(lib.saw_paged_decode_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
+                                                    int(num_seqs)))
+
+
+def saw_paged_decode_workspace_init(workspace: torch.Tensor, stream=None) -> None:
+    _need(workspace, "workspace", torch.uint8, 1)
+    rc = lib.saw_paged_decode_workspace_init(_ptr(workspace), workspace.numel(), _stream(stream))
+    _check(rc, "saw_paged_decode_workspace_init")
+
+
+def allocate_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: int,
+                       device="cuda") -> torch.Tensor:
+    """A zero-initialised decode workspace for this shape on the current device."""
+    n = saw_paged_decode_workspace_bytes(num_kv_heads, num_q_heads, num_seqs)
+    if n == 0:
+        raise SawError(SAW_ERR_CUDA, "saw_paged_decode_workspace_bytes")
+    ws = torch.empty(n, dtype=torch.uint8, device=device)
+    saw_paged_decode_workspace_init(ws)
+    return ws
+
+
+def _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace, dev_status):
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(out, "out", torch.float32, 3)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    desc = cache_desc(kv_pages)
+    S, hq, d = q.shape
+    if d != HEAD_DIM or tuple(out.shape) != (S, hq, HEAD_DIM):
+        raise ValueError("q and out must be [S][Hq][128]")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    return desc, S, hq
+
+
+def saw_paged_decode_attn(q, kv_pages, scales, block_table, seq_lens, out, workspace,
+                          sm_scale=None, dev_status=None, stream=None) -> None:
+    """Decode attention of q (bf16 [S][Hq][128]) over the INT4 paged cache into out (fp32)."""
+    desc, S, hq = _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace,
+                                 dev_status)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_paged_decode_attn(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages), _ptr(scales),
+                                   _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
+                                   float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                   _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_paged_decode_attn")
+
+
+def saw_decode_step(q, k_new, v_new, slot_mapping, kv_pages, scales, block_table, seq_lens, out,
+                    workspace, sm_scale=None, dev_status=None, stream=None) -> None:
+    """Append k_new / v_new (bf16 [T][Hkv][128]) at slot_mapping, then decode q."""
+    desc, S, hq = _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace,
+                                 dev_status)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    T = k_new.shape[0]
+    if tuple(k_new.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [T][Hkv][128] matching the cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have one entry per new token")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_decode_step(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new),
+                             _ptr(slot_mapping), T, _ptr(kv_pages), _ptr(scales),
+                             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
+                             float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                             _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_decode_step")

@@ -1,0 +1,144 @@
+/*
+ * saw.h -- C ABI of libsaw: SAW-INT4 paged INT4 KV-cache compression on NVIDIA B200 (sm_100a).
+ *
+ * The method ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving",
+ * Research Findings; restated on "Memory compression method reducing KV-cache size...", Core
+ * Innovation and Summary) quantizes every new key/value head vector token-wise to INT4 after a
+ * block-diagonal Hadamard rotation, inside one fused kernel that writes straight into a paged
+ * KV cache, and reads that cache back with fused attention.  This library implements the two
+ * halves of that path:
+ *
+ *   saw_rotate_quantize_paged  rotate + quantize + scatter new K/V vectors into the cache
+ *   saw_paged_decode_attn      decode attention over the INT4 paged cache (split-K, GQA)
+ *   saw_decode_step            one serving step: append one token per sequence, then decode
+ *
+ * Fixed build parameters (the pages give no numbers; these are the library's definition):
+ *   head_dim D = 128 = Hadamard block B; H is the Sylvester Hadamard matrix in natural order,
+ *   normalised by 1/sqrt(128), applied as an fp32 butterfly (stages h = 1, 2, ..., 64,
+ *   (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]), then a multiply by fp32(1/sqrt(128)),
+ *   every step one IEEE fp32 operation); per (token, kv head) and separately for K and V:
+ *   scale = (max - min) / 15 and zero = min in fp32, stored as fp16 (round to nearest even);
+ *   code_i = clamp(rint((y_i - min) / scale), 0, 15) with IEEE division and ties to even;
+ *   a vector whose fp32 scale is 0 stores scale +0 and all codes 0; a zero minimum is stored
+ *   as +0; two codes per byte, the even index in the low nibble; pages of 16 tokens.
+ *
+ * Memory layout (all buffers caller-owned device memory, C-contiguous, 16-byte aligned):
+ *   k, v (new tokens)   bf16   [T][Hkv][128]
+ *   slot_mapping        int64  [T]        slot = page * 16 + offset; slot < 0 skips the token
+ *   kv_pages            uint8  [num_pages][Hkv][2 (K, V)][16][64]
+ *                        so one (page, kv head) is one contiguous 2 KiB block: 1 KiB of K
+ *                        codes then 1 KiB of V codes, 64 bytes per token row
+ *   scales              fp16   [num_pages][Hkv][2 (K, V)][16][2 (scale, zero)]
+ *                        128 bytes per (page, kv head)
+ *   q                   bf16   [S][Hq][128]    query head hq reads kv head hq / (Hq / Hkv)
+ *   block_table         int32  [S][max_blocks_per_seq]  logical block -> page
+ *   seq_lens            int32  [S]    tokens of each sequence in the cache (including the
+ *                                     token appended by this step), 0 <= len <= 16 * max_blocks
+ *   out                 fp32   [S][Hq][128]
+ *
+ * Ownership and threading: the library allocates no device memory.  Every call is
+ * asynchronous on the given stream (a cudaStream_t passed as void*; NULL is the legacy
+ * default stream) and returns as soon as its kernels are queued.  Calls on different streams
+ * that share a workspace race.
+ *
+ * Errors: every entry point returns a saw_status.  Host-side checks (null pointers, sizes,
+ * alignment, unsupported shapes) return before anything is queued.  Errors that only the
+ * device can see -- a slot or page id out of range, a sequence length out of range, a bounded
+ * wait that gave up -- never trap: the kernel skips the offending access, ORs a SAW_DEV_* bit
+ * into *dev_status (when dev_status is not NULL) and carries on; the caller reads the word
+ * after synchronising.  NaN or Inf inputs are not supported (their codes are unspecified).
+ */
+#ifndef SAW_H_
+#define SAW_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum saw_status {
+    SAW_OK = 0,
+    SAW_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
+    SAW_ERR_UNSUPPORTED = 2,      /* head_dim != 128, page_size != 16, Hq / Hkv > 8 */
+    SAW_ERR_CUDA = 3,             /* a CUDA runtime call or kernel launch failed */
+    SAW_ERR_WORKSPACE = 4         /* workspace missing or smaller than required */
+} saw_status;
+
+/* Bits ORed into *dev_status by the kernels. */
+#define SAW_DEV_BAD_SLOT 0x1u     /* slot_mapping[t] >= num_pages * 16: token skipped */
+#define SAW_DEV_BAD_PAGE 0x2u     /* block_table entry outside [0, num_pages): page 0 read */
+#define SAW_DEV_BAD_SEQ_LEN 0x4u  /* seq_lens[s] < 0 or > 16 * max_blocks: output zeroed */
+#define SAW_DEV_WAIT_TIMEOUT 0x8u /* a bounded wait on a page copy gave up */
+
+typedef struct saw_cache_desc {
+    int32_t num_kv_heads; /* Hkv >= 1 */
+    int32_t head_dim;     /* must be 128 */
+    int32_t page_size;    /* must be 16 */
+    int64_t num_pages;    /* pages in kv_pages / scales; num_pages * Hkv * 32 < 2^31 */
+} saw_cache_desc;
+
+/* Rotate, quantize and scatter T new tokens into the paged cache.
+ * Follows "SAW-INT4" (Research Findings): the fused rotation-quantization kernel that writes
+ * token-wise INT4 codes of Hadamard-rotated vectors directly into the paged KV cache.
+ * k, v: bf16 [T][Hkv][128] device; slot_mapping: int64 [T] device; kv_pages, scales: the
+ * cache (device, updated in place); dev_status: device uint32 or NULL.  T == 0 is a no-op.
+ * Codes and scales are bit-identical to the definition above for every finite input. */
+int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const void *v,
+                              const int64_t *slot_mapping, int64_t num_tokens,
+                              uint8_t *kv_pages, void *scales, uint32_t *dev_status,
+                              void *stream);
+
+/* Bytes of workspace saw_paged_decode_attn / saw_decode_step need for this shape on the
+ * current device (split-K partial results and per-(seq, kv head) merge counters).  Returns 0
+ * for an unsupported or invalid shape. */
+size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                        int32_t num_seqs);
+
+/* Zero a workspace (cudaMemsetAsync on the stream).  Call once after allocating it: each
+ * decode call leaves its merge counters at zero for the next one, so the workspace can be
+ * reused without re-initialising unless a call was aborted. */
+int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
+
+/* Decode attention over the INT4 paged cache.
+ * Follows "SAW-INT4" (Research Findings: fused attention execution over a paged cache) and
+ * "BitDecoding-FP4" (abstract: stacked query heads over paged KV).  For each sequence s and
+ * query head hq (kv head h = hq / G, G = Hq / Hkv <= 8):
+ *     q_r = H q,   s_t = sm_scale * <q_r, zero_t + code_t * scale_t>  for t < seq_lens[s],
+ *     o_r = softmax(s) . (zero_t + code_t * scale_t) over the V side,   out = H o_r.
+ * The kernel computes in fp16 x fp16 -> fp32 tensor-core tiles on raw codes with the scale
+ * and zero applied in fp32 afterwards; results agree with an fp64 evaluation of the same
+ * formula to about 1e-3.  A sequence with seq_lens[s] == 0 gets an all-zero output.
+ * workspace: device memory of at least saw_paged_decode_workspace_bytes(), zeroed once by
+ * saw_paged_decode_workspace_init(). */
+int saw_paged_decode_attn(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                          const uint8_t *kv_pages, const void *scales,
+                          const int32_t *block_table, int32_t max_blocks_per_seq,
+                          const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                          float *out, void *workspace, size_t workspace_bytes,
+                          uint32_t *dev_status, void *stream);
+
+/* One serving step: saw_rotate_quantize_paged on the num_new_tokens tokens (k_new, v_new,
+ * slot_mapping), then saw_paged_decode_attn, queued back to back on the stream (the decode
+ * kernel is launched as a programmatic dependent of the append so that its launch and
+ * prologue overlap the append).  seq_lens must already count the appended tokens. */
+int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                    const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                    int64_t num_new_tokens, uint8_t *kv_pages, void *scales,
+                    const int32_t *block_table, int32_t max_blocks_per_seq,
+                    const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
+                    void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                    void *stream);
+
+/* Human-readable text of a saw_status (never NULL). */
+const char *saw_status_string(int status);
+
+/* Library ABI version: 100 * major + minor. */
+int saw_version(void);
+
+#ifdef __cplusplus
+} /* extern "C" */
+#endif
+
+#endif /* SAW_H_ */

@@ -1,0 +1,77 @@
+"""Shared helpers for the parity tests: the same seeded inputs go to the CUDA path (through
+the C ABI) and to the CPU oracle.  No expected value here comes from the CUDA path."""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+import torch
+
+import oracle
+from bit_paged_kv_block_b200 import synth
+
+NTHREADS = max(1, os.cpu_count() or 1)
+CANARY_CODE = 0xA5
+CANARY_SCALE = 0x5A5A
+
+# attention tolerance against the fp64 oracle
+MAX_ABS_TOL = 1e-2
+MEAN_ABS_TOL = 1e-3
+
+
+def u16(t: torch.Tensor) -> np.ndarray:
+    return t.detach().cpu().contiguous().view(torch.int16).numpy().view(np.uint16)
+
+
+def oracle_cache(wl, tokens="all", k=None, v=None, rotate=True):
+    """Oracle cache (numpy) holding the selected tokens of the workload, canary elsewhere."""
+    if k is None:
+        k = synth.kv_values(wl, "K", tokens=tokens)
+    if v is None:
+        v = synth.kv_values(wl, "V", tokens=tokens)
+    seq, pos = synth.token_index(wl, tokens)
+    slots = synth.slot_mapping(wl, seq, pos)
+    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
+    pages[:] = CANARY_CODE
+    scales[:] = CANARY_SCALE
+    bad = oracle.rotate_quantize_paged(u16(k), u16(v), slots, pages, scales, rotate=rotate,
+                                       nthreads=NTHREADS)
+    assert bad == 0
+    return pages, scales
+
+
+def device_cache_from(pages: np.ndarray, scales: np.ndarray, device):
+    kv = torch.from_numpy(pages).to(device)
+    sc = torch.from_numpy(scales.view(np.int16)).view(torch.float16).to(device)
+    return kv, sc
+
+
+def canary_device_cache(wl, device):
+    from bit_paged_kv_block_b200 import saw
+    kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, device)
+    kv.fill_(CANARY_CODE)
+    sc.view(torch.int16).fill_(CANARY_SCALE)
+    return kv, sc
+
+
+def attention_errors(got: np.ndarray, want: np.ndarray):
+    d = np.abs(got.astype(np.float64) - want)
+    return float(d.max()), float(d.mean())
+
+
+def assert_attention_close(got, want, what=""):
+    mx, mean = attention_errors(got, want)
+    assert np.isfinite(got).all(), f"{what}: non-finite output"
+    assert mx <= MAX_ABS_TOL and mean <= MEAN_ABS_TOL, f"{what}: max {mx:.3e} mean {mean:.3e}"
+    return mx, mean
+
+
+def subset(wl, seqs):
+    """The workload restricted to the given sequences (same pages and page ids)."""
+    seqs = np.asarray(seqs)
+    sub = synth.Workload(**{**wl.__dict__})
+    sub.num_seqs = len(seqs)
+    sub.seq_lens = wl.seq_lens[seqs].copy()
+    sub.new_tokens = wl.new_tokens[seqs].copy()
+    sub.block_table = np.ascontiguousarray(wl.block_table[seqs])
+    return sub

@@ -1,0 +1,109 @@
+"""The C-ABI library builds, loads and exports every entry point that include/saw.h declares;
+host-side argument checks return their status codes before any CUDA call (no GPU needed)."""
+import ctypes
+import os
+import re
+
+import pytest
+
+from bit_paged_kv_block_b200 import build, saw
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(__file__)), "include", "saw.h")
+
+
+def declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(saw_[a-z0-9_]+)\s*\(", text)))
+
+
+def test_library_is_built_in_tree():
+    assert build.up_to_date()
+    assert os.path.dirname(build.LIB) == os.path.dirname(saw.__file__)
+
+
+def test_every_declared_symbol_is_exported():
+    names = declared_functions()
+    assert {"saw_rotate_quantize_paged", "saw_paged_decode_attn", "saw_decode_step",
+            "saw_paged_decode_workspace_bytes", "saw_paged_decode_workspace_init",
+            "saw_status_string", "saw_version"} <= set(names)
+    lib = ctypes.CDLL(build.LIB)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_version_and_status_strings():
+    assert saw.saw_version() == 100
+    for code in range(5):
+        assert saw.saw_status_string(code)
+    assert saw.saw_status_string(99) == "unknown status"
+
+
+def _desc(hkv=8, d=128, p=16, pages=64):
+    return saw.saw_cache_desc(hkv, d, p, pages)
+
+
+def _rq(desc, T=4, k=16, v=16, slots=16, pages=16, scales=16):
+    P = ctypes.c_void_p
+    return saw.lib.saw_rotate_quantize_paged(
+        None if desc is None else ctypes.byref(desc), P(k), P(v), P(slots), T, P(pages),
+        P(scales), None, None)
+
+
+def test_append_argument_checks():
+    assert _rq(None) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _rq(_desc(d=64)) == saw.SAW_ERR_UNSUPPORTED
+    assert _rq(_desc(p=32)) == saw.SAW_ERR_UNSUPPORTED
+    assert _rq(_desc(hkv=0)) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _rq(_desc(pages=1 << 30)) == saw.SAW_ERR_UNSUPPORTED
+    assert _rq(_desc(), T=-1) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _rq(_desc(), k=0) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _rq(_desc(), k=8) == saw.SAW_ERR_INVALID_ARGUMENT          # not 16-byte aligned
+    assert _rq(_desc(), slots=4) == saw.SAW_ERR_INVALID_ARGUMENT      # not 8-byte aligned
+    assert _rq(_desc(), T=0, k=0, v=0, slots=0, pages=0, scales=0) == saw.SAW_OK  # no-op
+
+
+def _dec(desc, hq=32, S=2, q=16, out=16, bt=16, lens=16, ws=256, ws_bytes=1 << 20,
+         max_blocks=4, sm_scale=0.088):
+    P = ctypes.c_void_p
+    return saw.lib.saw_paged_decode_attn(
+        ctypes.byref(desc), hq, P(q), P(16), P(16), P(bt), max_blocks, P(lens), S, sm_scale,
+        P(out), P(ws), ws_bytes, None, None)
+
+
+def test_decode_argument_checks():
+    d = _desc()
+    assert _dec(d, hq=12) == saw.SAW_ERR_INVALID_ARGUMENT             # Hq % Hkv
+    assert _dec(d, hq=72) == saw.SAW_ERR_UNSUPPORTED                  # G = 9
+    assert _dec(d, S=-1) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, q=0) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, q=8) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, out=4) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, lens=2) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, max_blocks=0) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, sm_scale=float("nan")) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _dec(d, S=0) == saw.SAW_OK                                  # nothing to do
+    assert _dec(_desc(pages=0)) == saw.SAW_ERR_INVALID_ARGUMENT
+
+
+def test_workspace_init_checks():
+    assert saw.lib.saw_paged_decode_workspace_init(None, 16, None) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert saw.lib.saw_paged_decode_workspace_init(None, 0, None) == saw.SAW_OK
+
+
+def test_workspace_bytes_rejects_bad_shapes():
+    f = saw.lib.saw_paged_decode_workspace_bytes
+    assert f(ctypes.byref(_desc()), 12, 4) == 0
+    assert f(ctypes.byref(_desc()), 72, 4) == 0
+    assert f(ctypes.byref(_desc(d=64)), 32, 4) == 0
+
+
+def test_python_binding_rejects_cpu_tensors():
+    import torch
+    k = torch.zeros(2, 8, 128, dtype=torch.bfloat16)
+    kv = torch.zeros(4, 8, 2, 16, 64, dtype=torch.uint8)
+    sc = torch.zeros(4, 8, 2, 16, 2, dtype=torch.float16)
+    with pytest.raises(ValueError):
+        saw.saw_rotate_quantize_paged(k, k, torch.zeros(2, dtype=torch.int64), kv, sc)
+    with pytest.raises(TypeError):
+        saw.saw_rotate_quantize_paged(k.float(), k, torch.zeros(2, dtype=torch.int64), kv, sc)

@@ -1,0 +1,136 @@
+"""GPU parity of the rotate + quantize + scatter kernel against the CPU oracle: packed codes and
+fp16 scale / zero must be bit-identical ("SAW-INT4", Research Findings: the fused
+rotation-quantization kernel writing token-wise INT4 into the paged cache)."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_paged_kv_block_b200 import synth
+from helpers import CANARY_CODE, CANARY_SCALE, NTHREADS, canary_device_cache, oracle_cache, u16
+
+pytestmark = pytest.mark.gpu
+
+
+def gpu_append(wl, device, tokens="all", k=None, v=None, status=None):
+    from bit_paged_kv_block_b200 import saw
+    if k is None:
+        k = synth.kv_values(wl, "K", tokens=tokens)
+    if v is None:
+        v = synth.kv_values(wl, "V", tokens=tokens)
+    seq, pos = synth.token_index(wl, tokens)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(device)
+    kv, sc = canary_device_cache(wl, device)
+    saw.saw_rotate_quantize_paged(k.to(device), v.to(device), slots, kv, sc, dev_status=status)
+    torch.cuda.synchronize()
+    return kv, sc
+
+
+def assert_cache_equal(kv, sc, pages, scales):
+    got_p = kv.cpu().numpy()
+    got_s = u16(sc)
+    if not np.array_equal(got_p, pages):
+        bad = np.argwhere(got_p != pages)
+        raise AssertionError(f"{len(bad)} code bytes differ, first at {bad[0].tolist()}: "
+                             f"{got_p[tuple(bad[0])]:#x} vs {pages[tuple(bad[0])]:#x}")
+    if not np.array_equal(got_s, scales):
+        bad = np.argwhere(got_s != scales)
+        raise AssertionError(f"{len(bad)} scale words differ, first at {bad[0].tolist()}: "
+                             f"{got_s[tuple(bad[0])]:#x} vs {scales[tuple(bad[0])]:#x}")
+
+
+@pytest.mark.parametrize("name", ["tiny", "prefill", "decode", "long", "serving"])
+def test_rotate_quantize_bit_exact_workloads(cuda_device, name):
+    wl = synth.make_workload(name)
+    k = synth.kv_values(wl, "K")
+    v = synth.kv_values(wl, "V")
+    kv, sc = gpu_append(wl, cuda_device, k=k, v=v)
+    pages, scales = oracle_cache(wl, k=k, v=v)
+    assert_cache_equal(kv, sc, pages, scales)
+
+
+def _custom_tokens(T, Hkv, maker, seed=0):
+    g = torch.Generator().manual_seed(seed)
+    return maker(g, (T, Hkv, 128)).to(torch.bfloat16)
+
+
+@pytest.mark.parametrize("kind", ["small_ints", "zeros_and_constants", "tiny_magnitudes",
+                                  "huge_range", "signed_zero", "single_spike"])
+def test_rotate_quantize_edge_values(cuda_device, kind):
+    """Inputs chosen to hit exact ties, degenerate vectors, subnormal scales and the
+    reciprocal-path fallback; every code must still equal the IEEE-divide definition."""
+    T, Hkv = 203, 3                  # ragged: 609 vectors, not a multiple of 16 per warp
+    g = torch.Generator().manual_seed(7)
+    if kind == "small_ints":         # rotated values are multiples of c: many exact halves
+        x = torch.randint(-3, 4, (T, Hkv, 128), generator=g).float()
+    elif kind == "zeros_and_constants":
+        x = torch.zeros(T, Hkv, 128)
+        x[1::3] = torch.randn(T, Hkv, 1, generator=g)[1::3]        # constants
+        x[2::5, :, 7] = 1.0                                          # unit vectors
+    elif kind == "tiny_magnitudes":  # fp32 scales near / below the normal range
+        x = torch.randn(T, Hkv, 128, generator=g) * 1e-37
+        x[::2] *= 1e-2
+    elif kind == "huge_range":
+        x = torch.randn(T, Hkv, 128, generator=g) * (10.0 ** torch.randint(-3, 4, (T, Hkv, 1), generator=g))
+    elif kind == "signed_zero":
+        x = torch.zeros(T, Hkv, 128)
+        x[::2, :, 3] = -0.0
+        x[1::2, :, 5] = 1.0
+        x[::4] = -x[::4]
+    else:
+        x = torch.zeros(T, Hkv, 128)
+        x[torch.arange(T), :, torch.arange(T) % 128] = 50.0
+    k = x.to(torch.bfloat16)
+    v = (x.flip(-1) * 0.5).to(torch.bfloat16)
+    wl = synth.custom(kind, [T], num_q_heads=Hkv, num_kv_heads=Hkv, new_tokens=[T],
+                      num_pages=(T + 15) // 16 + 3)
+    kv, sc = gpu_append(wl, cuda_device, k=k, v=v)
+    pages, scales = oracle_cache(wl, k=k, v=v)
+    assert_cache_equal(kv, sc, pages, scales)
+
+
+def test_slots_skip_and_out_of_range(cuda_device):
+    """slot < 0 skips the token, slot >= num_pages * 16 skips it and sets SAW_DEV_BAD_SLOT;
+    everything not written keeps its canary."""
+    from bit_paged_kv_block_b200 import saw
+    T, Hkv, num_pages = 57, 2, 6
+    k = torch.randn(T, Hkv, 128).to(torch.bfloat16)
+    v = torch.randn(T, Hkv, 128).to(torch.bfloat16)
+    rng = np.random.default_rng(3)
+    slots = rng.permutation(num_pages * 16)[:T].astype(np.int64)
+    slots[::7] = -1
+    slots[5] = num_pages * 16 + 3
+    wl = synth.custom("slots", [T], num_q_heads=Hkv, num_kv_heads=Hkv, new_tokens=[T],
+                      num_pages=num_pages)
+    kv, sc = canary_device_cache(wl, cuda_device)
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    saw.saw_rotate_quantize_paged(k.to(cuda_device), v.to(cuda_device),
+                                  torch.from_numpy(slots).to(cuda_device), kv, sc,
+                                  dev_status=status)
+    torch.cuda.synchronize()
+    assert int(status.item()) == saw.SAW_DEV_BAD_SLOT
+    pages, scales = oracle.empty_cache(num_pages, Hkv)
+    pages[:] = CANARY_CODE
+    scales[:] = CANARY_SCALE
+    assert oracle.rotate_quantize_paged(u16(k), u16(v), slots, pages, scales) == 1
+    assert_cache_equal(kv, sc, pages, scales)
+
+
+def test_overwrite_in_place_and_repeat(cuda_device):
+    """Writing the same tokens twice gives the same bytes (the kernel is deterministic and
+    overwrites whole rows)."""
+    wl = synth.make_workload("tiny")
+    kv1, sc1 = gpu_append(wl, cuda_device)
+    kv2, sc2 = gpu_append(wl, cuda_device)
+    assert torch.equal(kv1, kv2) and torch.equal(sc1.view(torch.int16), sc2.view(torch.int16))
+
+
+def test_empty_append_is_noop(cuda_device):
+    from bit_paged_kv_block_b200 import saw
+    wl = synth.make_workload("tiny")
+    kv, sc = canary_device_cache(wl, cuda_device)
+    e = torch.empty(0, wl.num_kv_heads, 128, dtype=torch.bfloat16, device=cuda_device)
+    saw.saw_rotate_quantize_paged(e, e, torch.empty(0, dtype=torch.int64, device=cuda_device),
+                                  kv, sc)
+    torch.cuda.synchronize()
+    assert bool((kv == CANARY_CODE).all())
