@@ -1,0 +1,441 @@
+"""Benchmark of the SAW-INT4 paged INT4 KV-cache hot path on B200.
+
+One step = one serving step of the decode workload (Llama-3-8B layer shape: 64 sequences with
+lengths uniform on {512..8192}, 32 query / 8 kv heads, head_dim 128, 16-token pages): the new
+token of every sequence is rotated, INT4-quantized and scattered into the paged cache, then
+decode attention runs over the whole INT4 cache (saw_decode_step through the C ABI).  The
+headline value is decode tokens/s (sequences served per second, summed over ranks).  The same
+line also reports the rotate+quantize kernel's GB/s on the prefill workload (32 x 2048 tokens,
+8 kv heads), both kernels' fractions of the HBM roofline, an end-to-end number through host
+buffers, and the CPU oracle as a baseline.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+
+With --impl reference the script times the CPU oracle (the plain C reference in oracle/) on a
+bounded sample of the same workload and prints its line; under torchrun only rank 0 does so.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "INT4 paged decode tokens/s"
+UNIT = "tokens/s"
+HBM_TARGET_GBS = 8000.0            # the 8 TB/s roofline the targets are stated against
+CODE_ROW_BYTES = 64
+BYTES_PER_TOKEN_HEAD_DECODE = 2 * CODE_ROW_BYTES + 2 * 4          # K+V codes + scale/zero
+BYTES_PER_TOKEN_HEAD_APPEND = 2 * 128 * 2 + 2 * CODE_ROW_BYTES + 2 * 4   # bf16 in, codes+scales out
+WORKLOAD_TEXT = ("decode step, Llama-3-8B layer shape: batch 64, seq_lens uniform 512-8192, "
+                 "32 q / 8 kv heads, head_dim 128, page 16, one new token per seq appended "
+                 "(rotate + INT4 quantize + scatter) then INT4 paged decode attention; bf16 "
+                 "N(0,1) with 4 key outlier channels x U[10,30]")
+CPU_SAMPLE_SEQS = 8
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10000)
+    ap.add_argument("--warmup", type=int, default=100)
+    ap.add_argument("--impl", default="saw", choices=["saw", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    return ap.parse_args()
+
+
+def dist_env():
+    return (int(os.environ.get("RANK", "0")), int(os.environ.get("LOCAL_RANK", "0")),
+            int(os.environ.get("WORLD_SIZE", "1")))
+
+
+# ---- byte accounting (algorithmic bytes, not measured traffic) ----------------------------
+
+def decode_bytes(wl) -> int:
+    lens = wl.seq_lens.astype(np.int64)
+    pages = (lens + 15) // 16
+    per_seq = wl.num_q_heads * 128 * (2 + 4) + 4 + 4 * pages
+    return int((wl.num_kv_heads * lens * BYTES_PER_TOKEN_HEAD_DECODE).sum() + per_seq.sum())
+
+
+def append_bytes(num_tokens: int, hkv: int) -> int:
+    return num_tokens * (hkv * BYTES_PER_TOKEN_HEAD_APPEND + 8)
+
+
+# ---- clocks ----------------------------------------------------------------------------------
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    REASONS = {
+        "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
+        "hw_slowdown": 0x8, "sync_boost": 0x10, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+        "display_clock_setting": 0x100,
+    }
+
+    def __init__(self, device_index: int, period_s: float = 0.01):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.period = period_s
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            self.max_mhz = None
+        self._stop = threading.Event()
+        self._t = None
+
+    def _run(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for name, b in self.REASONS.items():
+                    if bits & b and name != "gpu_idle":
+                        self.reasons.add(name)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.ok:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *exc):
+        self._stop.set()
+        if self._t is not None:
+            self._t.join()
+
+    def summary(self):
+        return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
+                "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                "samples": len(self.samples), "source": "NVML during the timed region"}
+
+
+# ---- roofline denominators -----------------------------------------------------------------
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["hbm_gbs"]), "measured"
+    except Exception:
+        return 6650.0, "fallback"
+
+
+def kernel_traffic(kernel: str, units: float):
+    """dram bytes per launch from the committed ncu summary, if it was taken on the current
+    kernel source (scaled by `units` / the captured units); else None."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f)[kernel]
+        src = os.path.join(ROOT, "bit_paged_kv_block_b200", "csrc", rec["source"])
+        with open(src, "rb") as f:
+            digest = hashlib.sha256(f.read()).hexdigest()
+        if digest != rec["source_sha256"]:
+            return None
+        return rec["dram_bytes_per_launch"] * units / rec["units"]
+    except Exception:
+        return None
+
+
+# ---- the CPU oracle baseline ------------------------------------------------------------
+
+def oracle_sample(wl, seed_seqs: int = CPU_SAMPLE_SEQS):
+    """Oracle-built history cache for the first `seed_seqs` sequences (CPU only)."""
+    import oracle
+    from bit_paged_kv_block_b200 import synth
+    sub = synth.Workload(**{**wl.__dict__})
+    sel = np.arange(seed_seqs)
+    sub.num_seqs = seed_seqs
+    sub.seq_lens = wl.seq_lens[sel].copy()
+    sub.new_tokens = wl.new_tokens[sel].copy()
+    sub.block_table = np.ascontiguousarray(wl.block_table[sel])
+    nthreads = os.cpu_count() or 1
+    bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
+    seq, pos = synth.token_index(sub, "history")
+    oracle.rotate_quantize_paged(bits(synth.kv_values(sub, "K", tokens="history")),
+                                 bits(synth.kv_values(sub, "V", tokens="history")),
+                                 synth.slot_mapping(sub, seq, pos), pages, scales,
+                                 nthreads=nthreads)
+    seq, pos = synth.token_index(sub, "new")
+    new = (bits(synth.kv_values(sub, "K", tokens="new")),
+           bits(synth.kv_values(sub, "V", tokens="new")), synth.slot_mapping(sub, seq, pos))
+    q = bits(synth.q_values(wl))[sel].copy()
+    return sub, pages, scales, new, q, nthreads
+
+
+def oracle_step(sub, pages, scales, new, q, nthreads):
+    import oracle
+    oracle.rotate_quantize_paged(new[0], new[1], new[2], pages, scales, nthreads=nthreads)
+    return oracle.decode_fp64(q, pages, scales, sub.block_table, sub.seq_lens,
+                              nthreads=nthreads)
+
+
+def cpu_baseline(wl, min_seconds: float = 10.0):
+    sub, pages, scales, new, q, nthreads = oracle_sample(wl)
+    oracle_step(sub, pages, scales, new, q, nthreads)             # warm
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        oracle_step(sub, pages, scales, new, q, nthreads)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= min_seconds:
+            break
+    return {"value": sub.num_seqs * reps / el, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+            "sample": f"first {sub.num_seqs} of the 64 sequences ({int(sub.seq_lens.sum())} "
+                      f"cached tokens): oracle append of their new tokens + fp64 decode, "
+                      f"{reps} repetitions in {el:.1f} s, OpenMP over {nthreads} host threads"}
+
+
+def run_reference(args):
+    rank, _, world = dist_env()
+    if rank != 0:
+        return 0
+    from bit_paged_kv_block_b200 import synth
+    wl = synth.make_workload("decode", seed=0)
+    # size each step's sample so that warmup + K steps stay within about two minutes
+    sub, pages, scales, new, q, nthreads = oracle_sample(wl, 1)
+    t0 = time.perf_counter()
+    oracle_step(sub, pages, scales, new, q, nthreads)
+    per_seq = max(time.perf_counter() - t0, 1e-4)
+    n = int(max(1, min(CPU_SAMPLE_SEQS, 120.0 / (per_seq * (args.steps + args.warmup)))))
+    if n > 1:
+        sub, pages, scales, new, q, nthreads = oracle_sample(wl, n)
+    for _ in range(max(args.warmup, 0)):
+        oracle_step(sub, pages, scales, new, q, nthreads)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle_step(sub, pages, scales, new, q, nthreads)
+    el = time.perf_counter() - t0
+    value = sub.num_seqs * args.steps / el
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT,
+        "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": 1e3 * el / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT, "sample_seqs": sub.num_seqs},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": nthreads, "kind": "oracle",
+                         "sample": f"each step: first {sub.num_seqs} of the 64 sequences, "
+                                   f"oracle append + fp64 decode"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+# ---- the CUDA path --------------------------------------------------------------------------
+
+def run_saw(args):
+    import torch
+    from bit_paged_kv_block_b200 import saw, synth
+
+    rank, local_rank, world = dist_env()
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    pg = None
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=dev)
+        pg = dist
+
+    # ---- inputs: each rank serves its own batch (weak scaling, no exchange on the path) ----
+    wl = synth.make_workload("decode", seed=rank)
+    kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
+    seq, pos = synth.token_index(wl, "history")
+    saw.saw_rotate_quantize_paged(synth.kv_values(wl, "K", tokens="history", device=dev),
+                                  synth.kv_values(wl, "V", tokens="history", device=dev),
+                                  torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(dev),
+                                  kv, sc)
+    seq, pos = synth.token_index(wl, "new")
+    k_new = synth.kv_values(wl, "K", tokens="new", device=dev)
+    v_new = synth.kv_values(wl, "V", tokens="new", device=dev)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(dev)
+    q = synth.q_values(wl, device=dev)
+    table = torch.from_numpy(wl.block_table).to(dev)
+    lens = torch.from_numpy(wl.seq_lens).to(dev)
+    out = torch.empty((wl.num_seqs, wl.num_q_heads, 128), dtype=torch.float32, device=dev)
+    ws = saw.allocate_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
+    status = torch.zeros(1, dtype=torch.int32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step():
+        saw.saw_decode_step(q, k_new, v_new, slots, kv, sc, table, lens, out, ws,
+                            dev_status=status, stream=stream)
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+
+    # ---- timed region: exactly K steps, device events, max over ranks ----------------------
+    clocks = ClockSampler(local_rank)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    if pg:
+        pg.barrier()
+    torch.cuda.synchronize()
+    with clocks:
+        e0.record(stream)
+        for _ in range(args.steps):
+            step()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    ms = e0.elapsed_time(e1)
+    if pg:
+        pg.barrier()
+        t = torch.tensor([ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        ms = float(t.item())
+    if int(status.item()) != 0:
+        raise RuntimeError(f"device status {int(status.item()):#x}")
+    ms_per_step = ms / args.steps
+    value = world * wl.num_seqs / (ms_per_step / 1e3)
+
+    # ---- per-kernel durations (same inputs, events around each launch) ---------------------
+    n_kt = max(20, min(args.steps, 400))
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_kt)]
+    for i in range(n_kt):
+        ev[i][0].record(stream)
+        saw.saw_rotate_quantize_paged(k_new, v_new, slots, kv, sc, dev_status=status,
+                                      stream=stream)
+        ev[i][1].record(stream)
+        saw.saw_paged_decode_attn(q, kv, sc, table, lens, out, ws, dev_status=status,
+                                  stream=stream)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize()
+    t_append = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    t_decode = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    dec_bytes = decode_bytes(wl)
+    peak_gbs, peak_kind = measured_peaks()
+    dec_gbs = dec_bytes / (t_decode * 1e-3) / 1e9
+    roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peak_gbs, "unit": "GB/s",
+                "frac": dec_gbs / peak_gbs, "peak_kind": peak_kind,
+                "kernel": "paged_decode_kernel", "algorithmic_bytes_per_launch": dec_bytes,
+                "launch_ms": t_decode, "frac_of_8TBps": dec_gbs / HBM_TARGET_GBS,
+                "traffic": kernel_traffic("paged_decode_kernel", int(wl.seq_lens.sum()))}
+
+    # ---- prefill rotate+quantize throughput (the write side at full bandwidth) -------------
+    pre = synth.make_workload("prefill", seed=rank)
+    pkv, psc = saw.allocate_cache(pre.num_pages, pre.num_kv_heads, dev)
+    pseq, ppos = synth.token_index(pre, "all")
+    pk = synth.kv_values(pre, "K", device=dev)
+    pv = synth.kv_values(pre, "V", device=dev)
+    pslots = torch.from_numpy(synth.slot_mapping(pre, pseq, ppos)).to(dev)
+    for _ in range(3):
+        saw.saw_rotate_quantize_paged(pk, pv, pslots, pkv, psc, stream=stream)
+    n_rq = 50
+    evq = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_rq)]
+    for i in range(n_rq):
+        evq[i][0].record(stream)
+        saw.saw_rotate_quantize_paged(pk, pv, pslots, pkv, psc, stream=stream)
+        evq[i][1].record(stream)
+    torch.cuda.synchronize()
+    t_rq = statistics.mean(e[0].elapsed_time(e[1]) for e in evq)
+    rq_bytes = append_bytes(pre.total_tokens, pre.num_kv_heads)
+    rq_gbs = rq_bytes / (t_rq * 1e-3) / 1e9
+    rot_quant = {"workload": "prefill: 32 seqs x 2048 tokens, 8 kv heads, head_dim 128, page 16, "
+                             "pages by seeded permutation",
+                 "GBps": rq_gbs, "frac_of_8TBps": rq_gbs / HBM_TARGET_GBS,
+                 "frac_of_measured_peak": rq_gbs / peak_gbs, "launch_ms": t_rq,
+                 "algorithmic_bytes_per_launch": rq_bytes,
+                 "traffic": kernel_traffic("rotate_quantize_kernel", pre.total_tokens)}
+    del pk, pv, pkv, psc
+
+    # ---- end to end through the public API with host buffers ------------------------------
+    pin = lambda t: t.cpu().pin_memory()
+    h_q, h_k, h_v, h_slots, h_table, h_lens = (pin(q), pin(k_new), pin(v_new), pin(slots),
+                                               pin(table), pin(lens))
+    h_out = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+    h2d = sum(t.numel() * t.element_size() for t in (h_q, h_k, h_v, h_slots, h_table, h_lens))
+    d2h = h_out.numel() * h_out.element_size()
+
+    def e2e_step():
+        q.copy_(h_q, non_blocking=True)
+        k_new.copy_(h_k, non_blocking=True)
+        v_new.copy_(h_v, non_blocking=True)
+        slots.copy_(h_slots, non_blocking=True)
+        table.copy_(h_table, non_blocking=True)
+        lens.copy_(h_lens, non_blocking=True)
+        step()
+        h_out.copy_(out, non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    n_e2e = max(20, min(args.steps, 2000))
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_e2e):
+        e2e_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = e0.elapsed_time(e1) / n_e2e
+    if pg:
+        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
+        pg.all_reduce(t, op=pg.ReduceOp.MAX)
+        e2e_ms = float(t.item())
+    e2e = {"value": world * wl.num_seqs / (e2e_ms / 1e3), "unit": UNIT,
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
+           "ms_per_step": e2e_ms}
+
+    base = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        base = cpu_baseline(wl)
+
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": max(args.warmup, 3), "ms_per_step": ms_per_step, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "int4 codes; f32 quantizer; f16 mma, f32 accumulate",
+        "data": "synthetic",
+        "config": {"workload": WORKLOAD_TEXT, "batch": wl.num_seqs,
+                   "kv_tokens_per_step": int(wl.seq_lens.sum()), "parallelism": f"dp{world}",
+                   "l2": "inputs larger than L2 (the decode reads "
+                         f"{dec_bytes / 1e6:.0f} MB of INT4 cache per step > 126 MB)"},
+        "kv_tokens_per_s": world * int(wl.seq_lens.sum()) / (ms_per_step / 1e3),
+        "step_GBps": (dec_bytes + append_bytes(wl.num_seqs, wl.num_kv_heads)) / (ms_per_step * 1e-3) / 1e9,
+        "roofline": roofline,
+        "rot_quant": rot_quant,
+        "append_launch_ms": t_append,
+        "e2e": e2e,
+        "gpu_launches": 2 * args.steps,
+        "clocks": clocks.summary(),
+        "cpu_baseline": base,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+    if pg:
+        pg.barrier()
+        pg.destroy_process_group()
+    return 0
+
+
+def main():
+    args = parse()
+    if args.impl == "reference":
+        return run_reference(args)
+    return run_saw(args)
+
+
+if __name__ == "__main__":
+    sys.exit(main())

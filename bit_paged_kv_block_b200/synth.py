@@ -191,13 +191,14 @@ def _flat_offsets(wl: Workload) -> np.ndarray:
 
 
 def kv_values(wl: Workload, which: str = "K", *, tokens: str = "all",
-              device="cpu", chunk: int = 1 << 16) -> torch.Tensor:
+              device="cpu", chunk: int = 4096) -> torch.Tensor:
     """bf16 [T][Hkv][D] values of the selected tokens (see token_index).
 
     Each token's values depend only on (seed, workload name, K|V, its flat index among all
-    cached tokens), so 'history' + 'new' together give exactly 'all'.  Values are drawn in
-    chunks of `chunk` flat tokens from per-chunk generators on `device` (the CPU and CUDA
-    generators differ, so parity tests draw on the CPU)."""
+    cached tokens), so 'history' + 'new' together give exactly 'all', and a sequence's values
+    do not depend on how many sequences follow it.  Values are drawn in whole chunks of `chunk`
+    flat tokens from per-chunk generators on `device` (the CPU and CUDA generators differ, so
+    parity tests draw on the CPU)."""
     Hkv, D = wl.num_kv_heads, wl.head_dim
     seq, pos = token_index(wl, tokens)
     flat = _flat_offsets(wl)[seq] + pos
@@ -210,10 +211,9 @@ def kv_values(wl: Workload, which: str = "K", *, tokens: str = "all",
     dev = torch.device(device)
     for c in np.unique(flat // chunk).tolist():
         sel = torch.nonzero((flat_t // chunk) == c).flatten()
-        n_in_chunk = int(min(chunk, int(_flat_offsets(wl)[-1]) - c * chunk))
         g = torch.Generator(device=dev)
         g.manual_seed(_seed_for(wl.seed, wl.name, which, c))
-        vals = torch.randn((n_in_chunk, Hkv, D), generator=g, dtype=torch.float32, device=dev)
+        vals = torch.randn((chunk, Hkv, D), generator=g, dtype=torch.float32, device=dev)
         if which == "K":
             for h in range(Hkv):
                 vals[:, h, chan[h].to(dev)] *= fac[h].to(dev)
