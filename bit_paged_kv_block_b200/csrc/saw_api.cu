@@ -117,6 +117,9 @@ const char *saw_status_string(int status)
         return "CUDA runtime error";
     case SAW_ERR_WORKSPACE:
         return "workspace missing, misaligned or too small";
+    case SAW_ERR_SCRATCH_LIMIT:
+        return "shape too large for the fixed scratch of saw_paged_decode_attn_static "
+               "(num_seqs * num_kv_heads must be at most 2048)";
     default:
         return "unknown status";
     }

@@ -24,6 +24,7 @@ SAW_ERR_INVALID_ARGUMENT = 1
 SAW_ERR_UNSUPPORTED = 2
 SAW_ERR_CUDA = 3
 SAW_ERR_WORKSPACE = 4
+SAW_ERR_SCRATCH_LIMIT = 5
 
 SAW_DEV_BAD_SLOT = 0x1
 SAW_DEV_BAD_PAGE = 0x2
@@ -72,6 +73,11 @@ def _open_library() -> ctypes.CDLL:
 
 
 lib = _open_library()
+lib.saw_paged_decode_attn_static.argtypes = [
+    ctypes.POINTER(saw_cache_desc), ctypes.c_int32, ctypes.c_void_p, ctypes.c_void_p,
+    ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p, ctypes.c_int32,
+    ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]
+lib.saw_paged_decode_attn_static.restype = ctypes.c_int
 
 
 def saw_version() -> int:
@@ -230,3 +236,27 @@ def saw_decode_step(q, k_new, v_new, slot_mapping, kv_pages, scales, block_table
                              float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
                              _ptr(dev_status), _stream(stream))
     _check(rc, "saw_decode_step")
+
+
+def saw_paged_decode_attn_static(q, kv_pages, scales, block_table, seq_lens, out, sm_scale=None,
+                                 dev_status=None, stream=None) -> None:
+    """saw_paged_decode_attn without a workspace, for callers that cannot allocate device memory:
+    the scratch is a fixed array inside the library (num_seqs * num_kv_heads <= 2048).  Calls
+    share that array, so calls that can overlap on the GPU must be serialised by the caller."""
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(out, "out", torch.float32, 3)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    desc = cache_desc(kv_pages)
+    S, hq, _ = q.shape
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_paged_decode_attn_static(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages),
+                                          _ptr(scales), _ptr(block_table), block_table.shape[1],
+                                          _ptr(seq_lens), S, float(sm_scale), _ptr(out),
+                                          _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_paged_decode_attn_static")

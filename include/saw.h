@@ -63,7 +63,8 @@ typedef enum saw_status {
     SAW_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
     SAW_ERR_UNSUPPORTED = 2,      /* head_dim != 128, page_size != 16, Hq / Hkv > 8 */
     SAW_ERR_CUDA = 3,             /* a CUDA runtime call or kernel launch failed */
-    SAW_ERR_WORKSPACE = 4         /* workspace missing or smaller than required */
+    SAW_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required */
+    SAW_ERR_SCRATCH_LIMIT = 5     /* shape too large for saw_paged_decode_attn_static */
 } saw_status;
 
 /* Bits ORed into *dev_status by the kernels. */
@@ -130,6 +131,28 @@ int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void
                     const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
                     void *workspace, size_t workspace_bytes, uint32_t *dev_status,
                     void *stream);
+
+/* saw_paged_decode_attn for callers that cannot allocate device memory.
+ * The pages have no counterpart of this entry point: it exists for callers that are not allowed
+ * or not able to call cudaMalloc -- a plug-in inside a serving framework whose memory pool
+ * already owns the GPU, a request path that must not allocate (cudaMalloc synchronises the
+ * device), or a host library that is only ever handed input and output pointers.  It computes
+ * exactly what saw_paged_decode_attn computes, but its split-K scratch lives in one fixed array
+ * of 12.75 MiB inside this library's device code (present on every GPU that loads the library,
+ * until the process exits) instead of a caller workspace.  It allocates nothing.
+ * Limit: num_seqs * num_kv_heads <= 2048 and a decode grid of at most 1024 CTAs; larger
+ * shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
+ * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
+ * that device current); make that first call before any stream capture.  Every call clears the
+ * array's merge counters with cudaMemsetAsync on `stream`.  All calls on a device share the
+ * array and it keeps the previous call's contents, so calls that can overlap on the GPU (other
+ * streams, other host threads) race on it: the caller must serialise them.
+ * Arguments, layouts and the other status codes are those of saw_paged_decode_attn. */
+int saw_paged_decode_attn_static(const saw_cache_desc *cache, int32_t num_q_heads,
+                                 const void *q, const uint8_t *kv_pages, const void *scales,
+                                 const int32_t *block_table, int32_t max_blocks_per_seq,
+                                 const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                                 float *out, uint32_t *dev_status, void *stream);
 
 /* Human-readable text of a saw_status (never NULL). */
 const char *saw_status_string(int status);
