@@ -20,7 +20,7 @@
 // Per page (16 tokens x one kv head, 2 KiB of codes + 128 B of scales), per warp:
 //   * one elected lane queues a 2-D tensor copy of the 32 code rows (64B swizzle, so both the
 //     K reads and the transposed V reads below are bank-conflict free) and a 1-D bulk copy of
-//     the scales into a 6-stage ring, completion on an mbarrier (bounded wait);
+//     the scales into a 4-stage ring, completion on an mbarrier (bounded wait);
 //   * S^T[16 tok x 8 heads] = K_codes[16 x 128] . Q^T with mma.m16n8k16 (fp16 in, fp32 acc):
 //     the codes 0..15 are exact in fp16, and s = scale * acc + zero * sum(q) in fp32;
 //   * online softmax in the log2 domain (q carries sm_scale * log2 e);
@@ -39,7 +39,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 6;
+constexpr int kStages = 4;                              // power of two
 constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
 constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
@@ -102,21 +102,22 @@ __device__ __forceinline__ int64_t cta_of(int64_t pos, int64_t P, int64_t C)
 }
 
 // Unpack one 32-bit word of packed codes (bytes b0..b3, low nibble first) into four fp16x2
-// registers holding exact code values: (b0.lo, b2.lo), (b0.hi, b2.hi), (b1.lo, b3.lo),
-// (b1.hi, b3.hi).  OR-ing a nibble into the mantissa of 1024.0 gives 1024 + n (or 1024 + 16 n
-// for a high nibble), which one fp16 subtract / fma turns back into n exactly.
+// registers by masking alone: a nibble left in the low mantissa bits of an fp16 with a zero
+// exponent is the subnormal n * 2^-24 (low nibble) or 16 n * 2^-24 = n * 2^-20 (high nibble),
+// exactly.  y[0] = (b0.lo, b2.lo), y[1] = (b0.hi, b2.hi), y[2] = (b1.lo, b3.lo),
+// y[3] = (b1.hi, b3.hi).  The powers of two are folded into q (high nibbles use q / 16) and into
+// the scales, so the tensor-core products are exact.
 __device__ __forceinline__ void unpack_codes(uint32_t w, uint32_t y[4])
 {
-    const uint32_t magic = 0x64006400u;
     const uint32_t w8 = w >> 8;
-    const __half2 k1024 = __half2half2(__ushort_as_half(0x6400));   // 1024
-    const __half2 k1_16 = __half2half2(__ushort_as_half(0x2C00));   // 1/16
-    const __half2 km64 = __half2half2(__ushort_as_half(0xD400));    // -64
-    y[0] = half2_as_u32(__hsub2(u32_as_half2((w & 0x000F000Fu) | magic), k1024));
-    y[1] = half2_as_u32(__hfma2(u32_as_half2((w & 0x00F000F0u) | magic), k1_16, km64));
-    y[2] = half2_as_u32(__hsub2(u32_as_half2((w8 & 0x000F000Fu) | magic), k1024));
-    y[3] = half2_as_u32(__hfma2(u32_as_half2((w8 & 0x00F000F0u) | magic), k1_16, km64));
+    y[0] = w & 0x000F000Fu;
+    y[1] = w & 0x00F000F0u;
+    y[2] = w8 & 0x000F000Fu;
+    y[3] = w8 & 0x00F000F0u;
 }
+
+constexpr float kLowNibble = 16777216.0f;   // 2^24: undoes the low-nibble subnormal scale
+constexpr float kHighNibble = 1048576.0f;   // 2^20: undoes the high-nibble subnormal scale
 
 __device__ __forceinline__ float2 h2_to_f2(uint32_t u)
 {
@@ -189,12 +190,15 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, int s, int h, 
             x[l] = high ? o - x[l] : x[l] + o;
         }
     }
+    // Even d pair with low nibbles (weight 2^-24), odd d with high nibbles (weight 2^-20): odd
+    // entries carry q / 16 so that every product is q_d * code_d * 2^-24.
     float sq = 0.0f;
     __half hq[32];
 #pragma unroll
     for (int l = 0; l < 32; l++) {
-        hq[l] = __float2half_rn(x[l] * p.q_mult);
-        sq += __half2float(hq[l]);
+        const float qv = x[l] * p.q_mult;
+        hq[l] = __float2half_rn((l & 1) ? qv * 0.0625f : qv);
+        sq += (l & 1) ? 16.0f * __half2float(hq[l]) : __half2float(hq[l]);
     }
     sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
     sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
@@ -212,7 +216,9 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, int s, int h, 
     sq_out[1] = __shfl_sync(0xFFFFFFFFu, sq, 8 * t + 4);
 }
 
-// One page of one warp: QK^T, online softmax, PV.
+// One page of one warp: QK^T, online softmax, PV.  kMask: the page is the last of its
+// segment and only its first `valid` tokens exist.
+template <bool kMask>
 __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int valid,
                                              const uint32_t bq[8][2], const float sq[2],
                                              int lane, WarpState &st)
@@ -237,14 +243,21 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
     }
 
     // ---- logits (log2 domain) ---------------------------------------------------------------
-    const bool v0 = g < valid, v1 = g + 8 < valid;
+    const bool v0 = !kMask || g < valid, v1 = !kMask || g + 8 < valid;
     const float2 ksz0 = h2_to_f2(lds32(sbase + 4 * g));
     const float2 ksz1 = h2_to_f2(lds32(sbase + 4 * (g + 8)));
+    const float ks0 = ksz0.x * kLowNibble, ks1 = ksz1.x * kLowNibble;
     float s[4];
-    s[0] = v0 ? fmaf(ksz0.x, acc[0], ksz0.y * sq[0]) : -INFINITY;
-    s[1] = v0 ? fmaf(ksz0.x, acc[1], ksz0.y * sq[1]) : -INFINITY;
-    s[2] = v1 ? fmaf(ksz1.x, acc[2], ksz1.y * sq[0]) : -INFINITY;
-    s[3] = v1 ? fmaf(ksz1.x, acc[3], ksz1.y * sq[1]) : -INFINITY;
+    s[0] = fmaf(ks0, acc[0], ksz0.y * sq[0]);
+    s[1] = fmaf(ks0, acc[1], ksz0.y * sq[1]);
+    s[2] = fmaf(ks1, acc[2], ksz1.y * sq[0]);
+    s[3] = fmaf(ks1, acc[3], ksz1.y * sq[1]);
+    if (kMask) {
+        if (!v0)
+            s[0] = s[1] = -INFINITY;
+        if (!v1)
+            s[2] = s[3] = -INFINITY;
+    }
 
     float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
 #pragma unroll
@@ -281,10 +294,12 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
     // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
     float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));
     float2 vsz1 = h2_to_f2(lds32(sbase + 64 + 4 * (g + 8)));
-    if (!v0)
-        vsz0 = make_float2(0.0f, 0.0f);
-    if (!v1)
-        vsz1 = make_float2(0.0f, 0.0f);
+    if (kMask) {
+        if (!v0)
+            vsz0 = make_float2(0.0f, 0.0f);
+        if (!v1)
+            vsz1 = make_float2(0.0f, 0.0f);
+    }
     st.l[0] += pr[0] + pr[2];
     st.l[1] += pr[1] + pr[3];
     st.z[0] = fmaf(pr[0], vsz0.y, fmaf(pr[2], vsz1.y, st.z[0]));
@@ -415,7 +430,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, in
     }
 }
 
-__global__ void __launch_bounds__(kThreads, 3)
+__global__ void __launch_bounds__(kThreads, 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -516,7 +531,8 @@ __global__ void __launch_bounds__(kThreads, 3)
 
     int32_t look_cur = lookup(lane), look_nxt = lookup(32 + lane);
     int issued = 0;        // pages queued so far
-    bool aborted = false;
+    bool aborted = false;  // a page wait gave up: stop queueing and computing
+    int drain_from = 0;    // first page whose copy may still be in flight after an abort
     auto issue_next = [&]() {
         if (issued >= n_w || aborted)
             return;
@@ -527,7 +543,7 @@ __global__ void __launch_bounds__(kThreads, 3)
         }
         const int32_t row = __shfl_sync(0xFFFFFFFFu, look_cur, m & 31);
         if (lane == 0) {
-            const int stg = m % kStages;
+            const int stg = m & (kStages - 1);
             const uint32_t bar = bar0 + 8 * stg;
             mbar_arrive_expect_tx(bar, kTxBytes);
             tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, row, bar);
@@ -559,21 +575,26 @@ __global__ void __launch_bounds__(kThreads, 3)
             uint32_t bq[8][2];
             float sq[2];
             load_query(p, s, h, g, t, bq, sq);
-            for (; m < m_end; m++) {
+            int i = static_cast<int>(first + static_cast<int64_t>(kWarps) * m - seg_start);
+            for (; m < m_end; m++, i += kWarps) {
                 issue_next();
-                const int stg = m % kStages;
-                const bool ok = aborted ? false
-                                        : mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
-                if (!__all_sync(0xFFFFFFFFu, ok)) {
-                    if (!aborted && lane == 0)
-                        set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+                const int stg = m & (kStages - 1);
+                const bool ok = !aborted &&
+                                mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
+                if (__all_sync(0xFFFFFFFFu, ok)) {
+                    const uint32_t cb = code0 + stg * kCodeBytes, sb = scale0 + stg * kScaleBytes;
+                    if (i == n_s - 1)
+                        process_page<true>(cb, sb, len - kPageSize * i, bq, sq, lane, st);
+                    else
+                        process_page<false>(cb, sb, kPageSize, bq, sq, lane, st);
+                } else {
+                    if (!aborted) {
+                        if (lane == 0)
+                            set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+                        drain_from = m;
+                    }
                     aborted = true;
-                    continue;
                 }
-                const int i = static_cast<int>(first + static_cast<int64_t>(kWarps) * m - seg_start);
-                const int valid = len - kPageSize * i;
-                process_page(code0 + stg * kCodeBytes, scale0 + stg * kScaleBytes, valid, bq, sq,
-                             lane, st);
                 __syncwarp();
             }
             // reduce l and z over the 8 token rows (lanes differing in g)
@@ -585,12 +606,14 @@ __global__ void __launch_bounds__(kThreads, 3)
                     st.z[e] += __shfl_xor_sync(0xFFFFFFFFu, st.z[e], d);
                 }
             }
+            // undo the subnormal code scales (value rows g: low nibbles, g + 8: high nibbles)
+            // and add the zero-point term
 #pragma unroll
-            for (int i = 0; i < 8; i++) {
-                st.o[i][0] += st.z[0];
-                st.o[i][1] += st.z[1];
-                st.o[i][2] += st.z[0];
-                st.o[i][3] += st.z[1];
+            for (int i2 = 0; i2 < 8; i2++) {
+                st.o[i2][0] = fmaf(st.o[i2][0], kLowNibble, st.z[0]);
+                st.o[i2][1] = fmaf(st.o[i2][1], kLowNibble, st.z[1]);
+                st.o[i2][2] = fmaf(st.o[i2][2], kHighNibble, st.z[0]);
+                st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
             }
         }
 
@@ -645,11 +668,12 @@ __global__ void __launch_bounds__(kThreads, 3)
                     ticket = atomicAdd(p.tickets + seg, 1u);
                 ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
                 if (ticket == static_cast<uint32_t>(c_hi - c_lo)) {
-                    // last CTA of this segment: fold in every other CTA's partial
+                    // last CTA of this segment: fold in every CTA's partial, in CTA order
+                    // (its own included), so that the result does not depend on which CTA
+                    // finished last
                     __threadfence();
+                    state_reset(st);
                     for (int64_t c2 = c_lo; c2 <= c_hi; c2++) {
-                        if (c2 == cta)
-                            continue;
                         const float *o2 = p.partials + (seg + c2) * kSlotFloats;
                         const float4 *o24 = reinterpret_cast<const float4 *>(o2);
                         float4 bo[8];
@@ -671,7 +695,7 @@ __global__ void __launch_bounds__(kThreads, 3)
 
     // ---- 5. after an abort, let queued copies land before the CTA's shared memory is freed --
     if (aborted) {
-        for (int k = m; k < issued; k++)
+        for (int k = drain_from; k < issued; k++)
             mbar_wait_bounded(bar0 + 8 * (k % kStages), (k / kStages) & 1, kWaitLimitNs / 10);
     }
 }

@@ -134,7 +134,7 @@ __device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
 __device__ __forceinline__ float quantize_fast(uint64_t X[32], float mn, float r)
 {
     const uint64_t mn2 = f2_pack(mn, mn), r2 = f2_pack(r, r), m2 = f2_pack(kRoundMagic, kRoundMagic);
-    float worst = 0.0f;
+    float w[8];
 #pragma unroll
     for (int i = 0; i < 32; i++) {
         const uint64_t d = f2_sub(X[i], mn2);
@@ -143,10 +143,10 @@ __device__ __forceinline__ float quantize_fast(uint64_t X[32], float mn, float r
         const uint64_t res = f2_fma(d, r2, nk);     // d r - k, one rounding
         float a, c;
         f2_unpack(res, a, c);
-        worst = fmax3(worst, fabsf(a), fabsf(c));
+        w[i & 7] = (i < 8) ? fmaxf(fabsf(a), fabsf(c)) : fmax3(w[i & 7], fabsf(a), fabsf(c));
         X[i] = t;
     }
-    return worst;
+    return fmaxf(fmax3(w[0], w[1], w[2]), fmax3(fmax3(w[3], w[4], w[5]), w[6], w[7]));
 }
 
 // Codes through the IEEE divide, exactly as defined (used where quantize_fast cannot decide,
@@ -196,14 +196,16 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], const uint8_t *sr
                                                const RqParams &p)
 {
     // min / max over the pair's 128 elements
-    float mn = FLT_MAX, mx = -FLT_MAX;
+    float mns[8], mxs[8];
 #pragma unroll
     for (int i = 0; i < 32; i++) {
         float lo, hi;
         f2_unpack(X[i], lo, hi);
-        mn = fmin3(mn, lo, hi);
-        mx = fmax3(mx, lo, hi);
+        mns[i & 7] = (i < 8) ? fminf(lo, hi) : fmin3(mns[i & 7], lo, hi);
+        mxs[i & 7] = (i < 8) ? fmaxf(lo, hi) : fmax3(mxs[i & 7], lo, hi);
     }
+    float mn = fminf(fmin3(mns[0], mns[1], mns[2]), fmin3(fmin3(mns[3], mns[4], mns[5]), mns[6], mns[7]));
+    float mx = fmaxf(fmax3(mxs[0], mxs[1], mxs[2]), fmax3(fmax3(mxs[3], mxs[4], mxs[5]), mxs[6], mxs[7]));
     mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
     mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
 
