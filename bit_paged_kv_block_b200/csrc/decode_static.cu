@@ -1,19 +1,19 @@
 // decode_static.cu -- saw_paged_decode_attn_static: the decode entry point for callers that
 // cannot allocate device memory.
 //
-// saw_paged_decode_attn needs a caller-provided workspace (split-K partial results and merge
-// counters).  Some callers have no way to provide one: a plug-in running inside a serving
+// saw_paged_decode_attn needs a caller-provided workspace (split-K partial results).  Some
+// callers have no way to provide one: a plug-in running inside a serving
 // framework that has already reserved the whole GPU for its own memory pool, a request path
 // with a no-allocation rule (cudaMalloc synchronises the device and can stall every stream),
 // or a host library that only ever receives pointers to inputs and outputs.  For them this
 // entry point takes its scratch from one fixed array in device memory that is part of this
-// library itself: kScratchBytes (12.75 MiB) on every GPU that loads the library, held until
+// library itself: kScratchBytes (18.3 MiB) on every GPU that loads the library, held until
 // the process exits.  Nothing here calls cudaMalloc, cudaFree or any allocating routine.
 //
 // The scratch is shared by all calls on a device and keeps whatever the last call left in it,
 // so calls whose kernels can overlap on the GPU (different streams, or several host threads)
-// race on it and must be serialised by the caller.  The merge counters that must start at zero
-// are cleared with cudaMemsetAsync on the caller's stream at the start of every call.
+// race on it and must be serialised by the caller.  Nothing in it needs to start at zero: every
+// split-K partial is written by the decode kernel before the merge kernel reads it.
 #include <cuda_runtime.h>
 
 #include <mutex>
@@ -23,10 +23,10 @@
 
 namespace {
 
-// Room for num_seqs * num_kv_heads <= 2048 (sequence, kv head) pairs and a grid of up to 1024
-// CTAs: 2048 merge counters (8 KiB) plus (1024 + 2048) partial-result slots of 4160 bytes.
+// Room for num_seqs * num_kv_heads <= 2048 (sequence, kv head) pairs and a decode grid of up
+// to 2560 warps: (2560 + 2048) partial-result slots of 4160 bytes.
 constexpr int kScratchMaxSegments = 2048;
-constexpr size_t kScratchBytes = 8192 + (1024 + kScratchMaxSegments) * size_t(4160);
+constexpr size_t kScratchBytes = (2560 + kScratchMaxSegments) * size_t(4160);
 
 static __device__ __align__(256) unsigned char g_decode_scratch[kScratchBytes];
 
@@ -73,11 +73,6 @@ extern "C" int saw_paged_decode_attn_static(const saw_cache_desc *cache, int32_t
     const int rc = scratch_address(&scratch);
     if (rc != SAW_OK)
         return rc;
-    if (num_seqs > 0) {
-        const size_t counters = (size_t(num_seqs) * cache->num_kv_heads * 4 + 255) & ~size_t(255);
-        if (cudaMemsetAsync(scratch, 0, counters, static_cast<cudaStream_t>(stream)) != cudaSuccess)
-            return SAW_ERR_CUDA;
-    }
     return saw_paged_decode_attn(cache, num_q_heads, q, kv_pages, scales, block_table,
                                  max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, scratch,
                                  kScratchBytes, dev_status, stream);

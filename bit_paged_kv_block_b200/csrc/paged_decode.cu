@@ -7,29 +7,33 @@
 // Because H is orthogonal and symmetric, <q, k> = <Hq, Hk> and sum p_t v_t = H sum p_t (H v_t):
 // the kernel rotates q once, attends over the rotated codes and rotates the output back.
 //
-// Work split.  A (sequence s, kv head h) pair is a segment of ceil(len_s / 16) pages.  All
-// segments are laid end to end (seq-major, then kv head) and that flat page range P is cut into
-// C = min(gridDim.x, P / 4) equal slices, one per CTA; inside a CTA the 4 warps take every 4th
-// page.  Each
-// (segment, CTA) intersection is a piece: the warps' online-softmax states for a piece are
-// merged in shared memory; a segment that spans several CTAs has one partial per CTA in the
-// workspace (slot segment + CTA index, unique because both orders are monotone) and the CTA
-// that finishes it last (an atomic ticket, no waiting) merges them, rotates the result back
-// and writes it.
+// Work split.  A (sequence s, kv head h) pair is a segment of n = ceil(len_s / 16) pages.  All
+// segments are laid end to end (seq-major, then kv head) in a cost space where a segment costs
+// n + kKappa (kKappa pages' worth of per-segment work: query rotation and output rotation), and
+// that cost range is cut into W equal slices, one per warp of a persistent grid.  Each warp
+// owns the contiguous run of pages whose cost positions fall in its slice and works on it
+// independently: no barrier, atomic or fence between warps.  A segment that lies entirely in one
+// warp's run is finished by that warp; the pieces of a segment split across warps are written to
+// the workspace (slot segment + warp, unique because both orders are monotone) and combined by
+// a second kernel (paged_decode_merge_kernel), launched as a programmatic dependent.
 //
 // Per page (16 tokens x one kv head, 2 KiB of codes + 128 B of scales), per warp:
-//   * one elected lane queues a 2-D tensor copy of the 32 code rows (64B swizzle, so both the
-//     K reads and the transposed V reads below are bank-conflict free) and a 1-D bulk copy of
-//     the scales into a 4-stage ring, completion on an mbarrier (bounded wait);
+//   * the lane that looked the page up queues a 2-D tensor copy of the 32 code rows (64B
+//     swizzle, so the K reads and the transposed V reads below are bank-conflict free) and a
+//     1-D bulk copy of the scales into a 4-stage ring, completion on an mbarrier (bounded wait);
 //   * S^T[16 tok x 8 heads] = K_codes[16 x 128] . Q^T with mma.m16n8k16 (fp16 in, fp32 acc):
-//     the codes 0..15 are exact in fp16, and s = scale * acc + zero * sum(q) in fp32;
+//     the codes are exact fp16 subnormals, and s = scale * acc + zero * sum(q) in fp32;
 //   * online softmax in the log2 domain (q carries sm_scale * log2 e);
 //   * O^T[128 d x 8 heads] += V_codes^T . P'^T with P' = p * scale_V in fp16 and the zero
 //     point added in fp32 through sum_t p_t zero_t.
-// The query dimension d of QK and the value dimension of PV are consumed in a permuted order
-// (both sides permuted alike), which lets every thread unpack whole 32-bit code words.
+// The query of the next segment is bulk-copied into a per-warp buffer while the current one is
+// processed.  The query dimension d of QK and the value dimension of PV are consumed in a
+// permuted order (both sides permuted alike), which lets every thread unpack whole 32-bit code
+// words; the final inverse rotation undoes it.
 #include <cfloat>
 #include <cudaTypedefs.h>
+
+#include <mutex>
 
 #include "saw_device.cuh"
 #include "saw_internal.h"
@@ -43,22 +47,33 @@ constexpr int kStages = 4;                              // power of two
 constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
 constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
+constexpr int kQBytes = 8 * kHeadDim * 2;               // raw bf16 queries of one kv head (G <= 8)
 constexpr int kSlotFloats = 32 * 32 + 16;               // O (lane layout) + m[8] + l[8]
-constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a page wait after 1 s
+constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
+constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
 constexpr float kHadamardC = 0.0883883461356163f;
+constexpr int kMergeWarps = 4;
+constexpr int kMergeThreads = 32 * kMergeWarps;
 
-// shared memory carve-up (bytes, from a 1024-aligned base)
+// shared memory carve-up of the decode kernel (bytes, from a 1024-aligned base)
 constexpr int kSmemCodes = 0;
 constexpr int kSmemScales = kSmemCodes + kWarps * kStages * kCodeBytes;
-constexpr int kSmemBars = kSmemScales + kWarps * kStages * kScaleBytes;
-constexpr int kSmemMergeO = kSmemBars + kWarps * kStages * 8;
-constexpr int kSmemMergeML = kSmemMergeO + (kWarps - 1) * 32 * 32 * 4;
-constexpr int kSmemFlags = kSmemMergeML + (kWarps - 1) * 16 * 4;
+constexpr int kSmemQ = kSmemScales + kWarps * kStages * kScaleBytes;
+constexpr int kSmemBars = kSmemQ + kWarps * kQBytes;
+constexpr int kSmemFlags = kSmemBars + kWarps * (kStages + 1) * 8;
 constexpr int kSmemPrefix = kSmemFlags + 64;
+// merge kernel: per-warp partials, then the prefix
+constexpr int kMergeSmemSlots = 0;
+constexpr int kMergeSmemFlags = kMergeSmemSlots + (kMergeWarps - 1) * kSlotFloats * 4;
+constexpr int kMergeSmemPrefix = kMergeSmemFlags + 64;
 
 size_t decode_smem_bytes(int32_t num_seqs)
 {
     return 1024 + kSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
+}
+size_t merge_smem_bytes(int32_t num_seqs)
+{
+    return kMergeSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
 }
 
 struct DecodeParams {
@@ -67,8 +82,7 @@ struct DecodeParams {
     const int32_t *block_table;
     const int32_t *seq_lens;
     float *out;
-    uint32_t *tickets;
-    float *partials;
+    float *partials;             // workspace: (total warps + segments) slots
     uint32_t *status;
     int64_t num_pages;
     int32_t max_blocks;
@@ -76,10 +90,11 @@ struct DecodeParams {
     int32_t hq;
     int32_t hkv;
     int32_t group;
+    int32_t total_warps;         // warps of the decode grid (the plan's slice count bound)
     float q_mult;                // fp32(1/sqrt(128)) * sm_scale * log2(e)
 };
 
-// ---- small helpers ----------------------------------------------------------------------
+// ---- work plan ------------------------------------------------------------------------------
 
 // Largest s in [0, S) with hkv * pre[s] <= pos (pos < hkv * pre[S]).
 __device__ __forceinline__ int find_seq(const int32_t *pre, int S, int64_t pos, int64_t hkv)
@@ -95,11 +110,111 @@ __device__ __forceinline__ int find_seq(const int32_t *pre, int S, int64_t pos, 
     return lo;
 }
 
-// Index of the CTA whose slice [c P / C, (c + 1) P / C) holds flat page pos.
-__device__ __forceinline__ int64_t cta_of(int64_t pos, int64_t P, int64_t C)
+// Pages per sequence (0 for an invalid length, which is flagged) and their exclusive prefix
+// pre[0..S] in shared memory; every thread of the block takes part.
+__device__ void scan_pages(const DecodeParams &p, int32_t *pre, volatile int32_t *flags,
+                           bool report)
 {
-    return ((pos + 1) * C + P - 1) / P - 1;
+    const int S = p.num_seqs, nthreads = blockDim.x, tid = threadIdx.x;
+    const int lane = tid & 31, warp = tid >> 5;
+    const int per = (S + nthreads - 1) / nthreads;
+    const int s0 = tid * per, s1 = min(S, s0 + per);
+    int local = 0;
+    for (int s = s0; s < s1; s++) {
+        const int len = p.seq_lens[s];
+        const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
+        if (!ok && report)
+            set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
+        local += ok ? (len + kPageSize - 1) / kPageSize : 0;
+    }
+    int incl = local;
+#pragma unroll
+    for (int d = 1; d < 32; d <<= 1) {
+        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
+        if (lane >= d)
+            incl += o;
+    }
+    if (lane == 31)
+        flags[warp] = incl;
+    __syncthreads();
+    int base = 0;
+    for (int w = 0; w < warp; w++)
+        base += flags[w];
+    int run = base + incl - local;
+    for (int s = s0; s < s1; s++) {
+        pre[s] = run;
+        const int len = p.seq_lens[s];
+        const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
+        run += ok ? (len + kPageSize - 1) / kPageSize : 0;
+    }
+    if (tid == nthreads - 1)
+        pre[S] = base + incl;
+    __syncthreads();
 }
+
+// The cost-space split of the flat page range into warp runs.  Segment (s, h) spans the cost
+// range [seq_cost(s) + h (n_s + kKappa), + n_s + kKappa); its page i sits at cost
+// seq_cost(s) + h (n_s + kKappa) + kKappa + i.  Warp u owns the cost range
+// [b(u), b(u + 1)) with b(u) = u q + min(u, r), q = PT / W, r = PT % W (slices of q or q + 1,
+// never empty because W <= PT), i.e. the pages whose cost falls in it.
+struct Plan {
+    const int32_t *pre;
+    int S;
+    int64_t hkv;
+    int64_t P;    // pages
+    int64_t PT;   // cost
+    int64_t W;    // warps with a slice
+    int64_t q, r;
+
+    __device__ void init(const int32_t *pre_, int S_, int hkv_, int total_warps)
+    {
+        pre = pre_;
+        S = S_;
+        hkv = hkv_;
+        P = hkv * pre[S];
+        PT = hkv * (static_cast<int64_t>(pre[S]) + kKappa * S);
+        W = max(int64_t(1), min(static_cast<int64_t>(total_warps), PT));
+        q = PT / W;
+        r = PT - q * W;
+    }
+    __device__ int64_t seq_cost(int s) const
+    {
+        return hkv * (static_cast<int64_t>(pre[s]) + kKappa * s);
+    }
+    __device__ int64_t slice_begin(int64_t u) const { return u * q + min(u, r); }
+    // the warp whose cost slice holds cost position x (0 <= x < PT)
+    __device__ int64_t warp_of_cost(int64_t x) const
+    {
+        const int64_t big = r * (q + 1);
+        return x < big ? x / (q + 1) : r + (x - big) / q;
+    }
+    // cost position of page i of segment (s, h)
+    __device__ int64_t page_cost(int s, int h, int64_t i) const
+    {
+        return seq_cost(s) + static_cast<int64_t>(h) * (pre[s + 1] - pre[s] + kKappa) + kKappa + i;
+    }
+    // first flat page whose cost position is >= x
+    __device__ int64_t flat_of_cost(int64_t x) const
+    {
+        if (x >= PT)
+            return P;
+        int lo = 0, hi = S;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (seq_cost(mid) <= x)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        const int64_t n = pre[lo + 1] - pre[lo];
+        const int64_t within = x - seq_cost(lo);
+        const int64_t h = within / (n + kKappa);
+        const int64_t rr = within - h * (n + kKappa);
+        return hkv * pre[lo] + h * n + (rr < kKappa ? 0 : rr - kKappa);
+    }
+    // first flat page of warp u's run (u in [0, W]; the run of u is [begin(u), begin(u + 1)))
+    __device__ int64_t begin(int64_t u) const { return flat_of_cost(slice_begin(u)); }
+};
 
 // Unpack one 32-bit word of packed codes (bytes b0..b3, low nibble first) into four fp16x2
 // registers by masking alone: a nibble left in the low mantissa bits of an fp16 with a zero
@@ -148,17 +263,17 @@ __device__ __forceinline__ void state_reset(WarpState &st)
     }
 }
 
-// Rotated, scaled query of (seq s, kv head h) as fp16 mma B fragments.
+// Rotated, scaled query of (seq s, kv head h) as fp16 mma B fragments, from the raw bf16
+// queries of the group in shared memory ([G][128] at qbuf).
 // Thread (g, t) owns query head g of the group and d in [32t, 32t + 32).
-__device__ __forceinline__ void load_query(const DecodeParams &p, int s, int h, int g, int t,
+__device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int g, int t,
                                            uint32_t bq[8][2], float sq_out[2])
 {
     float x[32];
     if (g < p.group) {
-        const uint16_t *src = p.q + ((static_cast<int64_t>(s) * p.hq + h * p.group + g) * kHeadDim + 32 * t);
 #pragma unroll
         for (int c = 0; c < 4; c++) {
-            const uint4 u = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            const uint4 u = lds128(qbuf + g * (kHeadDim * 2) + 64 * t + 16 * c);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int k = 0; k < 4; k++) {
@@ -430,6 +545,37 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, in
     }
 }
 
+
+// Store this warp's (m, l, o) for one piece into workspace slot `slot`.
+__device__ __forceinline__ void store_partial(float *slot, int lane, const WarpState &st)
+{
+    const int g = lane >> 2, t = lane & 3;
+    float4 *so = reinterpret_cast<float4 *>(slot);
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        so[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
+    if (g == 0) {
+        slot[1024 + 2 * t] = st.m[0];
+        slot[1024 + 2 * t + 1] = st.m[1];
+        slot[1032 + 2 * t] = st.l[0];
+        slot[1032 + 2 * t + 1] = st.l[1];
+    }
+}
+
+__device__ __forceinline__ void load_partial(const float *slot, int lane, float bm[2], float bl[2],
+                                             float4 bo[8])
+{
+    const int t = lane & 3;
+    const float4 *so = reinterpret_cast<const float4 *>(slot);
+#pragma unroll
+    for (int i = 0; i < 8; i++)
+        bo[i] = so[i * 32 + lane];
+    bm[0] = slot[1024 + 2 * t];
+    bm[1] = slot[1024 + 2 * t + 1];
+    bl[0] = slot[1032 + 2 * t];
+    bl[1] = slot[1032 + 2 * t + 1];
+}
+
 __global__ void __launch_bounds__(kThreads, 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
 {
@@ -441,47 +587,9 @@ __global__ void __launch_bounds__(kThreads, 4)
     int32_t *pre = reinterpret_cast<int32_t *>(smem + kSmemPrefix);
     volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + kSmemFlags);
 
-    // ---- 1. pages per sequence and their exclusive prefix ---------------------------------
-    {
-        const int per = (S + kThreads - 1) / kThreads;
-        const int s0 = tid * per, s1 = min(S, s0 + per);
-        int local = 0;
-        for (int s = s0; s < s1; s++) {
-            const int len = p.seq_lens[s];
-            const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
-            if (!ok && blockIdx.x == 0)
-                set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
-            local += ok ? (len + kPageSize - 1) / kPageSize : 0;
-        }
-        int incl = local;
-#pragma unroll
-        for (int d = 1; d < 32; d <<= 1) {
-            const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-            if (lane >= d)
-                incl += o;
-        }
-        if (lane == 31)
-            flags[warp] = incl;
-        __syncthreads();
-        int base = 0;
-        for (int w = 0; w < warp; w++)
-            base += flags[w];
-        int run = base + incl - local;
-        for (int s = s0; s < s1; s++) {
-            pre[s] = run;
-            const int len = p.seq_lens[s];
-            const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
-            run += ok ? (len + kPageSize - 1) / kPageSize : 0;
-        }
-        if (tid == kThreads - 1)
-            pre[S] = base + incl;
-        __syncthreads();
-    }
-    const int64_t hkv = p.hkv;
-    const int64_t P = hkv * pre[S];
-    const int64_t cta = blockIdx.x;
-
-    // ---- 2. sequences with no pages get a zero output ---------------------------------------
+    // ---- 1. pages per sequence, the plan, zero outputs of empty sequences ------------------
+    scan_pages(p, pre, flags, blockIdx.x == 0);
+    pdl_launch_dependents();   // the merge kernel may start its own prologue
     for (int s = blockIdx.x; s < S; s += gridDim.x) {
         if (pre[s + 1] == pre[s]) {
             float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<int64_t>(s) * p.hq * kHeadDim);
@@ -489,36 +597,39 @@ __global__ void __launch_bounds__(kThreads, 4)
                 dst[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
     }
-    // Slice over C <= P / 4 CTAs so that every slice is non-empty (at least one page per
-    // warp); the remaining CTAs have no pages.  The merge counts rely on non-empty slices.
-    const int64_t C = max(int64_t(1), min(static_cast<int64_t>(gridDim.x), P / kWarps));
-    if (P == 0 || cta >= C)
+    Plan plan;
+    plan.init(pre, S, p.hkv, p.total_warps);
+    const int64_t u = static_cast<int64_t>(blockIdx.x) * kWarps + warp;
+    if (plan.P == 0 || u >= plan.W)
         return;
-    const int64_t Bc = (cta * P) / C, Bc1 = ((cta + 1) * P) / C;
+    const int64_t F0 = plan.begin(u), F1 = plan.begin(u + 1);
+    if (F0 >= F1)
+        return;
+    const int n_w = static_cast<int>(F1 - F0);
+    const int64_t hkv = p.hkv;
 
-    // ---- 3. this warp's page stream: flat positions Bc + warp + 4 m ----------------------------
+    // ---- 2. this warp's copy ring ---------------------------------------------------------------
     const uint32_t code0 = smem_u32(smem + kSmemCodes) + warp * kStages * kCodeBytes;
     const uint32_t scale0 = smem_u32(smem + kSmemScales) + warp * kStages * kScaleBytes;
-    const uint32_t bar0 = smem_u32(smem + kSmemBars) + warp * kStages * 8;
+    const uint32_t qbuf = smem_u32(smem + kSmemQ) + warp * kQBytes;
+    const uint32_t bar0 = smem_u32(smem + kSmemBars) + warp * (kStages + 1) * 8;
+    const uint32_t qbar = bar0 + kStages * 8;
     if (lane == 0)
-        for (int i = 0; i < kStages; i++)
+        for (int i = 0; i <= kStages; i++)
             mbar_init(bar0 + 8 * i, 1);
     mbar_init_fence();
     __syncwarp();
 
-    const int64_t first = Bc + warp;
-    const int n_w = first < Bc1 ? static_cast<int>((Bc1 - first + kWarps - 1) / kWarps) : 0;
-
-    // tensor-map row (page * Hkv + h) * 32 of this warp's page m (-1 past the end)
+    // tensor-map row (page * Hkv + h) * 32 of page m of this warp's run
     auto lookup = [&](int m) -> int32_t {
         if (m >= n_w)
-            return -1;
-        const int64_t pos = first + static_cast<int64_t>(kWarps) * m;
+            return 0;
+        const int64_t pos = F0 + m;
         const int s = find_seq(pre, S, pos, hkv);
         const int32_t n_s = pre[s + 1] - pre[s];
-        const int64_t u = pos - hkv * pre[s];
-        const int h = static_cast<int>(u / n_s);
-        const int i = static_cast<int>(u - static_cast<int64_t>(h) * n_s);
+        const int64_t rel = pos - hkv * pre[s];
+        const int h = static_cast<int>(rel / n_s);
+        const int i = static_cast<int>(rel - static_cast<int64_t>(h) * n_s);
         int32_t page = p.block_table[static_cast<int64_t>(s) * p.max_blocks + i];
         if (page < 0 || page >= p.num_pages) {
             set_status(p.status, SAW_DEV_BAD_PAGE);
@@ -526,12 +637,21 @@ __global__ void __launch_bounds__(kThreads, 4)
         }
         return (page * p.hkv + h) * 32;
     };
+    // queue the raw queries of (s, h) into the warp's query buffer
+    auto issue_query = [&](int s, int h) {
+        if (lane == 0) {
+            const uint32_t bytes = static_cast<uint32_t>(p.group) * kHeadDim * 2;
+            mbar_arrive_expect_tx(qbar, bytes);
+            bulk_g2s(qbuf, p.q + (static_cast<int64_t>(s) * p.hq + static_cast<int64_t>(h) * p.group) * kHeadDim,
+                     bytes, qbar);
+        }
+    };
 
     pdl_wait();   // the cache may be written by the kernel this one depends on
 
     int32_t look_cur = lookup(lane), look_nxt = lookup(32 + lane);
     int issued = 0;        // pages queued so far
-    bool aborted = false;  // a page wait gave up: stop queueing and computing
+    bool aborted = false;  // a wait gave up: stop queueing and computing
     int drain_from = 0;    // first page whose copy may still be in flight after an abort
     auto issue_next = [&]() {
         if (issued >= n_w || aborted)
@@ -541,162 +661,184 @@ __global__ void __launch_bounds__(kThreads, 4)
             look_cur = look_nxt;
             look_nxt = lookup(m + 32 + lane);
         }
-        const int32_t row = __shfl_sync(0xFFFFFFFFu, look_cur, m & 31);
-        if (lane == 0) {
+        if (lane == (m & 31)) {
             const int stg = m & (kStages - 1);
             const uint32_t bar = bar0 + 8 * stg;
             mbar_arrive_expect_tx(bar, kTxBytes);
-            tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, row, bar);
-            bulk_g2s(scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(row) * 4,
+            tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, look_cur, bar);
+            bulk_g2s(scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(look_cur) * 4,
                      kScaleBytes, bar);
         }
         issued++;
     };
+
+    // first piece's segment and its query
+    int s = find_seq(pre, S, F0, hkv);
+    int h = static_cast<int>((F0 - hkv * pre[s]) / (pre[s + 1] - pre[s]));
+    issue_query(s, h);
     for (int k = 0; k < kStages - 1; k++)
         issue_next();
 
-    // ---- 4. pieces ----------------------------------------------------------------------------
+    // ---- 3. pieces ------------------------------------------------------------------------------
     int m = 0;
-    int64_t pos = Bc;
+    uint32_t qphase = 0;
+    int64_t pos = F0;
     WarpState st;
-    while (pos < Bc1) {
-        const int s = find_seq(pre, S, pos, hkv);
+    while (pos < F1) {
         const int32_t n_s = pre[s + 1] - pre[s];
-        const int64_t seq_start = hkv * pre[s];
-        const int h = static_cast<int>((pos - seq_start) / n_s);
-        const int64_t seg_start = seq_start + static_cast<int64_t>(h) * n_s;
+        const int64_t seg_start = hkv * pre[s] + static_cast<int64_t>(h) * n_s;
         const int64_t seg_end = seg_start + n_s;
-        const int64_t piece_end = seg_end < Bc1 ? seg_end : Bc1;
-        const int m_end = piece_end > first ? static_cast<int>((piece_end - first + kWarps - 1) / kWarps) : 0;
+        const int64_t piece_end = seg_end < F1 ? seg_end : F1;
+        const int m_end = static_cast<int>(piece_end - F0);
         const int len = p.seq_lens[s];
 
-        state_reset(st);
-        if (m < m_end) {
-            uint32_t bq[8][2];
-            float sq[2];
-            load_query(p, s, h, g, t, bq, sq);
-            int i = static_cast<int>(first + static_cast<int64_t>(kWarps) * m - seg_start);
-            for (; m < m_end; m++, i += kWarps) {
-                issue_next();
-                const int stg = m & (kStages - 1);
-                const bool ok = !aborted &&
-                                mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
-                if (__all_sync(0xFFFFFFFFu, ok)) {
-                    const uint32_t cb = code0 + stg * kCodeBytes, sb = scale0 + stg * kScaleBytes;
-                    if (i == n_s - 1)
-                        process_page<true>(cb, sb, len - kPageSize * i, bq, sq, lane, st);
-                    else
-                        process_page<false>(cb, sb, kPageSize, bq, sq, lane, st);
-                } else {
-                    if (!aborted) {
-                        if (lane == 0)
-                            set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
-                        drain_from = m;
-                    }
-                    aborted = true;
-                }
-                __syncwarp();
+        // this piece's query: wait for its copy, build the fragments, then queue the next one
+        uint32_t bq[8][2];
+        float sq[2];
+        const bool qok = !aborted && mbar_wait_bounded(qbar, qphase, kWaitLimitNs);
+        if (!__all_sync(0xFFFFFFFFu, qok) && !aborted) {
+            if (lane == 0)
+                set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+            drain_from = m;
+            aborted = true;
+        }
+        qphase ^= 1;
+        load_query(p, qbuf, g, t, bq, sq);
+        __syncwarp();
+        int s_next = s, h_next = h;
+        if (piece_end < F1) {
+            if (++h_next == p.hkv) {
+                h_next = 0;
+                do {
+                    s_next++;
+                } while (pre[s_next + 1] == pre[s_next]);
             }
-            // reduce l and z over the 8 token rows (lanes differing in g)
-#pragma unroll
-            for (int e = 0; e < 2; e++) {
-#pragma unroll
-                for (int d = 4; d <= 16; d <<= 1) {
-                    st.l[e] += __shfl_xor_sync(0xFFFFFFFFu, st.l[e], d);
-                    st.z[e] += __shfl_xor_sync(0xFFFFFFFFu, st.z[e], d);
-                }
-            }
-            // undo the subnormal code scales (value rows g: low nibbles, g + 8: high nibbles)
-            // and add the zero-point term
-#pragma unroll
-            for (int i2 = 0; i2 < 8; i2++) {
-                st.o[i2][0] = fmaf(st.o[i2][0], kLowNibble, st.z[0]);
-                st.o[i2][1] = fmaf(st.o[i2][1], kLowNibble, st.z[1]);
-                st.o[i2][2] = fmaf(st.o[i2][2], kHighNibble, st.z[0]);
-                st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
-            }
+            if (!aborted)
+                issue_query(s_next, h_next);
         }
 
-        // ---- merge the 4 warps' partials of this piece ----------------------------------------
-        __syncthreads();   // warp 0 has finished reading the previous piece's buffers
-        float *mO = reinterpret_cast<float *>(smem + kSmemMergeO);
-        float *mML = reinterpret_cast<float *>(smem + kSmemMergeML);
-        if (warp > 0) {
-            float4 *dst = reinterpret_cast<float4 *>(mO) + (warp - 1) * 8 * 32;
+        state_reset(st);
+        int i = static_cast<int>(pos - seg_start);
+        for (; m < m_end; m++, i++) {
+            issue_next();
+            const int stg = m & (kStages - 1);
+            const bool ok = !aborted &&
+                            mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
+            if (__all_sync(0xFFFFFFFFu, ok)) {
+                const uint32_t cb = code0 + stg * kCodeBytes, sb = scale0 + stg * kScaleBytes;
+                if (i == n_s - 1)
+                    process_page<true>(cb, sb, len - kPageSize * i, bq, sq, lane, st);
+                else
+                    process_page<false>(cb, sb, kPageSize, bq, sq, lane, st);
+            } else {
+                if (!aborted) {
+                    if (lane == 0)
+                        set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+                    drain_from = m;
+                }
+                aborted = true;
+            }
+            __syncwarp();
+        }
+        // reduce l and z over the 8 token rows (lanes differing in g)
 #pragma unroll
-            for (int i = 0; i < 8; i++)
-                dst[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
-            if (g == 0) {
-                mML[(warp - 1) * 16 + 2 * t] = st.m[0];
-                mML[(warp - 1) * 16 + 2 * t + 1] = st.m[1];
-                mML[(warp - 1) * 16 + 8 + 2 * t] = st.l[0];
-                mML[(warp - 1) * 16 + 8 + 2 * t + 1] = st.l[1];
+        for (int e = 0; e < 2; e++) {
+#pragma unroll
+            for (int d = 4; d <= 16; d <<= 1) {
+                st.l[e] += __shfl_xor_sync(0xFFFFFFFFu, st.l[e], d);
+                st.z[e] += __shfl_xor_sync(0xFFFFFFFFu, st.z[e], d);
             }
         }
-        __syncthreads();
-        if (warp == 0) {
-            for (int w = 1; w < kWarps; w++) {
-                const float4 *src = reinterpret_cast<const float4 *>(mO) + (w - 1) * 8 * 32;
-                float4 bo[8];
+        // undo the subnormal code scales (value rows g: low nibbles, g + 8: high nibbles)
+        // and add the zero-point term
 #pragma unroll
-                for (int i = 0; i < 8; i++)
-                    bo[i] = src[i * 32 + lane];
-                const float bm[2] = {mML[(w - 1) * 16 + 2 * t], mML[(w - 1) * 16 + 2 * t + 1]};
-                const float bl[2] = {mML[(w - 1) * 16 + 8 + 2 * t], mML[(w - 1) * 16 + 8 + 2 * t + 1]};
-                merge_into(st.m, st.l, st.o, bm, bl, bo);
-            }
+        for (int i2 = 0; i2 < 8; i2++) {
+            st.o[i2][0] = fmaf(st.o[i2][0], kLowNibble, st.z[0]);
+            st.o[i2][1] = fmaf(st.o[i2][1], kLowNibble, st.z[1]);
+            st.o[i2][2] = fmaf(st.o[i2][2], kHighNibble, st.z[0]);
+            st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
+        }
+        if (seg_start >= F0 && seg_end <= F1) {
+            finalize(p, s, h, lane, st.o, st.l);
+        } else {
             const int64_t seg = static_cast<int64_t>(s) * hkv + h;
-            const int64_t c_lo = cta_of(seg_start, P, C), c_hi = cta_of(seg_end - 1, P, C);
-            if (c_lo == c_hi) {
-                finalize(p, s, h, lane, st.o, st.l);
-            } else {
-                float *slot = p.partials + (seg + cta) * kSlotFloats;
-                float4 *so = reinterpret_cast<float4 *>(slot);
-#pragma unroll
-                for (int i = 0; i < 8; i++)
-                    so[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
-                if (g == 0) {
-                    slot[1024 + 2 * t] = st.m[0];
-                    slot[1024 + 2 * t + 1] = st.m[1];
-                    slot[1024 + 8 + 2 * t] = st.l[0];
-                    slot[1024 + 8 + 2 * t + 1] = st.l[1];
-                }
-                __threadfence();
-                __syncwarp();
-                uint32_t ticket = 0;
-                if (lane == 0)
-                    ticket = atomicAdd(p.tickets + seg, 1u);
-                ticket = __shfl_sync(0xFFFFFFFFu, ticket, 0);
-                if (ticket == static_cast<uint32_t>(c_hi - c_lo)) {
-                    // last CTA of this segment: fold in every CTA's partial, in CTA order
-                    // (its own included), so that the result does not depend on which CTA
-                    // finished last
-                    __threadfence();
-                    state_reset(st);
-                    for (int64_t c2 = c_lo; c2 <= c_hi; c2++) {
-                        const float *o2 = p.partials + (seg + c2) * kSlotFloats;
-                        const float4 *o24 = reinterpret_cast<const float4 *>(o2);
-                        float4 bo[8];
-#pragma unroll
-                        for (int i = 0; i < 8; i++)
-                            bo[i] = __ldcg(o24 + i * 32 + lane);
-                        const float bm[2] = {__ldcg(o2 + 1024 + 2 * t), __ldcg(o2 + 1024 + 2 * t + 1)};
-                        const float bl[2] = {__ldcg(o2 + 1032 + 2 * t), __ldcg(o2 + 1032 + 2 * t + 1)};
-                        merge_into(st.m, st.l, st.o, bm, bl, bo);
-                    }
-                    finalize(p, s, h, lane, st.o, st.l);
-                    if (lane == 0)
-                        p.tickets[seg] = 0u;   // ready for the next call
-                }
-            }
+            store_partial(p.partials + (seg + u) * kSlotFloats, lane, st);
         }
         pos = piece_end;
+        s = s_next;
+        h = h_next;
     }
 
-    // ---- 5. after an abort, let queued copies land before the CTA's shared memory is freed --
+    // ---- 4. after an abort, let queued copies land before the shared memory is released ----
     if (aborted) {
         for (int k = drain_from; k < issued; k++)
-            mbar_wait_bounded(bar0 + 8 * (k % kStages), (k / kStages) & 1, kWaitLimitNs / 10);
+            mbar_wait_bounded(bar0 + 8 * (k & (kStages - 1)), (k / kStages) & 1, kWaitLimitNs / 10);
+        mbar_wait_bounded(qbar, qphase, kWaitLimitNs / 10);
+    }
+}
+
+// Combine the pieces of every segment that was split across warps: slot segment + u holds
+// warp u's (m, l, o); the warps of a block fold disjoint subsets in a fixed order, then warp 0
+// folds the other warps' results in warp order and writes the rotated-back output, so the
+// result does not depend on timing.
+__global__ void __launch_bounds__(kMergeThreads)
+    paged_decode_merge_kernel(const DecodeParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    int32_t *pre = reinterpret_cast<int32_t *>(smem + kMergeSmemPrefix);
+    volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + kMergeSmemFlags);
+    float *slots = reinterpret_cast<float *>(smem + kMergeSmemSlots);
+
+    scan_pages(p, pre, flags, false);
+    Plan plan;
+    plan.init(pre, p.num_seqs, p.hkv, p.total_warps);
+    pdl_wait();   // the decode kernel's partials
+    if (plan.P == 0)
+        return;
+    const int64_t hkv = p.hkv;
+    const int64_t J = static_cast<int64_t>(p.num_seqs) * hkv;
+    for (int64_t seg = blockIdx.x; seg < J; seg += gridDim.x) {
+        const int s = static_cast<int>(seg / hkv), h = static_cast<int>(seg - s * hkv);
+        const int32_t n_s = pre[s + 1] - pre[s];
+        if (n_s == 0)
+            continue;
+        const int64_t u_lo = plan.warp_of_cost(plan.page_cost(s, h, 0));
+        const int64_t u_hi = plan.warp_of_cost(plan.page_cost(s, h, n_s - 1));
+        if (u_lo == u_hi)
+            continue;
+        WarpState st;
+        state_reset(st);
+        // each warp folds every kMergeWarps-th partial; two loads in flight per step
+        int64_t uu = u_lo + warp;
+        for (; uu + kMergeWarps <= u_hi; uu += 2 * kMergeWarps) {
+            float bm0[2], bl0[2], bm1[2], bl1[2];
+            float4 bo0[8], bo1[8];
+            load_partial(p.partials + (seg + uu) * kSlotFloats, lane, bm0, bl0, bo0);
+            load_partial(p.partials + (seg + uu + kMergeWarps) * kSlotFloats, lane, bm1, bl1, bo1);
+            merge_into(st.m, st.l, st.o, bm0, bl0, bo0);
+            merge_into(st.m, st.l, st.o, bm1, bl1, bo1);
+        }
+        if (uu <= u_hi) {
+            float bm[2], bl[2];
+            float4 bo[8];
+            load_partial(p.partials + (seg + uu) * kSlotFloats, lane, bm, bl, bo);
+            merge_into(st.m, st.l, st.o, bm, bl, bo);
+        }
+        if (warp > 0)
+            store_partial(slots + (warp - 1) * kSlotFloats, lane, st);
+        __syncthreads();
+        if (warp == 0) {
+            for (int w = 1; w < kMergeWarps; w++) {
+                float bm[2], bl[2];
+                float4 bo[8];
+                load_partial(slots + (w - 1) * kSlotFloats, lane, bm, bl, bo);
+                merge_into(st.m, st.l, st.o, bm, bl, bo);
+            }
+            finalize(p, s, h, lane, st.o, st.l);
+        }
+        __syncthreads();
     }
 }
 
@@ -718,25 +860,60 @@ PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
 
 }  // namespace
 
+namespace {
+
+struct LaunchShape {
+    int sms = 0;
+    int occ = 0;
+};
+
+// Multiprocessor count and decode-kernel occupancy for the current device and smem size
+// (looked up once per (device, size) and cached).
+cudaError_t launch_shape(size_t smem, LaunchShape &out)
+{
+    static std::mutex mu;
+    static int cached_dev = -1;
+    static size_t cached_smem = 0;
+    static LaunchShape cached;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    std::lock_guard<std::mutex> lock(mu);
+    if (dev == cached_dev && smem == cached_smem) {
+        out = cached;
+        return cudaSuccess;
+    }
+    LaunchShape ls;
+    e = cudaDeviceGetAttribute(&ls.sms, cudaDevAttrMultiProcessorCount, dev);
+    if (e == cudaSuccess)
+        e = cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                 static_cast<int>(smem));
+    if (e == cudaSuccess)
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ls.occ, paged_decode_kernel, kThreads, smem);
+    if (e != cudaSuccess)
+        return e;
+    if (ls.occ <= 0)
+        return cudaErrorInvalidConfiguration;
+    cached_dev = dev;
+    cached_smem = smem;
+    cached = ls;
+    out = ls;
+    return cudaSuccess;
+}
+
+}  // namespace
+
 size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs)
 {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
-    int dev = 0, sms = 0, occ = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess ||
-        cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+    LaunchShape ls;
+    if (launch_shape(decode_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
-    const size_t smem = decode_smem_bytes(num_seqs);
-    if (cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem)) != cudaSuccess ||
-        cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, paged_decode_kernel, kThreads, smem) !=
-            cudaSuccess ||
-        occ <= 0)
-        return 0;
-    const size_t grid = static_cast<size_t>(sms) * occ;
+    const size_t warps = static_cast<size_t>(ls.sms) * ls.occ * kWarps;
     const size_t segs = static_cast<size_t>(num_seqs) * num_kv_heads;
-    const size_t ticket_bytes = (segs * 4 + 255) & ~size_t(255);
-    return ticket_bytes + (grid + segs) * kSlotFloats * sizeof(float);
+    return (warps + segs) * kSlotFloats * sizeof(float);
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
@@ -767,16 +944,19 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
         cache.rows = rows;
     }
 
+    const size_t smem = decode_smem_bytes(a.num_seqs);
+    LaunchShape ls;
+    cudaError_t e = launch_shape(smem, ls);
+    if (e != cudaSuccess)
+        return e;
+
     DecodeParams p;
     p.q = static_cast<const uint16_t *>(a.q);
     p.scales = static_cast<const uint8_t *>(a.scales);
     p.block_table = a.block_table;
     p.seq_lens = a.seq_lens;
     p.out = a.out;
-    const size_t segs = static_cast<size_t>(a.num_seqs) * a.num_kv_heads;
-    const size_t ticket_bytes = (segs * 4 + 255) & ~size_t(255);
-    p.tickets = static_cast<uint32_t *>(a.workspace);
-    p.partials = reinterpret_cast<float *>(static_cast<uint8_t *>(a.workspace) + ticket_bytes);
+    p.partials = static_cast<float *>(a.workspace);
     p.status = a.status;
     p.num_pages = a.num_pages;
     p.max_blocks = a.max_blocks;
@@ -784,34 +964,40 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     p.hq = a.num_q_heads;
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
+    p.total_warps = ls.sms * ls.occ * kWarps;
     p.q_mult = static_cast<float>(static_cast<double>(kHadamardC) * a.sm_scale * 1.4426950408889634);
 
-    int dev = 0, sms = 0, occ = 0;
-    cudaError_t e = cudaGetDevice(&dev);
-    if (e == cudaSuccess)
-        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-    const size_t smem = decode_smem_bytes(a.num_seqs);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, paged_decode_kernel, kThreads, smem);
-    if (e != cudaSuccess)
-        return e;
-    if (occ <= 0)
-        return cudaErrorInvalidConfiguration;
-
-    cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(sms * occ));
-    cfg.blockDim = dim3(kThreads);
-    cfg.dynamicSmemBytes = smem;
-    cfg.stream = stream;
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
+
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(ls.sms * ls.occ));
+    cfg.blockDim = dim3(kThreads);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
     e = cudaLaunchKernelEx(&cfg, paged_decode_kernel, cache.map, p);
+    if (e != cudaSuccess)
+        return e;
+
+    const size_t msmem = merge_smem_bytes(a.num_seqs);
+    static size_t merge_smem_set = 0;
+    if (msmem > merge_smem_set) {
+        e = cudaFuncSetAttribute(paged_decode_merge_kernel,
+                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(msmem));
+        if (e != cudaSuccess)
+            return e;
+        merge_smem_set = msmem;
+    }
+    const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+    cudaLaunchConfig_t mcfg = cfg;
+    mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
+    mcfg.blockDim = dim3(kMergeThreads);
+    mcfg.dynamicSmemBytes = msmem;
+    mcfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&mcfg, paged_decode_merge_kernel, p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();

@@ -92,14 +92,13 @@ int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const 
                               void *stream);
 
 /* Bytes of workspace saw_paged_decode_attn / saw_decode_step need for this shape on the
- * current device (split-K partial results and per-(seq, kv head) merge counters).  Returns 0
- * for an unsupported or invalid shape. */
+ * current device (split-K partial results: one slot per warp of the decode grid plus one per
+ * (seq, kv head)).  Returns 0 for an unsupported or invalid shape. */
 size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
                                         int32_t num_seqs);
 
-/* Zero a workspace (cudaMemsetAsync on the stream).  Call once after allocating it: each
- * decode call leaves its merge counters at zero for the next one, so the workspace can be
- * reused without re-initialising unless a call was aborted. */
+/* Zero a workspace (cudaMemsetAsync on the stream).  Optional: the decode never reads a
+ * workspace byte it has not written in the same call. */
 int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, void *stream);
 
 /* Decode attention over the INT4 paged cache.
@@ -111,8 +110,11 @@ int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, voi
  * The kernel computes in fp16 x fp16 -> fp32 tensor-core tiles on raw codes with the scale
  * and zero applied in fp32 afterwards; results agree with an fp64 evaluation of the same
  * formula to about 1e-3.  A sequence with seq_lens[s] == 0 gets an all-zero output.
- * workspace: device memory of at least saw_paged_decode_workspace_bytes(), zeroed once by
- * saw_paged_decode_workspace_init(). */
+ * The work is cut into equal-cost runs of pages, one per warp of a persistent grid; sequences
+ * split across warps are combined by a second kernel queued right after the first (as its
+ * programmatic dependent), so one call queues two kernels.
+ * workspace: device memory of at least saw_paged_decode_workspace_bytes() bytes, 256-byte
+ * aligned; its contents need no initialisation and are scratch after the call. */
 int saw_paged_decode_attn(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
                           const uint8_t *kv_pages, const void *scales,
                           const int32_t *block_table, int32_t max_blocks_per_seq,
@@ -123,7 +125,8 @@ int saw_paged_decode_attn(const saw_cache_desc *cache, int32_t num_q_heads, cons
 /* One serving step: saw_rotate_quantize_paged on the num_new_tokens tokens (k_new, v_new,
  * slot_mapping), then saw_paged_decode_attn, queued back to back on the stream (the decode
  * kernel is launched as a programmatic dependent of the append so that its launch and
- * prologue overlap the append).  seq_lens must already count the appended tokens. */
+ * prologue overlap the append; the split-K merge kernel follows the same way).  seq_lens must
+ * already count the appended tokens. */
 int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
                     const void *k_new, const void *v_new, const int64_t *slot_mapping,
                     int64_t num_new_tokens, uint8_t *kv_pages, void *scales,
@@ -138,15 +141,15 @@ int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void
  * already owns the GPU, a request path that must not allocate (cudaMalloc synchronises the
  * device), or a host library that is only ever handed input and output pointers.  It computes
  * exactly what saw_paged_decode_attn computes, but its split-K scratch lives in one fixed array
- * of 12.75 MiB inside this library's device code (present on every GPU that loads the library,
+ * of 18.3 MiB inside this library's device code (present on every GPU that loads the library,
  * until the process exits) instead of a caller workspace.  It allocates nothing.
- * Limit: num_seqs * num_kv_heads <= 2048 and a decode grid of at most 1024 CTAs; larger
- * shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
+ * Limit: num_seqs * num_kv_heads <= 2048 and a decode grid of at most 2560 warps (a B200 runs
+ * 2368); larger shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
- * that device current); make that first call before any stream capture.  Every call clears the
- * array's merge counters with cudaMemsetAsync on `stream`.  All calls on a device share the
- * array and it keeps the previous call's contents, so calls that can overlap on the GPU (other
- * streams, other host threads) race on it: the caller must serialise them.
+ * that device current); make that first call before any stream capture.  Nothing in the array
+ * needs to start at zero.  All calls on a device share the array and it keeps the previous
+ * call's contents, so calls that can overlap on the GPU (other streams, other host threads)
+ * race on it: the caller must serialise them.
  * Arguments, layouts and the other status codes are those of saw_paged_decode_attn. */
 int saw_paged_decode_attn_static(const saw_cache_desc *cache, int32_t num_q_heads,
                                  const void *q, const uint8_t *kv_pages, const void *scales,
