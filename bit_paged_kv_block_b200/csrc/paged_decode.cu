@@ -43,11 +43,10 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;                              // power of two
+constexpr int kStages = 4;
 constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
 constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
-constexpr int kQBytes = 8 * kHeadDim * 2;               // raw bf16 queries of one kv head (G <= 8)
 constexpr int kSlotFloats = 32 * 32 + 16;               // O (lane layout) + m[8] + l[8]
 constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
 constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
@@ -55,21 +54,23 @@ constexpr float kHadamardC = 0.0883883461356163f;
 constexpr int kMergeWarps = 4;
 constexpr int kMergeThreads = 32 * kMergeWarps;
 
-// shared memory carve-up of the decode kernel (bytes, from a 1024-aligned base)
+// shared memory carve-up of the decode kernel (bytes, from a 1024-aligned base); the query
+// buffers (G * 256 bytes per warp) and the sequence prefix follow at run-time offsets
 constexpr int kSmemCodes = 0;
 constexpr int kSmemScales = kSmemCodes + kWarps * kStages * kCodeBytes;
-constexpr int kSmemQ = kSmemScales + kWarps * kStages * kScaleBytes;
-constexpr int kSmemBars = kSmemQ + kWarps * kQBytes;
+constexpr int kSmemBars = kSmemScales + kWarps * kStages * kScaleBytes;
 constexpr int kSmemFlags = kSmemBars + kWarps * (kStages + 1) * 8;
-constexpr int kSmemPrefix = kSmemFlags + 64;
+constexpr int kSmemQ = kSmemFlags + 64;
+__host__ __device__ constexpr int q_bytes(int group) { return group * kHeadDim * 2; }
+__host__ __device__ constexpr int smem_prefix_offset(int group) { return kSmemQ + kWarps * q_bytes(group); }
 // merge kernel: per-warp partials, then the prefix
 constexpr int kMergeSmemSlots = 0;
 constexpr int kMergeSmemFlags = kMergeSmemSlots + (kMergeWarps - 1) * kSlotFloats * 4;
 constexpr int kMergeSmemPrefix = kMergeSmemFlags + 64;
 
-size_t decode_smem_bytes(int32_t num_seqs)
+size_t decode_smem_bytes(int32_t num_seqs, int32_t group)
 {
-    return 1024 + kSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
+    return 1024 + smem_prefix_offset(group) + 4 * (static_cast<size_t>(num_seqs) + 1);
 }
 size_t merge_smem_bytes(int32_t num_seqs)
 {
@@ -584,7 +585,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int g = lane >> 2, t = lane & 3;
     const int S = p.num_seqs;
-    int32_t *pre = reinterpret_cast<int32_t *>(smem + kSmemPrefix);
+    int32_t *pre = reinterpret_cast<int32_t *>(smem + smem_prefix_offset(p.group));
     volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + kSmemFlags);
 
     // ---- 1. pages per sequence, the plan, zero outputs of empty sequences ------------------
@@ -611,7 +612,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     // ---- 2. this warp's copy ring ---------------------------------------------------------------
     const uint32_t code0 = smem_u32(smem + kSmemCodes) + warp * kStages * kCodeBytes;
     const uint32_t scale0 = smem_u32(smem + kSmemScales) + warp * kStages * kScaleBytes;
-    const uint32_t qbuf = smem_u32(smem + kSmemQ) + warp * kQBytes;
+    const uint32_t qbuf = smem_u32(smem + kSmemQ) + warp * q_bytes(p.group);
     const uint32_t bar0 = smem_u32(smem + kSmemBars) + warp * (kStages + 1) * 8;
     const uint32_t qbar = bar0 + kStages * 8;
     if (lane == 0)
@@ -651,6 +652,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     int32_t look_cur = lookup(lane), look_nxt = lookup(32 + lane);
     int issued = 0;        // pages queued so far
+    int istg = 0;          // ring stage of the next page to queue
     bool aborted = false;  // a wait gave up: stop queueing and computing
     int drain_from = 0;    // first page whose copy may still be in flight after an abort
     auto issue_next = [&]() {
@@ -662,7 +664,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             look_nxt = lookup(m + 32 + lane);
         }
         if (lane == (m & 31)) {
-            const int stg = m & (kStages - 1);
+            const int stg = istg;
             const uint32_t bar = bar0 + 8 * stg;
             mbar_arrive_expect_tx(bar, kTxBytes);
             tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, look_cur, bar);
@@ -670,6 +672,8 @@ __global__ void __launch_bounds__(kThreads, 4)
                      kScaleBytes, bar);
         }
         issued++;
+        if (++istg == kStages)
+            istg = 0;
     };
 
     // first piece's segment and its query
@@ -681,6 +685,8 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     // ---- 3. pieces ------------------------------------------------------------------------------
     int m = 0;
+    int cstg = 0;          // ring stage of page m
+    uint32_t cphase = 0;   // its mbarrier phase parity
     uint32_t qphase = 0;
     int64_t pos = F0;
     WarpState st;
@@ -721,9 +727,12 @@ __global__ void __launch_bounds__(kThreads, 4)
         int i = static_cast<int>(pos - seg_start);
         for (; m < m_end; m++, i++) {
             issue_next();
-            const int stg = m & (kStages - 1);
-            const bool ok = !aborted &&
-                            mbar_wait_bounded(bar0 + 8 * stg, (m / kStages) & 1, kWaitLimitNs);
+            const int stg = cstg;
+            const bool ok = !aborted && mbar_wait_bounded(bar0 + 8 * stg, cphase, kWaitLimitNs);
+            if (++cstg == kStages) {
+                cstg = 0;
+                cphase ^= 1;
+            }
             if (__all_sync(0xFFFFFFFFu, ok)) {
                 const uint32_t cb = code0 + stg * kCodeBytes, sb = scale0 + stg * kScaleBytes;
                 if (i == n_s - 1)
@@ -772,7 +781,7 @@ __global__ void __launch_bounds__(kThreads, 4)
     // ---- 4. after an abort, let queued copies land before the shared memory is released ----
     if (aborted) {
         for (int k = drain_from; k < issued; k++)
-            mbar_wait_bounded(bar0 + 8 * (k & (kStages - 1)), (k / kStages) & 1, kWaitLimitNs / 10);
+            mbar_wait_bounded(bar0 + 8 * (k % kStages), (k / kStages) & 1, kWaitLimitNs / 10);
         mbar_wait_bounded(qbar, qphase, kWaitLimitNs / 10);
     }
 }
@@ -842,22 +851,6 @@ __global__ void __launch_bounds__(kMergeThreads)
     }
 }
 
-// Tensor map over kv_pages seen as [num_pages * Hkv * 32 rows][64 bytes], box 32 x 64
-// (one (page, kv head) block), 64-byte swizzle.
-PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn()
-{
-    static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
-    if (fn == nullptr) {
-        void *ptr = nullptr;
-        cudaDriverEntryPointQueryResult q;
-        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) ==
-                cudaSuccess &&
-            q == cudaDriverEntryPointSuccess)
-            fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
-    }
-    return fn;
-}
-
 }  // namespace
 
 namespace {
@@ -909,7 +902,7 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
     LaunchShape ls;
-    if (launch_shape(decode_smem_bytes(num_seqs), ls) != cudaSuccess)
+    if (launch_shape(decode_smem_bytes(num_seqs, num_q_heads / num_kv_heads), ls) != cudaSuccess)
         return 0;
     const size_t warps = static_cast<size_t>(ls.sms) * ls.occ * kWarps;
     const size_t segs = static_cast<size_t>(num_seqs) * num_kv_heads;
@@ -925,7 +918,7 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     } cache;
     const int64_t rows = a.num_pages * a.num_kv_heads * 32;
     if (cache.base != a.kv_pages || cache.rows != rows) {
-        auto encode = get_encode_fn();
+        auto encode = tensor_map_encoder();
         if (encode == nullptr)
             return cudaErrorNotSupported;
         const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
@@ -944,7 +937,7 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
         cache.rows = rows;
     }
 
-    const size_t smem = decode_smem_bytes(a.num_seqs);
+    const size_t smem = decode_smem_bytes(a.num_seqs, a.num_q_heads / a.num_kv_heads);
     LaunchShape ls;
     cudaError_t e = launch_shape(smem, ls);
     if (e != cudaSuccess)

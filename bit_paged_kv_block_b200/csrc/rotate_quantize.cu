@@ -15,12 +15,18 @@
 //     divide where it might not.
 // This translation unit is compiled with -fmad=false as a second guard against contraction.
 //
-// Thread layout: two threads per head vector, 16 vectors (token, kv head) per warp.  Thread
-// half b of a vector holds the 64 elements j = 16a + 8b + r (a, r in 0..7): the 16-byte load a
-// covers elements 16a + 8b .. +7, so the two threads of a pair read one contiguous 32-byte
-// sector per load.  Stage h = 8 is the only one that crosses the pair (one shuffle); the
-// 64 elements are kept as 32 packed pairs X[8a + r] = (x[a][r], x[a + 4][r]) for a < 4.
+// Data movement: every warp streams its own tiles of 8 consecutive (token, kv head) vectors of K
+// and of V (2 KiB each) into a private 3-stage shared-memory ring with 2-D tensor copies (TMA,
+// 128-byte swizzle) completing on mbarriers, so warps never wait for each other.  The warps of
+// the persistent grid take tiles round-robin.
+//
+// Thread layout: two threads per head vector; a warp's tile has its 8 K vectors in lanes 0-15
+// and its 8 V vectors in lanes 16-31.  Thread half b of a vector holds the 64 elements
+// j = 16a + 8b + r (a, r in 0..7), read as eight 16-byte shared-memory loads that the 128-byte
+// swizzle spreads over all banks.  Stage h = 8 is the only one that crosses the pair (one
+// shuffle); the 64 elements are kept as 32 packed pairs X[8a + r] = (x[a][r], x[a + 4][r]).
 #include <cfloat>
+#include <algorithm>
 
 #include "saw_device.cuh"
 #include "saw_internal.h"
@@ -28,8 +34,15 @@
 namespace saw {
 namespace {
 
-constexpr int kRqThreads = 256;
-constexpr int kRqVecsPerWarp = 16;
+constexpr int kTileVecs = 8;                           // (token, kv head) vectors per warp tile
+constexpr int kTileBytes = kTileVecs * kHeadDim * 2;   // 2 KiB of K (or of V) per tile
+constexpr int kRqStages = 3;
+constexpr int kRqWarps = 4;
+constexpr int kRqThreads = 32 * kRqWarps;
+constexpr int kRqStageBytes = 2 * kTileBytes;
+constexpr int kRqSmemBars = kRqWarps * kRqStages * kRqStageBytes;
+constexpr size_t kRqSmemBytes = 1024 + kRqSmemBars + kRqWarps * kRqStages * 8;
+constexpr uint64_t kRqWaitLimitNs = 1000000000ull;
 constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
 constexpr float kRoundMagic = 12582912.0f;           // 1.5 * 2^23
 // A code computed from the reciprocal is provably the IEEE-divide code unless the remainder
@@ -47,12 +60,17 @@ __device__ __forceinline__ uint64_t shfl_xor_u64(uint32_t mask, uint64_t v, int 
 __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-// Load this thread's 64 bf16 elements of one head vector (8 x 16 bytes).
-__device__ __forceinline__ void load_half_vec(const uint8_t *row, int b, uint4 raw[8])
+
+// This thread's 64 bf16 elements of tile vector vt (rows 2 vt and 2 vt + 1 of 128 bytes; the
+// 16-byte chunk c of row r sits at chunk c ^ (r & 7) under the 128-byte swizzle).
+__device__ __forceinline__ void load_half_vec(uint32_t tile, int vt, int b, uint4 raw[8])
 {
 #pragma unroll
-    for (int a = 0; a < 8; a++)
-        raw[a] = ldg_stream16(row + 32 * a + 16 * b);
+    for (int a = 0; a < 8; a++) {
+        const int row = 2 * vt + (a >> 2);
+        const int chunk = (2 * (a & 3) + b) ^ (row & 7);
+        raw[a] = lds128(tile + row * 128 + chunk * 16);
+    }
 }
 
 __device__ __forceinline__ void to_pairs(const uint4 raw[8], uint64_t X[32])
@@ -179,10 +197,9 @@ __device__ __forceinline__ uint32_t pack8(const uint32_t tt[8])
 }
 
 struct RqParams {
-    const uint8_t *k;
-    const uint8_t *v;
     const int64_t *slot_mapping;
     int64_t num_vecs;        // T * Hkv
+    int64_t num_tiles;
     int32_t hkv;
     int64_t num_slots;       // num_pages * 16
     uint8_t *kv_pages;
@@ -190,8 +207,8 @@ struct RqParams {
     uint32_t *status;
 };
 
-// Quantize the vector (held rotated in X) and store codes + scale for one of K (sel 0) / V (1).
-__device__ __forceinline__ void quantize_store(uint64_t X[32], const uint8_t *src_row, int b,
+// Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
+__device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, int vt, int b,
                                                int lane, bool store, int64_t row,
                                                const RqParams &p)
 {
@@ -232,7 +249,7 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], const uint8_t *sr
     if (pair_exact) {
         const uint32_t pair_mask = 3u << (lane & ~1);
         uint4 raw[8];
-        load_half_vec(src_row, b, raw);
+        load_half_vec(tile, vt, b, raw);
         to_pairs(raw, X);
         fwht128(X, b, pair_mask);
         quantize_exact(X, mn, scale);
@@ -258,46 +275,110 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], const uint8_t *sr
     }
 }
 
-__global__ void __launch_bounds__(kRqThreads, 2) rotate_quantize_kernel(const RqParams p)
+__global__ void __launch_bounds__(kRqThreads, 4)
+    rotate_quantize_kernel(const __grid_constant__ CUtensorMap tk,
+                           const __grid_constant__ CUtensorMap tv, const RqParams p)
 {
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
-    const int lane = threadIdx.x & 31;
+    // all indices below fit in 32 bits: the host limits num_vecs to 2^29
+    const uint32_t W = gridDim.x * kRqWarps;
+    const uint32_t wg = blockIdx.x * kRqWarps + warp;
+    const uint32_t num_tiles = static_cast<uint32_t>(p.num_tiles);
+    if (wg >= num_tiles)
+        return;
+    const int n = static_cast<int>((num_tiles - wg + W - 1) / W);   // this warp's tiles: wg + i W
+    const uint32_t ring = smem_u32(smem) + warp * kRqStages * kRqStageBytes;
+    const uint32_t bar0 = smem_u32(smem + kRqSmemBars) + warp * kRqStages * 8;
+    if (lane == 0)
+        for (int i = 0; i < kRqStages; i++)
+            mbar_init(bar0 + 8 * i, 1);
+    mbar_init_fence();
+    __syncwarp();
+
+    int issued = 0, istg = 0;
+    uint32_t itile = wg;
+    auto issue = [&]() {
+        if (issued < n) {
+            if (lane == 0) {
+                const uint32_t dst = ring + istg * kRqStageBytes;
+                const int32_t y = static_cast<int32_t>(itile * (2 * kTileVecs));
+                mbar_arrive_expect_tx(bar0 + 8 * istg, kRqStageBytes);
+                tma_load_2d(dst, &tk, 0, y, bar0 + 8 * istg);
+                tma_load_2d(dst + kTileBytes, &tv, 0, y, bar0 + 8 * istg);
+            }
+            issued++;
+            itile += W;
+            if (++istg == kRqStages)
+                istg = 0;
+        }
+    };
+    for (int k = 0; k < kRqStages - 1; k++)
+        issue();
+
+    const int half = lane >> 4;          // 0: K, 1: V
     const int b = lane & 1;
-    const int64_t warp_global = (static_cast<int64_t>(blockIdx.x) * kRqThreads + threadIdx.x) >> 5;
-    const int64_t vec_raw = warp_global * kRqVecsPerWarp + (lane >> 1);
-    if (warp_global * kRqVecsPerWarp >= p.num_vecs)
-        return;                                      // whole warp past the end
-    const bool in_range = vec_raw < p.num_vecs;
-    const int64_t vec = in_range ? vec_raw : p.num_vecs - 1;   // tail lanes recompute the last
-    const int64_t tok = vec / p.hkv;
-    const int h = static_cast<int>(vec - tok * p.hkv);
+    const int vt = (lane >> 1) & 7;
+    const uint32_t num_vecs = static_cast<uint32_t>(p.num_vecs);
+    const uint32_t hkv = static_cast<uint32_t>(p.hkv);
+    uint32_t tile = wg;
+    // slot of this thread's vector in the tile (prefetched one tile ahead)
+    auto slot_of = [&](uint32_t t, uint32_t &vec) -> int64_t {
+        const uint32_t vec_raw = t * kTileVecs + vt;
+        vec = vec_raw < num_vecs ? vec_raw : num_vecs - 1;
+        return p.slot_mapping[vec / hkv];
+    };
+    uint32_t vec_next;
+    int64_t slot_next = slot_of(tile, vec_next);
+    int cstg = 0;
+    uint32_t cphase = 0;
+    int i = 0;
+    for (; i < n; i++, tile += W) {
+        issue();
+        const uint32_t vec = vec_next;
+        const bool in_range = tile * kTileVecs + vt < num_vecs;
+        const int64_t slot = slot_next;
+        if (i + 1 < n)
+            slot_next = slot_of(tile + W, vec_next);
+        const int stg = cstg;
+        const bool ok = mbar_wait_bounded(bar0 + 8 * stg, cphase, kRqWaitLimitNs);
+        if (++cstg == kRqStages) {
+            cstg = 0;
+            cphase ^= 1;
+        }
+        if (!__all_sync(0xFFFFFFFFu, ok)) {
+            if (lane == 0)
+                set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+            break;
+        }
+        const uint32_t tok = vec / hkv;
+        const uint32_t h = vec - tok * hkv;
+        bool store = in_range && slot >= 0;
+        if (store && slot >= p.num_slots) {
+            if (b == 0 && half == 0)
+                set_status(p.status, SAW_DEV_BAD_SLOT);
+            store = false;
+        }
+        const int64_t page = store ? slot >> 4 : 0;    // slot / 16
+        const int64_t off = store ? slot & 15 : 0;
+        const int64_t row = ((page * p.hkv + h) * 2 + half) * kPageSize + off;
 
-    const int64_t slot = p.slot_mapping[tok];
-    bool store = in_range && slot >= 0;
-    if (store && slot >= p.num_slots) {
-        if (b == 0)
-            set_status(p.status, SAW_DEV_BAD_SLOT);
-        store = false;
+        const uint32_t tile_smem = ring + stg * kRqStageBytes + half * kTileBytes;
+        uint4 raw[8];
+        load_half_vec(tile_smem, vt, b, raw);
+        uint64_t X[32];
+        to_pairs(raw, X);
+        fwht128(X, b, 0xFFFFFFFFu);
+        quantize_store(X, tile_smem, vt, b, lane, store, row, p);
+        __syncwarp();
     }
-    const int64_t page = store ? slot / kPageSize : 0;
-    const int64_t off = store ? slot - page * kPageSize : 0;
-    const int64_t row_k = ((page * p.hkv + h) * 2 + 0) * kPageSize + off;
-    const int64_t row_v = row_k + kPageSize;
-
-    const uint8_t *k_row = p.k + vec * (kHeadDim * 2);
-    const uint8_t *v_row = p.v + vec * (kHeadDim * 2);
-    uint4 raw_k[8], raw_v[8];
-    load_half_vec(k_row, b, raw_k);
-    load_half_vec(v_row, b, raw_v);
-
-    uint64_t X[32];
-    to_pairs(raw_k, X);
-    fwht128(X, b, 0xFFFFFFFFu);
-    quantize_store(X, k_row, b, lane, store, row_k, p);
-
-    to_pairs(raw_v, X);
-    fwht128(X, b, 0xFFFFFFFFu);
-    quantize_store(X, v_row, b, lane, store, row_v, p);
+    if (i < n) {
+        // a wait gave up: let every queued copy land before the shared memory is released
+        for (int k = i; k < issued; k++)
+            mbar_wait_bounded(bar0 + 8 * (k % kRqStages), (k / kRqStages) & 1, kRqWaitLimitNs / 10);
+    }
 }
 
 }  // namespace
@@ -306,23 +387,72 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
                                    bool trigger_dependents)
 {
     (void)trigger_dependents;   // the kernel always releases dependents at its start
+    const int64_t num_vecs = a.num_tokens * a.num_kv_heads;
+    if (num_vecs == 0)
+        return cudaSuccess;
+    if (num_vecs > (int64_t(1) << 29))
+        return cudaErrorInvalidValue;       // tensor-map rows (2 per vector) must fit in int32
+
+    static thread_local struct {
+        const void *k = nullptr, *v = nullptr;
+        int64_t num_vecs = 0;
+        CUtensorMap mk, mv;
+    } cache;
+    if (cache.k != a.k || cache.v != a.v || cache.num_vecs != num_vecs) {
+        auto encode = tensor_map_encoder();
+        if (encode == nullptr)
+            return cudaErrorNotSupported;
+        const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(2 * num_vecs)};
+        const cuuint64_t strides[1] = {128};
+        const cuuint32_t box[2] = {128, 2 * kTileVecs};   // one warp tile: 16 rows of 128 B
+        const cuuint32_t estr[2] = {1, 1};
+        for (int which = 0; which < 2; which++) {
+            CUresult r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
+                                const_cast<void *>(which ? a.v : a.k), dims, strides, box, estr,
+                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            if (r != CUDA_SUCCESS) {
+                cache.k = nullptr;
+                return cudaErrorInvalidValue;
+            }
+        }
+        cache.k = a.k;
+        cache.v = a.v;
+        cache.num_vecs = num_vecs;
+    }
+
     RqParams p;
-    p.k = static_cast<const uint8_t *>(a.k);
-    p.v = static_cast<const uint8_t *>(a.v);
     p.slot_mapping = a.slot_mapping;
-    p.num_vecs = a.num_tokens * a.num_kv_heads;
+    p.num_vecs = num_vecs;
+    p.num_tiles = (num_vecs + kTileVecs - 1) / kTileVecs;
     p.hkv = a.num_kv_heads;
     p.num_slots = a.num_pages * kPageSize;
     p.kv_pages = a.kv_pages;
     p.scales = static_cast<uint32_t *>(a.scales);
     p.status = a.status;
-    if (p.num_vecs == 0)
-        return cudaSuccess;
-    const int64_t warps = (p.num_vecs + kRqVecsPerWarp - 1) / kRqVecsPerWarp;
-    const int64_t blocks = (warps * 32 + kRqThreads - 1) / kRqThreads;
-    if (blocks > 0x7FFFFFFF)
-        return cudaErrorInvalidValue;
-    rotate_quantize_kernel<<<static_cast<unsigned>(blocks), kRqThreads, 0, stream>>>(p);
+
+    static int sms = 0, occ = 0;
+    if (sms == 0) {
+        int dev = 0;
+        cudaError_t e = cudaGetDevice(&dev);
+        if (e == cudaSuccess)
+            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        if (e == cudaSuccess)
+            e = cudaFuncSetAttribute(rotate_quantize_kernel,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(kRqSmemBytes));
+        if (e == cudaSuccess)
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotate_quantize_kernel,
+                                                              kRqThreads, kRqSmemBytes);
+        if (e != cudaSuccess || occ <= 0) {
+            sms = 0;
+            return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
+        }
+    }
+    const int64_t grid = std::min<int64_t>((p.num_tiles + kRqWarps - 1) / kRqWarps,
+                                           static_cast<int64_t>(sms) * occ);
+    rotate_quantize_kernel<<<static_cast<unsigned>(grid), kRqThreads, kRqSmemBytes, stream>>>(cache.mk, cache.mv, p);
     return cudaGetLastError();
 }
 

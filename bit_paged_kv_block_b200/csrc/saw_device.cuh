@@ -132,6 +132,20 @@ __device__ __forceinline__ uint64_t globaltimer_ns()
     return t;
 }
 
+// Like mbar_try_wait, but the thread may sleep until the phase completes or about
+// `suspend_ns` nanoseconds have passed, instead of returning at once.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint32_t bar, uint32_t phase, uint32_t suspend_ns)
+{
+    uint32_t ok;
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "mbarrier.try_wait.parity.acquire.cta.shared::cta.b64 p, [%1], %2, %3;\n\t"
+                 "selp.u32 %0, 1, 0, p;\n\t}"
+                 : "=r"(ok)
+                 : "r"(bar), "r"(phase), "r"(suspend_ns)
+                 : "memory");
+    return ok != 0;
+}
+
 // Wait for phase `phase` of the mbarrier, giving up after `limit_ns` nanoseconds.
 __device__ __forceinline__ bool mbar_wait_bounded(uint32_t bar, uint32_t phase, uint64_t limit_ns)
 {

@@ -4,8 +4,24 @@
 #include <cstddef>
 #include <cstdint>
 #include <cuda_runtime.h>
+#include <cudaTypedefs.h>
 
 namespace saw {
+
+// cuTensorMapEncodeTiled from the driver, looked up through the runtime (no libcuda link).
+inline PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder()
+{
+    static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+        void *ptr = nullptr;
+        cudaDriverEntryPointQueryResult q;
+        if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+                cudaSuccess ||
+            q != cudaDriverEntryPointSuccess)
+            ptr = nullptr;
+        return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(ptr);
+    }();
+    return fn;
+}
 
 struct RotateQuantizeArgs {
     const void *k;               // bf16 [T][Hkv][128]
