@@ -60,6 +60,29 @@ def dist_env():
             int(os.environ.get("WORLD_SIZE", "1")))
 
 
+# ---- ranks (weak scaling: each rank serves its own batch; no exchange on the data path) ------
+
+def rank_workload(rank: int):
+    """The decode workload rank `rank` serves: the same shapes on every rank, its own seed."""
+    from bit_paged_kv_block_b200 import synth
+    return synth.make_workload("decode", seed=rank)
+
+
+def max_over_ranks(value: float, pg=None, device="cpu") -> float:
+    """The maximum of `value` over all ranks of the process group (the value itself alone)."""
+    if pg is None:
+        return float(value)
+    import torch
+    t = torch.tensor([float(value)], device=device, dtype=torch.float64)
+    pg.all_reduce(t, op=pg.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(units_per_rank: int, world: int, ms_per_step_max: float) -> float:
+    """Whole-job units per second: every rank's units over the slowest rank's step time."""
+    return world * units_per_rank / (ms_per_step_max / 1e3)
+
+
 # ---- byte accounting (algorithmic bytes, not measured traffic) ----------------------------
 
 def decode_bytes(wl) -> int:
@@ -263,7 +286,7 @@ def run_saw(args):
         pg = dist
 
     # ---- inputs: each rank serves its own batch (weak scaling, no exchange on the path) ----
-    wl = synth.make_workload("decode", seed=rank)
+    wl = rank_workload(rank)
     kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
     seq, pos = synth.token_index(wl, "history")
     saw.saw_rotate_quantize_paged(synth.kv_values(wl, "K", tokens="history", device=dev),
@@ -305,13 +328,11 @@ def run_saw(args):
     ms = e0.elapsed_time(e1)
     if pg:
         pg.barrier()
-        t = torch.tensor([ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ms, pg, dev)
     if int(status.item()) != 0:
         raise RuntimeError(f"device status {int(status.item()):#x}")
     ms_per_step = ms / args.steps
-    value = world * wl.num_seqs / (ms_per_step / 1e3)
+    value = job_throughput(wl.num_seqs, world, ms_per_step)
 
     # ---- per-kernel durations (same inputs, events around each launch) ---------------------
     n_kt = max(20, min(args.steps, 400))
@@ -390,12 +411,8 @@ def run_saw(args):
         e2e_step()
     e1.record(stream)
     torch.cuda.synchronize()
-    e2e_ms = e0.elapsed_time(e1) / n_e2e
-    if pg:
-        t = torch.tensor([e2e_ms], device=dev, dtype=torch.float64)
-        pg.all_reduce(t, op=pg.ReduceOp.MAX)
-        e2e_ms = float(t.item())
-    e2e = {"value": world * wl.num_seqs / (e2e_ms / 1e3), "unit": UNIT,
+    e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, pg, dev)
+    e2e = {"value": job_throughput(wl.num_seqs, world, e2e_ms), "unit": UNIT,
            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": n_e2e,
            "ms_per_step": e2e_ms}
 
