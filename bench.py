@@ -382,7 +382,46 @@ def run_saw(args):
                  "frac_of_measured_peak": rq_gbs / peak_gbs, "launch_ms": t_rq,
                  "algorithmic_bytes_per_launch": rq_bytes,
                  "traffic": kernel_traffic("rotate_quantize_kernel", pre.total_tokens)}
+
+    # ---- the plain INT4 baseline (no rotation) on the same workloads: rotation overhead -------
+    def mean_event_ms(fn, n):
+        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+        for e in evs:
+            e[0].record(stream)
+            fn()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+        return statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+
+    for _ in range(3):
+        saw.saw_quantize_paged_plain(pk, pv, pslots, pkv, psc, stream=stream)
+    t_rq_plain = mean_event_ms(lambda: saw.saw_quantize_paged_plain(pk, pv, pslots, pkv, psc,
+                                                                    stream=stream), n_rq)
     del pk, pv, pkv, psc
+    pkv2, psc2 = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
+    seq, pos = synth.token_index(wl, "history")
+    saw.saw_quantize_paged_plain(synth.kv_values(wl, "K", tokens="history", device=dev),
+                                 synth.kv_values(wl, "V", tokens="history", device=dev),
+                                 torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(dev),
+                                 pkv2, psc2)
+    plain_step = lambda: saw.saw_decode_step_plain(q, k_new, v_new, slots, pkv2, psc2, table, lens,
+                                                   out, ws, dev_status=status, stream=stream)
+    for _ in range(3):
+        plain_step()
+    torch.cuda.synchronize()
+    n_pl = max(20, min(args.steps, 2000))
+    e0.record(stream)
+    for _ in range(n_pl):
+        plain_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    pl_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
+    plain_int4 = {"what": "the same step and prefill quantize on a plain INT4 cache (H = I)",
+                  "step_ms": pl_ms, "tokens_per_s": job_throughput(wl.num_seqs, world, pl_ms),
+                  "step_rotation_overhead": ms_per_step / pl_ms - 1.0,
+                  "prefill_quant_launch_ms": t_rq_plain,
+                  "prefill_quant_rotation_overhead": t_rq / t_rq_plain - 1.0}
+    del pkv2, psc2
 
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
@@ -433,9 +472,10 @@ def run_saw(args):
         "step_GBps": (dec_bytes + append_bytes(wl.num_seqs, wl.num_kv_heads)) / (ms_per_step * 1e-3) / 1e9,
         "roofline": roofline,
         "rot_quant": rot_quant,
+        "plain_int4": plain_int4,
         "append_launch_ms": t_append,
         "e2e": e2e,
-        "gpu_launches": 2 * args.steps,
+        "gpu_launches": 3 * args.steps,
         "clocks": clocks.summary(),
         "cpu_baseline": base,
     }

@@ -267,6 +267,7 @@ __device__ __forceinline__ void state_reset(WarpState &st)
 // Rotated, scaled query of (seq s, kv head h) as fp16 mma B fragments, from the raw bf16
 // queries of the group in shared memory ([G][128] at qbuf).
 // Thread (g, t) owns query head g of the group and d in [32t, 32t + 32).
+template <bool kRotate>
 __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int g, int t,
                                            uint32_t bq[8][2], float sq_out[2])
 {
@@ -287,9 +288,10 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
         for (int l = 0; l < 32; l++)
             x[l] = 0.0f;
     }
-    // Hadamard butterfly: d bits 0..4 in registers, bits 5, 6 across lanes t ^ 1, t ^ 2.
+    // Hadamard butterfly: d bits 0..4 in registers, bits 5, 6 across lanes t ^ 1, t ^ 2
+    // (skipped for the plain INT4 cache).
 #pragma unroll
-    for (int hb = 1; hb < 32; hb <<= 1)
+    for (int hb = 1; kRotate && hb < 32; hb <<= 1)
 #pragma unroll
         for (int l = 0; l < 32; l++)
             if ((l & hb) == 0) {
@@ -298,7 +300,7 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
                 x[l + hb] = a - b;
             }
 #pragma unroll
-    for (int lb = 1; lb <= 2; lb <<= 1) {
+    for (int lb = 1; kRotate && lb <= 2; lb <<= 1) {
         const bool high = (t & lb) != 0;
 #pragma unroll
         for (int l = 0; l < 32; l++) {
@@ -476,7 +478,9 @@ __device__ __forceinline__ void merge_into(float am[2], float al[2], float ao[8]
     }
 }
 
-// o_r = o / l, out = H o_r for the heads this thread holds; written to out[s][h G + 2t + e].
+// o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the heads this thread
+// holds; written to out[s][h G + 2t + e].
+template <bool kRotate>
 __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, int lane,
                                          float o[8][4], const float l[2])
 {
@@ -494,7 +498,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, in
             v[e][c][3] = o[2 * c + 1][2 + e] * inv[e];
         }
 #pragma unroll
-    for (int e = 0; e < 2; e++) {
+    for (int e = 0; kRotate && e < 2; e++) {
         // d bits 0, 1 (j) and 5, 6 (c) in registers
 #pragma unroll
         for (int c = 0; c < 4; c++)
@@ -538,8 +542,9 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, in
             float *dst = p.out + ((static_cast<int64_t>(s) * p.hq + h * p.group + head) * kHeadDim);
 #pragma unroll
             for (int c = 0; c < 4; c++) {
-                const float4 val = make_float4(v[e][c][0] * kHadamardC, v[e][c][1] * kHadamardC,
-                                               v[e][c][2] * kHadamardC, v[e][c][3] * kHadamardC);
+                const float f = kRotate ? kHadamardC : 1.0f;
+                const float4 val = make_float4(v[e][c][0] * f, v[e][c][1] * f, v[e][c][2] * f,
+                                               v[e][c][3] * f);
                 *reinterpret_cast<float4 *>(dst + 32 * c + 4 * g) = val;
             }
         }
@@ -577,6 +582,7 @@ __device__ __forceinline__ void load_partial(const float *slot, int lane, float 
     bl[1] = slot[1032 + 2 * t + 1];
 }
 
+template <bool kRotate>
 __global__ void __launch_bounds__(kThreads, 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
 {
@@ -709,7 +715,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             aborted = true;
         }
         qphase ^= 1;
-        load_query(p, qbuf, g, t, bq, sq);
+        load_query<kRotate>(p, qbuf, g, t, bq, sq);
         __syncwarp();
         int s_next = s, h_next = h;
         if (piece_end < F1) {
@@ -768,7 +774,7 @@ __global__ void __launch_bounds__(kThreads, 4)
             st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
         }
         if (seg_start >= F0 && seg_end <= F1) {
-            finalize(p, s, h, lane, st.o, st.l);
+            finalize<kRotate>(p, s, h, lane, st.o, st.l);
         } else {
             const int64_t seg = static_cast<int64_t>(s) * hkv + h;
             store_partial(p.partials + (seg + u) * kSlotFloats, lane, st);
@@ -790,6 +796,7 @@ __global__ void __launch_bounds__(kThreads, 4)
 // warp u's (m, l, o); the warps of a block fold disjoint subsets in a fixed order, then warp 0
 // folds the other warps' results in warp order and writes the rotated-back output, so the
 // result does not depend on timing.
+template <bool kRotate>
 __global__ void __launch_bounds__(kMergeThreads)
     paged_decode_merge_kernel(const DecodeParams p)
 {
@@ -845,7 +852,7 @@ __global__ void __launch_bounds__(kMergeThreads)
                 load_partial(slots + (w - 1) * kSlotFloats, lane, bm, bl, bo);
                 merge_into(st.m, st.l, st.o, bm, bl, bo);
             }
-            finalize(p, s, h, lane, st.o, st.l);
+            finalize<kRotate>(p, s, h, lane, st.o, st.l);
         }
         __syncthreads();
     }
@@ -860,38 +867,59 @@ struct LaunchShape {
     int occ = 0;
 };
 
-// Multiprocessor count and decode-kernel occupancy for the current device and smem size
-// (looked up once per (device, size) and cached).
-cudaError_t launch_shape(size_t smem, LaunchShape &out)
+// Multiprocessor count and decode-kernel occupancy for the current device and smem size.  The
+// dynamic shared-memory attributes of both kernels (both variants) are raised per device as
+// needed; everything is cached per device.
+cudaError_t launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
 {
+    constexpr int kMaxDevices = 64;
+    struct DevState {
+        int sms = 0;
+        size_t decode_attr = 0, merge_attr = 0;
+        size_t occ_smem = 0;
+        int occ = 0;
+    };
     static std::mutex mu;
-    static int cached_dev = -1;
-    static size_t cached_smem = 0;
-    static LaunchShape cached;
+    static DevState st[kMaxDevices];
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
     std::lock_guard<std::mutex> lock(mu);
-    if (dev == cached_dev && smem == cached_smem) {
-        out = cached;
-        return cudaSuccess;
-    }
-    LaunchShape ls;
-    e = cudaDeviceGetAttribute(&ls.sms, cudaDevAttrMultiProcessorCount, dev);
-    if (e == cudaSuccess)
-        e = cudaFuncSetAttribute(paged_decode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                 static_cast<int>(smem));
-    if (e == cudaSuccess)
-        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&ls.occ, paged_decode_kernel, kThreads, smem);
-    if (e != cudaSuccess)
+    DevState &d = st[dev];
+    if (d.sms == 0 && (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
-    if (ls.occ <= 0)
-        return cudaErrorInvalidConfiguration;
-    cached_dev = dev;
-    cached_smem = smem;
-    cached = ls;
-    out = ls;
+    if (smem > d.decode_attr) {
+        for (int r = 0; r < 2 && e == cudaSuccess; r++)
+            e = cudaFuncSetAttribute(r ? paged_decode_kernel<true> : paged_decode_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(smem));
+        if (e != cudaSuccess)
+            return e;
+        d.decode_attr = smem;
+    }
+    if (merge_smem > d.merge_attr) {
+        for (int r = 0; r < 2 && e == cudaSuccess; r++)
+            e = cudaFuncSetAttribute(r ? paged_decode_merge_kernel<true> : paged_decode_merge_kernel<false>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(merge_smem));
+        if (e != cudaSuccess)
+            return e;
+        d.merge_attr = merge_smem;
+    }
+    if (smem != d.occ_smem) {
+        int occ = 0;
+        e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, paged_decode_kernel<true>, kThreads, smem);
+        if (e != cudaSuccess)
+            return e;
+        if (occ <= 0)
+            return cudaErrorInvalidConfiguration;
+        d.occ = occ;
+        d.occ_smem = smem;
+    }
+    out.sms = d.sms;
+    out.occ = d.occ;
     return cudaSuccess;
 }
 
@@ -902,7 +930,7 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
     LaunchShape ls;
-    if (launch_shape(decode_smem_bytes(num_seqs, num_q_heads / num_kv_heads), ls) != cudaSuccess)
+    if (launch_shape(decode_smem_bytes(num_seqs, num_q_heads / num_kv_heads), merge_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
     const size_t warps = static_cast<size_t>(ls.sms) * ls.occ * kWarps;
     const size_t segs = static_cast<size_t>(num_seqs) * num_kv_heads;
@@ -938,8 +966,9 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     }
 
     const size_t smem = decode_smem_bytes(a.num_seqs, a.num_q_heads / a.num_kv_heads);
+    const size_t msmem = merge_smem_bytes(a.num_seqs);
     LaunchShape ls;
-    cudaError_t e = launch_shape(smem, ls);
+    cudaError_t e = launch_shape(smem, msmem, ls);
     if (e != cudaSuccess)
         return e;
 
@@ -958,7 +987,9 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
     p.total_warps = ls.sms * ls.occ * kWarps;
-    p.q_mult = static_cast<float>(static_cast<double>(kHadamardC) * a.sm_scale * 1.4426950408889634);
+    // q carries sm_scale * log2(e), and 1/sqrt(128) of the (unnormalised) query butterfly
+    p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(kHadamardC) : 1.0) * a.sm_scale *
+                                  1.4426950408889634);
 
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
@@ -971,26 +1002,18 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, paged_decode_kernel, cache.map, p);
+    e = cudaLaunchKernelEx(&cfg, a.rotate ? paged_decode_kernel<true> : paged_decode_kernel<false>,
+                           cache.map, p);
     if (e != cudaSuccess)
         return e;
 
-    const size_t msmem = merge_smem_bytes(a.num_seqs);
-    static size_t merge_smem_set = 0;
-    if (msmem > merge_smem_set) {
-        e = cudaFuncSetAttribute(paged_decode_merge_kernel,
-                                 cudaFuncAttributeMaxDynamicSharedMemorySize, static_cast<int>(msmem));
-        if (e != cudaSuccess)
-            return e;
-        merge_smem_set = msmem;
-    }
     const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&mcfg, paged_decode_merge_kernel, p);
+    e = cudaLaunchKernelEx(&mcfg, a.rotate ? paged_decode_merge_kernel<true> : paged_decode_merge_kernel<false>, p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();

@@ -208,6 +208,8 @@ struct RqParams {
 };
 
 // Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
+// kRotate = false is the plain INT4 quantizer (H = I) used as the unrotated baseline.
+template <bool kRotate>
 __device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, int vt, int b,
                                                int lane, bool store, int64_t row,
                                                const RqParams &p)
@@ -251,7 +253,8 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, in
         uint4 raw[8];
         load_half_vec(tile, vt, b, raw);
         to_pairs(raw, X);
-        fwht128(X, b, pair_mask);
+        if (kRotate)
+            fwht128(X, b, pair_mask);
         quantize_exact(X, mn, scale);
     }
 
@@ -275,6 +278,7 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, in
     }
 }
 
+template <bool kRotate>
 __global__ void __launch_bounds__(kRqThreads, 4)
     rotate_quantize_kernel(const __grid_constant__ CUtensorMap tk,
                            const __grid_constant__ CUtensorMap tv, const RqParams p)
@@ -370,8 +374,9 @@ __global__ void __launch_bounds__(kRqThreads, 4)
         load_half_vec(tile_smem, vt, b, raw);
         uint64_t X[32];
         to_pairs(raw, X);
-        fwht128(X, b, 0xFFFFFFFFu);
-        quantize_store(X, tile_smem, vt, b, lane, store, row, p);
+        if (kRotate)
+            fwht128(X, b, 0xFFFFFFFFu);
+        quantize_store<kRotate>(X, tile_smem, vt, b, lane, store, row, p);
         __syncwarp();
     }
     if (i < n) {
@@ -432,27 +437,36 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     p.scales = static_cast<uint32_t *>(a.scales);
     p.status = a.status;
 
-    static int sms = 0, occ = 0;
-    if (sms == 0) {
-        int dev = 0;
-        cudaError_t e = cudaGetDevice(&dev);
-        if (e == cudaSuccess)
-            e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        if (e == cudaSuccess)
-            e = cudaFuncSetAttribute(rotate_quantize_kernel,
+    // per device: multiprocessor count, the shared-memory attribute and the occupancy
+    constexpr int kMaxDevices = 64;
+    static int sms_of[kMaxDevices] = {}, occ_of[kMaxDevices] = {};
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess)
+        return e;
+    if (dev < 0 || dev >= kMaxDevices)
+        return cudaErrorInvalidDevice;
+    auto kernel = a.rotate ? rotate_quantize_kernel<true> : rotate_quantize_kernel<false>;
+    if (sms_of[dev] == 0) {
+        int sms = 0, occ = 0;
+        e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+        for (int r = 0; r < 2 && e == cudaSuccess; r++)
+            e = cudaFuncSetAttribute(r ? rotate_quantize_kernel<true> : rotate_quantize_kernel<false>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kRqSmemBytes));
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotate_quantize_kernel,
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotate_quantize_kernel<true>,
                                                               kRqThreads, kRqSmemBytes);
-        if (e != cudaSuccess || occ <= 0) {
-            sms = 0;
-            return e != cudaSuccess ? e : cudaErrorInvalidConfiguration;
-        }
+        if (e != cudaSuccess)
+            return e;
+        if (occ <= 0)
+            return cudaErrorInvalidConfiguration;
+        occ_of[dev] = occ;
+        sms_of[dev] = sms;
     }
     const int64_t grid = std::min<int64_t>((p.num_tiles + kRqWarps - 1) / kRqWarps,
-                                           static_cast<int64_t>(sms) * occ);
-    rotate_quantize_kernel<<<static_cast<unsigned>(grid), kRqThreads, kRqSmemBytes, stream>>>(cache.mk, cache.mv, p);
+                                           static_cast<int64_t>(sms_of[dev]) * occ_of[dev]);
+    kernel<<<static_cast<unsigned>(grid), kRqThreads, kRqSmemBytes, stream>>>(cache.mk, cache.mv, p);
     return cudaGetLastError();
 }
 

@@ -125,17 +125,15 @@ const char *saw_status_string(int status)
     }
 }
 
-int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const void *v,
-                              const int64_t *slot_mapping, int64_t num_tokens,
-                              uint8_t *kv_pages, void *scales, uint32_t *dev_status,
-                              void *stream)
+}  // extern "C"
+
+namespace {
+
+saw::RotateQuantizeArgs append_args(const saw_cache_desc *cache, const void *k, const void *v,
+                                    const int64_t *slot_mapping, int64_t num_tokens,
+                                    uint8_t *kv_pages, void *scales, uint32_t *dev_status,
+                                    bool rotate)
 {
-    int rc = check_cache(cache);
-    if (rc != SAW_OK)
-        return rc;
-    rc = check_append(cache, k, v, slot_mapping, num_tokens, kv_pages, scales);
-    if (rc != SAW_OK || num_tokens == 0)
-        return rc;
     saw::RotateQuantizeArgs a;
     a.k = k;
     a.v = v;
@@ -146,9 +144,103 @@ int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const 
     a.kv_pages = kv_pages;
     a.scales = scales;
     a.status = dev_status;
+    a.rotate = rotate;
+    return a;
+}
+
+int append_impl(const saw_cache_desc *cache, const void *k, const void *v,
+                const int64_t *slot_mapping, int64_t num_tokens, uint8_t *kv_pages, void *scales,
+                uint32_t *dev_status, void *stream, bool rotate)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k, v, slot_mapping, num_tokens, kv_pages, scales);
+    if (rc != SAW_OK || num_tokens == 0)
+        return rc;
+    const saw::RotateQuantizeArgs a =
+        append_args(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status, rotate);
     return saw::launch_rotate_quantize(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
                ? SAW_OK
                : SAW_ERR_CUDA;
+}
+
+int decode_impl(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                const uint8_t *kv_pages, const void *scales, const int32_t *block_table,
+                int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                uint32_t *dev_status, void *stream, bool rotate)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    saw::DecodeArgs a =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    a.rotate = rotate;
+    return saw::launch_paged_decode(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? SAW_OK
+               : SAW_ERR_CUDA;
+}
+
+int step_impl(const saw_cache_desc *cache, int32_t num_q_heads, const void *q, const void *k_new,
+              const void *v_new, const int64_t *slot_mapping, int64_t num_new_tokens,
+              uint8_t *kv_pages, void *scales, const int32_t *block_table,
+              int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+              float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+              uint32_t *dev_status, void *stream, bool rotate)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k_new, v_new, slot_mapping, num_new_tokens, kv_pages, scales);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
+    if (rc != SAW_OK)
+        return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool appended = num_new_tokens > 0;
+    if (appended) {
+        const saw::RotateQuantizeArgs a = append_args(cache, k_new, v_new, slot_mapping,
+                                                      num_new_tokens, kv_pages, scales,
+                                                      dev_status, rotate);
+        if (saw::launch_rotate_quantize(a, s, true) != cudaSuccess)
+            return SAW_ERR_CUDA;
+    }
+    if (num_seqs == 0)
+        return SAW_OK;
+    saw::DecodeArgs d =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    d.rotate = rotate;
+    return saw::launch_paged_decode(d, s, appended) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const void *v,
+                              const int64_t *slot_mapping, int64_t num_tokens,
+                              uint8_t *kv_pages, void *scales, uint32_t *dev_status,
+                              void *stream)
+{
+    return append_impl(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status,
+                       stream, true);
+}
+
+int saw_quantize_paged_plain(const saw_cache_desc *cache, const void *k, const void *v,
+                             const int64_t *slot_mapping, int64_t num_tokens, uint8_t *kv_pages,
+                             void *scales, uint32_t *dev_status, void *stream)
+{
+    return append_impl(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status,
+                       stream, false);
 }
 
 size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
@@ -179,19 +271,21 @@ int saw_paged_decode_attn(const saw_cache_desc *cache, int32_t num_q_heads, cons
                           float *out, void *workspace, size_t workspace_bytes,
                           uint32_t *dev_status, void *stream)
 {
-    int rc = check_cache(cache);
-    if (rc != SAW_OK)
-        return rc;
-    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
-                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
-    if (rc != SAW_OK || num_seqs == 0)
-        return rc;
-    const saw::DecodeArgs a =
-        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
-                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
-    return saw::launch_paged_decode(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
-               ? SAW_OK
-               : SAW_ERR_CUDA;
+    return decode_impl(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                       seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status,
+                       stream, true);
+}
+
+int saw_paged_decode_attn_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                                const uint8_t *kv_pages, const void *scales,
+                                const int32_t *block_table, int32_t max_blocks_per_seq,
+                                const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                                float *out, void *workspace, size_t workspace_bytes,
+                                uint32_t *dev_status, void *stream)
+{
+    return decode_impl(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                       seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status,
+                       stream, false);
 }
 
 int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
@@ -202,38 +296,22 @@ int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void
                     void *workspace, size_t workspace_bytes, uint32_t *dev_status,
                     void *stream)
 {
-    int rc = check_cache(cache);
-    if (rc != SAW_OK)
-        return rc;
-    rc = check_append(cache, k_new, v_new, slot_mapping, num_new_tokens, kv_pages, scales);
-    if (rc != SAW_OK)
-        return rc;
-    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
-                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
-    if (rc != SAW_OK)
-        return rc;
-    const cudaStream_t s = static_cast<cudaStream_t>(stream);
-    const bool appended = num_new_tokens > 0;
-    if (appended) {
-        saw::RotateQuantizeArgs a;
-        a.k = k_new;
-        a.v = v_new;
-        a.slot_mapping = slot_mapping;
-        a.num_tokens = num_new_tokens;
-        a.num_kv_heads = cache->num_kv_heads;
-        a.num_pages = cache->num_pages;
-        a.kv_pages = kv_pages;
-        a.scales = scales;
-        a.status = dev_status;
-        if (saw::launch_rotate_quantize(a, s, true) != cudaSuccess)
-            return SAW_ERR_CUDA;
-    }
-    if (num_seqs == 0)
-        return SAW_OK;
-    const saw::DecodeArgs d =
-        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
-                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
-    return saw::launch_paged_decode(d, s, appended) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+    return step_impl(cache, num_q_heads, q, k_new, v_new, slot_mapping, num_new_tokens,
+                     kv_pages, scales, block_table, max_blocks_per_seq, seq_lens, num_seqs,
+                     sm_scale, out, workspace, workspace_bytes, dev_status, stream, true);
+}
+
+int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                          const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                          int64_t num_new_tokens, uint8_t *kv_pages, void *scales,
+                          const int32_t *block_table, int32_t max_blocks_per_seq,
+                          const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
+                          void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                          void *stream)
+{
+    return step_impl(cache, num_q_heads, q, k_new, v_new, slot_mapping, num_new_tokens,
+                     kv_pages, scales, block_table, max_blocks_per_seq, seq_lens, num_seqs,
+                     sm_scale, out, workspace, workspace_bytes, dev_status, stream, false);
 }
 
 }  // extern "C"

@@ -33,6 +33,7 @@ struct RotateQuantizeArgs {
     uint8_t *kv_pages;           // [num_pages][Hkv][2][16][64]
     void *scales;                // fp16 [num_pages][Hkv][2][16][2]
     uint32_t *status;            // nullable
+    bool rotate = true;          // false: plain INT4 (no Hadamard rotation)
 };
 
 struct DecodeArgs {
@@ -51,6 +52,7 @@ struct DecodeArgs {
     void *workspace;
     size_t workspace_bytes;
     uint32_t *status;
+    bool rotate = true;          // false: plain INT4 cache (no query / output rotation)
 };
 
 // Queue the rotate+quantize+scatter kernel.  `trigger_dependents` makes the kernel release

@@ -69,6 +69,12 @@ def _open_library() -> ctypes.CDLL:
     lib.saw_decode_step.argtypes = [D, i32, P, P, P, P, i64, P, P, P, i32, P, i32, f32, P, P,
                                     sz, P, P]
     lib.saw_decode_step.restype = ctypes.c_int
+    lib.saw_quantize_paged_plain.argtypes = lib.saw_rotate_quantize_paged.argtypes
+    lib.saw_quantize_paged_plain.restype = ctypes.c_int
+    lib.saw_paged_decode_attn_plain.argtypes = lib.saw_paged_decode_attn.argtypes
+    lib.saw_paged_decode_attn_plain.restype = ctypes.c_int
+    lib.saw_decode_step_plain.argtypes = lib.saw_decode_step.argtypes
+    lib.saw_decode_step_plain.restype = ctypes.c_int
     return lib
 
 
@@ -137,6 +143,18 @@ def allocate_cache(num_pages: int, num_kv_heads: int, device="cuda"):
 def saw_rotate_quantize_paged(k, v, slot_mapping, kv_pages, scales, dev_status=None,
                               stream=None) -> None:
     """Rotate, quantize and scatter new tokens k, v (bf16 [T][Hkv][128]) into the cache."""
+    _append(lib.saw_rotate_quantize_paged, "saw_rotate_quantize_paged", k, v, slot_mapping,
+            kv_pages, scales, dev_status, stream)
+
+
+def saw_quantize_paged_plain(k, v, slot_mapping, kv_pages, scales, dev_status=None,
+                             stream=None) -> None:
+    """Plain INT4 baseline: quantize and scatter without the Hadamard rotation."""
+    _append(lib.saw_quantize_paged_plain, "saw_quantize_paged_plain", k, v, slot_mapping,
+            kv_pages, scales, dev_status, stream)
+
+
+def _append(fn, name, k, v, slot_mapping, kv_pages, scales, dev_status, stream) -> None:
     _need(k, "k", torch.bfloat16, 3)
     _need(v, "v", torch.bfloat16, 3)
     _need(slot_mapping, "slot_mapping", torch.int64, 1)
@@ -152,10 +170,9 @@ def saw_rotate_quantize_paged(k, v, slot_mapping, kv_pages, scales, dev_status=N
         raise ValueError("scales must be [num_pages][Hkv][2][16][2]")
     if dev_status is not None:
         _need(dev_status, "dev_status", torch.int32, 1)
-    rc = lib.saw_rotate_quantize_paged(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(slot_mapping),
-                                       T, _ptr(kv_pages), _ptr(scales), _ptr(dev_status),
-                                       _stream(stream))
-    _check(rc, "saw_rotate_quantize_paged")
+    rc = fn(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(kv_pages),
+            _ptr(scales), _ptr(dev_status), _stream(stream))
+    _check(rc, name)
 
 
 def saw_paged_decode_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,
@@ -204,20 +221,45 @@ def _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace, d
 def saw_paged_decode_attn(q, kv_pages, scales, block_table, seq_lens, out, workspace,
                           sm_scale=None, dev_status=None, stream=None) -> None:
     """Decode attention of q (bf16 [S][Hq][128]) over the INT4 paged cache into out (fp32)."""
+    _decode(lib.saw_paged_decode_attn, "saw_paged_decode_attn", q, kv_pages, scales, block_table,
+            seq_lens, out, workspace, sm_scale, dev_status, stream)
+
+
+def saw_paged_decode_attn_plain(q, kv_pages, scales, block_table, seq_lens, out, workspace,
+                                sm_scale=None, dev_status=None, stream=None) -> None:
+    """Decode over a plain INT4 cache (written by saw_quantize_paged_plain)."""
+    _decode(lib.saw_paged_decode_attn_plain, "saw_paged_decode_attn_plain", q, kv_pages, scales,
+            block_table, seq_lens, out, workspace, sm_scale, dev_status, stream)
+
+
+def _decode(fn, name, q, kv_pages, scales, block_table, seq_lens, out, workspace, sm_scale,
+            dev_status, stream) -> None:
     desc, S, hq = _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace,
                                  dev_status)
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(HEAD_DIM)
-    rc = lib.saw_paged_decode_attn(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages), _ptr(scales),
-                                   _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
-                                   float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
-                                   _ptr(dev_status), _stream(stream))
-    _check(rc, "saw_paged_decode_attn")
+    rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages), _ptr(scales), _ptr(block_table),
+            block_table.shape[1], _ptr(seq_lens), S, float(sm_scale), _ptr(out), _ptr(workspace),
+            workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(rc, name)
 
 
 def saw_decode_step(q, k_new, v_new, slot_mapping, kv_pages, scales, block_table, seq_lens, out,
                     workspace, sm_scale=None, dev_status=None, stream=None) -> None:
     """Append k_new / v_new (bf16 [T][Hkv][128]) at slot_mapping, then decode q."""
+    _step(lib.saw_decode_step, "saw_decode_step", q, k_new, v_new, slot_mapping, kv_pages, scales,
+          block_table, seq_lens, out, workspace, sm_scale, dev_status, stream)
+
+
+def saw_decode_step_plain(q, k_new, v_new, slot_mapping, kv_pages, scales, block_table, seq_lens,
+                          out, workspace, sm_scale=None, dev_status=None, stream=None) -> None:
+    """The serving step on a plain INT4 cache (no rotation)."""
+    _step(lib.saw_decode_step_plain, "saw_decode_step_plain", q, k_new, v_new, slot_mapping,
+          kv_pages, scales, block_table, seq_lens, out, workspace, sm_scale, dev_status, stream)
+
+
+def _step(fn, name, q, k_new, v_new, slot_mapping, kv_pages, scales, block_table, seq_lens, out,
+          workspace, sm_scale, dev_status, stream) -> None:
     desc, S, hq = _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace,
                                  dev_status)
     _need(k_new, "k_new", torch.bfloat16, 3)
@@ -230,12 +272,11 @@ def saw_decode_step(q, k_new, v_new, slot_mapping, kv_pages, scales, block_table
         raise ValueError("slot_mapping must have one entry per new token")
     if sm_scale is None:
         sm_scale = 1.0 / math.sqrt(HEAD_DIM)
-    rc = lib.saw_decode_step(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new),
-                             _ptr(slot_mapping), T, _ptr(kv_pages), _ptr(scales),
-                             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
-                             float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
-                             _ptr(dev_status), _stream(stream))
-    _check(rc, "saw_decode_step")
+    rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T,
+            _ptr(kv_pages), _ptr(scales), _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
+            S, float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+            _stream(stream))
+    _check(rc, name)
 
 
 def saw_paged_decode_attn_static(q, kv_pages, scales, block_table, seq_lens, out, sm_scale=None,

@@ -135,6 +135,32 @@ int saw_decode_step(const saw_cache_desc *cache, int32_t num_q_heads, const void
                     void *workspace, size_t workspace_bytes, uint32_t *dev_status,
                     void *stream);
 
+/* Plain INT4 baseline (H = I): the same token-wise asymmetric INT4 quantizer, page layout and
+ * decode kernels without the Hadamard rotation -- the "naive INT4" the SAW-INT4 page compares
+ * against ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving",
+ * Concerns Raised: naive INT4 degrades accuracy; Research Findings: SAW-INT4 matches the
+ * throughput of plain INT4 and its fused rotation adds no measurable overhead).  Arguments,
+ * layouts, workspace and status codes are those of the rotated entry points; a cache written by
+ * saw_quantize_paged_plain must be read by the *_plain decode (codes are not rotated, and q and
+ * the output are not rotated either).  Codes and scales are bit-identical to the definition at
+ * the top of this file with the rotation step removed. */
+int saw_quantize_paged_plain(const saw_cache_desc *cache, const void *k, const void *v,
+                             const int64_t *slot_mapping, int64_t num_tokens, uint8_t *kv_pages,
+                             void *scales, uint32_t *dev_status, void *stream);
+int saw_paged_decode_attn_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                                const uint8_t *kv_pages, const void *scales,
+                                const int32_t *block_table, int32_t max_blocks_per_seq,
+                                const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
+                                float *out, void *workspace, size_t workspace_bytes,
+                                uint32_t *dev_status, void *stream);
+int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                          const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                          int64_t num_new_tokens, uint8_t *kv_pages, void *scales,
+                          const int32_t *block_table, int32_t max_blocks_per_seq,
+                          const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
+                          void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                          void *stream);
+
 /* saw_paged_decode_attn for callers that cannot allocate device memory.
  * The pages have no counterpart of this entry point: it exists for callers that are not allowed
  * or not able to call cudaMalloc -- a plug-in inside a serving framework whose memory pool
