@@ -18,9 +18,9 @@
 // a second kernel (paged_decode_merge_kernel), launched as a programmatic dependent.
 //
 // Per page (16 tokens x one kv head, 2 KiB of codes + 128 B of scales), per warp:
-//   * the lane that looked the page up queues a 2-D tensor copy of the 32 code rows (64B
-//     swizzle, so the K reads and the transposed V reads below are bank-conflict free) and a
-//     1-D bulk copy of the scales into a 4-stage ring, completion on an mbarrier (bounded wait);
+//   * one elected lane queues a 2-D tensor copy of the 32 code rows (64B swizzle, so the K
+//     reads and the transposed V reads below are bank-conflict free) and a 1-D bulk copy of the
+//     scales into a 4-stage ring, completion on an mbarrier (bounded wait), three pages ahead;
 //   * S^T[16 tok x 8 heads] = K_codes[16 x 128] . Q^T with mma.m16n8k16 (fp16 in, fp32 acc):
 //     the codes are exact fp16 subnormals, and s = scale * acc + zero * sum(q) in fp32;
 //   * online softmax in the log2 domain (q carries sm_scale * log2 e);
@@ -34,6 +34,7 @@
 #include <cudaTypedefs.h>
 
 #include <mutex>
+#include <type_traits>
 
 #include "saw_device.cuh"
 #include "saw_internal.h"
@@ -43,7 +44,7 @@ namespace {
 
 constexpr int kWarps = 4;
 constexpr int kThreads = 32 * kWarps;
-constexpr int kStages = 4;
+constexpr int kStages = 4;                              // power of two
 constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
 constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
@@ -377,15 +378,17 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
             s[2] = s[3] = -INFINITY;
     }
 
-    float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
-#pragma unroll
-    for (int e = 0; e < 2; e++) {
-        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
-        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 8));
-        mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 16));
-    }
-    const bool grow = mx[0] > st.m[0] || mx[1] > st.m[1];
+    // The running max only changes when some logit of the page exceeds it, so the cross-lane
+    // reduction is needed only then (rare once a piece is a few pages long).
+    const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
     if (__any_sync(0xFFFFFFFFu, grow)) {
+        float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 8));
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 16));
+        }
         float alpha[2];
 #pragma unroll
         for (int e = 0; e < 2; e++) {
@@ -582,6 +585,24 @@ __device__ __forceinline__ void load_partial(const float *slot, int lane, float 
     bl[1] = slot[1032 + 2 * t + 1];
 }
 
+// One elected lane of the (converged) warp arms the stage's mbarrier with the page's bytes and
+// queues the 2-D tensor copy of its code rows and the 1-D bulk copy of its scales; no branch.
+__device__ __forceinline__ void copy_page_elected(uint32_t bar, uint32_t dst_codes, const void *tmap,
+                                                  int32_t row, uint32_t dst_scales,
+                                                  const void *src_scales)
+{
+    asm volatile("{\n\t.reg .pred p;\n\t"
+                 "elect.sync _|p, 0xffffffff;\n\t"
+                 "@p mbarrier.arrive.expect_tx.release.cta.shared::cta.b64 _, [%0], %6;\n\t"
+                 "@p cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%1], [%2, {%7, %3}], [%0];\n\t"
+                 "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5], %8, [%0];\n\t"
+                 "}"
+                 ::"r"(bar), "r"(dst_codes), "l"(tmap), "r"(row), "r"(dst_scales), "l"(src_scales),
+                 "r"(kTxBytes), "r"(0), "r"(static_cast<uint32_t>(kScaleBytes))
+                 : "memory");
+}
+
 template <bool kRotate>
 __global__ void __launch_bounds__(kThreads, 4)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
@@ -656,57 +677,70 @@ __global__ void __launch_bounds__(kThreads, 4)
 
     pdl_wait();   // the cache may be written by the kernel this one depends on
 
-    int32_t look_cur = lookup(lane), look_nxt = lookup(32 + lane);
-    int issued = 0;        // pages queued so far
-    int istg = 0;          // ring stage of the next page to queue
+    // Lanes hold the tensor-map rows of pages [look_base, look_base + 32) of the run in look_a
+    // and of the 32 after them in look_b, whose block-table reads are thus in flight 32 pages
+    // ahead of their use.
+    int32_t look_a = lookup(lane), look_b = lookup(32 + lane);
+    int look_base = 0;
+    int issued = 0;        // pages queued so far (pages are queued in order)
     bool aborted = false;  // a wait gave up: stop queueing and computing
     int drain_from = 0;    // first page whose copy may still be in flight after an abort
+    // queue page `issued` of the run into ring stage issued % kStages (warp-uniform call)
     auto issue_next = [&]() {
-        if (issued >= n_w || aborted)
-            return;
-        const int m = issued;
-        if (m > 0 && (m & 31) == 0) {
-            look_cur = look_nxt;
-            look_nxt = lookup(m + 32 + lane);
+        const int j = issued++;
+        if (j >= look_base + 32) {
+            look_base += 32;
+            look_a = look_b;
+            look_b = lookup(look_base + 32 + lane);
         }
-        if (lane == (m & 31)) {
-            const int stg = istg;
-            const uint32_t bar = bar0 + 8 * stg;
-            mbar_arrive_expect_tx(bar, kTxBytes);
-            tma_load_2d(code0 + stg * kCodeBytes, &tmap, 0, look_cur, bar);
-            bulk_g2s(scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(look_cur) * 4,
-                     kScaleBytes, bar);
-        }
-        issued++;
-        if (++istg == kStages)
-            istg = 0;
+        const int32_t row = __shfl_sync(0xFFFFFFFFu, look_a, j & 31);
+        const int stg = j & (kStages - 1);
+        copy_page_elected(bar0 + 8 * stg, code0 + stg * kCodeBytes, &tmap, row,
+                          scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(row) * 4);
     };
 
     // first piece's segment and its query
     int s = find_seq(pre, S, F0, hkv);
     int h = static_cast<int>((F0 - hkv * pre[s]) / (pre[s + 1] - pre[s]));
     issue_query(s, h);
-    for (int k = 0; k < kStages - 1; k++)
+    while (issued < kStages - 1 && issued < n_w)
         issue_next();
+
+    WarpState st;
+    uint32_t bq[8][2];
+    float sq[2];
+    // Page m of the run: queue the page kStages - 1 ahead into the stage page m - 1 used, wait
+    // for page m and attend over its first `valid` tokens (kMask) or all of them.
+    auto step = [&](auto mask_tag, int m, int valid) {
+        if (issued < n_w && !aborted)
+            issue_next();
+        const int stg = m & (kStages - 1);
+        const uint32_t phase = (static_cast<uint32_t>(m) / kStages) & 1u;
+        const bool ok = !aborted && mbar_wait_bounded(bar0 + 8 * stg, phase, kWaitLimitNs);
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            process_page<decltype(mask_tag)::value>(code0 + stg * kCodeBytes, scale0 + stg * kScaleBytes,
+                                                    valid, bq, sq, lane, st);
+        } else if (!aborted) {
+            if (lane == 0)
+                set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+            drain_from = m;
+            aborted = true;
+        }
+        __syncwarp();
+    };
 
     // ---- 3. pieces ------------------------------------------------------------------------------
     int m = 0;
-    int cstg = 0;          // ring stage of page m
-    uint32_t cphase = 0;   // its mbarrier phase parity
     uint32_t qphase = 0;
     int64_t pos = F0;
-    WarpState st;
     while (pos < F1) {
         const int32_t n_s = pre[s + 1] - pre[s];
         const int64_t seg_start = hkv * pre[s] + static_cast<int64_t>(h) * n_s;
         const int64_t seg_end = seg_start + n_s;
-        const int64_t piece_end = seg_end < F1 ? seg_end : F1;
-        const int m_end = static_cast<int>(piece_end - F0);
-        const int len = p.seq_lens[s];
+        const bool ends_segment = seg_end <= F1;
+        const int m_end = static_cast<int>((ends_segment ? seg_end : F1) - F0);
 
         // this piece's query: wait for its copy, build the fragments, then queue the next one
-        uint32_t bq[8][2];
-        float sq[2];
         const bool qok = !aborted && mbar_wait_bounded(qbar, qphase, kWaitLimitNs);
         if (!__all_sync(0xFFFFFFFFu, qok) && !aborted) {
             if (lane == 0)
@@ -718,7 +752,7 @@ __global__ void __launch_bounds__(kThreads, 4)
         load_query<kRotate>(p, qbuf, g, t, bq, sq);
         __syncwarp();
         int s_next = s, h_next = h;
-        if (piece_end < F1) {
+        if (m_end < n_w) {
             if (++h_next == p.hkv) {
                 h_next = 0;
                 do {
@@ -729,32 +763,16 @@ __global__ void __launch_bounds__(kThreads, 4)
                 issue_query(s_next, h_next);
         }
 
+        // all pages but a segment's last are full
         state_reset(st);
-        int i = static_cast<int>(pos - seg_start);
-        for (; m < m_end; m++, i++) {
-            issue_next();
-            const int stg = cstg;
-            const bool ok = !aborted && mbar_wait_bounded(bar0 + 8 * stg, cphase, kWaitLimitNs);
-            if (++cstg == kStages) {
-                cstg = 0;
-                cphase ^= 1;
-            }
-            if (__all_sync(0xFFFFFFFFu, ok)) {
-                const uint32_t cb = code0 + stg * kCodeBytes, sb = scale0 + stg * kScaleBytes;
-                if (i == n_s - 1)
-                    process_page<true>(cb, sb, len - kPageSize * i, bq, sq, lane, st);
-                else
-                    process_page<false>(cb, sb, kPageSize, bq, sq, lane, st);
-            } else {
-                if (!aborted) {
-                    if (lane == 0)
-                        set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
-                    drain_from = m;
-                }
-                aborted = true;
-            }
-            __syncwarp();
+        const int m_full = ends_segment ? m_end - 1 : m_end;
+        for (; m < m_full; m++)
+            step(std::false_type(), m, kPageSize);
+        if (ends_segment) {
+            step(std::true_type(), m, p.seq_lens[s] - kPageSize * (n_s - 1));
+            m++;
         }
+
         // reduce l and z over the 8 token rows (lanes differing in g)
 #pragma unroll
         for (int e = 0; e < 2; e++) {
@@ -773,13 +791,13 @@ __global__ void __launch_bounds__(kThreads, 4)
             st.o[i2][2] = fmaf(st.o[i2][2], kHighNibble, st.z[0]);
             st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
         }
-        if (seg_start >= F0 && seg_end <= F1) {
+        if (seg_start >= F0 && ends_segment) {
             finalize<kRotate>(p, s, h, lane, st.o, st.l);
         } else {
             const int64_t seg = static_cast<int64_t>(s) * hkv + h;
             store_partial(p.partials + (seg + u) * kSlotFloats, lane, st);
         }
-        pos = piece_end;
+        pos = F0 + m_end;
         s = s_next;
         h = h_next;
     }
@@ -787,7 +805,8 @@ __global__ void __launch_bounds__(kThreads, 4)
     // ---- 4. after an abort, let queued copies land before the shared memory is released ----
     if (aborted) {
         for (int k = drain_from; k < issued; k++)
-            mbar_wait_bounded(bar0 + 8 * (k % kStages), (k / kStages) & 1, kWaitLimitNs / 10);
+            mbar_wait_bounded(bar0 + 8 * (k & (kStages - 1)), (static_cast<uint32_t>(k) / kStages) & 1u,
+                              kWaitLimitNs / 10);
         mbar_wait_bounded(qbar, qphase, kWaitLimitNs / 10);
     }
 }
