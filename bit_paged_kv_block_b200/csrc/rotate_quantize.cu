@@ -10,9 +10,9 @@
 //     Sylvester transform, stage h = 1, 2, ..., 64 in that order, then one multiply by
 //     fp32(1/sqrt(128)); two fp32 operations are issued per packed f32x2 instruction, each
 //     individually rounded, so the lane layout does not change any result;
-//   * scale = (max - min) / 15 uses the IEEE divide; the codes use a reciprocal, see
-//     quantize_fast() for why that gives the IEEE-divide code, and fall back to the IEEE
-//     divide where it might not.
+//   * scale = (max - min) / 15 uses the IEEE divide; the codes use a reciprocal (the note
+//     above code_bits_tie() shows why that gives the IEEE-divide code) and fall back to the
+//     IEEE divide where it might not.
 // This translation unit is compiled with -fmad=false as a second guard against contraction.
 //
 // Data movement: every warp streams its own tiles of 8 consecutive (token, kv head) vectors of K
@@ -46,7 +46,7 @@ constexpr uint64_t kRqWaitLimitNs = 1000000000ull;
 constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
 constexpr float kRoundMagic = 12582912.0f;           // 1.5 * 2^23
 // A code computed from the reciprocal is provably the IEEE-divide code unless the remainder
-// is within 2^-18 of one half (derivation at quantize_fast()).
+// is within 2^-18 of one half (derivation above code_bits_tie()).
 constexpr float kNearHalf = 0.5f - 1.0f / 262144.0f;
 
 __device__ __forceinline__ uint64_t shfl_xor_u64(uint32_t mask, uint64_t v, int delta)
@@ -147,40 +147,48 @@ __device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
 //   res = RN(d r - k) is the remainder to within 2^-26.
 // |d r - Q| <= Q 2^-24 < 2^-20 and |RN(Q) - Q| <= 2^-21, so if |res| < 0.5 - 2^-18 then
 // |RN(Q) - k| < 0.5 and rint(RN(d / s)) = k, which is the code the IEEE divide gives (no
-// clamp is needed: k <= 15).  Otherwise the caller recomputes with the IEEE divide.
-// On return X holds t (code = low 4 bits); the result is the largest |res| seen.
-__device__ __forceinline__ float quantize_fast(uint64_t X[32], float mn, float r)
+// clamp is needed: k <= 15).  Otherwise the code is decided as follows.
+//
+// Near a half-way quotient the code follows from the sign of one exact remainder instead of a
+// divide.  Let m = k +- 1/2 be the half-integer next to Q (0.5 <= m <= 14.5, since 0 <= Q <=
+// 15 (1 + 2^-23)) and E = d - m s.  RN(Q) = m exactly when |Q - m| <= ulp(m) / 2 (m has an even
+// last mantissa bit, so a tie also rounds to m), i.e. when |E| <= T = s ulp(m) / 2; then the
+// code is rint(m), the even neighbour.  Otherwise RN(Q) lies on the same side of m as Q and the
+// code is m + sign(E) / 2.  E is a multiple of ulp(s) / 4 (d and m s both are), and where
+// |E| <= 2 T it has at most 7 significant bits, so RN(E) = fma(-m, s, d) is E itself; where
+// |E| > 2 T, |RN(E)| >= 2 T.  The test |RN(E)| <= T is therefore exact, as are T (a power-of-two
+// multiple of s) and the sign, for s >= 2^-100; smaller scales divide.
+constexpr float kRemainderMinScale = 0x1p-100f;
+
+// Bits of M + code for an element whose reciprocal remainder `res` lies near one half (or any
+// element, for a subnormal scale: `fast` false), by the remainder test above, or by the IEEE
+// divide for scales below 2^-100.  Out of line: it runs for about one element in a thousand
+// of unrotated bf16 data and almost never for rotated data, and the many inlined call sites
+// stay small.
+__device__ __noinline__ uint32_t code_bits_tie(float d, float k, float res, float s, bool fast)
 {
-    const uint64_t mn2 = f2_pack(mn, mn), r2 = f2_pack(r, r), m2 = f2_pack(kRoundMagic, kRoundMagic);
-    float w[8];
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
-        const uint64_t d = f2_sub(X[i], mn2);
-        const uint64_t t = f2_fma(d, r2, m2);
-        const uint64_t nk = f2_sub(m2, t);          // -k, exact
-        const uint64_t res = f2_fma(d, r2, nk);     // d r - k, one rounding
-        float a, c;
-        f2_unpack(res, a, c);
-        w[i & 7] = (i < 8) ? fmaxf(fabsf(a), fabsf(c)) : fmax3(w[i & 7], fabsf(a), fabsf(c));
-        X[i] = t;
+    float code;
+    if (fast && s >= kRemainderMinScale) {
+        const float m = __fadd_rn(k, copysignf(0.5f, res));
+        const float e = __fmaf_rn(-m, s, d);
+        const float half_ulp = __int_as_float((__float_as_int(m) & 0x7F800000) - (24 << 23));
+        code = fabsf(e) <= __fmul_rn(s, half_ulp) ? m : __fadd_rn(m, copysignf(0.5f, e));
+    } else {
+        code = fminf(fmaxf(rintf(__fdiv_rn(d, s)), 0.0f), 15.0f);
     }
-    return fmaxf(fmax3(w[0], w[1], w[2]), fmax3(fmax3(w[3], w[4], w[5]), w[6], w[7]));
+    return __float_as_uint(__fadd_rn(code, kRoundMagic));   // m + M: a tie goes to even
 }
 
-// Codes through the IEEE divide, exactly as defined (used where quantize_fast cannot decide,
-// and when the scale is subnormal).
-__device__ __forceinline__ void quantize_exact(uint64_t X[32], float mn, float scale)
+// Bits of M + code for element value y, given the reciprocal result t_bits (M + k).
+__device__ __forceinline__ uint32_t code_bits_exact(float y, uint32_t t_bits, float mn, float s,
+                                                    float r, bool fast)
 {
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
-        float lo, hi;
-        f2_unpack(X[i], lo, hi);
-        float ql = rintf(__fdiv_rn(__fsub_rn(lo, mn), scale));
-        float qh = rintf(__fdiv_rn(__fsub_rn(hi, mn), scale));
-        ql = fminf(fmaxf(ql, 0.0f), 15.0f);
-        qh = fminf(fmaxf(qh, 0.0f), 15.0f);
-        X[i] = f2_pack(__fadd_rn(ql, kRoundMagic), __fadd_rn(qh, kRoundMagic));
-    }
+    const float d = __fsub_rn(y, mn);
+    const float k = __fsub_rn(__uint_as_float(t_bits), kRoundMagic);
+    const float res = __fmaf_rn(d, r, -k);
+    if (fast && fabsf(res) < kNearHalf)
+        return t_bits;
+    return code_bits_tie(d, k, res, s, fast);
 }
 
 // Gather the low nibbles of t_0..t_7 (codes of elements r = 0..7) into one word, element r at
@@ -210,9 +218,8 @@ struct RqParams {
 // Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
 // kRotate = false is the plain INT4 quantizer (H = I) used as the unrotated baseline.
 template <bool kRotate>
-__device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, int vt, int b,
-                                               int lane, bool store, int64_t row,
-                                               const RqParams &p)
+__device__ __forceinline__ void quantize_store(const uint64_t X[32], int b, bool store,
+                                               int64_t row, const RqParams &p)
 {
     // min / max over the pair's 128 elements
     float mns[8], mxs[8];
@@ -234,45 +241,53 @@ __device__ __forceinline__ void quantize_store(uint64_t X[32], uint32_t tile, in
         scale = 0.0f;                               // canonical +0
     const float zero = __fadd_rn(mn, 0.0f);         // a zero minimum is stored as +0
 
-    bool exact = false;
-    if (degenerate) {
-        const uint64_t m2 = f2_pack(kRoundMagic, kRoundMagic);
-#pragma unroll
-        for (int i = 0; i < 32; i++)
-            X[i] = m2;                              // every code 0
-    } else if (scale < FLT_MIN) {
-        exact = true;                               // subnormal scale: IEEE divide throughout
-    } else {
-        const float worst = quantize_fast(X, mn, __frcp_rn(scale));
-        exact = !(worst < kNearHalf);
-    }
-    // The two threads of a pair decide together (the recomputation shuffles within the pair).
-    const bool pair_exact = __shfl_xor_sync(0xFFFFFFFFu, exact ? 1 : 0, 1) != 0 || exact;
-    if (pair_exact) {
-        const uint32_t pair_mask = 3u << (lane & ~1);
-        uint4 raw[8];
-        load_half_vec(tile, vt, b, raw);
-        to_pairs(raw, X);
-        if (kRotate)
-            fwht128(X, b, pair_mask);
-        quantize_exact(X, mn, scale);
-    }
+    const bool fast = !degenerate && !(scale < FLT_MIN);
+    const float r = fast ? __frcp_rn(scale) : 0.0f;
+    const uint64_t mn2 = f2_pack(mn, mn), r2 = f2_pack(r, r);
+    const uint64_t m2 = f2_pack(kRoundMagic, kRoundMagic);
 
-    if (!store)
-        return;
+    // Codes and stores, two output words at a time: words a4 and a4 + 4 take the low and high
+    // halves of the packed pairs X[8 a4 + r].  Each code comes from the reciprocal (see the
+    // note above code_bits_tie()); the 16 elements of the two words go through
+    // code_bits_exact() when one of them lies near a half-way quotient, or for a subnormal
+    // scale.
     uint8_t *dst = p.kv_pages + row * kRowBytes;
 #pragma unroll
-    for (int a = 0; a < 8; a++) {
-        uint32_t tt[8];
+    for (int a4 = 0; a4 < 4; a4++) {
+        uint32_t tlo[8], thi[8];
+        float worst = 0.0f;
 #pragma unroll
-        for (int r = 0; r < 8; r++) {
-            float lo, hi;
-            f2_unpack(X[8 * (a & 3) + r], lo, hi);
-            tt[r] = __float_as_uint(a < 4 ? lo : hi);
+        for (int rr = 0; rr < 8; rr++) {
+            const uint64_t d = f2_sub(X[8 * a4 + rr], mn2);
+            const uint64_t t = f2_fma(d, r2, m2);
+            const uint64_t nk = f2_sub(m2, t);          // -k, exact
+            const uint64_t res = f2_fma(d, r2, nk);     // d r - k, one rounding
+            float tl, th, el, eh;
+            f2_unpack(t, tl, th);
+            f2_unpack(res, el, eh);
+            worst = fmax3(worst, fabsf(el), fabsf(eh));
+            tlo[rr] = __float_as_uint(tl);
+            thi[rr] = __float_as_uint(th);
         }
-        *reinterpret_cast<uint32_t *>(dst + 8 * a + 4 * b) = pack8(tt);
+        if (degenerate) {
+#pragma unroll
+            for (int rr = 0; rr < 8; rr++)
+                tlo[rr] = thi[rr] = __float_as_uint(kRoundMagic);   // every code 0
+        } else if (!fast || !(worst < kNearHalf)) {
+#pragma unroll
+            for (int rr = 0; rr < 8; rr++) {
+                float lo, hi;
+                f2_unpack(X[8 * a4 + rr], lo, hi);
+                tlo[rr] = code_bits_exact(lo, tlo[rr], mn, scale, r, fast);
+                thi[rr] = code_bits_exact(hi, thi[rr], mn, scale, r, fast);
+            }
+        }
+        if (store) {
+            *reinterpret_cast<uint32_t *>(dst + 8 * a4 + 4 * b) = pack8(tlo);
+            *reinterpret_cast<uint32_t *>(dst + 8 * (a4 + 4) + 4 * b) = pack8(thi);
+        }
     }
-    if (b == 0) {
+    if (store && b == 0) {
         const __half2 sz = __halves2half2(__float2half_rn(scale), __float2half_rn(zero));
         p.scales[row] = half2_as_u32(sz);
     }
@@ -376,7 +391,7 @@ __global__ void __launch_bounds__(kRqThreads, 4)
         to_pairs(raw, X);
         if (kRotate)
             fwht128(X, b, 0xFFFFFFFFu);
-        quantize_store<kRotate>(X, tile_smem, vt, b, lane, store, row, p);
+        quantize_store<kRotate>(X, b, store, row, p);
         __syncwarp();
     }
     if (i < n) {
