@@ -9,8 +9,8 @@ import torch
 
 import oracle
 from bit_paged_kv_block_b200 import synth
-from helpers import (NTHREADS, assert_attention_close, canary_device_cache, device_cache_from,
-                     oracle_cache, subset, u16)
+from helpers import (EDGE_KINDS, NTHREADS, assert_attention_close, canary_device_cache,
+                     device_cache_from, edge_kv, oracle_cache, subset, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -30,14 +30,14 @@ def test_plain_quantize_bit_exact(cuda_device, name):
     assert np.array_equal(u16(sc), scales)
 
 
-def test_plain_quantize_small_integer_ties(cuda_device):
-    """Unrotated small integers hit exact half-way quotients all the time."""
+@pytest.mark.parametrize("kind", EDGE_KINDS)
+def test_plain_quantize_edge_values(cuda_device, kind):
+    """Unrotated bf16 values land on exact half-way quotients all the time; these inputs add
+    degenerate vectors, subnormal scales and scales around 2^-100."""
     from bit_paged_kv_block_b200 import saw
     T, hkv = 137, 3
-    g = torch.Generator().manual_seed(3)
-    k = torch.randint(-7, 8, (T, hkv, 128), generator=g).to(torch.bfloat16)
-    v = torch.randint(0, 4, (T, hkv, 128), generator=g).to(torch.bfloat16)
-    wl = synth.custom("ints", [T], num_q_heads=hkv, num_kv_heads=hkv, new_tokens=[T])
+    k, v = edge_kv(kind, T, hkv)
+    wl = synth.custom(kind, [T], num_q_heads=hkv, num_kv_heads=hkv, new_tokens=[T])
     seq, pos = synth.token_index(wl)
     kv, sc = canary_device_cache(wl, cuda_device)
     saw.saw_quantize_paged_plain(k.to(cuda_device), v.to(cuda_device),

@@ -7,7 +7,8 @@ import torch
 
 import oracle
 from bit_paged_kv_block_b200 import synth
-from helpers import CANARY_CODE, CANARY_SCALE, NTHREADS, canary_device_cache, oracle_cache, u16
+from helpers import (CANARY_CODE, CANARY_SCALE, EDGE_KINDS, NTHREADS, canary_device_cache,
+                     edge_kv, oracle_cache, u16)
 
 pytestmark = pytest.mark.gpu
 
@@ -54,34 +55,13 @@ def _custom_tokens(T, Hkv, maker, seed=0):
     return maker(g, (T, Hkv, 128)).to(torch.bfloat16)
 
 
-@pytest.mark.parametrize("kind", ["small_ints", "zeros_and_constants", "tiny_magnitudes",
-                                  "huge_range", "signed_zero", "single_spike"])
+@pytest.mark.parametrize("kind", EDGE_KINDS)
 def test_rotate_quantize_edge_values(cuda_device, kind):
-    """Inputs chosen to hit exact ties, degenerate vectors, subnormal scales and the
-    reciprocal-path fallback; every code must still equal the IEEE-divide definition."""
+    """Inputs chosen to hit exact ties, degenerate vectors, subnormal scales and both sides of
+    the smallest scale the remainder test handles; every code must still equal the
+    IEEE-divide definition."""
     T, Hkv = 203, 3                  # ragged: 609 vectors, not a multiple of 16 per warp
-    g = torch.Generator().manual_seed(7)
-    if kind == "small_ints":         # rotated values are multiples of c: many exact halves
-        x = torch.randint(-3, 4, (T, Hkv, 128), generator=g).float()
-    elif kind == "zeros_and_constants":
-        x = torch.zeros(T, Hkv, 128)
-        x[1::3] = torch.randn(T, Hkv, 1, generator=g)[1::3]        # constants
-        x[2::5, :, 7] = 1.0                                          # unit vectors
-    elif kind == "tiny_magnitudes":  # fp32 scales near / below the normal range
-        x = torch.randn(T, Hkv, 128, generator=g) * 1e-37
-        x[::2] *= 1e-2
-    elif kind == "huge_range":
-        x = torch.randn(T, Hkv, 128, generator=g) * (10.0 ** torch.randint(-3, 4, (T, Hkv, 1), generator=g))
-    elif kind == "signed_zero":
-        x = torch.zeros(T, Hkv, 128)
-        x[::2, :, 3] = -0.0
-        x[1::2, :, 5] = 1.0
-        x[::4] = -x[::4]
-    else:
-        x = torch.zeros(T, Hkv, 128)
-        x[torch.arange(T), :, torch.arange(T) % 128] = 50.0
-    k = x.to(torch.bfloat16)
-    v = (x.flip(-1) * 0.5).to(torch.bfloat16)
+    k, v = edge_kv(kind, T, Hkv)
     wl = synth.custom(kind, [T], num_q_heads=Hkv, num_kv_heads=Hkv, new_tokens=[T],
                       num_pages=(T + 15) // 16 + 3)
     kv, sc = gpu_append(wl, cuda_device, k=k, v=v)
