@@ -77,6 +77,11 @@ def _load():
         lib.oracle_decode_fp64.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
                                            i32, P, i32]
         lib.oracle_decode_fp64.restype = None
+        lib.oracle_append_bf16.argtypes = [P, P, P, i64, i32, i32, i32, i64, P]
+        lib.oracle_append_bf16.restype = i64
+        lib.oracle_decode_bf16_fp64.argtypes = [P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
+                                                P, i32]
+        lib.oracle_decode_bf16_fp64.restype = None
         _lib = lib
         return lib
 
@@ -210,6 +215,45 @@ def decode_fp64(q_bits, kv_pages, scales, block_table, seq_lens, *, sm_scale=Non
     _load().oracle_decode_fp64(_ptr(q_bits), _ptr(kv_pages), _ptr(scales), _ptr(block_table),
                                block_table.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, page_size,
                                float(sm_scale), 1 if rotate else 0, _ptr(out), int(nthreads))
+    return out
+
+
+def empty_cache_bf16(num_pages: int, Hkv: int, D: int = 128, page_size: int = 16) -> np.ndarray:
+    """Zero-filled bf16 cache (uint16 bits) [num_pages][Hkv][2][page_size][D]."""
+    return np.zeros((num_pages, Hkv, 2, page_size, D), dtype=np.uint16)
+
+
+def append_bf16(k_bits, v_bits, slot_mapping, kv_bf16) -> int:
+    """Scatter bf16 K, V [T][Hkv][D] into the bf16 pages in place (the uncompressed baseline
+    cache).  Negative slots are skipped; slots past the cache are skipped and counted."""
+    k_bits = _as(k_bits, np.uint16)
+    v_bits = _as(v_bits, np.uint16)
+    slot_mapping = _as(slot_mapping, np.int64)
+    T, Hkv, D = k_bits.shape
+    num_pages, hkv2, _, page_size, d2 = kv_bf16.shape
+    assert hkv2 == Hkv and d2 == D and kv_bf16.dtype == np.uint16 and kv_bf16.flags.c_contiguous
+    return int(_load().oracle_append_bf16(_ptr(k_bits), _ptr(v_bits), _ptr(slot_mapping), T, Hkv,
+                                          D, page_size, num_pages, _ptr(kv_bf16)))
+
+
+def decode_bf16_fp64(q_bits, kv_bf16, block_table, seq_lens, *, sm_scale=None,
+                     nthreads=1) -> np.ndarray:
+    """fp64 decode attention over the bf16 paged cache (no rotation, no quantization).
+    Returns fp64 [S][Hq][D]."""
+    q_bits = _as(q_bits, np.uint16)
+    kv_bf16 = _as(kv_bf16, np.uint16)
+    block_table = _as(block_table, np.int32)
+    seq_lens = _as(seq_lens, np.int32)
+    S, Hq, D = q_bits.shape
+    num_pages, Hkv, _, page_size, d2 = kv_bf16.shape
+    assert d2 == D and Hq % Hkv == 0
+    assert block_table.ndim == 2 and block_table.shape[0] == S and seq_lens.shape == (S,)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    _load().oracle_decode_bf16_fp64(_ptr(q_bits), _ptr(kv_bf16), _ptr(block_table),
+                                    block_table.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, page_size,
+                                    float(sm_scale), _ptr(out), int(nthreads))
     return out
 
 

@@ -298,3 +298,92 @@ void oracle_decode_fp64(const uint16_t *q, const uint8_t *kv_pages, const uint16
         }
     }
 }
+
+/* ---- the BF16 paged-cache baseline ----------------------------------------------------- */
+/*
+ * The uncompressed cache the INT4 format is measured against ("SAW-INT4", Research Findings:
+ * its serving throughput gain is relative to a 16-bit KV cache; "BitDecoding-FP4", abstract:
+ * the speedup over BF16 KV decoding).  Layout (reading: the INT4 layout with 16-bit elements):
+ * kv_bf16 uint16 [num_pages][Hkv][2 (K,V)][page_size][D]; no scale, no rotation.
+ */
+
+/* Scatter T tokens of bf16 K and V into the bf16 pages.  A negative slot is skipped; a slot
+ * beyond the cache is skipped and counted.  Returns the count. */
+int64_t oracle_append_bf16(const uint16_t *k, const uint16_t *v, const int64_t *slot_mapping,
+                           int64_t T, int Hkv, int D, int page_size, int64_t num_pages,
+                           uint16_t *kv_bf16)
+{
+    int64_t bad = 0;
+    for (int64_t t = 0; t < T; t++) {
+        const int64_t slot = slot_mapping[t];
+        if (slot < 0)
+            continue;
+        if (slot >= num_pages * page_size) {
+            bad++;
+            continue;
+        }
+        const int64_t page = slot / page_size, off = slot % page_size;
+        for (int h = 0; h < Hkv; h++)
+            for (int sel = 0; sel < 2; sel++) {
+                const uint16_t *src = (sel ? v : k) + ((size_t)t * Hkv + h) * D;
+                uint16_t *dst = kv_bf16 + ((((size_t)page * Hkv + h) * 2 + sel) * page_size + off) * D;
+                for (int d = 0; d < D; d++)
+                    dst[d] = src[d];
+            }
+    }
+    return bad;
+}
+
+/* fp64 decode attention over the bf16 cache: s_t = sm_scale <q, k_t>, softmax over the
+ * seq_len valid tokens, out = sum_t p_t v_t; query head hq reads kv head hq / (Hq / Hkv). */
+void oracle_decode_bf16_fp64(const uint16_t *q, const uint16_t *kv_bf16,
+                             const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                             int S, int Hq, int Hkv, int D, int page_size, double sm_scale,
+                             double *out, int nthreads)
+{
+    const int G = Hq / Hkv;
+#pragma omp parallel for collapse(2) schedule(dynamic) num_threads(nthreads)
+    for (int s = 0; s < S; s++) {
+        for (int hq = 0; hq < Hq; hq++) {
+            const int h = hq / G;
+            const int L = seq_lens[s];
+            double qd[1024], o[1024];
+            double *dst = out + ((size_t)s * Hq + hq) * D;
+            if (L <= 0) {
+                for (int d = 0; d < D; d++)
+                    dst[d] = 0.0;
+                continue;
+            }
+            for (int d = 0; d < D; d++)
+                qd[d] = (double)oracle_bf16_to_f32(q[((size_t)s * Hq + hq) * D + d]);
+            double m = -INFINITY;
+            for (int t = 0; t < L; t++) {
+                const int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                const uint16_t *kr = kv_bf16 + ((((size_t)page * Hkv + h) * 2 + 0) * page_size + t % page_size) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qd[d] * (double)oracle_bf16_to_f32(kr[d]);
+                if (sm_scale * acc > m)
+                    m = sm_scale * acc;
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; d++)
+                o[d] = 0.0;
+            for (int t = 0; t < L; t++) {
+                const int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                const size_t base = (((size_t)page * Hkv + h) * 2) * page_size + t % page_size;
+                const uint16_t *kr = kv_bf16 + base * D;
+                const uint16_t *vr = kv_bf16 + (base + page_size) * D;
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qd[d] * (double)oracle_bf16_to_f32(kr[d]);
+                const double p = exp(sm_scale * acc - m);
+                l += p;
+                for (int d = 0; d < D; d++)
+                    o[d] += p * (double)oracle_bf16_to_f32(vr[d]);
+            }
+            for (int d = 0; d < D; d++)
+                dst[d] = o[d] / l;
+        }
+    }
+}

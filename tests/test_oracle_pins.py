@@ -503,3 +503,83 @@ def test_rotation_lowers_quantized_attention_error():
         errs[rotate] = (np.mean(o_err), np.mean(l_err))
     assert errs[True][0] < errs[False][0]
     assert errs[True][1] < errs[False][1]
+
+
+# ---- the BF16 paged-cache baseline (uncompressed; no rotation, no quantization) ---------------
+
+def _bf16_cache(wl):
+    """Oracle bf16 cache of every token of the workload, and the bf16 bits of K and V."""
+    k, v = synth.kv_values(wl, "K"), synth.kv_values(wl, "V")
+    seq, pos = synth.token_index(wl)
+    kv = oracle.empty_cache_bf16(wl.num_pages, wl.num_kv_heads)
+    assert oracle.append_bf16(synth.bf16_bits(k), synth.bf16_bits(v),
+                              synth.slot_mapping(wl, seq, pos), kv) == 0
+    return kv, synth.bf16_bits(k), synth.bf16_bits(v)
+
+
+def test_bf16_append_scatter_and_skips():
+    """Every row lands at page = slot / 16, offset slot % 16, (kv head, K|V) untouched otherwise;
+    negative slots are skipped, slots past the cache are skipped and counted."""
+    rng = np.random.default_rng(11)
+    T, Hkv, P = 40, 3, 4
+    k = rng.integers(0, 1 << 16, (T, Hkv, 128), dtype=np.uint16)
+    v = rng.integers(0, 1 << 16, (T, Hkv, 128), dtype=np.uint16)
+    slots = rng.permutation(P * 16)[:T].astype(np.int64)
+    slots[3] = -1
+    slots[7] = P * 16 + 5
+    kv = np.full((P, Hkv, 2, 16, 128), 0xABCD, dtype=np.uint16)
+    assert oracle.append_bf16(k, v, slots, kv) == 1
+    written = np.zeros((P, 16), dtype=bool)
+    for t, slot in enumerate(slots):
+        if 0 <= slot < P * 16:
+            page, off = divmod(int(slot), 16)
+            written[page, off] = True
+            assert np.array_equal(kv[page, :, 0, off], k[t]) and np.array_equal(kv[page, :, 1, off], v[t])
+    assert np.all(kv.transpose(0, 3, 1, 2, 4)[~written] == 0xABCD)
+
+
+def test_bf16_decode_matches_torch_sdpa_fp64():
+    wl = synth.custom("bf16sdpa", [1, 16, 17, 40], num_q_heads=4, num_kv_heads=4, seed=5)
+    kv, kb, vb = _bf16_cache(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    got = oracle.decode_bf16_fp64(qb, kv, wl.block_table, wl.seq_lens)
+    q = torch.from_numpy(qb.astype(np.uint32) << 16).view(torch.float32).double()
+    k = torch.from_numpy(kb.astype(np.uint32) << 16).view(torch.float32).double()
+    v = torch.from_numpy(vb.astype(np.uint32) << 16).view(torch.float32).double()
+    start = 0
+    for s, L in enumerate(wl.seq_lens.tolist()):
+        for hq in range(wl.num_q_heads):
+            ref = torch.nn.functional.scaled_dot_product_attention(
+                q[s, hq][None, None, None], k[start:start + L, hq][None, None],
+                v[start:start + L, hq][None, None])[0, 0, 0]
+            assert np.allclose(got[s, hq], ref.numpy(), atol=1e-12, rtol=1e-12)
+        start += L
+
+
+def test_bf16_decode_single_token_gqa_and_empty():
+    """seq_len 1 gives that token's value exactly; query head hq reads kv head hq / G; an empty
+    sequence gives zeros."""
+    wl = synth.custom("bf16g", [1, 0, 33], num_q_heads=8, num_kv_heads=2, seed=6)
+    kv, kb, vb = _bf16_cache(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_bf16_fp64(qb, kv, wl.block_table, wl.seq_lens)
+    vf = (vb.astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+    for hq in range(8):
+        assert np.array_equal(out[0, hq], vf[0, hq // 4])
+    assert np.all(out[1] == 0.0)
+    for hq in range(8):   # the same output as a single-head cache holding only kv head hq / G
+        sub = kv[:, hq // 4: hq // 4 + 1].copy()
+        one = oracle.decode_bf16_fp64(qb[2:3, hq:hq + 1], sub, wl.block_table[2:3], wl.seq_lens[2:3])
+        assert np.array_equal(one[0, 0], out[2, hq])
+
+
+def test_bf16_decode_page_permutation_invariance():
+    wl = synth.custom("bf16perm", [70], num_q_heads=2, num_kv_heads=2, seed=8)
+    kv, _, _ = _bf16_cache(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    base = oracle.decode_bf16_fp64(qb, kv, wl.block_table, wl.seq_lens)
+    perm = np.random.default_rng(3).permutation(wl.num_pages)
+    kv2 = np.empty_like(kv)
+    kv2[perm] = kv
+    table2 = np.where(wl.block_table >= 0, perm[np.maximum(wl.block_table, 0)], -1).astype(np.int32)
+    assert np.array_equal(oracle.decode_bf16_fp64(qb, kv2, table2, wl.seq_lens), base)
