@@ -77,8 +77,8 @@ __device__ __forceinline__ int find_seq(const int32_t *pre, int S, int64_t pos, 
 
 // Pages per sequence (0 for an invalid length, which is flagged) and their exclusive prefix
 // pre[0..S] in shared memory; every thread of the block takes part.
-__device__ void scan_pages(const DecodeParams &p, int32_t *pre, volatile int32_t *flags,
-                           bool report)
+__device__ inline void scan_pages(const DecodeParams &p, int32_t *pre, volatile int32_t *flags,
+                                  bool report)
 {
     const int S = p.num_seqs, nthreads = blockDim.x, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
@@ -205,6 +205,45 @@ __device__ __forceinline__ void state_reset(WarpState &st)
         st.l[e] = 0.0f;
         st.z[e] = 0.0f;
     }
+}
+
+// Online softmax over one page: s holds the logits (log2 domain) of tokens g, g + 8 for heads
+// 2t, 2t + 1 (-inf for masked tokens); returns p = 2^(s - m) with m the running max after the
+// page, and rescales o, l and z when m grows.  The running max only changes when some logit of
+// the page exceeds it, so the cross-lane reduction runs only then (rare once a piece is a few
+// pages long); the result equals reducing every page.
+__device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, float pr[4])
+{
+    const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
+    if (__any_sync(0xFFFFFFFFu, grow)) {
+        float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 8));
+            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 16));
+        }
+        float alpha[2];
+#pragma unroll
+        for (int e = 0; e < 2; e++) {
+            const float mn = fmaxf(st.m[e], mx[e]);
+            alpha[e] = ex2_approx(st.m[e] - mn);
+            st.m[e] = mn;
+            st.l[e] *= alpha[e];
+            st.z[e] *= alpha[e];
+        }
+#pragma unroll
+        for (int i = 0; i < 8; i++) {
+            st.o[i][0] *= alpha[0];
+            st.o[i][1] *= alpha[1];
+            st.o[i][2] *= alpha[0];
+            st.o[i][3] *= alpha[1];
+        }
+    }
+    pr[0] = ex2_approx(s[0] - st.m[0]);
+    pr[1] = ex2_approx(s[1] - st.m[1]);
+    pr[2] = ex2_approx(s[2] - st.m[0]);
+    pr[3] = ex2_approx(s[3] - st.m[1]);
 }
 
 // Fold (m, l, o) partial b (scaled by its own max) into the running partial a.

@@ -185,39 +185,8 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
             s[2] = s[3] = -INFINITY;
     }
 
-    // The running max only changes when some logit of the page exceeds it, so the cross-lane
-    // reduction is needed only then (rare once a piece is a few pages long).
-    const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
-    if (__any_sync(0xFFFFFFFFu, grow)) {
-        float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
-#pragma unroll
-        for (int e = 0; e < 2; e++) {
-            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
-            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 8));
-            mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 16));
-        }
-        float alpha[2];
-#pragma unroll
-        for (int e = 0; e < 2; e++) {
-            const float mn = fmaxf(st.m[e], mx[e]);
-            alpha[e] = ex2_approx(st.m[e] - mn);
-            st.m[e] = mn;
-            st.l[e] *= alpha[e];
-            st.z[e] *= alpha[e];
-        }
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            st.o[i][0] *= alpha[0];
-            st.o[i][1] *= alpha[1];
-            st.o[i][2] *= alpha[0];
-            st.o[i][3] *= alpha[1];
-        }
-    }
     float pr[4];
-    pr[0] = ex2_approx(s[0] - st.m[0]);
-    pr[1] = ex2_approx(s[1] - st.m[1]);
-    pr[2] = ex2_approx(s[2] - st.m[0]);
-    pr[3] = ex2_approx(s[3] - st.m[1]);
+    softmax_update(s, st, pr);
 
     // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
     float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));

@@ -24,18 +24,19 @@ int check_cache(const saw_cache_desc *c)
     return SAW_OK;
 }
 
+// bf16: the uncompressed baseline cache (no scales)
 int check_append(const saw_cache_desc *cache, const void *k, const void *v,
                  const int64_t *slot_mapping, int64_t num_tokens, const uint8_t *kv_pages,
-                 const void *scales)
+                 const void *scales, bool bf16 = false)
 {
     if (num_tokens < 0)
         return SAW_ERR_INVALID_ARGUMENT;
     if (num_tokens == 0)
         return SAW_OK;
-    if (!k || !v || !slot_mapping || !kv_pages || !scales)
+    if (!k || !v || !slot_mapping || !kv_pages || (!bf16 && !scales))
         return SAW_ERR_INVALID_ARGUMENT;
-    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(kv_pages, 16) || !aligned(scales, 16) ||
-        !aligned(slot_mapping, 8))
+    if (!aligned(k, 16) || !aligned(v, 16) || !aligned(kv_pages, 16) ||
+        (!bf16 && !aligned(scales, 16)) || !aligned(slot_mapping, 8))
         return SAW_ERR_INVALID_ARGUMENT;
     if (num_tokens > INT64_MAX / (int64_t(cache->num_kv_heads) * 256))
         return SAW_ERR_INVALID_ARGUMENT;
@@ -45,7 +46,8 @@ int check_append(const saw_cache_desc *cache, const void *k, const void *v,
 int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
                  const uint8_t *kv_pages, const void *scales, const int32_t *block_table,
                  int32_t max_blocks, const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
-                 const float *out, const void *workspace, size_t workspace_bytes)
+                 const float *out, const void *workspace, size_t workspace_bytes,
+                 bool bf16 = false)
 {
     if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
         return SAW_ERR_INVALID_ARGUMENT;
@@ -55,16 +57,17 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
         return SAW_ERR_INVALID_ARGUMENT;
     if (num_seqs == 0)
         return SAW_OK;
-    if (!q || !kv_pages || !scales || !block_table || !seq_lens || !out || max_blocks <= 0)
+    if (!q || !kv_pages || (!bf16 && !scales) || !block_table || !seq_lens || !out || max_blocks <= 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if (!aligned(q, 16) || !aligned(kv_pages, 16) || !aligned(scales, 16) || !aligned(out, 16) ||
+    if (!aligned(q, 16) || !aligned(kv_pages, 16) || (!bf16 && !aligned(scales, 16)) || !aligned(out, 16) ||
         !aligned(block_table, 4) || !aligned(seq_lens, 4))
         return SAW_ERR_INVALID_ARGUMENT;
     if (cache->num_pages == 0)
         return SAW_ERR_INVALID_ARGUMENT;
     if (int64_t(max_blocks) * 16 > INT32_MAX)
         return SAW_ERR_INVALID_ARGUMENT;
-    const size_t need = saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+    const size_t need = bf16 ? saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs)
+                             : saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
     if (need == 0)
         return SAW_ERR_CUDA;
     if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
@@ -312,6 +315,126 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
     return step_impl(cache, num_q_heads, q, k_new, v_new, slot_mapping, num_new_tokens,
                      kv_pages, scales, block_table, max_blocks_per_seq, seq_lens, num_seqs,
                      sm_scale, out, workspace, workspace_bytes, dev_status, stream, false);
+}
+
+// ---- the uncompressed BF16 paged cache (baseline) -------------------------------------------
+
+static int check_bf16_cache(const saw_cache_desc *cache)
+{
+    const int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    // tensor-map rows (page * Hkv + h) * 64 must stay below 2^31
+    if (cache->num_pages > (int64_t(1) << 31) / (int64_t(cache->num_kv_heads) * 64))
+        return SAW_ERR_UNSUPPORTED;
+    return SAW_OK;
+}
+
+static int append_bf16_impl(const saw_cache_desc *cache, const void *k, const void *v,
+                            const int64_t *slot_mapping, int64_t num_tokens, void *kv_bf16,
+                            uint32_t *dev_status, cudaStream_t stream)
+{
+    saw::AppendBf16Args a;
+    a.k = k;
+    a.v = v;
+    a.slot_mapping = slot_mapping;
+    a.num_tokens = num_tokens;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.num_pages = cache->num_pages;
+    a.kv = kv_bf16;
+    a.status = dev_status;
+    return saw::launch_append_bf16(a, stream) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+}
+
+int saw_append_bf16_paged(const saw_cache_desc *cache, const void *k, const void *v,
+                          const int64_t *slot_mapping, int64_t num_tokens, void *kv_bf16,
+                          uint32_t *dev_status, void *stream)
+{
+    int rc = check_bf16_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k, v, slot_mapping, num_tokens,
+                      static_cast<const uint8_t *>(kv_bf16), nullptr, true);
+    if (rc != SAW_OK || num_tokens == 0)
+        return rc;
+    return append_bf16_impl(cache, k, v, slot_mapping, num_tokens, kv_bf16, dev_status,
+                            static_cast<cudaStream_t>(stream));
+}
+
+size_t saw_paged_decode_bf16_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                             int32_t num_seqs)
+{
+    if (check_bf16_cache(cache) != SAW_OK)
+        return 0;
+    return saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+}
+
+static int decode_bf16_impl(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                            const void *kv_bf16, const int32_t *block_table,
+                            int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                            int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                            size_t workspace_bytes, uint32_t *dev_status, cudaStream_t stream,
+                            bool programmatic)
+{
+    saw::DecodeArgs a = decode_args(cache, num_q_heads, q, static_cast<const uint8_t *>(kv_bf16),
+                                    nullptr, block_table, max_blocks_per_seq, seq_lens, num_seqs,
+                                    sm_scale, out, workspace, workspace_bytes, dev_status);
+    a.rotate = false;
+    return saw::launch_paged_decode_bf16(a, stream, programmatic) == cudaSuccess ? SAW_OK
+                                                                                 : SAW_ERR_CUDA;
+}
+
+int saw_paged_decode_attn_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                               const void *kv_bf16, const int32_t *block_table,
+                               int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                               int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                               size_t workspace_bytes, uint32_t *dev_status, void *stream)
+{
+    int rc = check_bf16_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, static_cast<const uint8_t *>(kv_bf16), nullptr,
+                      block_table, max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out,
+                      workspace, workspace_bytes, true);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    return decode_bf16_impl(cache, num_q_heads, q, kv_bf16, block_table, max_blocks_per_seq,
+                            seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes,
+                            dev_status, static_cast<cudaStream_t>(stream), false);
+}
+
+int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                         const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                         int64_t num_new_tokens, void *kv_bf16, const int32_t *block_table,
+                         int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                         float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                         uint32_t *dev_status, void *stream)
+{
+    int rc = check_bf16_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_append(cache, k_new, v_new, slot_mapping, num_new_tokens,
+                      static_cast<const uint8_t *>(kv_bf16), nullptr, true);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode(cache, num_q_heads, q, static_cast<const uint8_t *>(kv_bf16), nullptr,
+                      block_table, max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out,
+                      workspace, workspace_bytes, true);
+    if (rc != SAW_OK)
+        return rc;
+    const cudaStream_t s = static_cast<cudaStream_t>(stream);
+    const bool appended = num_new_tokens > 0;
+    if (appended) {
+        rc = append_bf16_impl(cache, k_new, v_new, slot_mapping, num_new_tokens, kv_bf16,
+                              dev_status, s);
+        if (rc != SAW_OK)
+            return rc;
+    }
+    if (num_seqs == 0)
+        return SAW_OK;
+    return decode_bf16_impl(cache, num_q_heads, q, kv_bf16, block_table, max_blocks_per_seq,
+                            seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes,
+                            dev_status, s, appended);
 }
 
 }  // extern "C"

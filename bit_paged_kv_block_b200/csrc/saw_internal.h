@@ -55,6 +55,17 @@ struct DecodeArgs {
     bool rotate = true;          // false: plain INT4 cache (no query / output rotation)
 };
 
+struct AppendBf16Args {
+    const void *k;               // bf16 [T][Hkv][128]
+    const void *v;               // bf16 [T][Hkv][128]
+    const int64_t *slot_mapping; // [T]
+    int64_t num_tokens;
+    int32_t num_kv_heads;
+    int64_t num_pages;
+    void *kv;                    // bf16 [num_pages][Hkv][2][16][128]
+    uint32_t *status;            // nullable
+};
+
 // Queue the rotate+quantize+scatter kernel.  `trigger_dependents` makes the kernel release
 // a programmatic dependent launch early.  Returns a cudaError_t.
 cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t stream,
@@ -66,5 +77,11 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
 // Queue the decode kernel; `programmatic` launches it as a programmatic dependent of the
 // previous kernel on the stream.  Returns a cudaError_t.
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
+
+// The uncompressed BF16 paged cache (baseline): scatter, decode workspace size, decode
+// (DecodeArgs::kv_pages is the bf16 cache; scales and rotate are unused).
+cudaError_t launch_append_bf16(const AppendBf16Args &a, cudaStream_t stream);
+size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs);
+cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
 
 }  // namespace saw

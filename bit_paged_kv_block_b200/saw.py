@@ -75,6 +75,15 @@ def _open_library() -> ctypes.CDLL:
     lib.saw_paged_decode_attn_plain.restype = ctypes.c_int
     lib.saw_decode_step_plain.argtypes = lib.saw_decode_step.argtypes
     lib.saw_decode_step_plain.restype = ctypes.c_int
+    lib.saw_append_bf16_paged.argtypes = [D, P, P, P, i64, P, P, P]
+    lib.saw_append_bf16_paged.restype = ctypes.c_int
+    lib.saw_paged_decode_bf16_workspace_bytes.argtypes = [D, i32, i32]
+    lib.saw_paged_decode_bf16_workspace_bytes.restype = sz
+    lib.saw_paged_decode_attn_bf16.argtypes = [D, i32, P, P, P, i32, P, i32, f32, P, P, sz, P, P]
+    lib.saw_paged_decode_attn_bf16.restype = ctypes.c_int
+    lib.saw_decode_step_bf16.argtypes = [D, i32, P, P, P, P, i64, P, P, i32, P, i32, f32, P, P,
+                                         sz, P, P]
+    lib.saw_decode_step_bf16.restype = ctypes.c_int
     return lib
 
 
@@ -301,3 +310,109 @@ def saw_paged_decode_attn_static(q, kv_pages, scales, block_table, seq_lens, out
                                           _ptr(seq_lens), S, float(sm_scale), _ptr(out),
                                           _ptr(dev_status), _stream(stream))
     _check(rc, "saw_paged_decode_attn_static")
+
+
+# ---- the uncompressed BF16 paged cache (baseline) --------------------------------------------
+
+def cache_desc_bf16(kv_bf16: torch.Tensor) -> saw_cache_desc:
+    """Descriptor of a bf16 cache tensor [num_pages][Hkv][2][16][128]."""
+    _need(kv_bf16, "kv_bf16", torch.bfloat16, 5, cuda=False)
+    num_pages, hkv, two, page, d = kv_bf16.shape
+    if two != 2 or d != HEAD_DIM:
+        raise ValueError(f"kv_bf16 must be [num_pages][Hkv][2][16][128], got {tuple(kv_bf16.shape)}")
+    return saw_cache_desc(int(hkv), HEAD_DIM, int(page), int(num_pages))
+
+
+def allocate_cache_bf16(num_pages: int, num_kv_heads: int, device="cuda") -> torch.Tensor:
+    """Empty bf16 cache [P][Hkv][2][16][128]."""
+    return torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, HEAD_DIM), dtype=torch.bfloat16,
+                       device=device)
+
+
+def saw_append_bf16_paged(k, v, slot_mapping, kv_bf16, dev_status=None, stream=None) -> None:
+    """Scatter new tokens k, v (bf16 [T][Hkv][128]) into the bf16 cache."""
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    desc = cache_desc_bf16(kv_bf16)
+    _need(kv_bf16, "kv_bf16", torch.bfloat16, 5)
+    T = k.shape[0]
+    if tuple(k.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
+        raise ValueError("k and v must be [T][Hkv][128] matching the cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have one entry per token")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    rc = lib.saw_append_bf16_paged(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(slot_mapping), T,
+                                   _ptr(kv_bf16), _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_append_bf16_paged")
+
+
+def saw_paged_decode_bf16_workspace_bytes(num_kv_heads: int, num_q_heads: int,
+                                          num_seqs: int) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, 1)
+    return int(lib.saw_paged_decode_bf16_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
+                                                         int(num_seqs)))
+
+
+def allocate_workspace_bf16(num_kv_heads: int, num_q_heads: int, num_seqs: int,
+                            device="cuda") -> torch.Tensor:
+    n = saw_paged_decode_bf16_workspace_bytes(num_kv_heads, num_q_heads, num_seqs)
+    if n == 0:
+        raise SawError(SAW_ERR_CUDA, "saw_paged_decode_bf16_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _decode_checks_bf16(q, kv_bf16, block_table, seq_lens, out, workspace, dev_status):
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kv_bf16, "kv_bf16", torch.bfloat16, 5)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(out, "out", torch.float32, 3)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    desc = cache_desc_bf16(kv_bf16)
+    S, hq, d = q.shape
+    if d != HEAD_DIM or tuple(out.shape) != (S, hq, HEAD_DIM):
+        raise ValueError("q and out must be [S][Hq][128]")
+    if block_table.shape[0] != S or seq_lens.shape[0] != S:
+        raise ValueError("block_table and seq_lens need one row per sequence")
+    return desc, S, hq
+
+
+def saw_paged_decode_attn_bf16(q, kv_bf16, block_table, seq_lens, out, workspace, sm_scale=None,
+                               dev_status=None, stream=None) -> None:
+    """Decode attention of q (bf16 [S][Hq][128]) over the bf16 paged cache into out (fp32)."""
+    desc, S, hq = _decode_checks_bf16(q, kv_bf16, block_table, seq_lens, out, workspace,
+                                      dev_status)
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_paged_decode_attn_bf16(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_bf16),
+                                        _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
+                                        S, float(sm_scale), _ptr(out), _ptr(workspace),
+                                        workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_paged_decode_attn_bf16")
+
+
+def saw_decode_step_bf16(q, k_new, v_new, slot_mapping, kv_bf16, block_table, seq_lens, out,
+                         workspace, sm_scale=None, dev_status=None, stream=None) -> None:
+    """The serving step on the bf16 cache: append k_new / v_new, then decode q."""
+    desc, S, hq = _decode_checks_bf16(q, kv_bf16, block_table, seq_lens, out, workspace,
+                                      dev_status)
+    _need(k_new, "k_new", torch.bfloat16, 3)
+    _need(v_new, "v_new", torch.bfloat16, 3)
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    T = k_new.shape[0]
+    if tuple(k_new.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [T][Hkv][128] matching the cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have one entry per new token")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_decode_step_bf16(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new),
+                                  _ptr(slot_mapping), T, _ptr(kv_bf16), _ptr(block_table),
+                                  block_table.shape[1], _ptr(seq_lens), S, float(sm_scale),
+                                  _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
+                                  _stream(stream))
+    _check(rc, "saw_decode_step_bf16")

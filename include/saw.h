@@ -161,6 +161,37 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
                           void *workspace, size_t workspace_bytes, uint32_t *dev_status,
                           void *stream);
 
+/* The uncompressed BF16 paged KV cache: the baseline the INT4 format is measured against
+ * ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving", Research
+ * Findings: serving throughput against a 16-bit KV cache; "BitDecoding-FP4: Native FP4 KV
+ * Cache Decoding via Algorithm-System Co-Design", abstract: speedup over BF16 KV decoding).
+ * Same page geometry without quantization, scales or rotation:
+ *     kv_bf16: bf16 [num_pages][Hkv][2 (K, V)][16][128], 8 KiB per (page, kv head), 16-byte
+ *     aligned; num_pages * Hkv * 64 < 2^31.
+ * saw_append_bf16_paged scatters T tokens exactly (the stored bits are the input bits);
+ * saw_paged_decode_attn_bf16 computes, for each sequence s and query head hq (kv head
+ * h = hq / G, G <= 8), softmax(sm_scale <q, k_t>) . v over t < seq_lens[s] with bf16 x bf16
+ * tensor-core products accumulated in fp32 (results agree with fp64 to about 1e-3); its
+ * workspace comes from saw_paged_decode_bf16_workspace_bytes (no initialisation needed).
+ * saw_decode_step_bf16 is the append followed by the decode on one stream, as saw_decode_step.
+ * Arguments, ownership, alignment and status codes are those of the INT4 entry points. */
+int saw_append_bf16_paged(const saw_cache_desc *cache, const void *k, const void *v,
+                          const int64_t *slot_mapping, int64_t num_tokens, void *kv_bf16,
+                          uint32_t *dev_status, void *stream);
+size_t saw_paged_decode_bf16_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                             int32_t num_seqs);
+int saw_paged_decode_attn_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                               const void *kv_bf16, const int32_t *block_table,
+                               int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                               int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                               size_t workspace_bytes, uint32_t *dev_status, void *stream);
+int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                         const void *k_new, const void *v_new, const int64_t *slot_mapping,
+                         int64_t num_new_tokens, void *kv_bf16, const int32_t *block_table,
+                         int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                         float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                         uint32_t *dev_status, void *stream);
+
 /* saw_paged_decode_attn for callers that cannot allocate device memory.
  * The pages have no counterpart of this entry point: it exists for callers that are not allowed
  * or not able to call cudaMalloc -- a plug-in inside a serving framework whose memory pool
