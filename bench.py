@@ -92,6 +92,15 @@ def decode_bytes(wl) -> int:
     return int((wl.num_kv_heads * lens * BYTES_PER_TOKEN_HEAD_DECODE).sum() + per_seq.sum())
 
 
+def decode_bytes_bf16(wl) -> int:
+    """Algorithmic bytes of one decode over the uncompressed bf16 cache: 512 B per cached
+    token and kv head (K and V, 128 bf16 each) plus the same per-sequence terms."""
+    lens = wl.seq_lens.astype(np.int64)
+    pages = (lens + 15) // 16
+    per_seq = wl.num_q_heads * 128 * (2 + 4) + 4 + 4 * pages
+    return int((wl.num_kv_heads * lens * 512).sum() + per_seq.sum())
+
+
 def append_bytes(num_tokens: int, hkv: int) -> int:
     return num_tokens * (hkv * BYTES_PER_TOKEN_HEAD_APPEND + 8)
 
@@ -423,6 +432,35 @@ def run_saw(args):
                   "prefill_quant_rotation_overhead": t_rq / t_rq_plain - 1.0}
     del pkv2, psc2
 
+    # ---- the uncompressed BF16 cache on the same step: what the INT4 compression buys -------
+    kvb = saw.allocate_cache_bf16(wl.num_pages, wl.num_kv_heads, dev)
+    seq, pos = synth.token_index(wl, "history")
+    saw.saw_append_bf16_paged(synth.kv_values(wl, "K", tokens="history", device=dev),
+                              synth.kv_values(wl, "V", tokens="history", device=dev),
+                              torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(dev), kvb)
+    wsb = saw.allocate_workspace_bf16(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
+    bf16_step = lambda: saw.saw_decode_step_bf16(q, k_new, v_new, slots, kvb, table, lens, out, wsb,
+                                                 dev_status=status, stream=stream)
+    for _ in range(3):
+        bf16_step()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_pl):
+        bf16_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    bf_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
+    t_dec_bf16 = mean_event_ms(lambda: saw.saw_paged_decode_attn_bf16(
+        q, kvb, table, lens, out, wsb, dev_status=status, stream=stream), n_kt)
+    bf_gbs = decode_bytes_bf16(wl) / (t_dec_bf16 * 1e-3) / 1e9
+    bf16_baseline = {"what": "the same step on an uncompressed bf16 paged cache (4x the KV bytes)",
+                     "step_ms": bf_ms, "tokens_per_s": job_throughput(wl.num_seqs, world, bf_ms),
+                     "int4_step_speedup": bf_ms / ms_per_step,
+                     "decode_launch_ms": t_dec_bf16, "decode_GBps": bf_gbs,
+                     "decode_frac_of_measured_peak": bf_gbs / peak_gbs,
+                     "int4_decode_speedup": t_dec_bf16 / t_decode}
+    del kvb, wsb
+
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
     h_q, h_k, h_v, h_slots, h_table, h_lens = (pin(q), pin(k_new), pin(v_new), pin(slots),
@@ -473,6 +511,7 @@ def run_saw(args):
         "roofline": roofline,
         "rot_quant": rot_quant,
         "plain_int4": plain_int4,
+        "bf16_baseline": bf16_baseline,
         "append_launch_ms": t_append,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,
