@@ -3,7 +3,9 @@
 // per-warp online-softmax state, split-K partial slots in the workspace and the merge kernel
 // that folds a split segment's partials in a fixed order.
 //
-// A segment (sequence s, kv head h) of n = ceil(len_s / 16) pages costs n + kKappa in a cost
+// A segment (sequence s, kv head h, query sub-group: G > 8 query heads of one kv head are split
+// into ceil(G / 8) sub-groups, each its own segment reading the same pages, because the MMA
+// tiles stack at most 8 heads) of n = ceil(len_s / 16) pages costs n + kKappa in a cost
 // space where all segments lie end to end (sequence-major, then kv head); that range is cut
 // into equal slices, one per warp of a persistent grid, and a warp owns the pages whose cost
 // falls in its slice.  The pieces of a segment split across warps go to workspace slot
@@ -35,10 +37,21 @@ inline size_t merge_smem_bytes(int32_t num_seqs)
     return kMergeSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
 }
 
-// Workspace of a decode grid of `warps` warps over num_seqs * num_kv_heads segments.
-inline size_t workspace_bytes_for(size_t warps, int32_t num_seqs, int32_t num_kv_heads)
+// Query sub-groups of G = hq / hkv query heads per kv head (see DecodeParams).
+struct SubGroups {
+    int32_t nsub, gsub, hseg;
+};
+inline SubGroups sub_groups(int32_t num_kv_heads, int32_t num_q_heads)
 {
-    return (warps + static_cast<size_t>(num_seqs) * num_kv_heads) * kSlotFloats * sizeof(float);
+    const int32_t G = num_q_heads / num_kv_heads;
+    const int32_t nsub = (G + 7) / 8;
+    return {nsub, (G + nsub - 1) / nsub, num_kv_heads * nsub};
+}
+
+// Workspace of a decode grid of `warps` warps over num_seqs * segs_per_seq segments.
+inline size_t workspace_bytes_for(size_t warps, int32_t num_seqs, int32_t segs_per_seq)
+{
+    return (warps + static_cast<size_t>(num_seqs) * segs_per_seq) * kSlotFloats * sizeof(float);
 }
 
 struct DecodeParams {
@@ -54,9 +67,17 @@ struct DecodeParams {
     int32_t num_seqs;
     int32_t hq;
     int32_t hkv;
-    int32_t group;
+    int32_t group;               // G = hq / hkv
+    int32_t nsub;                // query sub-groups per kv head: ceil(G / 8) (MMA tiles are 8 wide)
+    int32_t gsub;                // query heads per sub-group: ceil(G / nsub) <= 8
+    int32_t hseg;                // segments per sequence: hkv * nsub
     int32_t total_warps;         // warps of the decode grid (the plan's slice count bound)
     float q_mult;                // the factor the kernel applies to q (or to the logits)
+
+    // Segment hv of a sequence is query sub-group hv % nsub of kv head hv / nsub.
+    __device__ int kv_head(int hv) const { return hv / nsub; }
+    __device__ int head_base(int hv) const { return (hv / nsub) * group + (hv % nsub) * gsub; }
+    __device__ int head_count(int hv) const { return min(gsub, group - (hv % nsub) * gsub); }
 };
 
 // ---- work plan ------------------------------------------------------------------------------
@@ -316,11 +337,11 @@ __global__ void __launch_bounds__(kMergeThreads)
 
     scan_pages(p, pre, flags, false);
     Plan plan;
-    plan.init(pre, p.num_seqs, p.hkv, p.total_warps);
+    plan.init(pre, p.num_seqs, p.hseg, p.total_warps);
     pdl_wait();   // the decode kernel's partials
     if (plan.P == 0)
         return;
-    const int64_t hkv = p.hkv;
+    const int64_t hkv = p.hseg;
     const int64_t J = static_cast<int64_t>(p.num_seqs) * hkv;
     for (int64_t seg = blockIdx.x; seg < J; seg += gridDim.x) {
         const int s = static_cast<int>(seg / hkv), h = static_cast<int>(seg - s * hkv);
@@ -376,13 +397,14 @@ __global__ void __launch_bounds__(kMergeThreads)
 //   Ring ring(base, warp)                          this warp's stage addresses;
 //   issue(ring, stg, bar, tmap, row, p)            queue a page's copies into stage stg,
 //                                                  completing on mbarrier bar (one elected lane);
-//   Query; load_query(p, qbuf, lane, q)            per-piece query fragments from the raw bf16
-//                                                  queries of the group in shared memory;
+//   Query; load_query(p, qbuf, n, lane, q)         per-piece query fragments from the raw bf16
+//                                                  queries of the segment's n <= 8 heads in
+//                                                  shared memory;
 //   page<kMask>(ring, stg, valid, q, lane, st)     attend over one staged page (first `valid`
 //                                                  tokens when kMask);
 //   piece_end(st)                                  reductions and corrections after a piece;
-//   finalize(p, s, h, lane, o, l)                  write a finished segment's output (also the
-//                                                  merge kernel's output step).
+//   finalize(p, s, hv, lane, o, l)                 write the output of segment hv of sequence s
+//                                                  (also the merge kernel's output step).
 // Shared memory: rings, then per warp (kStages + 1) mbarriers (the last for the query), 64 bytes
 // of flags, the per-warp query buffers (G * 256 bytes each) and the sequence page prefix.
 
@@ -415,7 +437,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int S = p.num_seqs;
-    int32_t *pre = reinterpret_cast<int32_t *>(smem + smem_prefix_offset<Fmt>(p.group));
+    int32_t *pre = reinterpret_cast<int32_t *>(smem + smem_prefix_offset<Fmt>(p.gsub));
     volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + smem_flags_offset<Fmt>());
 
     // ---- 1. pages per sequence, the plan, zero outputs of empty sequences ------------------
@@ -429,7 +451,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         }
     }
     Plan plan;
-    plan.init(pre, S, p.hkv, p.total_warps);
+    plan.init(pre, S, p.hseg, p.total_warps);
     const int64_t u = static_cast<int64_t>(blockIdx.x) * Fmt::kWarps + warp;
     if (plan.P == 0 || u >= plan.W)
         return;
@@ -437,12 +459,12 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     if (F0 >= F1)
         return;
     const int n_w = static_cast<int>(F1 - F0);
-    const int64_t hkv = p.hkv;
+    const int64_t hkv = p.hseg;   // segments per sequence
 
     // ---- 2. this warp's copy ring ---------------------------------------------------------------
     constexpr int kStages = Fmt::kStages;
     const typename Fmt::Ring ring = Fmt::ring(smem_u32(smem), warp);
-    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes(p.group);
+    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes(p.gsub);
     const uint32_t bar0 = smem_u32(smem + smem_bars_offset<Fmt>()) + warp * (kStages + 1) * 8;
     const uint32_t qbar = bar0 + kStages * 8;
     if (lane == 0)
@@ -466,14 +488,14 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
             set_status(p.status, SAW_DEV_BAD_PAGE);
             page = 0;
         }
-        return (page * p.hkv + h) * Fmt::kRowsPerPage;
+        return (page * p.hkv + p.kv_head(h)) * Fmt::kRowsPerPage;
     };
     // queue the raw queries of (s, h) into the warp's query buffer
     auto issue_query = [&](int s, int h) {
         if (lane == 0) {
-            const uint32_t bytes = static_cast<uint32_t>(p.group) * kHeadDim * 2;
+            const uint32_t bytes = static_cast<uint32_t>(p.head_count(h)) * kHeadDim * 2;
             mbar_arrive_expect_tx(qbar, bytes);
-            bulk_g2s(qbuf, p.q + (static_cast<int64_t>(s) * p.hq + static_cast<int64_t>(h) * p.group) * kHeadDim,
+            bulk_g2s(qbuf, p.q + (static_cast<int64_t>(s) * p.hq + p.head_base(h)) * kHeadDim,
                      bytes, qbar);
         }
     };
@@ -549,11 +571,11 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
             aborted = true;
         }
         qphase ^= 1;
-        Fmt::load_query(p, qbuf, lane, qf);
+        Fmt::load_query(p, qbuf, p.head_count(h), lane, qf);
         __syncwarp();
         int s_next = s, h_next = h;
         if (m_end < n_w) {
-            if (++h_next == p.hkv) {
+            if (++h_next == p.hseg) {
                 h_next = 0;
                 do {
                     s_next++;

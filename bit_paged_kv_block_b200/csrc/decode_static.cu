@@ -23,7 +23,7 @@
 
 namespace {
 
-// Room for num_seqs * num_kv_heads <= 2048 (sequence, kv head) pairs and a decode grid of up
+// Room for num_seqs * num_kv_heads * ceil(G / 8) <= 2048 decode segments and a decode grid of up
 // to 2560 warps: (2560 + 2048) partial-result slots of 4160 bytes.
 constexpr int kScratchMaxSegments = 2048;
 constexpr size_t kScratchBytes = (2560 + kScratchMaxSegments) * size_t(4160);
@@ -64,7 +64,10 @@ extern "C" int saw_paged_decode_attn_static(const saw_cache_desc *cache, int32_t
 {
     if (cache == nullptr || cache->num_kv_heads <= 0 || num_seqs < 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if (int64_t(num_seqs) * cache->num_kv_heads > kScratchMaxSegments)
+    if (num_q_heads <= 0 || num_q_heads % cache->num_kv_heads != 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    const int64_t group = num_q_heads / cache->num_kv_heads;
+    if (int64_t(num_seqs) * cache->num_kv_heads * ((group + 7) / 8) > kScratchMaxSegments)
         return SAW_ERR_SCRATCH_LIMIT;
     const size_t need = saw_paged_decode_workspace_bytes(cache, num_q_heads, num_seqs);
     if (num_seqs > 0 && need > kScratchBytes)

@@ -72,15 +72,15 @@ __device__ __forceinline__ float2 h2_to_f2(uint32_t u)
     return __half22float2(u32_as_half2(u));
 }
 
-// Rotated, scaled query of (seq s, kv head h) as fp16 mma B fragments, from the raw bf16
-// queries of the group in shared memory ([G][128] at qbuf).
+// Rotated, scaled query of one segment as fp16 mma B fragments, from the raw bf16 queries of
+// its nheads <= 8 heads in shared memory ([nheads][128] at qbuf).
 // Thread (g, t) owns query head g of the group and d in [32t, 32t + 32).
 template <bool kRotate>
-__device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int g, int t,
-                                           uint32_t bq[8][2], float sq_out[2])
+__device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int g,
+                                           int t, uint32_t bq[8][2], float sq_out[2])
 {
     float x[32];
-    if (g < p.group) {
+    if (g < nheads) {
 #pragma unroll
         for (int c = 0; c < 4; c++) {
             const uint4 u = lds128(qbuf + g * (kHeadDim * 2) + 64 * t + 16 * c);
@@ -236,9 +236,9 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
 
 
 // o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the heads this thread
-// holds; written to out[s][h G + 2t + e].
+// holds; written to out[s][head_base(hv) + 2t + e].
 template <bool kRotate>
-__device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, int lane,
+__device__ __forceinline__ void finalize(const DecodeParams &p, int s, int hv, int lane,
                                          float o[8][4], const float l[2])
 {
     const int g = lane >> 2, t = lane & 3;
@@ -295,8 +295,8 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int h, in
 #pragma unroll
     for (int e = 0; e < 2; e++) {
         const int head = 2 * t + e;
-        if (head < p.group) {
-            float *dst = p.out + ((static_cast<int64_t>(s) * p.hq + h * p.group + head) * kHeadDim);
+        if (head < p.head_count(hv)) {
+            float *dst = p.out + ((static_cast<int64_t>(s) * p.hq + p.head_base(hv) + head) * kHeadDim);
 #pragma unroll
             for (int c = 0; c < 4; c++) {
                 const float f = kRotate ? kHadamardC : 1.0f;
@@ -358,9 +358,10 @@ struct Int4Format {
         copy_page_elected(bar, r.code0 + stg * kCodeBytes, tmap, row, r.scale0 + stg * kScaleBytes,
                           p.scales + static_cast<int64_t>(row) * 4);
     }
-    __device__ static void load_query(const DecodeParams &p, uint32_t qbuf, int lane, Query &q)
+    __device__ static void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int lane,
+                                      Query &q)
     {
-        saw::load_query<kRotate>(p, qbuf, lane >> 2, lane & 3, q.bq, q.sq);
+        saw::load_query<kRotate>(p, qbuf, nheads, lane >> 2, lane & 3, q.bq, q.sq);
     }
     template <bool kMask>
     __device__ static void page(const Ring &r, int stg, int valid, const Query &q, int lane,
@@ -390,10 +391,10 @@ struct Int4Format {
             st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
         }
     }
-    __device__ static void finalize(const DecodeParams &p, int s, int h, int lane, float o[8][4],
+    __device__ static void finalize(const DecodeParams &p, int s, int hv, int lane, float o[8][4],
                                     const float l[2])
     {
-        saw::finalize<kRotate>(p, s, h, lane, o, l);
+        saw::finalize<kRotate>(p, s, hv, lane, o, l);
     }
 };
 
@@ -420,11 +421,12 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
     LaunchShape ls;
-    if (launch_shape(decode_smem_bytes<Int4Format<true>>(num_seqs, num_q_heads / num_kv_heads),
+    const SubGroups sg = sub_groups(num_kv_heads, num_q_heads);
+    if (launch_shape(decode_smem_bytes<Int4Format<true>>(num_seqs, sg.gsub),
                      merge_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
     return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Int4Format<true>::kWarps,
-                               num_seqs, num_kv_heads);
+                               num_seqs, sg.hseg);
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
@@ -456,7 +458,8 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     }
 
     using Fmt = Int4Format<true>;   // the layout is the same for both variants
-    const size_t smem = decode_smem_bytes<Fmt>(a.num_seqs, a.num_q_heads / a.num_kv_heads);
+    const SubGroups sg = sub_groups(a.num_kv_heads, a.num_q_heads);
+    const size_t smem = decode_smem_bytes<Fmt>(a.num_seqs, sg.gsub);
     const size_t msmem = merge_smem_bytes(a.num_seqs);
     LaunchShape ls;
     cudaError_t e = launch_shape(smem, msmem, ls);
@@ -477,6 +480,9 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     p.hq = a.num_q_heads;
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
+    p.nsub = sg.nsub;
+    p.gsub = sg.gsub;
+    p.hseg = sg.hseg;
     p.total_warps = ls.sms * ls.occ * Fmt::kWarps;
     // q carries sm_scale * log2(e), and 1/sqrt(128) of the (unnormalised) query butterfly
     p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(kHadamardC) : 1.0) * a.sm_scale *
@@ -498,7 +504,7 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     if (e != cudaSuccess)
         return e;
 
-    const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+    const int64_t segs = static_cast<int64_t>(a.num_seqs) * p.hseg;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
     mcfg.blockDim = dim3(kMergeThreads);

@@ -83,15 +83,16 @@ struct Bf16Format {
                      : "memory");
     }
 
-    // Thread (g, t) holds query head g of the group (zero for g >= G) as mma B fragments.
-    __device__ static void load_query(const DecodeParams &p, uint32_t qbuf, int lane, Query &q)
+    // Thread (g, t) holds query head g of the segment (zero for g >= nheads) as mma B fragments.
+    __device__ static void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int lane,
+                                      Query &q)
     {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
         for (int i = 0; i < 8; i++) {
             const uint32_t a = qbuf + g * (kHeadDim * 2) + (16 * i + 2 * t) * 2;
-            q.bq[i][0] = g < p.group ? lds32(a) : 0u;
-            q.bq[i][1] = g < p.group ? lds32(a + 16) : 0u;
+            q.bq[i][0] = g < nheads ? lds32(a) : 0u;
+            q.bq[i][1] = g < nheads ? lds32(a + 16) : 0u;
         }
         q.mult = p.q_mult;
     }
@@ -171,18 +172,18 @@ struct Bf16Format {
                 st.l[e] += __shfl_xor_sync(0xFFFFFFFFu, st.l[e], d);
     }
 
-    // out[s][h G + 2t + e][d] = o / l; tile c, rows g and g + 8 are d = 16 c + g (+ 8).
-    __device__ static void finalize(const DecodeParams &p, int s, int h, int lane, float o[8][4],
+    // out[s][head_base(hv) + 2t + e][d] = o / l; tile c, rows g and g + 8 are d = 16 c + g (+ 8).
+    __device__ static void finalize(const DecodeParams &p, int s, int hv, int lane, float o[8][4],
                                     const float l[2])
     {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const int head = 2 * t + e;
-            if (head >= p.group)
+            if (head >= p.head_count(hv))
                 continue;
             const float inv = 1.0f / l[e];
-            float *dst = p.out + (static_cast<int64_t>(s) * p.hq + h * p.group + head) * kHeadDim;
+            float *dst = p.out + (static_cast<int64_t>(s) * p.hq + p.head_base(hv) + head) * kHeadDim;
 #pragma unroll
             for (int c = 0; c < 8; c++) {
                 dst[16 * c + g] = o[c][e] * inv;
@@ -262,11 +263,12 @@ size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, in
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
     LaunchShape ls;
-    if (bf16_launch_shape(decode_smem_bytes<Bf16Format>(num_seqs, num_q_heads / num_kv_heads),
+    const SubGroups sg = sub_groups(num_kv_heads, num_q_heads);
+    if (bf16_launch_shape(decode_smem_bytes<Bf16Format>(num_seqs, sg.gsub),
                           merge_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
     return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Bf16Format::kWarps, num_seqs,
-                               num_kv_heads);
+                               sg.hseg);
 }
 
 cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
@@ -297,7 +299,8 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
         cache.rows = rows;
     }
 
-    const size_t smem = decode_smem_bytes<Bf16Format>(a.num_seqs, a.num_q_heads / a.num_kv_heads);
+    const SubGroups sg = sub_groups(a.num_kv_heads, a.num_q_heads);
+    const size_t smem = decode_smem_bytes<Bf16Format>(a.num_seqs, sg.gsub);
     const size_t msmem = merge_smem_bytes(a.num_seqs);
     LaunchShape ls;
     cudaError_t e = bf16_launch_shape(smem, msmem, ls);
@@ -318,6 +321,9 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     p.hq = a.num_q_heads;
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
+    p.nsub = sg.nsub;
+    p.gsub = sg.gsub;
+    p.hseg = sg.hseg;
     p.total_warps = ls.sms * ls.occ * Bf16Format::kWarps;
     p.q_mult = static_cast<float>(static_cast<double>(a.sm_scale) * 1.4426950408889634);
 
@@ -335,7 +341,7 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     if (e != cudaSuccess)
         return e;
 
-    const int64_t segs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+    const int64_t segs = static_cast<int64_t>(a.num_seqs) * p.hseg;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
     mcfg.blockDim = dim3(kMergeThreads);

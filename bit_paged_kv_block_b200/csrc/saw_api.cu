@@ -51,7 +51,7 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
 {
     if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if (num_q_heads / cache->num_kv_heads > 8)
+    if (num_q_heads / cache->num_kv_heads > 16)
         return SAW_ERR_UNSUPPORTED;
     if (!std::isfinite(sm_scale))
         return SAW_ERR_INVALID_ARGUMENT;
@@ -115,14 +115,14 @@ const char *saw_status_string(int status)
     case SAW_ERR_INVALID_ARGUMENT:
         return "invalid argument (null pointer, bad size or alignment, Hq not a multiple of Hkv)";
     case SAW_ERR_UNSUPPORTED:
-        return "unsupported shape (head_dim must be 128, page_size 16, Hq/Hkv at most 8)";
+        return "unsupported shape (head_dim must be 128, page_size 16, Hq/Hkv at most 16)";
     case SAW_ERR_CUDA:
         return "CUDA runtime error";
     case SAW_ERR_WORKSPACE:
         return "workspace missing, misaligned or too small";
     case SAW_ERR_SCRATCH_LIMIT:
         return "shape too large for the fixed scratch of saw_paged_decode_attn_static "
-               "(num_seqs * num_kv_heads must be at most 2048)";
+               "(num_seqs * num_kv_heads * ceil(Hq / Hkv / 8) must be at most 2048)";
     default:
         return "unknown status";
     }
@@ -250,7 +250,7 @@ size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num
                                         int32_t num_seqs)
 {
     if (check_cache(cache) != SAW_OK || num_q_heads <= 0 ||
-        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 8)
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
         return 0;
     return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
 }

@@ -291,7 +291,8 @@ def _step(fn, name, q, k_new, v_new, slot_mapping, kv_pages, scales, block_table
 def saw_paged_decode_attn_static(q, kv_pages, scales, block_table, seq_lens, out, sm_scale=None,
                                  dev_status=None, stream=None) -> None:
     """saw_paged_decode_attn without a workspace, for callers that cannot allocate device memory:
-    the scratch is a fixed array inside the library (num_seqs * num_kv_heads <= 2048).  Calls
+    the scratch is a fixed array inside the library (num_seqs * num_kv_heads * ceil(G / 8)
+    <= 2048).  Calls
     share that array, so calls that can overlap on the GPU must be serialised by the caller."""
     _need(q, "q", torch.bfloat16, 3)
     _need(kv_pages, "kv_pages", torch.uint8, 5)

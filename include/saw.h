@@ -61,7 +61,7 @@ extern "C" {
 typedef enum saw_status {
     SAW_OK = 0,
     SAW_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
-    SAW_ERR_UNSUPPORTED = 2,      /* head_dim != 128, page_size != 16, Hq / Hkv > 8 */
+    SAW_ERR_UNSUPPORTED = 2,      /* head_dim != 128, page_size != 16, Hq / Hkv > 16 */
     SAW_ERR_CUDA = 3,             /* a CUDA runtime call or kernel launch failed */
     SAW_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required */
     SAW_ERR_SCRATCH_LIMIT = 5     /* shape too large for saw_paged_decode_attn_static */
@@ -104,7 +104,8 @@ int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, voi
 /* Decode attention over the INT4 paged cache.
  * Follows "SAW-INT4" (Research Findings: fused attention execution over a paged cache) and
  * "BitDecoding-FP4" (abstract: stacked query heads over paged KV).  For each sequence s and
- * query head hq (kv head h = hq / G, G = Hq / Hkv <= 8):
+ * query head hq (kv head h = hq / G, G = Hq / Hkv <= 16; G > 8 runs as ceil(G / 8) groups of
+ * query heads that each read the kv head's pages):
  *     q_r = H q,   s_t = sm_scale * <q_r, zero_t + code_t * scale_t>  for t < seq_lens[s],
  *     o_r = softmax(s) . (zero_t + code_t * scale_t) over the V side,   out = H o_r.
  * The kernel computes in fp16 x fp16 -> fp32 tensor-core tiles on raw codes with the scale
@@ -170,7 +171,7 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
  *     aligned; num_pages * Hkv * 64 < 2^31.
  * saw_append_bf16_paged scatters T tokens exactly (the stored bits are the input bits);
  * saw_paged_decode_attn_bf16 computes, for each sequence s and query head hq (kv head
- * h = hq / G, G <= 8), softmax(sm_scale <q, k_t>) . v over t < seq_lens[s] with bf16 x bf16
+ * h = hq / G, G <= 16), softmax(sm_scale <q, k_t>) . v over t < seq_lens[s] with bf16 x bf16
  * tensor-core products accumulated in fp32 (results agree with fp64 to about 1e-3); its
  * workspace comes from saw_paged_decode_bf16_workspace_bytes (no initialisation needed).
  * saw_decode_step_bf16 is the append followed by the decode on one stream, as saw_decode_step.
@@ -200,8 +201,8 @@ int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const
  * exactly what saw_paged_decode_attn computes, but its split-K scratch lives in one fixed array
  * of 18.3 MiB inside this library's device code (present on every GPU that loads the library,
  * until the process exits) instead of a caller workspace.  It allocates nothing.
- * Limit: num_seqs * num_kv_heads <= 2048 and a decode grid of at most 2560 warps (a B200 runs
- * 2368); larger shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
+ * Limit: num_seqs * num_kv_heads * ceil(G / 8) <= 2048 and a decode grid of at most 2560 warps
+ * (a B200 runs 2368); larger shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
  * that device current); make that first call before any stream capture.  Nothing in the array
  * needs to start at zero.  All calls on a device share the array and it keeps the previous

@@ -74,7 +74,7 @@ def _dec(desc, hq=32, S=2, q=16, out=16, bt=16, lens=16, ws=256, ws_bytes=1 << 2
 def test_decode_argument_checks():
     d = _desc()
     assert _dec(d, hq=12) == saw.SAW_ERR_INVALID_ARGUMENT             # Hq % Hkv
-    assert _dec(d, hq=72) == saw.SAW_ERR_UNSUPPORTED                  # G = 9
+    assert _dec(d, hq=136) == saw.SAW_ERR_UNSUPPORTED                 # G = 17 (at most 16)
     assert _dec(d, S=-1) == saw.SAW_ERR_INVALID_ARGUMENT
     assert _dec(d, q=0) == saw.SAW_ERR_INVALID_ARGUMENT
     assert _dec(d, q=8) == saw.SAW_ERR_INVALID_ARGUMENT

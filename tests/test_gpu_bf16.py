@@ -82,7 +82,7 @@ def _decode_bf16(wl, kv, device, q, sm_scale=None):
 
 
 @pytest.mark.parametrize("G,lens", [(1, [1, 16, 17]), (2, [15, 31, 33, 64]), (4, [5, 300, 0, 129]),
-                                    (8, [1000, 1, 48])])
+                                    (8, [1000, 1, 48]), (12, [70, 1, 33]), (16, [257, 16])])
 def test_bf16_decode_matches_oracle(cuda_device, G, lens):
     hkv = 2
     wl = synth.custom(f"bf16dec{G}", lens, num_q_heads=G * hkv, num_kv_heads=hkv, seed=G + 20,

@@ -48,11 +48,12 @@ def test_decode_tiny(cuda_device):
     check(synth.make_workload("tiny"), cuda_device)
 
 
-@pytest.mark.parametrize("G", [1, 2, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8, 9, 12, 16])
 @pytest.mark.parametrize("lens", [[1], [15, 16, 17], [2, 31, 32, 33, 64, 100],
                                   [1000, 3, 257, 48, 16 * 37 + 5]])
 def test_decode_shapes(cuda_device, G, lens):
-    """Page boundaries (15/16/17, 31/32/33), single tokens, ragged lengths, every group size."""
+    """Page boundaries (15/16/17, 31/32/33), single tokens, ragged lengths, group sizes up to 16
+    (above 8 the query heads of a kv head run as ceil(G / 8) sub-groups, uneven for G = 9)."""
     hkv = 2 if G < 8 else 1
     wl = synth.custom(f"shape{G}_{len(lens)}", lens, num_q_heads=G * hkv, num_kv_heads=hkv,
                       seed=len(lens) * 10 + G, outlier_range=(10.0, 30.0))
@@ -149,3 +150,21 @@ def test_decode_step_full_size(cuda_device, name):
     sample = [0, 1, wl.num_seqs // 2, wl.num_seqs - 1]
     want = oracle_decode(subset(wl, sample), full_pages, full_scales, q=q[sample])
     assert_attention_close(got[sample], want, name + " step")
+
+
+def test_decode_g16_several_kv_heads_and_static_entry(cuda_device):
+    """G = 16 with 4 kv heads (8 segments per sequence), through both the workspace entry point
+    and the fixed-scratch one; the two results are bit-identical."""
+    from bit_paged_kv_block_b200 import saw
+    wl = synth.custom("g16", [300, 17, 1, 64], num_q_heads=64, num_kv_heads=4, seed=16,
+                      outlier_range=(10.0, 30.0))
+    pages, scales = oracle_cache(wl)
+    got, _ = run_decode(wl, pages, scales, cuda_device)
+    assert_attention_close(got, oracle_decode(wl, pages, scales), "g16")
+    kv, sc = device_cache_from(pages, scales, cuda_device)
+    out = torch.empty((wl.num_seqs, wl.num_q_heads, 128), device=cuda_device)
+    saw.saw_paged_decode_attn_static(synth.q_values(wl).to(cuda_device), kv, sc,
+                                     torch.from_numpy(wl.block_table).to(cuda_device),
+                                     torch.from_numpy(wl.seq_lens).to(cuda_device), out)
+    torch.cuda.synchronize()
+    assert np.array_equal(out.cpu().numpy(), got)
