@@ -213,6 +213,7 @@ struct RqParams {
     uint8_t *kv_pages;
     uint32_t *scales;        // fp16x2 (scale, zero) per row
     uint32_t *status;
+    bool strided;            // k / v through 3-D tensor maps with a token stride
 };
 
 // Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
@@ -319,14 +320,25 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 
     int issued = 0, istg = 0;
     uint32_t itile = wg;
+    const uint32_t hkv_u = static_cast<uint32_t>(p.hkv);
     auto issue = [&]() {
         if (issued < n) {
             if (lane == 0) {
                 const uint32_t dst = ring + istg * kRqStageBytes;
-                const int32_t y = static_cast<int32_t>(itile * (2 * kTileVecs));
-                mbar_arrive_expect_tx(bar0 + 8 * istg, kRqStageBytes);
-                tma_load_2d(dst, &tk, 0, y, bar0 + 8 * istg);
-                tma_load_2d(dst + kTileBytes, &tv, 0, y, bar0 + 8 * istg);
+                const uint32_t bar = bar0 + 8 * istg;
+                mbar_arrive_expect_tx(bar, kRqStageBytes);
+                if (p.strided) {
+                    // the tile's first vector: token and head (the box spans whole tiles)
+                    const uint32_t v0 = itile * kTileVecs;
+                    const int32_t tok = static_cast<int32_t>(v0 / hkv_u);
+                    const int32_t row = static_cast<int32_t>(2 * (v0 - tok * hkv_u));
+                    tma_load_3d(dst, &tk, 0, row, tok, bar);
+                    tma_load_3d(dst + kTileBytes, &tv, 0, row, tok, bar);
+                } else {
+                    const int32_t y = static_cast<int32_t>(itile * (2 * kTileVecs));
+                    tma_load_2d(dst, &tk, 0, y, bar);
+                    tma_load_2d(dst + kTileBytes, &tv, 0, y, bar);
+                }
             }
             issued++;
             itile += W;
@@ -413,25 +425,49 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     if (num_vecs > (int64_t(1) << 29))
         return cudaErrorInvalidValue;       // tensor-map rows (2 per vector) must fit in int32
 
+    // k / v: contiguous [T][Hkv][128] (k_stride = v_stride = 0) through a 2-D map of 128-byte
+    // rows, or with a token stride through 3-D maps whose box is one whole tile of 8 vectors
+    // (Hkv a multiple of 8: 8 heads of one token; Hkv dividing 8: 8 / Hkv tokens), so every
+    // copy lands on a 1024-byte aligned stage.
+    const bool strided = a.k_stride != 0 || a.v_stride != 0;
     static thread_local struct {
         const void *k = nullptr, *v = nullptr;
-        int64_t num_vecs = 0;
+        int64_t num_vecs = 0, k_stride = -1, v_stride = -1;
+        int32_t hkv = 0;
         CUtensorMap mk, mv;
     } cache;
-    if (cache.k != a.k || cache.v != a.v || cache.num_vecs != num_vecs) {
+    if (cache.k != a.k || cache.v != a.v || cache.num_vecs != num_vecs || cache.hkv != a.num_kv_heads ||
+        cache.k_stride != a.k_stride || cache.v_stride != a.v_stride) {
         auto encode = tensor_map_encoder();
         if (encode == nullptr)
             return cudaErrorNotSupported;
-        const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(2 * num_vecs)};
-        const cuuint64_t strides[1] = {128};
-        const cuuint32_t box[2] = {128, 2 * kTileVecs};   // one warp tile: 16 rows of 128 B
-        const cuuint32_t estr[2] = {1, 1};
+        const int64_t hkv = a.num_kv_heads;
+        if (strided && hkv % kTileVecs != 0 && kTileVecs % hkv != 0)
+            return cudaErrorInvalidValue;
+        const cuuint32_t estr[3] = {1, 1, 1};
         for (int which = 0; which < 2; which++) {
-            CUresult r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                                const_cast<void *>(which ? a.v : a.k), dims, strides, box, estr,
-                                CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                                CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
-                                CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            CUresult r;
+            void *base = const_cast<void *>(which ? a.v : a.k);
+            if (!strided) {
+                const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(2 * num_vecs)};
+                const cuuint64_t strides[1] = {128};
+                const cuuint32_t box[2] = {128, 2 * kTileVecs};   // one warp tile: 16 rows
+                r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
+                           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            } else {
+                const int64_t stride = which ? a.v_stride : a.k_stride;   // bf16 elements
+                const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(2 * hkv),
+                                            static_cast<cuuint64_t>(a.num_tokens)};
+                const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(stride * 2)};
+                const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(2 * std::min<int64_t>(hkv, kTileVecs)),
+                                           static_cast<cuuint32_t>(std::max<int64_t>(1, kTileVecs / hkv))};
+                r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base,
+                           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                           CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                           CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+            }
             if (r != CUDA_SUCCESS) {
                 cache.k = nullptr;
                 return cudaErrorInvalidValue;
@@ -440,6 +476,9 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         cache.k = a.k;
         cache.v = a.v;
         cache.num_vecs = num_vecs;
+        cache.hkv = a.num_kv_heads;
+        cache.k_stride = a.k_stride;
+        cache.v_stride = a.v_stride;
     }
 
     RqParams p;
@@ -451,6 +490,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     p.kv_pages = a.kv_pages;
     p.scales = static_cast<uint32_t *>(a.scales);
     p.status = a.status;
+    p.strided = strided;
 
     // per device: multiprocessor count, the shared-memory attribute and the occupancy
     constexpr int kMaxDevices = 64;

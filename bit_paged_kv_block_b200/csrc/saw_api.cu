@@ -151,18 +151,36 @@ saw::RotateQuantizeArgs append_args(const saw_cache_desc *cache, const void *k, 
     return a;
 }
 
+// k_stride / v_stride: bf16 elements between consecutive tokens of k / v (0: contiguous)
 int append_impl(const saw_cache_desc *cache, const void *k, const void *v,
                 const int64_t *slot_mapping, int64_t num_tokens, uint8_t *kv_pages, void *scales,
-                uint32_t *dev_status, void *stream, bool rotate)
+                uint32_t *dev_status, void *stream, bool rotate, int64_t k_stride = 0,
+                int64_t v_stride = 0)
 {
     int rc = check_cache(cache);
     if (rc != SAW_OK)
         return rc;
     rc = check_append(cache, k, v, slot_mapping, num_tokens, kv_pages, scales);
-    if (rc != SAW_OK || num_tokens == 0)
+    if (rc != SAW_OK)
         return rc;
-    const saw::RotateQuantizeArgs a =
+    if (k_stride != 0 || v_stride != 0) {
+        // strided rows: each token's Hkv head vectors are contiguous; tokens start every
+        // *_stride elements (a multiple of 8, so every token starts on 16 bytes)
+        const int64_t row = int64_t(cache->num_kv_heads) * 128;
+        if (k_stride < row || v_stride < row || k_stride % 8 != 0 || v_stride % 8 != 0 ||
+            k_stride > (int64_t(1) << 36) || v_stride > (int64_t(1) << 36))
+            return SAW_ERR_INVALID_ARGUMENT;
+        if (cache->num_kv_heads % 8 != 0 && 8 % cache->num_kv_heads != 0)
+            return SAW_ERR_UNSUPPORTED;
+        if (num_tokens > (int64_t(1) << 31) - 1)
+            return SAW_ERR_INVALID_ARGUMENT;
+    }
+    if (num_tokens == 0)
+        return SAW_OK;
+    saw::RotateQuantizeArgs a =
         append_args(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status, rotate);
+    a.k_stride = k_stride;
+    a.v_stride = v_stride;
     return saw::launch_rotate_quantize(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
                ? SAW_OK
                : SAW_ERR_CUDA;
@@ -244,6 +262,28 @@ int saw_quantize_paged_plain(const saw_cache_desc *cache, const void *k, const v
 {
     return append_impl(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status,
                        stream, false);
+}
+
+int saw_rotate_quantize_paged_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
+                                      const void *v, int64_t v_stride, const int64_t *slot_mapping,
+                                      int64_t num_tokens, uint8_t *kv_pages, void *scales,
+                                      uint32_t *dev_status, void *stream)
+{
+    if (k_stride == 0 || v_stride == 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    return append_impl(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status,
+                       stream, true, k_stride, v_stride);
+}
+
+int saw_quantize_paged_plain_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
+                                     const void *v, int64_t v_stride, const int64_t *slot_mapping,
+                                     int64_t num_tokens, uint8_t *kv_pages, void *scales,
+                                     uint32_t *dev_status, void *stream)
+{
+    if (k_stride == 0 || v_stride == 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    return append_impl(cache, k, v, slot_mapping, num_tokens, kv_pages, scales, dev_status,
+                       stream, false, k_stride, v_stride);
 }
 
 size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,

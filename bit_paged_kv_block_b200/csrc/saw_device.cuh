@@ -178,6 +178,16 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const void *tmap, int3
                  : "memory");
 }
 
+// 3-D tensor copy global -> shared through a tensor map (no multicast).
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const void *tmap, int32_t x, int32_t y,
+                                            int32_t z, uint32_t bar)
+{
+    asm volatile("cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+                 " [%0], [%1, {%2, %3, %4}], [%5];"
+                 ::"r"(dst), "l"(tmap), "r"(x), "r"(y), "r"(z), "r"(bar)
+                 : "memory");
+}
+
 __device__ __forceinline__ uint4 lds128(uint32_t addr)
 {
     uint4 r;

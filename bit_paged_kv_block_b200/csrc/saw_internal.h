@@ -34,6 +34,8 @@ struct RotateQuantizeArgs {
     void *scales;                // fp16 [num_pages][Hkv][2][16][2]
     uint32_t *status;            // nullable
     bool rotate = true;          // false: plain INT4 (no Hadamard rotation)
+    int64_t k_stride = 0;        // bf16 elements between tokens of k (0: contiguous, Hkv * 128)
+    int64_t v_stride = 0;        // the same for v
 };
 
 struct DecodeArgs {

@@ -75,6 +75,10 @@ def _open_library() -> ctypes.CDLL:
     lib.saw_paged_decode_attn_plain.restype = ctypes.c_int
     lib.saw_decode_step_plain.argtypes = lib.saw_decode_step.argtypes
     lib.saw_decode_step_plain.restype = ctypes.c_int
+    lib.saw_rotate_quantize_paged_strided.argtypes = [D, P, i64, P, i64, P, i64, P, P, P, P]
+    lib.saw_rotate_quantize_paged_strided.restype = ctypes.c_int
+    lib.saw_quantize_paged_plain_strided.argtypes = lib.saw_rotate_quantize_paged_strided.argtypes
+    lib.saw_quantize_paged_plain_strided.restype = ctypes.c_int
     lib.saw_append_bf16_paged.argtypes = [D, P, P, P, i64, P, P, P]
     lib.saw_append_bf16_paged.restype = ctypes.c_int
     lib.saw_paged_decode_bf16_workspace_bytes.argtypes = [D, i32, i32]
@@ -182,6 +186,33 @@ def _append(fn, name, k, v, slot_mapping, kv_pages, scales, dev_status, stream) 
     rc = fn(ctypes.byref(desc), _ptr(k), _ptr(v), _ptr(slot_mapping), T, _ptr(kv_pages),
             _ptr(scales), _ptr(dev_status), _stream(stream))
     _check(rc, name)
+
+
+def saw_rotate_quantize_paged_strided(k, v, slot_mapping, kv_pages, scales, dev_status=None,
+                                      stream=None, rotate=True) -> None:
+    """saw_rotate_quantize_paged for k, v that are token-strided views (e.g. slices of a fused
+    QKV output): [T][Hkv][128] with the heads of a token contiguous (strides (s, 128, 1)).
+    rotate=False is the plain INT4 quantizer."""
+    for t, name in ((k, "k"), (v, "v")):
+        if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device.type != "cuda":
+            raise TypeError(f"{name} must be a bf16 CUDA tensor")
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != HEAD_DIM:
+            raise ValueError(f"{name} must be [T][Hkv][128] with contiguous heads within a token")
+    _need(slot_mapping, "slot_mapping", torch.int64, 1)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    desc = cache_desc(kv_pages)
+    T = k.shape[0]
+    if tuple(k.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
+        raise ValueError("k and v must be [T][Hkv][128] matching the cache")
+    if slot_mapping.shape[0] != T:
+        raise ValueError("slot_mapping must have one entry per token")
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    fn = lib.saw_rotate_quantize_paged_strided if rotate else lib.saw_quantize_paged_plain_strided
+    rc = fn(ctypes.byref(desc), _ptr(k), k.stride(0), _ptr(v), v.stride(0), _ptr(slot_mapping), T,
+            _ptr(kv_pages), _ptr(scales), _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_rotate_quantize_paged_strided" if rotate else "saw_quantize_paged_plain_strided")
 
 
 def saw_paged_decode_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,

@@ -91,6 +91,23 @@ int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const 
                               uint8_t *kv_pages, void *scales, uint32_t *dev_status,
                               void *stream);
 
+/* saw_rotate_quantize_paged (and its plain INT4 counterpart) for k and v that are not
+ * contiguous, e.g. slices of a fused QKV projection output [T][(Hq + 2 Hkv) * 128]: each
+ * token's Hkv head vectors are contiguous (128 bf16 each, head-major), and token t starts at
+ * k + t * k_stride (v + t * v_stride) bf16 elements.  Strides are at least Hkv * 128 and a
+ * multiple of 8 (every token starts on 16 bytes; k and v themselves 16-byte aligned).
+ * Supported for Hkv a multiple of 8 or a divisor of 8 (else SAW_ERR_UNSUPPORTED): the kernel
+ * copies whole 8-vector tiles.  Results are bit-identical to the contiguous call on the same
+ * values. */
+int saw_rotate_quantize_paged_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
+                                      const void *v, int64_t v_stride, const int64_t *slot_mapping,
+                                      int64_t num_tokens, uint8_t *kv_pages, void *scales,
+                                      uint32_t *dev_status, void *stream);
+int saw_quantize_paged_plain_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
+                                     const void *v, int64_t v_stride, const int64_t *slot_mapping,
+                                     int64_t num_tokens, uint8_t *kv_pages, void *scales,
+                                     uint32_t *dev_status, void *stream);
+
 /* Bytes of workspace saw_paged_decode_attn / saw_decode_step need for this shape on the
  * current device (split-K partial results: one slot per warp of the decode grid plus one per
  * (seq, kv head)).  Returns 0 for an unsupported or invalid shape. */

@@ -107,3 +107,18 @@ def test_python_binding_rejects_cpu_tensors():
         saw.saw_rotate_quantize_paged(k, k, torch.zeros(2, dtype=torch.int64), kv, sc)
     with pytest.raises(TypeError):
         saw.saw_rotate_quantize_paged(k.float(), k, torch.zeros(2, dtype=torch.int64), kv, sc)
+
+
+def test_strided_append_argument_checks():
+    """Strides below a token's Hkv * 128 elements or not a multiple of 8 are invalid; Hkv that
+    neither divides nor is a multiple of 8 is unsupported (checked before any launch)."""
+    def call(hkv, ks, vs):
+        desc = saw.saw_cache_desc(hkv, 128, 16, 4)
+        return saw.lib.saw_rotate_quantize_paged_strided(
+            ctypes.byref(desc), ctypes.c_void_p(16), ks, ctypes.c_void_p(16), vs,
+            ctypes.c_void_p(16), 10, ctypes.c_void_p(16), ctypes.c_void_p(16), None, None)
+    assert call(2, 0, 256) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert call(2, 200, 256) == saw.SAW_ERR_INVALID_ARGUMENT       # < Hkv * 128
+    assert call(2, 260, 256) == saw.SAW_ERR_INVALID_ARGUMENT       # not a multiple of 8
+    assert call(3, 384, 384) == saw.SAW_ERR_UNSUPPORTED
+    assert call(12, 12 * 128, 12 * 128) == saw.SAW_ERR_UNSUPPORTED

@@ -114,3 +114,29 @@ def test_empty_append_is_noop(cuda_device):
                                   kv, sc)
     torch.cuda.synchronize()
     assert bool((kv == CANARY_CODE).all())
+
+
+@pytest.mark.parametrize("hkv", [1, 2, 8, 16])
+@pytest.mark.parametrize("rotate", [True, False])
+def test_strided_kv_from_fused_qkv(cuda_device, hkv, rotate):
+    """k and v as slices of a fused QKV projection output [T][(Hq + 2 Hkv) * 128] (token
+    stride (Hq + 2 Hkv) * 128): codes and scales bit-identical to the oracle on the same
+    values, for Hkv dividing 8 (one tile spans several tokens) and multiples of 8."""
+    from bit_paged_kv_block_b200 import saw
+    T, hq = 203, 4 * hkv
+    g = torch.Generator().manual_seed(hkv + 10 * rotate)
+    qkv = (torch.randn(T, (hq + 2 * hkv) * 128, generator=g) * 3.0).to(torch.bfloat16)
+    k = qkv[:, hq * 128:(hq + hkv) * 128].view(T, hkv, 128)
+    v = qkv[:, (hq + hkv) * 128:].view(T, hkv, 128)
+    wl = synth.custom(f"qkv{hkv}", [T], num_q_heads=hq, num_kv_heads=hkv, new_tokens=[T],
+                      num_pages=(T + 15) // 16 + 2)
+    seq, pos = synth.token_index(wl)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(cuda_device)
+    kv, sc = canary_device_cache(wl, cuda_device)
+    qkv_d = qkv.to(cuda_device)
+    saw.saw_rotate_quantize_paged_strided(qkv_d[:, hq * 128:(hq + hkv) * 128].view(T, hkv, 128),
+                                          qkv_d[:, (hq + hkv) * 128:].view(T, hkv, 128), slots,
+                                          kv, sc, rotate=rotate)
+    torch.cuda.synchronize()
+    pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous(), rotate=rotate)
+    assert_cache_equal(kv, sc, pages, scales)
