@@ -77,6 +77,9 @@ def _load():
         lib.oracle_decode_fp64.argtypes = [P, P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
                                            i32, P, i32]
         lib.oracle_decode_fp64.restype = None
+        lib.oracle_prefill_fp64.argtypes = [P, P, P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
+                                            i32, P, i32]
+        lib.oracle_prefill_fp64.restype = None
         lib.oracle_append_bf16.argtypes = [P, P, P, i64, i32, i32, i32, i64, P]
         lib.oracle_append_bf16.restype = i64
         lib.oracle_decode_bf16_fp64.argtypes = [P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
@@ -215,6 +218,31 @@ def decode_fp64(q_bits, kv_pages, scales, block_table, seq_lens, *, sm_scale=Non
     _load().oracle_decode_fp64(_ptr(q_bits), _ptr(kv_pages), _ptr(scales), _ptr(block_table),
                                block_table.shape[1], _ptr(seq_lens), S, Hq, Hkv, D, page_size,
                                float(sm_scale), 1 if rotate else 0, _ptr(out), int(nthreads))
+    return out
+
+
+def prefill_fp64(q_bits, q_start, kv_pages, scales, block_table, seq_lens, *, sm_scale=None,
+                 rotate=True, nthreads=1) -> np.ndarray:
+    """fp64 chunked-prefill attention over the INT4 paged cache: the C_s = q_start[s + 1] -
+    q_start[s] queries of sequence s (rows q_start[s].. of q_bits [total][Hq][D]) are its last
+    C_s cached tokens, query i attending causally to tokens 0 .. seq_lens[s] - C_s + i.
+    Returns fp64 [total][Hq][D]."""
+    q_bits = _as(q_bits, np.uint16)
+    q_start = _as(q_start, np.int32)
+    block_table = _as(block_table, np.int32)
+    seq_lens = _as(seq_lens, np.int32)
+    total, Hq, D = q_bits.shape
+    S = seq_lens.shape[0]
+    num_pages, Hkv, _, page_size, half = kv_pages.shape
+    assert half * 2 == D and Hq % Hkv == 0 and q_start.shape == (S + 1,) and q_start[S] == total
+    assert np.all(np.diff(q_start) >= 0) and np.all(np.diff(q_start) <= seq_lens)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.zeros((total, Hq, D), dtype=np.float64)
+    _load().oracle_prefill_fp64(_ptr(q_bits), _ptr(q_start), _ptr(kv_pages), _ptr(scales),
+                                _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S, Hq,
+                                Hkv, D, page_size, float(sm_scale), 1 if rotate else 0, _ptr(out),
+                                int(nthreads))
     return out
 
 

@@ -387,3 +387,73 @@ void oracle_decode_bf16_fp64(const uint16_t *q, const uint16_t *kv_bf16,
         }
     }
 }
+
+/* ---- chunked-prefill attention over the INT4 cache ------------------------------------- */
+/*
+ * The read step for a chunk of new tokens whose K/V are already in the paged cache ("SAW-INT4",
+ * Research Findings: the quantized cache must serve attention over paged memory; a prefill
+ * chunk is the multi-query case).  Sequence s has C_s = q_start[s + 1] - q_start[s] query
+ * tokens, the last C_s of its seq_lens[s] cached tokens: query i (row q_start[s] + i of q / out)
+ * sits at position L - C + i and attends causally to cache tokens 0 .. L - C + i.  Rotation,
+ * dequantization and the fp64 evaluation are those of oracle_decode_fp64.
+ */
+void oracle_prefill_fp64(const uint16_t *q, const int32_t *q_start, const uint8_t *kv_pages,
+                         const uint16_t *scales, const int32_t *block_table, int max_blocks,
+                         const int32_t *seq_lens, int S, int Hq, int Hkv, int D, int page_size,
+                         double sm_scale, int rotate, double *out, int nthreads)
+{
+    const int G = Hq / Hkv;
+    const int64_t total = q_start[S];
+#pragma omp parallel for collapse(2) schedule(dynamic) num_threads(nthreads)
+    for (int64_t row = 0; row < total; row++) {
+        for (int hq = 0; hq < Hq; hq++) {
+            int s = 0;
+            while (q_start[s + 1] <= row)
+                s++;
+            const int C = q_start[s + 1] - q_start[s];
+            const int i = (int)(row - q_start[s]);
+            const int L = seq_lens[s] - C + i + 1;   /* tokens this query sees */
+            const int h = hq / G;
+            double qr[1024], kv[1024], o[1024];
+            double *dst = out + ((size_t)row * Hq + hq) * D;
+            for (int d = 0; d < D; d++)
+                qr[d] = (double)oracle_bf16_to_f32(q[((size_t)row * Hq + hq) * D + d]);
+            if (rotate)
+                oracle_rotate_f64(qr, D);
+            double m = -INFINITY;
+            for (int t = 0; t < L; t++) {
+                const int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 0,
+                                       t % page_size, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qr[d] * kv[d];
+                if (sm_scale * acc > m)
+                    m = sm_scale * acc;
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; d++)
+                o[d] = 0.0;
+            for (int t = 0; t < L; t++) {
+                const int64_t page = block_table[(size_t)s * max_blocks + t / page_size];
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 0,
+                                       t % page_size, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qr[d] * kv[d];
+                const double p = exp(sm_scale * acc - m);
+                l += p;
+                oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, 1,
+                                       t % page_size, kv);
+                for (int d = 0; d < D; d++)
+                    o[d] += p * kv[d];
+            }
+            for (int d = 0; d < D; d++)
+                o[d] /= l;
+            if (rotate)
+                oracle_rotate_f64(o, D);
+            for (int d = 0; d < D; d++)
+                dst[d] = o[d];
+        }
+    }
+}

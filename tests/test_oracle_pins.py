@@ -583,3 +583,49 @@ def test_bf16_decode_page_permutation_invariance():
     kv2[perm] = kv
     table2 = np.where(wl.block_table >= 0, perm[np.maximum(wl.block_table, 0)], -1).astype(np.int32)
     assert np.array_equal(oracle.decode_bf16_fp64(qb, kv2, table2, wl.seq_lens), base)
+
+
+# ---- chunked prefill over the INT4 cache ------------------------------------------------------
+
+def _prefill_case(lens, chunks, hq, hkv, seed):
+    wl = synth.custom(f"pf{seed}", lens, num_q_heads=hq, num_kv_heads=hkv, seed=seed,
+                      outlier_range=(10.0, 30.0))
+    _, _, pages, scales = _cache_for(wl)
+    q_start = np.concatenate([[0], np.cumsum(chunks)]).astype(np.int32)
+    g = torch.Generator().manual_seed(seed)
+    qb = synth.bf16_bits(torch.randn(int(q_start[-1]), hq, 128, generator=g).to(torch.bfloat16))
+    return wl, pages, scales, q_start, qb
+
+
+def test_prefill_matches_torch_causal_sdpa_fp64():
+    """Each chunk query against torch fp64 SDPA with an explicit causal mask, on the rotated
+    query (Sylvester matrix from scipy) and the dequantized (rotated-domain) cache, rotated
+    back."""
+    lens, chunks = [40, 17, 33], [7, 17, 1]
+    wl, pages, scales, q_start, qb = _prefill_case(lens, chunks, hq=4, hkv=2, seed=3)
+    got = oracle.prefill_fp64(qb, q_start, pages, scales, wl.block_table, wl.seq_lens)
+    H = torch.from_numpy(hadamard(128).astype(np.float64)) / np.sqrt(128.0)
+    q = torch.from_numpy(qb.astype(np.uint32) << 16).view(torch.float32).double()
+    for s, (L, C) in enumerate(zip(lens, chunks)):
+        for hq in range(4):
+            h = hq // 2
+            k = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 0))[:L]
+            v = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 1))[:L]
+            qr = q[q_start[s]:q_start[s + 1], hq] @ H
+            mask = torch.arange(L)[None, :] <= (L - C + torch.arange(C))[:, None]
+            o = torch.nn.functional.scaled_dot_product_attention(
+                qr[None, None], k[None, None], v[None, None], attn_mask=mask[None, None])[0, 0]
+            assert np.allclose(got[q_start[s]:q_start[s + 1], hq], (o @ H).numpy(), atol=1e-10)
+
+
+def test_prefill_rows_equal_decode_on_their_prefix():
+    """Query i of a chunk is a decode over the first L - C + i + 1 tokens."""
+    lens, chunks = [50, 20], [9, 20]
+    wl, pages, scales, q_start, qb = _prefill_case(lens, chunks, hq=8, hkv=2, seed=4)
+    got = oracle.prefill_fp64(qb, q_start, pages, scales, wl.block_table, wl.seq_lens)
+    for s, (L, C) in enumerate(zip(lens, chunks)):
+        for i in range(C):
+            row = q_start[s] + i
+            dec = oracle.decode_fp64(qb[row:row + 1], pages, scales, wl.block_table[s:s + 1],
+                                     np.array([L - C + i + 1], dtype=np.int32))
+            assert np.allclose(got[row], dec[0], atol=1e-12, rtol=1e-12)
