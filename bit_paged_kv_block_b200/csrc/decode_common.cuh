@@ -1,14 +1,21 @@
-// decode_common.cuh -- the parts of the paged decode kernels that do not depend on the page
-// format: the cost-balanced split of all (sequence, kv head) segments into warp runs, the
-// per-warp online-softmax state, split-K partial slots in the workspace and the merge kernel
-// that folds a split segment's partials in a fixed order.
+// decode_common.cuh -- the parts of the paged attention kernels that do not depend on the page
+// format: the cost-balanced split of all segments into warp runs, the per-warp online-softmax
+// state, split-K partial slots in the workspace, the kernel body (generic over the page format)
+// and the merge kernel that folds a split segment's partials in a fixed order.
 //
-// A segment (sequence s, kv head h, query sub-group: G > 8 query heads of one kv head are split
-// into ceil(G / 8) sub-groups, each its own segment reading the same pages, because the MMA
-// tiles stack at most 8 heads) of n = ceil(len_s / 16) pages costs n + kKappa in a cost
-// space where all segments lie end to end (sequence-major, then kv head); that range is cut
-// into equal slices, one per warp of a persistent grid, and a warp owns the pages whose cost
-// falls in its slice.  The pieces of a segment split across warps go to workspace slot
+// Queries.  Sequence s has C_s query tokens: C_s = 1 for decode (query row s), or
+// q_start[s + 1] - q_start[s] for chunked prefill (query rows q_start[s] ..), the last C_s of
+// its L_s cached tokens.  Query token i sees cache tokens 0 .. L_s - C_s + i (causal; decode:
+// all L_s).  A query row of kv head h is a (query token, query head of h) pair, token-major:
+// row r is token r / G, head h G + r % G.
+//
+// Segments.  The C_s G rows of (sequence s, kv head h) are cut into blocks of at most 8 rows
+// (the MMA tiles stack 8 query columns); a segment is (s, h, block) and reads all
+// n_s = ceil(L_s / 16) pages of s, the rows' causal limits masking what each may not see.
+// Segment j of sequence s is kv head j / nb_s, block j % nb_s.  A segment of n pages costs
+// n + kKappa in a cost space where all segments lie end to end (sequence-major); that range
+// is cut into equal slices, one per warp of a persistent grid, and a warp owns the pages whose
+// cost falls in its slice.  The pieces of a segment split across warps go to workspace slot
 // segment + warp (unique, because both orders are monotone).
 #pragma once
 
@@ -25,148 +32,187 @@ namespace decode {
 constexpr int kSlotFloats = 32 * 32 + 16;               // O (lane layout) + m[8] + l[8]
 constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
 constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
+constexpr int kRowsPerBlock = 8;                        // query rows (MMA columns) per segment
 constexpr int kMergeWarps = 4;
 constexpr int kMergeThreads = 32 * kMergeWarps;
-// merge kernel shared memory: per-warp partials, flags, then the sequence prefix
+// per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
+constexpr int kSeqTableBytes = 20;
+// merge kernel shared memory: per-warp partials, flags, then the sequence tables
 constexpr int kMergeSmemSlots = 0;
 constexpr int kMergeSmemFlags = kMergeSmemSlots + (kMergeWarps - 1) * kSlotFloats * 4;
-constexpr int kMergeSmemPrefix = kMergeSmemFlags + 64;
+constexpr int kMergeSmemTables = kMergeSmemFlags + 64;
 
+inline size_t seq_table_bytes(int32_t num_seqs)
+{
+    return kSeqTableBytes * (static_cast<size_t>(num_seqs) + 1);
+}
 inline size_t merge_smem_bytes(int32_t num_seqs)
 {
-    return kMergeSmemPrefix + 4 * (static_cast<size_t>(num_seqs) + 1);
+    return kMergeSmemTables + seq_table_bytes(num_seqs);
 }
 
-// Query sub-groups of G = hq / hkv query heads per kv head (see DecodeParams).
-struct SubGroups {
-    int32_t nsub, gsub, hseg;
-};
-inline SubGroups sub_groups(int32_t num_kv_heads, int32_t num_q_heads)
+// Segments of a launch: decode, num_seqs * hkv * ceil(G / 8); chunked prefill over total_q
+// query tokens, at most hkv * (ceil(total_q G / 8) + num_seqs).
+inline int64_t max_segments(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                            int64_t total_q, bool prefill)
+{
+    const int64_t G = num_q_heads / num_kv_heads;
+    if (!prefill)
+        return static_cast<int64_t>(num_seqs) * num_kv_heads * ((G + kRowsPerBlock - 1) / kRowsPerBlock);
+    return num_kv_heads * ((total_q * G + kRowsPerBlock - 1) / kRowsPerBlock + num_seqs);
+}
+
+// Rows of each warp's query buffer: a decode block holds at most G rows; a prefill block 8.
+inline int32_t query_rows(int32_t num_kv_heads, int32_t num_q_heads, bool prefill)
 {
     const int32_t G = num_q_heads / num_kv_heads;
-    const int32_t nsub = (G + 7) / 8;
-    return {nsub, (G + nsub - 1) / nsub, num_kv_heads * nsub};
+    return prefill || G >= kRowsPerBlock ? kRowsPerBlock : G;
 }
 
-// Workspace of a decode grid of `warps` warps over num_seqs * segs_per_seq segments.
-inline size_t workspace_bytes_for(size_t warps, int32_t num_seqs, int32_t segs_per_seq)
+// Workspace of a decode grid of `warps` warps over `segments` segments.
+inline size_t workspace_bytes_for(size_t warps, int64_t segments)
 {
-    return (warps + static_cast<size_t>(num_seqs) * segs_per_seq) * kSlotFloats * sizeof(float);
+    return (warps + static_cast<size_t>(segments)) * kSlotFloats * sizeof(float);
 }
 
 struct DecodeParams {
     const uint16_t *q;
+    const int32_t *q_start;      // chunked prefill: [S + 1] query-row offsets; decode: null
     const uint8_t *scales;       // INT4 cache: bytes, 128 B per (page, kv head); else unused
     const int32_t *block_table;
     const int32_t *seq_lens;
     float *out;
-    float *partials;             // workspace: (total warps + segments) slots
+    float *partials;             // workspace: (total warps + max_segments) slots
     uint32_t *status;
     int64_t num_pages;
+    int64_t max_segments;        // segment slots the workspace holds
     int32_t max_blocks;
     int32_t num_seqs;
     int32_t hq;
     int32_t hkv;
     int32_t group;               // G = hq / hkv
-    int32_t nsub;                // query sub-groups per kv head: ceil(G / 8) (MMA tiles are 8 wide)
-    int32_t gsub;                // query heads per sub-group: ceil(G / nsub) <= 8
-    int32_t hseg;                // segments per sequence: hkv * nsub
     int32_t total_warps;         // warps of the decode grid (the plan's slice count bound)
+    int32_t qrows;               // rows of each warp's query buffer: min(8, C G) bound
     float q_mult;                // the factor the kernel applies to q (or to the logits)
-
-    // Segment hv of a sequence is query sub-group hv % nsub of kv head hv / nsub.
-    __device__ int kv_head(int hv) const { return hv / nsub; }
-    __device__ int head_base(int hv) const { return (hv / nsub) * group + (hv % nsub) * gsub; }
-    __device__ int head_count(int hv) const { return min(gsub, group - (hv % nsub) * gsub); }
 };
 
-// ---- work plan ------------------------------------------------------------------------------
+// ---- per-sequence tables and the work plan -----------------------------------------------------
 
-// Largest s in [0, S) with hkv * pre[s] <= pos (pos < hkv * pre[S]).
-__device__ __forceinline__ int find_seq(const int32_t *pre, int S, int64_t pos, int64_t hkv)
-{
-    int lo = 0, hi = S;
-    while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (hkv * pre[mid] <= pos)
-            lo = mid;
-        else
-            hi = mid;
+// Shared-memory tables over the sequences: fpre[s] flat pages (segments x pages) before s,
+// spre[s] segments before s, npg[s] pages of each segment of s, nbk[s] row blocks per kv head.
+struct SeqTables {
+    int64_t *fpre;
+    int32_t *spre, *npg, *nbk;
+
+    __device__ void bind(uint8_t *base, int S)
+    {
+        fpre = reinterpret_cast<int64_t *>(base);
+        spre = reinterpret_cast<int32_t *>(base + 8 * (S + 1));
+        npg = spre + (S + 1);
+        nbk = npg + (S + 1);
     }
-    return lo;
+};
+
+// Query tokens of sequence s (decode: 1) and its first query row.  kPrefill: a chunked
+// prefill (q_start given); the decode instantiation has none of the per-row arithmetic.
+template <bool kPrefill>
+__device__ __forceinline__ int query_tokens(const DecodeParams &p, int s)
+{
+    return kPrefill ? p.q_start[s + 1] - p.q_start[s] : 1;
+}
+template <bool kPrefill>
+__device__ __forceinline__ int64_t query_row0(const DecodeParams &p, int s)
+{
+    return kPrefill ? p.q_start[s] : s;
 }
 
-// Pages per sequence (0 for an invalid length, which is flagged) and their exclusive prefix
-// pre[0..S] in shared memory; every thread of the block takes part.
-__device__ inline void scan_pages(const DecodeParams &p, int32_t *pre, volatile int32_t *flags,
-                                  bool report)
+// Fill the tables (every thread of the block takes part).  A sequence with an invalid length
+// or query count (C > L, or C > 0 with L = 0 in prefill) is flagged and gets no segments; a
+// decode sequence of length 0 gets none either (its output row is zeroed).
+template <bool kPrefill>
+__device__ inline void scan_sequences(const DecodeParams &p, const SeqTables &tb,
+                                      volatile int64_t *flags, bool report)
 {
     const int S = p.num_seqs, nthreads = blockDim.x, tid = threadIdx.x;
     const int lane = tid & 31, warp = tid >> 5;
     const int per = (S + nthreads - 1) / nthreads;
     const int s0 = tid * per, s1 = min(S, s0 + per);
-    int local = 0;
+    int64_t local_pages = 0;
+    int32_t local_segs = 0;
     for (int s = s0; s < s1; s++) {
         const int len = p.seq_lens[s];
-        const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
-        if (!ok && report)
+        const int c = query_tokens<kPrefill>(p, s);
+        const bool len_ok = len >= 0 && len <= p.max_blocks * kPageSize;
+        const bool q_ok = !kPrefill || (c >= 0 && c <= len);
+        if (report && !(len_ok && q_ok))
             set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
-        local += ok ? (len + kPageSize - 1) / kPageSize : 0;
+        const int n = (len_ok && q_ok) ? (len + kPageSize - 1) / kPageSize : 0;
+        const int nb = n > 0 ? (c * p.group + kRowsPerBlock - 1) / kRowsPerBlock : 0;
+        tb.npg[s] = n;
+        tb.nbk[s] = nb;
+        local_segs += p.hkv * nb;
+        local_pages += static_cast<int64_t>(p.hkv) * nb * n;
     }
-    int incl = local;
+    int64_t ip = local_pages;
+    int32_t is = local_segs;
 #pragma unroll
     for (int d = 1; d < 32; d <<= 1) {
-        const int o = __shfl_up_sync(0xFFFFFFFFu, incl, d);
-        if (lane >= d)
-            incl += o;
+        const int64_t op = __shfl_up_sync(0xFFFFFFFFu, ip, d);
+        const int32_t os = __shfl_up_sync(0xFFFFFFFFu, is, d);
+        if (lane >= d) {
+            ip += op;
+            is += os;
+        }
     }
-    if (lane == 31)
-        flags[warp] = incl;
+    if (lane == 31) {
+        flags[2 * warp] = ip;
+        flags[2 * warp + 1] = is;
+    }
     __syncthreads();
-    int base = 0;
-    for (int w = 0; w < warp; w++)
-        base += flags[w];
-    int run = base + incl - local;
-    for (int s = s0; s < s1; s++) {
-        pre[s] = run;
-        const int len = p.seq_lens[s];
-        const bool ok = len >= 0 && len <= p.max_blocks * kPageSize;
-        run += ok ? (len + kPageSize - 1) / kPageSize : 0;
+    int64_t bp = 0, bs = 0;
+    for (int w = 0; w < warp; w++) {
+        bp += flags[2 * w];
+        bs += flags[2 * w + 1];
     }
-    if (tid == nthreads - 1)
-        pre[S] = base + incl;
+    int64_t rp = bp + ip - local_pages;
+    int32_t rs = static_cast<int32_t>(bs + is - local_segs);
+    for (int s = s0; s < s1; s++) {
+        tb.fpre[s] = rp;
+        tb.spre[s] = rs;
+        rs += p.hkv * tb.nbk[s];
+        rp += static_cast<int64_t>(p.hkv) * tb.nbk[s] * tb.npg[s];
+    }
+    if (tid == nthreads - 1) {
+        tb.fpre[S] = bp + ip;
+        tb.spre[S] = static_cast<int32_t>(bs + is);
+    }
     __syncthreads();
 }
 
-// The cost-space split of the flat page range into warp runs.  Segment (s, h) spans the cost
-// range [seq_cost(s) + h (n_s + kKappa), + n_s + kKappa); its page i sits at cost
-// seq_cost(s) + h (n_s + kKappa) + kKappa + i.  Warp u owns the cost range
-// [b(u), b(u + 1)) with b(u) = u q + min(u, r), q = PT / W, r = PT % W (slices of q or q + 1,
-// never empty because W <= PT), i.e. the pages whose cost falls in it.
+// The cost-space split of the flat page range into warp runs.  Segment j of sequence s spans
+// the cost range [cpre(s) + j (n_s + kKappa), + n_s + kKappa) with cpre(s) = fpre[s] +
+// kKappa spre[s]; its page i sits at cost cpre(s) + j (n_s + kKappa) + kKappa + i.  Warp u owns
+// the cost range [b(u), b(u + 1)) with b(u) = u q + min(u, r), q = PT / W, r = PT % W (slices of
+// q or q + 1, never empty because W <= PT), i.e. the pages whose cost falls in it.
 struct Plan {
-    const int32_t *pre;
+    SeqTables tb;
     int S;
-    int64_t hkv;
     int64_t P;    // pages
     int64_t PT;   // cost
     int64_t W;    // warps with a slice
     int64_t q, r;
 
-    __device__ void init(const int32_t *pre_, int S_, int hkv_, int total_warps)
+    __device__ void init(const SeqTables &tb_, int S_, int total_warps)
     {
-        pre = pre_;
+        tb = tb_;
         S = S_;
-        hkv = hkv_;
-        P = hkv * pre[S];
-        PT = hkv * (static_cast<int64_t>(pre[S]) + kKappa * S);
+        P = tb.fpre[S];
+        PT = P + kKappa * tb.spre[S];
         W = max(int64_t(1), min(static_cast<int64_t>(total_warps), PT));
         q = PT / W;
         r = PT - q * W;
     }
-    __device__ int64_t seq_cost(int s) const
-    {
-        return hkv * (static_cast<int64_t>(pre[s]) + kKappa * s);
-    }
+    __device__ int64_t seq_cost(int s) const { return tb.fpre[s] + kKappa * tb.spre[s]; }
     __device__ int64_t slice_begin(int64_t u) const { return u * q + min(u, r); }
     // the warp whose cost slice holds cost position x (0 <= x < PT)
     __device__ int64_t warp_of_cost(int64_t x) const
@@ -174,10 +220,36 @@ struct Plan {
         const int64_t big = r * (q + 1);
         return x < big ? x / (q + 1) : r + (x - big) / q;
     }
-    // cost position of page i of segment (s, h)
-    __device__ int64_t page_cost(int s, int h, int64_t i) const
+    // cost position of page i of segment j of sequence s
+    __device__ int64_t page_cost(int s, int j, int64_t i) const
     {
-        return seq_cost(s) + static_cast<int64_t>(h) * (pre[s + 1] - pre[s] + kKappa) + kKappa + i;
+        return seq_cost(s) + static_cast<int64_t>(j) * (tb.npg[s] + kKappa) + kKappa + i;
+    }
+    // the sequence holding flat page pos (0 <= pos < P): the largest s with fpre[s] <= pos
+    __device__ int seq_of_flat(int64_t pos) const
+    {
+        int lo = 0, hi = S;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tb.fpre[mid] <= pos)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        return lo;
+    }
+    // the sequence holding global segment g: the largest s with spre[s] <= g
+    __device__ int seq_of_segment(int64_t g) const
+    {
+        int lo = 0, hi = S;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (tb.spre[mid] <= g)
+                lo = mid;
+            else
+                hi = mid;
+        }
+        return lo;
     }
     // first flat page whose cost position is >= x
     __device__ int64_t flat_of_cost(int64_t x) const
@@ -192,15 +264,86 @@ struct Plan {
             else
                 hi = mid;
         }
-        const int64_t n = pre[lo + 1] - pre[lo];
+        const int64_t n = tb.npg[lo];
         const int64_t within = x - seq_cost(lo);
-        const int64_t h = within / (n + kKappa);
-        const int64_t rr = within - h * (n + kKappa);
-        return hkv * pre[lo] + h * n + (rr < kKappa ? 0 : rr - kKappa);
+        const int64_t j = within / (n + kKappa);
+        const int64_t rr = within - j * (n + kKappa);
+        return tb.fpre[lo] + j * n + (rr < kKappa ? 0 : rr - kKappa);
     }
     // first flat page of warp u's run (u in [0, W]; the run of u is [begin(u), begin(u + 1)))
     __device__ int64_t begin(int64_t u) const { return flat_of_cost(slice_begin(u)); }
 };
+
+// One segment: sequence s, its segment j = kv head h * nb + row block b.
+template <bool kPrefill>
+struct Segment {
+    int s, j, h, b;
+    int n;          // pages
+    int c;          // query tokens of the sequence
+    int len;        // cached tokens of the sequence
+    int row0;       // first row of the block (8 b)
+    int nrows;      // rows in the block (1..8)
+    int64_t qrow0;  // first query row of the sequence in q / out
+
+    __device__ void init(const DecodeParams &p, const SeqTables &tb, int s_, int j_)
+    {
+        s = s_;
+        j = j_;
+        const int nb = tb.nbk[s];
+        h = nb == 1 ? j : j / nb;
+        b = j - h * nb;
+        n = tb.npg[s];
+        c = query_tokens<kPrefill>(p, s);
+        len = p.seq_lens[s];
+        row0 = kRowsPerBlock * b;
+        nrows = min(kRowsPerBlock, c * p.group - row0);
+        qrow0 = query_row0<kPrefill>(p, s);
+    }
+    // query token and head (within the kv head's group) of block row e; a decode has one
+    // token, so no division there
+    __device__ int row_token(const DecodeParams &p, int e) const
+    {
+        return kPrefill ? (row0 + e) / p.group : 0;
+    }
+    // causal limit of block row e (0..7): the last cache token it sees
+    __device__ int limit(const DecodeParams &p, int e) const
+    {
+        return len - c + row_token(p, e);
+    }
+    // q / out element offset of block row e (e < nrows)
+    __device__ int64_t row_offset(const DecodeParams &p, int e) const
+    {
+        const int tok = row_token(p, e);
+        const int head = row0 + e - tok * p.group;
+        return ((qrow0 + tok) * p.hq + h * p.group + head) * kHeadDim;
+    }
+    // pages from this index on hold a token some row of the block may not see (or past len)
+    __device__ int first_masked_page(const DecodeParams &p) const
+    {
+        return (limit(p, 0) + 1) / kPageSize;
+    }
+};
+
+// Validity of one page for the MMA columns a thread holds (block rows 2t and 2t + 1):
+// tokens [0, valid) of the page exist (the rest were never written), and column e sees
+// tokens [0, col[e]).
+struct PageMask {
+    int valid;
+    int col[2];
+};
+
+// The mask of segment page `page` for a thread whose columns see tokens up to lim[0], lim[1]
+// of a sequence of len tokens.
+__device__ __forceinline__ PageMask page_mask(int len, const int lim[2], int page)
+{
+    const int base = kPageSize * page;
+    PageMask m;
+    m.valid = min(kPageSize, max(0, len - base));
+#pragma unroll
+    for (int e = 0; e < 2; e++)
+        m.col[e] = min(m.valid, max(0, lim[e] - base + 1));
+    return m;
+}
 
 // Per-warp running state of one piece: o holds O^T (128 value rows x 8 stacked query heads) as
 // eight m16n8 accumulator tiles, thread (g, t) holding heads 2t and 2t + 1 of rows g and g + 8
@@ -228,11 +371,13 @@ __device__ __forceinline__ void state_reset(WarpState &st)
     }
 }
 
-// Online softmax over one page: s holds the logits (log2 domain) of tokens g, g + 8 for heads
+// Online softmax over one page: s holds the logits (log2 domain) of tokens g, g + 8 for columns
 // 2t, 2t + 1 (-inf for masked tokens); returns p = 2^(s - m) with m the running max after the
 // page, and rescales o, l and z when m grows.  The running max only changes when some logit of
 // the page exceeds it, so the cross-lane reduction runs only then (rare once a piece is a few
-// pages long); the result equals reducing every page.
+// pages long); the result equals reducing every page.  kMask: a column may have seen only
+// masked tokens so far (m = -inf); its p stay 0 and nothing is rescaled by a NaN.
+template <bool kMask>
 __device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, float pr[4])
 {
     const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
@@ -248,7 +393,7 @@ __device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, 
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const float mn = fmaxf(st.m[e], mx[e]);
-            alpha[e] = ex2_approx(st.m[e] - mn);
+            alpha[e] = mn == -INFINITY ? 1.0f : ex2_approx(st.m[e] - mn);
             st.m[e] = mn;
             st.l[e] *= alpha[e];
             st.z[e] *= alpha[e];
@@ -265,6 +410,11 @@ __device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, 
     pr[1] = ex2_approx(s[1] - st.m[1]);
     pr[2] = ex2_approx(s[2] - st.m[0]);
     pr[3] = ex2_approx(s[3] - st.m[1]);
+    if (kMask) {
+#pragma unroll
+        for (int k = 0; k < 4; k++)
+            pr[k] = s[k] == -INFINITY ? 0.0f : pr[k];
+    }
 }
 
 // Fold (m, l, o) partial b (scaled by its own max) into the running partial a.
@@ -320,36 +470,35 @@ __device__ __forceinline__ void load_partial(const float *slot, int lane, float 
     bl[1] = slot[1032 + 2 * t + 1];
 }
 
-// Combine the pieces of every segment that was split across warps: slot segment + u holds
-// warp u's (m, l, o); the warps of a block fold disjoint subsets in a fixed order, then warp 0
-// folds the other warps' results in warp order and writes the output through the page format's
-// finalize step, so the result does not depend on timing.
-template <class Fmt>
+// Combine the pieces of every segment that was split across warps: slot g + u holds warp u's
+// (m, l, o) for global segment g; the warps of a block fold disjoint subsets in a fixed order,
+// then warp 0 folds the other warps' results in warp order and writes the output through the
+// page format's finalize step, so the result does not depend on timing.
+template <class Fmt, bool kPrefill>
 __global__ void __launch_bounds__(kMergeThreads)
     paged_decode_merge_kernel(const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    int32_t *pre = reinterpret_cast<int32_t *>(smem + kMergeSmemPrefix);
-    volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + kMergeSmemFlags);
+    SeqTables tb;
+    tb.bind(smem + kMergeSmemTables, p.num_seqs);
+    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + kMergeSmemFlags);
     float *slots = reinterpret_cast<float *>(smem + kMergeSmemSlots);
 
-    scan_pages(p, pre, flags, false);
+    scan_sequences<kPrefill>(p, tb, flags, false);
     Plan plan;
-    plan.init(pre, p.num_seqs, p.hseg, p.total_warps);
+    plan.init(tb, p.num_seqs, p.total_warps);
     pdl_wait();   // the decode kernel's partials
-    if (plan.P == 0)
+    if (plan.P == 0 || tb.spre[p.num_seqs] > p.max_segments)
         return;
-    const int64_t hkv = p.hseg;
-    const int64_t J = static_cast<int64_t>(p.num_seqs) * hkv;
-    for (int64_t seg = blockIdx.x; seg < J; seg += gridDim.x) {
-        const int s = static_cast<int>(seg / hkv), h = static_cast<int>(seg - s * hkv);
-        const int32_t n_s = pre[s + 1] - pre[s];
-        if (n_s == 0)
-            continue;
-        const int64_t u_lo = plan.warp_of_cost(plan.page_cost(s, h, 0));
-        const int64_t u_hi = plan.warp_of_cost(plan.page_cost(s, h, n_s - 1));
+    const int64_t J = tb.spre[p.num_seqs];
+    for (int64_t gseg = blockIdx.x; gseg < J; gseg += gridDim.x) {
+        const int s = plan.seq_of_segment(gseg);
+        const int j = static_cast<int>(gseg - tb.spre[s]);
+        const int32_t n_s = tb.npg[s];
+        const int64_t u_lo = plan.warp_of_cost(plan.page_cost(s, j, 0));
+        const int64_t u_hi = plan.warp_of_cost(plan.page_cost(s, j, n_s - 1));
         if (u_lo == u_hi)
             continue;
         WarpState st;
@@ -359,15 +508,15 @@ __global__ void __launch_bounds__(kMergeThreads)
         for (; uu + kMergeWarps <= u_hi; uu += 2 * kMergeWarps) {
             float bm0[2], bl0[2], bm1[2], bl1[2];
             float4 bo0[8], bo1[8];
-            load_partial(p.partials + (seg + uu) * kSlotFloats, lane, bm0, bl0, bo0);
-            load_partial(p.partials + (seg + uu + kMergeWarps) * kSlotFloats, lane, bm1, bl1, bo1);
+            load_partial(p.partials + (gseg + uu) * kSlotFloats, lane, bm0, bl0, bo0);
+            load_partial(p.partials + (gseg + uu + kMergeWarps) * kSlotFloats, lane, bm1, bl1, bo1);
             merge_into(st.m, st.l, st.o, bm0, bl0, bo0);
             merge_into(st.m, st.l, st.o, bm1, bl1, bo1);
         }
         if (uu <= u_hi) {
             float bm[2], bl[2];
             float4 bo[8];
-            load_partial(p.partials + (seg + uu) * kSlotFloats, lane, bm, bl, bo);
+            load_partial(p.partials + (gseg + uu) * kSlotFloats, lane, bm, bl, bo);
             merge_into(st.m, st.l, st.o, bm, bl, bo);
         }
         if (warp > 0)
@@ -380,13 +529,15 @@ __global__ void __launch_bounds__(kMergeThreads)
                 load_partial(slots + (w - 1) * kSlotFloats, lane, bm, bl, bo);
                 merge_into(st.m, st.l, st.o, bm, bl, bo);
             }
-            Fmt::finalize(p, s, h, lane, st.o, st.l);
+            Segment<kPrefill> sg;
+            sg.init(p, tb, s, j);
+            Fmt::finalize(p, sg, lane, st.o, st.l);
         }
         __syncthreads();
     }
 }
 
-// ---- the decode kernel, generic over the page format ----------------------------------------
+// ---- the attention kernel, generic over the page format --------------------------------------
 //
 // A page format Fmt supplies:
 //   kWarps, kStages (a power of two), kMinBlocks   warps per CTA, ring stages per warp, and the
@@ -397,18 +548,19 @@ __global__ void __launch_bounds__(kMergeThreads)
 //   Ring ring(base, warp)                          this warp's stage addresses;
 //   issue(ring, stg, bar, tmap, row, p)            queue a page's copies into stage stg,
 //                                                  completing on mbarrier bar (one elected lane);
-//   Query; load_query(p, qbuf, n, lane, q)         per-piece query fragments from the raw bf16
-//                                                  queries of the segment's n <= 8 heads in
-//                                                  shared memory;
-//   page<kMask>(ring, stg, valid, q, lane, st)     attend over one staged page (first `valid`
-//                                                  tokens when kMask);
+//   Query; load_query(p, qbuf, n, lane, q)         per-piece query fragments from the n <= 8
+//                                                  raw bf16 query rows in shared memory;
+//   page<kMask>(ring, stg, mask, q, lane, st)      attend over one staged page (PageMask when
+//                                                  kMask: never-written tokens, causal limits);
 //   piece_end(st)                                  reductions and corrections after a piece;
-//   finalize(p, s, hv, lane, o, l)                 write the output of segment hv of sequence s
+//   finalize(p, segment, lane, o, l)               write a finished segment's output rows (a
+//                                                  template on the segment type)
 //                                                  (also the merge kernel's output step).
-// Shared memory: rings, then per warp (kStages + 1) mbarriers (the last for the query), 64 bytes
-// of flags, the per-warp query buffers (G * 256 bytes each) and the sequence page prefix.
+// Shared memory: rings, then per warp (kStages + 1) mbarriers (the last for the query), 128 bytes
+// of flags, the per-warp query buffers (qrows * 256 bytes each) and the sequence tables.
 
-__host__ __device__ constexpr int query_bytes(int group) { return group * kHeadDim * 2; }
+constexpr int kSmemFlagBytes = 128;
+__host__ __device__ constexpr int query_bytes(int rows) { return rows * kHeadDim * 2; }
 template <class Fmt>
 __host__ __device__ constexpr int smem_bars_offset() { return Fmt::kRingBytes; }
 template <class Fmt>
@@ -417,19 +569,19 @@ __host__ __device__ constexpr int smem_flags_offset()
     return Fmt::kRingBytes + Fmt::kWarps * (Fmt::kStages + 1) * 8;
 }
 template <class Fmt>
-__host__ __device__ constexpr int smem_q_offset() { return smem_flags_offset<Fmt>() + 64; }
+__host__ __device__ constexpr int smem_q_offset() { return smem_flags_offset<Fmt>() + kSmemFlagBytes; }
 template <class Fmt>
-__host__ __device__ constexpr int smem_prefix_offset(int group)
+__host__ __device__ constexpr int smem_tables_offset(int qrows)
 {
-    return smem_q_offset<Fmt>() + Fmt::kWarps * query_bytes(group);
+    return smem_q_offset<Fmt>() + Fmt::kWarps * query_bytes(qrows);
 }
 template <class Fmt>
-inline size_t decode_smem_bytes(int32_t num_seqs, int32_t group)
+inline size_t decode_smem_bytes(int32_t num_seqs, int32_t qrows)
 {
-    return 1024 + smem_prefix_offset<Fmt>(group) + 4 * (static_cast<size_t>(num_seqs) + 1);
+    return 1024 + smem_tables_offset<Fmt>(qrows) + seq_table_bytes(num_seqs);
 }
 
-template <class Fmt>
+template <class Fmt, bool kPrefill>
 __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
 {
@@ -437,21 +589,28 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
     const int S = p.num_seqs;
-    int32_t *pre = reinterpret_cast<int32_t *>(smem + smem_prefix_offset<Fmt>(p.gsub));
-    volatile int32_t *flags = reinterpret_cast<volatile int32_t *>(smem + smem_flags_offset<Fmt>());
+    SeqTables tb;
+    tb.bind(smem + smem_tables_offset<Fmt>(p.qrows), S);
+    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + smem_flags_offset<Fmt>());
 
-    // ---- 1. pages per sequence, the plan, zero outputs of empty sequences ------------------
-    scan_pages(p, pre, flags, blockIdx.x == 0);
+    // ---- 1. sequence tables, the plan, zero the output rows that get no segment ----------------
+    scan_sequences<kPrefill>(p, tb, flags, blockIdx.x == 0);
     pdl_launch_dependents();   // the merge kernel may start its own prologue
     for (int s = blockIdx.x; s < S; s += gridDim.x) {
-        if (pre[s + 1] == pre[s]) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out + static_cast<int64_t>(s) * p.hq * kHeadDim);
-            for (int i = tid; i < p.hq * kHeadDim / 4; i += 32 * Fmt::kWarps)
+        const int c = query_tokens<kPrefill>(p, s);
+        if (tb.nbk[s] == 0 && c > 0 && (!kPrefill || c <= p.seq_lens[s])) {
+            float4 *dst = reinterpret_cast<float4 *>(p.out + query_row0<kPrefill>(p, s) * p.hq * kHeadDim);
+            for (int i = tid; i < c * p.hq * kHeadDim / 4; i += 32 * Fmt::kWarps)
                 dst[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
     }
+    if (tb.spre[S] > p.max_segments) {   // more query rows than the workspace was sized for
+        if (blockIdx.x == 0 && tid == 0)
+            set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
+        return;
+    }
     Plan plan;
-    plan.init(pre, S, p.hseg, p.total_warps);
+    plan.init(tb, S, p.total_warps);
     const int64_t u = static_cast<int64_t>(blockIdx.x) * Fmt::kWarps + warp;
     if (plan.P == 0 || u >= plan.W)
         return;
@@ -459,12 +618,11 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     if (F0 >= F1)
         return;
     const int n_w = static_cast<int>(F1 - F0);
-    const int64_t hkv = p.hseg;   // segments per sequence
 
     // ---- 2. this warp's copy ring ---------------------------------------------------------------
     constexpr int kStages = Fmt::kStages;
     const typename Fmt::Ring ring = Fmt::ring(smem_u32(smem), warp);
-    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes(p.gsub);
+    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes(p.qrows);
     const uint32_t bar0 = smem_u32(smem + smem_bars_offset<Fmt>()) + warp * (kStages + 1) * 8;
     const uint32_t qbar = bar0 + kStages * 8;
     if (lane == 0)
@@ -478,25 +636,32 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         if (m >= n_w)
             return 0;
         const int64_t pos = F0 + m;
-        const int s = find_seq(pre, S, pos, hkv);
-        const int32_t n_s = pre[s + 1] - pre[s];
-        const int64_t rel = pos - hkv * pre[s];
-        const int h = static_cast<int>(rel / n_s);
-        const int i = static_cast<int>(rel - static_cast<int64_t>(h) * n_s);
+        const int s = plan.seq_of_flat(pos);
+        const int32_t n_s = tb.npg[s];
+        const int64_t rel = pos - tb.fpre[s];
+        const int j = static_cast<int>(rel / n_s);
+        const int i = static_cast<int>(rel - static_cast<int64_t>(j) * n_s);
+        const int nb = tb.nbk[s];
+        const int h = nb == 1 ? j : j / nb;
         int32_t page = p.block_table[static_cast<int64_t>(s) * p.max_blocks + i];
         if (page < 0 || page >= p.num_pages) {
             set_status(p.status, SAW_DEV_BAD_PAGE);
             page = 0;
         }
-        return (page * p.hkv + p.kv_head(h)) * Fmt::kRowsPerPage;
+        return (page * p.hkv + h) * Fmt::kRowsPerPage;
     };
-    // queue the raw queries of (s, h) into the warp's query buffer
-    auto issue_query = [&](int s, int h) {
+    // queue a segment's raw query rows into the warp's query buffer: one bulk copy per run of
+    // rows of the same query token (its heads are contiguous)
+    auto issue_query = [&](const Segment<kPrefill> &sg) {
         if (lane == 0) {
-            const uint32_t bytes = static_cast<uint32_t>(p.head_count(h)) * kHeadDim * 2;
-            mbar_arrive_expect_tx(qbar, bytes);
-            bulk_g2s(qbuf, p.q + (static_cast<int64_t>(s) * p.hq + p.head_base(h)) * kHeadDim,
-                     bytes, qbar);
+            mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(sg.nrows) * kHeadDim * 2);
+            for (int e = 0; e < sg.nrows;) {
+                const int head = sg.row0 + e - sg.row_token(p, e) * p.group;
+                const int cnt = min(p.group - head, sg.nrows - e);
+                bulk_g2s(qbuf + e * kHeadDim * 2, p.q + sg.row_offset(p, e),
+                         static_cast<uint32_t>(cnt) * kHeadDim * 2, qbar);
+                e += cnt;
+            }
         }
     };
 
@@ -523,25 +688,30 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         Fmt::issue(ring, stg, bar0 + 8 * stg, &tmap, row, p);
     };
 
-    // first piece's segment and its query
-    int s = find_seq(pre, S, F0, hkv);
-    int h = static_cast<int>((F0 - hkv * pre[s]) / (pre[s + 1] - pre[s]));
-    issue_query(s, h);
+    // first piece's segment and its query; across pieces only (sequence, segment index) of the
+    // current and next segments stay live, the rest is rebuilt where needed
+    int cs = plan.seq_of_flat(F0);
+    int cj = static_cast<int>((F0 - tb.fpre[cs]) / tb.npg[cs]);
+    {
+        Segment<kPrefill> sg;
+        sg.init(p, tb, cs, cj);
+        issue_query(sg);
+    }
     while (issued < kStages - 1 && issued < n_w)
         issue_next();
 
     WarpState st;
     typename Fmt::Query qf;
     // Page m of the run: queue the page kStages - 1 ahead into the stage page m - 1 used, wait
-    // for page m and attend over its first `valid` tokens (kMask) or all of them.
-    auto step = [&](auto mask_tag, int m, int valid) {
+    // for page m and attend over it (through `mask` when kMask).
+    auto step = [&](auto mask_tag, int m, const PageMask &mask) {
         if (issued < n_w && !aborted)
             issue_next();
         const int stg = m & (kStages - 1);
         const uint32_t phase = (static_cast<uint32_t>(m) / kStages) & 1u;
         const bool ok = !aborted && mbar_wait_bounded(bar0 + 8 * stg, phase, kWaitLimitNs);
         if (__all_sync(0xFFFFFFFFu, ok)) {
-            Fmt::template page<decltype(mask_tag)::value>(ring, stg, valid, qf, lane, st);
+            Fmt::template page<decltype(mask_tag)::value>(ring, stg, mask, qf, lane, st);
         } else if (!aborted) {
             if (lane == 0)
                 set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
@@ -555,12 +725,23 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     int m = 0;
     uint32_t qphase = 0;
     int64_t pos = F0;
+    const int t4 = lane & 3;
     while (pos < F1) {
-        const int32_t n_s = pre[s + 1] - pre[s];
-        const int64_t seg_start = hkv * pre[s] + static_cast<int64_t>(h) * n_s;
+        const int n_s = tb.npg[cs];
+        const int64_t seg_start = tb.fpre[cs] + static_cast<int64_t>(cj) * n_s;
         const int64_t seg_end = seg_start + n_s;
         const bool ends_segment = seg_end <= F1;
         const int m_end = static_cast<int>((ends_segment ? seg_end : F1) - F0);
+        int len, lim[2], first_masked, nrows;
+        {
+            Segment<kPrefill> sg;
+            sg.init(p, tb, cs, cj);
+            len = sg.len;
+            lim[0] = sg.limit(p, 2 * t4);
+            lim[1] = sg.limit(p, 2 * t4 + 1);
+            first_masked = sg.first_masked_page(p);
+            nrows = sg.nrows;
+        }
 
         // this piece's query: wait for its copy, build the fragments, then queue the next one
         const bool qok = !aborted && mbar_wait_bounded(qbar, qphase, kWaitLimitNs);
@@ -571,40 +752,46 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
             aborted = true;
         }
         qphase ^= 1;
-        Fmt::load_query(p, qbuf, p.head_count(h), lane, qf);
+        Fmt::load_query(p, qbuf, nrows, lane, qf);
         __syncwarp();
-        int s_next = s, h_next = h;
+        int ns = cs, nj = cj;
         if (m_end < n_w) {
-            if (++h_next == p.hseg) {
-                h_next = 0;
+            if (cj + 1 < p.hkv * tb.nbk[cs]) {
+                nj = cj + 1;
+            } else {
                 do {
-                    s_next++;
-                } while (pre[s_next + 1] == pre[s_next]);
+                    ns++;
+                } while (tb.spre[ns + 1] == tb.spre[ns]);
+                nj = 0;
             }
-            if (!aborted)
-                issue_query(s_next, h_next);
+            if (!aborted) {
+                Segment<kPrefill> nx;
+                nx.init(p, tb, ns, nj);
+                issue_query(nx);
+            }
         }
 
-        // all pages but a segment's last are full
+        // pages before the block's first limit are whole for every row; the rest are masked
         state_reset(st);
-        const int m_full = ends_segment ? m_end - 1 : m_end;
+        const int i0 = static_cast<int>(pos - seg_start) - m;   // page index of run page m
+        const int m_full = min(m_end, max(m, first_masked - i0));
+        const PageMask whole = {kPageSize, {kPageSize, kPageSize}};
         for (; m < m_full; m++)
-            step(std::false_type(), m, kPageSize);
-        if (ends_segment) {
-            step(std::true_type(), m, p.seq_lens[s] - kPageSize * (n_s - 1));
-            m++;
-        }
+            step(std::false_type(), m, whole);
+        for (; m < m_end; m++)
+            step(std::true_type(), m, page_mask(len, lim, i0 + m));
 
         Fmt::piece_end(st);
         if (seg_start >= F0 && ends_segment) {
-            Fmt::finalize(p, s, h, lane, st.o, st.l);
+            Segment<kPrefill> sg;
+            sg.init(p, tb, cs, cj);
+            Fmt::finalize(p, sg, lane, st.o, st.l);
         } else {
-            const int64_t seg = static_cast<int64_t>(s) * hkv + h;
-            store_partial(p.partials + (seg + u) * kSlotFloats, lane, st);
+            store_partial(p.partials + (tb.spre[cs] + cj + u) * kSlotFloats, lane, st);
         }
         pos = F0 + m_end;
-        s = s_next;
-        h = h_next;
+        cs = ns;
+        cj = nj;
     }
 
     // ---- 4. after an abort, let queued copies land before the shared memory is released ----
@@ -616,13 +803,15 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     }
 }
 
+constexpr int kShapeVariants = 4;
+
 struct LaunchShape {
     int sms = 0;
     int occ = 0;
 };
 
-// Multiprocessor count and occupancy of one family of decode kernels (both variants of the
-// decode and of its merge kernel) for the current device and dynamic shared-memory sizes.  The
+// Multiprocessor count and occupancy of one family of decode kernels (the kShapeVariants
+// instantiations of the decode and of its merge kernel: rotation x decode / prefill) for the current device and dynamic shared-memory sizes.  The
 // shared-memory attributes are raised per device as needed; everything is cached per device
 // in `cache`.
 struct ShapeCache {
@@ -637,9 +826,9 @@ struct ShapeCache {
     Dev dev[kMaxDevices];
 };
 
-inline cudaError_t launch_shape(ShapeCache &cache, const void *const decode_kernels[2],
-                                const void *const merge_kernels[2], int threads, size_t smem,
-                                size_t merge_smem, LaunchShape &out)
+inline cudaError_t launch_shape(ShapeCache &cache, const void *const decode_kernels[kShapeVariants],
+                                const void *const merge_kernels[kShapeVariants], int threads,
+                                size_t smem, size_t merge_smem, LaunchShape &out)
 {
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
@@ -652,7 +841,7 @@ inline cudaError_t launch_shape(ShapeCache &cache, const void *const decode_kern
     if (d.sms == 0 && (e = cudaDeviceGetAttribute(&d.sms, cudaDevAttrMultiProcessorCount, dev)) != cudaSuccess)
         return e;
     if (smem > d.decode_attr) {
-        for (int r = 0; r < 2 && e == cudaSuccess; r++)
+        for (int r = 0; r < kShapeVariants && e == cudaSuccess; r++)
             e = cudaFuncSetAttribute(decode_kernels[r], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(smem));
         if (e != cudaSuccess)
@@ -660,7 +849,7 @@ inline cudaError_t launch_shape(ShapeCache &cache, const void *const decode_kern
         d.decode_attr = smem;
     }
     if (merge_smem > d.merge_attr) {
-        for (int r = 0; r < 2 && e == cudaSuccess; r++)
+        for (int r = 0; r < kShapeVariants && e == cudaSuccess; r++)
             e = cudaFuncSetAttribute(merge_kernels[r], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(merge_smem));
         if (e != cudaSuccess)

@@ -142,10 +142,11 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
     sq_out[1] = __shfl_sync(0xFFFFFFFFu, sq, 8 * t + 4);
 }
 
-// One page of one warp: QK^T, online softmax, PV.  kMask: the page is the last of its
-// segment and only its first `valid` tokens exist.
+// One page of one warp: QK^T, online softmax, PV.  kMask: tokens [0, mask.valid) of the page
+// exist (the rest were never written: their V scale and zero are replaced by 0) and column e
+// (block row 2t + e) sees tokens [0, mask.col[e]).
 template <bool kMask>
-__device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int valid,
+__device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, const PageMask &mask,
                                              const uint32_t bq[8][2], const float sq[2],
                                              int lane, WarpState &st)
 {
@@ -169,7 +170,7 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
     }
 
     // ---- logits (log2 domain) ---------------------------------------------------------------
-    const bool v0 = !kMask || g < valid, v1 = !kMask || g + 8 < valid;
+    const bool v0 = !kMask || g < mask.valid, v1 = !kMask || g + 8 < mask.valid;
     const float2 ksz0 = h2_to_f2(lds32(sbase + 4 * g));
     const float2 ksz1 = h2_to_f2(lds32(sbase + 4 * (g + 8)));
     const float ks0 = ksz0.x * kLowNibble, ks1 = ksz1.x * kLowNibble;
@@ -179,14 +180,18 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
     s[2] = fmaf(ks1, acc[2], ksz1.y * sq[0]);
     s[3] = fmaf(ks1, acc[3], ksz1.y * sq[1]);
     if (kMask) {
-        if (!v0)
-            s[0] = s[1] = -INFINITY;
-        if (!v1)
-            s[2] = s[3] = -INFINITY;
+        if (g >= mask.col[0])
+            s[0] = -INFINITY;
+        if (g >= mask.col[1])
+            s[1] = -INFINITY;
+        if (g + 8 >= mask.col[0])
+            s[2] = -INFINITY;
+        if (g + 8 >= mask.col[1])
+            s[3] = -INFINITY;
     }
 
     float pr[4];
-    softmax_update(s, st, pr);
+    softmax_update<kMask>(s, st, pr);
 
     // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
     float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));
@@ -235,10 +240,10 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, int
 }
 
 
-// o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the heads this thread
-// holds; written to out[s][head_base(hv) + 2t + e].
-template <bool kRotate>
-__device__ __forceinline__ void finalize(const DecodeParams &p, int s, int hv, int lane,
+// o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the block rows 2t, 2t + 1
+// this thread holds.
+template <bool kRotate, class Seg>
+__device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, int lane,
                                          float o[8][4], const float l[2])
 {
     const int g = lane >> 2, t = lane & 3;
@@ -295,8 +300,8 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, int s, int hv, i
 #pragma unroll
     for (int e = 0; e < 2; e++) {
         const int head = 2 * t + e;
-        if (head < p.head_count(hv)) {
-            float *dst = p.out + ((static_cast<int64_t>(s) * p.hq + p.head_base(hv) + head) * kHeadDim);
+        if (head < sg.nrows) {
+            float *dst = p.out + sg.row_offset(p, head);
 #pragma unroll
             for (int c = 0; c < 4; c++) {
                 const float f = kRotate ? kHadamardC : 1.0f;
@@ -364,10 +369,10 @@ struct Int4Format {
         saw::load_query<kRotate>(p, qbuf, nheads, lane >> 2, lane & 3, q.bq, q.sq);
     }
     template <bool kMask>
-    __device__ static void page(const Ring &r, int stg, int valid, const Query &q, int lane,
-                                WarpState &st)
+    __device__ static void page(const Ring &r, int stg, const PageMask &mask, const Query &q,
+                                int lane, WarpState &st)
     {
-        process_page<kMask>(r.code0 + stg * kCodeBytes, r.scale0 + stg * kScaleBytes, valid, q.bq,
+        process_page<kMask>(r.code0 + stg * kCodeBytes, r.scale0 + stg * kScaleBytes, mask, q.bq,
                             q.sq, lane, st);
     }
     __device__ static void piece_end(WarpState &st)
@@ -391,10 +396,11 @@ struct Int4Format {
             st.o[i2][3] = fmaf(st.o[i2][3], kHighNibble, st.z[1]);
         }
     }
-    __device__ static void finalize(const DecodeParams &p, int s, int hv, int lane, float o[8][4],
+    template <class Seg>
+    __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane, float o[8][4],
                                     const float l[2])
     {
-        saw::finalize<kRotate>(p, s, hv, lane, o, l);
+        saw::finalize<kRotate>(p, sg, lane, o, l);
     }
 };
 
@@ -404,29 +410,34 @@ ShapeCache g_shapes;
 // decode::launch_shape).
 cudaError_t launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
 {
-    static const void *const decode_kernels[2] = {
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true>>),
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false>>)};
-    static const void *const merge_kernels[2] = {
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true>>),
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false>>)};
-    return decode::launch_shape(g_shapes, decode_kernels, merge_kernels, 32 * Int4Format<true>::kWarps, smem, merge_smem,
-                                  out);
+    static const void *const decode_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true>, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false>, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true>, true>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false>, true>)};
+    static const void *const merge_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true>, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false>, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true>, true>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false>, true>)};
+    return decode::launch_shape(g_shapes, decode_kernels, merge_kernels,
+                                32 * Int4Format<true>::kWarps, smem, merge_smem, out);
 }
 
 }  // namespace
 
-size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs)
+size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                              int64_t total_q)
 {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
+    const bool prefill = total_q >= 0;
     LaunchShape ls;
-    const SubGroups sg = sub_groups(num_kv_heads, num_q_heads);
-    if (launch_shape(decode_smem_bytes<Int4Format<true>>(num_seqs, sg.gsub),
+    if (launch_shape(decode_smem_bytes<Int4Format<true>>(num_seqs, query_rows(num_kv_heads, num_q_heads, prefill)),
                      merge_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
     return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Int4Format<true>::kWarps,
-                               num_seqs, sg.hseg);
+                               max_segments(num_kv_heads, num_q_heads, num_seqs, total_q, prefill));
 }
 
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
@@ -458,8 +469,9 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     }
 
     using Fmt = Int4Format<true>;   // the layout is the same for both variants
-    const SubGroups sg = sub_groups(a.num_kv_heads, a.num_q_heads);
-    const size_t smem = decode_smem_bytes<Fmt>(a.num_seqs, sg.gsub);
+    const bool prefill = a.q_start != nullptr;
+    const int32_t qrows = query_rows(a.num_kv_heads, a.num_q_heads, prefill);
+    const size_t smem = decode_smem_bytes<Fmt>(a.num_seqs, qrows);
     const size_t msmem = merge_smem_bytes(a.num_seqs);
     LaunchShape ls;
     cudaError_t e = launch_shape(smem, msmem, ls);
@@ -468,6 +480,7 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
 
     DecodeParams p;
     p.q = static_cast<const uint16_t *>(a.q);
+    p.q_start = a.q_start;
     p.scales = static_cast<const uint8_t *>(a.scales);
     p.block_table = a.block_table;
     p.seq_lens = a.seq_lens;
@@ -480,9 +493,8 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     p.hq = a.num_q_heads;
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
-    p.nsub = sg.nsub;
-    p.gsub = sg.gsub;
-    p.hseg = sg.hseg;
+    p.qrows = qrows;
+    p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Fmt::kWarps;
     // q carries sm_scale * log2(e), and 1/sqrt(128) of the (unnormalised) query butterfly
     p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(kHadamardC) : 1.0) * a.sm_scale *
@@ -499,19 +511,25 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, a.rotate ? paged_decode_kernel<Int4Format<true>> : paged_decode_kernel<Int4Format<false>>,
-                           cache.map, p);
+    auto *kernel = a.rotate ? (prefill ? paged_decode_kernel<Int4Format<true>, true>
+                                       : paged_decode_kernel<Int4Format<true>, false>)
+                            : (prefill ? paged_decode_kernel<Int4Format<false>, true>
+                                       : paged_decode_kernel<Int4Format<false>, false>);
+    e = cudaLaunchKernelEx(&cfg, kernel, cache.map, p);
     if (e != cudaSuccess)
         return e;
 
-    const int64_t segs = static_cast<int64_t>(a.num_seqs) * p.hseg;
+    const int64_t segs = p.max_segments;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&mcfg, a.rotate ? paged_decode_merge_kernel<Int4Format<true>>
-                                     : paged_decode_merge_kernel<Int4Format<false>>, p);
+    auto *merge = a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true>, true>
+                                      : paged_decode_merge_kernel<Int4Format<true>, false>)
+                           : (prefill ? paged_decode_merge_kernel<Int4Format<false>, true>
+                                      : paged_decode_merge_kernel<Int4Format<false>, false>);
+    e = cudaLaunchKernelEx(&mcfg, merge, p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();

@@ -98,8 +98,8 @@ struct Bf16Format {
     }
 
     template <bool kMask>
-    __device__ static void page(const Ring &r, int stg, int valid, const Query &q, int lane,
-                                WarpState &st)
+    __device__ static void page(const Ring &r, int stg, const PageMask &mask, const Query &q,
+                                int lane, WarpState &st)
     {
         const uint32_t base = r.base + stg * kBf16PageBytes;
         const int g = lane >> 2, t = lane & 3;
@@ -115,15 +115,18 @@ struct Bf16Format {
             mma_16816_bf16(acc, a, q.bq[i][0], q.bq[i][1]);
         }
         float s[4] = {acc[0] * q.mult, acc[1] * q.mult, acc[2] * q.mult, acc[3] * q.mult};
-        const bool v0 = !kMask || g < valid, v1 = !kMask || g + 8 < valid;
-        if (kMask) {
-            if (!v0)
-                s[0] = s[1] = -INFINITY;
-            if (!v1)
-                s[2] = s[3] = -INFINITY;
+        if (kMask) {   // column e (block row 2t + e) sees tokens [0, mask.col[e])
+            if (g >= mask.col[0])
+                s[0] = -INFINITY;
+            if (g >= mask.col[1])
+                s[1] = -INFINITY;
+            if (g + 8 >= mask.col[0])
+                s[2] = -INFINITY;
+            if (g + 8 >= mask.col[1])
+                s[3] = -INFINITY;
         }
         float pr[4];
-        softmax_update(s, st, pr);
+        softmax_update<kMask>(s, st, pr);
         st.l[0] += pr[0] + pr[2];
         st.l[1] += pr[1] + pr[3];
 
@@ -138,13 +141,13 @@ struct Bf16Format {
         const uint32_t pl1 = movmatrix_trans(pack_bf16x2(lo[2], lo[3]));
 
         // O^T += V^T . P^T: ldmatrix.trans matrix j is (tokens 8 (j >> 1) .., d 8 (j & 1) ..),
-        // giving the A fragment of rows d = 16 c + (0..15) and columns tokens 0..15.  On the
-        // last page, tokens >= valid (never written: any bits) are zeroed so 0 * Inf cannot
-        // reach the output.
+        // giving the A fragment of rows d = 16 c + (0..15) and columns tokens 0..15.  Tokens
+        // >= mask.valid (never written: any bits) are zeroed so 0 * Inf cannot reach the output.
         const int vtok = (lane & 7) + 8 * (lane >> 4);
         const int vd = 8 * ((lane >> 3) & 1);
         uint32_t keep[2] = {0xFFFFFFFFu, 0xFFFFFFFFu};   // tokens 2t, 2t+1 | 2t+8, 2t+9
         if (kMask) {
+            const int valid = mask.valid;
             keep[0] = (2 * t < valid ? 0x0000FFFFu : 0u) | (2 * t + 1 < valid ? 0xFFFF0000u : 0u);
             keep[1] = (2 * t + 8 < valid ? 0x0000FFFFu : 0u) | (2 * t + 9 < valid ? 0xFFFF0000u : 0u);
         }
@@ -172,18 +175,19 @@ struct Bf16Format {
                 st.l[e] += __shfl_xor_sync(0xFFFFFFFFu, st.l[e], d);
     }
 
-    // out[s][head_base(hv) + 2t + e][d] = o / l; tile c, rows g and g + 8 are d = 16 c + g (+ 8).
-    __device__ static void finalize(const DecodeParams &p, int s, int hv, int lane, float o[8][4],
+    // block row 2t + e: out[row][d] = o / l; tile c, rows g and g + 8 are d = 16 c + g (+ 8).
+    template <class Seg>
+    __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane, float o[8][4],
                                     const float l[2])
     {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const int head = 2 * t + e;
-            if (head >= p.head_count(hv))
+            if (head >= sg.nrows)
                 continue;
             const float inv = 1.0f / l[e];
-            float *dst = p.out + (static_cast<int64_t>(s) * p.hq + p.head_base(hv) + head) * kHeadDim;
+            float *dst = p.out + sg.row_offset(p, head);
 #pragma unroll
             for (int c = 0; c < 8; c++) {
                 dst[16 * c + g] = o[c][e] * inv;
@@ -228,12 +232,16 @@ ShapeCache g_bf16_shapes;
 
 cudaError_t bf16_launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
 {
-    static const void *const decode_kernels[2] = {
-        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format>),
-        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format>)};
-    static const void *const merge_kernels[2] = {
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format>),
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format>)};
+    static const void *const decode_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format, true>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Bf16Format, true>)};
+    static const void *const merge_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format, true>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format, true>)};
     return decode::launch_shape(g_bf16_shapes, decode_kernels, merge_kernels,
                                 32 * Bf16Format::kWarps, smem, merge_smem, out);
 }
@@ -258,17 +266,18 @@ cudaError_t launch_append_bf16(const AppendBf16Args &a, cudaStream_t stream)
     return cudaGetLastError();
 }
 
-size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs)
+size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                                   int64_t total_q)
 {
     if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
         return 0;
+    const bool prefill = total_q >= 0;
     LaunchShape ls;
-    const SubGroups sg = sub_groups(num_kv_heads, num_q_heads);
-    if (bf16_launch_shape(decode_smem_bytes<Bf16Format>(num_seqs, sg.gsub),
+    if (bf16_launch_shape(decode_smem_bytes<Bf16Format>(num_seqs, query_rows(num_kv_heads, num_q_heads, prefill)),
                           merge_smem_bytes(num_seqs), ls) != cudaSuccess)
         return 0;
-    return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Bf16Format::kWarps, num_seqs,
-                               sg.hseg);
+    return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Bf16Format::kWarps,
+                               max_segments(num_kv_heads, num_q_heads, num_seqs, total_q, prefill));
 }
 
 cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
@@ -299,8 +308,9 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
         cache.rows = rows;
     }
 
-    const SubGroups sg = sub_groups(a.num_kv_heads, a.num_q_heads);
-    const size_t smem = decode_smem_bytes<Bf16Format>(a.num_seqs, sg.gsub);
+    const bool prefill = a.q_start != nullptr;
+    const int32_t qrows = query_rows(a.num_kv_heads, a.num_q_heads, prefill);
+    const size_t smem = decode_smem_bytes<Bf16Format>(a.num_seqs, qrows);
     const size_t msmem = merge_smem_bytes(a.num_seqs);
     LaunchShape ls;
     cudaError_t e = bf16_launch_shape(smem, msmem, ls);
@@ -309,6 +319,7 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
 
     DecodeParams p;
     p.q = static_cast<const uint16_t *>(a.q);
+    p.q_start = a.q_start;
     p.scales = nullptr;
     p.block_table = a.block_table;
     p.seq_lens = a.seq_lens;
@@ -321,9 +332,8 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     p.hq = a.num_q_heads;
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
-    p.nsub = sg.nsub;
-    p.gsub = sg.gsub;
-    p.hseg = sg.hseg;
+    p.qrows = qrows;
+    p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Bf16Format::kWarps;
     p.q_mult = static_cast<float>(static_cast<double>(a.sm_scale) * 1.4426950408889634);
 
@@ -337,17 +347,21 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, paged_decode_kernel<Bf16Format>, cache.map, p);
+    e = cudaLaunchKernelEx(&cfg, prefill ? paged_decode_kernel<Bf16Format, true>
+                                         : paged_decode_kernel<Bf16Format, false>,
+                           cache.map, p);
     if (e != cudaSuccess)
         return e;
 
-    const int64_t segs = static_cast<int64_t>(a.num_seqs) * p.hseg;
+    const int64_t segs = p.max_segments;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&mcfg, paged_decode_merge_kernel<Bf16Format>, p);
+    e = cudaLaunchKernelEx(&mcfg, prefill ? paged_decode_merge_kernel<Bf16Format, true>
+                                          : paged_decode_merge_kernel<Bf16Format, false>,
+                           p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();

@@ -47,7 +47,7 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
                  const uint8_t *kv_pages, const void *scales, const int32_t *block_table,
                  int32_t max_blocks, const int32_t *seq_lens, int32_t num_seqs, float sm_scale,
                  const float *out, const void *workspace, size_t workspace_bytes,
-                 bool bf16 = false)
+                 bool bf16 = false, int64_t total_q = -1)
 {
     if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
         return SAW_ERR_INVALID_ARGUMENT;
@@ -66,8 +66,9 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
         return SAW_ERR_INVALID_ARGUMENT;
     if (int64_t(max_blocks) * 16 > INT32_MAX)
         return SAW_ERR_INVALID_ARGUMENT;
-    const size_t need = bf16 ? saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs)
-                             : saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+    const size_t need =
+        bf16 ? saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q)
+             : saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q);
     if (need == 0)
         return SAW_ERR_CUDA;
     if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
@@ -475,6 +476,70 @@ int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const
     return decode_bf16_impl(cache, num_q_heads, q, kv_bf16, block_table, max_blocks_per_seq,
                             seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes,
                             dev_status, s, appended);
+}
+
+// ---- chunked-prefill attention over the INT4 cache -------------------------------------------
+
+size_t saw_paged_prefill_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                         int32_t num_seqs, int64_t total_q)
+{
+    if (check_cache(cache) != SAW_OK || num_q_heads <= 0 || total_q < 0 ||
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
+        return 0;
+    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q);
+}
+
+static int prefill_impl(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                        const int32_t *q_start, int64_t total_q, const uint8_t *kv_pages,
+                        const void *scales, const int32_t *block_table, int32_t max_blocks_per_seq,
+                        const int32_t *seq_lens, int32_t num_seqs, float sm_scale, float *out,
+                        void *workspace, size_t workspace_bytes, uint32_t *dev_status,
+                        void *stream, bool rotate)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    if (total_q < 0 || (num_seqs > 0 && (q_start == nullptr || !aligned(q_start, 4))) ||
+        total_q > (int64_t(1) << 31) - 1)
+        return SAW_ERR_INVALID_ARGUMENT;
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, false,
+                      total_q);
+    if (rc != SAW_OK || num_seqs == 0 || total_q == 0)
+        return rc;
+    saw::DecodeArgs a =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    a.rotate = rotate;
+    a.q_start = q_start;
+    a.total_q = total_q;
+    return saw::launch_paged_decode(a, static_cast<cudaStream_t>(stream), false) == cudaSuccess
+               ? SAW_OK
+               : SAW_ERR_CUDA;
+}
+
+int saw_paged_prefill_attn(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                           const int32_t *q_start, int64_t total_q, const uint8_t *kv_pages,
+                           const void *scales, const int32_t *block_table,
+                           int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                           float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                           uint32_t *dev_status, void *stream)
+{
+    return prefill_impl(cache, num_q_heads, q, q_start, total_q, kv_pages, scales, block_table,
+                        max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
+                        workspace_bytes, dev_status, stream, true);
+}
+
+int saw_paged_prefill_attn_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                                 const int32_t *q_start, int64_t total_q, const uint8_t *kv_pages,
+                                 const void *scales, const int32_t *block_table,
+                                 int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                                 int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                                 size_t workspace_bytes, uint32_t *dev_status, void *stream)
+{
+    return prefill_impl(cache, num_q_heads, q, q_start, total_q, kv_pages, scales, block_table,
+                        max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
+                        workspace_bytes, dev_status, stream, false);
 }
 
 }  // extern "C"

@@ -55,6 +55,8 @@ struct DecodeArgs {
     size_t workspace_bytes;
     uint32_t *status;
     bool rotate = true;          // false: plain INT4 cache (no query / output rotation)
+    const int32_t *q_start = nullptr;   // chunked prefill: [S + 1] query-row offsets (else decode)
+    int64_t total_q = 0;         // chunked prefill: query rows (q_start[S])
 };
 
 struct AppendBf16Args {
@@ -73,8 +75,10 @@ struct AppendBf16Args {
 cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t stream,
                                    bool trigger_dependents);
 
-// Workspace bytes the decode kernel needs on the current device (0 if the shape is invalid).
-size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs);
+// Workspace bytes the decode kernel needs on the current device (0 if the shape is invalid);
+// total_q >= 0: a chunked prefill over total_q query rows.
+size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                              int64_t total_q = -1);
 
 // Queue the decode kernel; `programmatic` launches it as a programmatic dependent of the
 // previous kernel on the stream.  Returns a cudaError_t.
@@ -83,7 +87,8 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
 // The uncompressed BF16 paged cache (baseline): scatter, decode workspace size, decode
 // (DecodeArgs::kv_pages is the bf16 cache; scales and rotate are unused).
 cudaError_t launch_append_bf16(const AppendBf16Args &a, cudaStream_t stream);
-size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs);
+size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                                   int64_t total_q = -1);
 cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
 
 }  // namespace saw

@@ -79,6 +79,13 @@ def _open_library() -> ctypes.CDLL:
     lib.saw_rotate_quantize_paged_strided.restype = ctypes.c_int
     lib.saw_quantize_paged_plain_strided.argtypes = lib.saw_rotate_quantize_paged_strided.argtypes
     lib.saw_quantize_paged_plain_strided.restype = ctypes.c_int
+    lib.saw_paged_prefill_workspace_bytes.argtypes = [D, i32, i32, i64]
+    lib.saw_paged_prefill_workspace_bytes.restype = sz
+    lib.saw_paged_prefill_attn.argtypes = [D, i32, P, P, i64, P, P, P, i32, P, i32, f32, P, P, sz,
+                                           P, P]
+    lib.saw_paged_prefill_attn.restype = ctypes.c_int
+    lib.saw_paged_prefill_attn_plain.argtypes = lib.saw_paged_prefill_attn.argtypes
+    lib.saw_paged_prefill_attn_plain.restype = ctypes.c_int
     lib.saw_append_bf16_paged.argtypes = [D, P, P, P, i64, P, P, P]
     lib.saw_append_bf16_paged.restype = ctypes.c_int
     lib.saw_paged_decode_bf16_workspace_bytes.argtypes = [D, i32, i32]
@@ -448,3 +455,52 @@ def saw_decode_step_bf16(q, k_new, v_new, slot_mapping, kv_bf16, block_table, se
                                   _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
                                   _stream(stream))
     _check(rc, "saw_decode_step_bf16")
+
+
+# ---- chunked-prefill attention over the INT4 cache -------------------------------------------
+
+def saw_paged_prefill_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,
+                                      total_q: int) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, 1)
+    return int(lib.saw_paged_prefill_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
+                                                     int(num_seqs), int(total_q)))
+
+
+def allocate_prefill_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: int, total_q: int,
+                               device="cuda") -> torch.Tensor:
+    n = saw_paged_prefill_workspace_bytes(num_kv_heads, num_q_heads, num_seqs, total_q)
+    if n == 0:
+        raise SawError(SAW_ERR_CUDA, "saw_paged_prefill_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def saw_paged_prefill_attn(q, q_start, kv_pages, scales, block_table, seq_lens, out, workspace,
+                           sm_scale=None, dev_status=None, stream=None, rotate=True) -> None:
+    """Causal attention of a chunk of query tokens (bf16 [total_q][Hq][128], sequence s owning
+    rows q_start[s] .. q_start[s + 1] - 1, the last tokens of its cached seq_lens[s]) over the
+    INT4 paged cache into out (fp32 [total_q][Hq][128]).  rotate=False reads a plain INT4
+    cache."""
+    _need(q_start, "q_start", torch.int32, 1)
+    _need(q, "q", torch.bfloat16, 3)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    _need(out, "out", torch.float32, 3)
+    _need(workspace, "workspace", torch.uint8, 1)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    desc = cache_desc(kv_pages)
+    total_q, hq, d = q.shape
+    S = seq_lens.shape[0]
+    if d != HEAD_DIM or tuple(out.shape) != (total_q, hq, HEAD_DIM):
+        raise ValueError("q and out must be [total_q][Hq][128]")
+    if q_start.shape[0] != S + 1 or block_table.shape[0] != S:
+        raise ValueError("q_start needs num_seqs + 1 entries and block_table one row per sequence")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    fn = lib.saw_paged_prefill_attn if rotate else lib.saw_paged_prefill_attn_plain
+    rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(q_start), total_q, _ptr(kv_pages), _ptr(scales),
+            _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S, float(sm_scale), _ptr(out),
+            _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_paged_prefill_attn" if rotate else "saw_paged_prefill_attn_plain")

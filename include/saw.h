@@ -179,6 +179,37 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
                           void *workspace, size_t workspace_bytes, uint32_t *dev_status,
                           void *stream);
 
+/* Chunked-prefill attention over the INT4 paged cache: the read step for a chunk of new tokens
+ * whose K/V were already appended with saw_rotate_quantize_paged ("SAW-INT4: System-Aware
+ * 4-Bit KV-Cache Quantization for Real-World LLM Serving", Research Findings: the quantized
+ * cache must serve fused attention over paged memory; a prefill chunk is its multi-query case).
+ * Sequence s has C_s = q_start[s + 1] - q_start[s] query tokens (rows q_start[s] .. of q and
+ * out), the last C_s of its seq_lens[s] cached tokens; query i sits at position
+ * seq_lens[s] - C_s + i and attends causally to cache tokens 0 .. seq_lens[s] - C_s + i, with
+ * the rotation, scales and arithmetic of saw_paged_decode_attn (a decode is the case C_s = 1).
+ *     q: bf16 [total_q][Hq][128]; out: fp32 [total_q][Hq][128]; q_start: int32 [num_seqs + 1],
+ *     device, non-decreasing, q_start[0] = 0, q_start[num_seqs] = total_q, 0 <= C_s <= seq_lens[s]
+ *     (a violating sequence is flagged SAW_DEV_BAD_SEQ_LEN and skipped).
+ * Every (query token, head) pair reads the pages of its sequence once per block of 8 such
+ * pairs, so the K/V traffic is about total_q G / 8 times that of one decode of the batch; the
+ * kernel and its work split are those of the decode.  workspace: at least
+ * saw_paged_prefill_workspace_bytes() bytes, 256-byte aligned, no initialisation needed.
+ * The _plain variant reads a cache written by saw_quantize_paged_plain. */
+size_t saw_paged_prefill_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                         int32_t num_seqs, int64_t total_q);
+int saw_paged_prefill_attn(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                           const int32_t *q_start, int64_t total_q, const uint8_t *kv_pages,
+                           const void *scales, const int32_t *block_table,
+                           int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                           float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                           uint32_t *dev_status, void *stream);
+int saw_paged_prefill_attn_plain(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,
+                                 const int32_t *q_start, int64_t total_q, const uint8_t *kv_pages,
+                                 const void *scales, const int32_t *block_table,
+                                 int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                                 int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                                 size_t workspace_bytes, uint32_t *dev_status, void *stream);
+
 /* The uncompressed BF16 paged KV cache: the baseline the INT4 format is measured against
  * ("SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving", Research
  * Findings: serving throughput against a 16-bit KV cache; "BitDecoding-FP4: Native FP4 KV
