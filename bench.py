@@ -461,6 +461,42 @@ def run_saw(args):
                      "int4_decode_speedup": t_dec_bf16 / t_decode}
     del kvb, wsb
 
+    # ---- chunked prefill over the INT4 cache: a 512-token chunk per sequence -----------------
+    pfl = synth.custom("chunked_prefill", [4096] * 8, num_q_heads=32, num_kv_heads=8,
+                       seed=40 + rank, outlier_range=(10.0, 30.0))
+    pkv3, psc3 = saw.allocate_cache(pfl.num_pages, pfl.num_kv_heads, dev)
+    seq, pos = synth.token_index(pfl)
+    saw.saw_rotate_quantize_paged(synth.kv_values(pfl, "K", device=dev),
+                                  synth.kv_values(pfl, "V", device=dev),
+                                  torch.from_numpy(synth.slot_mapping(pfl, seq, pos)).to(dev),
+                                  pkv3, psc3)
+    chunk = 512
+    q_start = torch.arange(0, (pfl.num_seqs + 1) * chunk, chunk, dtype=torch.int32, device=dev)
+    qpf = torch.randn(pfl.num_seqs * chunk, pfl.num_q_heads, 128, generator=torch.Generator(
+        device="cpu").manual_seed(41), ).to(torch.bfloat16).to(dev)
+    opf = torch.empty(qpf.shape, dtype=torch.float32, device=dev)
+    wpf = saw.allocate_prefill_workspace(pfl.num_kv_heads, pfl.num_q_heads, pfl.num_seqs,
+                                         int(qpf.shape[0]), dev)
+    tab3, len3 = torch.from_numpy(pfl.block_table).to(dev), torch.from_numpy(pfl.seq_lens).to(dev)
+    run_pf = lambda: saw.saw_paged_prefill_attn(qpf, q_start, pkv3, psc3, tab3, len3, opf, wpf,
+                                                dev_status=status, stream=stream)
+    for _ in range(3):
+        run_pf()
+    t_pf = mean_event_ms(run_pf, max(5, min(args.steps, 50)))
+    g = pfl.num_q_heads // pfl.num_kv_heads
+    blocks = pfl.num_seqs * pfl.num_kv_heads * (chunk * g // 8)
+    pages = int(((pfl.seq_lens + 15) // 16)[0])
+    # causal attention: query i of a chunk at the end of L tokens sees L - chunk + i + 1 tokens
+    visible = sum(4096 - chunk + i + 1 for i in range(chunk)) * pfl.num_seqs * pfl.num_q_heads
+    prefill_attn = {"workload": "8 seqs x 4096 cached tokens, last 512 of each as queries, 32 q / 8 kv heads",
+                    "launch_ms": t_pf,
+                    "query_tokens_per_s": world * pfl.num_seqs * chunk / (t_pf * 1e-3),
+                    "attention_TFLOPs": 4 * 128 * visible / (t_pf * 1e-3) / 1e12,
+                    "page_reads_per_launch": blocks * pages,
+                    "note": "each block of 8 (query token, head) rows reads its sequence's pages; "
+                            "the repeats come from L2"}
+    del pkv3, psc3, qpf, opf, wpf
+
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
     h_q, h_k, h_v, h_slots, h_table, h_lens = (pin(q), pin(k_new), pin(v_new), pin(slots),
@@ -512,6 +548,7 @@ def run_saw(args):
         "rot_quant": rot_quant,
         "plain_int4": plain_int4,
         "bf16_baseline": bf16_baseline,
+        "prefill_attn": prefill_attn,
         "append_launch_ms": t_append,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,
