@@ -34,8 +34,17 @@
 namespace saw {
 namespace {
 
-constexpr int kTileVecs = 8;                           // (token, kv head) vectors per warp tile
-constexpr int kTileBytes = kTileVecs * kHeadDim * 2;   // 2 KiB of K (or of V) per tile
+constexpr int kTileBytes = 2048;                       // K (or V) bytes of one warp tile: 16 rows
+// Head dimension D = 128 or 256 (two independent 128-point rotation blocks): a warp tile holds
+// 2048 / (2 D) vectors of K and as many of V, D / 64 threads per vector, each thread 64
+// elements of one 128-block; a vector is D / 64 tensor-map rows of 128 bytes.
+template <int kD>
+struct RqDims {
+    static constexpr int kTileVecs = kTileBytes / (2 * kD);   // 8 or 4
+    static constexpr int kThreadsPerVec = kD / 64;             // 2 or 4
+    static constexpr int kRowsPerVec = kD / 64;                // 128-byte rows per vector
+    static constexpr int kCodeBytes = kD / 2;                  // packed codes per vector
+};
 constexpr int kRqStages = 3;
 constexpr int kRqWarps = 4;
 constexpr int kRqThreads = 32 * kRqWarps;
@@ -61,13 +70,15 @@ __device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u 
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
 
-// This thread's 64 bf16 elements of tile vector vt (rows 2 vt and 2 vt + 1 of 128 bytes; the
-// 16-byte chunk c of row r sits at chunk c ^ (r & 7) under the 128-byte swizzle).
-__device__ __forceinline__ void load_half_vec(uint32_t tile, int vt, int b, uint4 raw[8])
+// This thread's 64 bf16 elements of 128-block blk of tile vector vt (rows (D / 64) vt + 2 blk
+// and the next of 128 bytes; the 16-byte chunk c of row r sits at chunk c ^ (r & 7) under the
+// 128-byte swizzle).
+template <int kD>
+__device__ __forceinline__ void load_half_vec(uint32_t tile, int vt, int blk, int b, uint4 raw[8])
 {
 #pragma unroll
     for (int a = 0; a < 8; a++) {
-        const int row = 2 * vt + (a >> 2);
+        const int row = RqDims<kD>::kRowsPerVec * vt + 2 * blk + (a >> 2);
         const int chunk = (2 * (a & 3) + b) ^ (row & 7);
         raw[a] = lds128(tile + row * 128 + chunk * 16);
     }
@@ -218,11 +229,11 @@ struct RqParams {
 
 // Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
 // kRotate = false is the plain INT4 quantizer (H = I) used as the unrotated baseline.
-template <bool kRotate>
-__device__ __forceinline__ void quantize_store(const uint64_t X[32], int b, bool store,
+template <bool kRotate, int kD>
+__device__ __forceinline__ void quantize_store(const uint64_t X[32], int blk, int b, bool store,
                                                int64_t row, const RqParams &p)
 {
-    // min / max over the pair's 128 elements
+    // min / max over the vector's D elements (its D / 64 threads)
     float mns[8], mxs[8];
 #pragma unroll
     for (int i = 0; i < 32; i++) {
@@ -233,8 +244,11 @@ __device__ __forceinline__ void quantize_store(const uint64_t X[32], int b, bool
     }
     float mn = fminf(fmin3(mns[0], mns[1], mns[2]), fmin3(fmin3(mns[3], mns[4], mns[5]), mns[6], mns[7]));
     float mx = fmaxf(fmax3(mxs[0], mxs[1], mxs[2]), fmax3(fmax3(mxs[3], mxs[4], mxs[5]), mxs[6], mxs[7]));
-    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
-    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+#pragma unroll
+    for (int d = 1; d < RqDims<kD>::kThreadsPerVec; d <<= 1) {
+        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
+        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+    }
 
     float scale = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
     const bool degenerate = !(scale != 0.0f);
@@ -252,7 +266,7 @@ __device__ __forceinline__ void quantize_store(const uint64_t X[32], int b, bool
     // note above code_bits_tie()); the 16 elements of the two words go through
     // code_bits_exact() when one of them lies near a half-way quotient, or for a subnormal
     // scale.
-    uint8_t *dst = p.kv_pages + row * kRowBytes;
+    uint8_t *dst = p.kv_pages + row * RqDims<kD>::kCodeBytes + 64 * blk;
 #pragma unroll
     for (int a4 = 0; a4 < 4; a4++) {
         uint32_t tlo[8], thi[8];
@@ -288,17 +302,19 @@ __device__ __forceinline__ void quantize_store(const uint64_t X[32], int b, bool
             *reinterpret_cast<uint32_t *>(dst + 8 * (a4 + 4) + 4 * b) = pack8(thi);
         }
     }
-    if (store && b == 0) {
+    if (store && b == 0 && blk == 0) {
         const __half2 sz = __halves2half2(__float2half_rn(scale), __float2half_rn(zero));
         p.scales[row] = half2_as_u32(sz);
     }
 }
 
-template <bool kRotate>
+template <bool kRotate, int kD>
 __global__ void __launch_bounds__(kRqThreads, 4)
     rotate_quantize_kernel(const __grid_constant__ CUtensorMap tk,
                            const __grid_constant__ CUtensorMap tv, const RqParams p)
 {
+    using Dims = RqDims<kD>;
+    constexpr int kTileVecs = Dims::kTileVecs;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -331,11 +347,11 @@ __global__ void __launch_bounds__(kRqThreads, 4)
                     // the tile's first vector: token and head (the box spans whole tiles)
                     const uint32_t v0 = itile * kTileVecs;
                     const int32_t tok = static_cast<int32_t>(v0 / hkv_u);
-                    const int32_t row = static_cast<int32_t>(2 * (v0 - tok * hkv_u));
+                    const int32_t row = static_cast<int32_t>(Dims::kRowsPerVec * (v0 - tok * hkv_u));
                     tma_load_3d(dst, &tk, 0, row, tok, bar);
                     tma_load_3d(dst + kTileBytes, &tv, 0, row, tok, bar);
                 } else {
-                    const int32_t y = static_cast<int32_t>(itile * (2 * kTileVecs));
+                    const int32_t y = static_cast<int32_t>(itile * (Dims::kRowsPerVec * kTileVecs));
                     tma_load_2d(dst, &tk, 0, y, bar);
                     tma_load_2d(dst + kTileBytes, &tv, 0, y, bar);
                 }
@@ -350,8 +366,9 @@ __global__ void __launch_bounds__(kRqThreads, 4)
         issue();
 
     const int half = lane >> 4;          // 0: K, 1: V
-    const int b = lane & 1;
-    const int vt = (lane >> 1) & 7;
+    const int b = lane & 1;              // half of a 128-block
+    const int blk = (lane >> 1) & (Dims::kThreadsPerVec / 2 - 1);   // 128-block of the vector
+    const int vt = (lane & 15) / Dims::kThreadsPerVec;              // vector of the tile
     const uint32_t num_vecs = static_cast<uint32_t>(p.num_vecs);
     const uint32_t hkv = static_cast<uint32_t>(p.hkv);
     uint32_t tile = wg;
@@ -398,12 +415,12 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 
         const uint32_t tile_smem = ring + stg * kRqStageBytes + half * kTileBytes;
         uint4 raw[8];
-        load_half_vec(tile_smem, vt, b, raw);
+        load_half_vec<kD>(tile_smem, vt, blk, b, raw);
         uint64_t X[32];
         to_pairs(raw, X);
         if (kRotate)
             fwht128(X, b, 0xFFFFFFFFu);
-        quantize_store<kRotate>(X, b, store, row, p);
+        quantize_store<kRotate, kD>(X, blk, b, store, row, p);
         __syncwarp();
     }
     if (i < n) {
@@ -422,47 +439,51 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     const int64_t num_vecs = a.num_tokens * a.num_kv_heads;
     if (num_vecs == 0)
         return cudaSuccess;
-    if (num_vecs > (int64_t(1) << 29))
-        return cudaErrorInvalidValue;       // tensor-map rows (2 per vector) must fit in int32
+    if (a.head_dim != 128 && a.head_dim != 256)
+        return cudaErrorInvalidValue;
+    const int64_t rows_per_vec = a.head_dim / 64;
+    const int64_t tile_vecs = kTileBytes / (2 * a.head_dim);
+    if (num_vecs * rows_per_vec > (int64_t(1) << 30))
+        return cudaErrorInvalidValue;       // tensor-map rows must fit in int32
 
-    // k / v: contiguous [T][Hkv][128] (k_stride = v_stride = 0) through a 2-D map of 128-byte
-    // rows, or with a token stride through 3-D maps whose box is one whole tile of 8 vectors
-    // (Hkv a multiple of 8: 8 heads of one token; Hkv dividing 8: 8 / Hkv tokens), so every
-    // copy lands on a 1024-byte aligned stage.
+    // k / v: contiguous [T][Hkv][D] (k_stride = v_stride = 0) through a 2-D map of 128-byte
+    // rows, or with a token stride through 3-D maps whose box is one whole tile of V vectors
+    // (V = 8 for D = 128, 4 for D = 256; Hkv a multiple of V: V heads of one token; Hkv dividing
+    // V: V / Hkv tokens), so every copy lands on a 1024-byte aligned stage.
     const bool strided = a.k_stride != 0 || a.v_stride != 0;
     static thread_local struct {
         const void *k = nullptr, *v = nullptr;
         int64_t num_vecs = 0, k_stride = -1, v_stride = -1;
-        int32_t hkv = 0;
+        int32_t hkv = 0, head_dim = 0;
         CUtensorMap mk, mv;
     } cache;
     if (cache.k != a.k || cache.v != a.v || cache.num_vecs != num_vecs || cache.hkv != a.num_kv_heads ||
-        cache.k_stride != a.k_stride || cache.v_stride != a.v_stride) {
+        cache.k_stride != a.k_stride || cache.v_stride != a.v_stride || cache.head_dim != a.head_dim) {
         auto encode = tensor_map_encoder();
         if (encode == nullptr)
             return cudaErrorNotSupported;
         const int64_t hkv = a.num_kv_heads;
-        if (strided && hkv % kTileVecs != 0 && kTileVecs % hkv != 0)
+        if (strided && hkv % tile_vecs != 0 && tile_vecs % hkv != 0)
             return cudaErrorInvalidValue;
         const cuuint32_t estr[3] = {1, 1, 1};
         for (int which = 0; which < 2; which++) {
             CUresult r;
             void *base = const_cast<void *>(which ? a.v : a.k);
             if (!strided) {
-                const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(2 * num_vecs)};
+                const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows_per_vec * num_vecs)};
                 const cuuint64_t strides[1] = {128};
-                const cuuint32_t box[2] = {128, 2 * kTileVecs};   // one warp tile: 16 rows
+                const cuuint32_t box[2] = {128, kTileBytes / 128};   // one warp tile: 16 rows
                 r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             } else {
                 const int64_t stride = which ? a.v_stride : a.k_stride;   // bf16 elements
-                const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(2 * hkv),
+                const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows_per_vec * hkv),
                                             static_cast<cuuint64_t>(a.num_tokens)};
                 const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(stride * 2)};
-                const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(2 * std::min<int64_t>(hkv, kTileVecs)),
-                                           static_cast<cuuint32_t>(std::max<int64_t>(1, kTileVecs / hkv))};
+                const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(rows_per_vec * std::min<int64_t>(hkv, tile_vecs)),
+                                           static_cast<cuuint32_t>(std::max<int64_t>(1, tile_vecs / hkv))};
                 r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base,
                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -477,6 +498,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         cache.v = a.v;
         cache.num_vecs = num_vecs;
         cache.hkv = a.num_kv_heads;
+        cache.head_dim = a.head_dim;
         cache.k_stride = a.k_stride;
         cache.v_stride = a.v_stride;
     }
@@ -484,7 +506,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     RqParams p;
     p.slot_mapping = a.slot_mapping;
     p.num_vecs = num_vecs;
-    p.num_tiles = (num_vecs + kTileVecs - 1) / kTileVecs;
+    p.num_tiles = (num_vecs + tile_vecs - 1) / tile_vecs;
     p.hkv = a.num_kv_heads;
     p.num_slots = a.num_pages * kPageSize;
     p.kv_pages = a.kv_pages;
@@ -501,17 +523,23 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         return e;
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
-    auto kernel = a.rotate ? rotate_quantize_kernel<true> : rotate_quantize_kernel<false>;
+    static const void *const kernels[4] = {
+        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 128>),
+        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 128>),
+        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 256>),
+        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 256>)};
+    auto kernel = a.head_dim == 128
+                      ? (a.rotate ? rotate_quantize_kernel<true, 128> : rotate_quantize_kernel<false, 128>)
+                      : (a.rotate ? rotate_quantize_kernel<true, 256> : rotate_quantize_kernel<false, 256>);
     if (sms_of[dev] == 0) {
         int sms = 0, occ = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        for (int r = 0; r < 2 && e == cudaSuccess; r++)
-            e = cudaFuncSetAttribute(r ? rotate_quantize_kernel<true> : rotate_quantize_kernel<false>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+        for (int r = 0; r < 4 && e == cudaSuccess; r++)
+            e = cudaFuncSetAttribute(kernels[r], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kRqSmemBytes));
         if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, rotate_quantize_kernel<true>,
-                                                              kRqThreads, kRqSmemBytes);
+            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernels[0], kRqThreads,
+                                                              kRqSmemBytes);
         if (e != cudaSuccess)
             return e;
         if (occ <= 0)

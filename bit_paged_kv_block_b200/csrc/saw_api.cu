@@ -16,7 +16,7 @@ int check_cache(const saw_cache_desc *c)
 {
     if (c == nullptr || c->num_kv_heads <= 0 || c->num_pages < 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if (c->head_dim != 128 || c->page_size != 16)
+    if ((c->head_dim != 128 && c->head_dim != 256) || c->page_size != 16)
         return SAW_ERR_UNSUPPORTED;
     // tensor-map rows (page * Hkv + h) * 32 must stay below 2^31
     if (c->num_pages > (int64_t(1) << 31) / (int64_t(c->num_kv_heads) * 32))
@@ -38,7 +38,7 @@ int check_append(const saw_cache_desc *cache, const void *k, const void *v,
     if (!aligned(k, 16) || !aligned(v, 16) || !aligned(kv_pages, 16) ||
         (!bf16 && !aligned(scales, 16)) || !aligned(slot_mapping, 8))
         return SAW_ERR_INVALID_ARGUMENT;
-    if (num_tokens > INT64_MAX / (int64_t(cache->num_kv_heads) * 256))
+    if (num_tokens > INT64_MAX / (int64_t(cache->num_kv_heads) * 2 * cache->head_dim))
         return SAW_ERR_INVALID_ARGUMENT;
     return SAW_OK;
 }
@@ -51,6 +51,8 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
 {
     if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
         return SAW_ERR_INVALID_ARGUMENT;
+    if (cache->head_dim != 128)
+        return SAW_ERR_UNSUPPORTED;   // attention kernels: D = 128
     if (num_q_heads / cache->num_kv_heads > 16)
         return SAW_ERR_UNSUPPORTED;
     if (!std::isfinite(sm_scale))
@@ -116,7 +118,8 @@ const char *saw_status_string(int status)
     case SAW_ERR_INVALID_ARGUMENT:
         return "invalid argument (null pointer, bad size or alignment, Hq not a multiple of Hkv)";
     case SAW_ERR_UNSUPPORTED:
-        return "unsupported shape (head_dim must be 128, page_size 16, Hq/Hkv at most 16)";
+        return "unsupported shape (head_dim 128, or 256 where supported; page_size 16; Hq/Hkv at "
+               "most 16)";
     case SAW_ERR_CUDA:
         return "CUDA runtime error";
     case SAW_ERR_WORKSPACE:
@@ -144,6 +147,7 @@ saw::RotateQuantizeArgs append_args(const saw_cache_desc *cache, const void *k, 
     a.slot_mapping = slot_mapping;
     a.num_tokens = num_tokens;
     a.num_kv_heads = cache->num_kv_heads;
+    a.head_dim = cache->head_dim;
     a.num_pages = cache->num_pages;
     a.kv_pages = kv_pages;
     a.scales = scales;
@@ -167,11 +171,12 @@ int append_impl(const saw_cache_desc *cache, const void *k, const void *v,
     if (k_stride != 0 || v_stride != 0) {
         // strided rows: each token's Hkv head vectors are contiguous; tokens start every
         // *_stride elements (a multiple of 8, so every token starts on 16 bytes)
-        const int64_t row = int64_t(cache->num_kv_heads) * 128;
+        const int64_t row = int64_t(cache->num_kv_heads) * cache->head_dim;
+        const int64_t tile_vecs = 1024 / cache->head_dim;   // vectors per quantizer tile
         if (k_stride < row || v_stride < row || k_stride % 8 != 0 || v_stride % 8 != 0 ||
             k_stride > (int64_t(1) << 36) || v_stride > (int64_t(1) << 36))
             return SAW_ERR_INVALID_ARGUMENT;
-        if (cache->num_kv_heads % 8 != 0 && 8 % cache->num_kv_heads != 0)
+        if (cache->num_kv_heads % tile_vecs != 0 && tile_vecs % cache->num_kv_heads != 0)
             return SAW_ERR_UNSUPPORTED;
         if (num_tokens > (int64_t(1) << 31) - 1)
             return SAW_ERR_INVALID_ARGUMENT;
@@ -291,7 +296,8 @@ size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num
                                         int32_t num_seqs)
 {
     if (check_cache(cache) != SAW_OK || num_q_heads <= 0 ||
-        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16 ||
+        cache->head_dim != 128)
         return 0;
     return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
 }
@@ -365,6 +371,8 @@ static int check_bf16_cache(const saw_cache_desc *cache)
     const int rc = check_cache(cache);
     if (rc != SAW_OK)
         return rc;
+    if (cache->head_dim != 128)
+        return SAW_ERR_UNSUPPORTED;
     // tensor-map rows (page * Hkv + h) * 64 must stay below 2^31
     if (cache->num_pages > (int64_t(1) << 31) / (int64_t(cache->num_kv_heads) * 64))
         return SAW_ERR_UNSUPPORTED;
@@ -484,7 +492,8 @@ size_t saw_paged_prefill_workspace_bytes(const saw_cache_desc *cache, int32_t nu
                                          int32_t num_seqs, int64_t total_q)
 {
     if (check_cache(cache) != SAW_OK || num_q_heads <= 0 || total_q < 0 ||
-        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16 ||
+        cache->head_dim != 128)
         return 0;
     return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q);
 }

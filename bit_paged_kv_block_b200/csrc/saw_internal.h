@@ -29,8 +29,9 @@ struct RotateQuantizeArgs {
     const int64_t *slot_mapping; // [T]
     int64_t num_tokens;
     int32_t num_kv_heads;
+    int32_t head_dim = 128;      // D: 128 or 256 (two 128-point rotation blocks)
     int64_t num_pages;
-    uint8_t *kv_pages;           // [num_pages][Hkv][2][16][64]
+    uint8_t *kv_pages;           // [num_pages][Hkv][2][16][D / 2]
     void *scales;                // fp16 [num_pages][Hkv][2][16][2]
     uint32_t *status;            // nullable
     bool rotate = true;          // false: plain INT4 (no Hadamard rotation)

@@ -143,17 +143,17 @@ def _need(t: torch.Tensor, name: str, dtype, ndim=None, cuda=True) -> None:
 
 
 def cache_desc(kv_pages: torch.Tensor) -> saw_cache_desc:
-    """Descriptor of a cache tensor uint8 [num_pages][Hkv][2][16][64]."""
+    """Descriptor of a cache tensor uint8 [num_pages][Hkv][2][16][D / 2] (D = 128 or 256)."""
     _need(kv_pages, "kv_pages", torch.uint8, 5, cuda=False)
     num_pages, hkv, two, page, half = kv_pages.shape
-    if two != 2 or half * 2 != HEAD_DIM:
-        raise ValueError(f"kv_pages must be [num_pages][Hkv][2][16][64], got {tuple(kv_pages.shape)}")
-    return saw_cache_desc(int(hkv), HEAD_DIM, int(page), int(num_pages))
+    if two != 2 or half * 2 not in (128, 256):
+        raise ValueError(f"kv_pages must be [num_pages][Hkv][2][16][D / 2], got {tuple(kv_pages.shape)}")
+    return saw_cache_desc(int(hkv), int(half * 2), int(page), int(num_pages))
 
 
-def allocate_cache(num_pages: int, num_kv_heads: int, device="cuda"):
-    """Empty cache tensors: kv_pages uint8 [P][Hkv][2][16][64], scales fp16 [P][Hkv][2][16][2]."""
-    kv = torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, HEAD_DIM // 2), dtype=torch.uint8,
+def allocate_cache(num_pages: int, num_kv_heads: int, device="cuda", head_dim: int = HEAD_DIM):
+    """Empty cache tensors: kv_pages uint8 [P][Hkv][2][16][D / 2], scales fp16 [P][Hkv][2][16][2]."""
+    kv = torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, head_dim // 2), dtype=torch.uint8,
                      device=device)
     sc = torch.empty((num_pages, num_kv_heads, 2, PAGE_SIZE, 2), dtype=torch.float16,
                      device=device)
@@ -182,8 +182,8 @@ def _append(fn, name, k, v, slot_mapping, kv_pages, scales, dev_status, stream) 
     _need(scales, "scales", torch.float16, 5)
     desc = cache_desc(kv_pages)
     T = k.shape[0]
-    if tuple(k.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
-        raise ValueError("k and v must be [T][Hkv][128] matching the cache")
+    if tuple(k.shape) != (T, desc.num_kv_heads, desc.head_dim) or v.shape != k.shape:
+        raise ValueError("k and v must be [T][Hkv][D] matching the cache")
     if slot_mapping.shape[0] != T:
         raise ValueError("slot_mapping must have one entry per token")
     if tuple(scales.shape) != (desc.num_pages, desc.num_kv_heads, 2, PAGE_SIZE, 2):
@@ -203,15 +203,15 @@ def saw_rotate_quantize_paged_strided(k, v, slot_mapping, kv_pages, scales, dev_
     for t, name in ((k, "k"), (v, "v")):
         if not isinstance(t, torch.Tensor) or t.dtype != torch.bfloat16 or t.device.type != "cuda":
             raise TypeError(f"{name} must be a bf16 CUDA tensor")
-        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != HEAD_DIM:
-            raise ValueError(f"{name} must be [T][Hkv][128] with contiguous heads within a token")
+        if t.dim() != 3 or t.stride(2) != 1 or t.stride(1) != t.shape[2]:
+            raise ValueError(f"{name} must be [T][Hkv][D] with contiguous heads within a token")
     _need(slot_mapping, "slot_mapping", torch.int64, 1)
     _need(kv_pages, "kv_pages", torch.uint8, 5)
     _need(scales, "scales", torch.float16, 5)
     desc = cache_desc(kv_pages)
     T = k.shape[0]
-    if tuple(k.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
-        raise ValueError("k and v must be [T][Hkv][128] matching the cache")
+    if tuple(k.shape) != (T, desc.num_kv_heads, desc.head_dim) or v.shape != k.shape:
+        raise ValueError("k and v must be [T][Hkv][D] matching the cache")
     if slot_mapping.shape[0] != T:
         raise ValueError("slot_mapping must have one entry per token")
     if dev_status is not None:

@@ -31,7 +31,7 @@ def oracle_cache(wl, tokens="all", k=None, v=None, rotate=True):
         v = synth.kv_values(wl, "V", tokens=tokens)
     seq, pos = synth.token_index(wl, tokens)
     slots = synth.slot_mapping(wl, seq, pos)
-    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
+    pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads, wl.head_dim)
     pages[:] = CANARY_CODE
     scales[:] = CANARY_SCALE
     bad = oracle.rotate_quantize_paged(u16(k), u16(v), slots, pages, scales, rotate=rotate,
@@ -48,7 +48,7 @@ def device_cache_from(pages: np.ndarray, scales: np.ndarray, device):
 
 def canary_device_cache(wl, device):
     from bit_paged_kv_block_b200 import saw
-    kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, device)
+    kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, device, head_dim=wl.head_dim)
     kv.fill_(CANARY_CODE)
     sc.view(torch.int16).fill_(CANARY_SCALE)
     return kv, sc

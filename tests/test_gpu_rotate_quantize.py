@@ -140,3 +140,52 @@ def test_strided_kv_from_fused_qkv(cuda_device, hkv, rotate):
     torch.cuda.synchronize()
     pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous(), rotate=rotate)
     assert_cache_equal(kv, sc, pages, scales)
+
+
+@pytest.mark.parametrize("hkv", [2, 4, 8])
+@pytest.mark.parametrize("rotate", [True, False])
+def test_head_dim_256_block_diagonal(cuda_device, hkv, rotate):
+    """D = 256: two independent 128-point rotation blocks per vector, one scale and zero over
+    all 256 elements, 128 code bytes per row; bit-exact against the oracle on outlier data and
+    on small integers (exact ties), ragged token counts."""
+    from bit_paged_kv_block_b200 import saw
+    for kind, T in (("randn", 137), ("small_ints", 61)):
+        wl = synth.custom(f"d256{kind}{hkv}", [T], num_q_heads=hkv, num_kv_heads=hkv,
+                          new_tokens=[T], head_dim=256, seed=hkv, outlier_range=(10.0, 30.0))
+        if kind == "randn":
+            k, v = synth.kv_values(wl, "K"), synth.kv_values(wl, "V")
+        else:
+            g = torch.Generator().manual_seed(hkv)
+            k = torch.randint(-3, 4, (T, hkv, 256), generator=g).to(torch.bfloat16)
+            v = torch.randint(0, 5, (T, hkv, 256), generator=g).to(torch.bfloat16)
+        seq, pos = synth.token_index(wl)
+        slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(cuda_device)
+        kv, sc = canary_device_cache(wl, cuda_device)
+        if rotate:
+            saw.saw_rotate_quantize_paged(k.to(cuda_device), v.to(cuda_device), slots, kv, sc)
+        else:
+            saw.saw_quantize_paged_plain(k.to(cuda_device), v.to(cuda_device), slots, kv, sc)
+        torch.cuda.synchronize()
+        pages, scales = oracle_cache(wl, k=k, v=v, rotate=rotate)
+        assert_cache_equal(kv, sc, pages, scales)
+
+
+def test_head_dim_256_strided(cuda_device):
+    """D = 256 k / v sliced from a fused QKV output (Hkv = 4: one tile of 4 vectors per token)."""
+    from bit_paged_kv_block_b200 import saw
+    T, hkv, hq = 90, 4, 16
+    g = torch.Generator().manual_seed(5)
+    qkv = (torch.randn(T, (hq + 2 * hkv) * 256, generator=g) * 2.0).to(torch.bfloat16)
+    k = qkv[:, hq * 256:(hq + hkv) * 256].view(T, hkv, 256)
+    v = qkv[:, (hq + hkv) * 256:].view(T, hkv, 256)
+    wl = synth.custom("d256qkv", [T], num_q_heads=hkv, num_kv_heads=hkv, new_tokens=[T],
+                      head_dim=256)
+    seq, pos = synth.token_index(wl)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(cuda_device)
+    kv, sc = canary_device_cache(wl, cuda_device)
+    qd = qkv.to(cuda_device)
+    saw.saw_rotate_quantize_paged_strided(qd[:, hq * 256:(hq + hkv) * 256].view(T, hkv, 256),
+                                          qd[:, (hq + hkv) * 256:].view(T, hkv, 256), slots, kv, sc)
+    torch.cuda.synchronize()
+    pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous())
+    assert_cache_equal(kv, sc, pages, scales)
