@@ -29,7 +29,9 @@
 namespace saw {
 namespace decode {
 
-constexpr int kSlotFloats = 32 * 32 + 16;               // O (lane layout) + m[8] + l[8]
+// workspace slot of one piece's partial: O in lane layout (kTiles x 32 float4), then m[8], l[8]
+template <int kTiles>
+__host__ __device__ constexpr int slot_floats() { return kTiles * 128 + 16; }
 constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
 constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
 constexpr int kRowsPerBlock = 8;                        // query rows (MMA columns) per segment
@@ -38,17 +40,19 @@ constexpr int kMergeThreads = 32 * kMergeWarps;
 // per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
 constexpr int kSeqTableBytes = 20;
 // merge kernel shared memory: per-warp partials, flags, then the sequence tables
-constexpr int kMergeSmemSlots = 0;
-constexpr int kMergeSmemFlags = kMergeSmemSlots + (kMergeWarps - 1) * kSlotFloats * 4;
-constexpr int kMergeSmemTables = kMergeSmemFlags + 64;
+template <int kTiles>
+__host__ __device__ constexpr int merge_smem_flags() { return (kMergeWarps - 1) * slot_floats<kTiles>() * 4; }
+template <int kTiles>
+__host__ __device__ constexpr int merge_smem_tables() { return merge_smem_flags<kTiles>() + 64; }
 
 inline size_t seq_table_bytes(int32_t num_seqs)
 {
     return kSeqTableBytes * (static_cast<size_t>(num_seqs) + 1);
 }
+template <int kTiles>
 inline size_t merge_smem_bytes(int32_t num_seqs)
 {
-    return kMergeSmemTables + seq_table_bytes(num_seqs);
+    return merge_smem_tables<kTiles>() + seq_table_bytes(num_seqs);
 }
 
 // Segments of a launch: decode, num_seqs * hkv * ceil(G / 8); chunked prefill over total_q
@@ -69,10 +73,11 @@ inline int32_t query_rows(int32_t num_kv_heads, int32_t num_q_heads, bool prefil
     return prefill || G >= kRowsPerBlock ? kRowsPerBlock : G;
 }
 
-// Workspace of a decode grid of `warps` warps over `segments` segments.
+// Workspace of a decode grid of `warps` warps over `segments` segments (kTiles output tiles).
+template <int kTiles>
 inline size_t workspace_bytes_for(size_t warps, int64_t segments)
 {
-    return (warps + static_cast<size_t>(segments)) * kSlotFloats * sizeof(float);
+    return (warps + static_cast<size_t>(segments)) * slot_floats<kTiles>() * sizeof(float);
 }
 
 struct DecodeParams {
@@ -310,12 +315,12 @@ struct Segment {
     {
         return len - c + row_token(p, e);
     }
-    // q / out element offset of block row e (e < nrows)
-    __device__ int64_t row_offset(const DecodeParams &p, int e) const
+    // q / out element offset of block row e (e < nrows) for head dimension d
+    __device__ int64_t row_offset(const DecodeParams &p, int e, int d) const
     {
         const int tok = row_token(p, e);
         const int head = row0 + e - tok * p.group;
-        return ((qrow0 + tok) * p.hq + h * p.group + head) * kHeadDim;
+        return ((qrow0 + tok) * p.hq + h * p.group + head) * d;
     }
     // pages from this index on hold a token some row of the block may not see (or past len)
     __device__ int first_masked_page(const DecodeParams &p) const
@@ -345,21 +350,24 @@ __device__ __forceinline__ PageMask page_mask(int len, const int lim[2], int pag
     return m;
 }
 
-// Per-warp running state of one piece: o holds O^T (128 value rows x 8 stacked query heads) as
-// eight m16n8 accumulator tiles, thread (g, t) holding heads 2t and 2t + 1 of rows g and g + 8
-// of each tile (which value dimension d a row is, is up to the kernel and its finalize step);
-// m, l: running max (log2 domain) and sum of the two heads; z: the kernel's zero-point sum.
+// Per-warp running state of one piece: o holds O^T (D value rows x 8 stacked query columns) as
+// kTiles = D / 16 m16n8 accumulator tiles, thread (g, t) holding columns 2t and 2t + 1 of rows g
+// and g + 8 of each tile (which value dimension d a row is, is up to the kernel and its finalize
+// step); m, l: running max (log2 domain) and sum of the two columns; z: the kernel's zero-point
+// sum.
+template <int kTiles>
 struct WarpState {
-    float o[8][4];
+    float o[kTiles][4];
     float m[2];
     float l[2];
     float z[2];
 };
 
-__device__ __forceinline__ void state_reset(WarpState &st)
+template <int kTiles>
+__device__ __forceinline__ void state_reset(WarpState<kTiles> &st)
 {
 #pragma unroll
-    for (int i = 0; i < 8; i++)
+    for (int i = 0; i < kTiles; i++)
 #pragma unroll
         for (int k = 0; k < 4; k++)
             st.o[i][k] = 0.0f;
@@ -377,8 +385,8 @@ __device__ __forceinline__ void state_reset(WarpState &st)
 // the page exceeds it, so the cross-lane reduction runs only then (rare once a piece is a few
 // pages long); the result equals reducing every page.  kMask: a column may have seen only
 // masked tokens so far (m = -inf); its p stay 0 and nothing is rescaled by a NaN.
-template <bool kMask>
-__device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, float pr[4])
+template <bool kMask, int kTiles>
+__device__ __forceinline__ void softmax_update(const float s[4], WarpState<kTiles> &st, float pr[4])
 {
     const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
     if (__any_sync(0xFFFFFFFFu, grow)) {
@@ -399,7 +407,7 @@ __device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, 
             st.z[e] *= alpha[e];
         }
 #pragma unroll
-        for (int i = 0; i < 8; i++) {
+        for (int i = 0; i < kTiles; i++) {
             st.o[i][0] *= alpha[0];
             st.o[i][1] *= alpha[1];
             st.o[i][2] *= alpha[0];
@@ -418,9 +426,10 @@ __device__ __forceinline__ void softmax_update(const float s[4], WarpState &st, 
 }
 
 // Fold (m, l, o) partial b (scaled by its own max) into the running partial a.
-__device__ __forceinline__ void merge_into(float am[2], float al[2], float ao[8][4],
+template <int kTiles>
+__device__ __forceinline__ void merge_into(float am[2], float al[2], float (&ao)[kTiles][4],
                                            const float bm[2], const float bl[2],
-                                           const float4 bo[8])
+                                           const float4 (&bo)[kTiles])
 {
     float fa[2], fb[2];
 #pragma unroll
@@ -432,7 +441,7 @@ __device__ __forceinline__ void merge_into(float am[2], float al[2], float ao[8]
         al[e] = al[e] * fa[e] + bl[e] * fb[e];
     }
 #pragma unroll
-    for (int i = 0; i < 8; i++) {
+    for (int i = 0; i < kTiles; i++) {
         ao[i][0] = ao[i][0] * fa[0] + bo[i].x * fb[0];
         ao[i][1] = ao[i][1] * fa[1] + bo[i].y * fb[1];
         ao[i][2] = ao[i][2] * fa[0] + bo[i].z * fb[0];
@@ -441,33 +450,37 @@ __device__ __forceinline__ void merge_into(float am[2], float al[2], float ao[8]
 }
 
 // Store this warp's (m, l, o) for one piece into workspace slot `slot`.
-__device__ __forceinline__ void store_partial(float *slot, int lane, const WarpState &st)
+template <int kTiles>
+__device__ __forceinline__ void store_partial(float *slot, int lane, const WarpState<kTiles> &st)
 {
     const int g = lane >> 2, t = lane & 3;
+    constexpr int kM = kTiles * 128;
     float4 *so = reinterpret_cast<float4 *>(slot);
 #pragma unroll
-    for (int i = 0; i < 8; i++)
+    for (int i = 0; i < kTiles; i++)
         so[i * 32 + lane] = make_float4(st.o[i][0], st.o[i][1], st.o[i][2], st.o[i][3]);
     if (g == 0) {
-        slot[1024 + 2 * t] = st.m[0];
-        slot[1024 + 2 * t + 1] = st.m[1];
-        slot[1032 + 2 * t] = st.l[0];
-        slot[1032 + 2 * t + 1] = st.l[1];
+        slot[kM + 2 * t] = st.m[0];
+        slot[kM + 2 * t + 1] = st.m[1];
+        slot[kM + 8 + 2 * t] = st.l[0];
+        slot[kM + 8 + 2 * t + 1] = st.l[1];
     }
 }
 
+template <int kTiles>
 __device__ __forceinline__ void load_partial(const float *slot, int lane, float bm[2], float bl[2],
-                                             float4 bo[8])
+                                             float4 (&bo)[kTiles])
 {
     const int t = lane & 3;
+    constexpr int kM = kTiles * 128;
     const float4 *so = reinterpret_cast<const float4 *>(slot);
 #pragma unroll
-    for (int i = 0; i < 8; i++)
+    for (int i = 0; i < kTiles; i++)
         bo[i] = so[i * 32 + lane];
-    bm[0] = slot[1024 + 2 * t];
-    bm[1] = slot[1024 + 2 * t + 1];
-    bl[0] = slot[1032 + 2 * t];
-    bl[1] = slot[1032 + 2 * t + 1];
+    bm[0] = slot[kM + 2 * t];
+    bm[1] = slot[kM + 2 * t + 1];
+    bl[0] = slot[kM + 8 + 2 * t];
+    bl[1] = slot[kM + 8 + 2 * t + 1];
 }
 
 // Combine the pieces of every segment that was split across warps: slot g + u holds warp u's
@@ -481,10 +494,12 @@ __global__ void __launch_bounds__(kMergeThreads)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 15) & ~uintptr_t(15));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    constexpr int kTiles = Fmt::kTiles;
+    constexpr int kSlot = slot_floats<kTiles>();
     SeqTables tb;
-    tb.bind(smem + kMergeSmemTables, p.num_seqs);
-    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + kMergeSmemFlags);
-    float *slots = reinterpret_cast<float *>(smem + kMergeSmemSlots);
+    tb.bind(smem + merge_smem_tables<kTiles>(), p.num_seqs);
+    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + merge_smem_flags<kTiles>());
+    float *slots = reinterpret_cast<float *>(smem);
 
     scan_sequences<kPrefill>(p, tb, flags, false);
     Plan plan;
@@ -501,32 +516,32 @@ __global__ void __launch_bounds__(kMergeThreads)
         const int64_t u_hi = plan.warp_of_cost(plan.page_cost(s, j, n_s - 1));
         if (u_lo == u_hi)
             continue;
-        WarpState st;
+        WarpState<kTiles> st;
         state_reset(st);
         // each warp folds every kMergeWarps-th partial; two loads in flight per step
         int64_t uu = u_lo + warp;
         for (; uu + kMergeWarps <= u_hi; uu += 2 * kMergeWarps) {
             float bm0[2], bl0[2], bm1[2], bl1[2];
-            float4 bo0[8], bo1[8];
-            load_partial(p.partials + (gseg + uu) * kSlotFloats, lane, bm0, bl0, bo0);
-            load_partial(p.partials + (gseg + uu + kMergeWarps) * kSlotFloats, lane, bm1, bl1, bo1);
+            float4 bo0[kTiles], bo1[kTiles];
+            load_partial(p.partials + (gseg + uu) * kSlot, lane, bm0, bl0, bo0);
+            load_partial(p.partials + (gseg + uu + kMergeWarps) * kSlot, lane, bm1, bl1, bo1);
             merge_into(st.m, st.l, st.o, bm0, bl0, bo0);
             merge_into(st.m, st.l, st.o, bm1, bl1, bo1);
         }
         if (uu <= u_hi) {
             float bm[2], bl[2];
-            float4 bo[8];
-            load_partial(p.partials + (gseg + uu) * kSlotFloats, lane, bm, bl, bo);
+            float4 bo[kTiles];
+            load_partial(p.partials + (gseg + uu) * kSlot, lane, bm, bl, bo);
             merge_into(st.m, st.l, st.o, bm, bl, bo);
         }
         if (warp > 0)
-            store_partial(slots + (warp - 1) * kSlotFloats, lane, st);
+            store_partial(slots + (warp - 1) * kSlot, lane, st);
         __syncthreads();
         if (warp == 0) {
             for (int w = 1; w < kMergeWarps; w++) {
                 float bm[2], bl[2];
-                float4 bo[8];
-                load_partial(slots + (w - 1) * kSlotFloats, lane, bm, bl, bo);
+                float4 bo[kTiles];
+                load_partial(slots + (w - 1) * kSlot, lane, bm, bl, bo);
                 merge_into(st.m, st.l, st.o, bm, bl, bo);
             }
             Segment<kPrefill> sg;
@@ -560,7 +575,9 @@ __global__ void __launch_bounds__(kMergeThreads)
 // of flags, the per-warp query buffers (qrows * 256 bytes each) and the sequence tables.
 
 constexpr int kSmemFlagBytes = 128;
-__host__ __device__ constexpr int query_bytes(int rows) { return rows * kHeadDim * 2; }
+// bytes of `rows` raw bf16 query rows of a format's head dimension
+template <class Fmt>
+__host__ __device__ constexpr int query_bytes(int rows) { return rows * Fmt::kDim * 2; }
 template <class Fmt>
 __host__ __device__ constexpr int smem_bars_offset() { return Fmt::kRingBytes; }
 template <class Fmt>
@@ -573,7 +590,7 @@ __host__ __device__ constexpr int smem_q_offset() { return smem_flags_offset<Fmt
 template <class Fmt>
 __host__ __device__ constexpr int smem_tables_offset(int qrows)
 {
-    return smem_q_offset<Fmt>() + Fmt::kWarps * query_bytes(qrows);
+    return smem_q_offset<Fmt>() + Fmt::kWarps * query_bytes<Fmt>(qrows);
 }
 template <class Fmt>
 inline size_t decode_smem_bytes(int32_t num_seqs, int32_t qrows)
@@ -599,8 +616,8 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     for (int s = blockIdx.x; s < S; s += gridDim.x) {
         const int c = query_tokens<kPrefill>(p, s);
         if (tb.nbk[s] == 0 && c > 0 && (!kPrefill || c <= p.seq_lens[s])) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out + query_row0<kPrefill>(p, s) * p.hq * kHeadDim);
-            for (int i = tid; i < c * p.hq * kHeadDim / 4; i += 32 * Fmt::kWarps)
+            float4 *dst = reinterpret_cast<float4 *>(p.out + query_row0<kPrefill>(p, s) * p.hq * Fmt::kDim);
+            for (int i = tid; i < c * p.hq * Fmt::kDim / 4; i += 32 * Fmt::kWarps)
                 dst[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
         }
     }
@@ -622,7 +639,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     // ---- 2. this warp's copy ring ---------------------------------------------------------------
     constexpr int kStages = Fmt::kStages;
     const typename Fmt::Ring ring = Fmt::ring(smem_u32(smem), warp);
-    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes(p.qrows);
+    const uint32_t qbuf = smem_u32(smem + smem_q_offset<Fmt>()) + warp * query_bytes<Fmt>(p.qrows);
     const uint32_t bar0 = smem_u32(smem + smem_bars_offset<Fmt>()) + warp * (kStages + 1) * 8;
     const uint32_t qbar = bar0 + kStages * 8;
     if (lane == 0)
@@ -654,12 +671,12 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     // rows of the same query token (its heads are contiguous)
     auto issue_query = [&](const Segment<kPrefill> &sg) {
         if (lane == 0) {
-            mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(sg.nrows) * kHeadDim * 2);
+            mbar_arrive_expect_tx(qbar, static_cast<uint32_t>(sg.nrows) * Fmt::kDim * 2);
             for (int e = 0; e < sg.nrows;) {
                 const int head = sg.row0 + e - sg.row_token(p, e) * p.group;
                 const int cnt = min(p.group - head, sg.nrows - e);
-                bulk_g2s(qbuf + e * kHeadDim * 2, p.q + sg.row_offset(p, e),
-                         static_cast<uint32_t>(cnt) * kHeadDim * 2, qbar);
+                bulk_g2s(qbuf + e * Fmt::kDim * 2, p.q + sg.row_offset(p, e, Fmt::kDim),
+                         static_cast<uint32_t>(cnt) * Fmt::kDim * 2, qbar);
                 e += cnt;
             }
         }
@@ -700,7 +717,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     while (issued < kStages - 1 && issued < n_w)
         issue_next();
 
-    WarpState st;
+    WarpState<Fmt::kTiles> st;
     typename Fmt::Query qf;
     // Page m of the run: queue the page kStages - 1 ahead into the stage page m - 1 used, wait
     // for page m and attend over it (through `mask` when kMask).
@@ -787,7 +804,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
             sg.init(p, tb, cs, cj);
             Fmt::finalize(p, sg, lane, st.o, st.l);
         } else {
-            store_partial(p.partials + (tb.spre[cs] + cj + u) * kSlotFloats, lane, st);
+            store_partial(p.partials + (tb.spre[cs] + cj + u) * slot_floats<Fmt::kTiles>(), lane, st);
         }
         pos = F0 + m_end;
         cs = ns;

@@ -44,9 +44,9 @@ namespace {
 
 using namespace decode;
 
-constexpr int kCodeBytes = 2 * kPageSize * kRowBytes;   // K + V codes of one (page, kv head)
+// K + V codes of one (page, kv head): 2 x 16 rows of D / 2 bytes
+__host__ __device__ constexpr int code_bytes(int d) { return 2 * kPageSize * d / 2; }
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
-constexpr uint32_t kTxBytes = kCodeBytes + kScaleBytes;
 constexpr float kHadamardC = 0.0883883461356163f;
 
 // Unpack one 32-bit word of packed codes (bytes b0..b3, low nibble first) into four fp16x2
@@ -73,17 +73,20 @@ __device__ __forceinline__ float2 h2_to_f2(uint32_t u)
 }
 
 // Rotated, scaled query of one segment as fp16 mma B fragments, from the raw bf16 queries of
-// its nheads <= 8 heads in shared memory ([nheads][128] at qbuf).
-// Thread (g, t) owns query head g of the group and d in [32t, 32t + 32).
-template <bool kRotate>
+// its nheads <= 8 heads in shared memory ([nheads][kD] at qbuf).
+// Thread (g, t) owns query head g of the group and d in [kQ t, kQ t + kQ), kQ = kD / 4.  The
+// rotation is the 128-point Hadamard transform of each 128-element block of d (for kD = 256
+// the two halves are independent blocks, as the quantizer rotates them).
+template <bool kRotate, int kD>
 __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int g,
-                                           int t, uint32_t bq[8][2], float sq_out[2])
+                                           int t, uint32_t bq[kD / 16][2], float sq_out[2])
 {
-    float x[32];
+    constexpr int kQ = kD / 4;
+    float x[kQ];
     if (g < nheads) {
 #pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const uint4 u = lds128(qbuf + g * (kHeadDim * 2) + 64 * t + 16 * c);
+        for (int c = 0; c < kQ / 8; c++) {
+            const uint4 u = lds128(qbuf + g * (kD * 2) + 2 * kQ * t + 16 * c);
             const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
             for (int k = 0; k < 4; k++) {
@@ -93,44 +96,45 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
         }
     } else {
 #pragma unroll
-        for (int l = 0; l < 32; l++)
+        for (int l = 0; l < kQ; l++)
             x[l] = 0.0f;
     }
-    // Hadamard butterfly: d bits 0..4 in registers, bits 5, 6 across lanes t ^ 1, t ^ 2
-    // (skipped for the plain INT4 cache).
+    // Hadamard butterfly (skipped for the plain INT4 cache): the low log2(kQ) bits of d in
+    // registers, the remaining bits of the 128-block across lanes t ^ 1 (and t ^ 2 for kD = 128).
 #pragma unroll
-    for (int hb = 1; kRotate && hb < 32; hb <<= 1)
+    for (int hb = 1; kRotate && hb < kQ; hb <<= 1)
 #pragma unroll
-        for (int l = 0; l < 32; l++)
+        for (int l = 0; l < kQ; l++)
             if ((l & hb) == 0) {
                 const float a = x[l], b = x[l + hb];
                 x[l] = a + b;
                 x[l + hb] = a - b;
             }
 #pragma unroll
-    for (int lb = 1; kRotate && lb <= 2; lb <<= 1) {
+    for (int lb = 1; kRotate && kQ * lb < 128; lb <<= 1) {
         const bool high = (t & lb) != 0;
 #pragma unroll
-        for (int l = 0; l < 32; l++) {
+        for (int l = 0; l < kQ; l++) {
             const float o = __shfl_xor_sync(0xFFFFFFFFu, x[l], lb);
             x[l] = high ? o - x[l] : x[l] + o;
         }
     }
     // Even d pair with low nibbles (weight 2^-24), odd d with high nibbles (weight 2^-20): odd
-    // entries carry q / 16 so that every product is q_d * code_d * 2^-24.
+    // entries carry q / 16 so that every product is q_d * code_d * 2^-24.  sum(q) runs over all
+    // kD elements: one (scale, zero) pair covers the whole head vector.
     float sq = 0.0f;
-    __half hq[32];
+    __half hq[kQ];
 #pragma unroll
-    for (int l = 0; l < 32; l++) {
+    for (int l = 0; l < kQ; l++) {
         const float qv = x[l] * p.q_mult;
         hq[l] = __float2half_rn((l & 1) ? qv * 0.0625f : qv);
         sq += (l & 1) ? 16.0f * __half2float(hq[l]) : __half2float(hq[l]);
     }
     sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 1);
     sq += __shfl_xor_sync(0xFFFFFFFFu, sq, 2);
-    // k-step (i, e): k slots (2t, 2t+1 | 2t+8, 2t+9) <-> d = 32t + 8i + 2e + (0, 4 | 1, 5)
+    // k-step (i, e): k slots (2t, 2t+1 | 2t+8, 2t+9) <-> d = kQ t + 8i + 2e + (0, 4 | 1, 5)
 #pragma unroll
-    for (int i = 0; i < 4; i++)
+    for (int i = 0; i < kQ / 8; i++)
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             const int l0 = 8 * i + 2 * e;
@@ -142,31 +146,49 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
     sq_out[1] = __shfl_sync(0xFFFFFFFFu, sq, 8 * t + 4);
 }
 
+// Byte offset of 16-byte chunk c of code row r in a staged page: rows of kD / 2 bytes with the
+// tensor copy's swizzle (64B for 64-byte rows: chunk ^ bits 1-2 of the row; 128B for 128-byte
+// rows: chunk ^ bits 0-2 of the row).
+template <int kD>
+__device__ __forceinline__ uint32_t code_offset(int r, int c)
+{
+    const int sw = kD == 128 ? (r >> 1) & 3 : r & 7;
+    return static_cast<uint32_t>(r * (kD / 2) + ((c ^ sw) << 4));
+}
+
 // One page of one warp: QK^T, online softmax, PV.  kMask: tokens [0, mask.valid) of the page
 // exist (the rest were never written: their V scale and zero are replaced by 0) and column e
 // (block row 2t + e) sees tokens [0, mask.col[e]).
-template <bool kMask>
+template <bool kMask, int kD>
 __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, const PageMask &mask,
-                                             const uint32_t bq[8][2], const float sq[2],
-                                             int lane, WarpState &st)
+                                             const uint32_t bq[kD / 16][2], const float sq[2],
+                                             int lane, WarpState<kD / 16> &st)
 {
     const int g = lane >> 2, t = lane & 3;
+    constexpr int kChunks = kD / 128;   // 16-byte code chunks of one row per thread
 
     // ---- S^T = K . Q^T over 16 tokens (rows g, g + 8) -----------------------------------
-    const uint4 k0 = lds128(cbase + g * 64 + ((t ^ ((g >> 1) & 3)) << 4));
-    const uint4 k1 = lds128(cbase + (g + 8) * 64 + ((t ^ (((g + 8) >> 1) & 3)) << 4));
-    const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
-    const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
+    // Thread t reads chunks kChunks t .. kChunks t + kChunks - 1 (d in [kD/4 t, kD/4 (t + 1))):
+    // within each quarter warp the two rows land in disjoint banks.
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int i = 0; i < 4; i++) {
-        uint32_t ya[4], yb[4];
-        unpack_codes(kw0[i], ya);
-        unpack_codes(kw1[i], yb);
-        const uint32_t a0[4] = {ya[0], yb[0], ya[1], yb[1]};
-        const uint32_t a1[4] = {ya[2], yb[2], ya[3], yb[3]};
-        mma_16816(acc, a0, bq[2 * i][0], bq[2 * i][1]);
-        mma_16816(acc, a1, bq[2 * i + 1][0], bq[2 * i + 1][1]);
+    for (int hf = 0; hf < kChunks; hf++) {
+        const int c = kChunks * t + hf;
+        const uint4 k0 = lds128(cbase + code_offset<kD>(g, c));
+        const uint4 k1 = lds128(cbase + code_offset<kD>(g + 8, c));
+        const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
+        const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            uint32_t ya[4], yb[4];
+            unpack_codes(kw0[i], ya);
+            unpack_codes(kw1[i], yb);
+            const uint32_t a0[4] = {ya[0], yb[0], ya[1], yb[1]};
+            const uint32_t a1[4] = {ya[2], yb[2], ya[3], yb[3]};
+            const int w = 4 * hf + i;
+            mma_16816(acc, a0, bq[2 * w][0], bq[2 * w][1]);
+            mma_16816(acc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
+        }
     }
 
     // ---- logits (log2 domain) ---------------------------------------------------------------
@@ -191,7 +213,7 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
     }
 
     float pr[4];
-    softmax_update<kMask>(s, st, pr);
+    softmax_update<kMask, kD / 16>(s, st, pr);
 
     // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
     float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));
@@ -214,15 +236,12 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
     // ---- O^T += V^T . P'^T -----------------------------------------------------------------
     // ldmatrix.trans: lane L addresses row (L & 7) of matrix L >> 3; matrices are
     // (tokens 0-7 | 8-15) x (16-byte chunk 2j | 2j + 1) of the V rows (rows 16..31).
-    const int vtok = ((lane >> 3) & 1) * 8 + (lane & 7);
-    const int vrow = 16 + vtok;
-    const uint32_t vrow_base = cbase + vrow * 64;
-    const int vsw = (vrow >> 1) & 3;
+    const int vrow = 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
 #pragma unroll
-    for (int j = 0; j < 2; j++) {
+    for (int j = 0; j < kD / 64; j++) {
         const int chunk = 2 * j + (lane >> 4);
         uint32_t r[4];
-        ldsm_x4_trans(vrow_base + ((chunk ^ vsw) << 4), r[0], r[1], r[2], r[3]);
+        ldsm_x4_trans(cbase + code_offset<kD>(vrow, chunk), r[0], r[1], r[2], r[3]);
         // r[0]: tokens 0-7, chunk 2j; r[1]: tokens 8-15, chunk 2j; r[2], r[3]: chunk 2j + 1
 #pragma unroll
         for (int cc = 0; cc < 2; cc++) {
@@ -241,17 +260,18 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
 
 
 // o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the block rows 2t, 2t + 1
-// this thread holds.
-template <bool kRotate, class Seg>
+// this thread holds; H acts on each 128-element block of d.
+template <bool kRotate, int kD, class Seg>
 __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, int lane,
-                                         float o[8][4], const float l[2])
+                                         float o[kD / 16][4], const float l[2])
 {
+    constexpr int kC = kD / 32;   // 32-element chunks of d
     const int g = lane >> 2, t = lane & 3;
     const float inv[2] = {1.0f / l[0], 1.0f / l[1]};
     // v[e][c][j]: head 2t + e, d = 32c + 4g + j
-    float v[2][4][4];
+    float v[2][kC][4];
 #pragma unroll
-    for (int c = 0; c < 4; c++)
+    for (int c = 0; c < kC; c++)
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             v[e][c][0] = o[2 * c][e] * inv[e];
@@ -261,9 +281,10 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
         }
 #pragma unroll
     for (int e = 0; kRotate && e < 2; e++) {
-        // d bits 0, 1 (j) and 5, 6 (c) in registers
+        // d bits 0, 1 (j) and 5, 6 (low bits of c) in registers; bit 7 (kD = 256) selects the
+        // 128-block and is not transformed
 #pragma unroll
-        for (int c = 0; c < 4; c++)
+        for (int c = 0; c < kC; c++)
 #pragma unroll
             for (int jb = 1; jb <= 2; jb <<= 1)
 #pragma unroll
@@ -276,7 +297,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
 #pragma unroll
         for (int cb = 1; cb <= 2; cb <<= 1)
 #pragma unroll
-            for (int c = 0; c < 4; c++)
+            for (int c = 0; c < kC; c++)
                 if ((c & cb) == 0)
 #pragma unroll
                     for (int j = 0; j < 4; j++) {
@@ -289,7 +310,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
         for (int gb = 1; gb <= 4; gb <<= 1) {
             const bool high = (g & gb) != 0;
 #pragma unroll
-            for (int c = 0; c < 4; c++)
+            for (int c = 0; c < kC; c++)
 #pragma unroll
                 for (int j = 0; j < 4; j++) {
                     const float other = __shfl_xor_sync(0xFFFFFFFFu, v[e][c][j], 4 * gb);
@@ -301,9 +322,9 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
     for (int e = 0; e < 2; e++) {
         const int head = 2 * t + e;
         if (head < sg.nrows) {
-            float *dst = p.out + sg.row_offset(p, head);
+            float *dst = p.out + sg.row_offset(p, head, kD);
 #pragma unroll
-            for (int c = 0; c < 4; c++) {
+            for (int c = 0; c < kC; c++) {
                 const float f = kRotate ? kHadamardC : 1.0f;
                 const float4 val = make_float4(v[e][c][0] * f, v[e][c][1] * f, v[e][c][2] * f,
                                                v[e][c][3] * f);
@@ -314,9 +335,9 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
 }
 
 
-
 // One elected lane of the (converged) warp arms the stage's mbarrier with the page's bytes and
 // queues the 2-D tensor copy of its code rows and the 1-D bulk copy of its scales; no branch.
+template <int kD>
 __device__ __forceinline__ void copy_page_elected(uint32_t bar, uint32_t dst_codes, const void *tmap,
                                                   int32_t row, uint32_t dst_scales,
                                                   const void *src_scales)
@@ -329,27 +350,34 @@ __device__ __forceinline__ void copy_page_elected(uint32_t bar, uint32_t dst_cod
                  "@p cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%4], [%5], %8, [%0];\n\t"
                  "}"
                  ::"r"(bar), "r"(dst_codes), "l"(tmap), "r"(row), "r"(dst_scales), "l"(src_scales),
-                 "r"(kTxBytes), "r"(0), "r"(static_cast<uint32_t>(kScaleBytes))
+                 "r"(static_cast<uint32_t>(code_bytes(kD) + kScaleBytes)), "r"(0), "r"(static_cast<uint32_t>(kScaleBytes))
                  : "memory");
 }
 
 
 
-// The INT4 page format for the generic decode kernel (decode_common.cuh): 4 warps per CTA, 4 CTAs
-// per SM, a 4-stage ring per warp; codes of all stages first (2 KiB each, 64B swizzle), then
-// the scales (128 B each); one (page, kv head) is 32 tensor-map rows of 64 B.
-template <bool kRotate>
+// The INT4 page format for the generic decode kernel (decode_common.cuh), head dimension kD:
+// 4 warps per CTA and a ring per warp whose stages hold the codes of one (page, kv head) (32
+// tensor-map rows of kD / 2 bytes: 2 KiB with the 64B swizzle for kD = 128, 4 KiB with the 128B
+// swizzle for kD = 256), codes of all stages first, then the scales (128 B each).  kD = 128:
+// 4 stages, 4 CTAs per SM; kD = 256 (twice the accumulators): 2 stages, 3 CTAs per SM, which
+// keeps about as many bytes in flight per SM.
+template <bool kRotate, int kD>
 struct Int4Format {
+    static_assert(kD == 128 || kD == 256, "head dimension");
+    static constexpr int kDim = kD;
+    static constexpr int kTiles = kD / 16;
     static constexpr int kWarps = 4;
-    static constexpr int kStages = 4;
-    static constexpr int kMinBlocks = 4;
+    static constexpr int kStages = kD == 128 ? 4 : 2;
+    static constexpr int kMinBlocks = kD == 128 ? 4 : 3;
     static constexpr int kRowsPerPage = 32;
+    static constexpr int kCodeBytes = code_bytes(kD);
     static constexpr int kRingBytes = kWarps * kStages * (kCodeBytes + kScaleBytes);
     struct Ring {
         uint32_t code0, scale0;
     };
     struct Query {
-        uint32_t bq[8][2];
+        uint32_t bq[kD / 16][2];
         float sq[2];
     };
     __device__ static Ring ring(uint32_t base, int warp)
@@ -360,22 +388,22 @@ struct Int4Format {
     __device__ static void issue(const Ring &r, int stg, uint32_t bar, const CUtensorMap *tmap,
                                  int32_t row, const DecodeParams &p)
     {
-        copy_page_elected(bar, r.code0 + stg * kCodeBytes, tmap, row, r.scale0 + stg * kScaleBytes,
-                          p.scales + static_cast<int64_t>(row) * 4);
+        copy_page_elected<kD>(bar, r.code0 + stg * kCodeBytes, tmap, row,
+                              r.scale0 + stg * kScaleBytes, p.scales + static_cast<int64_t>(row) * 4);
     }
     __device__ static void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int lane,
                                       Query &q)
     {
-        saw::load_query<kRotate>(p, qbuf, nheads, lane >> 2, lane & 3, q.bq, q.sq);
+        saw::load_query<kRotate, kD>(p, qbuf, nheads, lane >> 2, lane & 3, q.bq, q.sq);
     }
     template <bool kMask>
     __device__ static void page(const Ring &r, int stg, const PageMask &mask, const Query &q,
-                                int lane, WarpState &st)
+                                int lane, WarpState<kTiles> &st)
     {
-        process_page<kMask>(r.code0 + stg * kCodeBytes, r.scale0 + stg * kScaleBytes, mask, q.bq,
-                            q.sq, lane, st);
+        process_page<kMask, kD>(r.code0 + stg * kCodeBytes, r.scale0 + stg * kScaleBytes, mask,
+                                q.bq, q.sq, lane, st);
     }
-    __device__ static void piece_end(WarpState &st)
+    __device__ static void piece_end(WarpState<kTiles> &st)
     {
         // reduce l and z over the 8 token rows (lanes differing in g)
 #pragma unroll
@@ -389,7 +417,7 @@ struct Int4Format {
         // undo the subnormal code scales (value rows g: low nibbles, g + 8: high nibbles)
         // and add the zero-point term
 #pragma unroll
-        for (int i2 = 0; i2 < 8; i2++) {
+        for (int i2 = 0; i2 < kTiles; i2++) {
             st.o[i2][0] = fmaf(st.o[i2][0], kLowNibble, st.z[0]);
             st.o[i2][1] = fmaf(st.o[i2][1], kLowNibble, st.z[1]);
             st.o[i2][2] = fmaf(st.o[i2][2], kHighNibble, st.z[0]);
@@ -397,84 +425,94 @@ struct Int4Format {
         }
     }
     template <class Seg>
-    __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane, float o[8][4],
-                                    const float l[2])
+    __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane,
+                                    float o[kTiles][4], const float l[2])
     {
-        saw::finalize<kRotate>(p, sg, lane, o, l);
+        saw::finalize<kRotate, kD>(p, sg, lane, o, l);
     }
 };
 
-ShapeCache g_shapes;
-
-// Multiprocessor count and decode-kernel occupancy on the current device (see
-// decode::launch_shape).
+// Multiprocessor count and decode-kernel occupancy on the current device for head dimension kD
+// (see decode::launch_shape).
+template <int kD>
 cudaError_t launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
 {
+    static ShapeCache shapes;
     static const void *const decode_kernels[kShapeVariants] = {
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true>, false>),
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false>, false>),
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true>, true>),
-        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false>, true>)};
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true, kD>, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false, kD>, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<true, kD>, true>),
+        reinterpret_cast<const void *>(paged_decode_kernel<Int4Format<false, kD>, true>)};
     static const void *const merge_kernels[kShapeVariants] = {
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true>, false>),
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false>, false>),
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true>, true>),
-        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false>, true>)};
-    return decode::launch_shape(g_shapes, decode_kernels, merge_kernels,
-                                32 * Int4Format<true>::kWarps, smem, merge_smem, out);
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true, kD>, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false, kD>, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<true, kD>, true>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false, kD>, true>)};
+    return decode::launch_shape(shapes, decode_kernels, merge_kernels,
+                                32 * Int4Format<true, kD>::kWarps, smem, merge_smem, out);
 }
 
-}  // namespace
-
-size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
-                              int64_t total_q)
+template <int kD>
+size_t workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs, int64_t total_q)
 {
-    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
-        return 0;
+    using Fmt = Int4Format<true, kD>;
     const bool prefill = total_q >= 0;
     LaunchShape ls;
-    if (launch_shape(decode_smem_bytes<Int4Format<true>>(num_seqs, query_rows(num_kv_heads, num_q_heads, prefill)),
-                     merge_smem_bytes(num_seqs), ls) != cudaSuccess)
+    if (launch_shape<kD>(decode_smem_bytes<Fmt>(num_seqs, query_rows(num_kv_heads, num_q_heads, prefill)),
+                         merge_smem_bytes<Fmt::kTiles>(num_seqs), ls) != cudaSuccess)
         return 0;
-    return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Int4Format<true>::kWarps,
-                               max_segments(num_kv_heads, num_q_heads, num_seqs, total_q, prefill));
+    return workspace_bytes_for<Fmt::kTiles>(static_cast<size_t>(ls.sms) * ls.occ * Fmt::kWarps,
+                                            max_segments(num_kv_heads, num_q_heads, num_seqs,
+                                                         total_q, prefill));
 }
 
-cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
+// Tensor map of the code rows: [num_pages * Hkv * 32 rows][kD / 2 bytes], box = one (page, kv
+// head), cached per thread for the last cache seen.
+template <int kD>
+const CUtensorMap *code_tensor_map(const uint8_t *kv_pages, int64_t rows)
 {
     static thread_local struct {
         const void *base = nullptr;
         int64_t rows = 0;
         CUtensorMap map;
     } cache;
-    const int64_t rows = a.num_pages * a.num_kv_heads * 32;
-    if (cache.base != a.kv_pages || cache.rows != rows) {
+    if (cache.base != kv_pages || cache.rows != rows) {
         auto encode = tensor_map_encoder();
         if (encode == nullptr)
-            return cudaErrorNotSupported;
-        const cuuint64_t dims[2] = {64, static_cast<cuuint64_t>(rows)};
-        const cuuint64_t strides[1] = {64};
-        const cuuint32_t box[2] = {64, 32};
+            return nullptr;
+        const cuuint64_t dims[2] = {kD / 2, static_cast<cuuint64_t>(rows)};
+        const cuuint64_t strides[1] = {kD / 2};
+        const cuuint32_t box[2] = {kD / 2, 32};
         const cuuint32_t estr[2] = {1, 1};
         CUresult r = encode(&cache.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
-                            const_cast<uint8_t *>(a.kv_pages), dims, strides, box, estr,
-                            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_64B,
+                            const_cast<uint8_t *>(kv_pages), dims, strides, box, estr,
+                            CU_TENSOR_MAP_INTERLEAVE_NONE,
+                            kD == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
             cache.base = nullptr;
-            return cudaErrorInvalidValue;
+            return nullptr;
         }
-        cache.base = a.kv_pages;
+        cache.base = kv_pages;
         cache.rows = rows;
     }
+    return &cache.map;
+}
 
-    using Fmt = Int4Format<true>;   // the layout is the same for both variants
+template <int kD>
+cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
+{
+    const CUtensorMap *map = code_tensor_map<kD>(a.kv_pages, a.num_pages * a.num_kv_heads * 32);
+    if (map == nullptr)
+        return cudaErrorInvalidValue;
+
+    using Fmt = Int4Format<true, kD>;   // the layout is the same for both variants
     const bool prefill = a.q_start != nullptr;
     const int32_t qrows = query_rows(a.num_kv_heads, a.num_q_heads, prefill);
     const size_t smem = decode_smem_bytes<Fmt>(a.num_seqs, qrows);
-    const size_t msmem = merge_smem_bytes(a.num_seqs);
+    const size_t msmem = merge_smem_bytes<Fmt::kTiles>(a.num_seqs);
     LaunchShape ls;
-    cudaError_t e = launch_shape(smem, msmem, ls);
+    cudaError_t e = launch_shape<kD>(smem, msmem, ls);
     if (e != cudaSuccess)
         return e;
 
@@ -511,11 +549,11 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    auto *kernel = a.rotate ? (prefill ? paged_decode_kernel<Int4Format<true>, true>
-                                       : paged_decode_kernel<Int4Format<true>, false>)
-                            : (prefill ? paged_decode_kernel<Int4Format<false>, true>
-                                       : paged_decode_kernel<Int4Format<false>, false>);
-    e = cudaLaunchKernelEx(&cfg, kernel, cache.map, p);
+    auto *kernel = a.rotate ? (prefill ? paged_decode_kernel<Int4Format<true, kD>, true>
+                                       : paged_decode_kernel<Int4Format<true, kD>, false>)
+                            : (prefill ? paged_decode_kernel<Int4Format<false, kD>, true>
+                                       : paged_decode_kernel<Int4Format<false, kD>, false>);
+    e = cudaLaunchKernelEx(&cfg, kernel, *map, p);
     if (e != cudaSuccess)
         return e;
 
@@ -525,14 +563,37 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    auto *merge = a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true>, true>
-                                      : paged_decode_merge_kernel<Int4Format<true>, false>)
-                           : (prefill ? paged_decode_merge_kernel<Int4Format<false>, true>
-                                      : paged_decode_merge_kernel<Int4Format<false>, false>);
+    auto *merge = a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true>
+                                      : paged_decode_merge_kernel<Int4Format<true, kD>, false>)
+                           : (prefill ? paged_decode_merge_kernel<Int4Format<false, kD>, true>
+                                      : paged_decode_merge_kernel<Int4Format<false, kD>, false>);
     e = cudaLaunchKernelEx(&mcfg, merge, p);
     if (e != cudaSuccess)
         return e;
     return cudaGetLastError();
+}
+
+}  // namespace
+
+size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
+                              int64_t total_q, int32_t head_dim)
+{
+    if (num_kv_heads <= 0 || num_q_heads <= 0 || num_seqs < 0 || num_q_heads % num_kv_heads)
+        return 0;
+    if (head_dim == 128)
+        return workspace_bytes<128>(num_kv_heads, num_q_heads, num_seqs, total_q);
+    if (head_dim == 256)
+        return workspace_bytes<256>(num_kv_heads, num_q_heads, num_seqs, total_q);
+    return 0;
+}
+
+cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
+{
+    if (a.head_dim == 128)
+        return launch<128>(a, stream, programmatic);
+    if (a.head_dim == 256)
+        return launch<256>(a, stream, programmatic);
+    return cudaErrorInvalidValue;
 }
 
 }  // namespace saw

@@ -51,6 +51,8 @@ __device__ __forceinline__ uint32_t bf16_chunk(int sel, int tok, int d0)
 }
 
 struct Bf16Format {
+    static constexpr int kDim = kHeadDim;
+    static constexpr int kTiles = kHeadDim / 16;
     static constexpr int kWarps = 4;
     static constexpr int kStages = 2;
     static constexpr int kMinBlocks = 3;
@@ -99,7 +101,7 @@ struct Bf16Format {
 
     template <bool kMask>
     __device__ static void page(const Ring &r, int stg, const PageMask &mask, const Query &q,
-                                int lane, WarpState &st)
+                                int lane, WarpState<8> &st)
     {
         const uint32_t base = r.base + stg * kBf16PageBytes;
         const int g = lane >> 2, t = lane & 3;
@@ -126,7 +128,7 @@ struct Bf16Format {
                 s[3] = -INFINITY;
         }
         float pr[4];
-        softmax_update<kMask>(s, st, pr);
+        softmax_update<kMask, 8>(s, st, pr);
         st.l[0] += pr[0] + pr[2];
         st.l[1] += pr[1] + pr[3];
 
@@ -166,7 +168,7 @@ struct Bf16Format {
         }
     }
 
-    __device__ static void piece_end(WarpState &st)
+    __device__ static void piece_end(WarpState<8> &st)
     {
 #pragma unroll
         for (int e = 0; e < 2; e++)
@@ -187,7 +189,7 @@ struct Bf16Format {
             if (head >= sg.nrows)
                 continue;
             const float inv = 1.0f / l[e];
-            float *dst = p.out + sg.row_offset(p, head);
+            float *dst = p.out + sg.row_offset(p, head, kHeadDim);
 #pragma unroll
             for (int c = 0; c < 8; c++) {
                 dst[16 * c + g] = o[c][e] * inv;
@@ -274,9 +276,9 @@ size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, in
     const bool prefill = total_q >= 0;
     LaunchShape ls;
     if (bf16_launch_shape(decode_smem_bytes<Bf16Format>(num_seqs, query_rows(num_kv_heads, num_q_heads, prefill)),
-                          merge_smem_bytes(num_seqs), ls) != cudaSuccess)
+                          merge_smem_bytes<8>(num_seqs), ls) != cudaSuccess)
         return 0;
-    return workspace_bytes_for(static_cast<size_t>(ls.sms) * ls.occ * Bf16Format::kWarps,
+    return workspace_bytes_for<8>(static_cast<size_t>(ls.sms) * ls.occ * Bf16Format::kWarps,
                                max_segments(num_kv_heads, num_q_heads, num_seqs, total_q, prefill));
 }
 
@@ -311,7 +313,7 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     const bool prefill = a.q_start != nullptr;
     const int32_t qrows = query_rows(a.num_kv_heads, a.num_q_heads, prefill);
     const size_t smem = decode_smem_bytes<Bf16Format>(a.num_seqs, qrows);
-    const size_t msmem = merge_smem_bytes(a.num_seqs);
+    const size_t msmem = merge_smem_bytes<8>(a.num_seqs);
     LaunchShape ls;
     cudaError_t e = bf16_launch_shape(smem, msmem, ls);
     if (e != cudaSuccess)

@@ -51,8 +51,8 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
 {
     if (num_q_heads <= 0 || num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if (cache->head_dim != 128)
-        return SAW_ERR_UNSUPPORTED;   // attention kernels: D = 128
+    if (bf16 && cache->head_dim != 128)
+        return SAW_ERR_UNSUPPORTED;   // the BF16 baseline cache: D = 128
     if (num_q_heads / cache->num_kv_heads > 16)
         return SAW_ERR_UNSUPPORTED;
     if (!std::isfinite(sm_scale))
@@ -70,7 +70,8 @@ int check_decode(const saw_cache_desc *cache, int32_t num_q_heads, const void *q
         return SAW_ERR_INVALID_ARGUMENT;
     const size_t need =
         bf16 ? saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q)
-             : saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q);
+             : saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q,
+                                           cache->head_dim);
     if (need == 0)
         return SAW_ERR_CUDA;
     if (workspace == nullptr || workspace_bytes < need || !aligned(workspace, 256))
@@ -101,6 +102,7 @@ saw::DecodeArgs decode_args(const saw_cache_desc *cache, int32_t num_q_heads, co
     a.workspace = workspace;
     a.workspace_bytes = workspace_bytes;
     a.status = dev_status;
+    a.head_dim = cache->head_dim;
     return a;
 }
 
@@ -296,10 +298,10 @@ size_t saw_paged_decode_workspace_bytes(const saw_cache_desc *cache, int32_t num
                                         int32_t num_seqs)
 {
     if (check_cache(cache) != SAW_OK || num_q_heads <= 0 ||
-        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16 ||
-        cache->head_dim != 128)
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
         return 0;
-    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, -1,
+                                       cache->head_dim);
 }
 
 int saw_paged_decode_workspace_init(void *workspace, size_t workspace_bytes, void *stream)
@@ -492,10 +494,10 @@ size_t saw_paged_prefill_workspace_bytes(const saw_cache_desc *cache, int32_t nu
                                          int32_t num_seqs, int64_t total_q)
 {
     if (check_cache(cache) != SAW_OK || num_q_heads <= 0 || total_q < 0 ||
-        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16 ||
-        cache->head_dim != 128)
+        num_q_heads % cache->num_kv_heads != 0 || num_q_heads / cache->num_kv_heads > 16)
         return 0;
-    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q);
+    return saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, total_q,
+                                       cache->head_dim);
 }
 
 static int prefill_impl(const saw_cache_desc *cache, int32_t num_q_heads, const void *q,

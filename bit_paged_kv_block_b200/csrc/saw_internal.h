@@ -40,7 +40,7 @@ struct RotateQuantizeArgs {
 };
 
 struct DecodeArgs {
-    const void *q;               // bf16 [S][Hq][128]
+    const void *q;               // bf16 [S][Hq][D]
     const uint8_t *kv_pages;
     const void *scales;
     const int32_t *block_table;  // [S][max_blocks]
@@ -51,13 +51,14 @@ struct DecodeArgs {
     int32_t num_kv_heads;
     int64_t num_pages;
     float sm_scale;
-    float *out;                  // fp32 [S][Hq][128]
+    float *out;                  // fp32 [S][Hq][D]
     void *workspace;
     size_t workspace_bytes;
     uint32_t *status;
     bool rotate = true;          // false: plain INT4 cache (no query / output rotation)
     const int32_t *q_start = nullptr;   // chunked prefill: [S + 1] query-row offsets (else decode)
     int64_t total_q = 0;         // chunked prefill: query rows (q_start[S])
+    int32_t head_dim = 128;      // D: 128 or 256 (INT4 cache only)
 };
 
 struct AppendBf16Args {
@@ -79,7 +80,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
 // Workspace bytes the decode kernel needs on the current device (0 if the shape is invalid);
 // total_q >= 0: a chunked prefill over total_q query rows.
 size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
-                              int64_t total_q = -1);
+                              int64_t total_q = -1, int32_t head_dim = 128);
 
 // Queue the decode kernel; `programmatic` launches it as a programmatic dependent of the
 // previous kernel on the stream.  Returns a cudaError_t.

@@ -223,8 +223,8 @@ def saw_rotate_quantize_paged_strided(k, v, slot_mapping, kv_pages, scales, dev_
 
 
 def saw_paged_decode_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,
-                                     num_pages: int = 1) -> int:
-    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, int(num_pages))
+                                     num_pages: int = 1, head_dim: int = HEAD_DIM) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), int(head_dim), PAGE_SIZE, int(num_pages))
     return int(lib.saw_paged_decode_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
                                                     int(num_seqs)))
 
@@ -236,9 +236,9 @@ def saw_paged_decode_workspace_init(workspace: torch.Tensor, stream=None) -> Non
 
 
 def allocate_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: int,
-                       device="cuda") -> torch.Tensor:
+                       device="cuda", head_dim: int = HEAD_DIM) -> torch.Tensor:
     """A zero-initialised decode workspace for this shape on the current device."""
-    n = saw_paged_decode_workspace_bytes(num_kv_heads, num_q_heads, num_seqs)
+    n = saw_paged_decode_workspace_bytes(num_kv_heads, num_q_heads, num_seqs, head_dim=head_dim)
     if n == 0:
         raise SawError(SAW_ERR_CUDA, "saw_paged_decode_workspace_bytes")
     ws = torch.empty(n, dtype=torch.uint8, device=device)
@@ -258,8 +258,8 @@ def _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace, d
         _need(dev_status, "dev_status", torch.int32, 1)
     desc = cache_desc(kv_pages)
     S, hq, d = q.shape
-    if d != HEAD_DIM or tuple(out.shape) != (S, hq, HEAD_DIM):
-        raise ValueError("q and out must be [S][Hq][128]")
+    if d != desc.head_dim or tuple(out.shape) != (S, hq, desc.head_dim):
+        raise ValueError(f"q and out must be [S][Hq][{desc.head_dim}] matching the cache")
     if block_table.shape[0] != S or seq_lens.shape[0] != S:
         raise ValueError("block_table and seq_lens need one row per sequence")
     return desc, S, hq
@@ -267,7 +267,8 @@ def _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace, d
 
 def saw_paged_decode_attn(q, kv_pages, scales, block_table, seq_lens, out, workspace,
                           sm_scale=None, dev_status=None, stream=None) -> None:
-    """Decode attention of q (bf16 [S][Hq][128]) over the INT4 paged cache into out (fp32)."""
+    """Decode attention of q (bf16 [S][Hq][D], D = 128 or 256 as the cache) over the INT4 paged
+    cache into out (fp32 [S][Hq][D])."""
     _decode(lib.saw_paged_decode_attn, "saw_paged_decode_attn", q, kv_pages, scales, block_table,
             seq_lens, out, workspace, sm_scale, dev_status, stream)
 
@@ -284,7 +285,7 @@ def _decode(fn, name, q, kv_pages, scales, block_table, seq_lens, out, workspace
     desc, S, hq = _decode_checks(q, kv_pages, scales, block_table, seq_lens, out, workspace,
                                  dev_status)
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+        sm_scale = 1.0 / math.sqrt(desc.head_dim)
     rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages), _ptr(scales), _ptr(block_table),
             block_table.shape[1], _ptr(seq_lens), S, float(sm_scale), _ptr(out), _ptr(workspace),
             workspace.numel(), _ptr(dev_status), _stream(stream))
@@ -313,12 +314,12 @@ def _step(fn, name, q, k_new, v_new, slot_mapping, kv_pages, scales, block_table
     _need(v_new, "v_new", torch.bfloat16, 3)
     _need(slot_mapping, "slot_mapping", torch.int64, 1)
     T = k_new.shape[0]
-    if tuple(k_new.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v_new.shape != k_new.shape:
-        raise ValueError("k_new and v_new must be [T][Hkv][128] matching the cache")
+    if tuple(k_new.shape) != (T, desc.num_kv_heads, desc.head_dim) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [T][Hkv][D] matching the cache")
     if slot_mapping.shape[0] != T:
         raise ValueError("slot_mapping must have one entry per new token")
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+        sm_scale = 1.0 / math.sqrt(desc.head_dim)
     rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), T,
             _ptr(kv_pages), _ptr(scales), _ptr(block_table), block_table.shape[1], _ptr(seq_lens),
             S, float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(), _ptr(dev_status),
@@ -343,7 +344,7 @@ def saw_paged_decode_attn_static(q, kv_pages, scales, block_table, seq_lens, out
     desc = cache_desc(kv_pages)
     S, hq, _ = q.shape
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+        sm_scale = 1.0 / math.sqrt(desc.head_dim)
     rc = lib.saw_paged_decode_attn_static(ctypes.byref(desc), hq, _ptr(q), _ptr(kv_pages),
                                           _ptr(scales), _ptr(block_table), block_table.shape[1],
                                           _ptr(seq_lens), S, float(sm_scale), _ptr(out),
@@ -443,12 +444,12 @@ def saw_decode_step_bf16(q, k_new, v_new, slot_mapping, kv_bf16, block_table, se
     _need(v_new, "v_new", torch.bfloat16, 3)
     _need(slot_mapping, "slot_mapping", torch.int64, 1)
     T = k_new.shape[0]
-    if tuple(k_new.shape) != (T, desc.num_kv_heads, HEAD_DIM) or v_new.shape != k_new.shape:
-        raise ValueError("k_new and v_new must be [T][Hkv][128] matching the cache")
+    if tuple(k_new.shape) != (T, desc.num_kv_heads, desc.head_dim) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [T][Hkv][D] matching the cache")
     if slot_mapping.shape[0] != T:
         raise ValueError("slot_mapping must have one entry per new token")
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+        sm_scale = 1.0 / math.sqrt(desc.head_dim)
     rc = lib.saw_decode_step_bf16(ctypes.byref(desc), hq, _ptr(q), _ptr(k_new), _ptr(v_new),
                                   _ptr(slot_mapping), T, _ptr(kv_bf16), _ptr(block_table),
                                   block_table.shape[1], _ptr(seq_lens), S, float(sm_scale),
@@ -460,15 +461,16 @@ def saw_decode_step_bf16(q, k_new, v_new, slot_mapping, kv_bf16, block_table, se
 # ---- chunked-prefill attention over the INT4 cache -------------------------------------------
 
 def saw_paged_prefill_workspace_bytes(num_kv_heads: int, num_q_heads: int, num_seqs: int,
-                                      total_q: int) -> int:
-    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, 1)
+                                      total_q: int, head_dim: int = HEAD_DIM) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), int(head_dim), PAGE_SIZE, 1)
     return int(lib.saw_paged_prefill_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
                                                      int(num_seqs), int(total_q)))
 
 
 def allocate_prefill_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: int, total_q: int,
-                               device="cuda") -> torch.Tensor:
-    n = saw_paged_prefill_workspace_bytes(num_kv_heads, num_q_heads, num_seqs, total_q)
+                               device="cuda", head_dim: int = HEAD_DIM) -> torch.Tensor:
+    n = saw_paged_prefill_workspace_bytes(num_kv_heads, num_q_heads, num_seqs, total_q,
+                                          head_dim=head_dim)
     if n == 0:
         raise SawError(SAW_ERR_CUDA, "saw_paged_prefill_workspace_bytes")
     return torch.empty(n, dtype=torch.uint8, device=device)
@@ -476,9 +478,9 @@ def allocate_prefill_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: in
 
 def saw_paged_prefill_attn(q, q_start, kv_pages, scales, block_table, seq_lens, out, workspace,
                            sm_scale=None, dev_status=None, stream=None, rotate=True) -> None:
-    """Causal attention of a chunk of query tokens (bf16 [total_q][Hq][128], sequence s owning
+    """Causal attention of a chunk of query tokens (bf16 [total_q][Hq][D], sequence s owning
     rows q_start[s] .. q_start[s + 1] - 1, the last tokens of its cached seq_lens[s]) over the
-    INT4 paged cache into out (fp32 [total_q][Hq][128]).  rotate=False reads a plain INT4
+    INT4 paged cache into out (fp32 [total_q][Hq][D]).  rotate=False reads a plain INT4
     cache."""
     _need(q_start, "q_start", torch.int32, 1)
     _need(q, "q", torch.bfloat16, 3)
@@ -493,12 +495,12 @@ def saw_paged_prefill_attn(q, q_start, kv_pages, scales, block_table, seq_lens, 
     desc = cache_desc(kv_pages)
     total_q, hq, d = q.shape
     S = seq_lens.shape[0]
-    if d != HEAD_DIM or tuple(out.shape) != (total_q, hq, HEAD_DIM):
-        raise ValueError("q and out must be [total_q][Hq][128]")
+    if d != desc.head_dim or tuple(out.shape) != (total_q, hq, desc.head_dim):
+        raise ValueError(f"q and out must be [total_q][Hq][{desc.head_dim}] matching the cache")
     if q_start.shape[0] != S + 1 or block_table.shape[0] != S:
         raise ValueError("q_start needs num_seqs + 1 entries and block_table one row per sequence")
     if sm_scale is None:
-        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+        sm_scale = 1.0 / math.sqrt(desc.head_dim)
     fn = lib.saw_paged_prefill_attn if rotate else lib.saw_paged_prefill_attn_plain
     rc = fn(ctypes.byref(desc), hq, _ptr(q), _ptr(q_start), total_q, _ptr(kv_pages), _ptr(scales),
             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S, float(sm_scale), _ptr(out),

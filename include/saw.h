@@ -13,7 +13,9 @@
  *   saw_decode_step            one serving step: append one token per sequence, then decode
  *
  * Fixed build parameters (the pages give no numbers; these are the library's definition):
- *   head_dim D = 128 = Hadamard block B; H is the Sylvester Hadamard matrix in natural order,
+ *   head_dim D = 128 or 256; Hadamard block B = 128 (a D = 256 vector is rotated as two
+ *   independent 128-element blocks and keeps one (scale, zero) pair over all 256 elements);
+ *   H is the Sylvester Hadamard matrix in natural order,
  *   normalised by 1/sqrt(128), applied as an fp32 butterfly (stages h = 1, 2, ..., 64,
  *   (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]), then a multiply by fp32(1/sqrt(128)),
  *   every step one IEEE fp32 operation); per (token, kv head) and separately for K and V:
@@ -23,18 +25,18 @@
  *   as +0; two codes per byte, the even index in the low nibble; pages of 16 tokens.
  *
  * Memory layout (all buffers caller-owned device memory, C-contiguous, 16-byte aligned):
- *   k, v (new tokens)   bf16   [T][Hkv][128]
+ *   k, v (new tokens)   bf16   [T][Hkv][D]
  *   slot_mapping        int64  [T]        slot = page * 16 + offset; slot < 0 skips the token
- *   kv_pages            uint8  [num_pages][Hkv][2 (K, V)][16][64]
- *                        so one (page, kv head) is one contiguous 2 KiB block: 1 KiB of K
- *                        codes then 1 KiB of V codes, 64 bytes per token row
+ *   kv_pages            uint8  [num_pages][Hkv][2 (K, V)][16][D / 2]
+ *                        so one (page, kv head) is one contiguous block of 16 D bytes (2 KiB
+ *                        for D = 128): K codes then V codes, D / 2 bytes per token row
  *   scales              fp16   [num_pages][Hkv][2 (K, V)][16][2 (scale, zero)]
  *                        128 bytes per (page, kv head)
- *   q                   bf16   [S][Hq][128]    query head hq reads kv head hq / (Hq / Hkv)
+ *   q                   bf16   [S][Hq][D]      query head hq reads kv head hq / (Hq / Hkv)
  *   block_table         int32  [S][max_blocks_per_seq]  logical block -> page
  *   seq_lens            int32  [S]    tokens of each sequence in the cache (including the
  *                                     token appended by this step), 0 <= len <= 16 * max_blocks
- *   out                 fp32   [S][Hq][128]
+ *   out                 fp32   [S][Hq][D]
  *
  * Ownership and threading: the library allocates no device memory.  Every call is
  * asynchronous on the given stream (a cudaStream_t passed as void*; NULL is the legacy
@@ -61,7 +63,8 @@ extern "C" {
 typedef enum saw_status {
     SAW_OK = 0,
     SAW_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
-    SAW_ERR_UNSUPPORTED = 2,      /* head_dim != 128, page_size != 16, Hq / Hkv > 16 */
+    SAW_ERR_UNSUPPORTED = 2,      /* head_dim not 128 / 256 (BF16 cache: not 128), page_size
+                                     != 16, Hq / Hkv > 16 */
     SAW_ERR_CUDA = 3,             /* a CUDA runtime call or kernel launch failed */
     SAW_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required */
     SAW_ERR_SCRATCH_LIMIT = 5     /* shape too large for saw_paged_decode_attn_static */
@@ -75,7 +78,7 @@ typedef enum saw_status {
 
 typedef struct saw_cache_desc {
     int32_t num_kv_heads; /* Hkv >= 1 */
-    int32_t head_dim;     /* must be 128 */
+    int32_t head_dim;     /* 128 or 256 (the BF16 baseline cache: 128) */
     int32_t page_size;    /* must be 16 */
     int64_t num_pages;    /* pages in kv_pages / scales; num_pages * Hkv * 32 < 2^31 */
 } saw_cache_desc;
@@ -83,7 +86,7 @@ typedef struct saw_cache_desc {
 /* Rotate, quantize and scatter T new tokens into the paged cache.
  * Follows "SAW-INT4" (Research Findings): the fused rotation-quantization kernel that writes
  * token-wise INT4 codes of Hadamard-rotated vectors directly into the paged KV cache.
- * k, v: bf16 [T][Hkv][128] device; slot_mapping: int64 [T] device; kv_pages, scales: the
+ * k, v: bf16 [T][Hkv][D] device; slot_mapping: int64 [T] device; kv_pages, scales: the
  * cache (device, updated in place); dev_status: device uint32 or NULL.  T == 0 is a no-op.
  * Codes and scales are bit-identical to the definition above for every finite input. */
 int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const void *v,
@@ -92,12 +95,12 @@ int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const 
                               void *stream);
 
 /* saw_rotate_quantize_paged (and its plain INT4 counterpart) for k and v that are not
- * contiguous, e.g. slices of a fused QKV projection output [T][(Hq + 2 Hkv) * 128]: each
- * token's Hkv head vectors are contiguous (128 bf16 each, head-major), and token t starts at
- * k + t * k_stride (v + t * v_stride) bf16 elements.  Strides are at least Hkv * 128 and a
+ * contiguous, e.g. slices of a fused QKV projection output [T][(Hq + 2 Hkv) * D]: each
+ * token's Hkv head vectors are contiguous (D bf16 each, head-major), and token t starts at
+ * k + t * k_stride (v + t * v_stride) bf16 elements.  Strides are at least Hkv * D and a
  * multiple of 8 (every token starts on 16 bytes; k and v themselves 16-byte aligned).
- * Supported for Hkv a multiple of 8 or a divisor of 8 (else SAW_ERR_UNSUPPORTED): the kernel
- * copies whole 8-vector tiles.  Results are bit-identical to the contiguous call on the same
+ * Supported for Hkv a multiple or a divisor of the tile's 1024 / D vectors (8 for D = 128, 4 for
+ * D = 256; else SAW_ERR_UNSUPPORTED): the kernel copies whole tiles.  Results are bit-identical to the contiguous call on the same
  * values. */
 int saw_rotate_quantize_paged_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
                                       const void *v, int64_t v_stride, const int64_t *slot_mapping,
@@ -187,7 +190,7 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
  * out), the last C_s of its seq_lens[s] cached tokens; query i sits at position
  * seq_lens[s] - C_s + i and attends causally to cache tokens 0 .. seq_lens[s] - C_s + i, with
  * the rotation, scales and arithmetic of saw_paged_decode_attn (a decode is the case C_s = 1).
- *     q: bf16 [total_q][Hq][128]; out: fp32 [total_q][Hq][128]; q_start: int32 [num_seqs + 1],
+ *     q: bf16 [total_q][Hq][D]; out: fp32 [total_q][Hq][D]; q_start: int32 [num_seqs + 1],
  *     device, non-decreasing, q_start[0] = 0, q_start[num_seqs] = total_q, 0 <= C_s <= seq_lens[s]
  *     (a violating sequence is flagged SAW_DEV_BAD_SEQ_LEN and skipped).
  * Every (query token, head) pair reads the pages of its sequence once per block of 8 such
@@ -250,7 +253,9 @@ int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const
  * of 18.3 MiB inside this library's device code (present on every GPU that loads the library,
  * until the process exits) instead of a caller workspace.  It allocates nothing.
  * Limit: num_seqs * num_kv_heads * ceil(G / 8) <= 2048 and a decode grid of at most 2560 warps
- * (a B200 runs 2368); larger shapes return SAW_ERR_SCRATCH_LIMIT before anything is queued.
+ * (a B200 runs 2368), and the workspace the shape needs must fit the array (D = 256 slots are
+ * twice as large: about 550 segments on a B200); larger shapes return SAW_ERR_SCRATCH_LIMIT
+ * before anything is queued.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
  * that device current); make that first call before any stream capture.  Nothing in the array
  * needs to start at zero.  All calls on a device share the array and it keeps the previous

@@ -19,9 +19,10 @@ def run_decode(wl, pages, scales, device, q=None, sm_scale=None, status=None, ws
     kv, sc = device_cache_from(pages, scales, device)
     if q is None:
         q = synth.q_values(wl)
-    out = torch.full((wl.num_seqs, wl.num_q_heads, 128), float("nan"), device=device)
+    out = torch.full((wl.num_seqs, wl.num_q_heads, wl.head_dim), float("nan"), device=device)
     if ws is None:
-        ws = saw.allocate_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, device)
+        ws = saw.allocate_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, device,
+                                    head_dim=wl.head_dim)
     saw.saw_paged_decode_attn(q.to(device), kv, sc,
                               torch.from_numpy(wl.block_table).to(device),
                               torch.from_numpy(wl.seq_lens).to(device), out, ws,

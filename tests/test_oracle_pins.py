@@ -395,6 +395,28 @@ def test_decode_matches_torch_sdpa_fp64():
             assert torch.allclose(torch.from_numpy(out[s, h]), Hn @ o, atol=1e-12, rtol=0)
 
 
+def test_decode_d256_matches_torch_sdpa_fp64():
+    """D = 256: one (scale, zero) per 256-element vector, each 128-element half rotated on its
+    own, sm_scale 1/16.  The oracle equals torch's fp64 SDPA on the block-diagonally rotated
+    query and the dequantised cache, rotated back block by block."""
+    wl = synth.custom("sdpa256", [37, 16, 1, 50], num_q_heads=4, num_kv_heads=2, seed=21,
+                      head_dim=256)
+    _, _, pages, scales = _cache_for(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(qb, pages, scales, wl.block_table, wl.seq_lens)
+    Hn = H128 / np.sqrt(128.0)
+    R = torch.tensor(np.block([[Hn, np.zeros((128, 128))], [np.zeros((128, 128)), Hn]]))
+    qf = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).double()
+    for s in range(wl.num_seqs):
+        for hq in range(4):
+            h = hq // 2
+            K = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 0))
+            V = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 1))
+            o = torch.nn.functional.scaled_dot_product_attention(
+                (R @ qf[s, hq])[None, None, None], K[None, None], V[None, None])[0, 0, 0]
+            assert torch.allclose(torch.from_numpy(out[s, hq]), R @ o, atol=1e-12, rtol=0)
+
+
 def test_decode_identical_keys_and_zero_scale_give_mean():
     """If every key is the same, or sm_scale is 0, the weights are uniform: the output is the
     rotated mean of the dequantised values."""
