@@ -36,7 +36,6 @@ METRIC = "INT4 paged decode tokens/s"
 UNIT = "tokens/s"
 HBM_TARGET_GBS = 8000.0            # the 8 TB/s roofline the targets are stated against
 CODE_ROW_BYTES = 64
-BYTES_PER_TOKEN_HEAD_DECODE = 2 * CODE_ROW_BYTES + 2 * 4          # K+V codes + scale/zero
 BYTES_PER_TOKEN_HEAD_APPEND = 2 * 128 * 2 + 2 * CODE_ROW_BYTES + 2 * 4   # bf16 in, codes+scales out
 WORKLOAD_TEXT = ("decode step, Llama-3-8B layer shape: batch 64, seq_lens uniform 512-8192, "
                  "32 q / 8 kv heads, head_dim 128, page 16, one new token per seq appended "
@@ -86,10 +85,14 @@ def job_throughput(units_per_rank: int, world: int, ms_per_step_max: float) -> f
 # ---- byte accounting (algorithmic bytes, not measured traffic) ----------------------------
 
 def decode_bytes(wl) -> int:
+    """Algorithmic bytes of one INT4 decode: per cached token and kv head D / 2 bytes of codes
+    for K and for V plus 8 B of fp16 (scale, zero) pairs (136 B at D = 128); per sequence the
+    bf16 queries, fp32 outputs, its length and its block-table entries."""
+    D = wl.head_dim
     lens = wl.seq_lens.astype(np.int64)
     pages = (lens + 15) // 16
-    per_seq = wl.num_q_heads * 128 * (2 + 4) + 4 + 4 * pages
-    return int((wl.num_kv_heads * lens * BYTES_PER_TOKEN_HEAD_DECODE).sum() + per_seq.sum())
+    per_seq = wl.num_q_heads * D * (2 + 4) + 4 + 4 * pages
+    return int((wl.num_kv_heads * lens * (D + 8)).sum() + per_seq.sum())
 
 
 def decode_bytes_bf16(wl) -> int:
@@ -497,6 +500,31 @@ def run_saw(args):
                             "the repeats come from L2"}
     del pkv3, psc3, qpf, opf, wpf
 
+    # ---- head dimension 256: the decode workload's shape with 256-element head vectors -------
+    w256 = synth.custom("decode_d256", wl.seq_lens, num_q_heads=wl.num_q_heads,
+                        num_kv_heads=wl.num_kv_heads, seed=50 + rank, head_dim=256)
+    kv4, sc4 = saw.allocate_cache(w256.num_pages, w256.num_kv_heads, dev, head_dim=256)
+    seq, pos = synth.token_index(w256)
+    saw.saw_rotate_quantize_paged(synth.kv_values(w256, "K", device=dev),
+                                  synth.kv_values(w256, "V", device=dev),
+                                  torch.from_numpy(synth.slot_mapping(w256, seq, pos)).to(dev),
+                                  kv4, sc4)
+    q4 = synth.q_values(w256, device=dev)
+    o4 = torch.empty(q4.shape, dtype=torch.float32, device=dev)
+    ws4 = saw.allocate_workspace(w256.num_kv_heads, w256.num_q_heads, w256.num_seqs, dev,
+                                 head_dim=256)
+    tab4 = torch.from_numpy(w256.block_table).to(dev)
+    run_d4 = lambda: saw.saw_paged_decode_attn(q4, kv4, sc4, tab4, lens, o4, ws4,
+                                               dev_status=status, stream=stream)
+    for _ in range(3):
+        run_d4()
+    t_d4 = mean_event_ms(run_d4, n_kt)
+    d4_gbs = decode_bytes(w256) / (t_d4 * 1e-3) / 1e9
+    head_dim_256 = {"workload": "the decode batch (same lengths and heads) at head_dim 256",
+                    "decode_launch_ms": t_d4, "algorithmic_bytes_per_launch": decode_bytes(w256),
+                    "decode_GBps": d4_gbs, "decode_frac_of_measured_peak": d4_gbs / peak_gbs}
+    del kv4, sc4, q4, o4, ws4
+
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
     h_q, h_k, h_v, h_slots, h_table, h_lens = (pin(q), pin(k_new), pin(v_new), pin(slots),
@@ -549,6 +577,7 @@ def run_saw(args):
         "plain_int4": plain_int4,
         "bf16_baseline": bf16_baseline,
         "prefill_attn": prefill_attn,
+        "head_dim_256": head_dim_256,
         "append_launch_ms": t_append,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,
