@@ -130,7 +130,8 @@ def fwht_f32(x: np.ndarray) -> np.ndarray:
 
 
 def rotate_f32(x: np.ndarray) -> np.ndarray:
-    """Block-diagonal (128-wide blocks) normalised Hadamard rotation of each row, fp32."""
+    """Block-diagonal normalised Hadamard rotation of each row, fp32: 128-wide blocks, or the
+    whole row when it is 64 wide."""
     y = np.array(x, dtype=np.float32, copy=True, order="C")
     D = y.shape[-1]
     flat = y.reshape(-1, D)

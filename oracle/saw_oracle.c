@@ -15,9 +15,10 @@
  *     Summary): the same method restated.
  *   - "BitDecoding-FP4" (abstract): Hadamard rotation against key outliers under token-wise
  *     scaling; stacked-query attention over paged caches.
- * The pages give no formula.  The fixed build parameters used here are: Hadamard block B = 128,
- * normalised by 1/sqrt(B), applied as an fp32 butterfly (natural Sylvester order, stages
- * h = 1, 2, ..., 64, no FMA contraction: this file is compiled with -ffp-contract=off);
+ * The pages give no formula.  The fixed build parameters used here are: Hadamard block B = 128
+ * (B = D for the 64-wide head vectors, which hold no 128-point block), normalised by 1/sqrt(B),
+ * applied as an fp32 butterfly (natural Sylvester order, stages h = 1, 2, ..., B/2, no FMA
+ * contraction: this file is compiled with -ffp-contract=off);
  * asymmetric per-(token, kv-head) scale = (max - min) / 15 and zero = min computed in fp32 and
  * stored as fp16; code = clamp(rint((y - min) / scale), 0, 15); two codes per byte, the even
  * index in the low nibble; 16-token pages.
@@ -90,12 +91,17 @@ void oracle_fwht_f32(float *x, int n)
         x[j] = x[j] * c;
 }
 
-/* Block-diagonal rotation of a head vector of length D (a multiple of 128): each 128-wide
+/* Width of the diagonal blocks for a head vector of length D: the 128-point block, or the
+ * whole vector when it is shorter (D = 64: the 64-point transform, normalised by 1/sqrt(64)). */
+static int oracle_block(int D) { return D < ORACLE_HADAMARD_BLOCK ? D : ORACLE_HADAMARD_BLOCK; }
+
+/* Block-diagonal rotation of a head vector of length D (64, or a multiple of 128): each
  * block is rotated independently. */
 void oracle_rotate_f32(float *x, int D)
 {
-    for (int b = 0; b < D; b += ORACLE_HADAMARD_BLOCK)
-        oracle_fwht_f32(x + b, ORACLE_HADAMARD_BLOCK);
+    const int B = oracle_block(D);
+    for (int b = 0; b < D; b += B)
+        oracle_fwht_f32(x + b, B);
 }
 
 /* Same transform in fp64 (used on the decode side, where the reference is fp64). */
@@ -118,8 +124,9 @@ void oracle_fwht_f64(double *x, int n)
 
 void oracle_rotate_f64(double *x, int D)
 {
-    for (int b = 0; b < D; b += ORACLE_HADAMARD_BLOCK)
-        oracle_fwht_f64(x + b, ORACLE_HADAMARD_BLOCK);
+    const int B = oracle_block(D);
+    for (int b = 0; b < D; b += B)
+        oracle_fwht_f64(x + b, B);
 }
 
 /* ---- token-wise asymmetric INT4 quantizer -------------------------------------------- */

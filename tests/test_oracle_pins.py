@@ -100,6 +100,26 @@ def test_rotation_is_block_diagonal():
     assert np.abs(y - full).max() > 1e-2
 
 
+def test_rotation_d64_is_the_64_point_transform():
+    """A 64-wide head vector holds no 128-point block: it is rotated by the normalised 64-point
+    Sylvester transform (c = 1/8, exact in fp32)."""
+    rng = np.random.default_rng(6)
+    x = rng.standard_normal((6, 64)).astype(np.float32)
+    y = oracle.rotate_f32(x)
+    assert np.array_equal(y, oracle.fwht_f32(x))
+    H64 = hadamard(64).astype(np.float64)
+    ref = x.astype(np.float64) @ (H64 / 8.0).T
+    assert np.abs(y - ref).max() <= 2.5e-7 * np.abs(x).sum(axis=1).max()
+    for j in (0, 1, 37, 63):                       # unit vectors: column j times 1/8, exactly
+        e = np.zeros(64, np.float32)
+        e[j] = 1.0
+        assert np.array_equal(oracle.rotate_f32(e), (H64[:, j] / 8.0).astype(np.float32))
+    c = oracle.rotate_f32(np.full(64, 0.75, np.float32))
+    assert c[0] == np.float32(6.0) and np.all(c[1:] == 0)
+    xd = rng.standard_normal((5, 64))
+    assert np.abs(oracle.rotate_f64(xd) - xd @ (H64 / 8.0).T).max() <= 1e-12
+
+
 # ---------------------------------------------------------------------------------------
 # scalar conversions
 # ---------------------------------------------------------------------------------------
@@ -273,9 +293,10 @@ def test_quantizer_subnormal_scale():
 # scatter into the paged layout
 # ---------------------------------------------------------------------------------------
 
-def test_scatter_layout_and_skips():
+@pytest.mark.parametrize("D", [64, 128])
+def test_scatter_layout_and_skips(D):
     rng = np.random.default_rng(31)
-    T, Hkv, D, P, num_pages = 40, 3, 128, 16, 6
+    T, Hkv, P, num_pages = 40, 3, 16, 6
     k = synth.bf16_bits(torch.randn(T, Hkv, D).to(torch.bfloat16))
     v = synth.bf16_bits(torch.randn(T, Hkv, D).to(torch.bfloat16))
     slots = rng.permutation(num_pages * P)[:T].astype(np.int64)
@@ -406,6 +427,26 @@ def test_decode_d256_matches_torch_sdpa_fp64():
     out = oracle.decode_fp64(qb, pages, scales, wl.block_table, wl.seq_lens)
     Hn = H128 / np.sqrt(128.0)
     R = torch.tensor(np.block([[Hn, np.zeros((128, 128))], [np.zeros((128, 128)), Hn]]))
+    qf = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).double()
+    for s in range(wl.num_seqs):
+        for hq in range(4):
+            h = hq // 2
+            K = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 0))
+            V = torch.from_numpy(_dequant_seq(wl, pages, scales, s, h, 1))
+            o = torch.nn.functional.scaled_dot_product_attention(
+                (R @ qf[s, hq])[None, None, None], K[None, None], V[None, None])[0, 0, 0]
+            assert torch.allclose(torch.from_numpy(out[s, hq]), R @ o, atol=1e-12, rtol=0)
+
+
+def test_decode_d64_matches_torch_sdpa_fp64():
+    """D = 64: the 64-point rotation (1/8) and sm_scale 1/8; the oracle equals torch's fp64 SDPA
+    on the rotated query and the dequantised cache, rotated back."""
+    wl = synth.custom("sdpa64", [37, 16, 1, 50], num_q_heads=4, num_kv_heads=2, seed=22,
+                      head_dim=64)
+    _, _, pages, scales = _cache_for(wl)
+    qb = synth.bf16_bits(synth.q_values(wl))
+    out = oracle.decode_fp64(qb, pages, scales, wl.block_table, wl.seq_lens)
+    R = torch.tensor(hadamard(64).astype(np.float64) / 8.0)
     qf = torch.from_numpy(qb.view(np.int16)).view(torch.bfloat16).double()
     for s in range(wl.num_seqs):
         for hq in range(4):
