@@ -47,7 +47,8 @@ using namespace decode;
 // K + V codes of one (page, kv head): 2 x 16 rows of D / 2 bytes
 __host__ __device__ constexpr int code_bytes(int d) { return 2 * kPageSize * d / 2; }
 constexpr int kScaleBytes = 2 * kPageSize * 4;          // K + V (scale, zero) fp16 pairs
-constexpr float kHadamardC = 0.0883883461356163f;
+// 1/sqrt(B) of the rotation block B = min(D, 128): fp32(1/sqrt(128)), or 1/8 for D = 64
+__host__ __device__ constexpr float hadamard_c(int d) { return d == 64 ? 0.125f : 0.0883883461356163f; }
 
 // Unpack one 32-bit word of packed codes (bytes b0..b3, low nibble first) into four fp16x2
 // registers by masking alone: a nibble left in the low mantissa bits of an fp16 with a zero
@@ -75,13 +76,14 @@ __device__ __forceinline__ float2 h2_to_f2(uint32_t u)
 // Rotated, scaled query of one segment as fp16 mma B fragments, from the raw bf16 queries of
 // its nheads <= 8 heads in shared memory ([nheads][kD] at qbuf).
 // Thread (g, t) owns query head g of the group and d in [kQ t, kQ t + kQ), kQ = kD / 4.  The
-// rotation is the 128-point Hadamard transform of each 128-element block of d (for kD = 256
-// the two halves are independent blocks, as the quantizer rotates them).
+// rotation is the Hadamard transform of each block of B = min(kD, 128) elements of d (for
+// kD = 256 the two halves are independent blocks, as the quantizer rotates them).
 template <bool kRotate, int kD>
 __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf, int nheads, int g,
                                            int t, uint32_t bq[kD / 16][2], float sq_out[2])
 {
     constexpr int kQ = kD / 4;
+    constexpr int kBlock = kD < 128 ? kD : 128;
     float x[kQ];
     if (g < nheads) {
 #pragma unroll
@@ -100,7 +102,7 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
             x[l] = 0.0f;
     }
     // Hadamard butterfly (skipped for the plain INT4 cache): the low log2(kQ) bits of d in
-    // registers, the remaining bits of the 128-block across lanes t ^ 1 (and t ^ 2 for kD = 128).
+    // registers, the remaining bits of the block across lanes t ^ 1 (and t ^ 2 for kD <= 128).
 #pragma unroll
     for (int hb = 1; kRotate && hb < kQ; hb <<= 1)
 #pragma unroll
@@ -111,7 +113,7 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
                 x[l + hb] = a - b;
             }
 #pragma unroll
-    for (int lb = 1; kRotate && kQ * lb < 128; lb <<= 1) {
+    for (int lb = 1; kRotate && kQ * lb < kBlock; lb <<= 1) {
         const bool high = (t & lb) != 0;
 #pragma unroll
         for (int l = 0; l < kQ; l++) {
@@ -147,12 +149,12 @@ __device__ __forceinline__ void load_query(const DecodeParams &p, uint32_t qbuf,
 }
 
 // Byte offset of 16-byte chunk c of code row r in a staged page: rows of kD / 2 bytes with the
-// tensor copy's swizzle (64B for 64-byte rows: chunk ^ bits 1-2 of the row; 128B for 128-byte
-// rows: chunk ^ bits 0-2 of the row).
+// tensor copy's swizzle (32B for 32-byte rows: chunk ^ bit 2 of the row; 64B for 64-byte rows:
+// chunk ^ bits 1-2 of the row; 128B for 128-byte rows: chunk ^ bits 0-2 of the row).
 template <int kD>
 __device__ __forceinline__ uint32_t code_offset(int r, int c)
 {
-    const int sw = kD == 128 ? (r >> 1) & 3 : r & 7;
+    const int sw = kD == 64 ? (r >> 2) & 1 : kD == 128 ? (r >> 1) & 3 : r & 7;
     return static_cast<uint32_t>(r * (kD / 2) + ((c ^ sw) << 4));
 }
 
@@ -165,30 +167,47 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
                                              int lane, WarpState<kD / 16> &st)
 {
     const int g = lane >> 2, t = lane & 3;
-    constexpr int kChunks = kD / 128;   // 16-byte code chunks of one row per thread
+    constexpr int kWords = kD / 32;   // 32-bit code words of one row per thread
 
     // ---- S^T = K . Q^T over 16 tokens (rows g, g + 8) -----------------------------------
-    // Thread t reads chunks kChunks t .. kChunks t + kChunks - 1 (d in [kD/4 t, kD/4 (t + 1))):
-    // within each quarter warp the two rows land in disjoint banks.
+    // Thread t reads the kD / 4 codes of d in [kD/4 t, kD/4 (t + 1)) of rows g and g + 8: for
+    // kD >= 128 whole 16-byte chunks (within each quarter warp the two rows land in disjoint
+    // banks), for kD = 64 half a chunk (each half warp reads four whole 32-byte rows).
+    uint32_t kw0[kWords], kw1[kWords];
+    if constexpr (kD == 64) {
+        const uint32_t off = static_cast<uint32_t>(8 * (t & 1));
+        const uint2 k0 = lds64(cbase + code_offset<kD>(g, t >> 1) + off);
+        const uint2 k1 = lds64(cbase + code_offset<kD>(g + 8, t >> 1) + off);
+        kw0[0] = k0.x;
+        kw0[1] = k0.y;
+        kw1[0] = k1.x;
+        kw1[1] = k1.y;
+    } else {
+#pragma unroll
+        for (int hf = 0; hf < kD / 128; hf++) {
+            const int c = (kD / 128) * t + hf;
+            const uint4 k0 = lds128(cbase + code_offset<kD>(g, c));
+            const uint4 k1 = lds128(cbase + code_offset<kD>(g + 8, c));
+            kw0[4 * hf] = k0.x;
+            kw0[4 * hf + 1] = k0.y;
+            kw0[4 * hf + 2] = k0.z;
+            kw0[4 * hf + 3] = k0.w;
+            kw1[4 * hf] = k1.x;
+            kw1[4 * hf + 1] = k1.y;
+            kw1[4 * hf + 2] = k1.z;
+            kw1[4 * hf + 3] = k1.w;
+        }
+    }
     float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
-    for (int hf = 0; hf < kChunks; hf++) {
-        const int c = kChunks * t + hf;
-        const uint4 k0 = lds128(cbase + code_offset<kD>(g, c));
-        const uint4 k1 = lds128(cbase + code_offset<kD>(g + 8, c));
-        const uint32_t kw0[4] = {k0.x, k0.y, k0.z, k0.w};
-        const uint32_t kw1[4] = {k1.x, k1.y, k1.z, k1.w};
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            uint32_t ya[4], yb[4];
-            unpack_codes(kw0[i], ya);
-            unpack_codes(kw1[i], yb);
-            const uint32_t a0[4] = {ya[0], yb[0], ya[1], yb[1]};
-            const uint32_t a1[4] = {ya[2], yb[2], ya[3], yb[3]};
-            const int w = 4 * hf + i;
-            mma_16816(acc, a0, bq[2 * w][0], bq[2 * w][1]);
-            mma_16816(acc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
-        }
+    for (int w = 0; w < kWords; w++) {
+        uint32_t ya[4], yb[4];
+        unpack_codes(kw0[w], ya);
+        unpack_codes(kw1[w], yb);
+        const uint32_t a0[4] = {ya[0], yb[0], ya[1], yb[1]};
+        const uint32_t a1[4] = {ya[2], yb[2], ya[3], yb[3]};
+        mma_16816(acc, a0, bq[2 * w][0], bq[2 * w][1]);
+        mma_16816(acc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
     }
 
     // ---- logits (log2 domain) ---------------------------------------------------------------
@@ -281,8 +300,8 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
         }
 #pragma unroll
     for (int e = 0; kRotate && e < 2; e++) {
-        // d bits 0, 1 (j) and 5, 6 (low bits of c) in registers; bit 7 (kD = 256) selects the
-        // 128-block and is not transformed
+        // d bits 0, 1 (j) and 5, 6 (low bits of c; bit 5 only for kD = 64) in registers; bit 7
+        // (kD = 256) selects the 128-block and is not transformed
 #pragma unroll
         for (int c = 0; c < kC; c++)
 #pragma unroll
@@ -295,7 +314,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
                         v[e][c][j + jb] = a - b;
                     }
 #pragma unroll
-        for (int cb = 1; cb <= 2; cb <<= 1)
+        for (int cb = 1; cb <= 2 && cb < kC; cb <<= 1)
 #pragma unroll
             for (int c = 0; c < kC; c++)
                 if ((c & cb) == 0)
@@ -325,7 +344,7 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
             float *dst = p.out + sg.row_offset(p, head, kD);
 #pragma unroll
             for (int c = 0; c < kC; c++) {
-                const float f = kRotate ? kHadamardC : 1.0f;
+                const float f = kRotate ? hadamard_c(kD) : 1.0f;
                 const float4 val = make_float4(v[e][c][0] * f, v[e][c][1] * f, v[e][c][2] * f,
                                                v[e][c][3] * f);
                 *reinterpret_cast<float4 *>(dst + 32 * c + 4 * g) = val;
@@ -358,18 +377,20 @@ __device__ __forceinline__ void copy_page_elected(uint32_t bar, uint32_t dst_cod
 
 // The INT4 page format for the generic decode kernel (decode_common.cuh), head dimension kD:
 // 4 warps per CTA and a ring per warp whose stages hold the codes of one (page, kv head) (32
-// tensor-map rows of kD / 2 bytes: 2 KiB with the 64B swizzle for kD = 128, 4 KiB with the 128B
-// swizzle for kD = 256), codes of all stages first, then the scales (128 B each).  kD = 128:
-// 4 stages, 4 CTAs per SM; kD = 256 (twice the accumulators): 2 stages, 3 CTAs per SM, which
-// keeps about as many bytes in flight per SM.
+// tensor-map rows of kD / 2 bytes: 1 KiB with the 32B swizzle for kD = 64, 2 KiB with the 64B
+// swizzle for kD = 128, 4 KiB with the 128B swizzle for kD = 256), codes of all stages first,
+// then the scales (128 B each).  kD = 128: 4 stages, 4 CTAs per SM; kD = 256 (twice the
+// accumulators): 2 stages, 3 CTAs per SM, which keeps about as many bytes in flight per SM;
+// kD = 64 (half the registers, half the bytes per page): 4 stages, 6 CTAs per SM, since a warp
+// completes its page copies one after another and more warps keep more copies in flight.
 template <bool kRotate, int kD>
 struct Int4Format {
-    static_assert(kD == 128 || kD == 256, "head dimension");
+    static_assert(kD == 64 || kD == 128 || kD == 256, "head dimension");
     static constexpr int kDim = kD;
     static constexpr int kTiles = kD / 16;
     static constexpr int kWarps = 4;
-    static constexpr int kStages = kD == 128 ? 4 : 2;
-    static constexpr int kMinBlocks = kD == 128 ? 4 : 3;
+    static constexpr int kStages = kD == 256 ? 2 : 4;
+    static constexpr int kMinBlocks = kD == 64 ? 5 : kD == 128 ? 4 : 3;
     static constexpr int kRowsPerPage = 32;
     static constexpr int kCodeBytes = code_bytes(kD);
     static constexpr int kRingBytes = kWarps * kStages * (kCodeBytes + kScaleBytes);
@@ -487,7 +508,8 @@ const CUtensorMap *code_tensor_map(const uint8_t *kv_pages, int64_t rows)
         CUresult r = encode(&cache.map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2,
                             const_cast<uint8_t *>(kv_pages), dims, strides, box, estr,
                             CU_TENSOR_MAP_INTERLEAVE_NONE,
-                            kD == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
+                            kD == 64 ? CU_TENSOR_MAP_SWIZZLE_32B
+                            : kD == 128 ? CU_TENSOR_MAP_SWIZZLE_64B : CU_TENSOR_MAP_SWIZZLE_128B,
                             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
         if (r != CUDA_SUCCESS) {
             cache.base = nullptr;
@@ -534,8 +556,8 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     p.qrows = qrows;
     p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Fmt::kWarps;
-    // q carries sm_scale * log2(e), and 1/sqrt(128) of the (unnormalised) query butterfly
-    p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(kHadamardC) : 1.0) * a.sm_scale *
+    // q carries sm_scale * log2(e), and 1/sqrt(B) of the (unnormalised) query butterfly
+    p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(hadamard_c(kD)) : 1.0) * a.sm_scale *
                                   1.4426950408889634);
 
     cudaLaunchAttribute attr[1];
@@ -584,6 +606,8 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
         return workspace_bytes<128>(num_kv_heads, num_q_heads, num_seqs, total_q);
     if (head_dim == 256)
         return workspace_bytes<256>(num_kv_heads, num_q_heads, num_seqs, total_q);
+    if (head_dim == 64)
+        return workspace_bytes<64>(num_kv_heads, num_q_heads, num_seqs, total_q);
     return 0;
 }
 
@@ -593,6 +617,8 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
         return launch<128>(a, stream, programmatic);
     if (a.head_dim == 256)
         return launch<256>(a, stream, programmatic);
+    if (a.head_dim == 64)
+        return launch<64>(a, stream, programmatic);
     return cudaErrorInvalidValue;
 }
 

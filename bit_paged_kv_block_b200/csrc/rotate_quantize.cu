@@ -2,7 +2,8 @@
 //
 // Implements the fused rotation-quantization kernel of "SAW-INT4: System-Aware 4-Bit KV-Cache
 // Quantization for Real-World LLM Serving" (Research Findings): every new key and value head
-// vector is rotated by the normalised 128-point Hadamard transform, quantized token-wise to
+// vector is rotated by the normalised 128-point Hadamard transform (per 128-element block; a
+// 64-element head vector by the 64-point transform), quantized token-wise to
 // asymmetric INT4 and written straight into its page of the paged KV cache.
 //
 // Results are bit-identical to the definition in saw.h:
@@ -20,7 +21,9 @@
 // 128-byte swizzle) completing on mbarriers, so warps never wait for each other.  The warps of
 // the persistent grid take tiles round-robin.
 //
-// Thread layout: two threads per head vector; a warp's tile has its 8 K vectors in lanes 0-15
+// Thread layout (D = 128; D = 256 uses two such pairs per vector, one per 128-block, and D = 64
+// one thread per whole vector, 16 vectors of K and 16 of V per tile, the butterfly entirely in
+// registers): two threads per head vector; a warp's tile has its 8 K vectors in lanes 0-15
 // and its 8 V vectors in lanes 16-31.  Thread half b of a vector holds the 64 elements
 // j = 16a + 8b + r (a, r in 0..7), read as eight 16-byte shared-memory loads that the 128-byte
 // swizzle spreads over all banks.  Stage h = 8 is the only one that crosses the pair (one
@@ -35,13 +38,15 @@ namespace saw {
 namespace {
 
 constexpr int kTileBytes = 2048;                       // K (or V) bytes of one warp tile: 16 rows
-// Head dimension D = 128 or 256 (two independent 128-point rotation blocks): a warp tile holds
-// 2048 / (2 D) vectors of K and as many of V, D / 64 threads per vector, each thread 64
-// elements of one 128-block; a vector is D / 64 tensor-map rows of 128 bytes.
+// Head dimension D = 64 (the 64-point transform: no 128-point block fits), 128, or 256 (two
+// independent 128-point rotation blocks): a warp tile holds 2048 / (2 D) vectors of K and as
+// many of V, D / 64 threads per vector, each thread 64 elements of one rotation block; a vector
+// is D / 64 tensor-map rows of 128 bytes.
 template <int kD>
 struct RqDims {
-    static constexpr int kTileVecs = kTileBytes / (2 * kD);   // 8 or 4
-    static constexpr int kThreadsPerVec = kD / 64;             // 2 or 4
+    static_assert(kD == 64 || kD == 128 || kD == 256, "head dimension");
+    static constexpr int kTileVecs = kTileBytes / (2 * kD);   // 16, 8 or 4
+    static constexpr int kThreadsPerVec = kD / 64;             // 1, 2 or 4
     static constexpr int kRowsPerVec = kD / 64;                // 128-byte rows per vector
     static constexpr int kCodeBytes = kD / 2;                  // packed codes per vector
 };
@@ -53,6 +58,7 @@ constexpr int kRqSmemBars = kRqWarps * kRqStages * kRqStageBytes;
 constexpr size_t kRqSmemBytes = 1024 + kRqSmemBars + kRqWarps * kRqStages * 8;
 constexpr uint64_t kRqWaitLimitNs = 1000000000ull;
 constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
+constexpr float kHadamardC64 = 0.125f;               // 1/sqrt(64), exact
 constexpr float kRoundMagic = 12582912.0f;           // 1.5 * 2^23
 // A code computed from the reciprocal is provably the IEEE-divide code unless the remainder
 // is within 2^-18 of one half (derivation above code_bits_tie()).
@@ -82,6 +88,15 @@ __device__ __forceinline__ void load_half_vec(uint32_t tile, int vt, int blk, in
         const int chunk = (2 * (a & 3) + b) ^ (row & 7);
         raw[a] = lds128(tile + row * 128 + chunk * 16);
     }
+}
+
+// D = 64: this thread's whole vector vt of the tile, one 128-byte row (chunk a = elements
+// 8a .. 8a + 7 at chunk a ^ (vt & 7) under the 128-byte swizzle).
+__device__ __forceinline__ void load_vec64(uint32_t tile, int vt, uint4 raw[8])
+{
+#pragma unroll
+    for (int a = 0; a < 8; a++)
+        raw[a] = lds128(tile + vt * 128 + ((a ^ (vt & 7)) << 4));
 }
 
 __device__ __forceinline__ void to_pairs(const uint4 raw[8], uint64_t X[32])
@@ -146,6 +161,35 @@ __device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
         X[i] = f2_pack(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
     }
     const uint64_t cc = f2_pack(kHadamardC, kHadamardC);
+#pragma unroll
+    for (int i = 0; i < 32; i++)
+        X[i] = f2_mul(X[i], cc);
+}
+
+// Normalised 64-point Hadamard transform of the vector one thread holds as X[8 a + r] =
+// (x[8 a + r], x[8 (a + 4) + r]) (a < 4, r < 8): element bits 0-2 are index bits 0-2 of X
+// (h = 1, 2, 4), bits 3-4 index bits 3-4 (h = 8, 16), bit 5 the halves of each pair (h = 32);
+// then the multiply by 1/8.  The stages run in ascending h, every operation one IEEE fp32 op.
+__device__ __forceinline__ void fwht64(uint64_t X[32])
+{
+#pragma unroll
+    for (int hb = 1; hb <= 16; hb <<= 1) {
+#pragma unroll
+        for (int i = 0; i < 32; i++) {
+            if ((i & hb) == 0) {
+                const uint64_t lo = X[i], hi = X[i + hb];
+                X[i] = f2_add(lo, hi);
+                X[i + hb] = f2_sub(lo, hi);
+            }
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 32; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        X[i] = f2_pack(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+    }
+    const uint64_t cc = f2_pack(kHadamardC64, kHadamardC64);
 #pragma unroll
     for (int i = 0; i < 32; i++)
         X[i] = f2_mul(X[i], cc);
@@ -298,8 +342,12 @@ __device__ __forceinline__ void quantize_store(const uint64_t X[32], int blk, in
             }
         }
         if (store) {
-            *reinterpret_cast<uint32_t *>(dst + 8 * a4 + 4 * b) = pack8(tlo);
-            *reinterpret_cast<uint32_t *>(dst + 8 * (a4 + 4) + 4 * b) = pack8(thi);
+            // D = 64: elements 8 a + r of one thread, word a at byte 4 a; otherwise elements
+            // 16 a + 8 b + r of thread half b, word (a, b) at byte 8 a + 4 b of the block
+            const int w_lo = kD == 64 ? 4 * a4 : 8 * a4 + 4 * b;
+            const int w_hi = kD == 64 ? 4 * (a4 + 4) : 8 * (a4 + 4) + 4 * b;
+            *reinterpret_cast<uint32_t *>(dst + w_lo) = pack8(tlo);
+            *reinterpret_cast<uint32_t *>(dst + w_hi) = pack8(thi);
         }
     }
     if (store && b == 0 && blk == 0) {
@@ -366,9 +414,11 @@ __global__ void __launch_bounds__(kRqThreads, 4)
         issue();
 
     const int half = lane >> 4;          // 0: K, 1: V
-    const int b = lane & 1;              // half of a 128-block
-    const int blk = (lane >> 1) & (Dims::kThreadsPerVec / 2 - 1);   // 128-block of the vector
-    const int vt = (lane & 15) / Dims::kThreadsPerVec;              // vector of the tile
+    // half of a 128-block, 128-block of the vector, vector of the tile (D = 64: one thread
+    // holds a whole vector)
+    const int b = kD == 64 ? 0 : lane & 1;
+    const int blk = kD == 64 ? 0 : (lane >> 1) & (Dims::kThreadsPerVec / 2 - 1);
+    const int vt = (lane & 15) / Dims::kThreadsPerVec;
     const uint32_t num_vecs = static_cast<uint32_t>(p.num_vecs);
     const uint32_t hkv = static_cast<uint32_t>(p.hkv);
     uint32_t tile = wg;
@@ -415,11 +465,18 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 
         const uint32_t tile_smem = ring + stg * kRqStageBytes + half * kTileBytes;
         uint4 raw[8];
-        load_half_vec<kD>(tile_smem, vt, blk, b, raw);
+        if constexpr (kD == 64)
+            load_vec64(tile_smem, vt, raw);
+        else
+            load_half_vec<kD>(tile_smem, vt, blk, b, raw);
         uint64_t X[32];
         to_pairs(raw, X);
-        if (kRotate)
-            fwht128(X, b, 0xFFFFFFFFu);
+        if constexpr (kRotate) {
+            if constexpr (kD == 64)
+                fwht64(X);
+            else
+                fwht128(X, b, 0xFFFFFFFFu);
+        }
         quantize_store<kRotate, kD>(X, blk, b, store, row, p);
         __syncwarp();
     }
@@ -439,7 +496,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     const int64_t num_vecs = a.num_tokens * a.num_kv_heads;
     if (num_vecs == 0)
         return cudaSuccess;
-    if (a.head_dim != 128 && a.head_dim != 256)
+    if (a.head_dim != 64 && a.head_dim != 128 && a.head_dim != 256)
         return cudaErrorInvalidValue;
     const int64_t rows_per_vec = a.head_dim / 64;
     const int64_t tile_vecs = kTileBytes / (2 * a.head_dim);
@@ -448,7 +505,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
 
     // k / v: contiguous [T][Hkv][D] (k_stride = v_stride = 0) through a 2-D map of 128-byte
     // rows, or with a token stride through 3-D maps whose box is one whole tile of V vectors
-    // (V = 8 for D = 128, 4 for D = 256; Hkv a multiple of V: V heads of one token; Hkv dividing
+    // (V = 16 for D = 64, 8 for D = 128, 4 for D = 256; Hkv a multiple of V: V heads of one token; Hkv dividing
     // V: V / Hkv tokens), so every copy lands on a 1024-byte aligned stage.
     const bool strided = a.k_stride != 0 || a.v_stride != 0;
     static thread_local struct {
@@ -523,18 +580,22 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         return e;
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
-    static const void *const kernels[4] = {
+    static const void *const kernels[6] = {
         reinterpret_cast<const void *>(rotate_quantize_kernel<true, 128>),
         reinterpret_cast<const void *>(rotate_quantize_kernel<false, 128>),
         reinterpret_cast<const void *>(rotate_quantize_kernel<true, 256>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 256>)};
+        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 256>),
+        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 64>),
+        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 64>)};
     auto kernel = a.head_dim == 128
                       ? (a.rotate ? rotate_quantize_kernel<true, 128> : rotate_quantize_kernel<false, 128>)
-                      : (a.rotate ? rotate_quantize_kernel<true, 256> : rotate_quantize_kernel<false, 256>);
+                  : a.head_dim == 256
+                      ? (a.rotate ? rotate_quantize_kernel<true, 256> : rotate_quantize_kernel<false, 256>)
+                      : (a.rotate ? rotate_quantize_kernel<true, 64> : rotate_quantize_kernel<false, 64>);
     if (sms_of[dev] == 0) {
         int sms = 0, occ = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        for (int r = 0; r < 4 && e == cudaSuccess; r++)
+        for (int r = 0; r < 6 && e == cudaSuccess; r++)
             e = cudaFuncSetAttribute(kernels[r], cudaFuncAttributeMaxDynamicSharedMemorySize,
                                      static_cast<int>(kRqSmemBytes));
         if (e == cudaSuccess)

@@ -16,7 +16,7 @@ int check_cache(const saw_cache_desc *c)
 {
     if (c == nullptr || c->num_kv_heads <= 0 || c->num_pages < 0)
         return SAW_ERR_INVALID_ARGUMENT;
-    if ((c->head_dim != 128 && c->head_dim != 256) || c->page_size != 16)
+    if ((c->head_dim != 64 && c->head_dim != 128 && c->head_dim != 256) || c->page_size != 16)
         return SAW_ERR_UNSUPPORTED;
     // tensor-map rows (page * Hkv + h) * 32 must stay below 2^31
     if (c->num_pages > (int64_t(1) << 31) / (int64_t(c->num_kv_heads) * 32))
@@ -120,8 +120,8 @@ const char *saw_status_string(int status)
     case SAW_ERR_INVALID_ARGUMENT:
         return "invalid argument (null pointer, bad size or alignment, Hq not a multiple of Hkv)";
     case SAW_ERR_UNSUPPORTED:
-        return "unsupported shape (head_dim 128, or 256 where supported; page_size 16; Hq/Hkv at "
-               "most 16)";
+        return "unsupported shape (head_dim 64, 128 or 256, the BF16 cache 128; page_size 16; "
+               "Hq/Hkv at most 16)";
     case SAW_ERR_CUDA:
         return "CUDA runtime error";
     case SAW_ERR_WORKSPACE:

@@ -196,6 +196,12 @@ __device__ __forceinline__ uint4 lds128(uint32_t addr)
                  : "r"(addr));
     return r;
 }
+__device__ __forceinline__ uint2 lds64(uint32_t addr)
+{
+    uint2 r;
+    asm volatile("ld.shared.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "r"(addr));
+    return r;
+}
 __device__ __forceinline__ uint32_t lds32(uint32_t addr)
 {
     uint32_t r;

@@ -143,10 +143,10 @@ def _need(t: torch.Tensor, name: str, dtype, ndim=None, cuda=True) -> None:
 
 
 def cache_desc(kv_pages: torch.Tensor) -> saw_cache_desc:
-    """Descriptor of a cache tensor uint8 [num_pages][Hkv][2][16][D / 2] (D = 128 or 256)."""
+    """Descriptor of a cache tensor uint8 [num_pages][Hkv][2][16][D / 2] (D = 64, 128 or 256)."""
     _need(kv_pages, "kv_pages", torch.uint8, 5, cuda=False)
     num_pages, hkv, two, page, half = kv_pages.shape
-    if two != 2 or half * 2 not in (128, 256):
+    if two != 2 or half * 2 not in (64, 128, 256):
         raise ValueError(f"kv_pages must be [num_pages][Hkv][2][16][D / 2], got {tuple(kv_pages.shape)}")
     return saw_cache_desc(int(hkv), int(half * 2), int(page), int(num_pages))
 

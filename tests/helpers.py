@@ -81,36 +81,36 @@ EDGE_KINDS = ["small_ints", "zeros_and_constants", "tiny_magnitudes", "huge_rang
               "signed_zero", "single_spike", "scale_above_2m100", "scale_below_2m100"]
 
 
-def edge_kv(kind: str, T: int, Hkv: int):
-    """bf16 K, V [T][Hkv][128] whose quantization hits a corner of the code computation:
+def edge_kv(kind: str, T: int, Hkv: int, D: int = 128):
+    """bf16 K, V [T][Hkv][D] whose quantization hits a corner of the code computation:
     exact half-way quotients (small integers, before or after rotation), degenerate and
     constant vectors, subnormal scales, scales just above and just below 2^-100 (the smallest
     scale the kernel settles ties without a divide), huge dynamic range, signed zeros and one
     large spike per vector."""
     g = torch.Generator().manual_seed(7)
     if kind == "small_ints":
-        x = torch.randint(-3, 4, (T, Hkv, 128), generator=g).float()
+        x = torch.randint(-3, 4, (T, Hkv, D), generator=g).float()
     elif kind == "zeros_and_constants":
-        x = torch.zeros(T, Hkv, 128)
+        x = torch.zeros(T, Hkv, D)
         x[1::3] = torch.randn(T, Hkv, 1, generator=g)[1::3]
         x[2::5, :, 7] = 1.0
     elif kind == "tiny_magnitudes":
-        x = torch.randn(T, Hkv, 128, generator=g) * 1e-37
+        x = torch.randn(T, Hkv, D, generator=g) * 1e-37
         x[::2] *= 1e-2
     elif kind == "huge_range":
-        x = torch.randn(T, Hkv, 128, generator=g) * (10.0 ** torch.randint(-3, 4, (T, Hkv, 1), generator=g))
+        x = torch.randn(T, Hkv, D, generator=g) * (10.0 ** torch.randint(-3, 4, (T, Hkv, 1), generator=g))
     elif kind == "signed_zero":
-        x = torch.zeros(T, Hkv, 128)
+        x = torch.zeros(T, Hkv, D)
         x[::2, :, 3] = -0.0
         x[1::2, :, 5] = 1.0
         x[::4] = -x[::4]
     elif kind in ("scale_above_2m100", "scale_below_2m100"):
         # small integers times 2^-96 or 2^-103: scales just above and below 2^-100
         e = -96 if kind == "scale_above_2m100" else -103
-        x = torch.randint(-3, 4, (T, Hkv, 128), generator=g).float() * 2.0 ** e
+        x = torch.randint(-3, 4, (T, Hkv, D), generator=g).float() * 2.0 ** e
     elif kind == "single_spike":
-        x = torch.zeros(T, Hkv, 128)
-        x[torch.arange(T), :, torch.arange(T) % 128] = 50.0
+        x = torch.zeros(T, Hkv, D)
+        x[torch.arange(T), :, torch.arange(T) % D] = 50.0
     else:
         raise ValueError(kind)
     return x.to(torch.bfloat16), (x.flip(-1) * 0.5).to(torch.bfloat16)

@@ -52,7 +52,7 @@ def _rq(desc, T=4, k=16, v=16, slots=16, pages=16, scales=16):
 
 def test_append_argument_checks():
     assert _rq(None) == saw.SAW_ERR_INVALID_ARGUMENT
-    assert _rq(_desc(d=64)) == saw.SAW_ERR_UNSUPPORTED
+    assert _rq(_desc(d=96)) == saw.SAW_ERR_UNSUPPORTED
     assert _rq(_desc(p=32)) == saw.SAW_ERR_UNSUPPORTED
     assert _rq(_desc(hkv=0)) == saw.SAW_ERR_INVALID_ARGUMENT
     assert _rq(_desc(pages=1 << 30)) == saw.SAW_ERR_UNSUPPORTED
@@ -95,7 +95,7 @@ def test_workspace_bytes_rejects_bad_shapes():
     f = saw.lib.saw_paged_decode_workspace_bytes
     assert f(ctypes.byref(_desc()), 12, 4) == 0
     assert f(ctypes.byref(_desc()), 72, 4) == 0
-    assert f(ctypes.byref(_desc(d=64)), 32, 4) == 0
+    assert f(ctypes.byref(_desc(d=96)), 32, 4) == 0
 
 
 def test_python_binding_rejects_cpu_tensors():

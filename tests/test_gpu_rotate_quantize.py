@@ -189,3 +189,51 @@ def test_head_dim_256_strided(cuda_device):
     torch.cuda.synchronize()
     pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous())
     assert_cache_equal(kv, sc, pages, scales)
+
+
+@pytest.mark.parametrize("rotate", [True, False])
+@pytest.mark.parametrize("kind", ["randn"] + EDGE_KINDS)
+def test_head_dim_64(cuda_device, kind, rotate):
+    """D = 64: the whole vector is one 64-point rotation block (1/8), one thread per vector,
+    16 vectors of K and 16 of V per tile, 32 code bytes per row; bit-exact against the oracle on
+    outlier data and on every edge input, ragged token counts."""
+    from bit_paged_kv_block_b200 import saw
+    T, hkv = 203, 3
+    wl = synth.custom(f"d64{kind}", [T], num_q_heads=hkv, num_kv_heads=hkv, new_tokens=[T],
+                      head_dim=64, seed=3, outlier_range=(10.0, 30.0),
+                      num_pages=(T + 15) // 16 + 3)
+    if kind == "randn":
+        k, v = synth.kv_values(wl, "K"), synth.kv_values(wl, "V")
+    else:
+        k, v = edge_kv(kind, T, hkv, D=64)
+    seq, pos = synth.token_index(wl)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(cuda_device)
+    kv, sc = canary_device_cache(wl, cuda_device)
+    fn = saw.saw_rotate_quantize_paged if rotate else saw.saw_quantize_paged_plain
+    fn(k.to(cuda_device), v.to(cuda_device), slots, kv, sc)
+    torch.cuda.synchronize()
+    pages, scales = oracle_cache(wl, k=k, v=v, rotate=rotate)
+    assert_cache_equal(kv, sc, pages, scales)
+
+
+@pytest.mark.parametrize("hkv", [2, 8, 16])
+def test_head_dim_64_strided(cuda_device, hkv):
+    """D = 64 k / v sliced from a fused QKV output (tiles of 16 vectors: Hkv dividing or a
+    multiple of 16)."""
+    from bit_paged_kv_block_b200 import saw
+    T, hq = 77, 2 * hkv
+    g = torch.Generator().manual_seed(hkv)
+    qkv = (torch.randn(T, (hq + 2 * hkv) * 64, generator=g) * 2.0).to(torch.bfloat16)
+    k = qkv[:, hq * 64:(hq + hkv) * 64].view(T, hkv, 64)
+    v = qkv[:, (hq + hkv) * 64:].view(T, hkv, 64)
+    wl = synth.custom(f"d64qkv{hkv}", [T], num_q_heads=hkv, num_kv_heads=hkv, new_tokens=[T],
+                      head_dim=64)
+    seq, pos = synth.token_index(wl)
+    slots = torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(cuda_device)
+    kv, sc = canary_device_cache(wl, cuda_device)
+    qd = qkv.to(cuda_device)
+    saw.saw_rotate_quantize_paged_strided(qd[:, hq * 64:(hq + hkv) * 64].view(T, hkv, 64),
+                                          qd[:, (hq + hkv) * 64:].view(T, hkv, 64), slots, kv, sc)
+    torch.cuda.synchronize()
+    pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous())
+    assert_cache_equal(kv, sc, pages, scales)
