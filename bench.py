@@ -500,30 +500,33 @@ def run_saw(args):
                             "the repeats come from L2"}
     del pkv3, psc3, qpf, opf, wpf
 
-    # ---- head dimension 256: the decode workload's shape with 256-element head vectors -------
-    w256 = synth.custom("decode_d256", wl.seq_lens, num_q_heads=wl.num_q_heads,
-                        num_kv_heads=wl.num_kv_heads, seed=50 + rank, head_dim=256)
-    kv4, sc4 = saw.allocate_cache(w256.num_pages, w256.num_kv_heads, dev, head_dim=256)
-    seq, pos = synth.token_index(w256)
-    saw.saw_rotate_quantize_paged(synth.kv_values(w256, "K", device=dev),
-                                  synth.kv_values(w256, "V", device=dev),
-                                  torch.from_numpy(synth.slot_mapping(w256, seq, pos)).to(dev),
-                                  kv4, sc4)
-    q4 = synth.q_values(w256, device=dev)
-    o4 = torch.empty(q4.shape, dtype=torch.float32, device=dev)
-    ws4 = saw.allocate_workspace(w256.num_kv_heads, w256.num_q_heads, w256.num_seqs, dev,
-                                 head_dim=256)
-    tab4 = torch.from_numpy(w256.block_table).to(dev)
-    run_d4 = lambda: saw.saw_paged_decode_attn(q4, kv4, sc4, tab4, lens, o4, ws4,
-                                               dev_status=status, stream=stream)
-    for _ in range(3):
-        run_d4()
-    t_d4 = mean_event_ms(run_d4, n_kt)
-    d4_gbs = decode_bytes(w256) / (t_d4 * 1e-3) / 1e9
-    head_dim_256 = {"workload": "the decode batch (same lengths and heads) at head_dim 256",
-                    "decode_launch_ms": t_d4, "algorithmic_bytes_per_launch": decode_bytes(w256),
-                    "decode_GBps": d4_gbs, "decode_frac_of_measured_peak": d4_gbs / peak_gbs}
-    del kv4, sc4, q4, o4, ws4
+    # ---- head dimensions 64 and 256: the decode workload's shape with other head vectors -------
+    head_dims = {}
+    for hd in (64, 256):
+        whd = synth.custom(f"decode_d{hd}", wl.seq_lens, num_q_heads=wl.num_q_heads,
+                           num_kv_heads=wl.num_kv_heads, seed=50 + rank, head_dim=hd)
+        kv4, sc4 = saw.allocate_cache(whd.num_pages, whd.num_kv_heads, dev, head_dim=hd)
+        seq, pos = synth.token_index(whd)
+        saw.saw_rotate_quantize_paged(synth.kv_values(whd, "K", device=dev),
+                                      synth.kv_values(whd, "V", device=dev),
+                                      torch.from_numpy(synth.slot_mapping(whd, seq, pos)).to(dev),
+                                      kv4, sc4)
+        q4 = synth.q_values(whd, device=dev)
+        o4 = torch.empty(q4.shape, dtype=torch.float32, device=dev)
+        ws4 = saw.allocate_workspace(whd.num_kv_heads, whd.num_q_heads, whd.num_seqs, dev,
+                                     head_dim=hd)
+        tab4 = torch.from_numpy(whd.block_table).to(dev)
+        run_d4 = lambda: saw.saw_paged_decode_attn(q4, kv4, sc4, tab4, lens, o4, ws4,
+                                                   dev_status=status, stream=stream)
+        for _ in range(3):
+            run_d4()
+        t_d4 = mean_event_ms(run_d4, n_kt)
+        d4_gbs = decode_bytes(whd) / (t_d4 * 1e-3) / 1e9
+        head_dims[f"head_dim_{hd}"] = {
+            "workload": f"the decode batch (same lengths and heads) at head_dim {hd}",
+            "decode_launch_ms": t_d4, "algorithmic_bytes_per_launch": decode_bytes(whd),
+            "decode_GBps": d4_gbs, "decode_frac_of_measured_peak": d4_gbs / peak_gbs}
+        del kv4, sc4, q4, o4, ws4
 
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
@@ -577,7 +580,7 @@ def run_saw(args):
         "plain_int4": plain_int4,
         "bf16_baseline": bf16_baseline,
         "prefill_attn": prefill_attn,
-        "head_dim_256": head_dim_256,
+        **head_dims,
         "append_launch_ms": t_append,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,

@@ -13,11 +13,12 @@
  *   saw_decode_step            one serving step: append one token per sequence, then decode
  *
  * Fixed build parameters (the pages give no numbers; these are the library's definition):
- *   head_dim D = 128 or 256; Hadamard block B = 128 (a D = 256 vector is rotated as two
- *   independent 128-element blocks and keeps one (scale, zero) pair over all 256 elements);
- *   H is the Sylvester Hadamard matrix in natural order,
- *   normalised by 1/sqrt(128), applied as an fp32 butterfly (stages h = 1, 2, ..., 64,
- *   (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]), then a multiply by fp32(1/sqrt(128)),
+ *   head_dim D = 64, 128 or 256; Hadamard block B = min(D, 128) (a D = 256 vector is rotated
+ *   as two independent 128-element blocks and keeps one (scale, zero) pair over all 256
+ *   elements; a D = 64 vector holds no 128-element block and is rotated as one 64-element
+ *   block); H is the Sylvester Hadamard matrix of order B in natural order,
+ *   normalised by 1/sqrt(B), applied as an fp32 butterfly (stages h = 1, 2, ..., B/2,
+ *   (x[j], x[j+h]) <- (x[j] + x[j+h], x[j] - x[j+h]), then a multiply by fp32(1/sqrt(B)),
  *   every step one IEEE fp32 operation); per (token, kv head) and separately for K and V:
  *   scale = (max - min) / 15 and zero = min in fp32, stored as fp16 (round to nearest even);
  *   code_i = clamp(rint((y_i - min) / scale), 0, 15) with IEEE division and ties to even;
@@ -63,7 +64,7 @@ extern "C" {
 typedef enum saw_status {
     SAW_OK = 0,
     SAW_ERR_INVALID_ARGUMENT = 1, /* null pointer, bad size, misalignment, Hq % Hkv != 0 */
-    SAW_ERR_UNSUPPORTED = 2,      /* head_dim not 128 / 256 (BF16 cache: not 128), page_size
+    SAW_ERR_UNSUPPORTED = 2,      /* head_dim not 64 / 128 / 256 (BF16 cache: not 128), page_size
                                      != 16, Hq / Hkv > 16 */
     SAW_ERR_CUDA = 3,             /* a CUDA runtime call or kernel launch failed */
     SAW_ERR_WORKSPACE = 4,        /* workspace missing or smaller than required */
@@ -78,7 +79,7 @@ typedef enum saw_status {
 
 typedef struct saw_cache_desc {
     int32_t num_kv_heads; /* Hkv >= 1 */
-    int32_t head_dim;     /* 128 or 256 (the BF16 baseline cache: 128) */
+    int32_t head_dim;     /* 64, 128 or 256 (the BF16 baseline cache: 128) */
     int32_t page_size;    /* must be 16 */
     int64_t num_pages;    /* pages in kv_pages / scales; num_pages * Hkv * 32 < 2^31 */
 } saw_cache_desc;
@@ -99,8 +100,8 @@ int saw_rotate_quantize_paged(const saw_cache_desc *cache, const void *k, const 
  * token's Hkv head vectors are contiguous (D bf16 each, head-major), and token t starts at
  * k + t * k_stride (v + t * v_stride) bf16 elements.  Strides are at least Hkv * D and a
  * multiple of 8 (every token starts on 16 bytes; k and v themselves 16-byte aligned).
- * Supported for Hkv a multiple or a divisor of the tile's 1024 / D vectors (8 for D = 128, 4 for
- * D = 256; else SAW_ERR_UNSUPPORTED): the kernel copies whole tiles.  Results are bit-identical to the contiguous call on the same
+ * Supported for Hkv a multiple or a divisor of the tile's 1024 / D vectors (16 for D = 64, 8 for
+ * D = 128, 4 for D = 256; else SAW_ERR_UNSUPPORTED): the kernel copies whole tiles.  Results are bit-identical to the contiguous call on the same
  * values. */
 int saw_rotate_quantize_paged_strided(const saw_cache_desc *cache, const void *k, int64_t k_stride,
                                       const void *v, int64_t v_stride, const int64_t *slot_mapping,
