@@ -85,6 +85,9 @@ def _load():
         lib.oracle_decode_bf16_fp64.argtypes = [P, P, P, i32, P, i32, i32, i32, i32, i32, dbl,
                                                 P, i32]
         lib.oracle_decode_bf16_fp64.restype = None
+        lib.oracle_decode_window_fp64.argtypes = [P, P, P, i32, P, P, P, i32, P, i32, i32, i32,
+                                                  i32, i32, i32, i32, dbl, i32, P, i32]
+        lib.oracle_decode_window_fp64.restype = None
         _lib = lib
         return lib
 
@@ -290,3 +293,112 @@ def empty_cache(num_pages: int, Hkv: int, D: int = 128, page_size: int = 16):
     """Zero-filled cache arrays in the oracle's layout (pages, scales)."""
     return (np.zeros((num_pages, Hkv, 2, page_size, D // 2), dtype=np.uint8),
             np.zeros((num_pages, Hkv, 2, page_size, 2), dtype=np.uint16))
+
+
+# ---- full-precision sink / recent window beside the INT4 cache ----------------------------
+# "InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large Language Models",
+# Abstract and Figure 2.  The readings (which positions are sinks, recent or quantized, and
+# where each lives) are stated above oracle_decode_window_fp64 in saw_oracle.c.
+
+def window_slot(p: int, w_sink: int, w_recent: int) -> int:
+    """Window slot of position p (a sink or a recent token)."""
+    return p if p < w_sink else w_sink + (p - w_sink) % w_recent
+
+
+def _win_page_off(win_table, s, slot):
+    return int(win_table[s, slot // 16]), slot % 16
+
+
+def _q_slot(block_table, s, j):
+    return int(block_table[s, j // 16]) * 16 + j % 16
+
+
+def window_fill(k_bits, v_bits, seq_lens, w_sink, w_recent, win_kv, win_table, kv_pages, scales,
+                block_table, *, rotate=True):
+    """Place every token of each sequence where the window layout puts it: sinks and the last
+    w_recent positions (>= w_sink) into their window slots (bf16 bits), the others rotated and
+    quantized into the INT4 pages at their quantized index.  k_bits, v_bits: uint16
+    [S][Lmax][Hkv][D] (positions beyond seq_lens[s] ignored)."""
+    k_bits = _as(k_bits, np.uint16)
+    v_bits = _as(v_bits, np.uint16)
+    S = len(seq_lens)
+    for s in range(S):
+        L = int(seq_lens[s])
+        slots = []
+        for p in range(L):
+            if p < w_sink or p >= max(w_sink, L - w_recent):
+                pg, off = _win_page_off(win_table, s, window_slot(p, w_sink, w_recent))
+                win_kv[pg, :, 0, off] = k_bits[s, p]
+                win_kv[pg, :, 1, off] = v_bits[s, p]
+                slots.append(-1)
+            else:
+                slots.append(_q_slot(block_table, s, p - w_sink))
+        if L:
+            bad = rotate_quantize_paged(np.ascontiguousarray(k_bits[s, :L]),
+                                        np.ascontiguousarray(v_bits[s, :L]),
+                                        np.array(slots, dtype=np.int64), kv_pages, scales,
+                                        rotate=rotate)
+            assert bad == 0
+
+
+def window_append(k_bits, v_bits, seq_lens, w_sink, w_recent, win_kv, win_table, kv_pages,
+                  scales, block_table, *, rotate=True):
+    """One serving step: the new token of each sequence (k_bits, v_bits: uint16 [S][Hkv][D]) sits
+    at position p = seq_lens[s] - 1.  A sink goes to its window slot.  Otherwise the token that
+    leaves the recent window (position p - w_recent, if it is not a sink) is rotated and
+    quantized from its window slot into the INT4 pages at its quantized index, and the new
+    token takes that slot; with w_recent = 0 the new token itself is quantized.  Sequences with
+    seq_lens[s] <= 0 are skipped."""
+    k_bits = _as(k_bits, np.uint16)
+    v_bits = _as(v_bits, np.uint16)
+    for s in range(len(seq_lens)):
+        L = int(seq_lens[s])
+        if L <= 0:
+            continue
+        p = L - 1
+        if p < w_sink:
+            pg, off = _win_page_off(win_table, s, p)
+            win_kv[pg, :, 0, off] = k_bits[s]
+            win_kv[pg, :, 1, off] = v_bits[s]
+            continue
+        if w_recent == 0:
+            bad = rotate_quantize_paged(k_bits[s][None].copy(), v_bits[s][None].copy(),
+                                        np.array([_q_slot(block_table, s, p - w_sink)], np.int64),
+                                        kv_pages, scales, rotate=rotate)
+            assert bad == 0
+            continue
+        pg, off = _win_page_off(win_table, s, window_slot(p, w_sink, w_recent))
+        old = p - w_recent
+        if old >= w_sink:
+            bad = rotate_quantize_paged(win_kv[pg, :, 0, off][None].copy(),
+                                        win_kv[pg, :, 1, off][None].copy(),
+                                        np.array([_q_slot(block_table, s, old - w_sink)], np.int64),
+                                        kv_pages, scales, rotate=rotate)
+            assert bad == 0
+        win_kv[pg, :, 0, off] = k_bits[s]
+        win_kv[pg, :, 1, off] = v_bits[s]
+
+
+def decode_window_fp64(q_bits, win_kv, win_table, kv_pages, scales, block_table, seq_lens,
+                       w_sink, w_recent, *, sm_scale=None, rotate=True, nthreads=1) -> np.ndarray:
+    """fp64 decode attention over the window (bf16 pages [P_w][Hkv][2][16][D] through win_table)
+    and the quantized tokens (INT4 pages through block_table), one softmax over both, in the
+    original domain.  Returns fp64 [S][Hq][D]."""
+    q_bits = _as(q_bits, np.uint16)
+    win_kv = _as(win_kv, np.uint16)
+    win_table = _as(win_table, np.int32)
+    block_table = _as(block_table, np.int32)
+    seq_lens = _as(seq_lens, np.int32)
+    S, Hq, D = q_bits.shape
+    num_pages, Hkv, _, page_size, half = kv_pages.shape
+    assert half * 2 == D and Hq % Hkv == 0 and win_kv.shape[1:] == (Hkv, 2, page_size, D)
+    assert win_table.shape[0] == S and block_table.shape[0] == S and seq_lens.shape == (S,)
+    if sm_scale is None:
+        sm_scale = 1.0 / np.sqrt(D)
+    out = np.zeros((S, Hq, D), dtype=np.float64)
+    _load().oracle_decode_window_fp64(_ptr(q_bits), _ptr(win_kv), _ptr(win_table),
+                                      win_table.shape[1], _ptr(kv_pages), _ptr(scales),
+                                      _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
+                                      Hq, Hkv, D, page_size, int(w_sink), int(w_recent),
+                                      float(sm_scale), 1 if rotate else 0, _ptr(out), int(nthreads))
+    return out

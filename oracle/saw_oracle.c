@@ -395,6 +395,101 @@ void oracle_decode_bf16_fp64(const uint16_t *q, const uint16_t *kv_bf16,
     }
 }
 
+/* ---- full-precision sink / recent window beside the INT4 cache -------------------------- */
+/*
+ * "InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large Language Models",
+ * Abstract and Figure 2: a small high-precision window of attention-sink tokens and recent
+ * tokens is kept beside the quantized cache; the attention over the quantized part and over the
+ * window are computed separately and merged.  Readings (the pages give no layout):
+ *   - positions p < w_sink of a sequence of L tokens are sinks and positions
+ *     p >= max(w_sink, L - w_recent) are recent; both stay in bf16 in the window, the others are
+ *     quantized (rotated INT4) -- a sequence has min(L, W) window tokens and max(0, L - W)
+ *     quantized ones (W = w_sink + w_recent);
+ *   - window slot of position p: p for a sink, w_sink + (p - w_sink) mod w_recent for a recent
+ *     token; window slot i lives in bf16 page win_table[s][i / 16] at offset i mod 16 (the layout
+ *     of the bf16 baseline cache), so the occupied slots are always 0 .. min(L, W) - 1;
+ *   - the quantized tokens form their own paged INT4 sequence: position p is quantized index
+ *     j = p - w_sink, stored in page block_table[s][j / 16] at offset j mod 16.
+ * The reference attends in the original (unrotated) domain: each quantized key and value is
+ * dequantized and rotated back by the same normalised Hadamard transform, then one softmax runs
+ * over the window tokens and the quantized tokens together (the merged result the figure
+ * describes).  fp64 throughout. */
+static void oracle_window_token(const uint16_t *win_kv, const int32_t *win_table, int win_blocks,
+                                const uint8_t *kv_pages, const uint16_t *scales,
+                                const int32_t *block_table, int max_blocks, int s, int h,
+                                int Hkv, int D, int page_size, int L_w, int t, int sel,
+                                int rotate, double *y)
+{
+    if (t < L_w) {   /* window slot t */
+        const int64_t page = win_table[(size_t)s * win_blocks + t / page_size];
+        const uint16_t *r = win_kv + ((((size_t)page * Hkv + h) * 2 + sel) * page_size + t % page_size) * D;
+        for (int d = 0; d < D; d++)
+            y[d] = (double)oracle_bf16_to_f32(r[d]);
+    } else {         /* quantized index j */
+        const int j = t - L_w;
+        const int64_t page = block_table[(size_t)s * max_blocks + j / page_size];
+        oracle_dequant_row_f64(kv_pages, scales, Hkv, D, page_size, page, h, sel, j % page_size, y);
+        if (rotate)
+            oracle_rotate_f64(y, D);
+    }
+}
+
+void oracle_decode_window_fp64(const uint16_t *q, const uint16_t *win_kv, const int32_t *win_table,
+                               int win_blocks, const uint8_t *kv_pages, const uint16_t *scales,
+                               const int32_t *block_table, int max_blocks, const int32_t *seq_lens,
+                               int S, int Hq, int Hkv, int D, int page_size, int w_sink,
+                               int w_recent, double sm_scale, int rotate, double *out, int nthreads)
+{
+    const int G = Hq / Hkv;
+    const int W = w_sink + w_recent;
+#pragma omp parallel for collapse(2) schedule(dynamic) num_threads(nthreads)
+    for (int s = 0; s < S; s++) {
+        for (int hq = 0; hq < Hq; hq++) {
+            const int h = hq / G;
+            const int L = seq_lens[s];
+            double qd[1024], kv[1024], o[1024];
+            double *dst = out + ((size_t)s * Hq + hq) * D;
+            if (L <= 0) {
+                for (int d = 0; d < D; d++)
+                    dst[d] = 0.0;
+                continue;
+            }
+            const int L_w = L < W ? L : W;
+            const int n = L_w + (L > W ? L - W : 0);   /* every token once */
+            for (int d = 0; d < D; d++)
+                qd[d] = (double)oracle_bf16_to_f32(q[((size_t)s * Hq + hq) * D + d]);
+            double m = -INFINITY;
+            for (int t = 0; t < n; t++) {
+                oracle_window_token(win_kv, win_table, win_blocks, kv_pages, scales, block_table,
+                                    max_blocks, s, h, Hkv, D, page_size, L_w, t, 0, rotate, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qd[d] * kv[d];
+                if (sm_scale * acc > m)
+                    m = sm_scale * acc;
+            }
+            double l = 0.0;
+            for (int d = 0; d < D; d++)
+                o[d] = 0.0;
+            for (int t = 0; t < n; t++) {
+                oracle_window_token(win_kv, win_table, win_blocks, kv_pages, scales, block_table,
+                                    max_blocks, s, h, Hkv, D, page_size, L_w, t, 0, rotate, kv);
+                double acc = 0.0;
+                for (int d = 0; d < D; d++)
+                    acc += qd[d] * kv[d];
+                const double p = exp(sm_scale * acc - m);
+                l += p;
+                oracle_window_token(win_kv, win_table, win_blocks, kv_pages, scales, block_table,
+                                    max_blocks, s, h, Hkv, D, page_size, L_w, t, 1, rotate, kv);
+                for (int d = 0; d < D; d++)
+                    o[d] += p * kv[d];
+            }
+            for (int d = 0; d < D; d++)
+                dst[d] = o[d] / l;
+        }
+    }
+}
+
 /* ---- chunked-prefill attention over the INT4 cache ------------------------------------- */
 /*
  * The read step for a chunk of new tokens whose K/V are already in the paged cache ("SAW-INT4",

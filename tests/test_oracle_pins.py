@@ -692,3 +692,134 @@ def test_prefill_rows_equal_decode_on_their_prefix():
             dec = oracle.decode_fp64(qb[row:row + 1], pages, scales, wl.block_table[s:s + 1],
                                      np.array([L - C + i + 1], dtype=np.int32))
             assert np.allclose(got[row], dec[0], atol=1e-12, rtol=1e-12)
+
+
+# ---------------------------------------------------------------------------------------
+# full-precision sink / recent window ("InnerQ", Abstract and Figure 2)
+# ---------------------------------------------------------------------------------------
+
+def _window_state(lens, w_sink, w_recent, Hkv=2, D=128, seed=0, rotate=True):
+    """Token values for every position and the oracle window state after filling them."""
+    S, Lmax = len(lens), max(max(lens), 1)
+    g = torch.Generator().manual_seed(seed)
+    k = torch.randn(S, Lmax, Hkv, D, generator=g)
+    k[..., 3] *= 20.0                                   # an outlier key channel
+    k = synth.bf16_bits(k.to(torch.bfloat16))
+    v = synth.bf16_bits(torch.randn(S, Lmax, Hkv, D, generator=g).to(torch.bfloat16))
+    W = w_sink + w_recent
+    pw = max(1, (W + 15) // 16)
+    win_table = (np.arange(S * pw, dtype=np.int32).reshape(S, pw) * 7 + 3) % (S * pw)
+    win_kv = np.zeros((S * pw, Hkv, 2, 16, D), np.uint16)
+    nq = max(1, (Lmax + 15) // 16)
+    block_table = np.random.default_rng(seed).permutation(S * nq).astype(np.int32).reshape(S, nq)
+    pages, scales = oracle.empty_cache(S * nq, Hkv, D)
+    oracle.window_fill(k, v, np.array(lens), w_sink, w_recent, win_kv, win_table, pages, scales,
+                       block_table, rotate=rotate)
+    return k, v, win_kv, win_table, pages, scales, block_table
+
+
+def test_window_of_width_zero_is_the_int4_decode():
+    """w_sink = w_recent = 0: every token is quantized; the window decode (which rotates keys and
+    values back) equals the INT4 decode (which rotates the query and the output)."""
+    lens = [37, 1, 16, 70]
+    k, v, win_kv, win_table, pages, scales, bt = _window_state(lens, 0, 0, seed=1)
+    q = synth.bf16_bits(torch.randn(len(lens), 4, 128).to(torch.bfloat16))
+    a = oracle.decode_window_fp64(q, win_kv, win_table, pages, scales, bt,
+                                  np.array(lens, np.int32), 0, 0)
+    b = oracle.decode_fp64(q, pages, scales, bt, np.array(lens, np.int32))
+    assert np.abs(a - b).max() <= 1e-12
+
+
+@pytest.mark.parametrize("w_sink,w_recent", [(4, 60), (16, 112), (0, 40)])
+def test_window_covering_the_sequence_is_bf16_attention(w_sink, w_recent):
+    """L <= W: nothing is quantized; the output is fp64 SDPA over the bf16 keys and values."""
+    lens = [1, 5, w_sink + w_recent, 17]
+    k, v, win_kv, win_table, pages, scales, bt = _window_state(lens, w_sink, w_recent, seed=2)
+    q = synth.bf16_bits(torch.randn(len(lens), 2, 128).to(torch.bfloat16))
+    out = oracle.decode_window_fp64(q, win_kv, win_table, pages, scales, bt,
+                                    np.array(lens, np.int32), w_sink, w_recent)
+    tq = torch.from_numpy(q.view(np.int16)).view(torch.bfloat16).double()
+    tk = torch.from_numpy(k.view(np.int16)).view(torch.bfloat16).double()
+    tv = torch.from_numpy(v.view(np.int16)).view(torch.bfloat16).double()
+    for s, L in enumerate(lens):
+        for hq in range(2):
+            o = torch.nn.functional.scaled_dot_product_attention(
+                tq[s, hq][None, None, None], tk[s, :L, hq][None, None], tv[s, :L, hq][None, None])
+            assert torch.allclose(torch.from_numpy(out[s, hq]), o[0, 0, 0], atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("w_sink,w_recent", [(4, 12), (16, 112), (0, 32), (8, 0)])
+def test_window_matches_sdpa_over_bf16_window_and_dequantized_middle(w_sink, w_recent):
+    """Every position once: sinks and recent tokens with their bf16 values, the middle tokens
+    dequantized and rotated back; fp64 SDPA over that set equals the oracle."""
+    lens = [300, 3, 150, 128]
+    k, v, win_kv, win_table, pages, scales, bt = _window_state(lens, w_sink, w_recent, seed=3)
+    q = synth.bf16_bits(torch.randn(len(lens), 4, 128).to(torch.bfloat16))
+    out = oracle.decode_window_fp64(q, win_kv, win_table, pages, scales, bt,
+                                    np.array(lens, np.int32), w_sink, w_recent)
+    bf = lambda a: torch.from_numpy(a.view(np.int16)).view(torch.bfloat16).double()
+    tq, tk, tv = bf(q), bf(k), bf(v)
+    for s, L in enumerate(lens):
+        for hq in range(4):
+            h = hq // 2
+            keys, vals = [], []
+            for p in range(L):
+                if p < w_sink or p >= max(w_sink, L - w_recent):
+                    keys.append(tk[s, p, h])
+                    vals.append(tv[s, p, h])
+                else:
+                    j = p - w_sink
+                    pg, off = int(bt[s, j // 16]), j % 16
+                    keys.append(torch.from_numpy(oracle.rotate_f64(
+                        oracle.dequant_row_f64(pages, scales, pg, h, 0, off))))
+                    vals.append(torch.from_numpy(oracle.rotate_f64(
+                        oracle.dequant_row_f64(pages, scales, pg, h, 1, off))))
+            o = torch.nn.functional.scaled_dot_product_attention(
+                tq[s, hq][None, None, None], torch.stack(keys)[None, None],
+                torch.stack(vals)[None, None])[0, 0, 0]
+            assert torch.allclose(torch.from_numpy(out[s, hq]), o, atol=1e-12, rtol=0)
+
+
+@pytest.mark.parametrize("w_sink,w_recent", [(4, 12), (16, 112), (0, 32), (8, 0), (16, 16)])
+def test_window_append_steps_equal_fill(w_sink, w_recent):
+    """Appending tokens one step at a time (the quantized token is the one leaving the recent
+    window) reaches exactly the state that placing every token directly gives: window bits and
+    INT4 codes / scales bit-identical.  The window then holds the sinks and the last w_recent
+    tokens at their slots."""
+    L0, steps = [0, 3, 20, 140], 37
+    L1 = [x + steps for x in L0]
+    k, v, win_kv, win_table, pages, scales, bt = _window_state(L1, w_sink, w_recent, seed=4)
+    win2 = np.zeros_like(win_kv)
+    pages2, scales2 = oracle.empty_cache(*pages.shape[:2], 128)
+    oracle.window_fill(k, v, np.array(L0), w_sink, w_recent, win2, win_table, pages2, scales2, bt)
+    for i in range(1, steps + 1):
+        lens = np.array([x + i for x in L0])
+        kn = np.stack([k[s, lens[s] - 1] for s in range(len(L0))])
+        vn = np.stack([v[s, lens[s] - 1] for s in range(len(L0))])
+        oracle.window_append(kn, vn, lens, w_sink, w_recent, win2, win_table, pages2, scales2, bt)
+    assert np.array_equal(win2, win_kv)
+    assert np.array_equal(pages2, pages) and np.array_equal(scales2, scales)
+    s, L = 3, L1[3]                                   # direct check of the window contents
+    for p in list(range(min(L, w_sink))) + list(range(max(w_sink, L - w_recent), L)):
+        slot = oracle.window_slot(p, w_sink, w_recent)
+        pg = win_table[s, slot // 16]
+        assert np.array_equal(win_kv[pg, :, 0, slot % 16], k[s, p])
+        assert np.array_equal(win_kv[pg, :, 1, slot % 16], v[s, p])
+
+
+def test_window_decode_ignores_the_order_of_window_slots():
+    """The window is a set: moving its tokens to other slots (and pages) leaves the output."""
+    lens = [200, 90]
+    k, v, win_kv, win_table, pages, scales, bt = _window_state(lens, 16, 48, seed=5)
+    q = synth.bf16_bits(torch.randn(2, 4, 128).to(torch.bfloat16))
+    a = oracle.decode_window_fp64(q, win_kv, win_table, pages, scales, bt,
+                                  np.array(lens, np.int32), 16, 48)
+    perm = np.random.default_rng(0).permutation(64)
+    win_b = win_kv.copy()
+    for s in range(2):
+        for i in range(64):
+            j = perm[i]
+            win_b[win_table[s, j // 16], :, :, j % 16] = win_kv[win_table[s, i // 16], :, :, i % 16]
+    b = oracle.decode_window_fp64(q, win_b, win_table, pages, scales, bt,
+                                  np.array(lens, np.int32), 16, 48)
+    assert np.abs(a - b).max() <= 1e-12
