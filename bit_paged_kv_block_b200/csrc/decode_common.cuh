@@ -99,7 +99,25 @@ struct DecodeParams {
     int32_t total_warps;         // warps of the decode grid (the plan's slice count bound)
     int32_t qrows;               // rows of each warp's query buffer: min(8, C G) bound
     float q_mult;                // the factor the kernel applies to q (or to the logits)
+    // Full-precision window beside the quantized cache (decode only): win_part 1 attends over
+    // the min(L, W) window tokens of each sequence and writes out rows and lse[row] = the log2
+    // of the softmax denominator; win_part 2 attends over the max(0, L - W) quantized tokens
+    // and merges its result into the out rows part 1 wrote (W = win_sink + win_recent).
+    float *lse = nullptr;
+    int32_t win_part = 0;
+    int32_t win_sink = 0, win_recent = 0;
 };
+
+// Tokens this launch attends over in a sequence of seq_lens[s] tokens (a negative length is
+// passed through, to be flagged).
+__device__ __forceinline__ int attended_len(const DecodeParams &p, int s)
+{
+    const int L = p.seq_lens[s];
+    if (p.win_part == 0 || L < 0)
+        return L;
+    const int W = p.win_sink + p.win_recent;
+    return p.win_part == 1 ? min(L, W) : max(0, L - W);
+}
 
 // ---- per-sequence tables and the work plan -----------------------------------------------------
 
@@ -145,7 +163,7 @@ __device__ inline void scan_sequences(const DecodeParams &p, const SeqTables &tb
     int64_t local_pages = 0;
     int32_t local_segs = 0;
     for (int s = s0; s < s1; s++) {
-        const int len = p.seq_lens[s];
+        const int len = attended_len(p, s);
         const int c = query_tokens<kPrefill>(p, s);
         const bool len_ok = len >= 0 && len <= p.max_blocks * kPageSize;
         const bool q_ok = !kPrefill || (c >= 0 && c <= len);
@@ -299,7 +317,7 @@ struct Segment {
         b = j - h * nb;
         n = tb.npg[s];
         c = query_tokens<kPrefill>(p, s);
-        len = p.seq_lens[s];
+        len = attended_len(p, s);
         row0 = kRowsPerBlock * b;
         nrows = min(kRowsPerBlock, c * p.group - row0);
         qrow0 = query_row0<kPrefill>(p, s);
@@ -546,7 +564,7 @@ __global__ void __launch_bounds__(kMergeThreads)
             }
             Segment<kPrefill> sg;
             sg.init(p, tb, s, j);
-            Fmt::finalize(p, sg, lane, st.o, st.l);
+            Fmt::finalize(p, sg, lane, st.o, st.m, st.l);
         }
         __syncthreads();
     }
@@ -568,7 +586,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 //   page<kMask>(ring, stg, mask, q, lane, st)      attend over one staged page (PageMask when
 //                                                  kMask: never-written tokens, causal limits);
 //   piece_end(st)                                  reductions and corrections after a piece;
-//   finalize(p, segment, lane, o, l)               write a finished segment's output rows (a
+//   finalize(p, segment, lane, o, m, l)            write a finished segment's output rows (a
 //                                                  template on the segment type)
 //                                                  (also the merge kernel's output step).
 // Shared memory: rings, then per warp (kStages + 1) mbarriers (the last for the query), 128 bytes
@@ -613,12 +631,18 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     // ---- 1. sequence tables, the plan, zero the output rows that get no segment ----------------
     scan_sequences<kPrefill>(p, tb, flags, blockIdx.x == 0);
     pdl_launch_dependents();   // the merge kernel may start its own prologue
-    for (int s = blockIdx.x; s < S; s += gridDim.x) {
+    // (the quantized part of a windowed decode leaves such rows to the window part, which
+    // also marks their lse empty)
+    for (int s = blockIdx.x; s < S && p.win_part != 2; s += gridDim.x) {
         const int c = query_tokens<kPrefill>(p, s);
         if (tb.nbk[s] == 0 && c > 0 && (!kPrefill || c <= p.seq_lens[s])) {
-            float4 *dst = reinterpret_cast<float4 *>(p.out + query_row0<kPrefill>(p, s) * p.hq * Fmt::kDim);
+            const int64_t row0 = query_row0<kPrefill>(p, s) * p.hq;
+            float4 *dst = reinterpret_cast<float4 *>(p.out + row0 * Fmt::kDim);
             for (int i = tid; i < c * p.hq * Fmt::kDim / 4; i += 32 * Fmt::kWarps)
                 dst[i] = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+            if (p.lse != nullptr)
+                for (int i = tid; i < c * p.hq; i += 32 * Fmt::kWarps)
+                    p.lse[row0 + i] = -INFINITY;
         }
     }
     if (tb.spre[S] > p.max_segments) {   // more query rows than the workspace was sized for
@@ -802,7 +826,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         if (seg_start >= F0 && ends_segment) {
             Segment<kPrefill> sg;
             sg.init(p, tb, cs, cj);
-            Fmt::finalize(p, sg, lane, st.o, st.l);
+            Fmt::finalize(p, sg, lane, st.o, st.m, st.l);
         } else {
             store_partial(p.partials + (tb.spre[cs] + cj + u) * slot_floats<Fmt::kTiles>(), lane, st);
         }

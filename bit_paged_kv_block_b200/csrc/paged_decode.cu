@@ -279,10 +279,12 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
 
 
 // o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the block rows 2t, 2t + 1
-// this thread holds; H acts on each 128-element block of d.
-template <bool kRotate, int kD, class Seg>
+// this thread holds; H acts on each block of min(kD, 128) elements of d.  As the quantized part
+// of a windowed decode, out instead becomes the softmax-weighted merge of this result and the
+// window part's row already in out: weights 2^lse / (2^lse_q + 2^lse_w), lse_q = m + log2 l.
+template <bool kRotate, int kD, bool kMerge, class Seg>
 __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, int lane,
-                                         float o[kD / 16][4], const float l[2])
+                                         float o[kD / 16][4], const float m[2], const float l[2])
 {
     constexpr int kC = kD / 32;   // 32-element chunks of d
     const int g = lane >> 2, t = lane & 3;
@@ -341,13 +343,28 @@ __device__ __forceinline__ void finalize(const DecodeParams &p, const Seg &sg, i
     for (int e = 0; e < 2; e++) {
         const int head = 2 * t + e;
         if (head < sg.nrows) {
-            float *dst = p.out + sg.row_offset(p, head, kD);
+            const int64_t off = sg.row_offset(p, head, kD);
+            float *dst = p.out + off;
+            float f = kRotate ? hadamard_c(kD) : 1.0f, fw = 0.0f;
+            if (kMerge) {
+                const float lq = m[e] + log2f(l[e]), lw = p.lse[off / kD];
+                const float mx = fmaxf(lq, lw);
+                const float aq = exp2f(lq - mx), aw = exp2f(lw - mx);
+                const float inv = 1.0f / (aq + aw);
+                f *= aq * inv;
+                fw = aw * inv;
+            }
 #pragma unroll
             for (int c = 0; c < kC; c++) {
-                const float f = kRotate ? hadamard_c(kD) : 1.0f;
-                const float4 val = make_float4(v[e][c][0] * f, v[e][c][1] * f, v[e][c][2] * f,
-                                               v[e][c][3] * f);
-                *reinterpret_cast<float4 *>(dst + 32 * c + 4 * g) = val;
+                float4 val = make_float4(v[e][c][0] * f, v[e][c][1] * f, v[e][c][2] * f,
+                                         v[e][c][3] * f);
+                float4 *d4 = reinterpret_cast<float4 *>(dst + 32 * c + 4 * g);
+                if (kMerge) {
+                    const float4 w = *d4;
+                    val = make_float4(fmaf(fw, w.x, val.x), fmaf(fw, w.y, val.y),
+                                      fmaf(fw, w.z, val.z), fmaf(fw, w.w, val.w));
+                }
+                *d4 = val;
             }
         }
     }
@@ -381,9 +398,11 @@ __device__ __forceinline__ void copy_page_elected(uint32_t bar, uint32_t dst_cod
 // swizzle for kD = 128, 4 KiB with the 128B swizzle for kD = 256), codes of all stages first,
 // then the scales (128 B each).  kD = 128: 4 stages, 4 CTAs per SM; kD = 256 (twice the
 // accumulators): 2 stages, 3 CTAs per SM, which keeps about as many bytes in flight per SM;
-// kD = 64 (half the registers, half the bytes per page): 4 stages, 6 CTAs per SM, since a warp
+// kD = 64 (half the registers, half the bytes per page): 4 stages, 5 CTAs per SM, since a warp
 // completes its page copies one after another and more warps keep more copies in flight.
-template <bool kRotate, int kD>
+// kMerge: the quantized part of a windowed decode, whose finalize merges into the window part's
+// output rows (a separate instantiation, so the plain decode carries none of it).
+template <bool kRotate, int kD, bool kMerge = false>
 struct Int4Format {
     static_assert(kD == 64 || kD == 128 || kD == 256, "head dimension");
     static constexpr int kDim = kD;
@@ -447,9 +466,9 @@ struct Int4Format {
     }
     template <class Seg>
     __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane,
-                                    float o[kTiles][4], const float l[2])
+                                    float o[kTiles][4], const float m[2], const float l[2])
     {
-        saw::finalize<kRotate, kD>(p, sg, lane, o, l);
+        saw::finalize<kRotate, kD, kMerge>(p, sg, lane, o, m, l);
     }
 };
 
@@ -471,6 +490,28 @@ cudaError_t launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
         reinterpret_cast<const void *>(paged_decode_merge_kernel<Int4Format<false, kD>, true>)};
     return decode::launch_shape(shapes, decode_kernels, merge_kernels,
                                 32 * Int4Format<true, kD>::kWarps, smem, merge_smem, out);
+}
+
+// The windowed decode's quantized part (rotated, decode, head_dim 128): only the shared-memory
+// attributes are set here; its grid is the plain family's (same layout and launch bounds), which
+// the workspace is sized for.
+cudaError_t set_window_merge_attributes(size_t smem, size_t merge_smem)
+{
+    static ShapeCache shapes;
+    using W = Int4Format<true, 128, true>;
+    static const void *const decode_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>)};
+    static const void *const merge_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>)};
+    LaunchShape unused;
+    return decode::launch_shape(shapes, decode_kernels, merge_kernels, 32 * W::kWarps, smem,
+                                merge_smem, unused);
 }
 
 template <int kD>
@@ -554,6 +595,10 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
     p.qrows = qrows;
+    p.lse = a.lse;
+    p.win_part = a.win_part;
+    p.win_sink = a.win_sink;
+    p.win_recent = a.win_recent;
     p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Fmt::kWarps;
     // q carries sm_scale * log2(e), and 1/sqrt(B) of the (unnormalised) query butterfly
@@ -571,10 +616,16 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    auto *kernel = a.rotate ? (prefill ? paged_decode_kernel<Int4Format<true, kD>, true>
-                                       : paged_decode_kernel<Int4Format<true, kD>, false>)
-                            : (prefill ? paged_decode_kernel<Int4Format<false, kD>, true>
-                                       : paged_decode_kernel<Int4Format<false, kD>, false>);
+    const bool window_merge = a.win_part == 2;
+    if (window_merge && (kD != 128 || prefill || !a.rotate))
+        return cudaErrorInvalidValue;
+    if (window_merge && (e = set_window_merge_attributes(smem, msmem)) != cudaSuccess)
+        return e;
+    auto *kernel = window_merge ? paged_decode_kernel<Int4Format<true, kD, true>, false>
+                   : a.rotate   ? (prefill ? paged_decode_kernel<Int4Format<true, kD>, true>
+                                           : paged_decode_kernel<Int4Format<true, kD>, false>)
+                                : (prefill ? paged_decode_kernel<Int4Format<false, kD>, true>
+                                           : paged_decode_kernel<Int4Format<false, kD>, false>);
     e = cudaLaunchKernelEx(&cfg, kernel, *map, p);
     if (e != cudaSuccess)
         return e;
@@ -585,10 +636,11 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    auto *merge = a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true>
-                                      : paged_decode_merge_kernel<Int4Format<true, kD>, false>)
-                           : (prefill ? paged_decode_merge_kernel<Int4Format<false, kD>, true>
-                                      : paged_decode_merge_kernel<Int4Format<false, kD>, false>);
+    auto *merge = window_merge ? paged_decode_merge_kernel<Int4Format<true, kD, true>, false>
+                  : a.rotate   ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true>
+                                          : paged_decode_merge_kernel<Int4Format<true, kD>, false>)
+                               : (prefill ? paged_decode_merge_kernel<Int4Format<false, kD>, true>
+                                          : paged_decode_merge_kernel<Int4Format<false, kD>, false>);
     e = cudaLaunchKernelEx(&mcfg, merge, p);
     if (e != cudaSuccess)
         return e;

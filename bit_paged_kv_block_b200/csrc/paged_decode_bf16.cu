@@ -50,7 +50,10 @@ __device__ __forceinline__ uint32_t bf16_chunk(int sel, int tok, int d0)
     return row * kBf16RowBytes + ((chunk ^ (row & 7)) << 4);
 }
 
-struct Bf16Format {
+// kLse: the window part of a windowed decode, which also records each row's log2 softmax
+// denominator (a separate instantiation, so the plain decode carries none of it).
+template <bool kLse>
+struct Bf16FormatT {
     static constexpr int kDim = kHeadDim;
     static constexpr int kTiles = kHeadDim / 16;
     static constexpr int kWarps = 4;
@@ -178,9 +181,11 @@ struct Bf16Format {
     }
 
     // block row 2t + e: out[row][d] = o / l; tile c, rows g and g + 8 are d = 16 c + g (+ 8).
+    // As the window part of a windowed decode it also records lse[row] = m + log2 l, the log2 of
+    // the row's softmax denominator, for the quantized part to merge with.
     template <class Seg>
     __device__ static void finalize(const DecodeParams &p, const Seg &sg, int lane, float o[8][4],
-                                    const float l[2])
+                                    const float m[2], const float l[2])
     {
         const int g = lane >> 2, t = lane & 3;
 #pragma unroll
@@ -189,7 +194,10 @@ struct Bf16Format {
             if (head >= sg.nrows)
                 continue;
             const float inv = 1.0f / l[e];
-            float *dst = p.out + sg.row_offset(p, head, kHeadDim);
+            const int64_t off = sg.row_offset(p, head, kHeadDim);
+            float *dst = p.out + off;
+            if (kLse && g == 0)
+                p.lse[off / kHeadDim] = m[e] + log2f(l[e]);
 #pragma unroll
             for (int c = 0; c < 8; c++) {
                 dst[16 * c + g] = o[c][e] * inv;
@@ -198,6 +206,7 @@ struct Bf16Format {
         }
     }
 };
+using Bf16Format = Bf16FormatT<false>;
 
 // Scatter T tokens of bf16 K and V into the bf16 pages: one warp per (token, kv head), lanes
 // 0-15 moving the K vector and lanes 16-31 the V vector, 16 bytes each.
@@ -246,6 +255,27 @@ cudaError_t bf16_launch_shape(size_t smem, size_t merge_smem, LaunchShape &out)
         reinterpret_cast<const void *>(paged_decode_merge_kernel<Bf16Format, true>)};
     return decode::launch_shape(g_bf16_shapes, decode_kernels, merge_kernels,
                                 32 * Bf16Format::kWarps, smem, merge_smem, out);
+}
+
+// The window part of a windowed decode: only the shared-memory attributes are set here; its grid
+// is the plain family's (same layout and launch bounds), which the workspace is sized for.
+cudaError_t set_window_attributes(size_t smem, size_t merge_smem)
+{
+    static ShapeCache shapes;
+    using W = Bf16FormatT<true>;
+    static const void *const decode_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_kernel<W, false>)};
+    static const void *const merge_kernels[kShapeVariants] = {
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>),
+        reinterpret_cast<const void *>(paged_decode_merge_kernel<W, false>)};
+    LaunchShape unused;
+    return decode::launch_shape(shapes, decode_kernels, merge_kernels, 32 * W::kWarps, smem,
+                                merge_smem, unused);
 }
 
 }  // namespace
@@ -335,6 +365,10 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     p.hkv = a.num_kv_heads;
     p.group = a.num_q_heads / a.num_kv_heads;
     p.qrows = qrows;
+    p.lse = a.lse;
+    p.win_part = a.win_part;
+    p.win_sink = a.win_sink;
+    p.win_recent = a.win_recent;
     p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Bf16Format::kWarps;
     p.q_mult = static_cast<float>(static_cast<double>(a.sm_scale) * 1.4426950408889634);
@@ -349,8 +383,14 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     cfg.stream = stream;
     cfg.attrs = attr;
     cfg.numAttrs = programmatic ? 1 : 0;
-    e = cudaLaunchKernelEx(&cfg, prefill ? paged_decode_kernel<Bf16Format, true>
-                                         : paged_decode_kernel<Bf16Format, false>,
+    const bool window = a.win_part == 1;
+    if (window && prefill)
+        return cudaErrorInvalidValue;
+    if (window && (e = set_window_attributes(smem, msmem)) != cudaSuccess)
+        return e;
+    e = cudaLaunchKernelEx(&cfg, window    ? paged_decode_kernel<Bf16FormatT<true>, false>
+                                 : prefill ? paged_decode_kernel<Bf16Format, true>
+                                           : paged_decode_kernel<Bf16Format, false>,
                            cache.map, p);
     if (e != cudaSuccess)
         return e;
@@ -361,8 +401,9 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&mcfg, prefill ? paged_decode_merge_kernel<Bf16Format, true>
-                                          : paged_decode_merge_kernel<Bf16Format, false>,
+    e = cudaLaunchKernelEx(&mcfg, window    ? paged_decode_merge_kernel<Bf16FormatT<true>, false>
+                                  : prefill ? paged_decode_merge_kernel<Bf16Format, true>
+                                            : paged_decode_merge_kernel<Bf16Format, false>,
                            p);
     if (e != cudaSuccess)
         return e;

@@ -487,7 +487,147 @@ __global__ void __launch_bounds__(kRqThreads, 4)
     }
 }
 
+// ---- the full-precision window beside the INT4 cache: one serving step ----------------------
+//
+// "InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large Language Models",
+// Abstract and Figure 2: a small bf16 window of sink and recent tokens stays beside the quantized
+// cache.  Sequence s's new token sits at position p = seq_lens[s] - 1: a sink (p < w_sink) takes
+// window slot p; otherwise its slot in the recent ring is w_sink + (p - w_sink) mod w_recent, and
+// the token it displaces (position p - w_recent, when that is not a sink) is rotated, quantized
+// and scattered into the INT4 pages at quantized index p - w_recent - w_sink, bit-identically to
+// the rotate+quantize kernel (same device code).  With w_recent = 0 the new token itself is
+// quantized.  Window slot i lives in bf16 page win_table[s][i / 16] at offset i mod 16.
+//
+// Lanes as in the rotate+quantize kernel at D = 128: a warp takes 8 (sequence, kv head) pairs,
+// lanes 0-15 their K vectors and lanes 16-31 their V vectors, two threads per vector.  Each
+// thread reads exactly the 128 bytes of the displaced vector it later overwrites with the new
+// token, so the read and the write of a slot are ordered within one thread.
+struct WinAppendParams {
+    const uint16_t *k, *v;
+    const int32_t *seq_lens;
+    int32_t num_seqs, hkv, w_sink, w_recent;
+    uint16_t *win_kv;
+    const int32_t *win_table;
+    int32_t win_blocks;
+    int64_t num_win_pages;
+    const int32_t *block_table;
+    int32_t max_blocks;
+    int64_t num_pages;
+    RqParams q;        // kv_pages and scales for quantize_store; status
+};
+
+template <bool kRotate>
+__global__ void __launch_bounds__(kRqThreads)
+    window_append_kernel(const WinAppendParams p)
+{
+    pdl_launch_dependents();
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    const int half = lane >> 4, b = lane & 1, vt = (lane & 15) >> 1;
+    const int64_t pair = (static_cast<int64_t>(blockIdx.x) * kRqWarps + warp) * 8 + vt;
+    const bool live = pair < static_cast<int64_t>(p.num_seqs) * p.hkv;
+    const int s = live ? static_cast<int>(pair / p.hkv) : 0;
+    const int h = live ? static_cast<int>(pair - static_cast<int64_t>(s) * p.hkv) : 0;
+    const int L = live ? p.seq_lens[s] : 0;
+    const bool report = b == 0 && half == 0;
+
+    // where the new token goes and which token is quantized
+    bool to_win = false, quant = false, from_win = false;
+    int slot = 0, j = 0;
+    if (L > 0) {
+        const int pos = L - 1;
+        if (pos < p.w_sink) {
+            to_win = true;
+            slot = pos;
+        } else if (p.w_recent == 0) {
+            quant = true;
+            j = pos - p.w_sink;
+        } else {
+            to_win = true;
+            slot = p.w_sink + (pos - p.w_sink) % p.w_recent;
+            if (pos - p.w_recent >= p.w_sink) {
+                quant = from_win = true;
+                j = pos - p.w_recent - p.w_sink;
+            }
+        }
+    } else if (L < 0 && report) {
+        set_status(p.q.status, SAW_DEV_BAD_SEQ_LEN);
+    }
+    uint16_t *win = nullptr;
+    if (to_win) {
+        const int32_t page = p.win_table[static_cast<int64_t>(s) * p.win_blocks + slot / 16];
+        if (page < 0 || page >= p.num_win_pages) {
+            if (report)
+                set_status(p.q.status, SAW_DEV_BAD_PAGE);
+            to_win = quant = false;   // the displaced token cannot be read: leave the pair
+        } else {
+            win = p.win_kv + ((((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize) +
+                              slot % kPageSize) * 128;
+        }
+    }
+    int64_t row = 0;
+    if (quant) {
+        const int32_t page = j / kPageSize < p.max_blocks
+                                 ? p.block_table[static_cast<int64_t>(s) * p.max_blocks + j / kPageSize]
+                                 : -1;
+        if (page < 0 || page >= p.num_pages) {
+            if (report)
+                set_status(p.q.status, j / kPageSize < p.max_blocks ? SAW_DEV_BAD_PAGE : SAW_DEV_BAD_SEQ_LEN);
+            to_win = quant = false;   // keep the displaced token where it is
+        } else {
+            row = ((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize + j % kPageSize;
+        }
+    }
+
+    // this thread's 64 elements (16 a + 8 b + r) of the new vector and of the displaced one
+    uint4 fresh[8], raw[8];
+    const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128;
+#pragma unroll
+    for (int a = 0; a < 8; a++) {
+        fresh[a] = L > 0 ? *reinterpret_cast<const uint4 *>(src + 16 * a + 8 * b) : make_uint4(0, 0, 0, 0);
+        raw[a] = from_win && quant ? *reinterpret_cast<const uint4 *>(win + 16 * a + 8 * b) : fresh[a];
+    }
+    uint64_t X[32];
+    to_pairs(raw, X);
+    if constexpr (kRotate)
+        fwht128(X, b, 0xFFFFFFFFu);
+    quantize_store<kRotate, 128>(X, 0, b, quant, row, p.q);
+    if (to_win) {
+#pragma unroll
+        for (int a = 0; a < 8; a++)
+            *reinterpret_cast<uint4 *>(win + 16 * a + 8 * b) = fresh[a];
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_window_append(const WindowAppendArgs &a, cudaStream_t stream)
+{
+    const int64_t pairs = static_cast<int64_t>(a.num_seqs) * a.num_kv_heads;
+    if (pairs == 0)
+        return cudaSuccess;
+    WinAppendParams p;
+    p.k = static_cast<const uint16_t *>(a.k);
+    p.v = static_cast<const uint16_t *>(a.v);
+    p.seq_lens = a.seq_lens;
+    p.num_seqs = a.num_seqs;
+    p.hkv = a.num_kv_heads;
+    p.w_sink = a.w_sink;
+    p.w_recent = a.w_recent;
+    p.win_kv = static_cast<uint16_t *>(a.win_kv);
+    p.win_table = a.win_table;
+    p.win_blocks = a.win_blocks;
+    p.num_win_pages = a.num_win_pages;
+    p.block_table = a.block_table;
+    p.max_blocks = a.max_blocks;
+    p.num_pages = a.num_pages;
+    p.q = RqParams{};
+    p.q.kv_pages = a.kv_pages;
+    p.q.scales = static_cast<uint32_t *>(a.scales);
+    p.q.status = a.status;
+    const int64_t grid = (pairs + 8 * kRqWarps - 1) / (8 * kRqWarps);
+    window_append_kernel<true><<<static_cast<unsigned>(grid), kRqThreads, 0, stream>>>(p);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t stream,
                                    bool trigger_dependents)

@@ -2,6 +2,7 @@
 //
 // Argument validation, workspace sizing and kernel launches.  Nothing here allocates device
 // memory; every launch is asynchronous on the caller's stream.
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 
@@ -551,6 +552,217 @@ int saw_paged_prefill_attn_plain(const saw_cache_desc *cache, int32_t num_q_head
     return prefill_impl(cache, num_q_heads, q, q_start, total_q, kv_pages, scales, block_table,
                         max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
                         workspace_bytes, dev_status, stream, false);
+}
+
+// ---- full-precision sink / recent window beside the INT4 cache ------------------------------
+
+static int check_window(const saw_cache_desc *cache, const saw_window_cache *win, int32_t num_seqs)
+{
+    if (win == nullptr || win->sink < 0 || win->recent < 0 || win->blocks < 0)
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (cache->head_dim != 128)
+        return SAW_ERR_UNSUPPORTED;   // the window pages use the bf16 page format: D = 128
+    const int64_t W = int64_t(win->sink) + win->recent;
+    if (W > int64_t(16) * win->blocks || W > (int64_t(1) << 30))
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (num_seqs > 0 && W > 0) {
+        if (win->kv == nullptr || win->table == nullptr || win->num_pages <= 0 ||
+            !aligned(win->kv, 16) || !aligned(win->table, 4))
+            return SAW_ERR_INVALID_ARGUMENT;
+        // tensor-map rows (page * Hkv + h) * 64 of the window pages must stay below 2^31
+        if (win->num_pages > (int64_t(1) << 31) / (int64_t(cache->num_kv_heads) * 64))
+            return SAW_ERR_UNSUPPORTED;
+    }
+    return SAW_OK;
+}
+
+// workspace: the split-K slots of either part (they run one after the other), then the window
+// part's per-row lse
+static size_t window_partials_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                    int32_t num_seqs)
+{
+    const size_t a = saw::decode_bf16_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs);
+    const size_t b = saw::decode_workspace_bytes(cache->num_kv_heads, num_q_heads, num_seqs, -1, 128);
+    if (a == 0 || b == 0)
+        return 0;
+    return (std::max(a, b) + 255) / 256 * 256;
+}
+
+size_t saw_paged_decode_window_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                               int32_t num_seqs)
+{
+    if (check_cache(cache) != SAW_OK || cache->head_dim != 128 || num_q_heads <= 0 ||
+        num_seqs < 0 || num_q_heads % cache->num_kv_heads != 0 ||
+        num_q_heads / cache->num_kv_heads > 16)
+        return 0;
+    const size_t part = window_partials_bytes(cache, num_q_heads, num_seqs);
+    return part == 0 ? 0 : part + size_t(num_seqs) * num_q_heads * sizeof(float);
+}
+
+static int window_append_impl(const saw_cache_desc *cache, const saw_window_cache *win,
+                              const void *k, const void *v, const int32_t *seq_lens,
+                              int32_t num_seqs, uint8_t *kv_pages, void *scales,
+                              const int32_t *block_table, int32_t max_blocks_per_seq,
+                              uint32_t *dev_status, cudaStream_t stream)
+{
+    saw::WindowAppendArgs a;
+    a.k = k;
+    a.v = v;
+    a.seq_lens = seq_lens;
+    a.num_seqs = num_seqs;
+    a.num_kv_heads = cache->num_kv_heads;
+    a.w_sink = win->sink;
+    a.w_recent = win->recent;
+    a.win_kv = win->kv;
+    a.num_win_pages = win->num_pages;
+    a.win_table = win->table;
+    a.win_blocks = win->blocks;
+    a.kv_pages = kv_pages;
+    a.scales = scales;
+    a.num_pages = cache->num_pages;
+    a.block_table = block_table;
+    a.max_blocks = max_blocks_per_seq;
+    a.status = dev_status;
+    return saw::launch_window_append(a, stream) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+}
+
+static int check_window_append(const saw_cache_desc *cache, const saw_window_cache *win,
+                               const void *k, const void *v, const int32_t *seq_lens,
+                               int32_t num_seqs, const uint8_t *kv_pages, const void *scales,
+                               const int32_t *block_table, int32_t max_blocks_per_seq)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_window(cache, win, num_seqs);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    if (num_seqs < 0 || !k || !v || !seq_lens || !kv_pages || !scales || !block_table ||
+        max_blocks_per_seq <= 0 || !aligned(k, 16) || !aligned(v, 16) || !aligned(seq_lens, 4) ||
+        !aligned(kv_pages, 16) || !aligned(scales, 16) || !aligned(block_table, 4))
+        return SAW_ERR_INVALID_ARGUMENT;
+    if (win->sink + win->recent == 0 && win->blocks == 0)
+        return SAW_OK;
+    if (win->kv == nullptr || win->table == nullptr)
+        return SAW_ERR_INVALID_ARGUMENT;
+    return SAW_OK;
+}
+
+static int decode_window_impl(const saw_cache_desc *cache, const saw_window_cache *win,
+                              int32_t num_q_heads, const void *q, const uint8_t *kv_pages,
+                              const void *scales, const int32_t *block_table,
+                              int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                              int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                              size_t workspace_bytes, uint32_t *dev_status, cudaStream_t stream,
+                              bool programmatic)
+{
+    const size_t part = window_partials_bytes(cache, num_q_heads, num_seqs);
+    float *lse = reinterpret_cast<float *>(static_cast<uint8_t *>(workspace) + part);
+    saw::DecodeArgs a =
+        decode_args(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                    seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes, dev_status);
+    if (win->sink + win->recent == 0)   // no window: every token is quantized
+        return saw::launch_paged_decode(a, stream, programmatic) == cudaSuccess ? SAW_OK
+                                                                                : SAW_ERR_CUDA;
+    a.win_sink = win->sink;
+    a.win_recent = win->recent;
+    a.lse = lse;
+    // part 1: the window tokens from the bf16 window pages (writes out and lse)
+    saw::DecodeArgs w = a;
+    w.kv_pages = static_cast<const uint8_t *>(win->kv);
+    w.scales = nullptr;
+    w.block_table = win->table;
+    w.max_blocks = win->blocks;
+    w.num_pages = win->num_pages;
+    w.rotate = false;
+    w.win_part = 1;
+    if (saw::launch_paged_decode_bf16(w, stream, programmatic) != cudaSuccess)
+        return SAW_ERR_CUDA;
+    // part 2: the quantized tokens, merged into out by the lse of part 1
+    a.win_part = 2;
+    return saw::launch_paged_decode(a, stream, true) == cudaSuccess ? SAW_OK : SAW_ERR_CUDA;
+}
+
+static int check_decode_window(const saw_cache_desc *cache, const saw_window_cache *win,
+                               int32_t num_q_heads, const void *q, const uint8_t *kv_pages,
+                               const void *scales, const int32_t *block_table,
+                               int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                               int32_t num_seqs, float sm_scale, const float *out,
+                               const void *workspace, size_t workspace_bytes)
+{
+    int rc = check_cache(cache);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_window(cache, win, num_seqs);
+    if (rc != SAW_OK)
+        return rc;
+    const size_t need = saw_paged_decode_window_workspace_bytes(cache, num_q_heads, num_seqs);
+    // the INT4 checks, against the whole workspace (its first part holds the split-K slots)
+    rc = check_decode(cache, num_q_heads, q, kv_pages, scales, block_table, max_blocks_per_seq,
+                      seq_lens, num_seqs, sm_scale, out, workspace, workspace_bytes);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    if (need == 0)
+        return SAW_ERR_CUDA;
+    if (workspace_bytes < need)
+        return SAW_ERR_WORKSPACE;
+    return SAW_OK;
+}
+
+int saw_window_append(const saw_cache_desc *cache, const saw_window_cache *win, const void *k,
+                      const void *v, const int32_t *seq_lens, int32_t num_seqs, uint8_t *kv_pages,
+                      void *scales, const int32_t *block_table, int32_t max_blocks_per_seq,
+                      uint32_t *dev_status, void *stream)
+{
+    const int rc = check_window_append(cache, win, k, v, seq_lens, num_seqs, kv_pages, scales,
+                                       block_table, max_blocks_per_seq);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    return window_append_impl(cache, win, k, v, seq_lens, num_seqs, kv_pages, scales, block_table,
+                              max_blocks_per_seq, dev_status, static_cast<cudaStream_t>(stream));
+}
+
+int saw_paged_decode_attn_window(const saw_cache_desc *cache, const saw_window_cache *win,
+                                 int32_t num_q_heads, const void *q, const uint8_t *kv_pages,
+                                 const void *scales, const int32_t *block_table,
+                                 int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                                 int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                                 size_t workspace_bytes, uint32_t *dev_status, void *stream)
+{
+    const int rc = check_decode_window(cache, win, num_q_heads, q, kv_pages, scales, block_table,
+                                       max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out,
+                                       workspace, workspace_bytes);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    return decode_window_impl(cache, win, num_q_heads, q, kv_pages, scales, block_table,
+                              max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
+                              workspace_bytes, dev_status, static_cast<cudaStream_t>(stream), false);
+}
+
+int saw_decode_step_window(const saw_cache_desc *cache, const saw_window_cache *win,
+                           int32_t num_q_heads, const void *q, const void *k_new, const void *v_new,
+                           uint8_t *kv_pages, void *scales, const int32_t *block_table,
+                           int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                           float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                           uint32_t *dev_status, void *stream)
+{
+    int rc = check_window_append(cache, win, k_new, v_new, seq_lens, num_seqs, kv_pages, scales,
+                                 block_table, max_blocks_per_seq);
+    if (rc != SAW_OK)
+        return rc;
+    rc = check_decode_window(cache, win, num_q_heads, q, kv_pages, scales, block_table,
+                             max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
+                             workspace_bytes);
+    if (rc != SAW_OK || num_seqs == 0)
+        return rc;
+    const cudaStream_t st = static_cast<cudaStream_t>(stream);
+    rc = window_append_impl(cache, win, k_new, v_new, seq_lens, num_seqs, kv_pages, scales,
+                            block_table, max_blocks_per_seq, dev_status, st);
+    if (rc != SAW_OK)
+        return rc;
+    return decode_window_impl(cache, win, num_q_heads, q, kv_pages, scales, block_table,
+                              max_blocks_per_seq, seq_lens, num_seqs, sm_scale, out, workspace,
+                              workspace_bytes, dev_status, st, true);
 }
 
 }  // extern "C"

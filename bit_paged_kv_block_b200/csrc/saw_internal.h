@@ -58,7 +58,12 @@ struct DecodeArgs {
     bool rotate = true;          // false: plain INT4 cache (no query / output rotation)
     const int32_t *q_start = nullptr;   // chunked prefill: [S + 1] query-row offsets (else decode)
     int64_t total_q = 0;         // chunked prefill: query rows (q_start[S])
-    int32_t head_dim = 128;      // D: 128 or 256 (INT4 cache only)
+    int32_t head_dim = 128;      // D: 64, 128 or 256 (INT4 cache only)
+    // windowed decode: 1 = the window part (bf16 pages), 2 = the quantized part (merged into
+    // out with the window part's lse); 0 = a plain decode
+    int32_t win_part = 0;
+    int32_t win_sink = 0, win_recent = 0;
+    float *lse = nullptr;        // [S][Hq] log2 softmax denominators of the window part
 };
 
 struct AppendBf16Args {
@@ -89,6 +94,29 @@ cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool p
 // The uncompressed BF16 paged cache (baseline): scatter, decode workspace size, decode
 // (DecodeArgs::kv_pages is the bf16 cache; scales and rotate are unused).
 cudaError_t launch_append_bf16(const AppendBf16Args &a, cudaStream_t stream);
+
+struct WindowAppendArgs {
+    const void *k;               // new tokens, bf16 [S][Hkv][128]: one per sequence
+    const void *v;
+    const int32_t *seq_lens;     // [S], including the new token
+    int32_t num_seqs;
+    int32_t num_kv_heads;
+    int32_t w_sink, w_recent;
+    void *win_kv;                // bf16 window pages [num_win_pages][Hkv][2][16][128]
+    int64_t num_win_pages;
+    const int32_t *win_table;    // [S][win_blocks]
+    int32_t win_blocks;
+    uint8_t *kv_pages;           // INT4 pages of the quantized tokens
+    void *scales;
+    int64_t num_pages;
+    const int32_t *block_table;  // [S][max_blocks], indexed by quantized position
+    int32_t max_blocks;
+    uint32_t *status;            // nullable
+};
+
+// Queue the window append: per sequence and kv head, the token leaving the recent window is
+// rotated, quantized and scattered into the INT4 pages, and the new token takes its slot.
+cudaError_t launch_window_append(const WindowAppendArgs &a, cudaStream_t stream);
 size_t decode_bf16_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs,
                                    int64_t total_q = -1);
 cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, bool programmatic);

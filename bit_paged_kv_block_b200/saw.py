@@ -43,6 +43,12 @@ class saw_cache_desc(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int64)]
 
 
+class saw_window_cache(ctypes.Structure):
+    _fields_ = [("sink", ctypes.c_int32), ("recent", ctypes.c_int32), ("kv", ctypes.c_void_p),
+                ("num_pages", ctypes.c_int64), ("table", ctypes.c_void_p),
+                ("blocks", ctypes.c_int32)]
+
+
 def _open_library() -> ctypes.CDLL:
     path = _build.LIB
     if not _build.up_to_date():
@@ -95,6 +101,17 @@ def _open_library() -> ctypes.CDLL:
     lib.saw_decode_step_bf16.argtypes = [D, i32, P, P, P, P, i64, P, P, i32, P, i32, f32, P, P,
                                          sz, P, P]
     lib.saw_decode_step_bf16.restype = ctypes.c_int
+    Wc = ctypes.POINTER(saw_window_cache)
+    lib.saw_paged_decode_window_workspace_bytes.argtypes = [D, i32, i32]
+    lib.saw_paged_decode_window_workspace_bytes.restype = sz
+    lib.saw_window_append.argtypes = [D, Wc, P, P, P, i32, P, P, P, i32, P, P]
+    lib.saw_window_append.restype = ctypes.c_int
+    lib.saw_paged_decode_attn_window.argtypes = [D, Wc, i32, P, P, P, P, i32, P, i32, f32, P, P,
+                                                 sz, P, P]
+    lib.saw_paged_decode_attn_window.restype = ctypes.c_int
+    lib.saw_decode_step_window.argtypes = [D, Wc, i32, P, P, P, P, P, P, i32, P, i32, f32, P, P,
+                                           sz, P, P]
+    lib.saw_decode_step_window.restype = ctypes.c_int
     return lib
 
 
@@ -506,3 +523,118 @@ def saw_paged_prefill_attn(q, q_start, kv_pages, scales, block_table, seq_lens, 
             _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S, float(sm_scale), _ptr(out),
             _ptr(workspace), workspace.numel(), _ptr(dev_status), _stream(stream))
     _check(rc, "saw_paged_prefill_attn" if rotate else "saw_paged_prefill_attn_plain")
+
+
+# ---- full-precision sink / recent window beside the INT4 cache --------------------------------
+
+def allocate_window(num_seqs: int, num_kv_heads: int, sink: int, recent: int, device="cuda"):
+    """Window pages for num_seqs sequences: kv bf16 [num_seqs * blocks][Hkv][2][16][128] and the
+    table int32 [num_seqs][blocks] giving sequence s the pages s * blocks .. (blocks = the
+    16-token pages sink + recent tokens need, at least 1)."""
+    blocks = max(1, (sink + recent + PAGE_SIZE - 1) // PAGE_SIZE)
+    kv = torch.zeros((num_seqs * blocks, num_kv_heads, 2, PAGE_SIZE, HEAD_DIM), dtype=torch.bfloat16,
+                     device=device)
+    table = torch.arange(num_seqs * blocks, dtype=torch.int32, device=device).view(num_seqs, blocks)
+    return kv, table
+
+
+def window_desc(sink: int, recent: int, win_kv: torch.Tensor, win_table: torch.Tensor):
+    """The saw_window_cache of window pages win_kv (bf16 [P][Hkv][2][16][128]) and their table
+    (int32 [num_seqs][blocks])."""
+    _need(win_kv, "win_kv", torch.bfloat16, 5)
+    _need(win_table, "win_table", torch.int32, 2)
+    if tuple(win_kv.shape[2:]) != (2, PAGE_SIZE, HEAD_DIM):
+        raise ValueError(f"win_kv must be [P][Hkv][2][16][128], got {tuple(win_kv.shape)}")
+    return saw_window_cache(int(sink), int(recent), _ptr(win_kv), int(win_kv.shape[0]),
+                            _ptr(win_table), int(win_table.shape[1]))
+
+
+def saw_paged_decode_window_workspace_bytes(num_kv_heads: int, num_q_heads: int,
+                                            num_seqs: int) -> int:
+    desc = saw_cache_desc(int(num_kv_heads), HEAD_DIM, PAGE_SIZE, 1)
+    return int(lib.saw_paged_decode_window_workspace_bytes(ctypes.byref(desc), int(num_q_heads),
+                                                           int(num_seqs)))
+
+
+def allocate_window_workspace(num_kv_heads: int, num_q_heads: int, num_seqs: int,
+                              device="cuda") -> torch.Tensor:
+    n = saw_paged_decode_window_workspace_bytes(num_kv_heads, num_q_heads, num_seqs)
+    if n == 0:
+        raise SawError(SAW_ERR_CUDA, "saw_paged_decode_window_workspace_bytes")
+    return torch.empty(n, dtype=torch.uint8, device=device)
+
+
+def _window_checks(win, kv_pages, scales, block_table, seq_lens, dev_status):
+    sink, recent, win_kv, win_table = win
+    wd = window_desc(sink, recent, win_kv, win_table)
+    _need(kv_pages, "kv_pages", torch.uint8, 5)
+    _need(scales, "scales", torch.float16, 5)
+    _need(block_table, "block_table", torch.int32, 2)
+    _need(seq_lens, "seq_lens", torch.int32, 1)
+    if dev_status is not None:
+        _need(dev_status, "dev_status", torch.int32, 1)
+    desc = cache_desc(kv_pages)
+    S = seq_lens.shape[0]
+    if block_table.shape[0] != S or win_table.shape[0] != S:
+        raise ValueError("block_table and the window table need one row per sequence")
+    return wd, desc, S
+
+
+def saw_window_append(k, v, seq_lens, win, kv_pages, scales, block_table, dev_status=None,
+                      stream=None) -> None:
+    """One step's write into a windowed cache: k, v (bf16 [S][Hkv][128]) are the new tokens at
+    positions seq_lens - 1; win = (sink, recent, win_kv, win_table).  The token each one displaces
+    from the recent window is rotated, quantized and scattered into the INT4 pages."""
+    wd, desc, S = _window_checks(win, kv_pages, scales, block_table, seq_lens, dev_status)
+    _need(k, "k", torch.bfloat16, 3)
+    _need(v, "v", torch.bfloat16, 3)
+    if tuple(k.shape) != (S, desc.num_kv_heads, HEAD_DIM) or v.shape != k.shape:
+        raise ValueError("k and v must be [S][Hkv][128] matching the cache")
+    rc = lib.saw_window_append(ctypes.byref(desc), ctypes.byref(wd), _ptr(k), _ptr(v),
+                               _ptr(seq_lens), S, _ptr(kv_pages), _ptr(scales), _ptr(block_table),
+                               block_table.shape[1], _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_window_append")
+
+
+def saw_paged_decode_attn_window(q, win, kv_pages, scales, block_table, seq_lens, out, workspace,
+                                 sm_scale=None, dev_status=None, stream=None) -> None:
+    """Decode attention of q (bf16 [S][Hq][128]) over each sequence's bf16 window and its
+    quantized tokens, one softmax over both, into out (fp32 [S][Hq][128])."""
+    wd, desc, S = _window_checks(win, kv_pages, scales, block_table, seq_lens, dev_status)
+    _need(q, "q", torch.bfloat16, 3)
+    _need(out, "out", torch.float32, 3)
+    _need(workspace, "workspace", torch.uint8, 1)
+    hq = q.shape[1]
+    if tuple(q.shape) != (S, hq, HEAD_DIM) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [S][Hq][128]")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_paged_decode_attn_window(ctypes.byref(desc), ctypes.byref(wd), hq, _ptr(q),
+                                          _ptr(kv_pages), _ptr(scales), _ptr(block_table),
+                                          block_table.shape[1], _ptr(seq_lens), S, float(sm_scale),
+                                          _ptr(out), _ptr(workspace), workspace.numel(),
+                                          _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_paged_decode_attn_window")
+
+
+def saw_decode_step_window(q, k_new, v_new, win, kv_pages, scales, block_table, seq_lens, out,
+                           workspace, sm_scale=None, dev_status=None, stream=None) -> None:
+    """saw_window_append then saw_paged_decode_attn_window on one stream."""
+    wd, desc, S = _window_checks(win, kv_pages, scales, block_table, seq_lens, dev_status)
+    for t, name in ((q, "q"), (k_new, "k_new"), (v_new, "v_new")):
+        _need(t, name, torch.bfloat16, 3)
+    _need(out, "out", torch.float32, 3)
+    _need(workspace, "workspace", torch.uint8, 1)
+    hq = q.shape[1]
+    if tuple(k_new.shape) != (S, desc.num_kv_heads, HEAD_DIM) or v_new.shape != k_new.shape:
+        raise ValueError("k_new and v_new must be [S][Hkv][128] matching the cache")
+    if tuple(q.shape) != (S, hq, HEAD_DIM) or tuple(out.shape) != tuple(q.shape):
+        raise ValueError("q and out must be [S][Hq][128]")
+    if sm_scale is None:
+        sm_scale = 1.0 / math.sqrt(HEAD_DIM)
+    rc = lib.saw_decode_step_window(ctypes.byref(desc), ctypes.byref(wd), hq, _ptr(q),
+                                    _ptr(k_new), _ptr(v_new), _ptr(kv_pages), _ptr(scales),
+                                    _ptr(block_table), block_table.shape[1], _ptr(seq_lens), S,
+                                    float(sm_scale), _ptr(out), _ptr(workspace), workspace.numel(),
+                                    _ptr(dev_status), _stream(stream))
+    _check(rc, "saw_decode_step_window")

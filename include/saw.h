@@ -275,6 +275,71 @@ const char *saw_status_string(int status);
 /* Library ABI version: 100 * major + minor. */
 int saw_version(void);
 
+/* ---- full-precision sink / recent window beside the INT4 cache ----------------------------
+ *
+ * "InnerQ: Hardware-Aware Tuning-Free Quantization of KV Cache for Large Language Models",
+ * Abstract and Figure 2: a small high-precision window of attention-sink tokens and recent
+ * tokens is kept beside the quantized cache; the attention over the quantized part and over the
+ * window are computed separately and merged.  Layout (the pages give none; head_dim 128):
+ *   - of a sequence of L tokens, positions p < sink are sinks and positions
+ *     p >= max(sink, L - recent) are recent: min(L, W) window tokens, W = sink + recent, kept in
+ *     bf16.  Window slot of p: p for a sink, sink + (p - sink) mod recent for a recent token;
+ *     slot i of sequence s lives in window page table[s * blocks + i / 16] at offset i mod 16 of
+ *     kv, bf16 [num_pages][Hkv][2 (K, V)][16][128] (the layout of the bf16 baseline cache);
+ *   - the other max(0, L - W) tokens are rotated INT4 in the ordinary paged cache (kv_pages,
+ *     scales), as their own sequence: position p is quantized index j = p - sink, at page
+ *     block_table[s][j / 16], offset j mod 16.
+ * The decode attends over the window (bf16 arithmetic of saw_paged_decode_attn_bf16) and over the
+ * quantized tokens (that of saw_paged_decode_attn), and merges the two results by their softmax
+ * denominators, so the output is one softmax over all L tokens. */
+typedef struct saw_window_cache {
+    int32_t sink;            /* sink tokens kept in bf16, >= 0 */
+    int32_t recent;          /* most recent tokens kept in bf16, >= 0 */
+    void *kv;                /* device: bf16 window pages [num_pages][Hkv][2][16][128] */
+    int64_t num_pages;       /* pages in kv; num_pages * Hkv * 64 < 2^31 */
+    const int32_t *table;    /* device: int32 [num_seqs][blocks] window pages per sequence */
+    int32_t blocks;          /* row stride of table; sink + recent <= 16 * blocks */
+} saw_window_cache;
+
+/* Workspace bytes saw_paged_decode_attn_window / saw_decode_step_window need (0 if the shape is
+ * unsupported: head_dim != 128, Hq / Hkv > 16). */
+size_t saw_paged_decode_window_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
+                                               int32_t num_seqs);
+
+/* One serving step's write: sequence s's new token (k, v: bf16 [num_seqs][Hkv][128], device) sits
+ * at position p = seq_lens[s] - 1.  A sink takes window slot p.  Otherwise it takes its slot in the
+ * recent ring, and the token it displaces there (position p - recent, when that is not a sink) is
+ * rotated, quantized and scattered into kv_pages / scales at quantized index p - recent - sink,
+ * with the arithmetic of saw_rotate_quantize_paged (bit-identical codes and scales).  With
+ * recent = 0 the new token itself is quantized at index p - sink.  A sequence with
+ * seq_lens[s] <= 0 is skipped (negative: SAW_DEV_BAD_SEQ_LEN); a window or INT4 page id out of
+ * range, or a quantized index past max_blocks_per_seq, leaves the pair untouched and sets
+ * SAW_DEV_BAD_PAGE / SAW_DEV_BAD_SEQ_LEN. */
+int saw_window_append(const saw_cache_desc *cache, const saw_window_cache *win, const void *k,
+                      const void *v, const int32_t *seq_lens, int32_t num_seqs, uint8_t *kv_pages,
+                      void *scales, const int32_t *block_table, int32_t max_blocks_per_seq,
+                      uint32_t *dev_status, void *stream);
+
+/* Decode attention of q (bf16 [num_seqs][Hq][128]) over the window and the quantized tokens of
+ * each sequence (seq_lens[s] tokens in all, including the newest) into out (fp32
+ * [num_seqs][Hq][128]).  workspace: at least saw_paged_decode_window_workspace_bytes(), 256-byte
+ * aligned.  Launches the window part, then the quantized part as a programmatic dependent. */
+int saw_paged_decode_attn_window(const saw_cache_desc *cache, const saw_window_cache *win,
+                                 int32_t num_q_heads, const void *q, const uint8_t *kv_pages,
+                                 const void *scales, const int32_t *block_table,
+                                 int32_t max_blocks_per_seq, const int32_t *seq_lens,
+                                 int32_t num_seqs, float sm_scale, float *out, void *workspace,
+                                 size_t workspace_bytes, uint32_t *dev_status, void *stream);
+
+/* saw_window_append then saw_paged_decode_attn_window on one stream (the decode launched as a
+ * programmatic dependent of the append). */
+int saw_decode_step_window(const saw_cache_desc *cache, const saw_window_cache *win,
+                           int32_t num_q_heads, const void *q, const void *k_new, const void *v_new,
+                           uint8_t *kv_pages, void *scales, const int32_t *block_table,
+                           int32_t max_blocks_per_seq, const int32_t *seq_lens, int32_t num_seqs,
+                           float sm_scale, float *out, void *workspace, size_t workspace_bytes,
+                           uint32_t *dev_status, void *stream);
+
 #ifdef __cplusplus
 } /* extern "C" */
 #endif
