@@ -177,17 +177,23 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def sources_digest(sources) -> str:
+    """sha256 over the named csrc files, in order (the kernel's whole source)."""
+    h = hashlib.sha256()
+    for name in sources:
+        with open(os.path.join(ROOT, "bit_paged_kv_block_b200", "csrc", name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()
+
+
 def kernel_traffic(kernel: str, units: float):
     """dram bytes per launch from the committed ncu summary, if it was taken on the current
-    kernel source (scaled by `units` / the captured units); else None."""
+    kernel sources (scaled by `units` / the captured units); else None."""
     path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
     try:
         with open(path) as f:
             rec = json.load(f)[kernel]
-        src = os.path.join(ROOT, "bit_paged_kv_block_b200", "csrc", rec["source"])
-        with open(src, "rb") as f:
-            digest = hashlib.sha256(f.read()).hexdigest()
-        if digest != rec["source_sha256"]:
+        if sources_digest(rec["sources"]) != rec["sources_sha256"]:
             return None
         return rec["dram_bytes_per_launch"] * units / rec["units"]
     except Exception:
@@ -528,6 +534,53 @@ def run_saw(args):
             "decode_GBps": d4_gbs, "decode_frac_of_measured_peak": d4_gbs / peak_gbs}
         del kv4, sc4, q4, o4, ws4
 
+    # ---- full-precision sink / recent window ("InnerQ", Figure 2): W = 16 + 112 bf16 tokens ----
+    sink, recent = 16, 112
+    W = sink + recent
+    wkv, wtab = saw.allocate_window(wl.num_seqs, wl.num_kv_heads, sink, recent, dev)
+    wkv5, wsc5 = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
+    kh = synth.kv_values(wl, "K", tokens="history", device=dev)
+    vh = synth.kv_values(wl, "V", tokens="history", device=dev)
+    seqh, posh = synth.token_index(wl, "history")
+    Lh = wl.seq_lens[seqh] - 1                      # history length of each token's sequence
+    in_win = (posh < sink) | (posh >= np.maximum(sink, Lh - recent))
+    j = posh - sink
+    qslot = np.where(in_win, -1, wl.block_table[seqh, np.maximum(j, 0) // 16] * 16 + j % 16)
+    wslot = np.where(posh < sink, posh, sink + (posh - sink) % max(recent, 1))
+    wtab_np = wtab.cpu().numpy()
+    wslot = np.where(in_win, wtab_np[seqh, wslot // 16] * 16 + wslot % 16, -1)
+    saw.saw_rotate_quantize_paged(kh, vh, torch.from_numpy(qslot.astype(np.int64)).to(dev), wkv5, wsc5)
+    saw.saw_append_bf16_paged(kh, vh, torch.from_numpy(wslot.astype(np.int64)).to(dev), wkv)
+    del kh, vh
+    win = (sink, recent, wkv, wtab)
+    wsw = saw.allocate_window_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
+    win_step = lambda: saw.saw_decode_step_window(q, k_new, v_new, win, wkv5, wsc5, table, lens,
+                                                  out, wsw, dev_status=status, stream=stream)
+    win_decode = lambda: saw.saw_paged_decode_attn_window(q, win, wkv5, wsc5, table, lens, out, wsw,
+                                                          dev_status=status, stream=stream)
+    for _ in range(3):
+        win_step()
+    torch.cuda.synchronize()
+    e0.record(stream)
+    for _ in range(n_pl):
+        win_step()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    win_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
+    t_wdec = mean_event_ms(win_decode, n_kt)
+    win_tokens = int(np.minimum(wl.seq_lens, W).sum())
+    win_bytes = (decode_bytes(wl) - wl.num_kv_heads * win_tokens * 136
+                 + wl.num_kv_heads * win_tokens * 512)
+    window = {"what": f"the same step with a bf16 window of {sink} sink + {recent} recent tokens "
+                      "per sequence beside the INT4 cache (append with eviction, then the window "
+                      "part and the quantized part merged)",
+              "step_ms": win_ms, "tokens_per_s": job_throughput(wl.num_seqs, world, win_ms),
+              "step_vs_int4": win_ms / ms_per_step,
+              "decode_launch_ms": t_wdec,
+              "decode_algorithmic_bytes": win_bytes,
+              "decode_GBps": win_bytes / (t_wdec * 1e-3) / 1e9}
+    del wkv, wtab, wkv5, wsc5, wsw
+
     # ---- end to end through the public API with host buffers ------------------------------
     pin = lambda t: t.cpu().pin_memory()
     h_q, h_k, h_v, h_slots, h_table, h_lens = (pin(q), pin(k_new), pin(v_new), pin(slots),
@@ -581,6 +634,7 @@ def run_saw(args):
         "bf16_baseline": bf16_baseline,
         "prefill_attn": prefill_attn,
         **head_dims,
+        "window": window,
         "append_launch_ms": t_append,
         "e2e": e2e,
         "gpu_launches": 3 * args.steps,

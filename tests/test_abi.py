@@ -122,3 +122,44 @@ def test_strided_append_argument_checks():
     assert call(2, 260, 256) == saw.SAW_ERR_INVALID_ARGUMENT       # not a multiple of 8
     assert call(3, 384, 384) == saw.SAW_ERR_UNSUPPORTED
     assert call(12, 12 * 128, 12 * 128) == saw.SAW_ERR_UNSUPPORTED
+
+
+def _win(sink=16, recent=112, kv=16, pages=8, table=16, blocks=8):
+    return saw.saw_window_cache(sink, recent, kv, pages, table, blocks)
+
+
+def _wapp(desc, win, S=2, k=16, v=16, lens=16, pages=16, scales=16, bt=16, max_blocks=4):
+    P = ctypes.c_void_p
+    return saw.lib.saw_window_append(
+        ctypes.byref(desc), None if win is None else ctypes.byref(win), P(k), P(v), P(lens), S,
+        P(pages), P(scales), P(bt), max_blocks, None, None)
+
+
+def _wdec(desc, win, hq=32, S=2, q=16, out=16, ws=256, ws_bytes=1 << 30):
+    P = ctypes.c_void_p
+    return saw.lib.saw_paged_decode_attn_window(
+        ctypes.byref(desc), None if win is None else ctypes.byref(win), hq, P(q), P(16), P(16),
+        P(16), 4, P(16), S, 0.088, P(out), P(ws), ws_bytes, None, None)
+
+
+def test_window_argument_checks():
+    """The windowed entry points check the window description before any CUDA call."""
+    d = _desc()
+    assert _wapp(d, None) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wapp(d, _win(sink=-1)) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wapp(d, _win(recent=200, blocks=8)) == saw.SAW_ERR_INVALID_ARGUMENT   # W > 16 blocks
+    assert _wapp(d, _win(kv=0)) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wapp(d, _win(table=2)) == saw.SAW_ERR_INVALID_ARGUMENT                # misaligned
+    assert _wapp(d, _win(pages=1 << 30)) == saw.SAW_ERR_UNSUPPORTED               # 2^31 rows
+    assert _wapp(_desc(d=256), _win()) == saw.SAW_ERR_UNSUPPORTED                 # bf16 window
+    assert _wapp(d, _win(), k=8) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wapp(d, _win(), max_blocks=0) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wapp(d, _win(), S=0) == saw.SAW_OK                                    # nothing to do
+    assert _wdec(d, None) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _wdec(d, _win(), hq=12) == saw.SAW_ERR_INVALID_ARGUMENT                # Hq % Hkv
+    assert _wdec(d, _win(), hq=136) == saw.SAW_ERR_UNSUPPORTED                    # G = 17
+    assert _wdec(_desc(d=64), _win()) == saw.SAW_ERR_UNSUPPORTED
+    assert _wdec(d, _win(), S=0) == saw.SAW_OK
+    f = saw.lib.saw_paged_decode_window_workspace_bytes
+    assert f(ctypes.byref(_desc(d=256)), 32, 4) == 0
+    assert f(ctypes.byref(d), 12, 4) == 0
