@@ -20,8 +20,8 @@ COMMON = ["-O3", "-std=c++17", "-lineinfo", "-Xcompiler", "-fPIC", "-I", INCLUDE
           "-prec-div=true", "-ftz=false"]
 # per-file extra flags: the quantizer must not contract its IEEE operations into FMAs
 EXTRA = {"rotate_quantize.cu": ["-fmad=false"]}
-SOURCES = ["rotate_quantize.cu", "paged_decode.cu", "paged_decode_bf16.cu", "saw_api.cu",
-           "decode_static.cu"]
+SOURCES = ["rotate_quantize.cu", "paged_decode.cu", "paged_decode_bf16.cu", "prefill_tc.cu",
+           "saw_api.cu", "decode_static.cu"]
 HEADERS = ["saw_device.cuh", "saw_internal.h", "decode_common.cuh"]
 
 

@@ -565,6 +565,12 @@ const CUtensorMap *code_tensor_map(const uint8_t *kv_pages, int64_t rows)
 template <int kD>
 cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
 {
+    // Chunked prefill whose chunks average at least half a 128-row tile per sequence runs on the
+    // tensor cores (prefill_tc.cu); shorter chunks keep this kernel's split-K work split, which
+    // spreads a few long rows over every SM.
+    if (kD == 128 && a.q_start != nullptr && a.win_part == 0 &&
+        a.total_q * (a.num_q_heads / a.num_kv_heads) >= 64 * static_cast<int64_t>(a.num_seqs))
+        return launch_prefill_tc(a, stream, programmatic);
     const CUtensorMap *map = code_tensor_map<kD>(a.kv_pages, a.num_pages * a.num_kv_heads * 32);
     if (map == nullptr)
         return cudaErrorInvalidValue;

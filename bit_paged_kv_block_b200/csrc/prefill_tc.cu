@@ -1,0 +1,654 @@
+// prefill_tc.cu -- chunked-prefill attention over the INT4 paged cache on the 5th-generation
+// tensor cores (tcgen05.mma, accumulators in tensor memory).
+//
+// The read step for a chunk of new tokens whose K/V are already in the cache ("SAW-INT4:
+// System-Aware 4-Bit KV-Cache Quantization for Real-World LLM Serving", Research Findings: the
+// quantized cache must serve fused attention over paged memory; a prefill chunk is the
+// multi-query case).  Sequence s has C query tokens, the last C of its L cached tokens; query i
+// attends causally to cache tokens 0 .. L - C + i.  The arithmetic is the decode's: the query is
+// rotated by the same Hadamard transform and scaled by sm_scale log2(e) and 1/sqrt(128); logits
+// are s = scale_K acc + zero_K sum(q) over the raw codes; P' = p scale_V meets the raw V codes
+// and sum p zero_V is added in fp32; the output is rotated back.
+//
+// A CTA (4 warps) owns one tile of up to 128 query rows: T = 128 / G consecutive query tokens x
+// the G query heads of one kv head, row r = token (r / G), head (r % G).  It walks the tile's
+// causal range of the cache in blocks of 64 tokens (4 pages):
+//   1. the 4 pages' codes and scales are staged by cp.async (LSU path, one block ahead);
+//   2. all 128 threads unpack them once into fp16 tiles: K [64 tokens x 128 d] and
+//      V [64 tokens x 128 d], token rows of 128 B per half of d under the 128-byte swizzle;
+//   3. one thread issues S = Q K^T (M 128, N 64, K 128: 8 x tcgen05.mma.kind::f16) into tensor
+//      memory;
+//   4. each thread reads its row of S (tcgen05.ld), applies scales, zero points and the causal
+//      limit, and runs the online softmax for its row alone; P' (fp16) goes to a shared tile;
+//   5. one thread issues O += P' V (M 128, N 128, K 64: 4 MMAs, V read as the MN-major operand).
+// When a block's maximum exceeds a row's running maximum, the row's O accumulator is rescaled in
+// tensor memory (the warp's 32 rows together; rows without a change multiply by 1).  Letting the
+// maximum lag (weights up to 2^4) saved no measurable time and doubled the largest error.
+// The epilogue reads each thread's O row, adds the zero-point term, divides by the row sum and
+// rotates back.
+//
+// Codes enter the tensor cores as exact fp16 integers n = (1024 + n) - 1024 (a magic OR and one
+// half2 subtraction per pair).  These tensor cores flush fp16 subnormals, so the operands are kept
+// normal: the query enters scaled by 2^8 (logit = (scale_K acc + zero_K sq) / 2^8, sq the sum of the
+// fp16 query entries), and the weights as P' = 2^4 p scale_V with p <= 1 (O = O_acc / 2^4 +
+// sum p zero_V), so only weights below about 2^-14 of a row's maximum fall under fp16's normal
+// range.  A 32-bit word of 8 codes (d .. d + 7) gives the fp16 pairs (d, d+4), (d+1, d+5),
+// (d+2, d+6), (d+3, d+7); Q is written in that d order, and the epilogue reads O's columns back
+// through it.
+#include <cuda_fp16.h>
+#include <cudaTypedefs.h>
+
+#include <algorithm>
+
+#include "saw_device.cuh"
+#include "saw_internal.h"
+
+namespace saw {
+namespace {
+
+constexpr int kTcThreads = 128;
+constexpr int kTcRows = 128;                 // M of the MMAs: query rows per tile
+constexpr int kTcBlockTokens = 64;           // N of QK, K of PV: cache tokens per block
+constexpr int kTcBlockPages = kTcBlockTokens / kPageSize;
+constexpr int kTcPageBytes = 2 * kPageSize * kRowBytes + 2 * kPageSize * 4;   // codes + scales
+constexpr float kTcHadamardC = 0.0883883461356163f;
+constexpr float kTcRescale = 0.0f;           // move the running max whenever a block exceeds it
+constexpr float kTcQScale = 256.0f;          // query entries enter the MMA scaled by 2^8
+constexpr float kTcPScale = 16.0f;           // weights enter the MMA scaled by 2^4
+constexpr uint64_t kTcWaitLimitNs = 1000000000ull;
+
+// shared memory (from a 1024-byte aligned base)
+constexpr int kSmQ = 0;                                  // Q tile: 2 x [128 rows][128 B]
+constexpr int kSmK = kSmQ + 2 * kTcRows * 128;           // K tile: 2 x [64 tokens][128 B]
+constexpr int kSmV = kSmK + 2 * kTcBlockTokens * 128;    // V tile: 2 x [64 tokens][128 B]
+constexpr int kSmP = kSmV + 2 * kTcBlockTokens * 128;    // P tile: [128 rows][128 B]
+constexpr int kSmCodes = kSmP + kTcRows * 128;           // 2 stages x 4 pages (codes, scales)
+constexpr int kSmScales = kSmCodes + 2 * kTcBlockPages * kTcPageBytes;   // per token pair: float4 (K), float4 (V)
+constexpr int kSmBars = kSmScales + 4 * kTcBlockTokens * 4;              // 2 mbarriers + tmem addr
+constexpr int kSmTile = kSmBars + 32;                                    // tile descriptor
+constexpr int kSmBytes = kSmTile + 64;
+constexpr size_t kTcSmemBytes = 1024 + kSmBytes;
+constexpr uint32_t kTmemCols = 256;                      // O: columns 0..127, S: 128..191
+
+// byte offset of 16-bit element (row, k) in a tile of rows of 64 elements (128 B) per atom,
+// atom stride atom_bytes, 128-byte swizzle (16-byte chunk index XOR row mod 8)
+__device__ __forceinline__ uint32_t sw128_chunk(int row, int chunk16, uint32_t atom_bytes)
+{
+    return static_cast<uint32_t>((chunk16 >> 3) * atom_bytes + row * 128 + (((chunk16 & 7) ^ (row & 7)) << 4));
+}
+
+// tcgen05 shared-memory matrix descriptor: 128-byte swizzle, version 1 (sm_100), base offset 0
+__device__ __forceinline__ uint64_t umma_desc(uint32_t addr, uint32_t lbo, uint32_t sbo)
+{
+    uint64_t d = static_cast<uint64_t>((addr >> 4) & 0x3FFF);
+    d |= static_cast<uint64_t>((lbo >> 4) & 0x3FFF) << 16;
+    d |= static_cast<uint64_t>((sbo >> 4) & 0x3FFF) << 32;
+    d |= static_cast<uint64_t>(1) << 46;
+    d |= static_cast<uint64_t>(2) << 61;
+    return d;
+}
+
+// instruction descriptor of kind::f16: fp16 A and B, fp32 accumulator, M x N, A / B K- or
+// MN-major
+__host__ __device__ constexpr uint32_t umma_idesc(int m, int n, int a_mn, int b_mn)
+{
+    return (1u << 4) | (static_cast<uint32_t>(a_mn) << 15) | (static_cast<uint32_t>(b_mn) << 16) |
+           (static_cast<uint32_t>(n >> 3) << 17) | (static_cast<uint32_t>(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void umma_f16(uint32_t tmem_d, uint64_t a, uint64_t b, uint32_t idesc,
+                                         uint32_t accumulate)
+{
+    asm volatile("{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+                 "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}"
+                 ::"r"(tmem_d), "l"(a), "l"(b), "r"(idesc), "r"(accumulate)
+                 : "memory");
+}
+
+__device__ __forceinline__ void umma_commit(uint32_t bar)
+{
+    asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];"
+                 ::"r"(bar) : "memory");
+}
+
+__device__ __forceinline__ void tc_fence_before() { asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void tc_fence_after() { asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory"); }
+__device__ __forceinline__ void async_proxy_fence() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+// 32 consecutive fp32 columns of this thread's tensor-memory lane
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
+{
+    uint32_t r[32];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                 "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+                   "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]),
+                   "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]),
+                   "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]),
+                   "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 32; i++)
+        v[i] = __uint_as_float(r[i]);
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float v[32])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+                 "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
+                   "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
+                   "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
+                   "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
+                   "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
+                   "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
+                   "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
+                   "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
+                   "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
+                   "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
+                   "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
+{
+    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
+
+// d order of the 8 entries of a 16-byte chunk: position j holds d = 8 a + kPerm[j]
+__host__ __device__ constexpr int chunk_d(int j) { return (j >> 1) + ((j & 1) << 2); }
+
+struct TcParams {
+    const uint16_t *q;           // bf16 [total_q][Hq][128]
+    const int32_t *q_start;      // [S + 1]
+    const uint8_t *codes;        // INT4 pages [num_pages][Hkv][2][16][64]
+    const uint8_t *scales;       // fp16 pairs [num_pages][Hkv][2][16][2]
+    const int32_t *block_table;  // [S][max_blocks]
+    const int32_t *seq_lens;     // [S]
+    float *out;                  // fp32 [total_q][Hq][128]
+    uint32_t *status;
+    int64_t num_pages;
+    int32_t max_blocks, num_seqs, hq, hkv, group, tile_tokens;
+    float q_mult;
+};
+
+// Tile of CTA `cta`: sequence s, kv head h, first query token t0 of the chunk (tiles of T tokens
+// in sequence order, the kv heads of one tile on consecutive CTAs).  Returns false past the last
+// tile.  All threads of the CTA take part (block-wide scan over the sequences).
+__device__ bool find_tile(const TcParams &p, int cta, int &s_out, int &h_out, int &t0_out,
+                          int *sm_tile)
+{
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    __shared__ int warp_sums[kTcThreads / 32];
+    __shared__ int carry;
+    const int g_tile = cta / p.hkv;
+    if (tid == 0) {
+        carry = 0;
+        sm_tile[0] = -1;
+    }
+    __syncthreads();
+    for (int base = 0; base < p.num_seqs; base += kTcThreads) {
+        const int s = base + tid;
+        int n = 0;
+        if (s < p.num_seqs) {
+            const int c = p.q_start[s + 1] - p.q_start[s];
+            n = c > 0 ? (c + p.tile_tokens - 1) / p.tile_tokens : 0;
+        }
+        int x = n;   // inclusive scan over the chunk of sequences
+#pragma unroll
+        for (int d = 1; d < 32; d <<= 1) {
+            const int y = __shfl_up_sync(0xFFFFFFFFu, x, d);
+            if (lane >= d)
+                x += y;
+        }
+        if (lane == 31)
+            warp_sums[warp] = x;
+        __syncthreads();
+        int before = carry;
+        for (int w = 0; w < warp; w++)
+            before += warp_sums[w];
+        const int lo = before + x - n, hi = before + x;   // tiles [lo, hi) belong to s
+        if (n > 0 && g_tile >= lo && g_tile < hi) {
+            sm_tile[0] = s;
+            sm_tile[1] = g_tile - lo;
+        }
+        __syncthreads();
+        if (tid == kTcThreads - 1)
+            carry = before + x;
+        __syncthreads();
+        if (sm_tile[0] >= 0)
+            break;
+    }
+    if (sm_tile[0] < 0)
+        return false;
+    s_out = sm_tile[0];
+    h_out = cta - g_tile * p.hkv;
+    t0_out = sm_tile[1] * p.tile_tokens;
+    return true;
+}
+
+template <bool kRotate>
+__global__ void __launch_bounds__(kTcThreads, 1)
+    prefill_tc_kernel(const TcParams p)
+{
+    extern __shared__ uint8_t smem_raw[];
+    uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+    const int tid = threadIdx.x, warp = tid >> 5;
+    const uint32_t sbase = smem_u32(smem);
+    int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 16);
+    const uint32_t bar_s = sbase + kSmBars, bar_o = sbase + kSmBars + 8;
+    // kpar[j / 2] = (scale, zero, scale, zero) of K tokens j, j + 1 (logit factors); vpar likewise
+    // for V (P' factor, zero point)
+    float *kpar = reinterpret_cast<float *>(smem + kSmScales);
+    float *vpar = kpar + 2 * kTcBlockTokens;
+
+    pdl_launch_dependents();
+    int s, h, t0;
+    if (!find_tile(p, blockIdx.x, s, h, t0, sm_tile))
+        return;
+    const int G = p.group;
+    const int C = p.q_start[s + 1] - p.q_start[s];
+    const int L = p.seq_lens[s];
+    if (C > L || L > p.max_blocks * kPageSize) {   // a chunk longer than its sequence: skipped
+        if (tid == 0 && t0 == 0 && h == 0)
+            set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
+        return;
+    }
+    const int ntok = min(p.tile_tokens, C - t0);          // query tokens of this tile
+    const int nrows = ntok * G;
+    const int row = tid;                                   // this thread's row of the tile
+    const bool live = row < nrows;
+    const int tq = live ? row / G : 0, hg = live ? row - tq * G : 0;
+    const int limit = L - C + t0 + tq;                     // last visible cache token of the row
+    const int n_kv = L - C + t0 + ntok;                    // cache tokens any row sees
+    const int n_blocks = (n_kv + kTcBlockTokens - 1) / kTcBlockTokens;
+    const int n_pages = (n_kv + kPageSize - 1) / kPageSize;
+
+    // ---- tensor memory and barriers -----------------------------------------------------------
+    if (tid == 0) {
+        mbar_init(bar_s, 1);
+        mbar_init(bar_o, 1);
+    }
+    mbar_init_fence();
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;"
+                     ::"r"(smem_u32(tmem_slot)), "r"(kTmemCols) : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+
+    pdl_wait();   // the cache may be written by the kernel this one depends on
+
+    // ---- staging of a block's 4 pages (codes, then scales) by cp.async, one block ahead --------
+    // page ids of blocks kb + 1 (pid_a) and kb + 2 (pid_b), loaded a block before their use
+    const int64_t bt_row = static_cast<int64_t>(s) * p.max_blocks;
+    auto page_id = [&](int pg) -> int32_t {
+        if (pg >= n_pages)
+            return -1;   // past the tile's range: not staged
+        int32_t id = p.block_table[bt_row + pg];
+        if (id < 0 || id >= p.num_pages) {
+            set_status(p.status, SAW_DEV_BAD_PAGE);
+            id = 0;
+        }
+        return id;
+    };
+    auto stage_block = [&](int kb, const int32_t pid[kTcBlockPages]) {
+        const uint32_t dst0 = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
+        // 4 pages x 136 chunks of 16 B (128 of codes, 8 of scales)
+        for (int i = tid; i < kTcBlockPages * (kTcPageBytes / 16); i += kTcThreads) {
+            const int pg = i / (kTcPageBytes / 16), c = i - pg * (kTcPageBytes / 16);
+            const int32_t id = pg == 0 ? pid[0] : pg == 1 ? pid[1] : pg == 2 ? pid[2] : pid[3];
+            if (id < 0)
+                continue;
+            const int64_t ph = static_cast<int64_t>(id) * p.hkv + h;
+            const uint8_t *src = c < 128 ? p.codes + ph * (2 * kPageSize * kRowBytes) + c * 16
+                                         : p.scales + ph * (2 * kPageSize * 4) + (c - 128) * 16;
+            cp_async16(dst0 + pg * kTcPageBytes + c * 16, src);
+        }
+        cp_async_commit();
+    };
+    int32_t pid_a[kTcBlockPages], pid_b[kTcBlockPages];
+    {
+        int32_t pid0[kTcBlockPages];
+#pragma unroll
+        for (int i = 0; i < kTcBlockPages; i++) {
+            pid0[i] = page_id(i);
+            pid_a[i] = page_id(kTcBlockPages + i);
+            pid_b[i] = page_id(2 * kTcBlockPages + i);
+        }
+        stage_block(0, pid0);
+    }
+
+    // ---- the query tile: rotate, scale, fp16, in the codes' d order ------------------------------
+    float sq = 0.0f;
+    {
+        float x[128];
+        if (live) {
+            const uint4 *src = reinterpret_cast<const uint4 *>(
+                p.q + ((static_cast<int64_t>(p.q_start[s]) + t0 + tq) * p.hq + h * G + hg) * 128);
+#pragma unroll
+            for (int c = 0; c < 16; c++) {
+                const uint4 u = src[c];
+                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+                for (int k = 0; k < 4; k++) {
+                    x[8 * c + 2 * k] = __uint_as_float(w[k] << 16);
+                    x[8 * c + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+                }
+            }
+        } else {
+#pragma unroll
+            for (int i = 0; i < 128; i++)
+                x[i] = 0.0f;
+        }
+#pragma unroll
+        for (int hb = 1; kRotate && hb < 128; hb <<= 1)
+#pragma unroll
+            for (int i = 0; i < 128; i++)
+                if ((i & hb) == 0) {
+                    const float a = x[i], b = x[i + hb];
+                    x[i] = a + b;
+                    x[i + hb] = a - b;
+                }
+#pragma unroll
+        for (int c = 0; c < 16; c++) {
+            uint32_t wv[4];
+#pragma unroll
+            for (int k = 0; k < 4; k++) {
+                __half hh[2];
+#pragma unroll
+                for (int e = 0; e < 2; e++) {
+                    const int d = 8 * c + chunk_d(2 * k + e);
+                    hh[e] = __float2half_rn(x[d] * (p.q_mult * kTcQScale));
+                    sq += __half2float(hh[e]);
+                }
+                wv[k] = half2_as_u32(__halves2half2(hh[0], hh[1]));
+            }
+            const uint32_t a = sbase + kSmQ + sw128_chunk(row, c, kTcRows * 128);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(wv[0]), "r"(wv[1]),
+                         "r"(wv[2]), "r"(wv[3]) : "memory");
+        }
+    }
+
+    // ---- tensor-memory base, per-row softmax state -------------------------------------------
+    async_proxy_fence();   // the Q tile is read by the tensor cores
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = *tmem_slot;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
+    float m_ref = -INFINITY, l = 0.0f, z = 0.0f;
+    bool aborted = false;
+    int kb = 0;
+
+    for (; kb < n_blocks; kb++) {
+        // stage block kb + 1 (ids loaded a block ago) and load the ids of block kb + 3
+        if (kb + 1 < n_blocks)
+            stage_block(kb + 1, pid_a);
+        else
+            cp_async_commit();
+#pragma unroll
+        for (int i = 0; i < kTcBlockPages; i++) {
+            pid_a[i] = pid_b[i];
+            pid_b[i] = page_id(kTcBlockPages * (kb + 3) + i);
+        }
+        cp_async_wait1();   // this thread's copies of block kb have landed
+        // the previous block's P V has finished with the V and P tiles
+        bool ok = kb == 0 || mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs);
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+
+        // ---- unpack the 4 pages into the fp16 K and V tiles, and the scales ------------------
+        const uint32_t stage = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
+        // 4 pages x 32 code rows (16 K, 16 V) x 16 words: 16 words per thread
+#pragma unroll
+        for (int i = 0; i < 16; i++) {
+            const int w = tid + kTcThreads * i;
+            const int pg = w >> 9, qw = w & 511, r = qw >> 4, c4 = qw & 15;
+            const uint32_t word = lds32(stage + pg * kTcPageBytes + r * 64 + c4 * 4);
+            const int tok = pg * kPageSize + (r & 15);
+            // exact fp16 integers: (0x6400 | n) is 1024 + n, minus 1024
+            const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+            const uint32_t y0 = half2_as_u32(__hsub2(u32_as_half2((word & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y1 = half2_as_u32(__hsub2(u32_as_half2(((word >> 4) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y2 = half2_as_u32(__hsub2(u32_as_half2(((word >> 8) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y3 = half2_as_u32(__hsub2(u32_as_half2(((word >> 12) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t dst = sbase + (r < 16 ? kSmK : kSmV) + sw128_chunk(tok, c4, kTcBlockTokens * 128);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2),
+                         "r"(y3) : "memory");
+        }
+        {
+            const int pg = tid >> 5, sel = (tid >> 4) & 1, tk = pg * kPageSize + (tid & 15);
+            float2 sz = __half22float2(u32_as_half2(lds32(stage + pg * kTcPageBytes + 2 * kPageSize * kRowBytes +
+                                                          sel * 64 + (tid & 15) * 4)));
+            if (kb * kTcBlockTokens + tk >= n_kv)
+                sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
+            if (sel == 0) {   // logit = (scale acc + zero sq) / 2^8 (the query's scale)
+                kpar[2 * tk] = sz.x * (1.0f / kTcQScale);
+                kpar[2 * tk + 1] = sz.y * (1.0f / kTcQScale);
+            } else {          // P' = 2^4 p scale
+                vpar[2 * tk] = sz.x * kTcPScale;
+                vpar[2 * tk + 1] = sz.y;
+            }
+        }
+        async_proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- S = Q K^T into tensor-memory columns 128 .. 191 ----------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id_qk = umma_idesc(kTcRows, kTcBlockTokens, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++) {
+                const uint32_t oq = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
+                const uint32_t ok_ = (ks >> 2) * (kTcBlockTokens * 128) + (ks & 3) * 32;
+                umma_f16(tmem + 128, umma_desc(sbase + kSmQ + oq, 16, 1024),
+                         umma_desc(sbase + kSmK + ok_, 16, 1024), id_qk, ks > 0);
+            }
+            umma_commit(bar_s);
+        }
+        ok = mbar_wait_bounded(bar_s, static_cast<uint32_t>(kb) & 1u, kTcWaitLimitNs);
+        if (!__syncthreads_and(ok)) {
+            aborted = true;
+            break;
+        }
+        tc_fence_after();
+        float sv[kTcBlockTokens];
+        tmem_ld32(lane_base + 128, sv);
+        tmem_ld32(lane_base + 160, sv + 32);
+
+        // ---- online softmax of this thread's row ------------------------------------------------
+        const int tok0 = kb * kTcBlockTokens;
+        const float4 *kp4 = reinterpret_cast<const float4 *>(kpar);
+        const float4 *vp4 = reinterpret_cast<const float4 *>(vpar);
+        float mb = -INFINITY;
+#pragma unroll
+        for (int j = 0; j < kTcBlockTokens; j += 2) {
+            const float4 kp = kp4[j / 2];
+            sv[j] = fmaf(kp.x, sv[j], kp.y * sq);
+            sv[j + 1] = fmaf(kp.z, sv[j + 1], kp.w * sq);
+        }
+        // the causal limit (and the end of the cache) only reaches the last blocks of a tile
+        if (tok0 + kTcBlockTokens - 1 > L - C + t0) {
+#pragma unroll
+            for (int j = 0; j < kTcBlockTokens; j++)
+                if (tok0 + j > limit)
+                    sv[j] = -INFINITY;
+        }
+#pragma unroll
+        for (int j = 0; j < kTcBlockTokens; j++)
+            mb = fmaxf(mb, sv[j]);
+        if (!live)
+            mb = -INFINITY;
+        const bool grow = mb > m_ref + kTcRescale;
+        float alpha = 1.0f;
+        if (grow) {
+            alpha = ex2_approx(m_ref - mb);   // 0 on the first block a row sees
+            l *= alpha;
+            z *= alpha;
+            m_ref = mb;
+        }
+        // rescale the O row in tensor memory (warp-wide instructions; alpha 1 where no change)
+        if (kb > 0 && __any_sync(0xFFFFFFFFu, grow && alpha != 0.0f)) {
+#pragma unroll 1
+            for (int c = 0; c < 4; c++) {
+                float ov[32];
+                tmem_ld32(lane_base + 32 * c, ov);
+#pragma unroll
+                for (int i = 0; i < 32; i++)
+                    ov[i] *= alpha;
+                tmem_st32(lane_base + 32 * c, ov);
+            }
+        }
+        uint32_t pw[kTcBlockTokens / 2];
+        const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
+#pragma unroll
+        for (int j = 0; j < kTcBlockTokens; j += 2) {
+            const float4 vp = vp4[j / 2];
+            const float p0 = ex2_approx(sv[j] - mr);
+            const float p1 = ex2_approx(sv[j + 1] - mr);
+            l += p0 + p1;
+            z = fmaf(p0, vp.y, fmaf(p1, vp.w, z));
+            pw[j / 2] = half2_as_u32(__floats2half2_rn(p0 * vp.x, p1 * vp.z));
+        }
+#pragma unroll
+        for (int c = 0; c < 8; c++) {
+            const uint32_t a = sbase + kSmP + sw128_chunk(row, c, kTcRows * 128);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pw[4 * c]),
+                         "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3]) : "memory");
+        }
+        async_proxy_fence();
+        tc_fence_before();
+        __syncthreads();
+
+        // ---- O += P' V into tensor-memory columns 0 .. 127 -----------------------------------------
+        if (tid == 0) {
+            tc_fence_after();
+            constexpr uint32_t id_pv = umma_idesc(kTcRows, 128, 0, 1);
+#pragma unroll
+            for (int ks = 0; ks < 4; ks++)
+                umma_f16(tmem, umma_desc(sbase + kSmP + ks * 32, 16, 1024),
+                         umma_desc(sbase + kSmV + ks * 2048, kTcBlockTokens * 128, 1024), id_pv,
+                         kb > 0 || ks > 0);
+            umma_commit(bar_o);
+        }
+    }
+
+    // ---- epilogue: O row -> zero term, 1 / l, the nibble scales, inverse rotation ----------------
+    if (!aborted) {
+        const bool ok = mbar_wait_bounded(bar_o, static_cast<uint32_t>(n_blocks - 1) & 1u, kTcWaitLimitNs);
+        aborted = !__syncthreads_and(ok);
+    }
+    if (aborted) {
+        if (tid == 0)
+            set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+        asm volatile("cp.async.wait_all;" ::: "memory");
+        // let MMAs that may still be in flight finish before the tensor memory is released
+        mbar_wait_bounded(bar_s, static_cast<uint32_t>(kb) & 1u, kTcWaitLimitNs / 10);
+        if (kb > 0)
+            mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs / 10);
+    } else {
+        tc_fence_after();
+        float o[128];
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+            tmem_ld32(lane_base + 32 * c, o + 32 * c);
+        if (live) {
+            const float inv = 1.0f / l;
+            float v[128];
+#pragma unroll
+            for (int n = 0; n < 128; n++) {
+                const int d = (n & ~7) + chunk_d(n & 7);
+                v[d] = fmaf(o[n], 1.0f / kTcPScale, z) * inv;
+            }
+#pragma unroll
+            for (int hb = 1; kRotate && hb < 128; hb <<= 1)
+#pragma unroll
+                for (int i = 0; i < 128; i++)
+                    if ((i & hb) == 0) {
+                        const float a = v[i], b = v[i + hb];
+                        v[i] = a + b;
+                        v[i + hb] = a - b;
+                    }
+            const float f = kRotate ? kTcHadamardC : 1.0f;
+            float4 *dst = reinterpret_cast<float4 *>(
+                p.out + ((static_cast<int64_t>(p.q_start[s]) + t0 + tq) * p.hq + h * G + hg) * 128);
+#pragma unroll
+            for (int c = 0; c < 32; c++)
+                dst[c] = make_float4(v[4 * c] * f, v[4 * c + 1] * f, v[4 * c + 2] * f, v[4 * c + 3] * f);
+        }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem), "r"(kTmemCols)
+                     : "memory");
+}
+
+}  // namespace
+
+// Tiles of T = 128 / G query tokens; the grid covers the most tiles any chunk split can give.
+int64_t prefill_tc_grid(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs, int64_t total_q)
+{
+    const int32_t G = num_q_heads / num_kv_heads;
+    const int32_t T = std::max(1, kTcRows / G);
+    return static_cast<int64_t>(num_kv_heads) * ((total_q + T - 1) / T + num_seqs);
+}
+
+cudaError_t launch_prefill_tc(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
+{
+    TcParams p;
+    p.q = static_cast<const uint16_t *>(a.q);
+    p.q_start = a.q_start;
+    p.codes = a.kv_pages;
+    p.scales = static_cast<const uint8_t *>(a.scales);
+    p.block_table = a.block_table;
+    p.seq_lens = a.seq_lens;
+    p.out = a.out;
+    p.status = a.status;
+    p.num_pages = a.num_pages;
+    p.max_blocks = a.max_blocks;
+    p.num_seqs = a.num_seqs;
+    p.hq = a.num_q_heads;
+    p.hkv = a.num_kv_heads;
+    p.group = a.num_q_heads / a.num_kv_heads;
+    p.tile_tokens = std::max(1, kTcRows / p.group);
+    // q carries sm_scale * log2(e) and 1/sqrt(128) of the unnormalised butterfly
+    p.q_mult = static_cast<float>((a.rotate ? static_cast<double>(kTcHadamardC) : 1.0) * a.sm_scale *
+                                  1.4426950408889634);
+    static bool attr_set[2] = {false, false};
+    auto *kernel = a.rotate ? prefill_tc_kernel<true> : prefill_tc_kernel<false>;
+    if (!attr_set[a.rotate ? 1 : 0]) {
+        const cudaError_t e = cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                                   static_cast<int>(kTcSmemBytes));
+        if (e != cudaSuccess)
+            return e;
+        attr_set[a.rotate ? 1 : 0] = true;
+    }
+    const int64_t grid = prefill_tc_grid(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q);
+    if (grid <= 0)
+        return cudaSuccess;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(kTcThreads);
+    cfg.dynamicSmemBytes = kTcSmemBytes;
+    cfg.stream = stream;
+    cfg.attrs = attr;
+    cfg.numAttrs = programmatic ? 1 : 0;
+    const cudaError_t e = cudaLaunchKernelEx(&cfg, kernel, p);
+    if (e != cudaSuccess)
+        return e;
+    return cudaGetLastError();
+}
+
+}  // namespace saw

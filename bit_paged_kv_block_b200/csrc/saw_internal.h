@@ -91,6 +91,11 @@ size_t decode_workspace_bytes(int32_t num_kv_heads, int32_t num_q_heads, int32_t
 // previous kernel on the stream.  Returns a cudaError_t.
 cudaError_t launch_paged_decode(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
 
+// Chunked prefill at head_dim 128 on the tensor cores (tcgen05): one CTA per tile of up to 128
+// query rows; no workspace.  prefill_tc_grid: the CTAs a launch takes (an upper bound on tiles).
+cudaError_t launch_prefill_tc(const DecodeArgs &a, cudaStream_t stream, bool programmatic);
+int64_t prefill_tc_grid(int32_t num_kv_heads, int32_t num_q_heads, int32_t num_seqs, int64_t total_q);
+
 // The uncompressed BF16 paged cache (baseline): scatter, decode workspace size, decode
 // (DecodeArgs::kv_pages is the bf16 cache; scales and rotate are unused).
 cudaError_t launch_append_bf16(const AppendBf16Args &a, cudaStream_t stream);
