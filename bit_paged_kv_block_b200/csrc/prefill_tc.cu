@@ -10,22 +10,23 @@
 // are s = scale_K acc + zero_K sum(q) over the raw codes; P' = p scale_V meets the raw V codes
 // and sum p zero_V is added in fp32; the output is rotated back.
 //
-// A CTA (4 warps) owns one tile of up to 128 query rows: T = 128 / G consecutive query tokens x
+// A CTA (8 warps) owns one tile of up to 128 query rows: T = 128 / G consecutive query tokens x
 // the G query heads of one kv head, row r = token (r / G), head (r % G).  It walks the tile's
 // causal range of the cache in blocks of 64 tokens (4 pages):
 //   1. the 4 pages' codes and scales are staged by cp.async (LSU path, one block ahead);
-//   2. all 128 threads unpack them once into fp16 tiles: K [64 tokens x 128 d] and
+//   2. all 256 threads unpack them once into fp16 tiles: K [64 tokens x 128 d] and
 //      V [64 tokens x 128 d], token rows of 128 B per half of d under the 128-byte swizzle;
 //   3. one thread issues S = Q K^T (M 128, N 64, K 128: 8 x tcgen05.mma.kind::f16) into tensor
 //      memory;
-//   4. each thread reads its row of S (tcgen05.ld), applies scales, zero points and the causal
-//      limit, and runs the online softmax for its row alone; P' (fp16) goes to a shared tile;
+//   4. two threads per row each read half of the row of S (tcgen05.ld), apply scales, zero points
+//      and the causal limit, share the block maximum and run the online softmax; P' (fp16) goes
+//      to a shared tile;
 //   5. one thread issues O += P' V (M 128, N 128, K 64: 4 MMAs, V read as the MN-major operand).
 // When a block's maximum exceeds a row's running maximum, the row's O accumulator is rescaled in
 // tensor memory (the warp's 32 rows together; rows without a change multiply by 1).  Letting the
 // maximum lag (weights up to 2^4) saved no measurable time and doubled the largest error.
-// The epilogue reads each thread's O row, adds the zero-point term, divides by the row sum and
-// rotates back.
+// The epilogue reads each thread's half of its O row, adds the zero-point term, divides by the row
+// sum and rotates back (the last Hadamard stage pairs the halves through shared memory).
 //
 // Codes enter the tensor cores as exact fp16 integers n = (1024 + n) - 1024 (a magic OR and one
 // half2 subtraction per pair).  These tensor cores flush fp16 subnormals, so the operands are kept
@@ -46,7 +47,7 @@
 namespace saw {
 namespace {
 
-constexpr int kTcThreads = 128;
+constexpr int kTcThreads = 256;
 constexpr int kTcRows = 128;                 // M of the MMAs: query rows per tile
 constexpr int kTcBlockTokens = 64;           // N of QK, K of PV: cache tokens per block
 constexpr int kTcBlockPages = kTcBlockTokens / kPageSize;
@@ -64,7 +65,8 @@ constexpr int kSmV = kSmK + 2 * kTcBlockTokens * 128;    // V tile: 2 x [64 toke
 constexpr int kSmP = kSmV + 2 * kTcBlockTokens * 128;    // P tile: [128 rows][128 B]
 constexpr int kSmCodes = kSmP + kTcRows * 128;           // 2 stages x 4 pages (codes, scales)
 constexpr int kSmScales = kSmCodes + 2 * kTcBlockPages * kTcPageBytes;   // per token pair: float4 (K), float4 (V)
-constexpr int kSmBars = kSmScales + 4 * kTcBlockTokens * 4;              // 2 mbarriers + tmem addr
+constexpr int kSmXchg = kSmScales + 4 * kTcBlockTokens * 4;              // [4][128] fp32 between row halves
+constexpr int kSmBars = kSmXchg + 4 * kTcRows * 4;                       // 2 mbarriers + tmem addr
 constexpr int kSmTile = kSmBars + 32;                                    // tile descriptor
 constexpr int kSmBytes = kSmTile + 64;
 constexpr size_t kTcSmemBytes = 1024 + kSmBytes;
@@ -231,13 +233,19 @@ __device__ bool find_tile(const TcParams &p, int cta, int &s_out, int &h_out, in
     return true;
 }
 
+// Thread layout: 8 warps; warp w owns the 32 tile rows of tensor-memory lanes 32 (w mod 4) ..
+// (its lane quarter) and the half hf = w / 4 of each block's 64 tokens and of O's 128 columns.
+// The two threads of a row exchange only the block maximum (and, once, the sums of the query and
+// the final l, z and the last Hadamard stage) through shared memory.
 template <bool kRotate>
-__global__ void __launch_bounds__(kTcThreads, 1)
+__global__ void __launch_bounds__(kTcThreads, 2)
     prefill_tc_kernel(const TcParams p)
 {
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-    const int tid = threadIdx.x, warp = tid >> 5;
+    const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+    const int hf = warp >> 2;                             // token / column half
+    const int row = 32 * (warp & 3) + lane;               // tile row = tensor-memory lane
     const uint32_t sbase = smem_u32(smem);
     int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 16);
@@ -246,6 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     // for V (P' factor, zero point)
     float *kpar = reinterpret_cast<float *>(smem + kSmScales);
     float *vpar = kpar + 2 * kTcBlockTokens;
+    float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [2 halves][128 rows] x 4
 
     pdl_launch_dependents();
     int s, h, t0;
@@ -261,7 +270,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
     const int ntok = min(p.tile_tokens, C - t0);          // query tokens of this tile
     const int nrows = ntok * G;
-    const int row = tid;                                   // this thread's row of the tile
     const bool live = row < nrows;
     const int tq = live ? row / G : 0, hg = live ? row - tq * G : 0;
     const int limit = L - C + t0 + tq;                     // last visible cache token of the row
@@ -284,7 +292,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     pdl_wait();   // the cache may be written by the kernel this one depends on
 
     // ---- staging of a block's 4 pages (codes, then scales) by cp.async, one block ahead --------
-    // page ids of blocks kb + 1 (pid_a) and kb + 2 (pid_b), loaded a block before their use
+    // this thread's 16-byte chunks of a block are i = tid + 256 k (k < 3, i < 544): page
+    // i / 136, chunk i mod 136 (128 of codes, 8 of scales); the mapping is the same every block
     const int64_t bt_row = static_cast<int64_t>(s) * p.max_blocks;
     auto page_id = [&](int pg) -> int32_t {
         if (pg >= n_pages)
@@ -296,11 +305,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
         return id;
     };
+    constexpr int kChunksPerPage = kTcPageBytes / 16;
+    constexpr int kBlockChunks = kTcBlockPages * kChunksPerPage;
     auto stage_block = [&](int kb, const int32_t pid[kTcBlockPages]) {
         const uint32_t dst0 = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
-        // 4 pages x 136 chunks of 16 B (128 of codes, 8 of scales)
-        for (int i = tid; i < kTcBlockPages * (kTcPageBytes / 16); i += kTcThreads) {
-            const int pg = i / (kTcPageBytes / 16), c = i - pg * (kTcPageBytes / 16);
+#pragma unroll
+        for (int k = 0; k < (kBlockChunks + kTcThreads - 1) / kTcThreads; k++) {
+            const int i = tid + kTcThreads * k;
+            if (i >= kBlockChunks)
+                break;
+            const int pg = i / kChunksPerPage, c = i - pg * kChunksPerPage;
             const int32_t id = pg == 0 ? pid[0] : pg == 1 ? pid[1] : pg == 2 ? pid[2] : pid[3];
             if (id < 0)
                 continue;
@@ -323,65 +337,73 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         stage_block(0, pid0);
     }
 
-    // ---- the query tile: rotate, scale, fp16, in the codes' d order ------------------------------
-    float sq = 0.0f;
+    // ---- the query tile: rotate, scale, fp16, in the codes' d order --------------------------------
+    // This thread's half of d: the cross-half Hadamard stage (d, d + 64) first, from the whole
+    // row, then the 6 stages within the half (the order of the stages does not matter here: the
+    // query is not required to be bit-exact, only the quantized cache is).
     {
-        float x[128];
+        float x[64];
         if (live) {
             const uint4 *src = reinterpret_cast<const uint4 *>(
                 p.q + ((static_cast<int64_t>(p.q_start[s]) + t0 + tq) * p.hq + h * G + hg) * 128);
 #pragma unroll
-            for (int c = 0; c < 16; c++) {
-                const uint4 u = src[c];
-                const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+            for (int c = 0; c < 8; c++) {
+                const uint4 ua = src[c], ub = src[8 + c];   // d in [0, 64) and [64, 128)
+                const uint32_t wa[4] = {ua.x, ua.y, ua.z, ua.w}, wb[4] = {ub.x, ub.y, ub.z, ub.w};
 #pragma unroll
                 for (int k = 0; k < 4; k++) {
-                    x[8 * c + 2 * k] = __uint_as_float(w[k] << 16);
-                    x[8 * c + 2 * k + 1] = __uint_as_float(w[k] & 0xFFFF0000u);
+#pragma unroll
+                    for (int e = 0; e < 2; e++) {
+                        const float a = __uint_as_float(e ? (wa[k] & 0xFFFF0000u) : (wa[k] << 16));
+                        const float b = __uint_as_float(e ? (wb[k] & 0xFFFF0000u) : (wb[k] << 16));
+                        x[8 * c + 2 * k + e] = !kRotate ? (hf ? b : a) : (hf ? a - b : a + b);
+                    }
                 }
             }
         } else {
 #pragma unroll
-            for (int i = 0; i < 128; i++)
+            for (int i = 0; i < 64; i++)
                 x[i] = 0.0f;
         }
 #pragma unroll
-        for (int hb = 1; kRotate && hb < 128; hb <<= 1)
+        for (int hb = 1; kRotate && hb < 64; hb <<= 1)
 #pragma unroll
-            for (int i = 0; i < 128; i++)
+            for (int i = 0; i < 64; i++)
                 if ((i & hb) == 0) {
                     const float a = x[i], b = x[i + hb];
                     x[i] = a + b;
                     x[i + hb] = a - b;
                 }
+        float sq_half = 0.0f;
 #pragma unroll
-        for (int c = 0; c < 16; c++) {
+        for (int c = 0; c < 8; c++) {
             uint32_t wv[4];
 #pragma unroll
             for (int k = 0; k < 4; k++) {
                 __half hh[2];
 #pragma unroll
                 for (int e = 0; e < 2; e++) {
-                    const int d = 8 * c + chunk_d(2 * k + e);
-                    hh[e] = __float2half_rn(x[d] * (p.q_mult * kTcQScale));
-                    sq += __half2float(hh[e]);
+                    hh[e] = __float2half_rn(x[8 * c + chunk_d(2 * k + e)] * (p.q_mult * kTcQScale));
+                    sq_half += __half2float(hh[e]);
                 }
                 wv[k] = half2_as_u32(__halves2half2(hh[0], hh[1]));
             }
-            const uint32_t a = sbase + kSmQ + sw128_chunk(row, c, kTcRows * 128);
+            const uint32_t a = sbase + kSmQ + sw128_chunk(row, 8 * hf + c, kTcRows * 128);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(wv[0]), "r"(wv[1]),
                          "r"(wv[2]), "r"(wv[3]) : "memory");
         }
+        xchg[hf * kTcRows + row] = sq_half;
     }
 
-    // ---- tensor-memory base, per-row softmax state -------------------------------------------
+    // ---- tensor-memory base, the row's sum of q, per-row softmax state ------------------------------
     async_proxy_fence();   // the Q tile is read by the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * warp) << 16);
-    float m_ref = -INFINITY, l = 0.0f, z = 0.0f;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    const float sq = xchg[row] + xchg[kTcRows + row];
+    float m_ref = -INFINITY, l = 0.0f, z = 0.0f;   // l, z: this half's partial sums
     bool aborted = false;
     int kb = 0;
 
@@ -405,10 +427,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
 
         // ---- unpack the 4 pages into the fp16 K and V tiles, and the scales ------------------
+        // 4 pages x 32 code rows (16 K, 16 V) x 16 words: 8 words per thread
         const uint32_t stage = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
-        // 4 pages x 32 code rows (16 K, 16 V) x 16 words: 16 words per thread
 #pragma unroll
-        for (int i = 0; i < 16; i++) {
+        for (int i = 0; i < 8; i++) {
             const int w = tid + kTcThreads * i;
             const int pg = w >> 9, qw = w & 511, r = qw >> 4, c4 = qw & 15;
             const uint32_t word = lds32(stage + pg * kTcPageBytes + r * 64 + c4 * 4);
@@ -423,7 +445,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2),
                          "r"(y3) : "memory");
         }
-        {
+        if (tid < 2 * kTcBlockTokens) {
             const int pg = tid >> 5, sel = (tid >> 4) & 1, tk = pg * kPageSize + (tid & 15);
             float2 sz = __half22float2(u32_as_half2(lds32(stage + pg * kTcPageBytes + 2 * kPageSize * kRowBytes +
                                                           sel * 64 + (tid & 15) * 4)));
@@ -460,33 +482,35 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             break;
         }
         tc_fence_after();
-        float sv[kTcBlockTokens];
-        tmem_ld32(lane_base + 128, sv);
-        tmem_ld32(lane_base + 160, sv + 32);
+        float sv[32];   // tokens 32 hf .. 32 hf + 31 of the block
+        tmem_ld32(lane_base + 128 + 32 * hf, sv);
 
-        // ---- online softmax of this thread's row ------------------------------------------------
-        const int tok0 = kb * kTcBlockTokens;
-        const float4 *kp4 = reinterpret_cast<const float4 *>(kpar);
-        const float4 *vp4 = reinterpret_cast<const float4 *>(vpar);
-        float mb = -INFINITY;
+        // ---- online softmax: this half of the row, one shared maximum ---------------------------
+        const int tok0 = kb * kTcBlockTokens + 32 * hf;
+        const float4 *kp4 = reinterpret_cast<const float4 *>(kpar) + 16 * hf;
+        const float4 *vp4 = reinterpret_cast<const float4 *>(vpar) + 16 * hf;
 #pragma unroll
-        for (int j = 0; j < kTcBlockTokens; j += 2) {
+        for (int j = 0; j < 32; j += 2) {
             const float4 kp = kp4[j / 2];
             sv[j] = fmaf(kp.x, sv[j], kp.y * sq);
             sv[j + 1] = fmaf(kp.z, sv[j + 1], kp.w * sq);
         }
         // the causal limit (and the end of the cache) only reaches the last blocks of a tile
-        if (tok0 + kTcBlockTokens - 1 > L - C + t0) {
+        if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
 #pragma unroll
-            for (int j = 0; j < kTcBlockTokens; j++)
+            for (int j = 0; j < 32; j++)
                 if (tok0 + j > limit)
                     sv[j] = -INFINITY;
         }
+        float mb = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < kTcBlockTokens; j++)
+        for (int j = 0; j < 32; j++)
             mb = fmaxf(mb, sv[j]);
         if (!live)
             mb = -INFINITY;
+        xchg[2 * kTcRows + hf * kTcRows + row] = mb;
+        __syncthreads();
+        mb = fmaxf(mb, xchg[2 * kTcRows + (1 - hf) * kTcRows + row]);
         const bool grow = mb > m_ref + kTcRescale;
         float alpha = 1.0f;
         if (grow) {
@@ -495,22 +519,23 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             z *= alpha;
             m_ref = mb;
         }
-        // rescale the O row in tensor memory (warp-wide instructions; alpha 1 where no change)
+        // rescale this half of the O row in tensor memory (warp-wide instructions; alpha 1 where
+        // no change)
         if (kb > 0 && __any_sync(0xFFFFFFFFu, grow && alpha != 0.0f)) {
 #pragma unroll 1
-            for (int c = 0; c < 4; c++) {
+            for (int c = 0; c < 2; c++) {
                 float ov[32];
-                tmem_ld32(lane_base + 32 * c, ov);
+                tmem_ld32(lane_base + 64 * hf + 32 * c, ov);
 #pragma unroll
                 for (int i = 0; i < 32; i++)
                     ov[i] *= alpha;
-                tmem_st32(lane_base + 32 * c, ov);
+                tmem_st32(lane_base + 64 * hf + 32 * c, ov);
             }
         }
-        uint32_t pw[kTcBlockTokens / 2];
+        uint32_t pw[16];
         const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
 #pragma unroll
-        for (int j = 0; j < kTcBlockTokens; j += 2) {
+        for (int j = 0; j < 32; j += 2) {
             const float4 vp = vp4[j / 2];
             const float p0 = ex2_approx(sv[j] - mr);
             const float p1 = ex2_approx(sv[j + 1] - mr);
@@ -519,8 +544,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             pw[j / 2] = half2_as_u32(__floats2half2_rn(p0 * vp.x, p1 * vp.z));
         }
 #pragma unroll
-        for (int c = 0; c < 8; c++) {
-            const uint32_t a = sbase + kSmP + sw128_chunk(row, c, kTcRows * 128);
+        for (int c = 0; c < 4; c++) {
+            const uint32_t a = sbase + kSmP + sw128_chunk(row, 4 * hf + c, kTcRows * 128);
             asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pw[4 * c]),
                          "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3]) : "memory");
         }
@@ -541,7 +566,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         }
     }
 
-    // ---- epilogue: O row -> zero term, 1 / l, the nibble scales, inverse rotation ----------------
+    // ---- epilogue: O row -> zero term, 1 / l, the weights' scale, inverse rotation ----------------
     if (!aborted) {
         const bool ok = mbar_wait_bounded(bar_o, static_cast<uint32_t>(n_blocks - 1) & 1u, kTcWaitLimitNs);
         aborted = !__syncthreads_and(ok);
@@ -556,32 +581,55 @@ __global__ void __launch_bounds__(kTcThreads, 1)
             mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs / 10);
     } else {
         tc_fence_after();
-        float o[128];
+        // this half's 64 O columns = d in [64 hf, 64 hf + 64) (the d order permutes within 8)
+        float o[64];
+        tmem_ld32(lane_base + 64 * hf, o);
+        tmem_ld32(lane_base + 64 * hf + 32, o + 32);
+        xchg[hf * kTcRows + row] = l;
+        xchg[2 * kTcRows + hf * kTcRows + row] = z;
+        __syncthreads();
+        const float lt = xchg[row] + xchg[kTcRows + row];
+        const float zt = xchg[2 * kTcRows + row] + xchg[3 * kTcRows + row];
+        const float inv = live ? 1.0f / lt : 0.0f;
+        float v[64];
 #pragma unroll
-        for (int c = 0; c < 4; c++)
-            tmem_ld32(lane_base + 32 * c, o + 32 * c);
-        if (live) {
-            const float inv = 1.0f / l;
-            float v[128];
+        for (int n = 0; n < 64; n++) {
+            const int d = (n & ~7) + chunk_d(n & 7);
+            v[d] = fmaf(o[n], 1.0f / kTcPScale, zt) * inv;
+        }
+        // inverse rotation: the 6 stages within the half, then (d, d + 64) through shared memory
+        // (all tiles are free now: the exchange uses the Q, K and V tiles' 64 KB)
 #pragma unroll
-            for (int n = 0; n < 128; n++) {
-                const int d = (n & ~7) + chunk_d(n & 7);
-                v[d] = fmaf(o[n], 1.0f / kTcPScale, z) * inv;
+        for (int hb = 1; kRotate && hb < 64; hb <<= 1)
+#pragma unroll
+            for (int i = 0; i < 64; i++)
+                if ((i & hb) == 0) {
+                    const float a = v[i], b = v[i + hb];
+                    v[i] = a + b;
+                    v[i + hb] = a - b;
+                }
+        if (kRotate) {
+            float4 *mine = reinterpret_cast<float4 *>(smem + kSmQ) + (hf * kTcRows + row) * 16;
+            const float4 *other = reinterpret_cast<const float4 *>(smem + kSmQ) + ((1 - hf) * kTcRows + row) * 16;
+#pragma unroll
+            for (int c = 0; c < 16; c++)
+                mine[c] = make_float4(v[4 * c], v[4 * c + 1], v[4 * c + 2], v[4 * c + 3]);
+            __syncthreads();
+#pragma unroll
+            for (int c = 0; c < 16; c++) {
+                const float4 w = other[c];
+                const float b4[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+                for (int k = 0; k < 4; k++)   // low half: a + b; high half: a - b (a the low value)
+                    v[4 * c + k] = hf ? b4[k] - v[4 * c + k] : v[4 * c + k] + b4[k];
             }
-#pragma unroll
-            for (int hb = 1; kRotate && hb < 128; hb <<= 1)
-#pragma unroll
-                for (int i = 0; i < 128; i++)
-                    if ((i & hb) == 0) {
-                        const float a = v[i], b = v[i + hb];
-                        v[i] = a + b;
-                        v[i + hb] = a - b;
-                    }
+        }
+        if (live) {
             const float f = kRotate ? kTcHadamardC : 1.0f;
             float4 *dst = reinterpret_cast<float4 *>(
-                p.out + ((static_cast<int64_t>(p.q_start[s]) + t0 + tq) * p.hq + h * G + hg) * 128);
+                p.out + ((static_cast<int64_t>(p.q_start[s]) + t0 + tq) * p.hq + h * G + hg) * 128 + 64 * hf);
 #pragma unroll
-            for (int c = 0; c < 32; c++)
+            for (int c = 0; c < 16; c++)
                 dst[c] = make_float4(v[4 * c] * f, v[4 * c + 1] * f, v[4 * c + 2] * f, v[4 * c + 3] * f);
         }
     }
