@@ -250,8 +250,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
     uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 16);
     const uint32_t bar_s = sbase + kSmBars, bar_o = sbase + kSmBars + 8;
-    // kpar[j / 2] = (scale, zero, scale, zero) of K tokens j, j + 1 (logit factors); vpar likewise
-    // for V (P' factor, zero point)
+    // kpar[j / 2] = (scale_j, scale_j+1, zero_j, zero_j+1) of K tokens j, j + 1 (logit factors);
+    // vpar likewise for V (P' factors, zero points): two tokens per packed f32x2 operation
     float *kpar = reinterpret_cast<float *>(smem + kSmScales);
     float *vpar = kpar + 2 * kTcBlockTokens;
     float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [2 halves][128 rows] x 4
@@ -403,7 +403,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
     const float sq = xchg[row] + xchg[kTcRows + row];
-    float m_ref = -INFINITY, l = 0.0f, z = 0.0f;   // l, z: this half's partial sums
+    float m_ref = -INFINITY;
+    uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;   // this half's partial sums (two lanes each)
     bool aborted = false;
     int kb = 0;
 
@@ -451,12 +452,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                                                           sel * 64 + (tid & 15) * 4)));
             if (kb * kTcBlockTokens + tk >= n_kv)
                 sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
+            float *par = (sel == 0 ? kpar : vpar) + 4 * (tk >> 1) + (tk & 1);
             if (sel == 0) {   // logit = (scale acc + zero sq) / 2^8 (the query's scale)
-                kpar[2 * tk] = sz.x * (1.0f / kTcQScale);
-                kpar[2 * tk + 1] = sz.y * (1.0f / kTcQScale);
+                par[0] = sz.x * (1.0f / kTcQScale);
+                par[2] = sz.y * (1.0f / kTcQScale);
             } else {          // P' = 2^4 p scale
-                vpar[2 * tk] = sz.x * kTcPScale;
-                vpar[2 * tk + 1] = sz.y;
+                par[0] = sz.x * kTcPScale;
+                par[2] = sz.y;
             }
         }
         async_proxy_fence();
@@ -489,11 +491,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         const int tok0 = kb * kTcBlockTokens + 32 * hf;
         const float4 *kp4 = reinterpret_cast<const float4 *>(kpar) + 16 * hf;
         const float4 *vp4 = reinterpret_cast<const float4 *>(vpar) + 16 * hf;
+        const uint64_t sq2 = f2_pack(sq, sq);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
             const float4 kp = kp4[j / 2];
-            sv[j] = fmaf(kp.x, sv[j], kp.y * sq);
-            sv[j + 1] = fmaf(kp.z, sv[j + 1], kp.w * sq);
+            const uint64_t t = f2_fma(f2_pack(kp.x, kp.y), f2_pack(sv[j], sv[j + 1]),
+                                      f2_mul(f2_pack(kp.z, kp.w), sq2));
+            f2_unpack(t, sv[j], sv[j + 1]);
         }
         // the causal limit (and the end of the cache) only reaches the last blocks of a tile
         if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
@@ -504,8 +508,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
         float mb = -INFINITY;
 #pragma unroll
-        for (int j = 0; j < 32; j++)
-            mb = fmaxf(mb, sv[j]);
+        for (int j = 0; j < 32; j += 2)
+            mb = fmax3(mb, sv[j], sv[j + 1]);
         if (!live)
             mb = -INFINITY;
         xchg[2 * kTcRows + hf * kTcRows + row] = mb;
@@ -515,8 +519,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         float alpha = 1.0f;
         if (grow) {
             alpha = ex2_approx(m_ref - mb);   // 0 on the first block a row sees
-            l *= alpha;
-            z *= alpha;
+            const uint64_t a2 = f2_pack(alpha, alpha);
+            l2 = f2_mul(l2, a2);
+            z2 = f2_mul(z2, a2);
             m_ref = mb;
         }
         // rescale this half of the O row in tensor memory (warp-wide instructions; alpha 1 where
@@ -534,14 +539,18 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         }
         uint32_t pw[16];
         const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
+        const uint64_t mr2 = f2_pack(mr, mr);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
             const float4 vp = vp4[j / 2];
-            const float p0 = ex2_approx(sv[j] - mr);
-            const float p1 = ex2_approx(sv[j + 1] - mr);
-            l += p0 + p1;
-            z = fmaf(p0, vp.y, fmaf(p1, vp.w, z));
-            pw[j / 2] = half2_as_u32(__floats2half2_rn(p0 * vp.x, p1 * vp.z));
+            float d0, d1;
+            f2_unpack(f2_sub(f2_pack(sv[j], sv[j + 1]), mr2), d0, d1);
+            const uint64_t p2 = f2_pack(ex2_approx(d0), ex2_approx(d1));
+            l2 = f2_add(l2, p2);
+            z2 = f2_fma(p2, f2_pack(vp.z, vp.w), z2);
+            float w0, w1;
+            f2_unpack(f2_mul(p2, f2_pack(vp.x, vp.y)), w0, w1);
+            pw[j / 2] = half2_as_u32(__floats2half2_rn(w0, w1));
         }
 #pragma unroll
         for (int c = 0; c < 4; c++) {
@@ -585,8 +594,11 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         float o[64];
         tmem_ld32(lane_base + 64 * hf, o);
         tmem_ld32(lane_base + 64 * hf + 32, o + 32);
-        xchg[hf * kTcRows + row] = l;
-        xchg[2 * kTcRows + hf * kTcRows + row] = z;
+        float la, lb, za, zb;
+        f2_unpack(l2, la, lb);
+        f2_unpack(z2, za, zb);
+        xchg[hf * kTcRows + row] = la + lb;
+        xchg[2 * kTcRows + hf * kTcRows + row] = za + zb;
         __syncthreads();
         const float lt = xchg[row] + xchg[kTcRows + row];
         const float zt = xchg[2 * kTcRows + row] + xchg[3 * kTcRows + row];
