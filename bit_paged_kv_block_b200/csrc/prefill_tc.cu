@@ -13,15 +13,19 @@
 // A CTA (8 warps) owns one tile of up to 128 query rows: T = 128 / G consecutive query tokens x
 // the G query heads of one kv head, row r = token (r / G), head (r % G).  It walks the tile's
 // causal range of the cache in blocks of 64 tokens (4 pages):
-//   1. the 4 pages' codes and scales are staged by cp.async (LSU path, one block ahead);
+//   1. the 4 pages' codes and scales are staged by cp.async (LSU path) into one code stage;
 //   2. all 256 threads unpack them once into fp16 tiles: K [64 tokens x 128 d] and
 //      V [64 tokens x 128 d], token rows of 128 B per half of d under the 128-byte swizzle;
-//   3. one thread issues S = Q K^T (M 128, N 64, K 128: 8 x tcgen05.mma.kind::f16) into tensor
-//      memory;
+//   3. one thread issues S = Q K^T (M 128, N 64, K 128: 8 x tcgen05.mma.kind::f16) into one of
+//      two S buffers in tensor memory;
 //   4. two threads per row each read half of the row of S (tcgen05.ld), apply scales, zero points
 //      and the causal limit, share the block maximum and run the online softmax; P' (fp16) goes
 //      to a shared tile;
 //   5. one thread issues O += P' V (M 128, N 128, K 64: 4 MMAs, V read as the MN-major operand).
+// The loop is software-pipelined by one block: while the threads run the softmax of block kb, the
+// tensor cores compute S of block kb + 1 (unpacked and issued just before), and P V of block kb
+// runs while the threads unpack the K of block kb + 2; V and the scale tables are double-buffered,
+// the codes of block kb + 2 are in flight meanwhile, and the block table is read three blocks ahead.
 // When a block's maximum exceeds a row's running maximum, the row's O accumulator is rescaled in
 // tensor memory (the warp's 32 rows together; rows without a change multiply by 1).  Letting the
 // maximum lag (weights up to 2^4) saved no measurable time and doubled the largest error.
@@ -58,19 +62,22 @@ constexpr float kTcQScale = 256.0f;          // query entries enter the MMA scal
 constexpr float kTcPScale = 16.0f;           // weights enter the MMA scaled by 2^4
 constexpr uint64_t kTcWaitLimitNs = 1000000000ull;
 
-// shared memory (from a 1024-byte aligned base)
+// shared memory (from a 1024-byte aligned base); 2 CTAs fit on an SM
 constexpr int kSmQ = 0;                                  // Q tile: 2 x [128 rows][128 B]
 constexpr int kSmK = kSmQ + 2 * kTcRows * 128;           // K tile: 2 x [64 tokens][128 B]
-constexpr int kSmV = kSmK + 2 * kTcBlockTokens * 128;    // V tile: 2 x [64 tokens][128 B]
-constexpr int kSmP = kSmV + 2 * kTcBlockTokens * 128;    // P tile: [128 rows][128 B]
-constexpr int kSmCodes = kSmP + kTcRows * 128;           // 2 stages x 4 pages (codes, scales)
-constexpr int kSmScales = kSmCodes + 2 * kTcBlockPages * kTcPageBytes;   // per token pair: float4 (K), float4 (V)
-constexpr int kSmXchg = kSmScales + 4 * kTcBlockTokens * 4;              // [4][128] fp32 between row halves
-constexpr int kSmBars = kSmXchg + 4 * kTcRows * 4;                       // 2 mbarriers + tmem addr
-constexpr int kSmTile = kSmBars + 32;                                    // tile descriptor
+constexpr int kSmV = kSmK + 2 * kTcBlockTokens * 128;    // 2 V tiles: 2 x [64 tokens][128 B] each
+constexpr int kSmVTile = 2 * kTcBlockTokens * 128;
+constexpr int kSmP = kSmV + 2 * kSmVTile;                // P tile: [128 rows][128 B]
+constexpr int kSmCodes = kSmP + kTcRows * 128;           // one block's 4 pages (codes, scales)
+constexpr int kSmScales = kSmCodes + kTcBlockPages * kTcPageBytes;   // 2 x (K, V) token-pair factors
+constexpr int kSmScaleSet = 2 * 2 * kTcBlockTokens * 4;
+constexpr int kSmXchg = kSmScales + 2 * kSmScaleSet;     // [4][128] fp32 between row halves
+constexpr int kSmPid = kSmXchg + 4 * kTcRows * 4;        // page ids of 4 blocks (ring)
+constexpr int kSmBars = kSmPid + 4 * kTcBlockPages * 4;  // 2 mbarriers + tmem addr
+constexpr int kSmTile = kSmBars + 32;                    // tile descriptor
 constexpr int kSmBytes = kSmTile + 64;
 constexpr size_t kTcSmemBytes = 1024 + kSmBytes;
-constexpr uint32_t kTmemCols = 256;                      // O: columns 0..127, S: 128..191
+constexpr uint32_t kTmemCols = 256;                      // O: columns 0..127, S: 128..255 (2 x 64)
 
 // byte offset of 16-bit element (row, k) in a tile of rows of 64 elements (128 B) per atom,
 // atom stride atom_bytes, 128-byte swizzle (16-byte chunk index XOR row mod 8)
@@ -159,7 +166,6 @@ __device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
     asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-__device__ __forceinline__ void cp_async_wait1() { asm volatile("cp.async.wait_group 1;" ::: "memory"); }
 
 // d order of the 8 entries of a 16-byte chunk: position j holds d = 8 a + kPerm[j]
 __host__ __device__ constexpr int chunk_d(int j) { return (j >> 1) + ((j & 1) << 2); }
@@ -248,12 +254,9 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int row = 32 * (warp & 3) + lane;               // tile row = tensor-memory lane
     const uint32_t sbase = smem_u32(smem);
     int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 16);
-    const uint32_t bar_s = sbase + kSmBars, bar_o = sbase + kSmBars + 8;
-    // kpar[j / 2] = (scale_j, scale_j+1, zero_j, zero_j+1) of K tokens j, j + 1 (logit factors);
-    // vpar likewise for V (P' factors, zero points): two tokens per packed f32x2 operation
-    float *kpar = reinterpret_cast<float *>(smem + kSmScales);
-    float *vpar = kpar + 2 * kTcBlockTokens;
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 24);
+    // S of even / odd blocks (bar_s0, bar_s0 + 8), O += P V (bar_o)
+    const uint32_t bar_s0 = sbase + kSmBars, bar_o = sbase + kSmBars + 16;
     float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [2 halves][128 rows] x 4
 
     pdl_launch_dependents();
@@ -279,7 +282,8 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
     // ---- tensor memory and barriers -----------------------------------------------------------
     if (tid == 0) {
-        mbar_init(bar_s, 1);
+        mbar_init(bar_s0, 1);
+        mbar_init(bar_s0 + 8, 1);
         mbar_init(bar_o, 1);
     }
     mbar_init_fence();
@@ -291,51 +295,87 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
     pdl_wait();   // the cache may be written by the kernel this one depends on
 
-    // ---- staging of a block's 4 pages (codes, then scales) by cp.async, one block ahead --------
-    // this thread's 16-byte chunks of a block are i = tid + 256 k (k < 3, i < 544): page
-    // i / 136, chunk i mod 136 (128 of codes, 8 of scales); the mapping is the same every block
+    // ---- page ids: threads 0-3 load a block's 4 ids three blocks ahead and check them into a
+    //      shared ring of 4 blocks half an iteration later, so the loads never stall the loop ------
+    int32_t *pid_ring = reinterpret_cast<int32_t *>(smem + kSmPid);
     const int64_t bt_row = static_cast<int64_t>(s) * p.max_blocks;
-    auto page_id = [&](int pg) -> int32_t {
-        if (pg >= n_pages)
-            return -1;   // past the tile's range: not staged
-        int32_t id = p.block_table[bt_row + pg];
-        if (id < 0 || id >= p.num_pages) {
+    auto raw_id = [&](int pg) -> int32_t {
+        return pg < n_pages ? p.block_table[bt_row + pg] : -1;   // -1: past the tile's range
+    };
+    auto store_id = [&](int kb_, int32_t id) {   // thread tid < 4: page 4 kb_ + tid
+        const int pg = kTcBlockPages * kb_ + tid;
+        if (pg < n_pages && (id < 0 || id >= p.num_pages)) {
             set_status(p.status, SAW_DEV_BAD_PAGE);
             id = 0;
         }
-        return id;
+        pid_ring[(kb_ & 3) * kTcBlockPages + tid] = id;
     };
+    // ---- staging of a block's 4 pages (codes, then scales) by cp.async into the code stage ----
+    // this thread's 16-byte chunks are i = tid + 256 k (i < 544): page i / 136, chunk i mod 136
+    // (128 of codes, 8 of scales)
     constexpr int kChunksPerPage = kTcPageBytes / 16;
     constexpr int kBlockChunks = kTcBlockPages * kChunksPerPage;
-    auto stage_block = [&](int kb, const int32_t pid[kTcBlockPages]) {
-        const uint32_t dst0 = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
+    auto stage_block = [&](int kb_) {
+        const int32_t *pid = pid_ring + (kb_ & 3) * kTcBlockPages;
 #pragma unroll
         for (int k = 0; k < (kBlockChunks + kTcThreads - 1) / kTcThreads; k++) {
             const int i = tid + kTcThreads * k;
             if (i >= kBlockChunks)
                 break;
             const int pg = i / kChunksPerPage, c = i - pg * kChunksPerPage;
-            const int32_t id = pg == 0 ? pid[0] : pg == 1 ? pid[1] : pg == 2 ? pid[2] : pid[3];
+            const int32_t id = pid[pg];
             if (id < 0)
                 continue;
             const int64_t ph = static_cast<int64_t>(id) * p.hkv + h;
             const uint8_t *src = c < 128 ? p.codes + ph * (2 * kPageSize * kRowBytes) + c * 16
                                          : p.scales + ph * (2 * kPageSize * 4) + (c - 128) * 16;
-            cp_async16(dst0 + pg * kTcPageBytes + c * 16, src);
+            cp_async16(sbase + kSmCodes + pg * kTcPageBytes + c * 16, src);
         }
         cp_async_commit();
     };
-    int32_t pid_a[kTcBlockPages], pid_b[kTcBlockPages];
-    {
-        int32_t pid0[kTcBlockPages];
-#pragma unroll
-        for (int i = 0; i < kTcBlockPages; i++) {
-            pid0[i] = page_id(i);
-            pid_a[i] = page_id(kTcBlockPages + i);
-            pid_b[i] = page_id(2 * kTcBlockPages + i);
-        }
-        stage_block(0, pid0);
+    if (tid < kTcBlockPages) {
+        store_id(0, raw_id(tid));
+        store_id(1, raw_id(kTcBlockPages + tid));
+        store_id(2, raw_id(2 * kTcBlockPages + tid));
     }
+    __syncthreads();
+    stage_block(0);
+    int32_t praw = tid < kTcBlockPages ? raw_id(3 * kTcBlockPages + tid) : 0;   // ids of block 3
+
+    // ---- unpacking a staged block: exact fp16 integer codes ((0x6400 | n) - 1024), 128B swizzle --
+    // K rows (0-15) and V rows (16-31) of the 4 pages: 1024 words each, 4 per thread
+    auto unpack_rows = [&](uint32_t tile, int row_off) {
+        const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int w = tid + kTcThreads * i;
+            const int pg = w >> 8, qw = w & 255, r = qw >> 4, c4 = qw & 15;
+            const uint32_t word = lds32(sbase + kSmCodes + pg * kTcPageBytes + (row_off + r) * 64 + c4 * 4);
+            const int tok = pg * kPageSize + r;
+            const uint32_t y0 = half2_as_u32(__hsub2(u32_as_half2((word & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y1 = half2_as_u32(__hsub2(u32_as_half2(((word >> 4) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y2 = half2_as_u32(__hsub2(u32_as_half2(((word >> 8) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t y3 = half2_as_u32(__hsub2(u32_as_half2(((word >> 12) & 0x000F000Fu) | 0x64006400u), k1024));
+            const uint32_t dst = tile + sw128_chunk(tok, c4, kTcBlockTokens * 128);
+            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2),
+                         "r"(y3) : "memory");
+        }
+    };
+    // the block's token factors into scale set `set`: kpar[j / 2] = (scale_j, scale_j+1, zero_j,
+    // zero_j+1) of K (logit = (scale acc + zero sq) / 2^8), vpar likewise for V (P' = 2^4 p scale)
+    auto unpack_scales = [&](int kb_, int set) {
+        if (tid < 2 * kTcBlockTokens) {
+            const int pg = tid >> 5, sel = (tid >> 4) & 1, tk = pg * kPageSize + (tid & 15);
+            float2 sz = __half22float2(u32_as_half2(lds32(sbase + kSmCodes + pg * kTcPageBytes +
+                                                          2 * kPageSize * kRowBytes + sel * 64 + (tid & 15) * 4)));
+            if (kb_ * kTcBlockTokens + tk >= n_kv)
+                sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
+            float *par = reinterpret_cast<float *>(smem + kSmScales + set * kSmScaleSet) +
+                         sel * 2 * kTcBlockTokens + 4 * (tk >> 1) + (tk & 1);
+            par[0] = sel == 0 ? sz.x * (1.0f / kTcQScale) : sz.x * kTcPScale;
+            par[2] = sel == 0 ? sz.y * (1.0f / kTcQScale) : sz.y;
+        }
+    };
 
     // ---- the query tile: rotate, scale, fp16, in the codes' d order --------------------------------
     // This thread's half of d: the cross-half Hadamard stage (d, d + 64) first, from the whole
@@ -395,102 +435,83 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         xchg[hf * kTcRows + row] = sq_half;
     }
 
-    // ---- tensor-memory base, the row's sum of q, per-row softmax state ------------------------------
-    async_proxy_fence();   // the Q tile is read by the tensor cores
+
+    // ---- block 0: its pages, the Q tile and the query sums are in; unpack, issue S = Q K^T --------
+    auto issue_qk = [&](uint32_t tmem_, int kb_) {   // S of block kb_ into columns 128 + 64 (kb_ mod 2)
+        tc_fence_after();
+        constexpr uint32_t id_qk = umma_idesc(kTcRows, kTcBlockTokens, 0, 0);
+#pragma unroll
+        for (int ks = 0; ks < 8; ks++) {
+            const uint32_t oq = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
+            const uint32_t ok_ = (ks >> 2) * (kTcBlockTokens * 128) + (ks & 3) * 32;
+            umma_f16(tmem_ + 128 + 64 * (kb_ & 1), umma_desc(sbase + kSmQ + oq, 16, 1024),
+                     umma_desc(sbase + kSmK + ok_, 16, 1024), id_qk, ks > 0);
+        }
+        umma_commit(bar_s0 + 8 * (kb_ & 1));
+    };
+    asm volatile("cp.async.wait_all;" ::: "memory");
+    __syncthreads();
+    unpack_rows(sbase + kSmK, 0);
+    unpack_rows(sbase + kSmV, kPageSize);
+    unpack_scales(0, 0);
+    async_proxy_fence();   // the Q, K and V tiles are read by the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
+    if (tid == 0)
+        issue_qk(tmem, 0);
+    if (n_blocks > 1)
+        stage_block(1);
     const float sq = xchg[row] + xchg[kTcRows + row];
     float m_ref = -INFINITY;
     uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;   // this half's partial sums (two lanes each)
     bool aborted = false;
     int kb = 0;
 
+    // Iteration kb: (1) prepare block kb + 1 -- unpack its K (the K tile is free once S of block
+    // kb is done), its V into the other V tile (free once P V of block kb - 1 is done) and its
+    // scales, issue its S = Q K^T, stage block kb + 2; (2) the softmax of block kb from S in
+    // tensor memory, and O += P' V of block kb.  The tensor cores compute S of block kb + 1 while
+    // the threads run the softmax of block kb, and P V of block kb while they unpack block kb + 2.
     for (; kb < n_blocks; kb++) {
-        // stage block kb + 1 (ids loaded a block ago) and load the ids of block kb + 3
-        if (kb + 1 < n_blocks)
-            stage_block(kb + 1, pid_a);
-        else
-            cp_async_commit();
-#pragma unroll
-        for (int i = 0; i < kTcBlockPages; i++) {
-            pid_a[i] = pid_b[i];
-            pid_b[i] = page_id(kTcBlockPages * (kb + 3) + i);
-        }
-        cp_async_wait1();   // this thread's copies of block kb have landed
-        // the previous block's P V has finished with the V and P tiles
-        bool ok = kb == 0 || mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs);
+        const bool next = kb + 1 < n_blocks;
+        bool ok = mbar_wait_bounded(bar_s0 + 8 * (kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, kTcWaitLimitNs);
+        if (next)
+            asm volatile("cp.async.wait_all;" ::: "memory");   // block kb + 1's pages have landed
         if (!__syncthreads_and(ok)) {
             aborted = true;
             break;
         }
-
-        // ---- unpack the 4 pages into the fp16 K and V tiles, and the scales ------------------
-        // 4 pages x 32 code rows (16 K, 16 V) x 16 words: 8 words per thread
-        const uint32_t stage = sbase + kSmCodes + (kb & 1) * kTcBlockPages * kTcPageBytes;
-#pragma unroll
-        for (int i = 0; i < 8; i++) {
-            const int w = tid + kTcThreads * i;
-            const int pg = w >> 9, qw = w & 511, r = qw >> 4, c4 = qw & 15;
-            const uint32_t word = lds32(stage + pg * kTcPageBytes + r * 64 + c4 * 4);
-            const int tok = pg * kPageSize + (r & 15);
-            // exact fp16 integers: (0x6400 | n) is 1024 + n, minus 1024
-            const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
-            const uint32_t y0 = half2_as_u32(__hsub2(u32_as_half2((word & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y1 = half2_as_u32(__hsub2(u32_as_half2(((word >> 4) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y2 = half2_as_u32(__hsub2(u32_as_half2(((word >> 8) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y3 = half2_as_u32(__hsub2(u32_as_half2(((word >> 12) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t dst = sbase + (r < 16 ? kSmK : kSmV) + sw128_chunk(tok, c4, kTcBlockTokens * 128);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2),
-                         "r"(y3) : "memory");
+        if (next) {
+            unpack_rows(sbase + kSmK, 0);
+            unpack_scales(kb + 1, (kb + 1) & 1);
         }
-        if (tid < 2 * kTcBlockTokens) {
-            const int pg = tid >> 5, sel = (tid >> 4) & 1, tk = pg * kPageSize + (tid & 15);
-            float2 sz = __half22float2(u32_as_half2(lds32(stage + pg * kTcPageBytes + 2 * kPageSize * kRowBytes +
-                                                          sel * 64 + (tid & 15) * 4)));
-            if (kb * kTcBlockTokens + tk >= n_kv)
-                sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
-            float *par = (sel == 0 ? kpar : vpar) + 4 * (tk >> 1) + (tk & 1);
-            if (sel == 0) {   // logit = (scale acc + zero sq) / 2^8 (the query's scale)
-                par[0] = sz.x * (1.0f / kTcQScale);
-                par[2] = sz.y * (1.0f / kTcQScale);
-            } else {          // P' = 2^4 p scale
-                par[0] = sz.x * kTcPScale;
-                par[2] = sz.y;
-            }
-        }
+        ok = kb == 0 || mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs);
+        if (next && ok)
+            unpack_rows(sbase + kSmV + ((kb + 1) & 1) * kSmVTile, kPageSize);
         async_proxy_fence();
         tc_fence_before();
-        __syncthreads();
-
-        // ---- S = Q K^T into tensor-memory columns 128 .. 191 ----------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id_qk = umma_idesc(kTcRows, kTcBlockTokens, 0, 0);
-#pragma unroll
-            for (int ks = 0; ks < 8; ks++) {
-                const uint32_t oq = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
-                const uint32_t ok_ = (ks >> 2) * (kTcBlockTokens * 128) + (ks & 3) * 32;
-                umma_f16(tmem + 128, umma_desc(sbase + kSmQ + oq, 16, 1024),
-                         umma_desc(sbase + kSmK + ok_, 16, 1024), id_qk, ks > 0);
-            }
-            umma_commit(bar_s);
-        }
-        ok = mbar_wait_bounded(bar_s, static_cast<uint32_t>(kb) & 1u, kTcWaitLimitNs);
         if (!__syncthreads_and(ok)) {
             aborted = true;
             break;
+        }
+        if (next) {
+            if (tid == 0)
+                issue_qk(tmem, kb + 1);
+            if (kb + 2 < n_blocks)
+                stage_block(kb + 2);
         }
         tc_fence_after();
         float sv[32];   // tokens 32 hf .. 32 hf + 31 of the block
-        tmem_ld32(lane_base + 128 + 32 * hf, sv);
+        tmem_ld32(lane_base + 128 + 64 * (kb & 1) + 32 * hf, sv);
 
         // ---- online softmax: this half of the row, one shared maximum ---------------------------
         const int tok0 = kb * kTcBlockTokens + 32 * hf;
+        const float *kpar = reinterpret_cast<const float *>(smem + kSmScales + (kb & 1) * kSmScaleSet);
         const float4 *kp4 = reinterpret_cast<const float4 *>(kpar) + 16 * hf;
-        const float4 *vp4 = reinterpret_cast<const float4 *>(vpar) + 16 * hf;
+        const float4 *vp4 = reinterpret_cast<const float4 *>(kpar + 2 * kTcBlockTokens) + 16 * hf;
         const uint64_t sq2 = f2_pack(sq, sq);
 #pragma unroll
         for (int j = 0; j < 32; j += 2) {
@@ -515,6 +536,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         xchg[2 * kTcRows + hf * kTcRows + row] = mb;
         __syncthreads();
         mb = fmaxf(mb, xchg[2 * kTcRows + (1 - hf) * kTcRows + row]);
+        if (tid < kTcBlockPages) {   // the ids of block kb + 3 (loaded a block ago) into the ring
+            store_id(kb + 3, praw);
+            praw = raw_id(kTcBlockPages * (kb + 4) + tid);
+        }
         const bool grow = mb > m_ref + kTcRescale;
         float alpha = 1.0f;
         if (grow) {
@@ -569,7 +594,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 #pragma unroll
             for (int ks = 0; ks < 4; ks++)
                 umma_f16(tmem, umma_desc(sbase + kSmP + ks * 32, 16, 1024),
-                         umma_desc(sbase + kSmV + ks * 2048, kTcBlockTokens * 128, 1024), id_pv,
+                         umma_desc(sbase + kSmV + (kb & 1) * kSmVTile + ks * 2048, kTcBlockTokens * 128, 1024), id_pv,
                          kb > 0 || ks > 0);
             umma_commit(bar_o);
         }
@@ -585,9 +610,14 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
         asm volatile("cp.async.wait_all;" ::: "memory");
         // let MMAs that may still be in flight finish before the tensor memory is released
-        mbar_wait_bounded(bar_s, static_cast<uint32_t>(kb) & 1u, kTcWaitLimitNs / 10);
-        if (kb > 0)
+        // (S of blocks kb and kb - 1, P V of block kb - 1: the last ones issued)
+        if (kb < n_blocks)
+            mbar_wait_bounded(bar_s0 + 8 * (kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, kTcWaitLimitNs / 10);
+        if (kb > 0) {
+            mbar_wait_bounded(bar_s0 + 8 * ((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u,
+                              kTcWaitLimitNs / 10);
             mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs / 10);
+        }
     } else {
         tc_fence_after();
         // this half's 64 O columns = d in [64 hf, 64 hf + 64) (the d order permutes within 8)
