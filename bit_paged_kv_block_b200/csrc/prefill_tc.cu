@@ -55,7 +55,6 @@ constexpr int kTcThreads = 256;
 constexpr int kTcRows = 128;                 // M of the MMAs: query rows per tile
 constexpr int kTcBlockTokens = 64;           // N of QK, K of PV: cache tokens per block
 constexpr int kTcBlockPages = kTcBlockTokens / kPageSize;
-constexpr int kTcPageBytes = 2 * kPageSize * kRowBytes + 2 * kPageSize * 4;   // codes + scales
 constexpr float kTcHadamardC = 0.0883883461356163f;
 constexpr float kTcRescale = 0.0f;           // move the running max whenever a block exceeds it
 constexpr float kTcQScale = 256.0f;          // query entries enter the MMA scaled by 2^8
@@ -67,14 +66,12 @@ constexpr int kSmQ = 0;                                  // Q tile: 2 x [128 row
 constexpr int kSmK = kSmQ + 2 * kTcRows * 128;           // K tile: 2 x [64 tokens][128 B]
 constexpr int kSmV = kSmK + 2 * kTcBlockTokens * 128;    // 2 V tiles: 2 x [64 tokens][128 B] each
 constexpr int kSmVTile = 2 * kTcBlockTokens * 128;
-constexpr int kSmP = kSmV + 2 * kSmVTile;                // P tile: [128 rows][128 B]
-constexpr int kSmCodes = kSmP + kTcRows * 128;           // one block's 4 pages (codes, scales)
-constexpr int kSmScales = kSmCodes + kTcBlockPages * kTcPageBytes;   // 2 x (K, V) token-pair factors
+constexpr int kSmP = kSmV + 2 * kSmVTile;                // P' tile: [128 rows][128 B]
+constexpr int kSmScales = kSmP + kTcRows * 128;          // 4 x (K, V) token-pair factors
 constexpr int kSmScaleSet = 2 * 2 * kTcBlockTokens * 4;
-constexpr int kSmXchg = kSmScales + 2 * kSmScaleSet;     // [4][128] fp32 between row halves
-constexpr int kSmPid = kSmXchg + 4 * kTcRows * 4;        // page ids of 4 blocks (ring)
-constexpr int kSmBars = kSmPid + 4 * kTcBlockPages * 4;  // 2 mbarriers + tmem addr
-constexpr int kSmTile = kSmBars + 32;                    // tile descriptor
+constexpr int kSmXchg = kSmScales + 4 * kSmScaleSet;     // [4][128] fp32 between row halves
+constexpr int kSmBars = kSmXchg + 4 * kTcRows * 4;       // 12 mbarriers, tmem addr, flags
+constexpr int kSmTile = kSmBars + 128;                   // tile descriptor
 constexpr int kSmBytes = kSmTile + 64;
 constexpr size_t kTcSmemBytes = 1024 + kSmBytes;
 constexpr uint32_t kTmemCols = 256;                      // O: columns 0..127, S: 128..255 (2 x 64)
@@ -142,6 +139,65 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
         v[i] = __uint_as_float(r[i]);
 }
 
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16])
+{
+    uint32_t r[16];
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+#pragma unroll
+    for (int i = 0; i < 16; i++)
+        v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float v[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                   "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                   "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+                   "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+                   "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+                   "r"(__float_as_uint(v[15]))
+                 : "memory");
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// 16 consecutive fp32 columns of this thread's lane, without waiting (tmem_wait_ld before use)
+__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, float v[16])
+{
+    uint32_t *r = reinterpret_cast<uint32_t *>(v);
+    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
+                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
+                 : "r"(taddr));
+}
+// waits for this thread's tensor-memory loads; the 32 registers of `v` are tied to the wait so
+// that no use moves above it
+__device__ __forceinline__ void tmem_wait_ld32(float v[32])
+{
+    uint32_t *r = reinterpret_cast<uint32_t *>(v);
+    asm volatile("tcgen05.wait::ld.sync.aligned;"
+                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
+                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
+                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
+                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
+                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
+                 :: "memory");
+}
+__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const float v[16])
+{
+    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
+                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
+                   "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
+                   "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
+                   "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
+                   "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
+                   "r"(__float_as_uint(v[15]))
+                 : "memory");
+}
+
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float v[32])
 {
     asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
@@ -160,12 +216,6 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float v[32])
                  : "memory");
     asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void *src)
-{
-    asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(dst), "l"(src) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 
 // d order of the 8 entries of a 16-byte chunk: position j holds d = 8 a + kPerm[j]
 __host__ __device__ constexpr int chunk_d(int j) { return (j >> 1) + ((j & 1) << 2); }
@@ -239,10 +289,72 @@ __device__ bool find_tile(const TcParams &p, int cta, int &s_out, int &h_out, in
     return true;
 }
 
-// Thread layout: 8 warps; warp w owns the 32 tile rows of tensor-memory lanes 32 (w mod 4) ..
-// (its lane quarter) and the half hf = w / 4 of each block's 64 tokens and of O's 128 columns.
-// The two threads of a row exchange only the block maximum (and, once, the sums of the query and
-// the final l, z and the last Hadamard stage) through shared memory.
+__device__ __forceinline__ void tc_arrive(uint32_t bar)
+{
+    asm volatile("mbarrier.arrive.release.cta.shared::cta.b64 _, [%0];" ::"r"(bar) : "memory");
+}
+
+// Bounded wait on phase `parity` of an mbarrier that also gives up once the other role has
+// (the shared abort flag); a timeout raises the flag.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t parity, volatile int *abort_flag)
+{
+    if (mbar_try_wait(bar, parity))
+        return true;
+    const uint64_t t0 = globaltimer_ns();
+    while (true) {
+        if (mbar_try_wait(bar, parity))
+            return true;
+        if (*abort_flag != 0)
+            return false;
+        if (globaltimer_ns() - t0 > kTcWaitLimitNs) {
+            *abort_flag = 1;
+            return false;
+        }
+    }
+}
+
+// Named barrier of one role (128 threads: barrier 1 the producers, 2 the softmax warps) that
+// also ANDs a flag over them, so that the role leaves its loop as one.
+__device__ __forceinline__ bool role_bar_and(int id, bool v)
+{
+    uint32_t r;
+    asm volatile("{\n\t.reg .pred p, q;\n\tsetp.ne.u32 p, %1, 0;\n\t"
+                 "bar.red.and.pred q, %2, %3, p;\n\tselp.u32 %0, 1, 0, q;\n\t}"
+                 : "=r"(r)
+                 : "r"(static_cast<uint32_t>(v)), "r"(id), "r"(kTcThreads / 2)
+                 : "memory");
+    return r != 0;
+}
+
+__device__ __forceinline__ uint4 ldg_nc16(const void *p)
+{
+    uint4 r;
+    asm volatile("ld.global.nc.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w)
+                 : "l"(p));
+    return r;
+}
+
+// four fp16 pairs of the 8 codes of a 32-bit word as exact integers ((0x6400 | n) - 1024), stored
+// as one 16-byte chunk of an fp16 tile
+__device__ __forceinline__ void unpack_word_store(uint32_t dst, uint32_t word)
+{
+    const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
+    const uint32_t y0 = half2_as_u32(__hsub2(u32_as_half2((word & 0x000F000Fu) | 0x64006400u), k1024));
+    const uint32_t y1 = half2_as_u32(__hsub2(u32_as_half2(((word >> 4) & 0x000F000Fu) | 0x64006400u), k1024));
+    const uint32_t y2 = half2_as_u32(__hsub2(u32_as_half2(((word >> 8) & 0x000F000Fu) | 0x64006400u), k1024));
+    const uint32_t y3 = half2_as_u32(__hsub2(u32_as_half2(((word >> 12) & 0x000F000Fu) | 0x64006400u), k1024));
+    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+                 : "memory");
+}
+
+// Roles: warps 0-3 run the softmax, one query row per thread (row = thread = tensor-memory lane);
+// warps 4-7 are the producers: they load the pages of each block straight into registers (two
+// blocks ahead), unpack K and V into the fp16 tiles and write the scale table, and one of them
+// issues S = Q K^T.  Thread 0 issues O += P' V once the softmax warps have written P'.  The roles
+// hand off through mbarriers (the tensor cores' commits included) and two named barriers, one per
+// role, so neither waits for the other except where the data requires it.  Every wait is bounded;
+// a timeout sets the status bit and a shared abort flag that ends the other role's waits too.
 template <bool kRotate>
 __global__ void __launch_bounds__(kTcThreads, 2)
     prefill_tc_kernel(const TcParams p)
@@ -250,14 +362,24 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-    const int hf = warp >> 2;                             // token / column half
+    const int hf = warp >> 2;                             // prologue / epilogue: column half
     const int row = 32 * (warp & 3) + lane;               // tile row = tensor-memory lane
     const uint32_t sbase = smem_u32(smem);
     int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
-    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 24);
-    // S of even / odd blocks (bar_s0, bar_s0 + 8), O += P V (bar_o)
-    const uint32_t bar_s0 = sbase + kSmBars, bar_o = sbase + kSmBars + 16;
-    float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [2 halves][128 rows] x 4
+    float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [4][128] fp32 between row halves
+    const uint32_t bars = sbase + kSmBars;
+    // bar_s[b]: S of blocks b, b + 2, ... done (tensor-core commit); bar_sfree[b]: the softmax has
+    // read that S buffer (one arrival per softmax warp); bar_o[b]: P' V of blocks b, b + 2, ... done;
+    // bar_v[b]: V of those blocks unpacked (128 producer arrivals); bar_sc[i]: the scale table of
+    // blocks i, i + 4, ... written (128 producer arrivals)
+    auto bar_s = [&](int b) { return bars + 8 * b; };
+    auto bar_sfree = [&](int b) { return bars + 16 + 8 * b; };
+    auto bar_o = [&](int b) { return bars + 32 + 8 * b; };
+    auto bar_v = [&](int b) { return bars + 48 + 8 * b; };
+    auto bar_sc = [&](int i) { return bars + 64 + 8 * i; };
+    uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmBars + 96);
+    volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmBars + 100);
+    int *issued = reinterpret_cast<int *>(smem + kSmBars + 104);   // [0] S issued, [1] P' V issued
 
     pdl_launch_dependents();
     int s, h, t0;
@@ -282,9 +404,16 @@ __global__ void __launch_bounds__(kTcThreads, 2)
 
     // ---- tensor memory and barriers -----------------------------------------------------------
     if (tid == 0) {
-        mbar_init(bar_s0, 1);
-        mbar_init(bar_s0 + 8, 1);
-        mbar_init(bar_o, 1);
+        for (int b = 0; b < 2; b++) {
+            mbar_init(bar_s(b), 1);
+            mbar_init(bar_sfree(b), 4);
+            mbar_init(bar_o(b), 1);
+            mbar_init(bar_v(b), kTcThreads / 2);
+        }
+        for (int i = 0; i < 4; i++)
+            mbar_init(bar_sc(i), kTcThreads / 2);
+        *abort_flag = 0;
+        issued[0] = issued[1] = 0;
     }
     mbar_init_fence();
     if (warp == 0) {
@@ -294,88 +423,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
 
     pdl_wait();   // the cache may be written by the kernel this one depends on
-
-    // ---- page ids: threads 0-3 load a block's 4 ids three blocks ahead and check them into a
-    //      shared ring of 4 blocks half an iteration later, so the loads never stall the loop ------
-    int32_t *pid_ring = reinterpret_cast<int32_t *>(smem + kSmPid);
-    const int64_t bt_row = static_cast<int64_t>(s) * p.max_blocks;
-    auto raw_id = [&](int pg) -> int32_t {
-        return pg < n_pages ? p.block_table[bt_row + pg] : -1;   // -1: past the tile's range
-    };
-    auto store_id = [&](int kb_, int32_t id) {   // thread tid < 4: page 4 kb_ + tid
-        const int pg = kTcBlockPages * kb_ + tid;
-        if (pg < n_pages && (id < 0 || id >= p.num_pages)) {
-            set_status(p.status, SAW_DEV_BAD_PAGE);
-            id = 0;
-        }
-        pid_ring[(kb_ & 3) * kTcBlockPages + tid] = id;
-    };
-    // ---- staging of a block's 4 pages (codes, then scales) by cp.async into the code stage ----
-    // this thread's 16-byte chunks are i = tid + 256 k (i < 544): page i / 136, chunk i mod 136
-    // (128 of codes, 8 of scales)
-    constexpr int kChunksPerPage = kTcPageBytes / 16;
-    constexpr int kBlockChunks = kTcBlockPages * kChunksPerPage;
-    auto stage_block = [&](int kb_) {
-        const int32_t *pid = pid_ring + (kb_ & 3) * kTcBlockPages;
-#pragma unroll
-        for (int k = 0; k < (kBlockChunks + kTcThreads - 1) / kTcThreads; k++) {
-            const int i = tid + kTcThreads * k;
-            if (i >= kBlockChunks)
-                break;
-            const int pg = i / kChunksPerPage, c = i - pg * kChunksPerPage;
-            const int32_t id = pid[pg];
-            if (id < 0)
-                continue;
-            const int64_t ph = static_cast<int64_t>(id) * p.hkv + h;
-            const uint8_t *src = c < 128 ? p.codes + ph * (2 * kPageSize * kRowBytes) + c * 16
-                                         : p.scales + ph * (2 * kPageSize * 4) + (c - 128) * 16;
-            cp_async16(sbase + kSmCodes + pg * kTcPageBytes + c * 16, src);
-        }
-        cp_async_commit();
-    };
-    if (tid < kTcBlockPages) {
-        store_id(0, raw_id(tid));
-        store_id(1, raw_id(kTcBlockPages + tid));
-        store_id(2, raw_id(2 * kTcBlockPages + tid));
-    }
-    __syncthreads();
-    stage_block(0);
-    int32_t praw = tid < kTcBlockPages ? raw_id(3 * kTcBlockPages + tid) : 0;   // ids of block 3
-
-    // ---- unpacking a staged block: exact fp16 integer codes ((0x6400 | n) - 1024), 128B swizzle --
-    // K rows (0-15) and V rows (16-31) of the 4 pages: 1024 words each, 4 per thread
-    auto unpack_rows = [&](uint32_t tile, int row_off) {
-        const __half2 k1024 = __halves2half2(__ushort_as_half(0x6400), __ushort_as_half(0x6400));
-#pragma unroll
-        for (int i = 0; i < 4; i++) {
-            const int w = tid + kTcThreads * i;
-            const int pg = w >> 8, qw = w & 255, r = qw >> 4, c4 = qw & 15;
-            const uint32_t word = lds32(sbase + kSmCodes + pg * kTcPageBytes + (row_off + r) * 64 + c4 * 4);
-            const int tok = pg * kPageSize + r;
-            const uint32_t y0 = half2_as_u32(__hsub2(u32_as_half2((word & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y1 = half2_as_u32(__hsub2(u32_as_half2(((word >> 4) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y2 = half2_as_u32(__hsub2(u32_as_half2(((word >> 8) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t y3 = half2_as_u32(__hsub2(u32_as_half2(((word >> 12) & 0x000F000Fu) | 0x64006400u), k1024));
-            const uint32_t dst = tile + sw128_chunk(tok, c4, kTcBlockTokens * 128);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(dst), "r"(y0), "r"(y1), "r"(y2),
-                         "r"(y3) : "memory");
-        }
-    };
-    // the block's token factors into scale set `set`: kpar[j / 2] = (scale_j, scale_j+1, zero_j,
-    // zero_j+1) of K (logit = (scale acc + zero sq) / 2^8), vpar likewise for V (P' = 2^4 p scale)
-    auto unpack_scales = [&](int kb_, int set) {
-        if (tid < 2 * kTcBlockTokens) {
-            const int pg = tid >> 5, sel = (tid >> 4) & 1, tk = pg * kPageSize + (tid & 15);
-            float2 sz = __half22float2(u32_as_half2(lds32(sbase + kSmCodes + pg * kTcPageBytes +
-                                                          2 * kPageSize * kRowBytes + sel * 64 + (tid & 15) * 4)));
-            if (kb_ * kTcBlockTokens + tk >= n_kv)
-                sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
-            float *par = reinterpret_cast<float *>(smem + kSmScales + set * kSmScaleSet) +
-                         sel * 2 * kTcBlockTokens + 4 * (tk >> 1) + (tk & 1);
-            par[0] = sel == 0 ? sz.x * (1.0f / kTcQScale) : sz.x * kTcPScale;
-            par[2] = sel == 0 ? sz.y * (1.0f / kTcQScale) : sz.y;
-        }
-    };
 
     // ---- the query tile: rotate, scale, fp16, in the codes' d order --------------------------------
     // This thread's half of d: the cross-half Hadamard stage (d, d + 64) first, from the whole
@@ -436,187 +483,287 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     }
 
 
-    // ---- block 0: its pages, the Q tile and the query sums are in; unpack, issue S = Q K^T --------
-    auto issue_qk = [&](uint32_t tmem_, int kb_) {   // S of block kb_ into columns 128 + 64 (kb_ mod 2)
-        tc_fence_after();
-        constexpr uint32_t id_qk = umma_idesc(kTcRows, kTcBlockTokens, 0, 0);
-#pragma unroll
-        for (int ks = 0; ks < 8; ks++) {
-            const uint32_t oq = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
-            const uint32_t ok_ = (ks >> 2) * (kTcBlockTokens * 128) + (ks & 3) * 32;
-            umma_f16(tmem_ + 128 + 64 * (kb_ & 1), umma_desc(sbase + kSmQ + oq, 16, 1024),
-                     umma_desc(sbase + kSmK + ok_, 16, 1024), id_qk, ks > 0);
-        }
-        umma_commit(bar_s0 + 8 * (kb_ & 1));
-    };
-    asm volatile("cp.async.wait_all;" ::: "memory");
-    __syncthreads();
-    unpack_rows(sbase + kSmK, 0);
-    unpack_rows(sbase + kSmV, kPageSize);
-    unpack_scales(0, 0);
-    async_proxy_fence();   // the Q, K and V tiles are read by the tensor cores
+
+    // ---- tensor-memory base; the roles split here ----------------------------------------------
+    async_proxy_fence();   // the Q tile is read by the tensor cores
     tc_fence_before();
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-    if (tid == 0)
-        issue_qk(tmem, 0);
-    if (n_blocks > 1)
-        stage_block(1);
-    const float sq = xchg[row] + xchg[kTcRows + row];
-    float m_ref = -INFINITY;
-    uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;   // this half's partial sums (two lanes each)
-    bool aborted = false;
-    int kb = 0;
+    float l_row = 0.0f, z_row = 0.0f;   // softmax threads: the row's sums over all blocks
 
-    // Iteration kb: (1) prepare block kb + 1 -- unpack its K (the K tile is free once S of block
-    // kb is done), its V into the other V tile (free once P V of block kb - 1 is done) and its
-    // scales, issue its S = Q K^T, stage block kb + 2; (2) the softmax of block kb from S in
-    // tensor memory, and O += P' V of block kb.  The tensor cores compute S of block kb + 1 while
-    // the threads run the softmax of block kb, and P V of block kb while they unpack block kb + 2.
-    for (; kb < n_blocks; kb++) {
-        const bool next = kb + 1 < n_blocks;
-        bool ok = mbar_wait_bounded(bar_s0 + 8 * (kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, kTcWaitLimitNs);
-        if (next)
-            asm volatile("cp.async.wait_all;" ::: "memory");   // block kb + 1's pages have landed
-        if (!__syncthreads_and(ok)) {
-            aborted = true;
-            break;
-        }
-        if (next) {
-            unpack_rows(sbase + kSmK, 0);
-            unpack_scales(kb + 1, (kb + 1) & 1);
-        }
-        ok = kb == 0 || mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs);
-        if (next && ok)
-            unpack_rows(sbase + kSmV + ((kb + 1) & 1) * kSmVTile, kPageSize);
-        async_proxy_fence();
-        tc_fence_before();
-        if (!__syncthreads_and(ok)) {
-            aborted = true;
-            break;
-        }
-        if (next) {
-            if (tid == 0)
-                issue_qk(tmem, kb + 1);
+    if (warp >= 4) {
+        // ======== producers: pages -> registers (two blocks ahead) -> fp16 K / V tiles, scales ====
+        // Thread pt holds, of each block, the 16-byte quarter q4 of token rk's K and V rows in
+        // pages pgk and pgk + 2 (4 code words each), and the (scale, zero) pair `sel` of token tks
+        // of page pgs.
+        const int pt = tid - kTcThreads / 2;
+        const int pgk = pt >> 6, rk = (pt & 63) >> 2, q4 = pt & 3;
+        const int pgs = pt >> 5, sel = (pt >> 4) & 1, tks = pt & 15;
+        const int32_t *bt = p.block_table + static_cast<int64_t>(s) * p.max_blocks;
+        auto raw_id = [&](int pg) -> int32_t { return pg < n_pages ? __ldg(bt + pg) : -1; };
+        auto checked = [&](int pg, int32_t id) -> int32_t {   // -1 past the tile's range
+            if (pg < n_pages && (id < 0 || id >= p.num_pages)) {
+                set_status(p.status, SAW_DEV_BAD_PAGE);
+                return 0;
+            }
+            return id;
+        };
+        struct Words {
+            uint4 k0, k1, v0, v1;   // pages pgk, pgk + 2
+            uint32_t sc;
+        };
+        auto fetch = [&](int b, int32_t ia, int32_t ib, int32_t is) -> Words {
+            Words w;
+            const uint4 zero4 = make_uint4(0u, 0u, 0u, 0u);
+            ia = checked(kTcBlockPages * b + pgk, ia);
+            ib = checked(kTcBlockPages * b + pgk + 2, ib);
+            is = checked(kTcBlockPages * b + pgs, is);
+            const int off = rk * kRowBytes + q4 * 16;
+            const uint8_t *a = p.codes + (static_cast<int64_t>(ia) * p.hkv + h) * (2 * kPageSize * kRowBytes) + off;
+            const uint8_t *c = p.codes + (static_cast<int64_t>(ib) * p.hkv + h) * (2 * kPageSize * kRowBytes) + off;
+            w.k0 = ia >= 0 ? ldg_nc16(a) : zero4;
+            w.v0 = ia >= 0 ? ldg_nc16(a + kPageSize * kRowBytes) : zero4;
+            w.k1 = ib >= 0 ? ldg_nc16(c) : zero4;
+            w.v1 = ib >= 0 ? ldg_nc16(c + kPageSize * kRowBytes) : zero4;
+            w.sc = is >= 0 ? __ldg(reinterpret_cast<const uint32_t *>(
+                                 p.scales + (static_cast<int64_t>(is) * p.hkv + h) * (2 * kPageSize * 4) +
+                                 sel * (kPageSize * 4) + tks * 4))
+                           : 0u;
+            return w;
+        };
+        // S = Q K^T of block kb_ into S buffer kb_ mod 2
+        auto issue_qk = [&](int kb_) {
+            constexpr uint32_t id_qk = umma_idesc(kTcRows, kTcBlockTokens, 0, 0);
+#pragma unroll
+            for (int ks = 0; ks < 8; ks++) {
+                const uint32_t oq = (ks >> 2) * (kTcRows * 128) + (ks & 3) * 32;
+                const uint32_t ok_ = (ks >> 2) * (kTcBlockTokens * 128) + (ks & 3) * 32;
+                umma_f16(tmem + 128 + 64 * (kb_ & 1), umma_desc(sbase + kSmQ + oq, 16, 1024),
+                         umma_desc(sbase + kSmK + ok_, 16, 1024), id_qk, ks > 0);
+            }
+            umma_commit(bar_s(kb_ & 1));
+        };
+        // this thread's four fp16 chunks of a token row in a K or V tile (128-byte swizzle)
+        const int tk0 = pgk * kPageSize + rk, tk1 = (pgk + 2) * kPageSize + rk;
+        auto unpack4 = [&](uint32_t tile, int tok, const uint4 &w) {
+            unpack_word_store(tile + sw128_chunk(tok, 4 * q4 + 0, kTcBlockTokens * 128), w.x);
+            unpack_word_store(tile + sw128_chunk(tok, 4 * q4 + 1, kTcBlockTokens * 128), w.y);
+            unpack_word_store(tile + sw128_chunk(tok, 4 * q4 + 2, kTcBlockTokens * 128), w.z);
+            unpack_word_store(tile + sw128_chunk(tok, 4 * q4 + 3, kTcBlockTokens * 128), w.w);
+        };
+
+        int32_t ra = raw_id(pgk), rb = raw_id(pgk + 2), rs = raw_id(pgs);
+        Words w0 = fetch(0, ra, rb, rs);
+        ra = raw_id(kTcBlockPages + pgk), rb = raw_id(kTcBlockPages + pgk + 2), rs = raw_id(kTcBlockPages + pgs);
+        Words w1 = fetch(1, ra, rb, rs);
+        ra = raw_id(2 * kTcBlockPages + pgk), rb = raw_id(2 * kTcBlockPages + pgk + 2);
+        rs = raw_id(2 * kTcBlockPages + pgs);
+        bool ok = true;
+        for (int kb = 0; kb < n_blocks; kb++) {
+            // the words of block kb + 2 (ids read a block ago) and the ids of block kb + 3
+            Words w2 = {};
             if (kb + 2 < n_blocks)
-                stage_block(kb + 2);
-        }
-        tc_fence_after();
-        float sv[32];   // tokens 32 hf .. 32 hf + 31 of the block
-        tmem_ld32(lane_base + 128 + 64 * (kb & 1) + 32 * hf, sv);
+                w2 = fetch(kb + 2, ra, rb, rs);
+            const int nb = kTcBlockPages * (kb + 3);
+            ra = raw_id(nb + pgk), rb = raw_id(nb + pgk + 2), rs = raw_id(nb + pgs);
 
-        // ---- online softmax: this half of the row, one shared maximum ---------------------------
-        const int tok0 = kb * kTcBlockTokens + 32 * hf;
-        const float *kpar = reinterpret_cast<const float *>(smem + kSmScales + (kb & 1) * kSmScaleSet);
-        const float4 *kp4 = reinterpret_cast<const float4 *>(kpar) + 16 * hf;
-        const float4 *vp4 = reinterpret_cast<const float4 *>(kpar + 2 * kTcBlockTokens) + 16 * hf;
+            // V of block kb into V tile kb mod 2, once P' V of block kb - 2 has read it
+            if (kb >= 2)
+                ok = ok && tc_wait(bar_o(kb & 1), static_cast<uint32_t>((kb - 2) >> 1) & 1u, abort_flag);
+            if (ok) {
+                const uint32_t vt = sbase + kSmV + (kb & 1) * kSmVTile;
+                unpack4(vt, tk0, w0.v0);
+                unpack4(vt, tk1, w0.v1);
+                async_proxy_fence();
+                tc_arrive(bar_v(kb & 1));
+            }
+            // K of block kb and its scale table, once S of block kb - 1 has read the K tile
+            if (kb >= 1)
+                ok = ok && tc_wait(bar_s((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u, abort_flag);
+            if (ok) {
+                unpack4(sbase + kSmK, tk0, w0.k0);
+                unpack4(sbase + kSmK, tk1, w0.k1);
+                const int tk = pgs * kPageSize + tks;
+                float2 sz = __half22float2(u32_as_half2(w0.sc));
+                if (kb * kTcBlockTokens + tk >= n_kv)
+                    sz = make_float2(0.0f, 0.0f);   // past the tile's range: no weight, no NaN
+                float *par = reinterpret_cast<float *>(smem + kSmScales + (kb & 3) * kSmScaleSet) +
+                             sel * 2 * kTcBlockTokens + 4 * (tk >> 1) + (tk & 1);
+                // K: logit = (scale acc + zero sq) / 2^8; V: P' = 2^4 p scale, zero point
+                par[0] = sel == 0 ? sz.x * (1.0f / kTcQScale) : sz.x * kTcPScale;
+                par[2] = sel == 0 ? sz.y * (1.0f / kTcQScale) : sz.y;
+                async_proxy_fence();
+                tc_arrive(bar_sc(kb & 3));
+            }
+            ok = role_bar_and(1, ok);
+            if (!ok)
+                break;
+            if (pt == 0) {
+                // the S buffer of block kb - 2 has been read by the softmax
+                ok = kb < 2 || tc_wait(bar_sfree(kb & 1), static_cast<uint32_t>((kb - 2) >> 1) & 1u, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    issue_qk(kb);
+                    issued[0] = kb + 1;
+                }
+            }
+            w0 = w1;
+            w1 = w2;
+        }
+    } else {
+        // ======== softmax: thread `row` owns one query row over all 64 tokens of each block =======
+        const float sq = xchg[row] + xchg[kTcRows + row];
         const uint64_t sq2 = f2_pack(sq, sq);
+        float m_ref = -INFINITY;
+        uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;   // the row's sums (two lanes each)
+        bool ok = true;
+        for (int kb = 0; kb < n_blocks; kb++) {
+            // S of block kb and its scale table
+            ok = ok && tc_wait(bar_s(kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, abort_flag);
+            ok = ok && tc_wait(bar_sc(kb & 3), static_cast<uint32_t>(kb >> 2) & 1u, abort_flag);
+            ok = __all_sync(0xFFFFFFFFu, ok);   // tensor-memory loads are warp-wide
+            float sv[64];   // the block's 64 logits of this row
+            bool grow = false;
+            float alpha = 1.0f;
+            if (ok) {
+                tc_fence_after();
+                tmem_ld32(lane_base + 128 + 64 * (kb & 1), sv);
+                tmem_ld32(lane_base + 128 + 64 * (kb & 1) + 32, sv + 32);
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0)
+                    tc_arrive(bar_sfree(kb & 1));   // the S buffer may be overwritten
+
+                const float4 *kp4 = reinterpret_cast<const float4 *>(smem + kSmScales + (kb & 3) * kSmScaleSet);
 #pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-            const float4 kp = kp4[j / 2];
-            const uint64_t t = f2_fma(f2_pack(kp.x, kp.y), f2_pack(sv[j], sv[j + 1]),
-                                      f2_mul(f2_pack(kp.z, kp.w), sq2));
-            f2_unpack(t, sv[j], sv[j + 1]);
-        }
-        // the causal limit (and the end of the cache) only reaches the last blocks of a tile
-        if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
+                for (int j = 0; j < 64; j += 2) {
+                    const float4 kp = kp4[j / 2];
+                    const uint64_t t = f2_fma(f2_pack(kp.x, kp.y), f2_pack(sv[j], sv[j + 1]),
+                                              f2_mul(f2_pack(kp.z, kp.w), sq2));
+                    f2_unpack(t, sv[j], sv[j + 1]);
+                }
+                // the causal limit (and the end of the cache) only reaches the last blocks of a tile
+                if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
+                    const int tok0 = kb * kTcBlockTokens;
 #pragma unroll
-            for (int j = 0; j < 32; j++)
-                if (tok0 + j > limit)
-                    sv[j] = -INFINITY;
-        }
-        float mb = -INFINITY;
+                    for (int j = 0; j < 64; j++)
+                        if (tok0 + j > limit)
+                            sv[j] = -INFINITY;
+                }
+                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // 4 short chains
 #pragma unroll
-        for (int j = 0; j < 32; j += 2)
-            mb = fmax3(mb, sv[j], sv[j + 1]);
-        if (!live)
-            mb = -INFINITY;
-        xchg[2 * kTcRows + hf * kTcRows + row] = mb;
-        __syncthreads();
-        mb = fmaxf(mb, xchg[2 * kTcRows + (1 - hf) * kTcRows + row]);
-        if (tid < kTcBlockPages) {   // the ids of block kb + 3 (loaded a block ago) into the ring
-            store_id(kb + 3, praw);
-            praw = raw_id(kTcBlockPages * (kb + 4) + tid);
-        }
-        const bool grow = mb > m_ref + kTcRescale;
-        float alpha = 1.0f;
-        if (grow) {
-            alpha = ex2_approx(m_ref - mb);   // 0 on the first block a row sees
-            const uint64_t a2 = f2_pack(alpha, alpha);
-            l2 = f2_mul(l2, a2);
-            z2 = f2_mul(z2, a2);
-            m_ref = mb;
-        }
-        // rescale this half of the O row in tensor memory (warp-wide instructions; alpha 1 where
-        // no change)
-        if (kb > 0 && __any_sync(0xFFFFFFFFu, grow && alpha != 0.0f)) {
+                for (int j = 0; j < 64; j += 2)
+                    m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], sv[j], sv[j + 1]);
+                float mb = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
+                if (!live)
+                    mb = -INFINITY;
+                grow = mb > m_ref + kTcRescale;
+                if (grow) {
+                    alpha = ex2_approx(m_ref - mb);   // 0 on the first block a row sees
+                    const uint64_t a2 = f2_pack(alpha, alpha);
+                    l2 = f2_mul(l2, a2);
+                    z2 = f2_mul(z2, a2);
+                    m_ref = mb;
+                }
+            }
+            // P' V of block kb - 1 has finished with the P' tile and the O accumulator
+            if (kb >= 1)
+                ok = ok && tc_wait(bar_o((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u, abort_flag);
+            ok = __all_sync(0xFFFFFFFFu, ok);
+            if (ok) {
+                tc_fence_after();
+                // the weights, 8 tokens (one 16-byte chunk of the P' row) at a time
+                const float4 *vp4 = reinterpret_cast<const float4 *>(smem + kSmScales + (kb & 3) * kSmScaleSet) +
+                                    kTcBlockTokens / 2;
+                const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
+                const uint64_t mr2 = f2_pack(mr, mr);
+#pragma unroll
+                for (int c = 0; c < 8; c++) {
+                    uint32_t pw[4];
+#pragma unroll
+                    for (int k = 0; k < 4; k++) {
+                        const int j = 8 * c + 2 * k;
+                        const float4 vp = vp4[j / 2];
+                        float d0, d1;
+                        f2_unpack(f2_sub(f2_pack(sv[j], sv[j + 1]), mr2), d0, d1);
+                        const uint64_t p2 = f2_pack(ex2_approx(d0), ex2_approx(d1));
+                        l2 = f2_add(l2, p2);
+                        z2 = f2_fma(p2, f2_pack(vp.z, vp.w), z2);
+                        float q0, q1;
+                        f2_unpack(f2_mul(p2, f2_pack(vp.x, vp.y)), q0, q1);
+                        pw[k] = half2_as_u32(__floats2half2_rn(q0, q1));
+                    }
+                    const uint32_t a = sbase + kSmP + sw128_chunk(row, c, kTcRows * 128);
+                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pw[0]), "r"(pw[1]),
+                                 "r"(pw[2]), "r"(pw[3]) : "memory");
+                }
+                // rescale the O row in tensor memory (warp-wide; alpha 1 where no change): four
+                // rounds of 32 columns, the stores waited for once
+                if (kb > 0 && __any_sync(0xFFFFFFFFu, grow && alpha != 0.0f)) {
 #pragma unroll 1
-            for (int c = 0; c < 2; c++) {
-                float ov[32];
-                tmem_ld32(lane_base + 64 * hf + 32 * c, ov);
+                    for (int c = 0; c < 4; c++) {
+                        float ov[32];
+                        tmem_ld16_nowait(lane_base + 32 * c, ov);
+                        tmem_ld16_nowait(lane_base + 32 * c + 16, ov + 16);
+                        tmem_wait_ld32(ov);
 #pragma unroll
-                for (int i = 0; i < 32; i++)
-                    ov[i] *= alpha;
-                tmem_st32(lane_base + 64 * hf + 32 * c, ov);
+                        for (int i = 0; i < 32; i += 2) {
+                            const uint64_t r = f2_mul(f2_pack(ov[i], ov[i + 1]), f2_pack(alpha, alpha));
+                            f2_unpack(r, ov[i], ov[i + 1]);
+                        }
+                        tmem_st16_nowait(lane_base + 32 * c, ov);
+                        tmem_st16_nowait(lane_base + 32 * c + 16, ov + 16);
+                    }
+                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                }
+                async_proxy_fence();
+                tc_fence_before();
+            }
+            ok = role_bar_and(2, ok);
+            if (!ok)
+                break;
+            if (tid == 0) {
+                // O += P' V of block kb, once the producers have written V of block kb
+                ok = tc_wait(bar_v(kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, abort_flag);
+                if (ok) {
+                    tc_fence_after();
+                    constexpr uint32_t id_pv = umma_idesc(kTcRows, 128, 0, 1);
+#pragma unroll
+                    for (int ks = 0; ks < 4; ks++)
+                        umma_f16(tmem, umma_desc(sbase + kSmP + ks * 32, 16, 1024),
+                                 umma_desc(sbase + kSmV + (kb & 1) * kSmVTile + ks * 2048,
+                                           kTcBlockTokens * 128, 1024),
+                                 id_pv, kb > 0 || ks > 0);
+                    umma_commit(bar_o(kb & 1));
+                    issued[1] = kb + 1;
+                }
             }
         }
-        uint32_t pw[16];
-        const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
-        const uint64_t mr2 = f2_pack(mr, mr);
-#pragma unroll
-        for (int j = 0; j < 32; j += 2) {
-            const float4 vp = vp4[j / 2];
-            float d0, d1;
-            f2_unpack(f2_sub(f2_pack(sv[j], sv[j + 1]), mr2), d0, d1);
-            const uint64_t p2 = f2_pack(ex2_approx(d0), ex2_approx(d1));
-            l2 = f2_add(l2, p2);
-            z2 = f2_fma(p2, f2_pack(vp.z, vp.w), z2);
-            float w0, w1;
-            f2_unpack(f2_mul(p2, f2_pack(vp.x, vp.y)), w0, w1);
-            pw[j / 2] = half2_as_u32(__floats2half2_rn(w0, w1));
-        }
-#pragma unroll
-        for (int c = 0; c < 4; c++) {
-            const uint32_t a = sbase + kSmP + sw128_chunk(row, 4 * hf + c, kTcRows * 128);
-            asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pw[4 * c]),
-                         "r"(pw[4 * c + 1]), "r"(pw[4 * c + 2]), "r"(pw[4 * c + 3]) : "memory");
-        }
-        async_proxy_fence();
-        tc_fence_before();
-        __syncthreads();
-
-        // ---- O += P' V into tensor-memory columns 0 .. 127 -----------------------------------------
-        if (tid == 0) {
-            tc_fence_after();
-            constexpr uint32_t id_pv = umma_idesc(kTcRows, 128, 0, 1);
-#pragma unroll
-            for (int ks = 0; ks < 4; ks++)
-                umma_f16(tmem, umma_desc(sbase + kSmP + ks * 32, 16, 1024),
-                         umma_desc(sbase + kSmV + (kb & 1) * kSmVTile + ks * 2048, kTcBlockTokens * 128, 1024), id_pv,
-                         kb > 0 || ks > 0);
-            umma_commit(bar_o);
-        }
+        float la, lb, za, zb;
+        f2_unpack(l2, la, lb);
+        f2_unpack(z2, za, zb);
+        l_row = la + lb;
+        z_row = za + zb;
     }
 
     // ---- epilogue: O row -> zero term, 1 / l, the weights' scale, inverse rotation ----------------
-    if (!aborted) {
-        const bool ok = mbar_wait_bounded(bar_o, static_cast<uint32_t>(n_blocks - 1) & 1u, kTcWaitLimitNs);
-        aborted = !__syncthreads_and(ok);
+    __syncthreads();
+    bool fine = *abort_flag == 0;
+    if (fine) {
+        const int last = n_blocks - 1;
+        const bool ok = tc_wait(bar_o(last & 1), static_cast<uint32_t>(last >> 1) & 1u, abort_flag);
+        fine = __syncthreads_and(ok);
     }
-    if (aborted) {
-        if (tid == 0)
+    if (!fine) {
+        if (tid == 0) {
             set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
-        asm volatile("cp.async.wait_all;" ::: "memory");
-        // let MMAs that may still be in flight finish before the tensor memory is released
-        // (S of blocks kb and kb - 1, P V of block kb - 1: the last ones issued)
-        if (kb < n_blocks)
-            mbar_wait_bounded(bar_s0 + 8 * (kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, kTcWaitLimitNs / 10);
-        if (kb > 0) {
-            mbar_wait_bounded(bar_s0 + 8 * ((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u,
-                              kTcWaitLimitNs / 10);
-            mbar_wait_bounded(bar_o, static_cast<uint32_t>(kb - 1) & 1u, kTcWaitLimitNs / 10);
+            // let the MMAs that may still be in flight finish before the tensor memory is released
+            for (int b = max(0, issued[0] - 2); b < issued[0]; b++)
+                mbar_wait_bounded(bar_s(b & 1), static_cast<uint32_t>(b >> 1) & 1u, kTcWaitLimitNs / 10);
+            for (int b = max(0, issued[1] - 2); b < issued[1]; b++)
+                mbar_wait_bounded(bar_o(b & 1), static_cast<uint32_t>(b >> 1) & 1u, kTcWaitLimitNs / 10);
         }
     } else {
         tc_fence_after();
@@ -624,14 +771,13 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         float o[64];
         tmem_ld32(lane_base + 64 * hf, o);
         tmem_ld32(lane_base + 64 * hf + 32, o + 32);
-        float la, lb, za, zb;
-        f2_unpack(l2, la, lb);
-        f2_unpack(z2, za, zb);
-        xchg[hf * kTcRows + row] = la + lb;
-        xchg[2 * kTcRows + hf * kTcRows + row] = za + zb;
+        if (hf == 0) {
+            xchg[row] = l_row;
+            xchg[kTcRows + row] = z_row;
+        }
         __syncthreads();
-        const float lt = xchg[row] + xchg[kTcRows + row];
-        const float zt = xchg[2 * kTcRows + row] + xchg[3 * kTcRows + row];
+        const float lt = xchg[row];
+        const float zt = xchg[kTcRows + row];
         const float inv = live ? 1.0f / lt : 0.0f;
         float v[64];
 #pragma unroll
