@@ -10,27 +10,30 @@
 // are s = scale_K acc + zero_K sum(q) over the raw codes; P' = p scale_V meets the raw V codes
 // and sum p zero_V is added in fp32; the output is rotated back.
 //
-// A CTA (8 warps) owns one tile of up to 128 query rows: T = 128 / G consecutive query tokens x
-// the G query heads of one kv head, row r = token (r / G), head (r % G).  It walks the tile's
-// causal range of the cache in blocks of 64 tokens (4 pages):
-//   1. the 4 pages' codes and scales are staged by cp.async (LSU path) into one code stage;
-//   2. all 256 threads unpack them once into fp16 tiles: K [64 tokens x 128 d] and
-//      V [64 tokens x 128 d], token rows of 128 B per half of d under the 128-byte swizzle;
-//   3. one thread issues S = Q K^T (M 128, N 64, K 128: 8 x tcgen05.mma.kind::f16) into one of
-//      two S buffers in tensor memory;
-//   4. two threads per row each read half of the row of S (tcgen05.ld), apply scales, zero points
-//      and the causal limit, share the block maximum and run the online softmax; P' (fp16) goes
-//      to a shared tile;
-//   5. one thread issues O += P' V (M 128, N 128, K 64: 4 MMAs, V read as the MN-major operand).
-// The loop is software-pipelined by one block: while the threads run the softmax of block kb, the
-// tensor cores compute S of block kb + 1 (unpacked and issued just before), and P V of block kb
-// runs while the threads unpack the K of block kb + 2; V and the scale tables are double-buffered,
-// the codes of block kb + 2 are in flight meanwhile, and the block table is read three blocks ahead.
-// When a block's maximum exceeds a row's running maximum, the row's O accumulator is rescaled in
-// tensor memory (the warp's 32 rows together; rows without a change multiply by 1).  Letting the
-// maximum lag (weights up to 2^4) saved no measurable time and doubled the largest error.
-// The epilogue reads each thread's half of its O row, adds the zero-point term, divides by the row
-// sum and rotates back (the last Hadamard stage pairs the halves through shared memory).
+// A CTA (8 warps, 2 per SM) owns one tile of up to 128 query rows: T = 128 / G consecutive query
+// tokens x the G query heads of one kv head, row r = token (r / G), head (r % G).  It walks the
+// tile's causal range of the cache in blocks of 64 tokens (4 pages) with two roles:
+//   - producers (warps 4-7) load each block's code words and scales straight into registers, two
+//     blocks ahead (block-table ids three ahead), unpack them into fp16 tiles K and V [64 tokens x
+//     128 d] (V double-buffered; token rows of 128 B per half of d, 128-byte swizzle), write the
+//     block's scale table (a ring of 4), and one of them issues S = Q K^T (M 128, N 64, K 128:
+//     8 x tcgen05.mma.kind::f16) into one of two S buffers in tensor memory;
+//   - softmax warps (0-3) read S with tcgen05.ld.16x256b, which gives each thread 4 rows x 16
+//     tokens (rows r, r + 8 of each 16-lane half, r = lane / 4; tokens 8 k + 2 (lane % 4), + 1), so
+//     a scale-table entry loaded once serves 4 rows and a row's maximum is combined over the 4
+//     threads of a quad by two shuffles; they apply scales, zero points and the causal limit, run
+//     the online softmax one 16-lane half at a time, write P' (fp16) to a shared tile by stmatrix,
+//     and thread 0 issues O += P' V (M 128, N 128, K 64: 4 MMAs, V the MN-major operand).
+// The roles hand off through mbarriers: the tensor cores' commits (S and P' V done), the softmax's
+// release of an S buffer, and the producers' V and scale-table arrivals; each role also meets at
+// its own named barrier once per block.  So the tensor cores compute S of block kb + 1 while the
+// softmax runs on block kb, and the producers unpack block kb + 2 meanwhile.  When a block's
+// maximum exceeds a row's running maximum, the row's O accumulator is rescaled in tensor memory
+// (a half warp's rows together; rows without a change multiply by 1).  Letting the maximum lag
+// saved little time and doubled the largest error (weights kept in fp16's normal range then flush
+// more of the small ones).  The epilogue reads each half of an O row (two threads per row), adds
+// the zero-point term, divides by the row sum and rotates back (the last Hadamard stage pairs the
+// halves through shared memory).
 //
 // Codes enter the tensor cores as exact fp16 integers n = (1024 + n) - 1024 (a magic OR and one
 // half2 subtraction per pair).  These tensor cores flush fp16 subnormals, so the operands are kept
@@ -140,81 +143,41 @@ __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float v[32])
 }
 
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, float v[16])
+// tcgen05.ld.16x256b.x8 of one 16-lane half (32 columns per thread's pair of rows), waited for
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t ta, float v[32])
 {
-    uint32_t r[16];
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-#pragma unroll
-    for (int i = 0; i < 16; i++)
-        v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void tmem_st16(uint32_t taddr, const float v[16])
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-                   "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-                   "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-                   "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-                   "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-                   "r"(__float_as_uint(v[15]))
-                 : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-}
-// 16 consecutive fp32 columns of this thread's lane, without waiting (tmem_wait_ld before use)
-__device__ __forceinline__ void tmem_ld16_nowait(uint32_t taddr, float v[16])
-{
-    uint32_t *r = reinterpret_cast<uint32_t *>(v);
-    asm volatile("tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];"
-                 : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
-                   "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15])
-                 : "r"(taddr));
-}
-// waits for this thread's tensor-memory loads; the 32 registers of `v` are tied to the wait so
-// that no use moves above it
-__device__ __forceinline__ void tmem_wait_ld32(float v[32])
-{
-    uint32_t *r = reinterpret_cast<uint32_t *>(v);
-    asm volatile("tcgen05.wait::ld.sync.aligned;"
-                 : "+r"(r[0]), "+r"(r[1]), "+r"(r[2]), "+r"(r[3]), "+r"(r[4]), "+r"(r[5]), "+r"(r[6]), "+r"(r[7]),
-                   "+r"(r[8]), "+r"(r[9]), "+r"(r[10]), "+r"(r[11]), "+r"(r[12]), "+r"(r[13]), "+r"(r[14]),
-                   "+r"(r[15]), "+r"(r[16]), "+r"(r[17]), "+r"(r[18]), "+r"(r[19]), "+r"(r[20]), "+r"(r[21]),
-                   "+r"(r[22]), "+r"(r[23]), "+r"(r[24]), "+r"(r[25]), "+r"(r[26]), "+r"(r[27]), "+r"(r[28]),
-                   "+r"(r[29]), "+r"(r[30]), "+r"(r[31])
-                 :: "memory");
-}
-__device__ __forceinline__ void tmem_st16_nowait(uint32_t taddr, const float v[16])
-{
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};"
-                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])), "r"(__float_as_uint(v[2])),
-                   "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])), "r"(__float_as_uint(v[5])),
-                   "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])), "r"(__float_as_uint(v[8])),
-                   "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])), "r"(__float_as_uint(v[11])),
-                   "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])), "r"(__float_as_uint(v[14])),
-                   "r"(__float_as_uint(v[15]))
+    uint32_t *a = reinterpret_cast<uint32_t *>(v);
+    asm volatile("tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];\n\t"
+                 "tcgen05.wait::ld.sync.aligned;"
+                 : "=r"(a[0]), "=r"(a[1]), "=r"(a[2]), "=r"(a[3]), "=r"(a[4]), "=r"(a[5]), "=r"(a[6]), "=r"(a[7]),
+                   "=r"(a[8]), "=r"(a[9]), "=r"(a[10]), "=r"(a[11]), "=r"(a[12]), "=r"(a[13]), "=r"(a[14]), "=r"(a[15]),
+                   "=r"(a[16]), "=r"(a[17]), "=r"(a[18]), "=r"(a[19]), "=r"(a[20]), "=r"(a[21]), "=r"(a[22]), "=r"(a[23]),
+                   "=r"(a[24]), "=r"(a[25]), "=r"(a[26]), "=r"(a[27]), "=r"(a[28]), "=r"(a[29]), "=r"(a[30]), "=r"(a[31])
+                 : "r"(ta)
                  : "memory");
 }
 
-__device__ __forceinline__ void tmem_st32(uint32_t taddr, const float v[32])
+// the matching store (no wait)
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t ta, const float v[32])
 {
-    asm volatile("tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-                 "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
-                 ::"r"(taddr), "r"(__float_as_uint(v[0])), "r"(__float_as_uint(v[1])),
-                   "r"(__float_as_uint(v[2])), "r"(__float_as_uint(v[3])), "r"(__float_as_uint(v[4])),
-                   "r"(__float_as_uint(v[5])), "r"(__float_as_uint(v[6])), "r"(__float_as_uint(v[7])),
-                   "r"(__float_as_uint(v[8])), "r"(__float_as_uint(v[9])), "r"(__float_as_uint(v[10])),
-                   "r"(__float_as_uint(v[11])), "r"(__float_as_uint(v[12])), "r"(__float_as_uint(v[13])),
-                   "r"(__float_as_uint(v[14])), "r"(__float_as_uint(v[15])), "r"(__float_as_uint(v[16])),
-                   "r"(__float_as_uint(v[17])), "r"(__float_as_uint(v[18])), "r"(__float_as_uint(v[19])),
-                   "r"(__float_as_uint(v[20])), "r"(__float_as_uint(v[21])), "r"(__float_as_uint(v[22])),
-                   "r"(__float_as_uint(v[23])), "r"(__float_as_uint(v[24])), "r"(__float_as_uint(v[25])),
-                   "r"(__float_as_uint(v[26])), "r"(__float_as_uint(v[27])), "r"(__float_as_uint(v[28])),
-                   "r"(__float_as_uint(v[29])), "r"(__float_as_uint(v[30])), "r"(__float_as_uint(v[31]))
+    const uint32_t *a = reinterpret_cast<const uint32_t *>(v);
+    asm volatile("tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,"
+                 "%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+                 ::"r"(ta), "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(a[4]), "r"(a[5]), "r"(a[6]), "r"(a[7]),
+                   "r"(a[8]), "r"(a[9]), "r"(a[10]), "r"(a[11]), "r"(a[12]), "r"(a[13]), "r"(a[14]), "r"(a[15]),
+                   "r"(a[16]), "r"(a[17]), "r"(a[18]), "r"(a[19]), "r"(a[20]), "r"(a[21]), "r"(a[22]), "r"(a[23]),
+                   "r"(a[24]), "r"(a[25]), "r"(a[26]), "r"(a[27]), "r"(a[28]), "r"(a[29]), "r"(a[30]), "r"(a[31])
                  : "memory");
-    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// four 8x8 fp16 matrices from the fragment layout (thread t: row t / 4, columns 2 (t % 4), + 1 of
+// each); thread t gives the shared address of row t % 8 of matrix t / 8
+__device__ __forceinline__ void stmatrix_x4(uint32_t addr, const uint32_t r[4])
+{
+    asm volatile("stmatrix.sync.aligned.m8n8.x4.shared.b16 [%0], {%1, %2, %3, %4};" ::"r"(addr), "r"(r[0]), "r"(r[1]),
+                 "r"(r[2]), "r"(r[3])
+                 : "memory");
 }
 
 // d order of the 8 entries of a 16-byte chunk: position j holds d = 8 a + kPerm[j]
@@ -397,7 +360,6 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int nrows = ntok * G;
     const bool live = row < nrows;
     const int tq = live ? row / G : 0, hg = live ? row - tq * G : 0;
-    const int limit = L - C + t0 + tq;                     // last visible cache token of the row
     const int n_kv = L - C + t0 + ntok;                    // cache tokens any row sees
     const int n_blocks = (n_kv + kTcBlockTokens - 1) / kTcBlockTokens;
     const int n_pages = (n_kv + kPageSize - 1) / kPageSize;
@@ -491,7 +453,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     tc_fence_after();
     const uint32_t tmem = *tmem_slot;
     const uint32_t lane_base = tmem + (static_cast<uint32_t>(32 * (warp & 3)) << 16);
-    float l_row = 0.0f, z_row = 0.0f;   // softmax threads: the row's sums over all blocks
+    float l_quad[4] = {0.0f, 0.0f, 0.0f, 0.0f}, z_quad[4] = {0.0f, 0.0f, 0.0f, 0.0f};   // softmax: row sums
 
     if (warp >= 4) {
         // ======== producers: pages -> registers (two blocks ahead) -> fp16 K / V tiles, scales ====
@@ -613,111 +575,157 @@ __global__ void __launch_bounds__(kTcThreads, 2)
             w1 = w2;
         }
     } else {
-        // ======== softmax: thread `row` owns one query row over all 64 tokens of each block =======
-        const float sq = xchg[row] + xchg[kTcRows + row];
-        const uint64_t sq2 = f2_pack(sq, sq);
-        float m_ref = -INFINITY;
-        uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;   // the row's sums (two lanes each)
+        // ======== softmax: fragment layout ===========================================================
+        // S is read with tcgen05.ld.16x256b: in each 16-lane half of its quarter, thread (r = lane / 4,
+        // c = lane % 4) gets rows r and r + 8 at columns 8 k + 2 c, 8 k + 2 c + 1 (k = 0 .. 7).  So a
+        // thread holds 4 rows (slots i: row 32 w + r + 8 i) x 16 tokens, and each of its 16 scale-table
+        // loads serves 4 rows; the row maximum is combined over the 4 threads of a quad by shuffles, and
+        // the sums l, z stay per thread until the end.
+        const int fr = lane >> 2, fc = lane & 3;
+        float sq[4], m_ref[4];
+        uint64_t l2[4], z2[4];   // this thread's share of the row sums (two lanes each)
+        bool live_i[4];
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            const int ri = 32 * warp + fr + 8 * i;
+            sq[i] = xchg[ri] + xchg[kTcRows + ri];
+            m_ref[i] = -INFINITY;
+            l2[i] = f2_pack(0.0f, 0.0f);
+            z2[i] = l2[i];
+            live_i[i] = ri < nrows;
+        }
+        const uint32_t quarter = tmem + (static_cast<uint32_t>(32 * warp) << 16);
         bool ok = true;
         for (int kb = 0; kb < n_blocks; kb++) {
             // S of block kb and its scale table
             ok = ok && tc_wait(bar_s(kb & 1), static_cast<uint32_t>(kb >> 1) & 1u, abort_flag);
             ok = ok && tc_wait(bar_sc(kb & 3), static_cast<uint32_t>(kb >> 2) & 1u, abort_flag);
             ok = __all_sync(0xFFFFFFFFu, ok);   // tensor-memory loads are warp-wide
-            float sv[64];   // the block's 64 logits of this row
-            bool grow = false;
-            float alpha = 1.0f;
-            if (ok) {
-                tc_fence_after();
-                tmem_ld32(lane_base + 128 + 64 * (kb & 1), sv);
-                tmem_ld32(lane_base + 128 + 64 * (kb & 1) + 32, sv + 32);
-                tc_fence_before();
-                __syncwarp();
-                if (lane == 0)
-                    tc_arrive(bar_sfree(kb & 1));   // the S buffer may be overwritten
-
-                const float4 *kp4 = reinterpret_cast<const float4 *>(smem + kSmScales + (kb & 3) * kSmScaleSet);
+            const float4 *kp4 = reinterpret_cast<const float4 *>(smem + kSmScales + (kb & 3) * kSmScaleSet);
+            const float4 *vp4 = kp4 + kTcBlockTokens / 2;
+            const uint32_t cb = 128 + 64 * (kb & 1);
+            // the two 16-lane halves of the quarter are independent rows: one at a time
 #pragma unroll
-                for (int j = 0; j < 64; j += 2) {
-                    const float4 kp = kp4[j / 2];
-                    const uint64_t t = f2_fma(f2_pack(kp.x, kp.y), f2_pack(sv[j], sv[j + 1]),
-                                              f2_mul(f2_pack(kp.z, kp.w), sq2));
-                    f2_unpack(t, sv[j], sv[j + 1]);
+            for (int h = 0; h < 2; h++) {
+                float s[32];   // s[4 k + e]: row slot 2 h + e / 2, token 8 k + 2 c + e % 2
+                bool grow = false;
+                float alpha[2] = {1.0f, 1.0f};
+                if (ok) {
+                    tc_fence_after();
+                    tmem_ld_16x256b_x8(quarter + (static_cast<uint32_t>(16 * h) << 16) + cb, s);
+                    if (h == 1) {
+                        tc_fence_before();
+                        __syncwarp();
+                        if (lane == 0)
+                            tc_arrive(bar_sfree(kb & 1));   // the S buffer may be overwritten
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; k++) {
+                        const float4 kp = kp4[4 * k + fc];   // tokens 8 k + 2 c, + 1
+                        const uint64_t sk2 = f2_pack(kp.x, kp.y), zk2 = f2_pack(kp.z, kp.w);
+#pragma unroll
+                        for (int j = 0; j < 2; j++) {
+                            float &a = s[4 * k + 2 * j], &b = s[4 * k + 2 * j + 1];
+                            const float q = sq[2 * h + j];
+                            const uint64_t t = f2_fma(sk2, f2_pack(a, b), f2_mul(zk2, f2_pack(q, q)));
+                            f2_unpack(t, a, b);
+                        }
+                    }
+                    // the causal limit (and the end of the cache) only reaches the last blocks of a tile
+                    if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
+                        const int tok0 = kb * kTcBlockTokens + 2 * fc;
+#pragma unroll
+                        for (int j = 0; j < 2; j++) {
+                            const int ri = 32 * warp + fr + 8 * (2 * h + j);
+                            const int lim = L - C + t0 + (live_i[2 * h + j] ? ri / G : 0);
+#pragma unroll
+                            for (int k = 0; k < 8; k++)
+#pragma unroll
+                                for (int e = 0; e < 2; e++)
+                                    if (tok0 + 8 * k + e > lim)
+                                        s[4 * k + 2 * j + e] = -INFINITY;
+                        }
+                    }
+#pragma unroll
+                    for (int j = 0; j < 2; j++) {
+                        const int i = 2 * h + j;
+                        float m = -INFINITY;
+#pragma unroll
+                        for (int k = 0; k < 8; k++)
+                            m = fmax3(m, s[4 * k + 2 * j], s[4 * k + 2 * j + 1]);
+                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+                        m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+                        if (!live_i[i])
+                            m = -INFINITY;
+                        if (m > m_ref[i] + kTcRescale) {
+                            alpha[j] = ex2_approx(m_ref[i] - m);   // 0 on the first block a row sees
+                            const uint64_t a2 = f2_pack(alpha[j], alpha[j]);
+                            l2[i] = f2_mul(l2[i], a2);
+                            z2[i] = f2_mul(z2[i], a2);
+                            m_ref[i] = m;
+                            grow |= alpha[j] != 0.0f;
+                        }
+                    }
                 }
-                // the causal limit (and the end of the cache) only reaches the last blocks of a tile
-                if (kb * kTcBlockTokens + kTcBlockTokens - 1 > L - C + t0) {
-                    const int tok0 = kb * kTcBlockTokens;
-#pragma unroll
-                    for (int j = 0; j < 64; j++)
-                        if (tok0 + j > limit)
-                            sv[j] = -INFINITY;
+                if (h == 0) {
+                    // P' V of block kb - 1 has finished with the P' tile and the O accumulator
+                    if (kb >= 1)
+                        ok = ok && tc_wait(bar_o((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u, abort_flag);
+                    ok = __all_sync(0xFFFFFFFFu, ok);
                 }
-                float m4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};   // 4 short chains
+                if (ok) {
+                    tc_fence_after();
+                    // the weights of the half's two rows, two 8-token chunks per stmatrix (matrices:
+                    // (row slot 2 h, chunk k), (2 h + 1, k), (2 h, k + 1), (2 h + 1, k + 1))
 #pragma unroll
-                for (int j = 0; j < 64; j += 2)
-                    m4[(j >> 1) & 3] = fmax3(m4[(j >> 1) & 3], sv[j], sv[j + 1]);
-                float mb = fmaxf(fmax3(m4[0], m4[1], m4[2]), m4[3]);
-                if (!live)
-                    mb = -INFINITY;
-                grow = mb > m_ref + kTcRescale;
-                if (grow) {
-                    alpha = ex2_approx(m_ref - mb);   // 0 on the first block a row sees
-                    const uint64_t a2 = f2_pack(alpha, alpha);
-                    l2 = f2_mul(l2, a2);
-                    z2 = f2_mul(z2, a2);
-                    m_ref = mb;
+                    for (int k = 0; k < 8; k += 2) {
+                        uint32_t pw[4];
+#pragma unroll
+                        for (int kk = 0; kk < 2; kk++) {
+                            const float4 vp = vp4[4 * (k + kk) + fc];
+                            const uint64_t sv2 = f2_pack(vp.x, vp.y), zv2 = f2_pack(vp.z, vp.w);
+#pragma unroll
+                            for (int j = 0; j < 2; j++) {
+                                const int i = 2 * h + j;
+                                const float mr = live_i[i] ? m_ref[i] : INFINITY;   // rows past the tile: 0
+                                float d0, d1;
+                                f2_unpack(f2_sub(f2_pack(s[4 * (k + kk) + 2 * j], s[4 * (k + kk) + 2 * j + 1]),
+                                                 f2_pack(mr, mr)),
+                                          d0, d1);
+                                const uint64_t p2 = f2_pack(ex2_approx(d0), ex2_approx(d1));
+                                l2[i] = f2_add(l2[i], p2);
+                                z2[i] = f2_fma(p2, zv2, z2[i]);
+                                float q0, q1;
+                                f2_unpack(f2_mul(p2, sv2), q0, q1);
+                                pw[2 * kk + j] = half2_as_u32(__floats2half2_rn(q0, q1));
+                            }
+                        }
+                        // thread t: row 32 w + 16 h + t % 16 of chunk k + t / 16
+                        stmatrix_x4(sbase + kSmP + sw128_chunk(32 * warp + 16 * h + (lane & 15), k + (lane >> 4),
+                                                                kTcRows * 128),
+                                    pw);
+                    }
+                    // rescale the half's O rows in tensor memory (warp-wide; alpha 1 where no change)
+                    if (kb > 0 && __any_sync(0xFFFFFFFFu, grow)) {
+#pragma unroll 1
+                        for (int c = 0; c < 2; c++) {   // 64 columns at a time
+                            const uint32_t ta = quarter + (static_cast<uint32_t>(16 * h) << 16) + 64 * c;
+                            float ov[32];
+                            tmem_ld_16x256b_x8(ta, ov);
+#pragma unroll
+                            for (int j = 0; j < 32; j += 4) {
+                                ov[j] *= alpha[0];
+                                ov[j + 1] *= alpha[0];
+                                ov[j + 2] *= alpha[1];
+                                ov[j + 3] *= alpha[1];
+                            }
+                            tmem_st_16x256b_x8(ta, ov);
+                        }
+                        asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+                    }
                 }
             }
-            // P' V of block kb - 1 has finished with the P' tile and the O accumulator
-            if (kb >= 1)
-                ok = ok && tc_wait(bar_o((kb - 1) & 1), static_cast<uint32_t>((kb - 1) >> 1) & 1u, abort_flag);
-            ok = __all_sync(0xFFFFFFFFu, ok);
             if (ok) {
-                tc_fence_after();
-                // the weights, 8 tokens (one 16-byte chunk of the P' row) at a time
-                const float4 *vp4 = reinterpret_cast<const float4 *>(smem + kSmScales + (kb & 3) * kSmScaleSet) +
-                                    kTcBlockTokens / 2;
-                const float mr = live ? m_ref : INFINITY;   // rows past the tile: every weight 0
-                const uint64_t mr2 = f2_pack(mr, mr);
-#pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    uint32_t pw[4];
-#pragma unroll
-                    for (int k = 0; k < 4; k++) {
-                        const int j = 8 * c + 2 * k;
-                        const float4 vp = vp4[j / 2];
-                        float d0, d1;
-                        f2_unpack(f2_sub(f2_pack(sv[j], sv[j + 1]), mr2), d0, d1);
-                        const uint64_t p2 = f2_pack(ex2_approx(d0), ex2_approx(d1));
-                        l2 = f2_add(l2, p2);
-                        z2 = f2_fma(p2, f2_pack(vp.z, vp.w), z2);
-                        float q0, q1;
-                        f2_unpack(f2_mul(p2, f2_pack(vp.x, vp.y)), q0, q1);
-                        pw[k] = half2_as_u32(__floats2half2_rn(q0, q1));
-                    }
-                    const uint32_t a = sbase + kSmP + sw128_chunk(row, c, kTcRows * 128);
-                    asm volatile("st.shared.v4.u32 [%0], {%1, %2, %3, %4};" ::"r"(a), "r"(pw[0]), "r"(pw[1]),
-                                 "r"(pw[2]), "r"(pw[3]) : "memory");
-                }
-                // rescale the O row in tensor memory (warp-wide; alpha 1 where no change): four
-                // rounds of 32 columns, the stores waited for once
-                if (kb > 0 && __any_sync(0xFFFFFFFFu, grow && alpha != 0.0f)) {
-#pragma unroll 1
-                    for (int c = 0; c < 4; c++) {
-                        float ov[32];
-                        tmem_ld16_nowait(lane_base + 32 * c, ov);
-                        tmem_ld16_nowait(lane_base + 32 * c + 16, ov + 16);
-                        tmem_wait_ld32(ov);
-#pragma unroll
-                        for (int i = 0; i < 32; i += 2) {
-                            const uint64_t r = f2_mul(f2_pack(ov[i], ov[i + 1]), f2_pack(alpha, alpha));
-                            f2_unpack(r, ov[i], ov[i + 1]);
-                        }
-                        tmem_st16_nowait(lane_base + 32 * c, ov);
-                        tmem_st16_nowait(lane_base + 32 * c + 16, ov + 16);
-                    }
-                    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
-                }
                 async_proxy_fence();
                 tc_fence_before();
             }
@@ -741,11 +749,20 @@ __global__ void __launch_bounds__(kTcThreads, 2)
                 }
             }
         }
-        float la, lb, za, zb;
-        f2_unpack(l2, la, lb);
-        f2_unpack(z2, za, zb);
-        l_row = la + lb;
-        z_row = za + zb;
+        // the row sums over the quad, for the epilogue
+#pragma unroll
+        for (int i = 0; i < 4; i++) {
+            float la, lb, za, zb;
+            f2_unpack(l2[i], la, lb);
+            f2_unpack(z2[i], za, zb);
+            float lt = la + lb, zt = za + zb;
+            lt += __shfl_xor_sync(0xFFFFFFFFu, lt, 1);
+            zt += __shfl_xor_sync(0xFFFFFFFFu, zt, 1);
+            lt += __shfl_xor_sync(0xFFFFFFFFu, lt, 2);
+            zt += __shfl_xor_sync(0xFFFFFFFFu, zt, 2);
+            l_quad[i] = lt;
+            z_quad[i] = zt;
+        }
     }
 
     // ---- epilogue: O row -> zero term, 1 / l, the weights' scale, inverse rotation ----------------
@@ -771,9 +788,12 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         float o[64];
         tmem_ld32(lane_base + 64 * hf, o);
         tmem_ld32(lane_base + 64 * hf + 32, o + 32);
-        if (hf == 0) {
-            xchg[row] = l_row;
-            xchg[kTcRows + row] = z_row;
+        if (warp < 4 && (lane & 3) == 0) {
+#pragma unroll
+            for (int i = 0; i < 4; i++) {
+                xchg[32 * warp + (lane >> 2) + 8 * i] = l_quad[i];
+                xchg[kTcRows + 32 * warp + (lane >> 2) + 8 * i] = z_quad[i];
+            }
         }
         __syncthreads();
         const float lt = xchg[row];
