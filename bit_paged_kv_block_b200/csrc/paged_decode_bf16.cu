@@ -371,13 +371,18 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     p.win_recent = a.win_recent;
     p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Bf16Format::kWarps;
+    // The window part's segments are short (at most sink + recent tokens each): one warp per
+    // segment, so windows of equal length are never split and its merge has nothing to fold,
+    // instead of runs of a page or two whose fixed costs dominate.
+    if (a.win_part == 1)
+        p.total_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(p.total_warps, p.max_segments)));
     p.q_mult = static_cast<float>(static_cast<double>(a.sm_scale) * 1.4426950408889634);
 
     cudaLaunchAttribute attr[1];
     attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cudaLaunchConfig_t cfg = {};
-    cfg.gridDim = dim3(static_cast<unsigned>(ls.sms * ls.occ));
+    cfg.gridDim = dim3(static_cast<unsigned>((p.total_warps + Bf16Format::kWarps - 1) / Bf16Format::kWarps));
     cfg.blockDim = dim3(32 * Bf16Format::kWarps);
     cfg.dynamicSmemBytes = smem;
     cfg.stream = stream;
