@@ -194,10 +194,15 @@ int saw_decode_step_plain(const saw_cache_desc *cache, int32_t num_q_heads, cons
  *     q: bf16 [total_q][Hq][D]; out: fp32 [total_q][Hq][D]; q_start: int32 [num_seqs + 1],
  *     device, non-decreasing, q_start[0] = 0, q_start[num_seqs] = total_q, 0 <= C_s <= seq_lens[s]
  *     (a violating sequence is flagged SAW_DEV_BAD_SEQ_LEN and skipped).
- * Every (query token, head) pair reads the pages of its sequence once per block of 8 such
- * pairs, so the K/V traffic is about total_q G / 8 times that of one decode of the batch; the
- * kernel and its work split are those of the decode.  workspace: at least
- * saw_paged_prefill_workspace_bytes() bytes, 256-byte aligned, no initialisation needed.
+ * Two kernels serve the call.  At D = 128, when the chunks average at least half a 128-row tile
+ * per sequence (total_q G >= 64 num_seqs), a tensor-core kernel (tcgen05) takes tiles of 128 / G
+ * query tokens x G heads and walks each tile's causal range of the cache once (the repeated reads
+ * of a page by the tiles of one sequence come from L2).  Otherwise, and at D = 64 or 256, the
+ * decode kernel runs with segments of 8 (query token, head) rows, whose K/V traffic is about
+ * total_q G / 8 times that of one decode of the batch.  The tensor-core kernel's arithmetic
+ * keeps its fp16 operands in fp16's normal range (queries scaled by 2^8, weights by 2^4): results
+ * agree with the decode kernel's within the attention tolerance, not bit for bit.  workspace: at
+ * least saw_paged_prefill_workspace_bytes() bytes, 256-byte aligned, no initialisation needed.
  * The _plain variant reads a cache written by saw_quantize_paged_plain. */
 size_t saw_paged_prefill_workspace_bytes(const saw_cache_desc *cache, int32_t num_q_heads,
                                          int32_t num_seqs, int64_t total_q);
