@@ -87,3 +87,24 @@ def test_prefill_tc_rows_match_decode(cuda_device):
                                   np.array([lens[s] - chunks[s] + i + 1], dtype=np.int32),
                                   nthreads=NTHREADS)
         assert_attention_close(got[r:r + 1], want, f"row {r}")
+
+
+def test_prefill_tc_bench_workload_sampled(cuda_device):
+    """The bench's chunked-prefill workload itself (8 sequences of 4096 cached tokens, the last
+    512 of each as queries, 32 q / 8 kv heads, the bench's seeds), in the launch configuration the
+    bench times; sampled rows at tile boundaries against the oracle's decode of their prefix."""
+    from bit_paged_kv_block_b200 import saw
+    wl = synth.custom("chunked_prefill", [4096] * 8, num_q_heads=32, num_kv_heads=8, seed=40,
+                      outlier_range=(10.0, 30.0))
+    pages, scales = oracle_cache(wl)
+    chunk = 512
+    q_start = np.arange(0, 9 * chunk, chunk, dtype=np.int32)
+    q = torch.randn(8 * chunk, 32, 128, generator=torch.Generator(device="cpu").manual_seed(41)).to(torch.bfloat16)
+    got = _run(wl, pages, scales, q, q_start, cuda_device)
+    for s in (0, 3, 7):
+        for i in (0, 31, 32, 255, 480, 511):   # tiles are 32 query tokens at G = 4
+            r = s * chunk + i
+            want = oracle.decode_fp64(u16(q[r:r + 1]), pages, scales, wl.block_table[s:s + 1],
+                                      np.array([4096 - chunk + i + 1], dtype=np.int32),
+                                      nthreads=NTHREADS)
+            assert_attention_close(got[r:r + 1], want, f"sequence {s} query {i}")
