@@ -108,3 +108,17 @@ def test_prefill_tc_bench_workload_sampled(cuda_device):
                                       np.array([4096 - chunk + i + 1], dtype=np.int32),
                                       nthreads=NTHREADS)
             assert_attention_close(got[r:r + 1], want, f"sequence {s} query {i}")
+
+
+def test_prefill_tc_many_sequences(cuda_device):
+    """300 sequences (the tile search scans the sequences 256 at a time, so a second pass finds
+    the tiles of the last 44), short ragged lengths and 16-token chunks: at G = 4 that is 64 rows
+    per sequence, the tensor-core path."""
+    rng = np.random.default_rng(77)
+    lens = [int(x) for x in rng.integers(16, 200, size=300)]
+    chunks = [16] * 300
+    wl, pages, scales, q, q_start = _case(lens, chunks, 4, 2, seed=34)
+    got = _run(wl, pages, scales, q, q_start, cuda_device)
+    want = oracle.prefill_fp64(u16(q), q_start, pages, scales, wl.block_table, wl.seq_lens,
+                               nthreads=NTHREADS)
+    assert_attention_close(got, want, "tensor-core prefill, 300 sequences")
