@@ -35,15 +35,16 @@ __host__ __device__ constexpr int slot_floats() { return kTiles * 128 + 16; }
 constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
 constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
 constexpr int kRowsPerBlock = 8;                        // query rows (MMA columns) per segment
-constexpr int kMergeWarps = 4;
+constexpr int kMergeWarps = 8;
 constexpr int kMergeThreads = 32 * kMergeWarps;
 // per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
 constexpr int kSeqTableBytes = 20;
 // merge kernel shared memory: per-warp partials, flags, then the sequence tables
 template <int kTiles>
 __host__ __device__ constexpr int merge_smem_flags() { return (kMergeWarps - 1) * slot_floats<kTiles>() * 4; }
+// the flags hold scan_sequences' two int64 partial sums per warp
 template <int kTiles>
-__host__ __device__ constexpr int merge_smem_tables() { return merge_smem_flags<kTiles>() + 64; }
+__host__ __device__ constexpr int merge_smem_tables() { return merge_smem_flags<kTiles>() + 16 * kMergeWarps; }
 
 inline size_t seq_table_bytes(int32_t num_seqs)
 {
@@ -592,7 +593,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 // Shared memory: rings, then per warp (kStages + 1) mbarriers (the last for the query), 128 bytes
 // of flags, the per-warp query buffers (qrows * 256 bytes each) and the sequence tables.
 
-constexpr int kSmemFlagBytes = 128;
+constexpr int kSmemFlagBytes = 128;   // scan_sequences' two int64 partial sums per warp
 // bytes of `rows` raw bf16 query rows of a format's head dimension
 template <class Fmt>
 __host__ __device__ constexpr int query_bytes(int rows) { return rows * Fmt::kDim * 2; }
@@ -620,6 +621,7 @@ template <class Fmt, bool kPrefill>
 __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     paged_decode_kernel(const __grid_constant__ CUtensorMap tmap, const DecodeParams p)
 {
+    static_assert(16 * Fmt::kWarps <= kSmemFlagBytes, "the flags hold two int64 per warp");
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
