@@ -35,7 +35,7 @@ __host__ __device__ constexpr int slot_floats() { return kTiles * 128 + 16; }
 constexpr int64_t kKappa = 2;                           // per-segment cost, in pages
 constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait after 1 s
 constexpr int kRowsPerBlock = 8;                        // query rows (MMA columns) per segment
-constexpr int kMergeWarps = 8;
+constexpr int kMergeWarps = 4;
 constexpr int kMergeThreads = 32 * kMergeWarps;
 // per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
 constexpr int kSeqTableBytes = 20;
