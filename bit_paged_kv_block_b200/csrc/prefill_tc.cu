@@ -72,7 +72,7 @@ constexpr int kSmVTile = 2 * kTcBlockTokens * 128;
 constexpr int kSmP = kSmV + 2 * kSmVTile;                // P' tile: [128 rows][128 B]
 constexpr int kSmScales = kSmP + kTcRows * 128;          // 4 x (K, V) token-pair factors
 constexpr int kSmScaleSet = 2 * 2 * kTcBlockTokens * 4;
-constexpr int kSmXchg = kSmScales + 4 * kSmScaleSet;     // [4][128] fp32 between row halves
+constexpr int kSmXchg = kSmScales + 4 * kSmScaleSet;     // per row: the query halves' sums, then l, z
 constexpr int kSmBars = kSmXchg + 4 * kTcRows * 4;       // 12 mbarriers, tmem addr, flags
 constexpr int kSmTile = kSmBars + 128;                   // tile descriptor
 constexpr int kSmBytes = kSmTile + 64;
@@ -329,7 +329,7 @@ __global__ void __launch_bounds__(kTcThreads, 2)
     const int row = 32 * (warp & 3) + lane;               // tile row = tensor-memory lane
     const uint32_t sbase = smem_u32(smem);
     int *sm_tile = reinterpret_cast<int *>(smem + kSmTile);
-    float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [4][128] fp32 between row halves
+    float *xchg = reinterpret_cast<float *>(smem + kSmXchg);   // [2][128] fp32 per-row hand-overs
     const uint32_t bars = sbase + kSmBars;
     // bar_s[b]: S of blocks b, b + 2, ... done (tensor-core commit); bar_sfree[b]: the softmax has
     // read that S buffer (one arrival per softmax warp); bar_o[b]: P' V of blocks b, b + 2, ... done;
@@ -578,9 +578,10 @@ __global__ void __launch_bounds__(kTcThreads, 2)
         // ======== softmax: fragment layout ===========================================================
         // S is read with tcgen05.ld.16x256b: in each 16-lane half of its quarter, thread (r = lane / 4,
         // c = lane % 4) gets rows r and r + 8 at columns 8 k + 2 c, 8 k + 2 c + 1 (k = 0 .. 7).  So a
-        // thread holds 4 rows (slots i: row 32 w + r + 8 i) x 16 tokens, and each of its 16 scale-table
-        // loads serves 4 rows; the row maximum is combined over the 4 threads of a quad by shuffles, and
-        // the sums l, z stay per thread until the end.
+        // thread holds 4 rows (slots i: row 32 w + r + 8 i) x 16 tokens.  The halves are processed
+        // one after the other (32 live S values); each scale-table entry a thread loads (8 for K and
+        // 8 for V per half) serves the half's 2 rows, the row maximum is combined over the 4 threads
+        // of a quad by shuffles, and the sums l, z stay per thread until the end.
         const int fr = lane >> 2, fc = lane & 3;
         float sq[4], m_ref[4];
         uint64_t l2[4], z2[4];   // this thread's share of the row sums (two lanes each)
