@@ -163,3 +163,28 @@ def test_window_argument_checks():
     f = saw.lib.saw_paged_decode_window_workspace_bytes
     assert f(ctypes.byref(_desc(d=256)), 32, 4) == 0
     assert f(ctypes.byref(d), 12, 4) == 0
+
+
+def _pf(desc, hq=32, S=2, q=16, q_start=16, total_q=64, out=16, bt=16, lens=16, ws=256,
+        ws_bytes=1 << 20, max_blocks=4, sm_scale=0.088):
+    P = ctypes.c_void_p
+    return saw.lib.saw_paged_prefill_attn(
+        None if desc is None else ctypes.byref(desc), hq, P(q), P(q_start), total_q, P(16), P(16),
+        P(bt), max_blocks, P(lens), S, sm_scale, P(out), P(ws), ws_bytes, None, None)
+
+
+def test_prefill_argument_checks():
+    """The chunked-prefill entry point rejects bad arguments on the host, before any CUDA call."""
+    d = _desc()
+    assert _pf(None) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _pf(_desc(d=96)) == saw.SAW_ERR_UNSUPPORTED
+    assert _pf(d, total_q=-1) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _pf(d, total_q=1 << 31) == saw.SAW_ERR_INVALID_ARGUMENT     # more rows than int32
+    assert _pf(d, q_start=0) == saw.SAW_ERR_INVALID_ARGUMENT           # no chunk starts
+    assert _pf(d, q_start=2) == saw.SAW_ERR_INVALID_ARGUMENT           # not 4-byte aligned
+    assert _pf(d, hq=12) == saw.SAW_ERR_INVALID_ARGUMENT               # Hq % Hkv
+    assert _pf(d, hq=136) == saw.SAW_ERR_UNSUPPORTED                   # G = 17
+    assert _pf(d, q=8) == saw.SAW_ERR_INVALID_ARGUMENT                 # q not 16-byte aligned
+    assert _pf(d, out=0) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _pf(d, sm_scale=float("inf")) == saw.SAW_ERR_INVALID_ARGUMENT
+    assert _pf(d, S=0, q_start=0) == saw.SAW_OK                          # nothing to do
