@@ -179,6 +179,18 @@ def measured_peaks():
         return 6650.0, "fallback"
 
 
+def measured_tensor_peak():
+    """Dense bf16 tensor-core TFLOP/s measured on this machine (the burst figure: the prefill kernel
+    is timed alone); fp16 runs at the same nominal rate.  Fallback: 1590."""
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return float(d["bf16_tflops"]), "measured"
+    except Exception:
+        return 1590.0, "fallback"
+
+
 def sources_digest(sources) -> str:
     """sha256 over the named csrc files, in order (the kernel's whole source)."""
     h = hashlib.sha256()
@@ -495,17 +507,27 @@ def run_saw(args):
         run_pf()
     t_pf = mean_event_ms(run_pf, max(5, min(args.steps, 50)))
     g = pfl.num_q_heads // pfl.num_kv_heads
-    blocks = pfl.num_seqs * pfl.num_kv_heads * (chunk * g // 8)
-    pages = int(((pfl.seq_lens + 15) // 16)[0])
+    # the tensor-core kernel's tiles: 128 / G query tokens each, reading their causal range
+    tile_tok = 128 // g
+    page_reads = pfl.num_seqs * pfl.num_kv_heads * sum(
+        (4096 - chunk + t0 + min(tile_tok, chunk - t0) + 15) // 16 for t0 in range(0, chunk, tile_tok))
     # causal attention: query i of a chunk at the end of L tokens sees L - chunk + i + 1 tokens
     visible = sum(4096 - chunk + i + 1 for i in range(chunk)) * pfl.num_seqs * pfl.num_q_heads
+    tc_peak, tc_peak_kind = measured_tensor_peak()
     prefill_attn = {"workload": "8 seqs x 4096 cached tokens, last 512 of each as queries, 32 q / 8 kv heads",
                     "launch_ms": t_pf,
                     "query_tokens_per_s": world * pfl.num_seqs * chunk / (t_pf * 1e-3),
                     "attention_TFLOPs": 4 * 128 * visible / (t_pf * 1e-3) / 1e12,
-                    "page_reads_per_launch": blocks * pages,
-                    "note": "each block of 8 (query token, head) rows reads its sequence's pages; "
-                            "the repeats come from L2"}
+                    "roofline": {"bound": "tensor", "kernel": "prefill_tc_kernel",
+                                 "achieved": 4 * 128 * visible / (t_pf * 1e-3) / 1e12,
+                                 "peak": tc_peak, "unit": "TFLOP/s",
+                                 "frac": 4 * 128 * visible / (t_pf * 1e-3) / 1e12 / tc_peak,
+                                 "peak_kind": tc_peak_kind,
+                                 "note": "fp16 operands at the dense bf16 rate; flops = 4 D per "
+                                         "visible (query, head, cache token)"},
+                    "page_reads_per_launch": page_reads,
+                    "note": "each 128-row tile (32 query tokens x 4 heads) reads its causal range of "
+                            "the sequence's pages once; the repeats across tiles come from L2"}
     del pkv3, psc3, qpf, opf, wpf
 
     # ---- head dimensions 64 and 256: the decode workload's shape with other head vectors -------
