@@ -44,6 +44,15 @@ WORKLOAD_TEXT = ("decode step, Llama-3-8B layer shape: batch 64, seq_lens unifor
                  "(rotate + INT4 quantize + scatter) then INT4 paged decode attention; bf16 "
                  "N(0,1) with 4 key outlier channels x U[10,30]")
 CPU_SAMPLE_SEQS = 8
+WORKLOADS = {
+    "long": "long-context decode: batch 8 x 32768 tokens, 64 q / 8 kv heads, head_dim 128, page 16, "
+            "block table a shuffled permutation of 16384 pages, decode only; bf16 N(0,1) with 4 "
+            "key outlier channels x20",
+    "serving": "high-concurrency serving step: batch 256, seq_lens round(lognormal(ln 1024, 1.0)) "
+               "clipped to [64, 16384], 32 q / 8 kv heads, head_dim 128, page 16, one new token per "
+               "seq appended then decoded (fused step); bf16 N(0,1) with 4 key outlier channels "
+               "x U[10,30]",
+}
 
 
 def parse():
@@ -113,7 +122,11 @@ def append_bytes(num_tokens: int, hkv: int) -> int:
 # ---- clocks ----------------------------------------------------------------------------------
 
 class ClockSampler:
-    """Samples SM clock and clock-event reasons through NVML while running."""
+    """Samples SM clock and clock-event reasons through NVML while a timed loop runs.
+
+    The sampling thread lives for the whole benchmark but records only inside `with
+    sampler.timed():` blocks, so the record covers every timed region (the headline steps and
+    the per-kernel and per-line loops) and none of the set-up work between them."""
 
     REASONS = {
         "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4,
@@ -122,8 +135,9 @@ class ClockSampler:
         "display_clock_setting": 0x100,
     }
 
-    def __init__(self, device_index: int, period_s: float = 0.01):
+    def __init__(self, device_index: int, period_s: float = 0.005):
         self.samples, self.reasons, self.ok = [], set(), False
+        self.headline_samples = 0
         self.period = period_s
         try:
             import pynvml
@@ -135,36 +149,59 @@ class ClockSampler:
         except Exception:
             self.max_mhz = None
         self._stop = threading.Event()
+        self._active = threading.Event()
         self._t = None
 
-    def _run(self):
+    def _sample(self):
         nv = self.nv
-        while not self._stop.is_set():
-            try:
-                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
-                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
-                for name, b in self.REASONS.items():
-                    if bits & b and name != "gpu_idle":
-                        self.reasons.add(name)
-            except Exception:
-                pass
-            time.sleep(self.period)
+        try:
+            self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+            bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+            for name, b in self.REASONS.items():
+                if bits & b and name != "gpu_idle":
+                    self.reasons.add(name)
+        except Exception:
+            pass
 
-    def __enter__(self):
+    def _run(self):
+        while not self._stop.is_set():
+            if self._active.wait(0.05):
+                self._sample()
+                time.sleep(self.period)
+
+    def start(self):
         if self.ok:
             self._t = threading.Thread(target=self._run, daemon=True)
             self._t.start()
         return self
 
-    def __exit__(self, *exc):
+    def stop(self):
         self._stop.set()
+        self._active.set()
         if self._t is not None:
             self._t.join()
+
+    class _Timed:
+        def __init__(self, owner):
+            self.owner = owner
+
+        def __enter__(self):
+            if self.owner.ok:
+                self.owner._sample()          # at least one sample per region
+            self.owner._active.set()
+
+        def __exit__(self, *exc):
+            self.owner._active.clear()
+
+    def timed(self):
+        return ClockSampler._Timed(self)
 
     def summary(self):
         return {"sm_mhz": statistics.median(self.samples) if self.samples else None,
                 "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
-                "samples": len(self.samples), "source": "NVML during the timed region"}
+                "samples": len(self.samples), "headline_region_samples": self.headline_samples,
+                "source": "NVML every 5 ms inside every timed region of this run (the headline "
+                          "steps and each per-kernel / per-line timing loop)"}
 
 
 # ---- roofline denominators -----------------------------------------------------------------
@@ -214,9 +251,79 @@ def kernel_traffic(kernel: str, units: float):
         return None
 
 
+
+# ---- timing helpers ----------------------------------------------------------------------------
+
+MIN_LAUNCHES = 200        # per-launch loops: at least this many launches ...
+MIN_LOOP_SECONDS = 0.5    # ... and at least this long, whatever --steps is
+
+
+def loop_count(fn, stream, min_launches=MIN_LAUNCHES, min_seconds=MIN_LOOP_SECONDS, cap=20000):
+    """Launches a timing loop needs to reach both bounds (estimated from 10 back-to-back runs)."""
+    import torch
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(10):
+        fn()
+    e1.record(stream)
+    torch.cuda.synchronize()
+    est = max(e0.elapsed_time(e1) / 10 / 1e3, 1e-6)
+    return int(min(cap, max(min_launches, math.ceil(min_seconds / est))))
+
+
+def per_launch_ms(fn, stream, clocks, n=None):
+    """Mean CUDA-event duration of one call of fn (events around each call, on its stream)."""
+    import torch
+    for _ in range(3):
+        fn()
+    if n is None:
+        n = loop_count(fn, stream)
+    evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
+    torch.cuda.synchronize()
+    with clocks.timed():
+        for e in evs:
+            e[0].record(stream)
+            fn()
+            e[1].record(stream)
+        torch.cuda.synchronize()
+    return statistics.mean(e[0].elapsed_time(e[1]) for e in evs), n
+
+
+def back_to_back_ms(fn, stream, clocks, n=None, pg=None, dev="cpu"):
+    """Mean time of one call of fn in a loop of n back-to-back calls (one event pair), max over
+    ranks."""
+    import torch
+    for _ in range(3):
+        fn()
+    if n is None:
+        n = loop_count(fn, stream)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    with clocks.timed():
+        e0.record(stream)
+        for _ in range(n):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+    return max_over_ranks(e0.elapsed_time(e1) / n, pg, dev), n
+
+
+def host_cpu():
+    """The host's CPU model (from /proc/cpuinfo) and its logical CPU count."""
+    model = None
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    model = line.split(":", 1)[1].strip()
+                    break
+    except OSError:
+        pass
+    return model, os.cpu_count() or 1
+
 # ---- the CPU oracle baseline ------------------------------------------------------------
 
-def oracle_sample(wl, seed_seqs: int = CPU_SAMPLE_SEQS):
+def oracle_sample(wl, seed_seqs: int = CPU_SAMPLE_SEQS, nthreads=None):
     """Oracle-built history cache for the first `seed_seqs` sequences (CPU only)."""
     import oracle
     from bit_paged_kv_block_b200 import synth
@@ -226,14 +333,15 @@ def oracle_sample(wl, seed_seqs: int = CPU_SAMPLE_SEQS):
     sub.seq_lens = wl.seq_lens[sel].copy()
     sub.new_tokens = wl.new_tokens[sel].copy()
     sub.block_table = np.ascontiguousarray(wl.block_table[sel])
-    nthreads = os.cpu_count() or 1
+    if nthreads is None:
+        nthreads = os.cpu_count() or 1
     bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
     pages, scales = oracle.empty_cache(wl.num_pages, wl.num_kv_heads)
     seq, pos = synth.token_index(sub, "history")
     oracle.rotate_quantize_paged(bits(synth.kv_values(sub, "K", tokens="history")),
                                  bits(synth.kv_values(sub, "V", tokens="history")),
                                  synth.slot_mapping(sub, seq, pos), pages, scales,
-                                 nthreads=nthreads)
+                                 nthreads=os.cpu_count() or 1)
     seq, pos = synth.token_index(sub, "new")
     new = (bits(synth.kv_values(sub, "K", tokens="new")),
            bits(synth.kv_values(sub, "V", tokens="new")), synth.slot_mapping(sub, seq, pos))
@@ -248,20 +356,59 @@ def oracle_step(sub, pages, scales, new, q, nthreads):
                               nthreads=nthreads)
 
 
-def cpu_baseline(wl, min_seconds: float = 10.0):
-    sub, pages, scales, new, q, nthreads = oracle_sample(wl)
-    oracle_step(sub, pages, scales, new, q, nthreads)             # warm
+def _timed_reps(fn, min_seconds):
+    fn()                                               # warm
     reps, t0 = 0, time.perf_counter()
     while True:
-        oracle_step(sub, pages, scales, new, q, nthreads)
+        fn()
         reps += 1
         el = time.perf_counter() - t0
         if el >= min_seconds:
-            break
-    return {"value": sub.num_seqs * reps / el, "unit": UNIT, "cores": nthreads, "kind": "oracle",
-            "sample": f"first {sub.num_seqs} of the 64 sequences ({int(sub.seq_lens.sum())} "
-                      f"cached tokens): oracle append of their new tokens + fp64 decode, "
-                      f"{reps} repetitions in {el:.1f} s, OpenMP over {nthreads} host threads"}
+            return reps, el
+
+
+def cpu_baseline(wl, seconds_each: float = 6.0):
+    """The oracle as it stands on the host cores: the decode step on a sample of the decode
+    workload (all host threads, then one thread) and the rotate + quantize + scatter on a sample
+    of the prefill workload (same two thread counts)."""
+    import oracle
+    from bit_paged_kv_block_b200 import synth
+    model, ncpu = host_cpu()
+    out = {"unit": UNIT, "kind": "oracle", "cpu_model": model, "nproc": ncpu}
+    # decode step, all threads (8 sequences) and one thread (2 sequences)
+    for key, nseq, nth in (("all_cores", CPU_SAMPLE_SEQS, ncpu), ("single_thread", 2, 1)):
+        sub, pages, scales, new, q, nthreads = oracle_sample(wl, nseq, nthreads=nth)
+        reps, el = _timed_reps(lambda: oracle_step(sub, pages, scales, new, q, nthreads), seconds_each)
+        out[key] = {"value": sub.num_seqs * reps / el, "unit": UNIT, "cores": nthreads,
+                    "sample": f"first {sub.num_seqs} of the 64 sequences ({int(sub.seq_lens.sum())} "
+                              f"cached tokens): oracle append of their new tokens + fp64 decode, "
+                              f"{reps} repetitions in {el:.1f} s on {nthreads} thread(s)"}
+    out["value"] = out["all_cores"]["value"]
+    out["cores"] = out["all_cores"]["cores"]
+    out["sample"] = out["all_cores"]["sample"]
+    # rotate + quantize + scatter on the prefill workload's first 2 sequences (4096 tokens)
+    pre = synth.make_workload("prefill", seed=0)
+    sub = synth.Workload(**{**pre.__dict__})
+    sub.num_seqs = 2
+    sub.seq_lens = pre.seq_lens[:2].copy()
+    sub.new_tokens = pre.new_tokens[:2].copy()
+    sub.block_table = np.ascontiguousarray(pre.block_table[:2])
+    bits = lambda t: t.contiguous().view(__import__("torch").int16).numpy().view(np.uint16)
+    seq, pos = synth.token_index(sub, "all")
+    kb, vb = bits(synth.kv_values(sub, "K")), bits(synth.kv_values(sub, "V"))
+    slots = synth.slot_mapping(sub, seq, pos)
+    pages, scales = oracle.empty_cache(pre.num_pages, pre.num_kv_heads)
+    nbytes = append_bytes(len(seq), pre.num_kv_heads)
+    quant = {"workload": "prefill rotate + INT4 quantize + scatter (32 x 2048 tokens, 8 kv heads), "
+                         f"sample: its first 2 sequences ({len(seq)} tokens), same byte accounting "
+                         "as the GPU line", "unit": "GB/s"}
+    for key, nth in (("all_cores", ncpu), ("single_thread", 1)):
+        reps, el = _timed_reps(lambda: oracle.rotate_quantize_paged(kb, vb, slots, pages, scales,
+                                                                     nthreads=nth), seconds_each / 2)
+        quant[key] = {"GBps": nbytes * reps / el / 1e9, "cores": nth, "repetitions": reps,
+                      "seconds": el}
+    out["rot_quant"] = quant
+    return out
 
 
 def run_reference(args):
@@ -346,17 +493,18 @@ def run_saw(args):
     torch.cuda.synchronize()
 
     # ---- timed region: exactly K steps, device events, max over ranks ----------------------
-    clocks = ClockSampler(local_rank)
+    clocks = ClockSampler(local_rank).start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     if pg:
         pg.barrier()
     torch.cuda.synchronize()
-    with clocks:
+    with clocks.timed():
         e0.record(stream)
         for _ in range(args.steps):
             step()
         e1.record(stream)
         torch.cuda.synchronize()
+    clocks.headline_samples = len(clocks.samples)
     ms = e0.elapsed_time(e1)
     if pg:
         pg.barrier()
@@ -366,28 +514,72 @@ def run_saw(args):
     ms_per_step = ms / args.steps
     value = job_throughput(wl.num_seqs, world, ms_per_step)
 
-    # ---- per-kernel durations (same inputs, events around each launch) ---------------------
-    n_kt = max(20, min(args.steps, 400))
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(n_kt)]
-    for i in range(n_kt):
-        ev[i][0].record(stream)
-        saw.saw_rotate_quantize_paged(k_new, v_new, slots, kv, sc, dev_status=status,
-                                      stream=stream)
-        ev[i][1].record(stream)
-        saw.saw_paged_decode_attn(q, kv, sc, table, lens, out, ws, dev_status=status,
-                                  stream=stream)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize()
-    t_append = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    t_decode = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    # ---- per-kernel durations (same inputs, events around each launch, >= 200 launches and
+    # >= 0.5 s per loop whatever --steps is) ---------------------------------------------------
+    t_append, n_app = per_launch_ms(lambda: saw.saw_rotate_quantize_paged(
+        k_new, v_new, slots, kv, sc, dev_status=status, stream=stream), stream, clocks)
+    decode_call = lambda: saw.saw_paged_decode_attn(q, kv, sc, table, lens, out, ws,
+                                                    dev_status=status, stream=stream)
+    t_decode, n_kt = per_launch_ms(decode_call, stream, clocks)
     dec_bytes = decode_bytes(wl)
     peak_gbs, peak_kind = measured_peaks()
     dec_gbs = dec_bytes / (t_decode * 1e-3) / 1e9
     roofline = {"bound": "hbm", "achieved": dec_gbs, "peak": peak_gbs, "unit": "GB/s",
                 "frac": dec_gbs / peak_gbs, "peak_kind": peak_kind,
                 "kernel": "paged_decode_kernel", "algorithmic_bytes_per_launch": dec_bytes,
-                "launch_ms": t_decode, "frac_of_8TBps": dec_gbs / HBM_TARGET_GBS,
+                "launch_ms": t_decode, "launches_timed": n_kt,
+                "frac_of_8TBps": dec_gbs / HBM_TARGET_GBS,
                 "traffic": kernel_traffic("paged_decode_kernel", int(wl.seq_lens.sum()))}
+
+    # ---- the long-context and high-concurrency workloads: one line each ------------------------
+    def workload_line(name, fused):
+        """Decode-only (long context) or fused append + decode (serving) on another workload."""
+        w2 = synth.make_workload(name, seed=rank)
+        kv2, sc2 = saw.allocate_cache(w2.num_pages, w2.num_kv_heads, dev)
+        sq, sp = synth.token_index(w2, "history")
+        saw.saw_rotate_quantize_paged(synth.kv_values(w2, "K", tokens="history", device=dev),
+                                      synth.kv_values(w2, "V", tokens="history", device=dev),
+                                      torch.from_numpy(synth.slot_mapping(w2, sq, sp)).to(dev),
+                                      kv2, sc2)
+        sq, sp = synth.token_index(w2, "new")
+        kn2 = synth.kv_values(w2, "K", tokens="new", device=dev)
+        vn2 = synth.kv_values(w2, "V", tokens="new", device=dev)
+        sl2 = torch.from_numpy(synth.slot_mapping(w2, sq, sp)).to(dev)
+        q2 = synth.q_values(w2, device=dev)
+        tab2 = torch.from_numpy(w2.block_table).to(dev)
+        len2 = torch.from_numpy(w2.seq_lens).to(dev)
+        out2 = torch.empty((w2.num_seqs, w2.num_q_heads, 128), dtype=torch.float32, device=dev)
+        ws2 = saw.allocate_workspace(w2.num_kv_heads, w2.num_q_heads, w2.num_seqs, dev)
+        dec2 = lambda: saw.saw_paged_decode_attn(q2, kv2, sc2, tab2, len2, out2, ws2,
+                                                 dev_status=status, stream=stream)
+        if fused:
+            step2 = lambda: saw.saw_decode_step(q2, kn2, vn2, sl2, kv2, sc2, tab2, len2, out2, ws2,
+                                                dev_status=status, stream=stream)
+        else:
+            step2 = dec2
+        st_ms, st_n = back_to_back_ms(step2, stream, clocks, pg=pg, dev=dev)
+        d_ms, d_n = per_launch_ms(dec2, stream, clocks)
+        torch.cuda.synchronize()
+        if int(status.item()) != 0:
+            raise RuntimeError(f"device status {int(status.item()):#x} on {name}")
+        b2 = decode_bytes(w2)
+        g2 = b2 / (d_ms * 1e-3) / 1e9
+        step_bytes = b2 + (append_bytes(int(w2.new_tokens.sum()), w2.num_kv_heads) if fused else 0)
+        line2 = {"workload": WORKLOADS[name], "batch": w2.num_seqs,
+                 "kv_tokens": int(w2.seq_lens.sum()),
+                 "step": "append one new token per sequence + decode" if fused else "decode only",
+                 "step_ms": st_ms, "steps_timed": st_n,
+                 "tokens_per_s": job_throughput(w2.num_seqs, world, st_ms),
+                 "kv_tokens_per_s": world * int(w2.seq_lens.sum()) / (st_ms * 1e-3),
+                 "step_GBps": step_bytes / (st_ms * 1e-3) / 1e9,
+                 "launch_ms": d_ms, "launches_timed": d_n,
+                 "algorithmic_bytes_per_launch": b2, "decode_GBps": g2,
+                 "frac_of_measured_peak": g2 / peak_gbs, "frac_of_8TBps": g2 / HBM_TARGET_GBS}
+        del kv2, sc2, kn2, vn2, q2, out2, ws2
+        return line2
+
+    long_ctx = workload_line("long", fused=False)
+    serving = workload_line("serving", fused=True)
 
     # ---- prefill rotate+quantize throughput (the write side at full bandwidth) -------------
     pre = synth.make_workload("prefill", seed=rank)
@@ -396,39 +588,23 @@ def run_saw(args):
     pk = synth.kv_values(pre, "K", device=dev)
     pv = synth.kv_values(pre, "V", device=dev)
     pslots = torch.from_numpy(synth.slot_mapping(pre, pseq, ppos)).to(dev)
-    for _ in range(3):
-        saw.saw_rotate_quantize_paged(pk, pv, pslots, pkv, psc, stream=stream)
-    n_rq = 50
-    evq = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n_rq)]
-    for i in range(n_rq):
-        evq[i][0].record(stream)
-        saw.saw_rotate_quantize_paged(pk, pv, pslots, pkv, psc, stream=stream)
-        evq[i][1].record(stream)
-    torch.cuda.synchronize()
-    t_rq = statistics.mean(e[0].elapsed_time(e[1]) for e in evq)
+    t_rq, n_rq = per_launch_ms(lambda: saw.saw_rotate_quantize_paged(pk, pv, pslots, pkv, psc,
+                                                                     stream=stream), stream, clocks)
     rq_bytes = append_bytes(pre.total_tokens, pre.num_kv_heads)
     rq_gbs = rq_bytes / (t_rq * 1e-3) / 1e9
     rot_quant = {"workload": "prefill: 32 seqs x 2048 tokens, 8 kv heads, head_dim 128, page 16, "
                              "pages by seeded permutation",
                  "GBps": rq_gbs, "frac_of_8TBps": rq_gbs / HBM_TARGET_GBS,
                  "frac_of_measured_peak": rq_gbs / peak_gbs, "launch_ms": t_rq,
-                 "algorithmic_bytes_per_launch": rq_bytes,
+                 "launches_timed": n_rq, "algorithmic_bytes_per_launch": rq_bytes,
                  "traffic": kernel_traffic("rotate_quantize_kernel", pre.total_tokens)}
 
     # ---- the plain INT4 baseline (no rotation) on the same workloads: rotation overhead -------
-    def mean_event_ms(fn, n):
-        evs = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(n)]
-        for e in evs:
-            e[0].record(stream)
-            fn()
-            e[1].record(stream)
-        torch.cuda.synchronize()
-        return statistics.mean(e[0].elapsed_time(e[1]) for e in evs)
+    def mean_event_ms(fn, n=None):
+        return per_launch_ms(fn, stream, clocks, n)[0]
 
-    for _ in range(3):
-        saw.saw_quantize_paged_plain(pk, pv, pslots, pkv, psc, stream=stream)
     t_rq_plain = mean_event_ms(lambda: saw.saw_quantize_paged_plain(pk, pv, pslots, pkv, psc,
-                                                                    stream=stream), n_rq)
+                                                                    stream=stream))
     del pk, pv, pkv, psc
     pkv2, psc2 = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
     seq, pos = synth.token_index(wl, "history")
@@ -438,16 +614,7 @@ def run_saw(args):
                                  pkv2, psc2)
     plain_step = lambda: saw.saw_decode_step_plain(q, k_new, v_new, slots, pkv2, psc2, table, lens,
                                                    out, ws, dev_status=status, stream=stream)
-    for _ in range(3):
-        plain_step()
-    torch.cuda.synchronize()
-    n_pl = max(20, min(args.steps, 2000))
-    e0.record(stream)
-    for _ in range(n_pl):
-        plain_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    pl_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
+    pl_ms, _ = back_to_back_ms(plain_step, stream, clocks, pg=pg, dev=dev)
     plain_int4 = {"what": "the same step and prefill quantize on a plain INT4 cache (H = I)",
                   "step_ms": pl_ms, "tokens_per_s": job_throughput(wl.num_seqs, world, pl_ms),
                   "step_rotation_overhead": ms_per_step / pl_ms - 1.0,
@@ -464,17 +631,9 @@ def run_saw(args):
     wsb = saw.allocate_workspace_bf16(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
     bf16_step = lambda: saw.saw_decode_step_bf16(q, k_new, v_new, slots, kvb, table, lens, out, wsb,
                                                  dev_status=status, stream=stream)
-    for _ in range(3):
-        bf16_step()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(n_pl):
-        bf16_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    bf_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
+    bf_ms, _ = back_to_back_ms(bf16_step, stream, clocks, pg=pg, dev=dev)
     t_dec_bf16 = mean_event_ms(lambda: saw.saw_paged_decode_attn_bf16(
-        q, kvb, table, lens, out, wsb, dev_status=status, stream=stream), n_kt)
+        q, kvb, table, lens, out, wsb, dev_status=status, stream=stream))
     bf_gbs = decode_bytes_bf16(wl) / (t_dec_bf16 * 1e-3) / 1e9
     bf16_baseline = {"what": "the same step on an uncompressed bf16 paged cache (4x the KV bytes)",
                      "step_ms": bf_ms, "tokens_per_s": job_throughput(wl.num_seqs, world, bf_ms),
@@ -505,7 +664,7 @@ def run_saw(args):
                                                 dev_status=status, stream=stream)
     for _ in range(3):
         run_pf()
-    t_pf = mean_event_ms(run_pf, max(5, min(args.steps, 50)))
+    t_pf = mean_event_ms(run_pf)
     g = pfl.num_q_heads // pfl.num_kv_heads
     # the tensor-core kernel's tiles: 128 / G query tokens each, reading their causal range
     tile_tok = 128 // g
@@ -550,7 +709,7 @@ def run_saw(args):
                                                    dev_status=status, stream=stream)
         for _ in range(3):
             run_d4()
-        t_d4 = mean_event_ms(run_d4, n_kt)
+        t_d4 = mean_event_ms(run_d4)
         d4_gbs = decode_bytes(whd) / (t_d4 * 1e-3) / 1e9
         head_dims[f"head_dim_{hd}"] = {
             "workload": f"the decode batch (same lengths and heads) at head_dim {hd}",
@@ -582,16 +741,8 @@ def run_saw(args):
                                                   out, wsw, dev_status=status, stream=stream)
     win_decode = lambda: saw.saw_paged_decode_attn_window(q, win, wkv5, wsc5, table, lens, out, wsw,
                                                           dev_status=status, stream=stream)
-    for _ in range(3):
-        win_step()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(n_pl):
-        win_step()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    win_ms = max_over_ranks(e0.elapsed_time(e1) / n_pl, pg, dev)
-    t_wdec = mean_event_ms(win_decode, n_kt)
+    win_ms, _ = back_to_back_ms(win_step, stream, clocks, pg=pg, dev=dev)
+    t_wdec = mean_event_ms(win_decode)
     win_tokens = int(np.minimum(wl.seq_lens, W).sum())
     win_bytes = (decode_bytes(wl) - wl.num_kv_heads * win_tokens * 136
                  + wl.num_kv_heads * win_tokens * 512)
@@ -655,16 +806,18 @@ def run_saw(args):
 
     for i in range(4):
         e2e_step(i)
-    n_e2e = max(20, min(args.steps, 2000))
+    n_e2e = loop_count(step, stream)
+    n_e2e += n_e2e & 1
     torch.cuda.synchronize()
-    e0.record(stream)
-    s_in.wait_event(e0)
-    s_out.wait_event(e0)
-    for i in range(n_e2e):
-        e2e_step(i)
-    stream.wait_stream(s_out)
-    e1.record(stream)
-    torch.cuda.synchronize()
+    with clocks.timed():
+        e0.record(stream)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i in range(n_e2e):
+            e2e_step(i)
+        stream.wait_stream(s_out)
+        e1.record(stream)
+        torch.cuda.synchronize()
     e2e_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, pg, dev)
     # the same copies and step without overlap (one stream: copy in, step, copy out), for context
     def e2e_serial():
@@ -674,15 +827,7 @@ def run_saw(args):
                             dev_status=status, stream=stream)
         h_out[0].copy_(d_out[0], non_blocking=True)
 
-    for _ in range(3):
-        e2e_serial()
-    torch.cuda.synchronize()
-    e0.record(stream)
-    for _ in range(n_e2e):
-        e2e_serial()
-    e1.record(stream)
-    torch.cuda.synchronize()
-    serial_ms = max_over_ranks(e0.elapsed_time(e1) / n_e2e, pg, dev)
+    serial_ms, _ = back_to_back_ms(e2e_serial, stream, clocks, n=n_e2e, pg=pg, dev=dev)
     step()   # the device-only step on the same inputs, for the check below
     torch.cuda.synchronize()
     e2e_matches = bool(torch.equal(h_out[(n_e2e - 1) & 1], out.cpu()))
@@ -696,6 +841,7 @@ def run_saw(args):
            "serial": {"value": job_throughput(wl.num_seqs, world, serial_ms), "ms_per_step": serial_ms,
                       "how": "the same two copies and step on one stream, no overlap"}}
 
+    clocks.stop()
     base = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         base = cpu_baseline(wl)
@@ -712,7 +858,12 @@ def run_saw(args):
         "kv_tokens_per_s": world * int(wl.seq_lens.sum()) / (ms_per_step / 1e3),
         "step_GBps": (dec_bytes + append_bytes(wl.num_seqs, wl.num_kv_heads)) / (ms_per_step * 1e-3) / 1e9,
         "roofline": roofline,
+        "rot_quant_GBps": rq_gbs,
+        "rot_quant_frac": rq_gbs / peak_gbs,
+        "rot_quant_frac_of_8TBps": rq_gbs / HBM_TARGET_GBS,
         "rot_quant": rot_quant,
+        "long_context": long_ctx,
+        "serving": serving,
         "plain_int4": plain_int4,
         "bf16_baseline": bf16_baseline,
         "prefill_attn": prefill_attn,

@@ -34,7 +34,8 @@ constexpr int kMaxDevices = 64;
 std::mutex g_setup_mutex;
 void *g_scratch_ptr[kMaxDevices] = {};
 
-// Device address of g_decode_scratch on the current device, looked up once per device.
+// Device address of g_decode_scratch on the current device, looked up once per device and kept
+// for the life of the process (a device reset would invalidate it; the header says so).
 // In host code the symbol is only a host-side stand-in; the real address comes from
 // cudaGetSymbolAddress with that device current.
 int scratch_address(void **out)

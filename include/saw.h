@@ -263,7 +263,10 @@ int saw_decode_step_bf16(const saw_cache_desc *cache, int32_t num_q_heads, const
  * twice as large: about 550 segments on a B200); larger shapes return SAW_ERR_SCRATCH_LIMIT
  * before anything is queued.
  * The first call on each device looks up the array's device address (cudaGetSymbolAddress with
- * that device current); make that first call before any stream capture.  Nothing in the array
+ * that device current) and keeps it for the life of the process; make that first call before
+ * any stream capture.  A cudaDeviceReset (or any other teardown of the device's primary
+ * context) invalidates the kept address: do not call this entry point on that device after
+ * one.  Nothing in the array
  * needs to start at zero.  All calls on a device share the array and it keeps the previous
  * call's contents, so calls that can overlap on the GPU (other streams, other host threads)
  * race on it: the caller must serialise them.
