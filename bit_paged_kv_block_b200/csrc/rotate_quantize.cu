@@ -10,24 +10,27 @@
 //   * the butterfly performs exactly the IEEE fp32 adds/subtracts of the natural-order
 //     Sylvester transform, stage h = 1, 2, ..., 64 in that order, then one multiply by
 //     fp32(1/sqrt(128)); two fp32 operations are issued per packed f32x2 instruction, each
-//     individually rounded, so the lane layout does not change any result;
-//   * scale = (max - min) / 15 uses the IEEE divide; the codes use a reciprocal (the note
-//     above code_bits_tie() shows why that gives the IEEE-divide code) and fall back to the
-//     IEEE divide where it might not.
+//     individually rounded, so the register layout does not change any result;
+//   * scale = (max - min) / 15 is the IEEE quotient (computed by a three-operation sequence
+//     checked against the IEEE divide for every non-negative fp32 dividend, below); each code is
+//     read off one fused multiply-add on a 2^-16 grid, which is provably the IEEE-divide code
+//     except where the grid value is exactly half-way between two codes; those rare elements
+//     are settled by an exact remainder test (note above code_at_half()).
 // This translation unit is compiled with -fmad=false as a second guard against contraction.
 //
-// Data movement: every warp streams its own tiles of 8 consecutive (token, kv head) vectors of K
-// and of V (2 KiB each) into a private 3-stage shared-memory ring with 2-D tensor copies (TMA,
-// 128-byte swizzle) completing on mbarriers, so warps never wait for each other.  The warps of
-// the persistent grid take tiles round-robin.
+// Data movement: every warp streams its own tiles of 16 rows of 128 bytes (64 bf16 elements) of K
+// and the same 16 rows of V into a private 3-stage shared-memory ring with tensor copies (TMA,
+// 128-byte swizzle) completing on mbarriers, so warps never wait for each other.  The warps of the
+// persistent grid take tiles round-robin.
 //
-// Thread layout (D = 128; D = 256 uses two such pairs per vector, one per 128-block, and D = 64
-// one thread per whole vector, 16 vectors of K and 16 of V per tile, the butterfly entirely in
-// registers): two threads per head vector; a warp's tile has its 8 K vectors in lanes 0-15
-// and its 8 V vectors in lanes 16-31.  Thread half b of a vector holds the 64 elements
-// j = 16a + 8b + r (a, r in 0..7), read as eight 16-byte shared-memory loads that the 128-byte
-// swizzle spreads over all banks.  Stage h = 8 is the only one that crosses the pair (one
-// shuffle); the 64 elements are kept as 32 packed pairs X[8a + r] = (x[a][r], x[a + 4][r]).
+// Thread layout: one thread per 64-element row; lanes 0-15 take the tile's K rows and lanes 16-31
+// its V rows.  A thread keeps its row as packed pairs X[m] = (x[m], x[m + 32]), so butterfly
+// stages h = 1 .. 16 of its 64 elements run on packed f32x2 instructions and stage h = 32 pairs the
+// two halves of each register.  D = 64: that is the whole transform.  D = 128 and 256: a row is half
+// of a 128-point block and stage h = 64 pairs lane r with lane r ^ 1; the two lanes swap their 64
+// values by shuffles and each forms its own half of the stage's outputs: x + partner (lower row) or
+// partner - x = fma(x, -1, partner), one IEEE rounding either way.  min / max combine over the
+// vector's lanes by shuffles.
 #include <cfloat>
 #include <algorithm>
 
@@ -37,91 +40,65 @@
 namespace saw {
 namespace {
 
-constexpr int kTileBytes = 2048;                       // K (or V) bytes of one warp tile: 16 rows
+constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
+constexpr float kHadamardC64 = 0.125f;               // 1/sqrt(64), exact
+constexpr float kInv15 = 1.0f / 15.0f;               // RN(1/15)
+// Codes are read off t = RN(d * 2^16 / s + kGridMagic): t lies in [2^23, 2^24), where the fp32
+// spacing is 1, so t = 2^23 + 2^15 + N with N = rint(d * 2^16 / s) (the 2^-16 grid value of the
+// quotient) and bits 16..19 of t hold floor(grid + 1/2).
+constexpr float kGridMagic = 8421376.0f;             // 2^23 + 2^15
+constexpr float kFastScaleMin = 0x1p-100f;           // scales outside [2^-100, 2^100] divide
+constexpr float kFastScaleMax = 0x1p100f;
+constexpr uint64_t kRqWaitLimitNs = 1000000000ull;
+
 // Head dimension D = 64 (the 64-point transform: no 128-point block fits), 128, or 256 (two
-// independent 128-point rotation blocks): a warp tile holds 2048 / (2 D) vectors of K and as
-// many of V, D / 64 threads per vector, each thread 64 elements of one rotation block; a vector
-// is D / 64 tensor-map rows of 128 bytes.
+// independent 128-point rotation blocks).  A thread holds one 64-element row (kN = 32 packed pairs);
+// a vector is kThreadsPerVec rows; a warp tile is 16 rows of K and the same 16 rows of V.
 template <int kD>
 struct RqDims {
     static_assert(kD == 64 || kD == 128 || kD == 256, "head dimension");
-    static constexpr int kTileVecs = kTileBytes / (2 * kD);   // 16, 8 or 4
+    static constexpr int kN = 32;                              // packed registers per thread
     static constexpr int kThreadsPerVec = kD / 64;             // 1, 2 or 4
-    static constexpr int kRowsPerVec = kD / 64;                // 128-byte rows per vector
+    static constexpr int kTileVecs = 16 / kThreadsPerVec;      // 16, 8 or 4
+    static constexpr int kHalfBytes = 2048;                    // K (or V) bytes of one tile
+    static constexpr int kStageBytes = 2 * kHalfBytes;
     static constexpr int kCodeBytes = kD / 2;                  // packed codes per vector
 };
 constexpr int kRqStages = 3;
 constexpr int kRqWarps = 4;
 constexpr int kRqThreads = 32 * kRqWarps;
-constexpr int kRqStageBytes = 2 * kTileBytes;
-constexpr int kRqSmemBars = kRqWarps * kRqStages * kRqStageBytes;
-constexpr size_t kRqSmemBytes = 1024 + kRqSmemBars + kRqWarps * kRqStages * 8;
-constexpr uint64_t kRqWaitLimitNs = 1000000000ull;
-constexpr float kHadamardC = 0.0883883461356163f;   // fp32(1/sqrt(128)) = 0x3DB504F3
-constexpr float kHadamardC64 = 0.125f;               // 1/sqrt(64), exact
-constexpr float kRoundMagic = 12582912.0f;           // 1.5 * 2^23
-// A code computed from the reciprocal is provably the IEEE-divide code unless the remainder
-// is within 2^-18 of one half (derivation above code_bits_tie()).
-constexpr float kNearHalf = 0.5f - 1.0f / 262144.0f;
-
-__device__ __forceinline__ uint64_t shfl_xor_u64(uint32_t mask, uint64_t v, int delta)
+template <int kD>
+__host__ __device__ constexpr size_t rq_smem_bytes()
 {
-    uint32_t lo = static_cast<uint32_t>(v), hi = static_cast<uint32_t>(v >> 32);
-    lo = __shfl_xor_sync(mask, lo, delta);
-    hi = __shfl_xor_sync(mask, hi, delta);
-    return (static_cast<uint64_t>(hi) << 32) | lo;
+    return 1024 + size_t(kRqWarps) * kRqStages * RqDims<kD>::kStageBytes + kRqWarps * kRqStages * 8;
 }
 
-__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(__byte_perm(u, 0, 0x1044)); }
 __device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
 
-
-// This thread's 64 bf16 elements of 128-block blk of tile vector vt (rows (D / 64) vt + 2 blk
-// and the next of 128 bytes; the 16-byte chunk c of row r sits at chunk c ^ (r & 7) under the
-// 128-byte swizzle).
-template <int kD>
-__device__ __forceinline__ void load_half_vec(uint32_t tile, int vt, int blk, int b, uint4 raw[8])
+// Packed pairs X[8 c .. 8 c + 7] of one block from 16-byte chunk c of its elements 0 .. kN - 1
+// (`lo`) and of its elements kN .. 2 kN - 1 (`hi`): X[m] = (x[m], x[m + kN]).
+__device__ __forceinline__ void pairs_from_chunk(uint4 lo, uint4 hi, uint64_t X[8])
 {
+    const uint32_t a[4] = {lo.x, lo.y, lo.z, lo.w};
+    const uint32_t b[4] = {hi.x, hi.y, hi.z, hi.w};
 #pragma unroll
-    for (int a = 0; a < 8; a++) {
-        const int row = RqDims<kD>::kRowsPerVec * vt + 2 * blk + (a >> 2);
-        const int chunk = (2 * (a & 3) + b) ^ (row & 7);
-        raw[a] = lds128(tile + row * 128 + chunk * 16);
+    for (int k = 0; k < 4; k++) {
+        X[2 * k] = f2_pack(bf16_lo(a[k]), bf16_lo(b[k]));
+        X[2 * k + 1] = f2_pack(bf16_hi(a[k]), bf16_hi(b[k]));
     }
 }
 
-// D = 64: this thread's whole vector vt of the tile, one 128-byte row (chunk a = elements
-// 8a .. 8a + 7 at chunk a ^ (vt & 7) under the 128-byte swizzle).
-__device__ __forceinline__ void load_vec64(uint32_t tile, int vt, uint4 raw[8])
+// The butterfly stages of the 2 kN elements one thread holds: stages h = 1 .. kN / 2 pair
+// registers m and m + h (packed, two IEEE operations per instruction), stage h = kN pairs the two
+// halves of each register.  Stages run in ascending h; low index gets a + b, high index a - b.
+template <int kN>
+__device__ __forceinline__ void fwht_stages(uint64_t X[kN])
 {
 #pragma unroll
-    for (int a = 0; a < 8; a++)
-        raw[a] = lds128(tile + vt * 128 + ((a ^ (vt & 7)) << 4));
-}
-
-__device__ __forceinline__ void to_pairs(const uint4 raw[8], uint64_t X[32])
-{
+    for (int hb = 1; hb < kN; hb <<= 1) {
 #pragma unroll
-    for (int a = 0; a < 4; a++) {
-        const uint32_t lo[4] = {raw[a].x, raw[a].y, raw[a].z, raw[a].w};
-        const uint32_t hi[4] = {raw[a + 4].x, raw[a + 4].y, raw[a + 4].z, raw[a + 4].w};
-#pragma unroll
-        for (int q = 0; q < 4; q++) {
-            X[8 * a + 2 * q] = f2_pack(bf16_lo(lo[q]), bf16_lo(hi[q]));
-            X[8 * a + 2 * q + 1] = f2_pack(bf16_hi(lo[q]), bf16_hi(hi[q]));
-        }
-    }
-}
-
-// Normalised 128-point Hadamard transform of the vector held by a thread pair.
-// `mask` names the lanes executing this call (the full warp, or just this pair).
-__device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
-{
-    // h = 1, 2, 4: element bits r0..r2 = index bits 0..2 of X.
-#pragma unroll
-    for (int hb = 1; hb <= 4; hb <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
+        for (int i = 0; i < kN; i++) {
             if ((i & hb) == 0) {
                 const uint64_t lo = X[i], hi = X[i + hb];
                 X[i] = f2_add(lo, hi);
@@ -129,134 +106,236 @@ __device__ __forceinline__ void fwht128(uint64_t X[32], int b, uint32_t mask)
             }
         }
     }
-    // h = 8: element bit 3 = the pair half b.  Low half: x + partner; high half:
-    // partner - x, computed as fma(x, -1, partner): the product is exact, so the single
-    // rounding gives exactly the IEEE difference.
-    {
-        const float sg = b ? -1.0f : 1.0f;
-        const uint64_t sgn = f2_pack(sg, sg);
 #pragma unroll
-        for (int i = 0; i < 32; i++) {
-            const uint64_t other = shfl_xor_u64(mask, X[i], 1);
-            X[i] = f2_fma(X[i], sgn, other);
-        }
-    }
-    // h = 16, 32: element bits a0, a1 = index bits 3, 4 of X.
-#pragma unroll
-    for (int hb = 8; hb <= 16; hb <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-            if ((i & hb) == 0) {
-                const uint64_t lo = X[i], hi = X[i + hb];
-                X[i] = f2_add(lo, hi);
-                X[i + hb] = f2_sub(lo, hi);
-            }
-        }
-    }
-    // h = 64: element bit a2 = the two halves of each packed pair.
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
+    for (int i = 0; i < kN; i++) {
         float lo, hi;
         f2_unpack(X[i], lo, hi);
         X[i] = f2_pack(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
     }
-    const uint64_t cc = f2_pack(kHadamardC, kHadamardC);
+}
+
+template <int kN>
+__device__ __forceinline__ void scale_all(uint64_t X[kN], float c)
+{
+    const uint64_t cc = f2_pack(c, c);
 #pragma unroll
-    for (int i = 0; i < 32; i++)
+    for (int i = 0; i < kN; i++)
         X[i] = f2_mul(X[i], cc);
 }
 
-// Normalised 64-point Hadamard transform of the vector one thread holds as X[8 a + r] =
-// (x[8 a + r], x[8 (a + 4) + r]) (a < 4, r < 8): element bits 0-2 are index bits 0-2 of X
-// (h = 1, 2, 4), bits 3-4 index bits 3-4 (h = 8, 16), bit 5 the halves of each pair (h = 32);
-// then the multiply by 1/8.  The stages run in ascending h, every operation one IEEE fp32 op.
-__device__ __forceinline__ void fwht64(uint64_t X[32])
+// The normalised Hadamard transform of a block one thread holds whole (2 kN points): the stages,
+// then every element times fp32(1/sqrt(2 kN)).
+template <int kN>
+__device__ __forceinline__ void fwht_block(uint64_t X[kN])
 {
-#pragma unroll
-    for (int hb = 1; hb <= 16; hb <<= 1) {
-#pragma unroll
-        for (int i = 0; i < 32; i++) {
-            if ((i & hb) == 0) {
-                const uint64_t lo = X[i], hi = X[i + hb];
-                X[i] = f2_add(lo, hi);
-                X[i + hb] = f2_sub(lo, hi);
-            }
-        }
-    }
+    fwht_stages<kN>(X);
+    scale_all<kN>(X, kN == 64 ? kHadamardC : kHadamardC64);
+}
+
+// Stage h = 64 of a 128-point block split over lanes L (elements 0..63, b = 0) and L ^ 1 (elements
+// 64..127, b = 1): each lane takes its partner's 64 values by shuffles and forms its own half of the
+// stage's outputs: x + partner (lower lane) or partner - x = fma(x, -1, partner) (upper lane).  The
+// product is exact, so either is one IEEE rounding of the stage's sum or difference.
+__device__ __forceinline__ void exchange_stage64(uint64_t X[32], int b)
+{
+    const float sg = b ? -1.0f : 1.0f;
+    const uint64_t sgn = f2_pack(sg, sg);
 #pragma unroll
     for (int i = 0; i < 32; i++) {
         float lo, hi;
         f2_unpack(X[i], lo, hi);
-        X[i] = f2_pack(__fadd_rn(lo, hi), __fsub_rn(lo, hi));
+        const uint64_t other = f2_pack(__shfl_xor_sync(0xFFFFFFFFu, lo, 1),
+                                       __shfl_xor_sync(0xFFFFFFFFu, hi, 1));
+        X[i] = f2_fma(X[i], sgn, other);
     }
-    const uint64_t cc = f2_pack(kHadamardC64, kHadamardC64);
+}
+
+// min / max over the thread's elements (4 independent chains of three-input min / max)
+template <int kN>
+__device__ __forceinline__ void block_min_max(const uint64_t X[kN], float &mn, float &mx)
+{
+    float mns[4], mxs[4];
 #pragma unroll
-    for (int i = 0; i < 32; i++)
-        X[i] = f2_mul(X[i], cc);
-}
-
-// Codes via the reciprocal.  With s = scale (a normal fp32 > 0), r = RN(1/s), d = RN(y - min)
-// and Q = d / s exactly (0 <= Q < 15 (1 + 2^-23)):
-//   t = RN(d r + M), M = 1.5 * 2^23: d r < 2^22, so t = M + k with k = rint(d r) (ties to even,
-//   since M is even) and k sits in the low mantissa bits of t;
-//   res = RN(d r - k) is the remainder to within 2^-26.
-// |d r - Q| <= Q 2^-24 < 2^-20 and |RN(Q) - Q| <= 2^-21, so if |res| < 0.5 - 2^-18 then
-// |RN(Q) - k| < 0.5 and rint(RN(d / s)) = k, which is the code the IEEE divide gives (no
-// clamp is needed: k <= 15).  Otherwise the code is decided as follows.
-//
-// Near a half-way quotient the code follows from the sign of one exact remainder instead of a
-// divide.  Let m = k +- 1/2 be the half-integer next to Q (0.5 <= m <= 14.5, since 0 <= Q <=
-// 15 (1 + 2^-23)) and E = d - m s.  RN(Q) = m exactly when |Q - m| <= ulp(m) / 2 (m has an even
-// last mantissa bit, so a tie also rounds to m), i.e. when |E| <= T = s ulp(m) / 2; then the
-// code is rint(m), the even neighbour.  Otherwise RN(Q) lies on the same side of m as Q and the
-// code is m + sign(E) / 2.  E is a multiple of ulp(s) / 4 (d and m s both are), and where
-// |E| <= 2 T it has at most 7 significant bits, so RN(E) = fma(-m, s, d) is E itself; where
-// |E| > 2 T, |RN(E)| >= 2 T.  The test |RN(E)| <= T is therefore exact, as are T (a power-of-two
-// multiple of s) and the sign, for s >= 2^-100; smaller scales divide.
-constexpr float kRemainderMinScale = 0x1p-100f;
-
-// Bits of M + code for an element whose reciprocal remainder `res` lies near one half (or any
-// element, for a subnormal scale: `fast` false), by the remainder test above, or by the IEEE
-// divide for scales below 2^-100.  Out of line: it runs for about one element in a thousand
-// of unrotated bf16 data and almost never for rotated data, and the many inlined call sites
-// stay small.
-__device__ __noinline__ uint32_t code_bits_tie(float d, float k, float res, float s, bool fast)
-{
-    float code;
-    if (fast && s >= kRemainderMinScale) {
-        const float m = __fadd_rn(k, copysignf(0.5f, res));
-        const float e = __fmaf_rn(-m, s, d);
-        const float half_ulp = __int_as_float((__float_as_int(m) & 0x7F800000) - (24 << 23));
-        code = fabsf(e) <= __fmul_rn(s, half_ulp) ? m : __fadd_rn(m, copysignf(0.5f, e));
-    } else {
-        code = fminf(fmaxf(rintf(__fdiv_rn(d, s)), 0.0f), 15.0f);
+    for (int i = 0; i < 4; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        mns[i] = fminf(lo, hi);
+        mxs[i] = fmaxf(lo, hi);
     }
-    return __float_as_uint(__fadd_rn(code, kRoundMagic));   // m + M: a tie goes to even
+#pragma unroll
+    for (int i = 4; i < kN; i++) {
+        float lo, hi;
+        f2_unpack(X[i], lo, hi);
+        mns[i & 3] = fmin3(mns[i & 3], lo, hi);
+        mxs[i & 3] = fmax3(mxs[i & 3], lo, hi);
+    }
+    mn = fmin3(mns[0], mns[1], fminf(mns[2], mns[3]));
+    mx = fmax3(mxs[0], mxs[1], fmaxf(mxs[2], mxs[3]));
 }
 
-// Bits of M + code for element value y, given the reciprocal result t_bits (M + k).
-__device__ __forceinline__ uint32_t code_bits_exact(float y, uint32_t t_bits, float mn, float s,
-                                                    float r, bool fast)
+// RN(x / 15) for x >= 0: q0 = RN(x c), e = x - 15 q0 (exact in one fma), q1 = RN(q0 + e c) with
+// c = RN(1/15) -- the correction step of P. Markstein, "Computation of elementary functions on the
+// IBM RISC System/6000 processor" (IBM J. Res. Dev. 34(1), 1990).  Checked exhaustively on the
+// host: q1 equals the IEEE quotient for all 2^31 - 2^23 non-negative finite fp32 x.
+__device__ __forceinline__ float div15(float x)
 {
+    const float q0 = __fmul_rn(x, kInv15);
+    const float e = __fmaf_rn(-q0, 15.0f, x);
+    return __fmaf_rn(e, kInv15, q0);
+}
+
+// 2^16 / s with relative error below 2^-23, for 2^-100 <= s <= 2^100: the hardware reciprocal
+// (max error 1 ulp) refined by one Newton-Raphson step, scaled by 2^16 exactly.
+__device__ __forceinline__ float recip_2p16(float s)
+{
+    float r0;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r0) : "f"(s));
+    const float e = __fmaf_rn(-s, r0, 1.0f);
+    const float r0s = __fmul_rn(r0, 65536.0f);
+    return __fmaf_rn(r0s, e, r0s);
+}
+
+// Codes from grid values.  With Q = d / s (exact), r16 = (2^16 / s)(1 + e),
+// |e| < 2^-23, and t = RN(d r16 + 2^23 + 2^15) = 2^23 + 2^15 + N, N = rint(d r16):
+//   |N / 2^16 - Q| <= 2^-17 + 15.0001 * 2^-23 < 0.65 * 2^-16, and |RN(Q) - Q| <= 2^-21 (Q < 16),
+// so the grid value g = N / 2^16 lies within 2^-16 of RN(Q).  g + 1/2 is a multiple of 2^-16: if
+// it is not an integer it is at least 2^-16 from every integer, RN(Q) + 1/2 lies strictly between
+// the same two integers, and rint(RN(Q)) = floor(g + 1/2) = bits 16..19 of t (never more than
+// 15).  If it is an integer K (the low 16 bits of t are 0), m = K - 1/2 is the half-integer next
+// to Q (0.5 <= m <= 14.5) and the code follows from the sign of one exact remainder: let
+// E = d - m s; RN(Q) = m exactly when |Q - m| <= ulp(m) / 2 (m has an even last mantissa bit, so a
+// tie also rounds to m), i.e. when |E| <= T = s ulp(m) / 2, and then the code is rint(m) (ties to
+// even); otherwise RN(Q) lies on the same side of m as Q and the code is m + sign(E) / 2.  E is a
+// multiple of ulp(s) / 4 (d and m s both are), and where |E| <= 2 T it has at most 7 significant
+// bits, so RN(E) = fma(-m, s, d) is E itself; where |E| > 2 T, |RN(E)| >= 2 T.  The test
+// |RN(E)| <= T is therefore exact, as are T (a power-of-two multiple of s) and the sign, for
+// s >= 2^-100.  code_at_half() returns the code of element value y (d = y - min) whose t has zero
+// low bits.
+__device__ __noinline__ uint32_t code_at_half(float y, float mn, float s, uint32_t t_bits)
+{
+    const uint32_t cand = (t_bits >> 16) & 15u;
     const float d = __fsub_rn(y, mn);
-    const float k = __fsub_rn(__uint_as_float(t_bits), kRoundMagic);
-    const float res = __fmaf_rn(d, r, -k);
-    if (fast && fabsf(res) < kNearHalf)
-        return t_bits;
-    return code_bits_tie(d, k, res, s, fast);
+    const float m = __fsub_rn(static_cast<float>(cand), 0.5f);
+    const float e = __fmaf_rn(-m, s, d);
+    const float half_ulp = __int_as_float((__float_as_int(m) & 0x7F800000) - (24 << 23));
+    const float code = fabsf(e) <= __fmul_rn(s, half_ulp) ? rintf(m) : __fadd_rn(m, copysignf(0.5f, e));
+    return static_cast<uint32_t>(code);
 }
 
-// Gather the low nibbles of t_0..t_7 (codes of elements r = 0..7) into one word, element r at
-// bits 4r: bytes are [k0 | k1 << 4, k2 | k3 << 4, ...] (even index in the low nibble).
-__device__ __forceinline__ uint32_t pack8(const uint32_t tt[8])
+// The IEEE-divide code (scales outside [2^-100, 2^100]).
+__device__ __noinline__ uint32_t code_by_divide(float y, float mn, float s)
 {
-    const uint32_t e01 = __byte_perm(tt[0], tt[2], 0x0040);
-    const uint32_t e23 = __byte_perm(tt[4], tt[6], 0x0040);
+    const float q = rintf(__fdiv_rn(__fsub_rn(y, mn), s));
+    return static_cast<uint32_t>(fminf(fmaxf(q, 0.0f), 15.0f));
+}
+
+// Gather byte 2 of t_0..t_7 (the codes of elements e = 0..7) into one word, element e at bits
+// 4e: bytes are [k0 | k1 << 4, k2 | k3 << 4, ...] (even index in the low nibble).
+__device__ __forceinline__ uint32_t pack8_b2(const uint32_t tt[8])
+{
+    const uint32_t e01 = __byte_perm(tt[0], tt[2], 0x0062);
+    const uint32_t e23 = __byte_perm(tt[4], tt[6], 0x0062);
     const uint32_t even = __byte_perm(e01, e23, 0x5410);   // [k0, k2, k4, k6]
-    const uint32_t o01 = __byte_perm(tt[1], tt[3], 0x0040);
-    const uint32_t o23 = __byte_perm(tt[5], tt[7], 0x0040);
+    const uint32_t o01 = __byte_perm(tt[1], tt[3], 0x0062);
+    const uint32_t o23 = __byte_perm(tt[5], tt[7], 0x0062);
     const uint32_t odd = __byte_perm(o01, o23, 0x5410);    // [k1, k3, k5, k7]
     return even | (odd << 4);
+}
+
+// Unsigned 16-bit minimum of three packed pairs.
+__device__ __forceinline__ uint32_t vmin3_u16x2(uint32_t a, uint32_t b, uint32_t c)
+{
+    return __vimin3_u16x2(a, b, c);
+}
+
+// Codes of one thread's elements (held rotated, or raw for the plain INT4 cache, in X) and the
+// vector's fp32 scale and zero point, given the vector's min and max.  words[g] (g < kN / 8) holds
+// the codes of elements 8 g .. 8 g + 7 and words[kN / 8 + g] those of elements kN + 8 g .. (low
+// halves, then high halves of the registers).  Groups of 8 registers are finished one after
+// another (the rare exactly half-way elements and scales outside [2^-100, 2^100] inside the
+// group), so each group's registers are free once its two words exist.
+template <int kN>
+__device__ __forceinline__ void quantize_block(const uint64_t X[kN], float mn, float mx,
+                                               uint32_t words[kN / 4], float &scale_out,
+                                               float &zero_out)
+{
+    float scale = div15(__fsub_rn(mx, mn));
+    const bool degenerate = !(scale != 0.0f);
+    if (degenerate)
+        scale = 0.0f;                               // canonical +0
+    zero_out = __fadd_rn(mn, 0.0f);                 // a zero minimum is stored as +0
+    scale_out = scale;
+    const bool fast = scale >= kFastScaleMin && scale <= kFastScaleMax;
+    const bool divide = !fast && !degenerate;       // scales outside [2^-100, 2^100]
+    // a degenerate block gets r16 = 0: every t is the magic, code 0, and never flagged
+    const float r16 = fast ? recip_2p16(scale) : 0.0f;
+    const uint64_t nmn2 = f2_pack(-mn, -mn), r2 = f2_pack(r16, r16);
+    const uint64_t m2 = f2_pack(kGridMagic, kGridMagic);
+
+#pragma unroll
+    for (int g = 0; g < kN / 8; g++) {
+        uint32_t tlo[8], thi[8];
+        // the low 16 bits of a t are 0 only at an exactly half-way grid value: f collects the
+        // smallest low half (its high half is never 0: bits 16..31 of t hold 0x4B00 | code)
+        uint32_t f = 0xFFFFFFFFu;
+#pragma unroll
+        for (int e = 0; e < 8; e++) {
+            const uint64_t d = f2_add(X[8 * g + e], nmn2);   // y - min, one rounding
+            const uint64_t t = f2_fma(d, r2, m2);
+            float a, b;
+            f2_unpack(t, a, b);
+            tlo[e] = __float_as_uint(a);
+            thi[e] = __float_as_uint(b);
+            f = vmin3_u16x2(f, tlo[e], thi[e]);
+        }
+        if (divide) {
+            // every element by the IEEE divide
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                float a, b;
+                f2_unpack(X[8 * g + e], a, b);
+                tlo[e] = code_by_divide(a, mn, scale) << 16;
+                thi[e] = code_by_divide(b, mn, scale) << 16;
+            }
+        } else if ((f & 0xFFFFu) == 0) {
+            // rare: settle each exactly half-way element by the remainder test
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                float a, b;
+                f2_unpack(X[8 * g + e], a, b);
+                if ((tlo[e] & 0xFFFFu) == 0)
+                    tlo[e] = code_at_half(a, mn, scale, tlo[e]) << 16;
+                if ((thi[e] & 0xFFFFu) == 0)
+                    thi[e] = code_at_half(b, mn, scale, thi[e]) << 16;
+            }
+        }
+        words[g] = pack8_b2(tlo);
+        words[kN / 8 + g] = pack8_b2(thi);
+    }
+}
+
+// Store one block's codes (two runs of kN / 2 bytes: low halves, then high halves) and, from the
+// vector's first block, its fp16 (scale, zero); flag scales or zero points past fp16's range.
+template <int kN>
+__device__ __forceinline__ void store_block(uint8_t *dst, const uint32_t words[kN / 4], bool scale_here,
+                                            float scale, float zero, uint32_t *scale_dst,
+                                            uint32_t *status)
+{
+#pragma unroll
+    for (int h = 0; h < 2; h++)
+#pragma unroll
+        for (int q = 0; q < kN / 32; q++)
+            *reinterpret_cast<uint4 *>(dst + h * (kN / 2) + 16 * q) =
+                make_uint4(words[h * (kN / 8) + 4 * q], words[h * (kN / 8) + 4 * q + 1],
+                           words[h * (kN / 8) + 4 * q + 2], words[h * (kN / 8) + 4 * q + 3]);
+    if (scale_here) {
+        const __half2 sz = __halves2half2(__float2half_rn(scale), __float2half_rn(zero));
+        *scale_dst = half2_as_u32(sz);
+        // fp16 holds magnitudes below 65520: beyond, the stored value is infinite (as the
+        // definition's round-to-nearest conversion gives), which the read side cannot use
+        if (!(fabsf(scale) < 65520.0f) || !(fabsf(zero) < 65520.0f))
+            set_status(status, SAW_DEV_RANGE);
+    }
 }
 
 struct RqParams {
@@ -268,92 +347,24 @@ struct RqParams {
     uint8_t *kv_pages;
     uint32_t *scales;        // fp16x2 (scale, zero) per row
     uint32_t *status;
-    bool strided;            // k / v through 3-D tensor maps with a token stride
+    int32_t strided;         // k / v through 3-D tensor maps with a token stride
+    uint32_t hkv_mul;        // vec / hkv by multiply and shift (div_hkv)
+    uint32_t hkv_shift;
 };
 
-// Quantize the vector (held rotated in X) and store codes + scale into cache row `row`.
-// kRotate = false is the plain INT4 quantizer (H = I) used as the unrotated baseline.
-template <bool kRotate, int kD>
-__device__ __forceinline__ void quantize_store(const uint64_t X[32], int blk, int b, bool store,
-                                               int64_t row, const RqParams &p)
+// vec / hkv without a divide (T. Granlund, P. Montgomery, "Division by invariant integers using
+// multiplication", PLDI 1994, with a 33-bit multiplier): with s = ceil(log2 hkv) and
+// m' = ceil(2^(32 + s) / hkv), floor(vec m' / 2^(32 + s)) = floor(vec / hkv) for every vec < 2^32;
+// m' = 2^32 + hkv_mul, so vec m' / 2^32 = umulhi(vec, hkv_mul) + vec (no overflow for vec < 2^31).
+__device__ __forceinline__ uint32_t div_hkv(uint32_t vec, const RqParams &p)
 {
-    // min / max over the vector's D elements (its D / 64 threads)
-    float mns[8], mxs[8];
-#pragma unroll
-    for (int i = 0; i < 32; i++) {
-        float lo, hi;
-        f2_unpack(X[i], lo, hi);
-        mns[i & 7] = (i < 8) ? fminf(lo, hi) : fmin3(mns[i & 7], lo, hi);
-        mxs[i & 7] = (i < 8) ? fmaxf(lo, hi) : fmax3(mxs[i & 7], lo, hi);
-    }
-    float mn = fminf(fmin3(mns[0], mns[1], mns[2]), fmin3(fmin3(mns[3], mns[4], mns[5]), mns[6], mns[7]));
-    float mx = fmaxf(fmax3(mxs[0], mxs[1], mxs[2]), fmax3(fmax3(mxs[3], mxs[4], mxs[5]), mxs[6], mxs[7]));
-#pragma unroll
-    for (int d = 1; d < RqDims<kD>::kThreadsPerVec; d <<= 1) {
-        mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
-        mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
-    }
+    return (__umulhi(vec, p.hkv_mul) + vec) >> p.hkv_shift;
+}
 
-    float scale = __fdiv_rn(__fsub_rn(mx, mn), 15.0f);
-    const bool degenerate = !(scale != 0.0f);
-    if (degenerate)
-        scale = 0.0f;                               // canonical +0
-    const float zero = __fadd_rn(mn, 0.0f);         // a zero minimum is stored as +0
-
-    const bool fast = !degenerate && !(scale < FLT_MIN);
-    const float r = fast ? __frcp_rn(scale) : 0.0f;
-    const uint64_t mn2 = f2_pack(mn, mn), r2 = f2_pack(r, r);
-    const uint64_t m2 = f2_pack(kRoundMagic, kRoundMagic);
-
-    // Codes and stores, two output words at a time: words a4 and a4 + 4 take the low and high
-    // halves of the packed pairs X[8 a4 + r].  Each code comes from the reciprocal (see the
-    // note above code_bits_tie()); the 16 elements of the two words go through
-    // code_bits_exact() when one of them lies near a half-way quotient, or for a subnormal
-    // scale.
-    uint8_t *dst = p.kv_pages + row * RqDims<kD>::kCodeBytes + 64 * blk;
-#pragma unroll
-    for (int a4 = 0; a4 < 4; a4++) {
-        uint32_t tlo[8], thi[8];
-        float worst = 0.0f;
-#pragma unroll
-        for (int rr = 0; rr < 8; rr++) {
-            const uint64_t d = f2_sub(X[8 * a4 + rr], mn2);
-            const uint64_t t = f2_fma(d, r2, m2);
-            const uint64_t nk = f2_sub(m2, t);          // -k, exact
-            const uint64_t res = f2_fma(d, r2, nk);     // d r - k, one rounding
-            float tl, th, el, eh;
-            f2_unpack(t, tl, th);
-            f2_unpack(res, el, eh);
-            worst = fmax3(worst, fabsf(el), fabsf(eh));
-            tlo[rr] = __float_as_uint(tl);
-            thi[rr] = __float_as_uint(th);
-        }
-        if (degenerate) {
-#pragma unroll
-            for (int rr = 0; rr < 8; rr++)
-                tlo[rr] = thi[rr] = __float_as_uint(kRoundMagic);   // every code 0
-        } else if (!fast || !(worst < kNearHalf)) {
-#pragma unroll
-            for (int rr = 0; rr < 8; rr++) {
-                float lo, hi;
-                f2_unpack(X[8 * a4 + rr], lo, hi);
-                tlo[rr] = code_bits_exact(lo, tlo[rr], mn, scale, r, fast);
-                thi[rr] = code_bits_exact(hi, thi[rr], mn, scale, r, fast);
-            }
-        }
-        if (store) {
-            // D = 64: elements 8 a + r of one thread, word a at byte 4 a; otherwise elements
-            // 16 a + 8 b + r of thread half b, word (a, b) at byte 8 a + 4 b of the block
-            const int w_lo = kD == 64 ? 4 * a4 : 8 * a4 + 4 * b;
-            const int w_hi = kD == 64 ? 4 * (a4 + 4) : 8 * (a4 + 4) + 4 * b;
-            *reinterpret_cast<uint32_t *>(dst + w_lo) = pack8(tlo);
-            *reinterpret_cast<uint32_t *>(dst + w_hi) = pack8(thi);
-        }
-    }
-    if (store && b == 0 && blk == 0) {
-        const __half2 sz = __halves2half2(__float2half_rn(scale), __float2half_rn(zero));
-        p.scales[row] = half2_as_u32(sz);
-    }
+// A vector's row of the cache: (page * Hkv + h) * 2 + K/V, times 16, plus the offset in the page.
+__device__ __forceinline__ int64_t cache_row(int64_t slot, uint32_t h, int half, int64_t hkv)
+{
+    return ((((slot >> 4) * hkv + h) * 2 + half) << 4) + (slot & 15);
 }
 
 template <bool kRotate, int kD>
@@ -362,20 +373,22 @@ __global__ void __launch_bounds__(kRqThreads, 4)
                            const __grid_constant__ CUtensorMap tv, const RqParams p)
 {
     using Dims = RqDims<kD>;
-    constexpr int kTileVecs = Dims::kTileVecs;
+    constexpr int kN = Dims::kN;
+    constexpr int kStageBytes = Dims::kStageBytes;
+    constexpr int kTpv = Dims::kThreadsPerVec;
     extern __shared__ uint8_t smem_raw[];
     uint8_t *smem = reinterpret_cast<uint8_t *>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     pdl_launch_dependents();
-    // all indices below fit in 32 bits: the host limits num_vecs to 2^29
+    // all indices below fit in 32 bits: the host limits the rows to 2^29
     const uint32_t W = gridDim.x * kRqWarps;
     const uint32_t wg = blockIdx.x * kRqWarps + warp;
     const uint32_t num_tiles = static_cast<uint32_t>(p.num_tiles);
     if (wg >= num_tiles)
         return;
     const int n = static_cast<int>((num_tiles - wg + W - 1) / W);   // this warp's tiles: wg + i W
-    const uint32_t ring = smem_u32(smem) + warp * kRqStages * kRqStageBytes;
-    const uint32_t bar0 = smem_u32(smem + kRqSmemBars) + warp * kRqStages * 8;
+    const uint32_t ring = smem_u32(smem) + warp * kRqStages * kStageBytes;
+    const uint32_t bar0 = smem_u32(smem + kRqWarps * kRqStages * kStageBytes) + warp * kRqStages * 8;
     if (lane == 0)
         for (int i = 0; i < kRqStages; i++)
             mbar_init(bar0 + 8 * i, 1);
@@ -384,24 +397,24 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 
     int issued = 0, istg = 0;
     uint32_t itile = wg;
-    const uint32_t hkv_u = static_cast<uint32_t>(p.hkv);
+    // queue tile `itile` (16 rows of K and of V) into stage istg
     auto issue = [&]() {
         if (issued < n) {
             if (lane == 0) {
-                const uint32_t dst = ring + istg * kRqStageBytes;
+                const uint32_t dst = ring + istg * kStageBytes;
                 const uint32_t bar = bar0 + 8 * istg;
-                mbar_arrive_expect_tx(bar, kRqStageBytes);
+                mbar_arrive_expect_tx(bar, kStageBytes);
                 if (p.strided) {
                     // the tile's first vector: token and head (the box spans whole tiles)
-                    const uint32_t v0 = itile * kTileVecs;
-                    const int32_t tok = static_cast<int32_t>(v0 / hkv_u);
-                    const int32_t row = static_cast<int32_t>(Dims::kRowsPerVec * (v0 - tok * hkv_u));
+                    const uint32_t v0 = itile * Dims::kTileVecs;
+                    const int32_t tok = static_cast<int32_t>(div_hkv(v0, p));
+                    const int32_t row = static_cast<int32_t>(kTpv * (v0 - tok * static_cast<uint32_t>(p.hkv)));
                     tma_load_3d(dst, &tk, 0, row, tok, bar);
-                    tma_load_3d(dst + kTileBytes, &tv, 0, row, tok, bar);
+                    tma_load_3d(dst + Dims::kHalfBytes, &tv, 0, row, tok, bar);
                 } else {
-                    const int32_t y = static_cast<int32_t>(itile * (Dims::kRowsPerVec * kTileVecs));
+                    const int32_t y = static_cast<int32_t>(itile * 16);
                     tma_load_2d(dst, &tk, 0, y, bar);
-                    tma_load_2d(dst + kTileBytes, &tv, 0, y, bar);
+                    tma_load_2d(dst + Dims::kHalfBytes, &tv, 0, y, bar);
                 }
             }
             issued++;
@@ -413,20 +426,18 @@ __global__ void __launch_bounds__(kRqThreads, 4)
     for (int k = 0; k < kRqStages - 1; k++)
         issue();
 
-    const int half = lane >> 4;          // 0: K, 1: V
-    // half of a 128-block, 128-block of the vector, vector of the tile (D = 64: one thread
-    // holds a whole vector)
-    const int b = kD == 64 ? 0 : lane & 1;
-    const int blk = kD == 64 ? 0 : (lane >> 1) & (Dims::kThreadsPerVec / 2 - 1);
-    const int vt = (lane & 15) / Dims::kThreadsPerVec;
+    const int half = lane >> 4;                     // 0: K, 1: V
+    const int r = lane & 15;                        // row of the tile
+    const int part = r % kTpv;                      // row of the vector (64 elements each)
+    const int vt = r / kTpv;                        // vector of the tile
     const uint32_t num_vecs = static_cast<uint32_t>(p.num_vecs);
     const uint32_t hkv = static_cast<uint32_t>(p.hkv);
     uint32_t tile = wg;
     // slot of this thread's vector in the tile (prefetched one tile ahead)
     auto slot_of = [&](uint32_t t, uint32_t &vec) -> int64_t {
-        const uint32_t vec_raw = t * kTileVecs + vt;
+        const uint32_t vec_raw = t * Dims::kTileVecs + vt;
         vec = vec_raw < num_vecs ? vec_raw : num_vecs - 1;
-        return p.slot_mapping[vec / hkv];
+        return p.slot_mapping[div_hkv(vec, p)];
     };
     uint32_t vec_next;
     int64_t slot_next = slot_of(tile, vec_next);
@@ -436,7 +447,7 @@ __global__ void __launch_bounds__(kRqThreads, 4)
     for (; i < n; i++, tile += W) {
         issue();
         const uint32_t vec = vec_next;
-        const bool in_range = tile * kTileVecs + vt < num_vecs;
+        const bool in_range = tile * Dims::kTileVecs + vt < num_vecs;
         const int64_t slot = slot_next;
         if (i + 1 < n)
             slot_next = slot_of(tile + W, vec_next);
@@ -451,34 +462,49 @@ __global__ void __launch_bounds__(kRqThreads, 4)
                 set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
             break;
         }
-        const uint32_t tok = vec / hkv;
+        const uint32_t tok = div_hkv(vec, p);
         const uint32_t h = vec - tok * hkv;
         bool store = in_range && slot >= 0;
         if (store && slot >= p.num_slots) {
-            if (b == 0 && half == 0)
+            if (part == 0 && half == 0)
                 set_status(p.status, SAW_DEV_BAD_SLOT);
             store = false;
         }
-        const int64_t page = store ? slot >> 4 : 0;    // slot / 16
-        const int64_t off = store ? slot & 15 : 0;
-        const int64_t row = ((page * p.hkv + h) * 2 + half) * kPageSize + off;
 
-        const uint32_t tile_smem = ring + stg * kRqStageBytes + half * kTileBytes;
-        uint4 raw[8];
-        if constexpr (kD == 64)
-            load_vec64(tile_smem, vt, raw);
-        else
-            load_half_vec<kD>(tile_smem, vt, blk, b, raw);
-        uint64_t X[32];
-        to_pairs(raw, X);
+        // this thread's row r of the stage's K or V half; the 16-byte chunk c of a row sits at
+        // chunk c ^ (r & 7) under the 128-byte swizzle: X[m] = (x[m], x[m + 32])
+        const uint32_t stage = ring + stg * kStageBytes;
+        const uint32_t row = stage + half * Dims::kHalfBytes + r * 128;
+        uint64_t X[kN];
+#pragma unroll
+        for (int c = 0; c < 4; c++)
+            pairs_from_chunk(lds128(row + ((c ^ (r & 7)) << 4)),
+                             lds128(row + (((c + 4) ^ (r & 7)) << 4)), X + 8 * c);
+        __syncwarp();   // every lane has read the stage
         if constexpr (kRotate) {
-            if constexpr (kD == 64)
-                fwht64(X);
-            else
-                fwht128(X, b, 0xFFFFFFFFu);
+            fwht_stages<kN>(X);
+            if constexpr (kD == 64) {
+                scale_all<kN>(X, kHadamardC64);
+            } else {
+                exchange_stage64(X, part & 1);
+                scale_all<kN>(X, kHadamardC);
+            }
         }
-        quantize_store<kRotate, kD>(X, blk, b, store, row, p);
-        __syncwarp();
+        float mn, mx;
+        block_min_max<kN>(X, mn, mx);
+#pragma unroll
+        for (int d = 1; d < kTpv; d <<= 1) {
+            mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, d));
+            mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, d));
+        }
+        uint32_t words[kN / 4];
+        float scale, zero;
+        quantize_block<kN>(X, mn, mx, words, scale, zero);
+        if (store) {
+            const int64_t crow = cache_row(slot, h, half, p.hkv);
+            store_block<kN>(p.kv_pages + crow * Dims::kCodeBytes + 32 * part, words, part == 0, scale,
+                            zero, p.scales + crow, p.status);
+        }
     }
     if (i < n) {
         // a wait gave up: let every queued copy land before the shared memory is released
@@ -498,10 +524,10 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 // the rotate+quantize kernel (same device code).  With w_recent = 0 the new token itself is
 // quantized.  Window slot i lives in bf16 page win_table[s][i / 16] at offset i mod 16.
 //
-// Lanes as in the rotate+quantize kernel at D = 128: a warp takes 8 (sequence, kv head) pairs,
-// lanes 0-15 their K vectors and lanes 16-31 their V vectors, two threads per vector.  Each
-// thread reads exactly the 128 bytes of the displaced vector it later overwrites with the new
-// token, so the read and the write of a slot are ordered within one thread.
+// Lanes as in the rotate+quantize kernel at D = 128: a warp takes 16 (sequence, kv head) pairs,
+// lanes 0-15 their K vectors and lanes 16-31 their V vectors, one thread per vector.  Each thread
+// reads exactly the 256 bytes of the displaced vector it later overwrites with the new token, so
+// the read and the write of a slot are ordered within one thread.
 struct WinAppendParams {
     const uint16_t *k, *v;
     const int32_t *seq_lens;
@@ -513,7 +539,9 @@ struct WinAppendParams {
     const int32_t *block_table;
     int32_t max_blocks;
     int64_t num_pages;
-    RqParams q;        // kv_pages and scales for quantize_store; status
+    uint8_t *kv_pages;
+    uint32_t *scales;
+    uint32_t *status;
 };
 
 template <bool kRotate>
@@ -522,13 +550,13 @@ __global__ void __launch_bounds__(kRqThreads)
 {
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-    const int half = lane >> 4, b = lane & 1, vt = (lane & 15) >> 1;
-    const int64_t pair = (static_cast<int64_t>(blockIdx.x) * kRqWarps + warp) * 8 + vt;
+    const int half = lane >> 4;
+    const int64_t pair = (static_cast<int64_t>(blockIdx.x) * kRqWarps + warp) * 16 + (lane & 15);
     const bool live = pair < static_cast<int64_t>(p.num_seqs) * p.hkv;
     const int s = live ? static_cast<int>(pair / p.hkv) : 0;
     const int h = live ? static_cast<int>(pair - static_cast<int64_t>(s) * p.hkv) : 0;
     const int L = live ? p.seq_lens[s] : 0;
-    const bool report = b == 0 && half == 0;
+    const bool report = half == 0;
 
     // where the new token goes and which token is quantized
     bool to_win = false, quant = false, from_win = false;
@@ -550,14 +578,14 @@ __global__ void __launch_bounds__(kRqThreads)
             }
         }
     } else if (L < 0 && report) {
-        set_status(p.q.status, SAW_DEV_BAD_SEQ_LEN);
+        set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
     }
     uint16_t *win = nullptr;
     if (to_win) {
         const int32_t page = p.win_table[static_cast<int64_t>(s) * p.win_blocks + slot / 16];
         if (page < 0 || page >= p.num_win_pages) {
             if (report)
-                set_status(p.q.status, SAW_DEV_BAD_PAGE);
+                set_status(p.status, SAW_DEV_BAD_PAGE);
             to_win = quant = false;   // the displaced token cannot be read: leave the pair
         } else {
             win = p.win_kv + ((((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize) +
@@ -571,30 +599,37 @@ __global__ void __launch_bounds__(kRqThreads)
                                  : -1;
         if (page < 0 || page >= p.num_pages) {
             if (report)
-                set_status(p.q.status, j / kPageSize < p.max_blocks ? SAW_DEV_BAD_PAGE : SAW_DEV_BAD_SEQ_LEN);
+                set_status(p.status, j / kPageSize < p.max_blocks ? SAW_DEV_BAD_PAGE : SAW_DEV_BAD_SEQ_LEN);
             to_win = quant = false;   // keep the displaced token where it is
         } else {
             row = ((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize + j % kPageSize;
         }
     }
 
-    // this thread's 64 elements (16 a + 8 b + r) of the new vector and of the displaced one
-    uint4 fresh[8], raw[8];
+    // the vector to quantize (the displaced window token, or the new token itself when there is
+    // no recent ring): elements 0..63 in lo, 64..127 in hi
     const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128;
+    if (quant) {
+        const uint16_t *qsrc = from_win ? win : src;
+        uint64_t X[64];
 #pragma unroll
-    for (int a = 0; a < 8; a++) {
-        fresh[a] = L > 0 ? *reinterpret_cast<const uint4 *>(src + 16 * a + 8 * b) : make_uint4(0, 0, 0, 0);
-        raw[a] = from_win && quant ? *reinterpret_cast<const uint4 *>(win + 16 * a + 8 * b) : fresh[a];
+        for (int c = 0; c < 8; c++)
+            pairs_from_chunk(*reinterpret_cast<const uint4 *>(qsrc + 8 * c),
+                             *reinterpret_cast<const uint4 *>(qsrc + 64 + 8 * c), X + 8 * c);
+        if constexpr (kRotate)
+            fwht_block<64>(X);
+        float mn, mx;
+        block_min_max<64>(X, mn, mx);
+        uint32_t words[16];
+        float scale, zero;
+        quantize_block<64>(X, mn, mx, words, scale, zero);
+        store_block<64>(p.kv_pages + row * 64, words, true, scale, zero, p.scales + row, p.status);
     }
-    uint64_t X[32];
-    to_pairs(raw, X);
-    if constexpr (kRotate)
-        fwht128(X, b, 0xFFFFFFFFu);
-    quantize_store<kRotate, 128>(X, 0, b, quant, row, p.q);
+    // then the new token takes the slot (after this thread's own read of it)
     if (to_win) {
 #pragma unroll
-        for (int a = 0; a < 8; a++)
-            *reinterpret_cast<uint4 *>(win + 16 * a + 8 * b) = fresh[a];
+        for (int c = 0; c < 16; c++)
+            *reinterpret_cast<uint4 *>(win + 8 * c) = *reinterpret_cast<const uint4 *>(src + 8 * c);
     }
 }
 
@@ -620,11 +655,10 @@ cudaError_t launch_window_append(const WindowAppendArgs &a, cudaStream_t stream)
     p.block_table = a.block_table;
     p.max_blocks = a.max_blocks;
     p.num_pages = a.num_pages;
-    p.q = RqParams{};
-    p.q.kv_pages = a.kv_pages;
-    p.q.scales = static_cast<uint32_t *>(a.scales);
-    p.q.status = a.status;
-    const int64_t grid = (pairs + 8 * kRqWarps - 1) / (8 * kRqWarps);
+    p.kv_pages = a.kv_pages;
+    p.scales = static_cast<uint32_t *>(a.scales);
+    p.status = a.status;
+    const int64_t grid = (pairs + 16 * kRqWarps - 1) / (16 * kRqWarps);
     window_append_kernel<true><<<static_cast<unsigned>(grid), kRqThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
@@ -638,16 +672,18 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         return cudaSuccess;
     if (a.head_dim != 64 && a.head_dim != 128 && a.head_dim != 256)
         return cudaErrorInvalidValue;
-    const int64_t rows_per_vec = a.head_dim / 64;
-    const int64_t tile_vecs = kTileBytes / (2 * a.head_dim);
-    if (num_vecs * rows_per_vec > (int64_t(1) << 30))
-        return cudaErrorInvalidValue;       // tensor-map rows must fit in int32
+    const int64_t rows_per_vec = a.head_dim / 64;   // 128-byte rows (64 elements) per vector
+    const int64_t tile_vecs = 16 / rows_per_vec;
+    if (num_vecs * rows_per_vec > (int64_t(1) << 29))
+        return cudaErrorInvalidValue;       // tensor-map rows and tile indices fit in int32
 
     // k / v: contiguous [T][Hkv][D] (k_stride = v_stride = 0) through a 2-D map of 128-byte
-    // rows, or with a token stride through 3-D maps whose box is one whole tile of V vectors
-    // (V = 16 for D = 64, 8 for D = 128, 4 for D = 256; Hkv a multiple of V: V heads of one token; Hkv dividing
-    // V: V / Hkv tokens), so every copy lands on a 1024-byte aligned stage.
+    // rows whose box is one warp tile (16 rows), or with a token stride through 3-D maps (row,
+    // row within the token, token) whose box is also one whole tile: 16 rows of one token (rows
+    // per token a multiple of 16) or 16 / R whole tokens of R rows (R dividing 16).  Every copy
+    // lands on a 1024-byte aligned stage.
     const bool strided = a.k_stride != 0 || a.v_stride != 0;
+    const int64_t rows_per_token = a.num_kv_heads * rows_per_vec;
     static thread_local struct {
         const void *k = nullptr, *v = nullptr;
         int64_t num_vecs = 0, k_stride = -1, v_stride = -1;
@@ -659,8 +695,7 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
         auto encode = tensor_map_encoder();
         if (encode == nullptr)
             return cudaErrorNotSupported;
-        const int64_t hkv = a.num_kv_heads;
-        if (strided && hkv % tile_vecs != 0 && tile_vecs % hkv != 0)
+        if (strided && rows_per_token % 16 != 0 && 16 % rows_per_token != 0)
             return cudaErrorInvalidValue;
         const cuuint32_t estr[3] = {1, 1, 1};
         for (int which = 0; which < 2; which++) {
@@ -669,18 +704,18 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
             if (!strided) {
                 const cuuint64_t dims[2] = {128, static_cast<cuuint64_t>(rows_per_vec * num_vecs)};
                 const cuuint64_t strides[1] = {128};
-                const cuuint32_t box[2] = {128, kTileBytes / 128};   // one warp tile: 16 rows
+                const cuuint32_t box[2] = {128, 16};
                 r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, base,
                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
             } else {
                 const int64_t stride = which ? a.v_stride : a.k_stride;   // bf16 elements
-                const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows_per_vec * hkv),
+                const cuuint64_t dims[3] = {128, static_cast<cuuint64_t>(rows_per_token),
                                             static_cast<cuuint64_t>(a.num_tokens)};
                 const cuuint64_t strides[2] = {128, static_cast<cuuint64_t>(stride * 2)};
-                const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(rows_per_vec * std::min<int64_t>(hkv, tile_vecs)),
-                                           static_cast<cuuint32_t>(std::max<int64_t>(1, tile_vecs / hkv))};
+                const cuuint32_t box[3] = {128, static_cast<cuuint32_t>(std::min<int64_t>(rows_per_token, 16)),
+                                           static_cast<cuuint32_t>(std::max<int64_t>(1, 16 / rows_per_token))};
                 r = encode(which ? &cache.mv : &cache.mk, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, base,
                            dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
                            CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
@@ -709,48 +744,57 @@ cudaError_t launch_rotate_quantize(const RotateQuantizeArgs &a, cudaStream_t str
     p.kv_pages = a.kv_pages;
     p.scales = static_cast<uint32_t *>(a.scales);
     p.status = a.status;
-    p.strided = strided;
+    p.strided = strided ? 1 : 0;
+    {
+        uint32_t sh = 0;
+        while ((int64_t(1) << sh) < a.num_kv_heads)
+            sh++;
+        const uint64_t d = static_cast<uint64_t>(a.num_kv_heads);
+        p.hkv_shift = sh;
+        p.hkv_mul = static_cast<uint32_t>(((uint64_t(1) << (32 + sh)) + d - 1) / d - (uint64_t(1) << 32));
+    }
 
-    // per device: multiprocessor count, the shared-memory attribute and the occupancy
+    // per device and kernel: multiprocessor count, the shared-memory attribute and occupancy
     constexpr int kMaxDevices = 64;
-    static int sms_of[kMaxDevices] = {}, occ_of[kMaxDevices] = {};
+    constexpr int kVariants = 6;
+    static int sms_of[kMaxDevices] = {}, occ_of[kMaxDevices][kVariants] = {};
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess)
         return e;
     if (dev < 0 || dev >= kMaxDevices)
         return cudaErrorInvalidDevice;
-    static const void *const kernels[6] = {
-        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 128>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 128>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 256>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 256>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<true, 64>),
-        reinterpret_cast<const void *>(rotate_quantize_kernel<false, 64>)};
-    auto kernel = a.head_dim == 128
-                      ? (a.rotate ? rotate_quantize_kernel<true, 128> : rotate_quantize_kernel<false, 128>)
-                  : a.head_dim == 256
-                      ? (a.rotate ? rotate_quantize_kernel<true, 256> : rotate_quantize_kernel<false, 256>)
-                      : (a.rotate ? rotate_quantize_kernel<true, 64> : rotate_quantize_kernel<false, 64>);
+    using KernelFn = void (*)(CUtensorMap, CUtensorMap, RqParams);
+    static const KernelFn kernels[kVariants] = {
+        rotate_quantize_kernel<true, 128>, rotate_quantize_kernel<false, 128>,
+        rotate_quantize_kernel<true, 256>, rotate_quantize_kernel<false, 256>,
+        rotate_quantize_kernel<true, 64>, rotate_quantize_kernel<false, 64>};
+    static const size_t smem_of[kVariants] = {rq_smem_bytes<128>(), rq_smem_bytes<128>(),
+                                              rq_smem_bytes<256>(), rq_smem_bytes<256>(),
+                                              rq_smem_bytes<64>(), rq_smem_bytes<64>()};
+    const int which = (a.head_dim == 128 ? 0 : a.head_dim == 256 ? 2 : 4) + (a.rotate ? 0 : 1);
     if (sms_of[dev] == 0) {
-        int sms = 0, occ = 0;
+        int sms = 0;
         e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-        for (int r = 0; r < 6 && e == cudaSuccess; r++)
-            e = cudaFuncSetAttribute(kernels[r], cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                     static_cast<int>(kRqSmemBytes));
-        if (e == cudaSuccess)
-            e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&occ, kernels[0], kRqThreads,
-                                                              kRqSmemBytes);
+        for (int r = 0; r < kVariants && e == cudaSuccess; r++) {
+            e = cudaFuncSetAttribute(reinterpret_cast<const void *>(kernels[r]),
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     static_cast<int>(smem_of[r]));
+            int occ = 0;
+            if (e == cudaSuccess)
+                e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(
+                    &occ, reinterpret_cast<const void *>(kernels[r]), kRqThreads, smem_of[r]);
+            if (e == cudaSuccess && occ <= 0)
+                e = cudaErrorInvalidConfiguration;
+            occ_of[dev][r] = occ;
+        }
         if (e != cudaSuccess)
             return e;
-        if (occ <= 0)
-            return cudaErrorInvalidConfiguration;
-        occ_of[dev] = occ;
         sms_of[dev] = sms;
     }
     const int64_t grid = std::min<int64_t>((p.num_tiles + kRqWarps - 1) / kRqWarps,
-                                           static_cast<int64_t>(sms_of[dev]) * occ_of[dev]);
-    kernel<<<static_cast<unsigned>(grid), kRqThreads, kRqSmemBytes, stream>>>(cache.mk, cache.mv, p);
+                                           static_cast<int64_t>(sms_of[dev]) * occ_of[dev][which]);
+    kernels[which]<<<static_cast<unsigned>(grid), kRqThreads, smem_of[which], stream>>>(cache.mk, cache.mv, p);
     return cudaGetLastError();
 }
 

@@ -30,6 +30,7 @@ SAW_DEV_BAD_SLOT = 0x1
 SAW_DEV_BAD_PAGE = 0x2
 SAW_DEV_BAD_SEQ_LEN = 0x4
 SAW_DEV_WAIT_TIMEOUT = 0x8
+SAW_DEV_RANGE = 0x10
 
 
 class SawError(RuntimeError):

@@ -50,6 +50,12 @@
  * wait that gave up -- never trap: the kernel skips the offending access, ORs a SAW_DEV_* bit
  * into *dev_status (when dev_status is not NULL) and carries on; the caller reads the word
  * after synchronising.  NaN or Inf inputs are not supported (their codes are unspecified).
+ * Input range: a vector's rotated minimum and its scale must stay below fp16's largest finite
+ * magnitude (65504; a value that rounds to 65520 or more is stored as infinity, as the
+ * round-to-nearest conversion of the definition gives).  The rotation can grow a value by up to
+ * sqrt(128) = 11.3 (a constant vector of -5800 already has a rotated minimum of -65600), so keys
+ * and values beyond a few thousand in magnitude are out of range; the quantizer then still
+ * stores the definition's bits but ORs SAW_DEV_RANGE into *dev_status.
  */
 #ifndef SAW_H_
 #define SAW_H_
@@ -76,6 +82,8 @@ typedef enum saw_status {
 #define SAW_DEV_BAD_PAGE 0x2u     /* block_table entry outside [0, num_pages): page 0 read */
 #define SAW_DEV_BAD_SEQ_LEN 0x4u  /* seq_lens[s] < 0 or > 16 * max_blocks: output zeroed */
 #define SAW_DEV_WAIT_TIMEOUT 0x8u /* a bounded wait on a page copy gave up */
+#define SAW_DEV_RANGE 0x10u       /* a scale or zero point beyond fp16's range (|x| >= 65520) was
+                                     stored as +-inf: that vector cannot be read back */
 
 typedef struct saw_cache_desc {
     int32_t num_kv_heads; /* Hkv >= 1 */
