@@ -398,18 +398,24 @@ __device__ __forceinline__ void state_reset(WarpState<kTiles> &st)
     }
 }
 
-// Online softmax over one page: s holds the logits (log2 domain) of tokens g, g + 8 for columns
-// 2t, 2t + 1 (-inf for masked tokens); returns p = 2^(s - m) with m the running max after the
-// page, and rescales o, l and z when m grows.  The running max only changes when some logit of
-// the page exceeds it, so the cross-lane reduction runs only then (rare once a piece is a few
-// pages long); the result equals reducing every page.  kMask: a column may have seen only
-// masked tokens so far (m = -inf); its p stay 0 and nothing is rescaled by a NaN.
-template <bool kMask, int kTiles>
-__device__ __forceinline__ void softmax_update(const float s[4], WarpState<kTiles> &st, float pr[4])
+// Online softmax over one page (kN = 4) or two (kN = 8): s holds the logits (log2 domain) of
+// tokens g, g + 8 (then g + 16, g + 24 of the second page) for columns 2t, 2t + 1 (s[k] belongs to
+// column k & 1; -inf for masked tokens); returns p = 2^(s - m) with m the running max after the
+// page(s), and rescales o, l and z when m grows.  The running max only changes when some logit
+// exceeds it, so the cross-lane reduction runs only then (rare once a piece is a few pages long);
+// the result equals reducing every page.  kMask: a column may have seen only masked tokens so far
+// (m = -inf); its p stay 0 and nothing is rescaled by a NaN.
+template <bool kMask, int kTiles, int kN = 4>
+__device__ __forceinline__ void softmax_update(const float s[kN], WarpState<kTiles> &st, float pr[kN])
 {
-    const bool grow = fmaxf(s[0], s[2]) > st.m[0] || fmaxf(s[1], s[3]) > st.m[1];
+    float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
+#pragma unroll
+    for (int k = 4; k < kN; k += 2) {
+        mx[0] = fmaxf(mx[0], s[k]);
+        mx[1] = fmaxf(mx[1], s[k + 1]);
+    }
+    const bool grow = mx[0] > st.m[0] || mx[1] > st.m[1];
     if (__any_sync(0xFFFFFFFFu, grow)) {
-        float mx[2] = {fmaxf(s[0], s[2]), fmaxf(s[1], s[3])};
 #pragma unroll
         for (int e = 0; e < 2; e++) {
             mx[e] = fmaxf(mx[e], __shfl_xor_sync(0xFFFFFFFFu, mx[e], 4));
@@ -433,13 +439,10 @@ __device__ __forceinline__ void softmax_update(const float s[4], WarpState<kTile
             st.o[i][3] *= alpha[1];
         }
     }
-    pr[0] = ex2_approx(s[0] - st.m[0]);
-    pr[1] = ex2_approx(s[1] - st.m[1]);
-    pr[2] = ex2_approx(s[2] - st.m[0]);
-    pr[3] = ex2_approx(s[3] - st.m[1]);
-    if (kMask) {
 #pragma unroll
-        for (int k = 0; k < 4; k++)
+    for (int k = 0; k < kN; k++) {
+        pr[k] = ex2_approx(s[k] - st.m[k & 1]);
+        if (kMask)
             pr[k] = s[k] == -INFINITY ? 0.0f : pr[k];
     }
 }
@@ -574,7 +577,7 @@ __global__ void __launch_bounds__(kMergeThreads)
 // ---- the attention kernel, generic over the page format --------------------------------------
 //
 // A page format Fmt supplies:
-//   kWarps, kStages (a power of two), kMinBlocks   warps per CTA, ring stages per warp, and the
+//   kWarps, kStages, kMinBlocks                    warps per CTA, ring stages per warp, and the
 //                                                  CTAs per SM the launch bounds ask for;
 //   kRingBytes                                     the rings of all warps, from a 1024-byte
 //                                                  aligned base;
@@ -586,6 +589,8 @@ __global__ void __launch_bounds__(kMergeThreads)
 //                                                  raw bf16 query rows in shared memory;
 //   page<kMask>(ring, stg, mask, q, lane, st)      attend over one staged page (PageMask when
 //                                                  kMask: never-written tokens, causal limits);
+//   kPairs; page2(ring, stg0, stg1, q, lane, st)   whether whole pages go two at a time, and
+//                                                  the two-page step (one softmax update);
 //   piece_end(st)                                  reductions and corrections after a piece;
 //   finalize(p, segment, lane, o, m, l)            write a finished segment's output rows (a
 //                                                  template on the segment type)
@@ -727,7 +732,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
             look_b = lookup(look_base + 32 + lane);
         }
         const int32_t row = __shfl_sync(0xFFFFFFFFu, look_a, j & 31);
-        const int stg = j & (kStages - 1);
+        const int stg = j % kStages;
         Fmt::issue(ring, stg, bar0 + 8 * stg, &tmap, row, p);
     };
 
@@ -750,11 +755,32 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     auto step = [&](auto mask_tag, int m, const PageMask &mask) {
         if (issued < n_w && !aborted)
             issue_next();
-        const int stg = m & (kStages - 1);
+        const int stg = m % kStages;
         const uint32_t phase = (static_cast<uint32_t>(m) / kStages) & 1u;
         const bool ok = !aborted && mbar_wait_bounded(bar0 + 8 * stg, phase, kWaitLimitNs);
         if (__all_sync(0xFFFFFFFFu, ok)) {
             Fmt::template page<decltype(mask_tag)::value>(ring, stg, mask, qf, lane, st);
+        } else if (!aborted) {
+            if (lane == 0)
+                set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
+            drain_from = m;
+            aborted = true;
+        }
+        __syncwarp();
+    };
+
+    // Whole pages m and m + 1 as one step (formats with kPairs): queue pages up to m + kStages - 1
+    // (the stages pages m - 2 and m - 1 used), wait for both pages, attend over both.
+    auto step2 = [&](int m) {
+        while (issued <= m + kStages - 1 && issued < n_w && !aborted)
+            issue_next();
+        const int stg0 = m % kStages, stg1 = (m + 1) % kStages;
+        const bool ok = !aborted &&
+                        mbar_wait_bounded(bar0 + 8 * stg0, (static_cast<uint32_t>(m) / kStages) & 1u, kWaitLimitNs) &&
+                        mbar_wait_bounded(bar0 + 8 * stg1, (static_cast<uint32_t>(m + 1) / kStages) & 1u, kWaitLimitNs);
+        if (__all_sync(0xFFFFFFFFu, ok)) {
+            if constexpr (Fmt::kPairs)
+                Fmt::page2(ring, stg0, stg1, qf, lane, st);
         } else if (!aborted) {
             if (lane == 0)
                 set_status(p.status, SAW_DEV_WAIT_TIMEOUT);
@@ -819,6 +845,10 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         const int i0 = static_cast<int>(pos - seg_start) - m;   // page index of run page m
         const int m_full = min(m_end, max(m, first_masked - i0));
         const PageMask whole = {kPageSize, {kPageSize, kPageSize}};
+        if constexpr (Fmt::kPairs) {
+            for (; m + 1 < m_full; m += 2)
+                step2(m);
+        }
         for (; m < m_full; m++)
             step(std::false_type(), m, whole);
         for (; m < m_end; m++)
@@ -840,7 +870,7 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
     // ---- 4. after an abort, let queued copies land before the shared memory is released ----
     if (aborted) {
         for (int k = drain_from; k < issued; k++)
-            mbar_wait_bounded(bar0 + 8 * (k & (kStages - 1)), (static_cast<uint32_t>(k) / kStages) & 1u,
+            mbar_wait_bounded(bar0 + 8 * (k % kStages), (static_cast<uint32_t>(k) / kStages) & 1u,
                               kWaitLimitNs / 10);
         mbar_wait_bounded(qbar, qphase, kWaitLimitNs / 10);
     }

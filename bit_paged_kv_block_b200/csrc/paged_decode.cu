@@ -158,18 +158,18 @@ __device__ __forceinline__ uint32_t code_offset(int r, int c)
     return static_cast<uint32_t>(r * (kD / 2) + ((c ^ sw) << 4));
 }
 
-// One page of one warp: QK^T, online softmax, PV.  kMask: tokens [0, mask.valid) of the page
-// exist (the rest were never written: their V scale and zero are replaced by 0) and column e
-// (block row 2t + e) sees tokens [0, mask.col[e]).
+// The logits of one page (log2 domain): S^T = K . Q^T over its 16 tokens (rows g, g + 8), then
+// s = scale * acc + zero * sum(q) per (token, query column); tokens a column may not see get
+// -inf.  kMask: tokens [0, mask.valid) of the page exist and column e (block row 2t + e) sees
+// tokens [0, mask.col[e]).
 template <bool kMask, int kD>
-__device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, const PageMask &mask,
-                                             const uint32_t bq[kD / 16][2], const float sq[2],
-                                             int lane, WarpState<kD / 16> &st)
+__device__ __forceinline__ void page_logits(uint32_t cbase, uint32_t sbase, const PageMask &mask,
+                                            const uint32_t bq[kD / 16][2], const float sq[2],
+                                            int lane, float s[4])
 {
     const int g = lane >> 2, t = lane & 3;
     constexpr int kWords = kD / 32;   // 32-bit code words of one row per thread
 
-    // ---- S^T = K . Q^T over 16 tokens (rows g, g + 8) -----------------------------------
     // Thread t reads the kD / 4 codes of d in [kD/4 t, kD/4 (t + 1)) of rows g and g + 8: for
     // kD >= 128 whole 16-byte chunks (within each quarter warp the two rows land in disjoint
     // banks), for kD = 64 half a chunk (each half warp reads four whole 32-byte rows).
@@ -210,12 +210,9 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
         mma_16816(acc, a1, bq[2 * w + 1][0], bq[2 * w + 1][1]);
     }
 
-    // ---- logits (log2 domain) ---------------------------------------------------------------
-    const bool v0 = !kMask || g < mask.valid, v1 = !kMask || g + 8 < mask.valid;
     const float2 ksz0 = h2_to_f2(lds32(sbase + 4 * g));
     const float2 ksz1 = h2_to_f2(lds32(sbase + 4 * (g + 8)));
     const float ks0 = ksz0.x * kLowNibble, ks1 = ksz1.x * kLowNibble;
-    float s[4];
     s[0] = fmaf(ks0, acc[0], ksz0.y * sq[0]);
     s[1] = fmaf(ks0, acc[1], ksz0.y * sq[1]);
     s[2] = fmaf(ks1, acc[2], ksz1.y * sq[0]);
@@ -230,11 +227,18 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
         if (g + 8 >= mask.col[1])
             s[3] = -INFINITY;
     }
+}
 
-    float pr[4];
-    softmax_update<kMask, kD / 16>(s, st, pr);
-
-    // V-side scale / zero of tokens g, g + 8 (masked tokens contribute exactly 0)
+// O^T += V^T . P'^T for one page with weights pr (tokens g, g + 8 of columns 2t, 2t + 1), and the
+// running sums l (weights) and z (weights times the V zero points).  kMask: tokens past
+// mask.valid were never written; their V scale and zero are replaced by 0, so they contribute
+// exactly 0 whatever bits their rows hold.
+template <bool kMask, int kD>
+__device__ __forceinline__ void page_pv(uint32_t cbase, uint32_t sbase, const PageMask &mask,
+                                        const float pr[4], int lane, WarpState<kD / 16> &st)
+{
+    const int g = lane >> 2;
+    const bool v0 = !kMask || g < mask.valid, v1 = !kMask || g + 8 < mask.valid;
     float2 vsz0 = h2_to_f2(lds32(sbase + 64 + 4 * g));
     float2 vsz1 = h2_to_f2(lds32(sbase + 64 + 4 * (g + 8)));
     if (kMask) {
@@ -252,7 +256,6 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
     const uint32_t pb0 = movmatrix_trans(p01);   // B fragment: tokens 2t, 2t+1 of head g
     const uint32_t pb1 = movmatrix_trans(p23);   // tokens 2t + 8, 2t + 9
 
-    // ---- O^T += V^T . P'^T -----------------------------------------------------------------
     // ldmatrix.trans: lane L addresses row (L & 7) of matrix L >> 3; matrices are
     // (tokens 0-7 | 8-15) x (16-byte chunk 2j | 2j + 1) of the V rows (rows 16..31).
     const int vrow = 16 + ((lane >> 3) & 1) * 8 + (lane & 7);
@@ -277,6 +280,33 @@ __device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, con
     }
 }
 
+// One page of one warp: QK^T, online softmax, PV.
+template <bool kMask, int kD>
+__device__ __forceinline__ void process_page(uint32_t cbase, uint32_t sbase, const PageMask &mask,
+                                             const uint32_t bq[kD / 16][2], const float sq[2],
+                                             int lane, WarpState<kD / 16> &st)
+{
+    float s[4], pr[4];
+    page_logits<kMask, kD>(cbase, sbase, mask, bq, sq, lane, s);
+    softmax_update<kMask, kD / 16, 4>(s, st, pr);
+    page_pv<kMask, kD>(cbase, sbase, mask, pr, lane, st);
+}
+
+// Two whole pages of one warp as one step: both pages' logits (two independent tensor-core
+// chains), one online-softmax update over their 32 tokens, then PV for both.
+template <int kD>
+__device__ __forceinline__ void process_pages2(uint32_t cbase0, uint32_t sbase0, uint32_t cbase1,
+                                               uint32_t sbase1, const uint32_t bq[kD / 16][2],
+                                               const float sq[2], int lane, WarpState<kD / 16> &st)
+{
+    const PageMask whole = {kPageSize, {kPageSize, kPageSize}};
+    float s[8], pr[8];
+    page_logits<false, kD>(cbase0, sbase0, whole, bq, sq, lane, s);
+    page_logits<false, kD>(cbase1, sbase1, whole, bq, sq, lane, s + 4);
+    softmax_update<false, kD / 16, 8>(s, st, pr);
+    page_pv<false, kD>(cbase0, sbase0, whole, pr, lane, st);
+    page_pv<false, kD>(cbase1, sbase1, whole, pr + 4, lane, st);
+}
 
 // o_r = o / l, out = H o_r (o_r itself for the plain INT4 cache) for the block rows 2t, 2t + 1
 // this thread holds; H acts on each block of min(kD, 128) elements of d.  As the quantized part
@@ -442,6 +472,14 @@ struct Int4Format {
     {
         process_page<kMask, kD>(r.code0 + stg * kCodeBytes, r.scale0 + stg * kScaleBytes, mask,
                                 q.bq, q.sq, lane, st);
+    }
+    static constexpr bool kPairs = kD != 256;   // two whole pages as one step (page2)
+    __device__ static void page2(const Ring &r, int stg0, int stg1, const Query &q, int lane,
+                                 WarpState<kTiles> &st)
+    {
+        process_pages2<kD>(r.code0 + stg0 * kCodeBytes, r.scale0 + stg0 * kScaleBytes,
+                           r.code0 + stg1 * kCodeBytes, r.scale0 + stg1 * kScaleBytes, q.bq, q.sq,
+                           lane, st);
     }
     __device__ static void piece_end(WarpState<kTiles> &st)
     {

@@ -59,6 +59,7 @@ struct Bf16FormatT {
     static constexpr int kWarps = 4;
     static constexpr int kStages = 2;
     static constexpr int kMinBlocks = 3;
+    static constexpr bool kPairs = false;
     static constexpr int kRowsPerPage = kBf16PageBytes / kBf16RowBytes;   // 64
     static constexpr int kRingBytes = kWarps * kStages * kBf16PageBytes;
     struct Ring {
@@ -131,7 +132,7 @@ struct Bf16FormatT {
                 s[3] = -INFINITY;
         }
         float pr[4];
-        softmax_update<kMask, 8>(s, st, pr);
+        softmax_update<kMask, 8, 4>(s, st, pr);
         st.l[0] += pr[0] + pr[2];
         st.l[1] += pr[1] + pr[3];
 

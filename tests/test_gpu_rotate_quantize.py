@@ -237,3 +237,25 @@ def test_head_dim_64_strided(cuda_device, hkv):
     torch.cuda.synchronize()
     pages, scales = oracle_cache(wl, k=k.contiguous(), v=v.contiguous())
     assert_cache_equal(kv, sc, pages, scales)
+
+
+def test_rotate_quantize_out_of_fp16_range_sets_status(cuda_device):
+    """A constant vector of -6000 rotates to (-6000 sqrt(128), 0, ..., 0): its minimum -67882 lies
+    beyond fp16's range, so the stored zero point is -inf (the round-to-nearest conversion of the
+    definition, bit-identical to the oracle) and the kernel reports SAW_DEV_RANGE.  Vectors in
+    range in the same call are stored as usual and leave the bit alone when they are alone."""
+    from bit_paged_kv_block_b200 import saw
+    wl = synth.custom("range", [32], num_q_heads=8, num_kv_heads=2, seed=3, new_tokens=[32])
+    k = torch.randn(32, 2, 128, generator=torch.Generator().manual_seed(3)).to(torch.bfloat16)
+    v = k.flip(-1).clone()
+    k[5, 1] = -6000.0                                  # out of range: K of token 5, head 1
+    status = torch.zeros(1, dtype=torch.int32, device=cuda_device)
+    kv, sc = gpu_append(wl, cuda_device, k=k, v=v, status=status)
+    assert int(status.item()) & saw.SAW_DEV_RANGE
+    pages, scales = oracle_cache(wl, k=k, v=v)
+    assert_cache_equal(kv, sc, pages, scales)
+    k_ok = k.clone()
+    k_ok[5, 1] = -100.0
+    status.zero_()
+    gpu_append(wl, cuda_device, k=k_ok, v=v, status=status)
+    assert int(status.item()) == 0
