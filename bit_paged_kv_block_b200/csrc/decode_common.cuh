@@ -637,7 +637,11 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
 
     // ---- 1. sequence tables, the plan, zero the output rows that get no segment ----------------
     scan_sequences<kPrefill>(p, tb, flags, blockIdx.x == 0);
-    pdl_launch_dependents();   // the merge kernel may start its own prologue
+    // The merge kernel may start its own prologue.  The window part of a windowed decode holds
+    // its dependent (the quantized part) back until the cache writes it waits for are complete
+    // (below), so that the quantized part can read the cache at once.
+    if (p.win_part != 1)
+        pdl_launch_dependents();
     // (the quantized part of a windowed decode leaves such rows to the window part, which
     // also marks their lse empty)
     for (int s = blockIdx.x; s < S && p.win_part != 2; s += gridDim.x) {
@@ -652,19 +656,46 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
                     p.lse[row0 + i] = -INFINITY;
         }
     }
+    // Leaving early keeps a windowed decode's order: the window part waits for the cache writes
+    // before it releases the quantized part, and the quantized part completes only after the
+    // window part (its merge kernel reads the window part's rows).
+    auto pdl_exit = [&]() {
+        if (p.win_part != 0)
+            pdl_wait();
+        if (p.win_part == 1)
+            pdl_launch_dependents();
+    };
     if (tb.spre[S] > p.max_segments) {   // more query rows than the workspace was sized for
         if (blockIdx.x == 0 && tid == 0)
             set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
+        pdl_exit();
         return;
     }
     Plan plan;
     plan.init(tb, S, p.total_warps);
     const int64_t u = static_cast<int64_t>(blockIdx.x) * Fmt::kWarps + warp;
-    if (plan.P == 0 || u >= plan.W)
+    int64_t F0, F1;
+    if (p.win_part == 1) {
+        // the window part: warp u takes segment u whole (no split, so no partials to merge)
+        if (u >= tb.spre[S]) {
+            pdl_exit();
+            return;
+        }
+        const int s = plan.seq_of_segment(u);
+        F0 = tb.fpre[s] + (u - tb.spre[s]) * tb.npg[s];
+        F1 = F0 + tb.npg[s];
+    } else {
+        if (plan.P == 0 || u >= plan.W) {
+            pdl_exit();
+            return;
+        }
+        F0 = plan.begin(u);
+        F1 = plan.begin(u + 1);
+    }
+    if (F0 >= F1) {
+        pdl_exit();
         return;
-    const int64_t F0 = plan.begin(u), F1 = plan.begin(u + 1);
-    if (F0 >= F1)
-        return;
+    }
     const int n_w = static_cast<int>(F1 - F0);
 
     // ---- 2. this warp's copy ring ---------------------------------------------------------------
@@ -713,7 +744,13 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         }
     };
 
-    pdl_wait();   // the cache may be written by the kernel this one depends on
+    // The cache may be written by the kernel this one depends on.  The quantized part of a
+    // windowed decode depends on the window part, which released it only after that kernel's
+    // writes were complete: it waits only where it needs the window part's rows (finalize).
+    if (p.win_part != 2)
+        pdl_wait();
+    if (p.win_part == 1)
+        pdl_launch_dependents();
 
     // Lanes hold the tensor-map rows of pages [look_base, look_base + 32) of the run in look_a
     // and of the 32 after them in look_b, whose block-table reads are thus in flight 32 pages
@@ -858,6 +895,8 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
         if (seg_start >= F0 && ends_segment) {
             Segment<kPrefill> sg;
             sg.init(p, tb, cs, cj);
+            if (p.win_part == 2)
+                pdl_wait();   // the window part's rows and lse
             Fmt::finalize(p, sg, lane, st.o, st.m, st.l);
         } else {
             store_partial(p.partials + (tb.spre[cs] + cj + u) * slot_floats<Fmt::kTiles>(), lane, st);
@@ -874,6 +913,8 @@ __global__ void __launch_bounds__(32 * Fmt::kWarps, Fmt::kMinBlocks)
                               kWaitLimitNs / 10);
         mbar_wait_bounded(qbar, qphase, kWaitLimitNs / 10);
     }
+    if (p.win_part == 2)
+        pdl_wait();   // complete only after the window part (the merge kernel reads its rows)
 }
 
 constexpr int kShapeVariants = 4;

@@ -373,10 +373,10 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     p.max_segments = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, a.total_q, prefill);
     p.total_warps = ls.sms * ls.occ * Bf16Format::kWarps;
     // The window part's segments are short (at most sink + recent tokens each): one warp per
-    // segment, so windows of equal length are never split and its merge has nothing to fold,
-    // instead of runs of a page or two whose fixed costs dominate.
+    // segment, never split, so it needs no merge kernel; the quantized part follows it directly
+    // and overlaps it, waiting for its rows only at finalize.
     if (a.win_part == 1)
-        p.total_warps = static_cast<int32_t>(std::max<int64_t>(1, std::min<int64_t>(p.total_warps, p.max_segments)));
+        p.total_warps = static_cast<int32_t>(std::max<int64_t>(1, p.max_segments));
     p.q_mult = static_cast<float>(static_cast<double>(a.sm_scale) * 1.4426950408889634);
 
     cudaLaunchAttribute attr[1];
@@ -401,6 +401,8 @@ cudaError_t launch_paged_decode_bf16(const DecodeArgs &a, cudaStream_t stream, b
     if (e != cudaSuccess)
         return e;
 
+    if (window)
+        return cudaGetLastError();
     const int64_t segs = p.max_segments;
     cudaLaunchConfig_t mcfg = cfg;
     mcfg.gridDim = dim3(static_cast<unsigned>(std::max<int64_t>(1, std::min<int64_t>(segs, 8 * ls.sms))));
