@@ -252,8 +252,8 @@ __device__ __forceinline__ uint32_t vmin3_u16x2(uint32_t a, uint32_t b, uint32_t
 // vector's fp32 scale and zero point, given the vector's min and max.  words[g] (g < kN / 8) holds
 // the codes of elements 8 g .. 8 g + 7 and words[kN / 8 + g] those of elements kN + 8 g .. (low
 // halves, then high halves of the registers).  Groups of 8 registers are finished one after
-// another (the rare exactly half-way elements and scales outside [2^-100, 2^100] inside the
-// group), so each group's registers are free once its two words exist.
+// another (the rare exactly half-way elements inside the group), so each group's registers are
+// free once its two words exist; scales outside [2^-100, 2^100] take the IEEE divide throughout.
 template <int kN>
 __device__ __forceinline__ void quantize_block(const uint64_t X[kN], float mn, float mx,
                                                uint32_t words[kN / 4], float &scale_out,
@@ -272,6 +272,23 @@ __device__ __forceinline__ void quantize_block(const uint64_t X[kN], float mn, f
     const uint64_t nmn2 = f2_pack(-mn, -mn), r2 = f2_pack(r16, r16);
     const uint64_t m2 = f2_pack(kGridMagic, kGridMagic);
 
+    if (divide) {
+        // scales outside [2^-100, 2^100] (rare): every element by the IEEE divide
+#pragma unroll
+        for (int g = 0; g < kN / 8; g++) {
+            uint32_t wl = 0, wh = 0;
+#pragma unroll
+            for (int e = 0; e < 8; e++) {
+                float a, b;
+                f2_unpack(X[8 * g + e], a, b);
+                wl |= code_by_divide(a, mn, scale) << (4 * e);
+                wh |= code_by_divide(b, mn, scale) << (4 * e);
+            }
+            words[g] = wl;
+            words[kN / 8 + g] = wh;
+        }
+        return;
+    }
 #pragma unroll
     for (int g = 0; g < kN / 8; g++) {
         uint32_t tlo[8], thi[8];
@@ -288,16 +305,7 @@ __device__ __forceinline__ void quantize_block(const uint64_t X[kN], float mn, f
             thi[e] = __float_as_uint(b);
             f = vmin3_u16x2(f, tlo[e], thi[e]);
         }
-        if (divide) {
-            // every element by the IEEE divide
-#pragma unroll
-            for (int e = 0; e < 8; e++) {
-                float a, b;
-                f2_unpack(X[8 * g + e], a, b);
-                tlo[e] = code_by_divide(a, mn, scale) << 16;
-                thi[e] = code_by_divide(b, mn, scale) << 16;
-            }
-        } else if ((f & 0xFFFFu) == 0) {
+        if ((f & 0xFFFFu) == 0) {
             // rare: settle each exactly half-way element by the remainder test
 #pragma unroll
             for (int e = 0; e < 8; e++) {
