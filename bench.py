@@ -15,6 +15,11 @@ beside it), and the CPU oracle as a baseline.
 
 With --impl reference the script times the CPU oracle (the plain C reference in oracle/) on a
 bounded sample of the same workload and prints its line; under torchrun only rank 0 does so.
+
+Profiling aids (their numbers are not bench values): --loop-launches L --loop-seconds 0 cuts every
+per-kernel timing loop to L launches, so that a one-pass ncu launch list covers the whole bench;
+--profile rot_quant|decode builds one kernel's workload and launches that kernel six times, for a
+full ncu capture of a single launch.
 """
 from __future__ import annotations
 
@@ -62,6 +67,14 @@ def parse():
     ap.add_argument("--warmup", type=int, default=100)
     ap.add_argument("--impl", default="saw", choices=["saw", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    # profiling aids: shorter per-kernel loops (for a launch list under ncu), or one kernel's
+    # workload alone, launched a few times (for a full ncu capture of one launch)
+    ap.add_argument("--loop-launches", type=int, default=200,
+                    help="per-kernel timing loops run at least this many launches")
+    ap.add_argument("--loop-seconds", type=float, default=0.5,
+                    help="... and at least this long (0: exactly --loop-launches)")
+    ap.add_argument("--profile", choices=["rot_quant", "decode"],
+                    help="run only this kernel on its workload (3 warm-ups, then 3 launches)")
     return ap.parse_args()
 
 
@@ -258,9 +271,13 @@ MIN_LAUNCHES = 200        # per-launch loops: at least this many launches ...
 MIN_LOOP_SECONDS = 0.5    # ... and at least this long, whatever --steps is
 
 
-def loop_count(fn, stream, min_launches=MIN_LAUNCHES, min_seconds=MIN_LOOP_SECONDS, cap=20000):
+def loop_count(fn, stream, min_launches=None, min_seconds=None, cap=20000):
     """Launches a timing loop needs to reach both bounds (estimated from 10 back-to-back runs)."""
     import torch
+    min_launches = MIN_LAUNCHES if min_launches is None else min_launches
+    min_seconds = MIN_LOOP_SECONDS if min_seconds is None else min_seconds
+    if min_seconds <= 0:
+        return min_launches
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record(stream)
     for _ in range(10):
@@ -883,10 +900,47 @@ def run_saw(args):
     return 0
 
 
+def run_profile(args):
+    """One kernel on its workload, 3 warm-up launches then 3 more, nothing else (for ncu)."""
+    import torch
+    from bit_paged_kv_block_b200 import saw, synth
+    dev = torch.device("cuda", 0)
+    if args.profile == "rot_quant":
+        pre = synth.make_workload("prefill")
+        kv, sc = saw.allocate_cache(pre.num_pages, pre.num_kv_heads, dev)
+        seq, pos = synth.token_index(pre, "all")
+        k = synth.kv_values(pre, "K", device=dev)
+        v = synth.kv_values(pre, "V", device=dev)
+        slots = torch.from_numpy(synth.slot_mapping(pre, seq, pos)).to(dev)
+        fn = lambda: saw.saw_rotate_quantize_paged(k, v, slots, kv, sc)
+    else:
+        wl = synth.make_workload("decode")
+        kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
+        seq, pos = synth.token_index(wl, "all")
+        saw.saw_rotate_quantize_paged(synth.kv_values(wl, "K", device=dev),
+                                      synth.kv_values(wl, "V", device=dev),
+                                      torch.from_numpy(synth.slot_mapping(wl, seq, pos)).to(dev), kv, sc)
+        q = synth.q_values(wl, device=dev)
+        tab = torch.from_numpy(wl.block_table).to(dev)
+        lens = torch.from_numpy(wl.seq_lens).to(dev)
+        out = torch.empty((wl.num_seqs, wl.num_q_heads, 128), dtype=torch.float32, device=dev)
+        ws = saw.allocate_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
+        fn = lambda: saw.saw_paged_decode_attn(q, kv, sc, tab, lens, out, ws)
+    for _ in range(6):
+        fn()
+    torch.cuda.synchronize()
+    print(json.dumps({"profile": args.profile, "launches": 6}), flush=True)
+    return 0
+
+
 def main():
     args = parse()
+    global MIN_LAUNCHES, MIN_LOOP_SECONDS
+    MIN_LAUNCHES, MIN_LOOP_SECONDS = args.loop_launches, args.loop_seconds
     if args.impl == "reference":
         return run_reference(args)
+    if args.profile:
+        return run_profile(args)
     return run_saw(args)
 
 
