@@ -123,15 +123,6 @@ __device__ __forceinline__ void scale_all(uint64_t X[kN], float c)
         X[i] = f2_mul(X[i], cc);
 }
 
-// The normalised Hadamard transform of a block one thread holds whole (2 kN points): the stages,
-// then every element times fp32(1/sqrt(2 kN)).
-template <int kN>
-__device__ __forceinline__ void fwht_block(uint64_t X[kN])
-{
-    fwht_stages<kN>(X);
-    scale_all<kN>(X, kN == 64 ? kHadamardC : kHadamardC64);
-}
-
 // Stage h = 64 of a 128-point block split over lanes L (elements 0..63, b = 0) and L ^ 1 (elements
 // 64..127, b = 1): each lane takes its partner's 64 values by shuffles and forms its own half of the
 // stage's outputs: x + partner (lower lane) or partner - x = fma(x, -1, partner) (upper lane).  The
@@ -532,10 +523,11 @@ __global__ void __launch_bounds__(kRqThreads, 4)
 // the rotate+quantize kernel (same device code).  With w_recent = 0 the new token itself is
 // quantized.  Window slot i lives in bf16 page win_table[s][i / 16] at offset i mod 16.
 //
-// Lanes as in the rotate+quantize kernel at D = 128: a warp takes 16 (sequence, kv head) pairs,
-// lanes 0-15 their K vectors and lanes 16-31 their V vectors, one thread per vector.  Each thread
-// reads exactly the 256 bytes of the displaced vector it later overwrites with the new token, so
-// the read and the write of a slot are ordered within one thread.
+// Lanes as in the rotate+quantize kernel at D = 128: a warp takes 8 (sequence, kv head) pairs,
+// lanes 0-15 their K vectors and lanes 16-31 their V vectors, two lanes per vector (lane 2 i + b
+// holds elements 64 b .. 64 b + 63 of pair i; stage h = 64 is the shuffle exchange).  Each thread
+// reads exactly the 128 bytes of the displaced vector that it later overwrites with the new
+// token, so the read and the write of those bytes are ordered within one thread.
 struct WinAppendParams {
     const uint16_t *k, *v;
     const int32_t *seq_lens;
@@ -559,12 +551,13 @@ __global__ void __launch_bounds__(kRqThreads)
     pdl_launch_dependents();
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const int half = lane >> 4;
-    const int64_t pair = (static_cast<int64_t>(blockIdx.x) * kRqWarps + warp) * 16 + (lane & 15);
+    const int part = lane & 1;
+    const int64_t pair = (static_cast<int64_t>(blockIdx.x) * kRqWarps + warp) * 8 + ((lane & 15) >> 1);
     const bool live = pair < static_cast<int64_t>(p.num_seqs) * p.hkv;
     const int s = live ? static_cast<int>(pair / p.hkv) : 0;
     const int h = live ? static_cast<int>(pair - static_cast<int64_t>(s) * p.hkv) : 0;
     const int L = live ? p.seq_lens[s] : 0;
-    const bool report = half == 0;
+    const bool report = half == 0 && part == 0;
 
     // where the new token goes and which token is quantized
     bool to_win = false, quant = false, from_win = false;
@@ -588,7 +581,7 @@ __global__ void __launch_bounds__(kRqThreads)
     } else if (L < 0 && report) {
         set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
     }
-    uint16_t *win = nullptr;
+    uint16_t *win = nullptr;   // this thread's 64 elements of the window slot
     if (to_win) {
         const int32_t page = p.win_table[static_cast<int64_t>(s) * p.win_blocks + slot / 16];
         if (page < 0 || page >= p.num_win_pages) {
@@ -597,7 +590,7 @@ __global__ void __launch_bounds__(kRqThreads)
             to_win = quant = false;   // the displaced token cannot be read: leave the pair
         } else {
             win = p.win_kv + ((((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize) +
-                              slot % kPageSize) * 128;
+                              slot % kPageSize) * 128 + 64 * part;
         }
     }
     int64_t row = 0;
@@ -615,28 +608,41 @@ __global__ void __launch_bounds__(kRqThreads)
     }
 
     // the vector to quantize (the displaced window token, or the new token itself when there is
-    // no recent ring): elements 0..63 in lo, 64..127 in hi
-    const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128;
+    // no recent ring); both lanes of a vector decide alike, and every lane runs the transform
+    // (its stage h = 64 pairs lanes 2 i and 2 i + 1): lanes with nothing to quantize run it on
+    // zeros and store nothing
+    const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128 + 64 * part;
+    uint64_t X[32];
     if (quant) {
         const uint16_t *qsrc = from_win ? win : src;
-        uint64_t X[64];
 #pragma unroll
-        for (int c = 0; c < 8; c++)
+        for (int c = 0; c < 4; c++)
             pairs_from_chunk(*reinterpret_cast<const uint4 *>(qsrc + 8 * c),
-                             *reinterpret_cast<const uint4 *>(qsrc + 64 + 8 * c), X + 8 * c);
-        if constexpr (kRotate)
-            fwht_block<64>(X);
-        float mn, mx;
-        block_min_max<64>(X, mn, mx);
-        uint32_t words[16];
-        float scale, zero;
-        quantize_block<64>(X, mn, mx, words, scale, zero);
-        store_block<64>(p.kv_pages + row * 64, words, true, scale, zero, p.scales + row, p.status);
+                             *reinterpret_cast<const uint4 *>(qsrc + 32 + 8 * c), X + 8 * c);
+    } else {
+#pragma unroll
+        for (int i = 0; i < 32; i++)
+            X[i] = 0;
     }
-    // then the new token takes the slot (after this thread's own read of it)
+    if constexpr (kRotate) {
+        fwht_stages<32>(X);
+        exchange_stage64(X, part);
+        scale_all<32>(X, kHadamardC);
+    }
+    float mn, mx;
+    block_min_max<32>(X, mn, mx);
+    mn = fminf(mn, __shfl_xor_sync(0xFFFFFFFFu, mn, 1));
+    mx = fmaxf(mx, __shfl_xor_sync(0xFFFFFFFFu, mx, 1));
+    uint32_t words[8];
+    float scale, zero;
+    quantize_block<32>(X, mn, mx, words, scale, zero);
+    if (quant)
+        store_block<32>(p.kv_pages + row * 64 + 32 * part, words, part == 0, scale, zero, p.scales + row,
+                        p.status);
+    // then the new token takes the slot (after this thread's own read of these bytes)
     if (to_win) {
 #pragma unroll
-        for (int c = 0; c < 16; c++)
+        for (int c = 0; c < 8; c++)
             *reinterpret_cast<uint4 *>(win + 8 * c) = *reinterpret_cast<const uint4 *>(src + 8 * c);
     }
 }
@@ -666,7 +672,7 @@ cudaError_t launch_window_append(const WindowAppendArgs &a, cudaStream_t stream)
     p.kv_pages = a.kv_pages;
     p.scales = static_cast<uint32_t *>(a.scales);
     p.status = a.status;
-    const int64_t grid = (pairs + 16 * kRqWarps - 1) / (16 * kRqWarps);
+    const int64_t grid = (pairs + 8 * kRqWarps - 1) / (8 * kRqWarps);
     window_append_kernel<true><<<static_cast<unsigned>(grid), kRqThreads, 0, stream>>>(p);
     return cudaGetLastError();
 }
