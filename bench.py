@@ -19,7 +19,7 @@ bounded sample of the same workload and prints its line; under torchrun only ran
 Profiling aids (their numbers are not bench values): --loop-launches L --loop-seconds 0 cuts every
 per-kernel timing loop to L launches, so that a one-pass ncu launch list covers the whole bench;
 --profile rot_quant|decode builds one kernel's workload and launches that kernel six times, for a
-full ncu capture of a single launch.
+full ncu capture of a single launch; --profile window runs the windowed serving step six times.
 """
 from __future__ import annotations
 
@@ -73,8 +73,8 @@ def parse():
                     help="per-kernel timing loops run at least this many launches")
     ap.add_argument("--loop-seconds", type=float, default=0.5,
                     help="... and at least this long (0: exactly --loop-launches)")
-    ap.add_argument("--profile", choices=["rot_quant", "decode"],
-                    help="run only this kernel on its workload (3 warm-ups, then 3 launches)")
+    ap.add_argument("--profile", choices=["rot_quant", "decode", "window"],
+                    help="run only this kernel (window: the windowed step) on its workload, 6 times")
     return ap.parse_args()
 
 
@@ -900,6 +900,34 @@ def run_saw(args):
     return 0
 
 
+def window_profile_step(wl, q, tab, lens, out, dev):
+    """The windowed serving step of the bench's window line (16 sink + 112 recent bf16 tokens) on
+    the decode workload: the cache and window filled from the history tokens, the step appends the
+    new tokens (window append with eviction) and decodes (window part + quantized part + merge)."""
+    import torch
+    from bit_paged_kv_block_b200 import saw, synth
+    sink, recent = 16, 112
+    wkv, wtab = saw.allocate_window(wl.num_seqs, wl.num_kv_heads, sink, recent, dev)
+    kv, sc = saw.allocate_cache(wl.num_pages, wl.num_kv_heads, dev)
+    kh = synth.kv_values(wl, "K", tokens="history", device=dev)
+    vh = synth.kv_values(wl, "V", tokens="history", device=dev)
+    seqh, posh = synth.token_index(wl, "history")
+    lh = wl.seq_lens[seqh] - 1
+    in_win = (posh < sink) | (posh >= np.maximum(sink, lh - recent))
+    j = posh - sink
+    qslot = np.where(in_win, -1, wl.block_table[seqh, np.maximum(j, 0) // 16] * 16 + j % 16)
+    wslot = np.where(posh < sink, posh, sink + (posh - sink) % max(recent, 1))
+    wtab_np = wtab.cpu().numpy()
+    wslot = np.where(in_win, wtab_np[seqh, wslot // 16] * 16 + wslot % 16, -1)
+    saw.saw_rotate_quantize_paged(kh, vh, torch.from_numpy(qslot.astype(np.int64)).to(dev), kv, sc)
+    saw.saw_append_bf16_paged(kh, vh, torch.from_numpy(wslot.astype(np.int64)).to(dev), wkv)
+    win = (sink, recent, wkv, wtab)
+    ws = saw.allocate_window_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
+    k_new = synth.kv_values(wl, "K", tokens="new", device=dev)
+    v_new = synth.kv_values(wl, "V", tokens="new", device=dev)
+    return lambda: saw.saw_decode_step_window(q, k_new, v_new, win, kv, sc, tab, lens, out, ws)
+
+
 def run_profile(args):
     """One kernel on its workload, 3 warm-up launches then 3 more, nothing else (for ncu)."""
     import torch
@@ -926,6 +954,8 @@ def run_profile(args):
         out = torch.empty((wl.num_seqs, wl.num_q_heads, 128), dtype=torch.float32, device=dev)
         ws = saw.allocate_workspace(wl.num_kv_heads, wl.num_q_heads, wl.num_seqs, dev)
         fn = lambda: saw.saw_paged_decode_attn(q, kv, sc, tab, lens, out, ws)
+        if args.profile == "window":
+            fn = window_profile_step(wl, q, tab, lens, out, dev)
     for _ in range(6):
         fn()
     torch.cuda.synchronize()
