@@ -558,6 +558,15 @@ __global__ void __launch_bounds__(kRqThreads)
     const int h = live ? static_cast<int>(pair - static_cast<int64_t>(s) * p.hkv) : 0;
     const int L = live ? p.seq_lens[s] : 0;
     const bool report = half == 0 && part == 0;
+    // this thread's 64 elements of the new token, loaded now: nothing below depends on them, so
+    // their latency overlaps the table lookups instead of following the quantization
+    const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128 + 64 * part;
+    uint4 fresh[8];
+    if (live) {
+#pragma unroll
+        for (int c = 0; c < 8; c++)
+            fresh[c] = *reinterpret_cast<const uint4 *>(src + 8 * c);
+    }
 
     // where the new token goes and which token is quantized
     bool to_win = false, quant = false, from_win = false;
@@ -611,7 +620,6 @@ __global__ void __launch_bounds__(kRqThreads)
     // no recent ring); both lanes of a vector decide alike, and every lane runs the transform
     // (its stage h = 64 pairs lanes 2 i and 2 i + 1): lanes with nothing to quantize run it on
     // zeros and store nothing
-    const uint16_t *src = (half ? p.v : p.k) + (static_cast<int64_t>(s) * p.hkv + h) * 128 + 64 * part;
     uint64_t X[32];
     if (quant) {
         const uint16_t *qsrc = from_win ? win : src;
@@ -643,7 +651,7 @@ __global__ void __launch_bounds__(kRqThreads)
     if (to_win) {
 #pragma unroll
         for (int c = 0; c < 8; c++)
-            *reinterpret_cast<uint4 *>(win + 8 * c) = *reinterpret_cast<const uint4 *>(src + 8 * c);
+            *reinterpret_cast<uint4 *>(win + 8 * c) = fresh[c];
     }
 }
 
