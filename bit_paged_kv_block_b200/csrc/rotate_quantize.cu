@@ -590,9 +590,15 @@ __global__ void __launch_bounds__(kRqThreads)
     } else if (L < 0 && report) {
         set_status(p.status, SAW_DEV_BAD_SEQ_LEN);
     }
+    // both table lookups depend only on the length: issue them together
+    const bool q_in_table = j / kPageSize < p.max_blocks;
+    const int32_t wpage = to_win ? p.win_table[static_cast<int64_t>(s) * p.win_blocks + slot / 16] : 0;
+    const int32_t qpage = quant && q_in_table
+                              ? p.block_table[static_cast<int64_t>(s) * p.max_blocks + j / kPageSize]
+                              : -1;
     uint16_t *win = nullptr;   // this thread's 64 elements of the window slot
     if (to_win) {
-        const int32_t page = p.win_table[static_cast<int64_t>(s) * p.win_blocks + slot / 16];
+        const int32_t page = wpage;
         if (page < 0 || page >= p.num_win_pages) {
             if (report)
                 set_status(p.status, SAW_DEV_BAD_PAGE);
@@ -604,12 +610,10 @@ __global__ void __launch_bounds__(kRqThreads)
     }
     int64_t row = 0;
     if (quant) {
-        const int32_t page = j / kPageSize < p.max_blocks
-                                 ? p.block_table[static_cast<int64_t>(s) * p.max_blocks + j / kPageSize]
-                                 : -1;
+        const int32_t page = qpage;
         if (page < 0 || page >= p.num_pages) {
             if (report)
-                set_status(p.status, j / kPageSize < p.max_blocks ? SAW_DEV_BAD_PAGE : SAW_DEV_BAD_SEQ_LEN);
+                set_status(p.status, q_in_table ? SAW_DEV_BAD_PAGE : SAW_DEV_BAD_SEQ_LEN);
             to_win = quant = false;   // keep the displaced token where it is
         } else {
             row = ((static_cast<int64_t>(page) * p.hkv + h) * 2 + half) * kPageSize + j % kPageSize;
