@@ -37,23 +37,26 @@ constexpr uint64_t kWaitLimitNs = 1000000000ull;        // give up a copy wait a
 constexpr int kRowsPerBlock = 8;                        // query rows (MMA columns) per segment
 constexpr int kMergeWarps = 4;
 constexpr int kMergeThreads = 32 * kMergeWarps;
+// a launch with at most one segment per SM (few, long sequences: each split over tens of warps)
+// folds each segment's partials with this many warps
+constexpr int kMergeWarpsWide = 8;
 // per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
 constexpr int kSeqTableBytes = 20;
 // merge kernel shared memory: per-warp partials, flags, then the sequence tables
-template <int kTiles>
-__host__ __device__ constexpr int merge_smem_flags() { return (kMergeWarps - 1) * slot_floats<kTiles>() * 4; }
+template <int kTiles, int kMW = kMergeWarps>
+__host__ __device__ constexpr int merge_smem_flags() { return (kMW - 1) * slot_floats<kTiles>() * 4; }
 // the flags hold scan_sequences' two int64 partial sums per warp
-template <int kTiles>
-__host__ __device__ constexpr int merge_smem_tables() { return merge_smem_flags<kTiles>() + 16 * kMergeWarps; }
+template <int kTiles, int kMW = kMergeWarps>
+__host__ __device__ constexpr int merge_smem_tables() { return merge_smem_flags<kTiles, kMW>() + 16 * kMW; }
 
 inline size_t seq_table_bytes(int32_t num_seqs)
 {
     return kSeqTableBytes * (static_cast<size_t>(num_seqs) + 1);
 }
-template <int kTiles>
+template <int kTiles, int kMW = kMergeWarps>
 inline size_t merge_smem_bytes(int32_t num_seqs)
 {
-    return merge_smem_tables<kTiles>() + seq_table_bytes(num_seqs);
+    return merge_smem_tables<kTiles, kMW>() + seq_table_bytes(num_seqs);
 }
 
 // Segments of a launch: decode, num_seqs * hkv * ceil(G / 8); chunked prefill over total_q
@@ -509,8 +512,8 @@ __device__ __forceinline__ void load_partial(const float *slot, int lane, float 
 // (m, l, o) for global segment g; the warps of a block fold disjoint subsets in a fixed order,
 // then warp 0 folds the other warps' results in warp order and writes the output through the
 // page format's finalize step, so the result does not depend on timing.
-template <class Fmt, bool kPrefill>
-__global__ void __launch_bounds__(kMergeThreads)
+template <class Fmt, bool kPrefill, int kMW = kMergeWarps>
+__global__ void __launch_bounds__(32 * kMW)
     paged_decode_merge_kernel(const DecodeParams p)
 {
     extern __shared__ uint8_t smem_raw[];
@@ -519,8 +522,8 @@ __global__ void __launch_bounds__(kMergeThreads)
     constexpr int kTiles = Fmt::kTiles;
     constexpr int kSlot = slot_floats<kTiles>();
     SeqTables tb;
-    tb.bind(smem + merge_smem_tables<kTiles>(), p.num_seqs);
-    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + merge_smem_flags<kTiles>());
+    tb.bind(smem + merge_smem_tables<kTiles, kMW>(), p.num_seqs);
+    volatile int64_t *flags = reinterpret_cast<volatile int64_t *>(smem + merge_smem_flags<kTiles, kMW>());
     float *slots = reinterpret_cast<float *>(smem);
 
     scan_sequences<kPrefill>(p, tb, flags, false);
@@ -540,13 +543,13 @@ __global__ void __launch_bounds__(kMergeThreads)
             continue;
         WarpState<kTiles> st;
         state_reset(st);
-        // each warp folds every kMergeWarps-th partial; two loads in flight per step
+        // each warp folds every kMW-th partial; two loads in flight per step
         int64_t uu = u_lo + warp;
-        for (; uu + kMergeWarps <= u_hi; uu += 2 * kMergeWarps) {
+        for (; uu + kMW <= u_hi; uu += 2 * kMW) {
             float bm0[2], bl0[2], bm1[2], bl1[2];
             float4 bo0[kTiles], bo1[kTiles];
             load_partial(p.partials + (gseg + uu) * kSlot, lane, bm0, bl0, bo0);
-            load_partial(p.partials + (gseg + uu + kMergeWarps) * kSlot, lane, bm1, bl1, bo1);
+            load_partial(p.partials + (gseg + uu + kMW) * kSlot, lane, bm1, bl1, bo1);
             merge_into(st.m, st.l, st.o, bm0, bl0, bo0);
             merge_into(st.m, st.l, st.o, bm1, bl1, bo1);
         }
@@ -560,7 +563,7 @@ __global__ void __launch_bounds__(kMergeThreads)
             store_partial(slots + (warp - 1) * kSlot, lane, st);
         __syncthreads();
         if (warp == 0) {
-            for (int w = 1; w < kMergeWarps; w++) {
+            for (int w = 1; w < kMW; w++) {
                 float bm[2], bl[2];
                 float4 bo[kTiles];
                 load_partial(slots + (w - 1) * kSlot, lane, bm, bl, bo);

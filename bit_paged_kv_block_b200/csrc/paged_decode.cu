@@ -680,6 +680,19 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     mcfg.blockDim = dim3(kMergeThreads);
     mcfg.dynamicSmemBytes = msmem;
     mcfg.numAttrs = 1;
+    // at most one segment per SM: every segment is split over tens of warps, whose partials the
+    // wider merge folds in fewer rounds (its shared memory stays below the default 48 KiB)
+    if (kD <= 128 && !prefill && !window_merge && segs <= ls.sms) {
+        constexpr int kW = kMergeWarpsWide;
+        mcfg.blockDim = dim3(32 * kW);
+        mcfg.dynamicSmemBytes = merge_smem_bytes<Fmt::kTiles, kW>(a.num_seqs);
+        e = cudaLaunchKernelEx(&mcfg, a.rotate ? paged_decode_merge_kernel<Int4Format<true, kD>, false, kW>
+                                               : paged_decode_merge_kernel<Int4Format<false, kD>, false, kW>,
+                               p);
+        if (e != cudaSuccess)
+            return e;
+        return cudaGetLastError();
+    }
     auto *merge = window_merge ? paged_decode_merge_kernel<Int4Format<true, kD, true>, false>
                   : a.rotate   ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true>
                                           : paged_decode_merge_kernel<Int4Format<true, kD>, false>)
