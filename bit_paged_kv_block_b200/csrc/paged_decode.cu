@@ -682,12 +682,16 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     mcfg.numAttrs = 1;
     // at most one segment per SM: every segment is split over tens of warps, whose partials the
     // wider merge folds in fewer rounds (its shared memory stays below the default 48 KiB)
-    if (kD <= 128 && !prefill && !window_merge && segs <= ls.sms) {
+    // (the chunked prefill on this kernel takes the same choice, so that a one-token chunk stays
+    // bit-identical to the decode)
+    if (kD <= 128 && !window_merge && segs <= ls.sms) {
         constexpr int kW = kMergeWarpsWide;
         mcfg.blockDim = dim3(32 * kW);
         mcfg.dynamicSmemBytes = merge_smem_bytes<Fmt::kTiles, kW>(a.num_seqs);
-        e = cudaLaunchKernelEx(&mcfg, a.rotate ? paged_decode_merge_kernel<Int4Format<true, kD>, false, kW>
-                                               : paged_decode_merge_kernel<Int4Format<false, kD>, false, kW>,
+        e = cudaLaunchKernelEx(&mcfg, a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true, kW>
+                                                          : paged_decode_merge_kernel<Int4Format<true, kD>, false, kW>)
+                                               : (prefill ? paged_decode_merge_kernel<Int4Format<false, kD>, true, kW>
+                                                          : paged_decode_merge_kernel<Int4Format<false, kD>, false, kW>),
                                p);
         if (e != cudaSuccess)
             return e;
