@@ -682,9 +682,10 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
     mcfg.numAttrs = 1;
     // at most one segment per SM: every segment is split over tens of warps, whose partials the
     // wider merge folds in fewer rounds (its shared memory stays below the default 48 KiB)
-    // (the chunked prefill on this kernel takes the same choice, so that a one-token chunk stays
-    // bit-identical to the decode)
-    if (kD <= 128 && !window_merge && segs <= ls.sms) {
+    // (the chunked prefill on this kernel takes the same choice from the same count, the decode's
+    // segments, so that a one-token chunk stays bit-identical to the decode)
+    const int64_t decode_segs = max_segments(a.num_kv_heads, a.num_q_heads, a.num_seqs, 0, false);
+    if (kD <= 128 && !window_merge && decode_segs <= ls.sms) {
         constexpr int kW = kMergeWarpsWide;
         mcfg.blockDim = dim3(32 * kW);
         mcfg.dynamicSmemBytes = merge_smem_bytes<Fmt::kTiles, kW>(a.num_seqs);

@@ -64,18 +64,24 @@ def test_prefill_plain_cache(cuda_device):
     assert_attention_close(got, want, "prefill plain")
 
 
-def test_prefill_of_one_token_is_the_decode(cuda_device):
-    """C_s = 1 for every sequence is a decode: the same segments and split, so the outputs are
-    bit-identical to saw_paged_decode_attn."""
+@pytest.mark.parametrize("lens,hq", [
+    ([300, 17, 1, 64, 1000], 8),
+    # 70 sequences x 2 kv heads at G = 1: 140 decode segments, at most one per SM of a B200, while
+    # the prefill's segment bound is larger; both must still pick the same split-K merge
+    ([2000 + 37 * i for i in range(70)], 2),
+])
+def test_prefill_of_one_token_is_the_decode(cuda_device, lens, hq):
+    """C_s = 1 for every sequence is a decode: the same segments, split and merge, so the outputs
+    are bit-identical to saw_paged_decode_attn."""
     from bit_paged_kv_block_b200 import saw
-    wl = synth.custom("pf1", [300, 17, 1, 64, 1000], num_q_heads=8, num_kv_heads=2, seed=12)
+    wl = synth.custom("pf1", lens, num_q_heads=hq, num_kv_heads=2, seed=12)
     pages, scales = oracle_cache(wl)
     q = synth.q_values(wl)
     q_start = np.arange(wl.num_seqs + 1, dtype=np.int32)
     got = _prefill(wl, pages, scales, q, q_start, cuda_device)
     kv, sc = device_cache_from(pages, scales, cuda_device)
-    out = torch.empty((wl.num_seqs, 8, 128), device=cuda_device)
-    ws = saw.allocate_workspace(2, 8, wl.num_seqs, cuda_device)
+    out = torch.empty((wl.num_seqs, hq, 128), device=cuda_device)
+    ws = saw.allocate_workspace(2, hq, wl.num_seqs, cuda_device)
     saw.saw_paged_decode_attn(q.to(cuda_device), kv, sc,
                               torch.from_numpy(wl.block_table).to(cuda_device),
                               torch.from_numpy(wl.seq_lens).to(cuda_device), out, ws)
