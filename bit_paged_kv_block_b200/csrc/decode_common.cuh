@@ -40,6 +40,8 @@ constexpr int kMergeThreads = 32 * kMergeWarps;
 // a launch with at most one segment per SM (few, long sequences: each split over tens of warps)
 // folds each segment's partials with this many warps
 constexpr int kMergeWarpsWide = 8;
+// ... and a launch with more than 4 segments per SM (many short sequences) with this many
+constexpr int kMergeWarpsNarrow = 1;
 // per-sequence shared-memory tables (fpre int64, spre int32, npg int32, nbk int32) + ends
 constexpr int kSeqTableBytes = 20;
 // merge kernel shared memory: per-warp partials, flags, then the sequence tables

@@ -698,6 +698,22 @@ cudaError_t launch(const DecodeArgs &a, cudaStream_t stream, bool programmatic)
             return e;
         return cudaGetLastError();
     }
+    // many short segments (more than 4 per SM, each split over one or two warps): fewer warps per
+    // segment, and enough CTAs for one wave over them
+    if (kD <= 128 && !window_merge && decode_segs > 4 * static_cast<int64_t>(ls.sms)) {
+        constexpr int kW = kMergeWarpsNarrow;
+        mcfg.gridDim = dim3(static_cast<unsigned>(std::min<int64_t>(segs, (32 / kW) * ls.sms)));
+        mcfg.blockDim = dim3(32 * kW);
+        mcfg.dynamicSmemBytes = merge_smem_bytes<Fmt::kTiles, kW>(a.num_seqs);
+        e = cudaLaunchKernelEx(&mcfg, a.rotate ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true, kW>
+                                                          : paged_decode_merge_kernel<Int4Format<true, kD>, false, kW>)
+                                               : (prefill ? paged_decode_merge_kernel<Int4Format<false, kD>, true, kW>
+                                                          : paged_decode_merge_kernel<Int4Format<false, kD>, false, kW>),
+                               p);
+        if (e != cudaSuccess)
+            return e;
+        return cudaGetLastError();
+    }
     auto *merge = window_merge ? paged_decode_merge_kernel<Int4Format<true, kD, true>, false>
                   : a.rotate   ? (prefill ? paged_decode_merge_kernel<Int4Format<true, kD>, true>
                                           : paged_decode_merge_kernel<Int4Format<true, kD>, false>)
